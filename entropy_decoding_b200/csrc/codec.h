@@ -1,0 +1,71 @@
+// codec.h -- host side of libdf11: code construction, decode-table building,
+// the multi-threaded encoder, the container and the device image.
+#pragma once
+
+#include <cstdint>
+#include <memory>
+#include <string>
+#include <vector>
+
+#include "df11_internal.h"
+
+namespace df11 {
+
+enum Dtype : int { kBF16 = 0, kE4M3 = 1 };
+
+inline int nsym_of(int dtype) { return dtype == kBF16 ? 256 : 16; }
+
+struct Codebook {
+    int dtype = kBF16;
+    int nsym = 256;
+    uint8_t lengths[256] = {};
+    uint32_t codes[256] = {};
+    int max_len_used = 0;
+    int min_len_used = 0;
+    std::vector<uint16_t> meta;  // kMultiEntries
+    std::vector<uint32_t> syms;  // kMultiEntries
+    std::vector<uint16_t> lut;   // n_luts * kLutEntries
+    int n_luts() const { return static_cast<int>(lut.size() / kLutEntries); }
+};
+
+struct Blob {
+    int dtype = kBF16;
+    int chunk_bits = 128;
+    int tile_threads = 256;
+    uint64_t n = 0;
+    uint64_t total_bits = 0;
+    uint64_t n_tiles = 0;
+    uint64_t max_span = 0;
+    std::shared_ptr<const Codebook> cb;
+    std::vector<uint8_t> stream;    // ceil(total_bits / 8)
+    std::vector<uint8_t> plane;     // n (BF16) or ceil(n / 2) (E4M3)
+    std::vector<uint8_t> gaps;      // n_tiles * tile_threads
+    std::vector<uint64_t> out_off;  // n_tiles + 1
+    const uint8_t *dev_image = nullptr;
+    uint64_t dev_cap = 0;
+    std::vector<uint8_t> host_image;  // staging copy kept alive for df11_blob_upload
+};
+
+// Code construction.  Returns false when the arguments admit no code.
+bool code_lengths(const uint64_t *counts, int nsym, int max_len, uint8_t *lengths);
+bool canonical_codes(const uint8_t *lengths, int nsym, uint32_t *codes);  // false: not a prefix code
+std::shared_ptr<Codebook> make_codebook(int dtype, const uint8_t *lengths);  // nullptr if invalid
+
+// Histogram of the exponent field, added into counts[256].
+void histogram(int dtype, const void *src, uint64_t n, uint64_t *counts, int n_threads);
+
+// Encoder: returns an empty string on success, else the reason.
+std::string encode(std::shared_ptr<const Codebook> cb, const void *src, uint64_t n, int chunk_bits,
+                   int tile_threads, int n_threads, Blob *out);
+
+uint64_t plane_bytes(int dtype, uint64_t n);
+uint64_t serialized_bytes(const Blob &b);
+void serialize(const Blob &b, uint8_t *dst);
+std::string deserialize(const uint8_t *src, uint64_t len, Blob *out);
+
+ImageLayout image_layout(const Blob &b);
+void write_image(const Blob &b, uint8_t *dst);
+
+bool valid_layout(int chunk_bits, int tile_threads);
+
+}  // namespace df11

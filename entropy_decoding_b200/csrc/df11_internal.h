@@ -1,0 +1,83 @@
+// df11_internal.h -- layout constants and structures shared by the host codec
+// (codec.cpp), the C-ABI (capi.cpp) and the decode kernels (decode.cu).
+//
+// Decode tables (the "compact, hierarchical lookup tables that fit within GPU
+// SRAM" of the DFloat11 Abstract, item (i)):
+//   * hierarchical LUT: levels of 256 u16 entries indexed by the next 8 stream
+//     bits.  Table 0 is the root.  Entry forms:
+//       leaf     bit15 = 0: bits 0..7 symbol, bits 8..13 full code length
+//       pointer  bit15 = 1: bits 0..14 index of the next-level table
+//       invalid  bit14 = 1 (leaf form, length 1): no codeword has this prefix
+//     A 32-bit code needs at most 4 levels.
+//   * multi-symbol table (an addition for sm_100a's instruction budget): 4096
+//     entries indexed by the next 12 stream bits.  meta[v] = consumed bits
+//     (bits 0..5) | symbols decoded (bits 8..10), for the longest run of up
+//     to 4 whole codes inside the 12-bit window; meta[v] = kMetaLong when the
+//     first code is longer than 12 bits.  syms[v] holds those symbols, first
+//     in the low byte.
+#pragma once
+
+#include <cstdint>
+
+namespace df11 {
+
+constexpr int kMultiBits = 12;
+constexpr int kMultiEntries = 1 << kMultiBits;
+constexpr int kMultiMaxSyms = 4;
+constexpr uint16_t kMetaLong = 0x0040;
+
+constexpr int kLutEntries = 256;
+constexpr uint16_t kLutPointer = 0x8000;
+constexpr uint16_t kLutInvalid = 0x4000 | (1u << 8);
+constexpr int kMaxLutTables = 0x7FFF;
+constexpr int kSmemLutTables = 16;  // hierarchical tables staged in shared memory; the rest stay in global
+
+constexpr int kMaxCodeLen = 32;
+constexpr int kMaxTensorsPerLaunch = 64;
+constexpr uint64_t kImageAlign = 256;
+constexpr uint64_t kStreamTail = 16;  // zero bytes after the last tile: look-ahead of the last thread
+constexpr uint64_t kPlaneTail = 32;
+
+inline uint64_t align_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
+
+// Offsets of the sections inside one blob's device image.
+struct ImageLayout {
+    uint64_t meta, syms, lut, gaps, out_off, stream, plane, total;
+};
+
+// Header at offset 0 of every device image (kept for inspection; the kernel
+// takes everything it needs from its launch parameters).
+struct ImageHeader {
+    char magic[8];  // "DF11IMG1"
+    uint32_t dtype, chunk_bits, tile_threads, n_luts;
+    uint64_t n_elems, total_bits, n_tiles, max_span;
+    ImageLayout layout;
+};
+
+// One tensor of a batched launch.  Tiles of all tensors are numbered
+// consecutively: tensor i owns global tiles [tile_begin, tile_begin + n_tiles).
+struct TensorDesc {
+    const uint8_t *stream;
+    const uint8_t *plane;
+    const uint8_t *gaps;
+    const uint64_t *out_off;
+    void *dst;
+    uint64_t n;
+    uint64_t total_bits;
+    uint32_t n_tiles;
+    uint32_t tile_begin;
+};
+
+struct DecodeParams {
+    const uint16_t *meta;
+    const uint32_t *syms;
+    const uint16_t *lut;
+    int *err;
+    int32_t n_luts;
+    int32_t n_tensors;
+    uint32_t total_tiles;
+    uint32_t max_span;  // largest per-tile span over the launch's tensors
+    TensorDesc t[kMaxTensorsPerLaunch];
+};
+
+}  // namespace df11

@@ -1,0 +1,287 @@
+"""Thin ctypes binding of libdf11 (C-ABI declared in include/df11.h).
+
+Every function here only marshals arguments into the library call of the same
+name; encoding runs in the library's host code, decoding in its sm_100a
+kernel.  There is no Python or CPU fallback: importing this module raises
+when libdf11.so has not been built (``python -m entropy_decoding_b200.build``).
+
+PyTorch is used only as a source of device memory and streams: device
+pointers are plain integers (``tensor.data_ptr()``), streams are
+``torch.cuda.Stream.cuda_stream`` integers (0 = default stream).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdf11.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "df11.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libdf11.so not built at {LIB_PATH}; run `python -m entropy_decoding_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+DF11_OK, DF11_EINVAL, DF11_ENOMEM, DF11_ECUDA, DF11_ECORRUPT, DF11_EUNSUPPORTED = range(6)
+DF11_BF16, DF11_FP8_E4M3 = 0, 1
+DTYPES = {"bf16": DF11_BF16, "e4m3": DF11_FP8_E4M3}
+DEV_ERR_SPAN, DEV_ERR_CODE, DEV_ERR_AUX, DEV_ERR_TIMEOUT = 1, 2, 4, 8
+
+
+class Df11Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {_lib.df11_status_string(status).decode()} ({status})")
+
+
+class BlobInfo(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int32), ("chunk_bits", ctypes.c_int32), ("tile_threads", ctypes.c_int32),
+                ("max_code_len", ctypes.c_int32), ("n_elems", ctypes.c_uint64), ("total_bits", ctypes.c_uint64),
+                ("n_tiles", ctypes.c_uint64), ("max_span", ctypes.c_uint64), ("stream_bytes", ctypes.c_uint64),
+                ("plane_bytes", ctypes.c_uint64), ("gaps_bytes", ctypes.c_uint64),
+                ("out_off_bytes", ctypes.c_uint64), ("serialized_bytes", ctypes.c_uint64),
+                ("device_bytes", ctypes.c_uint64), ("uncompressed_bytes", ctypes.c_uint64)]
+
+    def as_dict(self) -> dict:
+        return {k: getattr(self, k) for k, _ in self._fields_}
+
+
+_P = ctypes.c_void_p
+_PP = ctypes.POINTER(ctypes.c_void_p)
+_U64 = ctypes.c_uint64
+_I = ctypes.c_int
+_S = ctypes.c_int  # df11_status
+
+_SIGS = {
+    "df11_version": ([], _I),
+    "df11_status_string": ([_I], ctypes.c_char_p),
+    "df11_build_codebook": ([_I, _PP, ctypes.POINTER(_U64), _I, _I, _PP], _S),
+    "df11_codebook_from_lengths": ([_I, _P, _I, _PP], _S),
+    "df11_codebook_lengths": ([_P, _P], _S),
+    "df11_codebook_free": ([_P], None),
+    "df11_encode": ([_P, _P, _U64, _PP], _S),
+    "df11_encode_ex": ([_P, _P, _U64, _I, _I, _I, _PP], _S),
+    "df11_layout_supported": ([_I, _I, _I], _I),
+    "df11_blob_free": ([_P], None),
+    "df11_blob_get_info": ([_P, ctypes.POINTER(BlobInfo)], _S),
+    "df11_blob_sections": ([_P, _PP, _PP, _PP, _PP], _S),
+    "df11_blob_lengths": ([_P, _P], _S),
+    "df11_serialize": ([_P, _P, _U64, ctypes.POINTER(_U64)], _S),
+    "df11_deserialize": ([_P, _U64, _PP], _S),
+    "df11_blob_device_image": ([_P, _P, _U64], _S),
+    "df11_blob_bind": ([_P, _P, _U64], _S),
+    "df11_blob_upload": ([_P, _P, _U64, _P], _S),
+    "df11_decode": ([_PP, _PP, _I, _P, _P], _S),
+    "df11_decode_host": ([_PP, _PP, _PP, _PP, _PP, _I, _P, _P], _S),
+    "df11_decode_launch_shape": ([_PP, _I, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I)], _S),
+}
+for _name, (_args, _res) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.argtypes = _args
+    _f.restype = _res
+
+
+def exported_names() -> list[str]:
+    """Function names declared in include/df11.h (for the symbol check)."""
+    with open(HEADER_PATH) as f:
+        src = f.read()
+    return sorted(set(re.findall(r"\b(df11_[a-z_0-9]+)\s*\(", src)))
+
+
+def _check(status: int, what: str):
+    if status != DF11_OK:
+        raise Df11Error(status, what)
+
+
+def _ptr_array(ptrs) -> ctypes.Array:
+    return (ctypes.c_void_p * len(ptrs))(*[int(p) if p is not None else None for p in ptrs])
+
+
+# ----------------------------------------------------------------- objects
+
+class Codebook:
+    def __init__(self, handle: int, dtype: str):
+        self._h = ctypes.c_void_p(handle)
+        self.dtype = dtype
+
+    @property
+    def handle(self):
+        return self._h
+
+    def lengths(self) -> np.ndarray:
+        out = np.zeros(256, np.uint8)
+        _check(_lib.df11_codebook_lengths(self._h, out.ctypes.data), "df11_codebook_lengths")
+        return out[: 256 if self.dtype == "bf16" else 16]
+
+    def __del__(self):
+        if getattr(self, "_h", None) and self._h.value:
+            _lib.df11_codebook_free(self._h)
+            self._h = ctypes.c_void_p(0)
+
+
+class Blob:
+    def __init__(self, handle: int):
+        self._h = ctypes.c_void_p(handle)
+        self._keep = None  # device image owner (e.g. a torch tensor)
+
+    @property
+    def handle(self):
+        return self._h
+
+    def info(self) -> BlobInfo:
+        i = BlobInfo()
+        _check(_lib.df11_blob_get_info(self._h, ctypes.byref(i)), "df11_blob_get_info")
+        return i
+
+    @property
+    def dtype(self) -> str:
+        return "bf16" if self.info().dtype == DF11_BF16 else "e4m3"
+
+    def sections(self) -> dict:
+        """Copies of the host sections: stream, plane, gaps, out_off."""
+        i = self.info()
+        ptrs = [ctypes.c_void_p() for _ in range(4)]
+        _check(_lib.df11_blob_sections(self._h, *[ctypes.byref(p) for p in ptrs]), "df11_blob_sections")
+
+        def grab(p, n, dt):
+            if n == 0:
+                return np.zeros(0, dt)
+            return np.ctypeslib.as_array(ctypes.cast(p, ctypes.POINTER(ctypes.c_uint8)), (n,)).view(dt).copy()
+
+        return {"stream": grab(ptrs[0], i.stream_bytes, np.uint8),
+                "plane": grab(ptrs[1], i.plane_bytes, np.uint8),
+                "gaps": grab(ptrs[2], i.gaps_bytes, np.uint8),
+                "out_off": grab(ptrs[3], i.out_off_bytes, np.uint64)}
+
+    def lengths(self) -> np.ndarray:
+        out = np.zeros(256, np.uint8)
+        _check(_lib.df11_blob_lengths(self._h, out.ctypes.data), "df11_blob_lengths")
+        return out
+
+    def __del__(self):
+        if getattr(self, "_h", None) and self._h.value:
+            _lib.df11_blob_free(self._h)
+            self._h = ctypes.c_void_p(0)
+
+
+# ----------------------------------------------------------------- functions (same names as the C-ABI)
+
+def df11_version() -> int:
+    return _lib.df11_version()
+
+
+def df11_build_codebook(dtype: str, tensors, max_code_len: int = 0) -> Codebook:
+    arrs = [np.ascontiguousarray(t).reshape(-1) for t in tensors]
+    ptrs = _ptr_array([a.ctypes.data if a.size else None for a in arrs])
+    ns = (_U64 * len(arrs))(*[a.size for a in arrs])
+    out = ctypes.c_void_p()
+    _check(_lib.df11_build_codebook(DTYPES[dtype], ptrs, ns, len(arrs), max_code_len, ctypes.byref(out)),
+           "df11_build_codebook")
+    return Codebook(out.value, dtype)
+
+
+def df11_codebook_from_lengths(dtype: str, lengths) -> Codebook:
+    ln = np.ascontiguousarray(lengths, np.uint8)
+    out = ctypes.c_void_p()
+    _check(_lib.df11_codebook_from_lengths(DTYPES[dtype], ln.ctypes.data, ln.size, ctypes.byref(out)),
+           "df11_codebook_from_lengths")
+    return Codebook(out.value, dtype)
+
+
+def df11_encode(cb: Codebook, x: np.ndarray, chunk_bits: int = 128, tile_threads: int = 256,
+                n_threads: int = 0) -> Blob:
+    a = np.ascontiguousarray(x).reshape(-1)
+    out = ctypes.c_void_p()
+    _check(_lib.df11_encode_ex(cb.handle, a.ctypes.data if a.size else None, a.size, chunk_bits, tile_threads,
+                               n_threads, ctypes.byref(out)), "df11_encode")
+    return Blob(out.value)
+
+
+def df11_layout_supported(dtype: str, chunk_bits: int, tile_threads: int) -> bool:
+    return bool(_lib.df11_layout_supported(DTYPES[dtype], chunk_bits, tile_threads))
+
+
+def df11_serialize(blob: Blob) -> bytes:
+    used = _U64()
+    _lib.df11_serialize(blob.handle, None, 0, ctypes.byref(used))
+    buf = np.zeros(used.value, np.uint8)
+    _check(_lib.df11_serialize(blob.handle, buf.ctypes.data, buf.size, ctypes.byref(used)), "df11_serialize")
+    return buf.tobytes()
+
+
+def df11_deserialize(data) -> Blob:
+    buf = np.frombuffer(data, np.uint8)
+    if buf.size == 0:
+        buf = np.zeros(1, np.uint8)
+        n = 0
+    else:
+        n = buf.size
+    out = ctypes.c_void_p()
+    _check(_lib.df11_deserialize(buf.ctypes.data, n, ctypes.byref(out)), "df11_deserialize")
+    return Blob(out.value)
+
+
+def df11_blob_device_image(blob: Blob, host_dst_ptr: int, cap: int):
+    _check(_lib.df11_blob_device_image(blob.handle, host_dst_ptr, cap), "df11_blob_device_image")
+
+
+def df11_blob_bind(blob: Blob, dev_image_ptr: int, cap: int, keep=None):
+    _check(_lib.df11_blob_bind(blob.handle, dev_image_ptr, cap), "df11_blob_bind")
+    blob._keep = keep
+
+
+def df11_blob_upload(blob: Blob, dev_dst_ptr: int, cap: int, stream: int = 0, keep=None):
+    _check(_lib.df11_blob_upload(blob.handle, dev_dst_ptr, cap, stream or None), "df11_blob_upload")
+    blob._keep = keep
+
+
+def df11_decode(blobs, dst_ptrs, err_ptr: int | None = None, stream: int = 0):
+    hs = _ptr_array([b.handle.value for b in blobs])
+    ds = _ptr_array(dst_ptrs)
+    _check(_lib.df11_decode(hs, ds, len(blobs), err_ptr or None, stream or None), "df11_decode")
+
+
+def df11_decode_host(blobs, host_image_ptrs, dev_image_ptrs, dst_dev_ptrs, dst_host_ptrs,
+                     err_ptr: int | None = None, stream: int = 0):
+    _check(_lib.df11_decode_host(_ptr_array([b.handle.value for b in blobs]), _ptr_array(host_image_ptrs),
+                                 _ptr_array(dev_image_ptrs), _ptr_array(dst_dev_ptrs), _ptr_array(dst_host_ptrs),
+                                 len(blobs), err_ptr or None, stream or None), "df11_decode_host")
+
+
+def df11_decode_launch_shape(blobs) -> tuple[int, int, int]:
+    g, b, s = _I(), _I(), _I()
+    _check(_lib.df11_decode_launch_shape(_ptr_array([x.handle.value for x in blobs]), len(blobs),
+                                         ctypes.byref(g), ctypes.byref(b), ctypes.byref(s)),
+           "df11_decode_launch_shape")
+    return g.value, b.value, s.value
+
+
+# ----------------------------------------------------------------- torch-side helpers (device memory only)
+
+def upload(blob: Blob, stream=None):
+    """Allocates the device image with torch, copies it there and binds it.
+    Returns the torch tensor that owns the image (also kept on the blob)."""
+    import torch
+    n = blob.info().device_bytes
+    dev = torch.empty(n + 256, dtype=torch.uint8, device="cuda")
+    base = dev.data_ptr()
+    off = (-base) % 256
+    s = stream.cuda_stream if stream is not None else torch.cuda.current_stream().cuda_stream
+    df11_blob_upload(blob, base + off, n, s, keep=dev)
+    return dev
+
+
+def elem_bytes(dtype: str) -> int:
+    return 2 if dtype == "bf16" else 1
+
+
+def empty_output(blob: Blob):
+    """A device buffer (torch uint8, 16-byte aligned) for the decoded tensor."""
+    import torch
+    i = blob.info()
+    nbytes = i.n_elems * (2 if i.dtype == DF11_BF16 else 1)
+    return torch.empty(max(nbytes, 16), dtype=torch.uint8, device="cuda")

@@ -1,0 +1,244 @@
+/*
+ * df11.h -- C-ABI of libdf11: lossless BF16 / FP8-E4M3 weight compression by
+ * Huffman-coding the exponent field, with a B200 (sm_100a) decode kernel.
+ *
+ * The operations follow "70% Size, 100% Accuracy: Lossless LLM Compression
+ * for Efficient GPU Inference via Dynamic-Length Float (DFloat11)", Abstract:
+ *   - frequency-based dynamic-length (Huffman) codes for the low-entropy part
+ *     of each weight, built offline ............. df11_build_codebook
+ *   - the compressed tensor: raw sign+mantissa plane, packed code stream and
+ *     lightweight auxiliary variables that coordinate thread read/write
+ *     positions ................................. df11_encode
+ *   - online GPU decompression with lookup tables in on-chip SRAM and a
+ *     two-phase kernel, one launch per transformer block (all matrices of the
+ *     block in one launch) ...................... df11_decode
+ * and "Compressing LLMs without Compromise" summary page, section "Where the
+ * redundancy lives" (BF16 = 1 sign + 8 exponent + 7 mantissa bits; only the
+ * exponent is low-entropy) and section "Three ways to spend the savings"
+ * (exponents Huffman-coded offline, lookup tables in GPU shared memory);
+ * "To Compress or Not? ... Exponent Concentration", Abstract (FP8 variant).
+ *
+ * Conventions for every function:
+ *   - Host pointers are ordinary CPU memory; "device" pointers are CUDA
+ *     global-memory addresses of the current device.  No function takes or
+ *     returns framework (torch) objects.
+ *   - Objects (df11_codebook, df11_blob) are created by the library and owned
+ *     by the caller, who frees them with the matching *_free function.  Input
+ *     buffers are only read during the call unless stated otherwise.
+ *   - Errors are returned synchronously as df11_status; nothing aborts or
+ *     prints.  Calls are thread-safe for distinct objects.
+ *   - Decoding never allocates memory and never synchronises: the caller
+ *     provides every device buffer and owns the stream.
+ */
+#ifndef DF11_H
+#define DF11_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DF11_OK = 0,
+    DF11_EINVAL = 1,       /* bad argument (null pointer, size, alignment, mixed codes) */
+    DF11_ENOMEM = 2,       /* host allocation failed, or a caller buffer is too small */
+    DF11_ECUDA = 3,        /* a CUDA runtime call or kernel launch failed */
+    DF11_ECORRUPT = 4,     /* a serialized container failed validation */
+    DF11_EUNSUPPORTED = 5  /* a valid request this build has no kernel for */
+} df11_status;
+
+typedef enum {
+    DF11_BF16 = 0,      /* 16-bit words: sign | 8-bit exponent | 7-bit mantissa */
+    DF11_FP8_E4M3 = 1   /* bytes: sign | 4-bit exponent | 3-bit mantissa */
+} df11_dtype;
+
+/* Bits the decode kernel ORs into the caller's device error word.  Any
+ * non-zero value means some output of that call is not valid; the kernel
+ * still never writes outside the destination buffers it was given. */
+#define DF11_DEV_ERR_SPAN 1u     /* a tile decoded a different number of codes than its out_off span */
+#define DF11_DEV_ERR_CODE 2u     /* the stream held a bit pattern that is no codeword */
+#define DF11_DEV_ERR_AUX 4u      /* an auxiliary value (gap, out_off) out of its valid range */
+#define DF11_DEV_ERR_TIMEOUT 8u  /* a bounded wait on an on-chip barrier gave up */
+
+/* Same type as cudaStream_t; pass 0 for the legacy default stream. */
+typedef struct CUstream_st *df11_stream;
+
+typedef struct df11_codebook df11_codebook; /* host object: code lengths + decode tables */
+typedef struct df11_blob df11_blob;         /* host object: one compressed tensor */
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int df11_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *df11_status_string(df11_status status);
+
+/* ---------------------------------------------------------------------
+ * Codebook  (DFloat11 Abstract: "dynamic-length encodings ... based on
+ * frequency"; summary page: "Huffman-codes the exponents offline")
+ * ------------------------------------------------------------------ */
+
+/* Builds one code for a group of tensors (e.g. every matrix of one transformer
+ * block): the exponent histogram is summed over all n_tensors tensors, Huffman
+ * code lengths are computed (ties broken by (count, symbol) with merged nodes
+ * after leaves in creation order) and limited to max_code_len bits by
+ * package-merge when needed; codes are canonical.
+ *   dtype          DF11_BF16 (exponent = 8 bits, 256 symbols) or
+ *                  DF11_FP8_E4M3 (4 bits, 16 symbols).
+ *   host_tensors   n_tensors host pointers to the raw weights (uint16 words
+ *                  for BF16, bytes for E4M3); a pointer may be NULL only when
+ *                  its n_elems is 0.
+ *   n_elems        n_tensors element counts.
+ *   max_code_len   1..32, or 0 for 32; must allow a complete code
+ *                  (2^max_code_len >= number of distinct symbols).
+ *   out            receives the new codebook (caller frees).
+ * Errors: DF11_EINVAL for bad arguments, DF11_ENOMEM. */
+df11_status df11_build_codebook(df11_dtype dtype, const void *const *host_tensors,
+                                const uint64_t *n_elems, int n_tensors, int max_code_len,
+                                df11_codebook **out);
+
+/* Builds a codebook from explicit code lengths (n_lengths = 256 for BF16, 16
+ * for E4M3; 0 = symbol unused).  The lengths must form a prefix code (Kraft
+ * sum <= 1) with every length <= 32.  Errors: DF11_EINVAL. */
+df11_status df11_codebook_from_lengths(df11_dtype dtype, const uint8_t *lengths, int n_lengths,
+                                       df11_codebook **out);
+
+/* Copies the code length of every symbol into lengths[0..255] (E4M3 uses the
+ * first 16; the rest are 0). */
+df11_status df11_codebook_lengths(const df11_codebook *cb, uint8_t *lengths);
+
+void df11_codebook_free(df11_codebook *cb);
+
+/* ---------------------------------------------------------------------
+ * Encoding  (DFloat11 Abstract: "lightweight auxiliary variables")
+ * ------------------------------------------------------------------ */
+
+/* Compresses one tensor with a codebook (whose code must cover every exponent
+ * the tensor holds).  Default layout: chunk_bits = 128 stream bits per decode
+ * thread, tile_threads = 256 threads per tile; all host cores are used.
+ * The blob holds, in host memory:
+ *   plane    n bytes (BF16: sign << 7 | mantissa) or ceil(n/2) bytes (E4M3:
+ *            nibble sign << 3 | mantissa, element 2i in the low nibble)
+ *   stream   the canonical codes of the exponents in element order, most
+ *            significant bit first (stream bit k = bit 7 - k%8 of byte k/8)
+ *   gaps     one byte per chunk: offset of the first code that starts in the
+ *            chunk (padded with 0 to whole tiles)
+ *   out_off  n_tiles + 1 uint64 values: codes starting before each tile
+ * Errors: DF11_EINVAL (bad layout, or a symbol the code does not cover),
+ * DF11_ENOMEM. */
+df11_status df11_encode(const df11_codebook *cb, const void *host_src, uint64_t n_elems,
+                        df11_blob **out);
+
+/* df11_encode with an explicit layout: chunk_bits in {64, 128, 256},
+ * tile_threads in {128, 256, 512}; n_threads host threads (0 = all cores).
+ * df11_decode supports the layouts listed by df11_layout_supported. */
+df11_status df11_encode_ex(const df11_codebook *cb, const void *host_src, uint64_t n_elems,
+                           int chunk_bits, int tile_threads, int n_threads, df11_blob **out);
+
+/* 1 when df11_decode has a kernel for this (dtype, chunk_bits, tile_threads). */
+int df11_layout_supported(df11_dtype dtype, int chunk_bits, int tile_threads);
+
+void df11_blob_free(df11_blob *blob);
+
+typedef struct {
+    int32_t dtype;            /* df11_dtype */
+    int32_t chunk_bits;
+    int32_t tile_threads;
+    int32_t max_code_len;     /* longest code actually used */
+    uint64_t n_elems;
+    uint64_t total_bits;      /* stream length in bits */
+    uint64_t n_tiles;
+    uint64_t max_span;        /* most codes that start in one tile */
+    uint64_t stream_bytes;    /* ceil(total_bits / 8) */
+    uint64_t plane_bytes;
+    uint64_t gaps_bytes;
+    uint64_t out_off_bytes;
+    uint64_t serialized_bytes;/* size of df11_serialize's output: the container */
+    uint64_t device_bytes;    /* size of the device image (df11_blob_device_image) */
+    uint64_t uncompressed_bytes;
+} df11_blob_info;
+
+df11_status df11_blob_get_info(const df11_blob *blob, df11_blob_info *info);
+
+/* Read-only host views of the blob's sections (valid until the blob is freed);
+ * any output pointer may be NULL. */
+df11_status df11_blob_sections(const df11_blob *blob, const uint8_t **stream, const uint8_t **plane,
+                               const uint8_t **gaps, const uint64_t **out_off);
+
+/* Copies the code lengths the blob was encoded with into lengths[0..255]. */
+df11_status df11_blob_lengths(const df11_blob *blob, uint8_t *lengths);
+
+/* ---------------------------------------------------------------------
+ * Container (the offline, on-disk form)
+ * ------------------------------------------------------------------ */
+
+/* Writes the container (header with code lengths, gaps, out_off, stream,
+ * plane; sections 16-byte aligned) into buf[0..cap).  *used receives
+ * info.serialized_bytes.  Errors: DF11_ENOMEM when cap is too small. */
+df11_status df11_serialize(const df11_blob *blob, void *buf, uint64_t cap, uint64_t *used);
+
+/* Reads a container; validates the header, the code (Kraft sum, lengths),
+ * the section sizes and every auxiliary value against the layout rules.
+ * Errors: DF11_ECORRUPT for any inconsistency, DF11_ENOMEM. */
+df11_status df11_deserialize(const void *buf, uint64_t len, df11_blob **out);
+
+/* ---------------------------------------------------------------------
+ * Device image and decoding  (DFloat11 Abstract: hierarchical lookup tables
+ * in SRAM, two-phase kernel, transformer-block-level decompression)
+ * ------------------------------------------------------------------ */
+
+/* Writes the blob's device image into host memory host_dst[0..cap) (cap >=
+ * info.device_bytes; pinned memory makes the later copy asynchronous).  The
+ * image is one buffer with 256-byte aligned sections: the decode tables
+ * built from the code lengths, gaps, out_off, the stream padded with zeros
+ * to whole tiles plus 16 bytes, and the plane padded to 16 bytes plus 32. */
+df11_status df11_blob_device_image(const df11_blob *blob, void *host_dst, uint64_t cap);
+
+/* Records that the blob's device image is at device address dev_image
+ * (256-byte aligned, cap >= info.device_bytes), placed there by the caller.
+ * The memory stays owned by the caller and must outlive the decodes. */
+df11_status df11_blob_bind(df11_blob *blob, const void *dev_image, uint64_t cap);
+
+/* Convenience: builds the image in a host buffer held by the blob, copies it
+ * to dev_dst with cudaMemcpyAsync on `stream`, and binds it.  The caller owns
+ * dev_dst.  Errors: DF11_EINVAL, DF11_ENOMEM, DF11_ECUDA. */
+df11_status df11_blob_upload(df11_blob *blob, void *dev_dst, uint64_t cap, df11_stream stream);
+
+/* Decodes n_blobs bound blobs in ONE kernel launch on `stream`, asynchronously.
+ *   blobs        all encoded with the same code lengths, dtype and layout (a
+ *                transformer block shares one codebook); otherwise DF11_EINVAL.
+ *   dst_dev      n_blobs device pointers, 16-byte aligned, each holding
+ *                n_elems * 2 bytes (BF16) or n_elems bytes (E4M3); written
+ *                with the exact original bit patterns.  Buffers must not
+ *                overlap each other or the images.
+ *   n_blobs      1..64 per launch (more: DF11_EINVAL; split the call).
+ *   dev_err_flag device int, or NULL.  The kernel ORs DF11_DEV_ERR_* bits into
+ *                it when the data is inconsistent; the caller zeroes it.
+ * Never allocates, never synchronises.  Errors: DF11_EINVAL (unbound blob,
+ * misaligned or NULL pointer, mixed codes), DF11_EUNSUPPORTED (layout without
+ * a kernel), DF11_ECUDA (launch failure). */
+df11_status df11_decode(const df11_blob *const *blobs, void *const *dst_dev, int n_blobs,
+                        int *dev_err_flag, df11_stream stream);
+
+/* End-to-end decode from host memory to host memory, all on `stream` and
+ * asynchronous (the caller synchronises the stream before reading dst_host):
+ * for each blob, cudaMemcpyAsync host_images[i] (its device image, e.g. from
+ * df11_blob_device_image into pinned memory) to dev_images[i] and bind it;
+ * one df11_decode launch into dst_dev; then cudaMemcpyAsync dst_dev[i] to
+ * dst_host[i].  All buffers are the caller's.  Errors as df11_decode. */
+df11_status df11_decode_host(df11_blob *const *blobs, const void *const *host_images,
+                             void *const *dev_images, void *const *dst_dev, void *const *dst_host,
+                             int n_blobs, int *dev_err_flag, df11_stream stream);
+
+/* Launch shape df11_decode would use for these blobs on the current device:
+ * grid (persistent CTAs), threads per CTA and dynamic shared memory bytes.
+ * Any output pointer may be NULL. */
+df11_status df11_decode_launch_shape(const df11_blob *const *blobs, int n_blobs, int *grid,
+                                     int *block, int *smem_bytes);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DF11_H */

@@ -1,0 +1,209 @@
+"""GPU parity: the sm_100a decode kernel, called through the C-ABI, against the
+CPU oracle, element by element (bit-exact: the method is lossless, "70% Size,
+100% Accuracy ... (DFloat11)", Abstract: bit-for-bit identical outputs)."""
+import numpy as np
+import pytest
+import torch
+
+from entropy_decoding_b200 import synth
+from gpu_util import decode_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def df11():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from entropy_decoding_b200 import build
+    build.build()
+    from entropy_decoding_b200 import df11 as mod
+    return mod
+
+
+def _roundtrip(df11, oracle_mod, x, dt, chunk_bits=128, tile_threads=256, max_len=0, check_oracle=True):
+    cb = df11.df11_build_codebook(dt, [x], max_len)
+    blob = df11.df11_encode(cb, x, chunk_bits, tile_threads)
+    (out,), err, guards = decode_gpu(df11, [blob])
+    assert err == 0
+    assert guards
+    assert out.shape == x.shape
+    assert np.array_equal(out, x)
+    if check_oracle:
+        o = oracle_mod.compress(x, dt, lengths=cb.lengths(), chunk_bits=chunk_bits, tile_threads=tile_threads)
+        assert np.array_equal(out, oracle_mod.decompress(o))
+    return blob
+
+
+SMALL = {
+    "normal_1m": ("bf16", lambda: synth.single_matrix(0)[0].tensors[0].bits),
+    "heavy_2m": ("bf16", lambda: synth.heavy_tail_matrix(0)[0].tensors[0].bits[: 2 * 10 ** 6 + 3]),
+    "all_bf16": ("bf16", synth.all_bf16_patterns),
+    "single_symbol": ("bf16", lambda: synth.constant_bf16(100003, 0.0)),
+    "fib26": ("bf16", lambda: synth.powers_of_two_bf16(synth.fibonacci_counts(26), first_exponent=-20)),
+    "uniform_random": ("bf16", lambda: synth.random_bits(700001, "bf16", 1)),
+    "e4m3_normal": ("e4m3", lambda: synth.normal_e4m3(np.random.SeedSequence(0), 1000003)),
+    "e4m3_all": ("e4m3", synth.all_e4m3_patterns),
+    "e4m3_random": ("e4m3", lambda: synth.random_bits(500001, "e4m3", 2)),
+}
+
+
+@pytest.mark.parametrize("case", list(SMALL))
+def test_parity_small(df11, oracle_mod, case):
+    dt, make = SMALL[case]
+    _roundtrip(df11, oracle_mod, make(), dt)
+
+
+@pytest.mark.parametrize("n", [1, 2, 7, 8, 15, 16, 17, 31, 32, 33, 47, 1000, 4095, 4096, 4097])
+@pytest.mark.parametrize("dt", ["bf16", "e4m3"])
+def test_parity_ragged_sizes(df11, oracle_mod, dt, n):
+    x = synth.random_bits(n, dt, n) if n < 40 else (
+        synth.single_matrix(n)[0].tensors[0].bits[:n] if dt == "bf16"
+        else synth.normal_e4m3(np.random.SeedSequence(n), n))
+    _roundtrip(df11, oracle_mod, x, dt)
+
+
+LAYOUTS = [(128, 256), (256, 128), (64, 512), (128, 128), (128, 512), (256, 256)]
+
+
+@pytest.mark.parametrize("layout", LAYOUTS)
+@pytest.mark.parametrize("case", ["heavy_2m", "e4m3_normal", "single_symbol", "uniform_random"])
+def test_parity_layouts(df11, oracle_mod, layout, case):
+    dt, make = SMALL[case]
+    _roundtrip(df11, oracle_mod, make(), dt, *layout)
+
+
+def test_parity_32_bit_codes(df11, oracle_mod):
+    """Fibonacci counts F1..F34: package-merge limits the code to 32 bits, so
+    the decoder walks all four hierarchical levels."""
+    x = synth.powers_of_two_bf16(synth.fibonacci_counts(34), first_exponent=-40)
+    blob = _roundtrip(df11, oracle_mod, x, "bf16")
+    assert blob.info().max_code_len == 32
+
+
+@pytest.mark.parametrize("limit", [9, 12, 16])
+def test_parity_length_limited(df11, oracle_mod, limit):
+    x = synth.heavy_tail_matrix(1)[0].tensors[0].bits[:500000]
+    blob = _roundtrip(df11, oracle_mod, x, "bf16", max_len=limit)
+    assert blob.info().max_code_len <= limit
+
+
+def test_empty_tensor(df11):
+    x = np.zeros(0, np.uint16)
+    cb = df11.df11_build_codebook("bf16", [synth.random_bits(100, "bf16")])
+    blob = df11.df11_encode(cb, x)
+    assert blob.info().n_tiles == 0
+    outs, err, _ = decode_gpu(df11, [blob])
+    assert err == 0 and outs[0].size == 0
+
+
+def test_batched_block_launch_scaled(df11, oracle_mod):
+    """Seven Llama-3-8B-shaped matrices (scaled by 1/32) sharing one code,
+    decoded in ONE launch (DFloat11 Abstract, item (iii))."""
+    g = synth.transformer_block(0)[0]
+    xs = [t.bits[: t.bits.size // 32 + 77 * i] for i, t in enumerate(g.tensors)]
+    cb = df11.df11_build_codebook("bf16", xs)
+    blobs = [df11.df11_encode(cb, x) for x in xs]
+    outs, err, guards = decode_gpu(df11, blobs)
+    assert err == 0 and guards
+    lengths = cb.lengths()
+    for x, out in zip(xs, outs):
+        assert np.array_equal(out, x)
+        assert np.array_equal(out, oracle_mod.decompress(oracle_mod.compress(x, "bf16", lengths=lengths)))
+
+
+def test_mixed_codes_rejected(df11):
+    a = synth.single_matrix(0)[0].tensors[0].bits[:5000]
+    b = synth.heavy_tail_matrix(0)[0].tensors[0].bits[:5000]
+    ba = df11.df11_encode(df11.df11_build_codebook("bf16", [a]), a)
+    bb = df11.df11_encode(df11.df11_build_codebook("bf16", [b]), b)
+    df11.upload(ba)
+    df11.upload(bb)
+    outs = [df11.empty_output(ba), df11.empty_output(bb)]
+    with pytest.raises(df11.Df11Error) as e:
+        df11.df11_decode([ba, bb], [o.data_ptr() for o in outs])
+    assert e.value.status == df11.DF11_EINVAL
+
+
+def test_unbound_and_misaligned_rejected(df11):
+    x = synth.single_matrix(0)[0].tensors[0].bits[:5000]
+    blob = df11.df11_encode(df11.df11_build_codebook("bf16", [x]), x)
+    out = df11.empty_output(blob)
+    with pytest.raises(df11.Df11Error):
+        df11.df11_decode([blob], [out.data_ptr()])  # not bound yet
+    df11.upload(blob)
+    with pytest.raises(df11.Df11Error):
+        df11.df11_decode([blob], [out.data_ptr() + 2])  # 2-byte aligned destination
+
+
+def test_deterministic_and_stream(df11):
+    x = synth.heavy_tail_matrix(2)[0].tensors[0].bits[:3000001]
+    blob = df11.df11_encode(df11.df11_build_codebook("bf16", [x]), x)
+    s = torch.cuda.Stream()
+    a, ea, _ = decode_gpu(df11, [blob], stream=s)
+    b, eb, _ = decode_gpu(df11, [blob])
+    assert ea == eb == 0
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[0], x)
+
+
+def test_corrupted_device_data_sets_error_flag(df11):
+    """Damaged auxiliary data on the device: the kernel flags it and writes
+    nothing outside the destination (guard bytes intact)."""
+    x = synth.single_matrix(4)[0].tensors[0].bits
+    blob = df11.df11_encode(df11.df11_build_codebook("bf16", [x]), x)
+    import struct
+    n = blob.info().device_bytes
+    img = np.zeros(n, np.uint8)
+    df11.df11_blob_device_image(blob, img.ctypes.data, n)
+    out_off_at = struct.unpack_from("<Q", img.tobytes(), 56 + 8 * 4)[0]
+    gaps_at = struct.unpack_from("<Q", img.tobytes(), 56 + 8 * 3)[0]
+    for what in ("out_off", "gap"):
+        bad = img.copy()
+        if what == "out_off":
+            bad[out_off_at + 8 * 3: out_off_at + 8 * 4] = np.frombuffer(struct.pack("<Q", 10 ** 12), np.uint8)
+        else:
+            bad[gaps_at + 5] = (int(bad[gaps_at + 5]) + 3) % 32
+        dev = torch.from_numpy(bad).cuda()
+        df11.df11_blob_bind(blob, dev.data_ptr(), n, keep=dev)
+        guard = 64
+        nbytes = 2 * x.size
+        buf = torch.full((nbytes + 2 * guard,), 0xA5, dtype=torch.uint8, device="cuda")
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        df11.df11_decode([blob], [buf.data_ptr() + guard], err.data_ptr())
+        torch.cuda.synchronize()
+        e = int(err.item())
+        g = buf.cpu().numpy()
+        assert (g[:guard] == 0xA5).all() and (g[guard + nbytes:] == 0xA5).all()
+        if what == "out_off":
+            assert e & df11.DEV_ERR_AUX
+        # a shifted gap is caught when it changes the tile's code count; when
+        # the parse resynchronises to the same count the output is wrong but
+        # still inside the destination, which is what is checked above
+
+
+def test_decode_host_end_to_end(df11):
+    """Host image in pinned memory -> device -> decode -> host output, one call."""
+    x = synth.single_matrix(5)[0].tensors[0].bits
+    blob = df11.df11_encode(df11.df11_build_codebook("bf16", [x]), x)
+    n = blob.info().device_bytes
+    himg = torch.empty(n, dtype=torch.uint8, pin_memory=True)
+    df11.df11_blob_device_image(blob, himg.data_ptr(), n)
+    dimg = torch.empty(n + 256, dtype=torch.uint8, device="cuda")
+    dptr = dimg.data_ptr() + (-dimg.data_ptr()) % 256
+    dout = torch.empty(2 * x.size, dtype=torch.uint8, device="cuda")
+    hout = torch.empty(2 * x.size, dtype=torch.uint8, pin_memory=True)
+    s = torch.cuda.current_stream()
+    df11.df11_decode_host([blob], [himg.data_ptr()], [dptr], [dout.data_ptr()], [hout.data_ptr()],
+                          None, s.cuda_stream)
+    s.synchronize()
+    assert np.array_equal(hout.numpy().view(np.uint16), x)
+
+
+def test_launch_shape_is_persistent(df11):
+    x = synth.heavy_tail_matrix(0)[0].tensors[0].bits
+    blob = df11.df11_encode(df11.df11_build_codebook("bf16", [x]), x)
+    df11.upload(blob)
+    grid, block, smem = df11.df11_decode_launch_shape([blob])
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert block == 256 + 32
+    assert grid == min(blob.info().n_tiles, grid) and grid % sms == 0 or grid == blob.info().n_tiles
+    assert 0 < smem <= 227 * 1024

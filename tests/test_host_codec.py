@@ -1,0 +1,261 @@
+"""Host side of the library (code construction, encoder, container, device
+image) against the CPU oracle and against independent recomputation.  No GPU
+needed: nothing here launches a kernel."""
+import ctypes
+import struct
+
+import numpy as np
+import pytest
+
+from entropy_decoding_b200 import synth
+
+
+@pytest.fixture(scope="module")
+def df11():
+    from entropy_decoding_b200 import build
+    build.build()
+    from entropy_decoding_b200 import df11 as mod
+    return mod
+
+
+def test_library_exports_every_declared_symbol(df11):
+    names = df11.exported_names()
+    assert len(names) >= 20
+    lib = ctypes.CDLL(df11.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert df11.df11_version() == 10000
+
+
+def _cases():
+    return {
+        "normal": ("bf16", lambda: synth.single_matrix(0)[0].tensors[0].bits[:400000]),
+        "heavy": ("bf16", lambda: synth.heavy_tail_matrix(0)[0].tensors[0].bits[:600000]),
+        "all_bf16": ("bf16", synth.all_bf16_patterns),
+        "single": ("bf16", lambda: synth.constant_bf16(50000, 1.0)),
+        "fib": ("bf16", lambda: synth.powers_of_two_bf16(synth.fibonacci_counts(28), first_exponent=-24)),
+        "random": ("bf16", lambda: synth.random_bits(123457, "bf16", 4)),
+        "tiny": ("bf16", lambda: synth.random_bits(9, "bf16", 5)),
+        "e4m3": ("e4m3", lambda: synth.normal_e4m3(np.random.SeedSequence(1), 300001)),
+        "e4m3_all": ("e4m3", synth.all_e4m3_patterns),
+    }
+
+
+@pytest.mark.parametrize("case", list(_cases()))
+def test_lengths_and_sections_match_oracle(df11, oracle_mod, case):
+    dt, make = _cases()[case]
+    x = make()
+    cb = df11.df11_build_codebook(dt, [x])
+    want = oracle_mod.build_lengths([x], dt)
+    assert np.array_equal(cb.lengths(), want)
+    for chunk_bits, tile_threads in [(128, 256), (64, 512), (256, 128)]:
+        blob = df11.df11_encode(cb, x, chunk_bits, tile_threads)
+        o = oracle_mod.compress(x, dt, lengths=want, chunk_bits=chunk_bits, tile_threads=tile_threads)
+        info = blob.info()
+        s = blob.sections()
+        assert info.total_bits == o.total_bits
+        assert info.n_tiles == o.n_tiles
+        assert info.max_span == o.max_span
+        assert np.array_equal(s["stream"], o.stream)
+        assert np.array_equal(s["plane"], o.plane)
+        assert np.array_equal(s["gaps"], o.gaps)
+        assert np.array_equal(s["out_off"], o.out_off)
+
+
+def test_shared_codebook_over_a_group(df11, oracle_mod):
+    g = synth.transformer_block(0)[0]
+    xs = [t.bits[: 100000 + 1000 * i] for i, t in enumerate(g.tensors)]
+    cb = df11.df11_build_codebook("bf16", xs)
+    assert np.array_equal(cb.lengths(), oracle_mod.build_lengths(xs, "bf16"))
+
+
+def test_length_limit_matches_oracle(df11, oracle_mod):
+    x = synth.powers_of_two_bf16(synth.fibonacci_counts(30), first_exponent=-25)
+    for lim in (32, 20, 12, 9):
+        cb = df11.df11_build_codebook("bf16", [x], lim)
+        want = oracle_mod.build_lengths([x], "bf16", lim)
+        assert np.array_equal(cb.lengths(), want), lim
+        assert cb.lengths().max() <= lim
+
+
+def test_fibonacci_34_reaches_32_bit_codes(df11, oracle_mod):
+    """The 34-symbol Fibonacci histogram (unlimited depth 33) through the
+    library: package-merge lengths equal the oracle's, longest code 32."""
+    counts = np.zeros(256, np.uint64)
+    counts[100:134] = synth.fibonacci_counts(34)
+    want = oracle_mod.code_lengths(counts, 256, 32)
+    assert want.max() == 32
+    cb = df11.df11_codebook_from_lengths("bf16", want)
+    assert np.array_equal(cb.lengths(), want)
+
+
+def _image_layout(img: bytes):
+    magic = img[:8]
+    assert magic == b"DF11IMG1"
+    dtype, chunk, tile, n_luts = struct.unpack_from("<4I", img, 8)
+    n, total, n_tiles, max_span = struct.unpack_from("<4Q", img, 24)
+    keys = ["meta", "syms", "lut", "gaps", "out_off", "stream", "plane", "total"]
+    lay = dict(zip(keys, struct.unpack_from("<8Q", img, 56)))
+    return dict(dtype=dtype, chunk=chunk, tile=tile, n_luts=n_luts, n=n, total_bits=total, n_tiles=n_tiles,
+                max_span=max_span, **lay)
+
+
+def _image(df11, blob):
+    n = blob.info().device_bytes
+    buf = np.zeros(n, np.uint8)
+    df11.df11_blob_device_image(blob, buf.ctypes.data, n)
+    return buf
+
+
+def _prefix_decoder(lengths, codes):
+    table = {}
+    for s, l in enumerate(lengths):
+        if l:
+            table[(int(l), int(codes[s]))] = s
+    return table
+
+
+def _first_code(table, bits, nbits):
+    """(symbol, length) of the code at the top of a `nbits`-bit value, or None."""
+    for l in range(1, nbits + 1):
+        v = bits >> (nbits - l)
+        if (l, v) in table:
+            return table[(l, v)], l
+    return None
+
+
+@pytest.mark.parametrize("case", ["normal", "heavy", "fib", "single", "e4m3"])
+def test_decode_tables_match_independent_prefix_decode(df11, oracle_mod, case):
+    """The device image's 12-bit multi-symbol table and hierarchical 256-entry
+    tables, checked entry by entry against a dictionary prefix decode over the
+    oracle's canonical codes."""
+    dt, make = _cases()[case]
+    x = make()
+    cb = df11.df11_build_codebook(dt, [x])
+    blob = df11.df11_encode(cb, x)
+    img = _image(df11, blob)
+    lay = _image_layout(img.tobytes()[:128])
+    lengths = oracle_mod.build_lengths([x], dt)
+    codes = oracle_mod.canonical_codes(lengths)
+    table = _prefix_decoder(lengths, codes)
+    meta = img[lay["meta"]:lay["meta"] + 8192].view(np.uint16)
+    syms = img[lay["syms"]:lay["syms"] + 16384].view(np.uint32)
+    for v in range(4096):
+        pos, got = 0, []
+        while len(got) < 4:
+            r = _first_code(table, v & ((1 << (12 - pos)) - 1), 12 - pos) if pos < 12 else None
+            if r is None:
+                break
+            got.append(r[0])
+            pos += r[1]
+        if not got:
+            assert meta[v] == 0x40, v
+        else:
+            assert meta[v] == pos | (len(got) << 8), v
+            assert [(int(syms[v]) >> (8 * i)) & 0xFF for i in range(len(got))] == got
+    lut = img[lay["lut"]:lay["lut"] + lay["n_luts"] * 512].view(np.uint16)
+    rng = np.random.default_rng(0)
+    wins = list(rng.integers(0, 2 ** 32, 3000, dtype=np.uint64))
+    for s, l in enumerate(lengths):  # every codeword at least once, random tail
+        if l:
+            wins.append((int(codes[s]) << (32 - int(l))) | int(rng.integers(0, 2 ** (32 - int(l)))))
+    for win in wins:
+        win = int(win)
+        e = int(lut[win >> 24])
+        lvl = 1
+        while e & 0x8000 and lvl < 4:
+            e = int(lut[(e & 0x7FFF) * 256 + ((win >> (24 - 8 * lvl)) & 0xFF)])
+            lvl += 1
+        r = _first_code(table, win, 32)
+        if r is None:
+            assert e & 0x4000
+        else:
+            assert not e & 0xC000
+            assert (e & 0xFF, (e >> 8) & 0x3F) == r
+
+
+def test_serialize_roundtrip_and_size(df11, oracle_mod):
+    x = synth.single_matrix(2)[0].tensors[0].bits
+    cb = df11.df11_build_codebook("bf16", [x])
+    blob = df11.df11_encode(cb, x)
+    data = df11.df11_serialize(blob)
+    info = blob.info()
+    assert len(data) == info.serialized_bytes
+    # near the pages' ~70% of BF16 ("70% Size", DFloat11 title / Abstract)
+    assert 0.62 < info.serialized_bytes / info.uncompressed_bytes < 0.72
+    b2 = df11.df11_deserialize(data)
+    s1, s2 = blob.sections(), b2.sections()
+    for k in s1:
+        assert np.array_equal(s1[k], s2[k])
+    assert np.array_equal(b2.lengths(), blob.lengths())
+    assert df11.df11_serialize(b2) == data
+
+
+def test_deserialize_rejects_corruption(df11):
+    x = synth.heavy_tail_matrix(0)[0].tensors[0].bits[:200000]
+    cb = df11.df11_build_codebook("bf16", [x])
+    blob = df11.df11_encode(cb, x)
+    good = bytearray(df11.df11_serialize(blob))
+    info = blob.info()
+
+    def rejected(buf):
+        with pytest.raises(df11.Df11Error) as e:
+            df11.df11_deserialize(bytes(buf))
+        assert e.value.status == df11.DF11_ECORRUPT
+
+    rejected(good[:-16])                       # truncated
+    bad = bytearray(good); bad[0] ^= 1; rejected(bad)          # magic
+    bad = bytearray(good); bad[8] = 9; rejected(bad)           # version
+    bad = bytearray(good); bad[16] ^= 1; rejected(bad)         # element count
+    lengths_off = 64
+    bad = bytearray(good); bad[lengths_off + 120] = 1; rejected(bad)  # Kraft sum > 1
+    gaps_off = (64 + 256 + 15) // 16 * 16
+    bad = bytearray(good); bad[gaps_off + 3] = 200; rejected(bad)     # gap out of range
+    oo = (gaps_off + info.gaps_bytes + 15) // 16 * 16
+    bad = bytearray(good); struct.pack_into("<Q", bad, oo + 8 * 2, 0); rejected(bad)  # out_off not monotone
+    bad = bytearray(good); struct.pack_into("<Q", bad, oo, 5); rejected(bad)          # out_off[0] != 0
+    with pytest.raises(df11.Df11Error):
+        df11.df11_deserialize(b"")
+
+
+def test_encode_rejects_uncovered_symbol(df11):
+    x = synth.single_matrix(0)[0].tensors[0].bits[:1000]
+    cb = df11.df11_build_codebook("bf16", [x])
+    y = x.copy()
+    y[5] = 0x7F80  # +inf: exponent 255, absent from the code
+    with pytest.raises(df11.Df11Error) as e:
+        df11.df11_encode(cb, y)
+    assert e.value.status == df11.DF11_EINVAL
+
+
+def test_invalid_arguments(df11):
+    with pytest.raises(df11.Df11Error):
+        df11.df11_build_codebook("bf16", [np.zeros(4, np.uint16)], 40)
+    with pytest.raises(df11.Df11Error):
+        df11.df11_codebook_from_lengths("bf16", np.full(256, 1, np.uint8))  # Kraft sum 128
+    cb = df11.df11_build_codebook("bf16", [synth.random_bits(100, "bf16")])
+    with pytest.raises(df11.Df11Error):
+        df11.df11_encode(cb, synth.random_bits(100, "bf16"), chunk_bits=96)
+    assert df11.df11_layout_supported("bf16", 128, 256)
+    assert df11.df11_layout_supported("e4m3", 128, 256)
+    assert not df11.df11_layout_supported("bf16", 96, 256)
+
+
+def test_device_image_layout(df11):
+    x = synth.random_bits(300000, "bf16", 9)
+    cb = df11.df11_build_codebook("bf16", [x])
+    blob = df11.df11_encode(cb, x)
+    img = _image(df11, blob)
+    lay = _image_layout(img.tobytes()[:128])
+    info = blob.info()
+    assert lay["total"] == info.device_bytes == img.size
+    for k in ("meta", "syms", "lut", "gaps", "out_off", "stream", "plane"):
+        assert lay[k] % 256 == 0
+    s = blob.sections()
+    tile_bytes = info.chunk_bits // 8 * info.tile_threads
+    stream = img[lay["stream"]:lay["plane"]]
+    assert np.array_equal(stream[: s["stream"].size], s["stream"])
+    assert stream.size >= info.n_tiles * tile_bytes + 16
+    assert not stream[s["stream"].size:].any()
+    assert np.array_equal(img[lay["plane"]:lay["plane"] + info.plane_bytes], s["plane"])
+    assert lay["total"] - lay["plane"] >= info.plane_bytes + 32
