@@ -1,0 +1,518 @@
+#!/usr/bin/env python
+"""Decode throughput of libdf11 on B200: decompressed BF16 GB/s, fraction of
+the HBM roofline, and compression ratio, on seeded synthetic weights shaped
+like a whole Llama-3-8B model (32 transformer blocks + embedding + LM head,
+8,029,995,008 BF16 weights, one codebook per block, one decode launch per
+block, 34 launches back to back per step).
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--workload ...]
+
+One step = one decode of the whole model (every launch of the hot path) with
+the compressed images resident in HBM.  Inputs (10.8 GB compressed, 16 GB
+decoded) are far larger than the 126 MB L2, so no flush is needed.  Rank 0
+prints one JSON line.  Multi-GPU (torchrun): every rank decodes its own
+replica of the model (weak scaling, no collective on the data path); the
+timed region is bracketed by barriers and the reported time is the max over
+ranks.  `--impl reference` times the CPU oracle decoder (the method written
+out plainly, single-threaded) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from entropy_decoding_b200 import synth  # noqa: E402
+
+METRIC = "decompressed BF16 GB/s"
+HBM_FALLBACK_GBS = 6650.0
+KERNEL_SRC = os.path.join(ROOT, "entropy_decoding_b200", "csrc", "decode.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", choices=["whole_model", "block", "e4m3"], default="whole_model")
+    p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--cpu-seconds", type=float, default=10.0)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu", action="store_true")
+    p.add_argument("--chunk-bits", type=int, default=128)
+    p.add_argument("--tile-threads", type=int, default=256)
+    p.add_argument("--chunks-per-thread", type=int, default=0, help="decode launch option (0 = library default)")
+    p.add_argument("--ctas-per-sm", type=int, default=0, help="decode launch option (0 = as many as fit)")
+    return p.parse_args()
+
+
+# ------------------------------------------------------------------ workload description
+
+def workload_config(name: str) -> dict:
+    if name == "whole_model":
+        n = sum(s[0] * s[1] for _, ts in synth.whole_model_specs() for _, s, _ in ts)
+        return {"workload": "whole Llama-3-8B-shaped model: 32 blocks (q,k,v,o,gate,up,down) + embedding + "
+                            "LM head, per-block codebooks, 34 decode launches per step",
+                "n_weights": n, "launches_per_step": 34, "dtype_in": "bf16"}
+    if name == "block":
+        n = sum(s[0] * s[1] for _, s in synth.BLOCK_SHAPES)
+        return {"workload": "one Llama-3-8B-shaped transformer block, shared codebook, 1 launch",
+                "n_weights": n, "launches_per_step": 1, "dtype_in": "bf16"}
+    return {"workload": "8192x28672 FP8 E4M3, N(0,0.02) scaled to E4M3 range, 1 launch",
+            "n_weights": 8192 * 28672, "launches_per_step": 1, "dtype_in": "e4m3"}
+
+
+def full_config(args, world: int) -> dict:
+    """The `config` object of the JSON line (identical for both arms)."""
+    cfg = workload_config(args.workload)
+    out_gb = cfg["n_weights"] * (2 if cfg["dtype_in"] == "bf16" else 1) / 1e9
+    return {**cfg, "seed": args.seed, "chunk_bits": args.chunk_bits, "tile_threads": args.tile_threads,
+            "chunks_per_thread": args.chunks_per_thread or 2, "ctas_per_sm": args.ctas_per_sm or "max",
+            "l2": f"no flush: inputs larger than L2 (decoded output {out_gb:.1f} GB, compressed images "
+                  f"about 0.68x that, vs 126 MB L2)",
+            "parallelism": f"replicas x{world} (each GPU decodes its own copy)"}
+
+
+def group_count(name: str) -> int:
+    return len(synth.whole_model_specs()) if name == "whole_model" else 1
+
+
+def make_group(name: str, seed: int, gi: int) -> synth.Group:
+    if name == "whole_model":
+        return synth.whole_model_group(seed, gi)
+    if name == "block":
+        return synth.transformer_block(seed)[0]
+    return synth.e4m3_matrix(seed)[0]
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="df11_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) == len(self.FIELDS):
+                    rows.append(parts)
+        os.unlink(self.path)
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max((float(r[2]) for r in rows if r[2].replace(".", "").isdigit()), default=None)}
+
+
+# ------------------------------------------------------------------ helpers
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, copy bandwidth)"
+    except (OSError, KeyError, ValueError):
+        return HBM_FALLBACK_GBS, "fallback (profiling recipe: 6.65 TB/s)"
+
+
+def kernel_hash() -> str:
+    with open(KERNEL_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def traffic_per_weight():
+    """DRAM bytes per weight from a committed ncu capture of the current
+    kernel source, or None when the kernel changed since."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None, None
+    if t.get("kernel_sha256_16") != kernel_hash():
+        return None, "stale"
+    return float(t["dram_bytes_per_weight"]), t.get("source")
+
+
+def host_threads(world: int) -> int:
+    try:
+        c = len(os.sched_getaffinity(0))
+    except AttributeError:
+        c = os.cpu_count() or 1
+    return max(1, c // max(world, 1))
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def oracle_decode_sample(groups_host, seconds: float):
+    """Times the CPU oracle decoder (single-threaded) on whole tensors of the
+    workload, in order, until `seconds` of decode time have accumulated.
+    The oracle decodes the same compressed stream the GPU decodes."""
+    import oracle
+    oracle.build()
+    done_w, spent, names = 0, 0.0, []
+    for gname, tensors in groups_host:
+        for tname, dt, n, lengths, sec in tensors:
+            nsym = 256 if dt == "bf16" else 16
+            t0 = time.perf_counter()
+            exps = oracle.decode(sec["stream"], int(sec["total_bits"]), lengths[:nsym], 0, n)
+            oracle.merge(exps, sec["plane"], n, dt)
+            spent += time.perf_counter() - t0
+            done_w += n
+            names.append(f"{gname}.{tname}")
+            if spent >= seconds:
+                return done_w, spent, names
+    return done_w, spent, names
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return
+    cfg = full_config(args, world)
+    gi = 1 if args.workload == "whole_model" else 0
+    g = make_group(args.workload, args.seed, gi)
+    from entropy_decoding_b200 import df11
+    import oracle
+    oracle.build()
+    t = g.tensors[0]
+    dt = "bf16" if t.bits.dtype == np.uint16 else "e4m3"
+    cb = df11.df11_build_codebook(dt, [x.bits for x in g.tensors])
+    blob = df11.df11_encode(cb, t.bits)
+    sec = blob.sections()
+    info = blob.info()
+    lengths = cb.lengths()
+    n = t.bits.size
+
+    def step():
+        exps = oracle.decode(sec["stream"], int(info.total_bits), lengths, 0, n)
+        return oracle.merge(exps, sec["plane"], n, dt)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        out = step()
+    el = time.perf_counter() - t0
+    assert np.array_equal(out, t.bits)
+    out_bytes = n * (2 if dt == "bf16" else 1)
+    value = out_bytes * args.steps / el / 1e9
+    sample = (f"{g.name}.{t.name} ({n} weights) per step, decoded by the single-threaded CPU oracle "
+              f"from the library's compressed stream")
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u32", "data": "synthetic",
+            "config": cfg, "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+    from entropy_decoding_b200 import df11
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    cfg = workload_config(args.workload)
+    threads = host_threads(world)
+
+    # ---- build: generate, encode, upload, one group at a time (host memory stays bounded)
+    t_setup = time.time()
+    groups = []  # (name, blobs, dsts, algo bytes, n weights, out bytes)
+    host_for_cpu = []
+    samples = []  # (group index, tensor index, positions, values)
+    out_bytes_total = 0
+    ser_total = 0
+    dev_total = 0
+    uncompressed_total = 0
+    max_len = 0
+    tensors_meta = []
+    rng = np.random.default_rng(12345)
+    for gi in range(group_count(args.workload)):
+        g = make_group(args.workload, args.seed, gi)
+        dt = "bf16" if g.tensors[0].bits.dtype == np.uint16 else "e4m3"
+        cb = df11.df11_build_codebook(dt, [t.bits for t in g.tensors])
+        blobs = [df11.df11_encode(cb, t.bits, args.chunk_bits, args.tile_threads, threads) for t in g.tensors]
+        for ti, (t, b) in enumerate(zip(g.tensors, blobs)):
+            pos = np.unique(np.concatenate([np.arange(min(4096, t.bits.size)),
+                                            np.arange(max(0, t.bits.size - 4096), t.bits.size),
+                                            rng.integers(0, t.bits.size, 32768)]))
+            samples.append((gi, ti, pos, t.bits[pos].copy()))
+            i = b.info()
+            ser_total += i.serialized_bytes
+            dev_total += i.device_bytes
+            uncompressed_total += i.uncompressed_bytes
+            max_len = max(max_len, i.max_code_len)
+            tensors_meta.append(i)
+        if rank == 0 and not args.no_cpu and gi in (1, 2, 3):
+            lengths = cb.lengths()
+            host_for_cpu.append((g.name, [(t.name, dt, t.bits.size, lengths, {**b.sections(),
+                                 "total_bits": b.info().total_bits}) for t, b in zip(g.tensors, blobs)]))
+        groups.append([g.name, blobs, dt])
+        del g
+    setup_s = time.time() - t_setup
+
+    # device images (torch-owned memory) and one output buffer, 256-byte aligned slices
+    with torch.cuda.stream(stream):
+        for _, blobs, _ in groups:
+            for b in blobs:
+                df11.upload(b, stream)
+        sizes = []
+        for _, blobs, dt in groups:
+            sizes.append([b.info().n_elems * (2 if dt == "bf16" else 1) for b in blobs])
+        total_out = sum(((s + 255) // 256) * 256 for ss in sizes for s in ss)
+        out = torch.empty(total_out, dtype=torch.uint8, device=dev)
+        base = out.data_ptr()
+        off = 0
+        for gi, (ss, grp) in enumerate(zip(sizes, groups)):
+            dsts = []
+            for s in ss:
+                dsts.append((base + off, off, s))
+                off += ((s + 255) // 256) * 256
+            grp.append(dsts)
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream.synchronize()
+    out_bytes_total = sum(sum(ss) for ss in sizes)
+
+    # algorithmic bytes per launch: compressed sections read + output written
+    algo = []
+    k = 0
+    for name, blobs, dt, dsts in groups:
+        a = 0
+        for b in blobs:
+            i = tensors_meta[k]
+            k += 1
+            a += i.stream_bytes + i.plane_bytes + i.gaps_bytes + i.out_off_bytes + i.uncompressed_bytes
+        algo.append(a)
+
+    def one_step(events=None):
+        for gi, (name, blobs, dt, dsts) in enumerate(groups):
+            if events is not None:
+                events[gi][0].record(stream)
+            df11.df11_decode_ex(blobs, [d[0] for d in dsts], err.data_ptr(), stream.cuda_stream,
+                                args.chunks_per_thread, args.ctas_per_sm)
+            if events is not None:
+                events[gi][1].record(stream)
+
+    for _ in range(args.warmup):
+        one_step()
+    stream.synchronize()
+
+    ev = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+           for _ in groups] for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                          else local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)  # let the sampler attach before the region
+    start.record(stream)
+    for s_ in range(args.steps):
+        one_step(ev[s_])
+    end.record(stream)
+    end.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    elapsed_ms = start.elapsed_time(end)
+    launch_ms = [[e[0].elapsed_time(e[1]) for e in step] for step in ev]
+    if world > 1:
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    # ---- correctness outside the timed region: error word + sampled positions
+    e = int(err.item())
+    host_out = {}
+    bad = 0
+    for gi, ti, pos, vals in samples:
+        name, blobs, dt, dsts = groups[gi]
+        ptr, o, s = dsts[ti]
+        if dt == "bf16":
+            v = out[o:o + s].view(torch.int16)
+            got = v[torch.from_numpy(pos).to(dev)].cpu().numpy().view(np.uint16)
+        else:
+            got = out[o:o + s][torch.from_numpy(pos).to(dev)].cpu().numpy()
+        bad += int((got != vals).sum())
+    assert e == 0, f"device error word {e}"
+    assert bad == 0, f"{bad} sampled outputs differ from the source weights"
+
+    # ---- end to end through the C-ABI with host buffers (pinned)
+    e2e = None
+    if not args.no_e2e:
+        himgs = []
+        for name, blobs, dt, dsts in groups:
+            hs = []
+            for b in blobs:
+                nb = b.info().device_bytes
+                h = torch.empty(nb, dtype=torch.uint8, pin_memory=True)
+                df11.df11_blob_device_image(b, h.data_ptr(), nb)
+                hs.append(h)
+            himgs.append(hs)
+        max_group_out = max(sum(((s + 255) // 256) * 256 for s in ss) for ss in sizes)
+        hout = torch.empty(max_group_out, dtype=torch.uint8, pin_memory=True)
+        h2d = sum(h.numel() for hs in himgs for h in hs)
+        d2h = out_bytes_total
+
+        def e2e_step():
+            for gi, (name, blobs, dt, dsts) in enumerate(groups):
+                hp = []
+                o = 0
+                for (_, _, s) in dsts:
+                    hp.append(hout.data_ptr() + o)
+                    o += ((s + 255) // 256) * 256
+                dimg = [b._keep.data_ptr() + (-b._keep.data_ptr()) % 256 for b in blobs]
+                df11.df11_decode_host(blobs, [h.data_ptr() for h in himgs[gi]], dimg, [d[0] for d in dsts], hp,
+                                      err.data_ptr(), stream.cuda_stream)
+
+        e2e_step()
+        stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        s1.record(stream)
+        s1.synchronize()
+        e2e_ms = s0.elapsed_time(s1) / args.e2e_steps
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        assert int(err.item()) == 0
+        e2e = {"value": world * out_bytes_total / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+               "path": "df11_decode_host: pinned host image -> H2D -> decode launch -> D2H of every output"}
+        del himgs, hout
+
+    # ---- CPU oracle baseline (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu and host_for_cpu:
+        w, sec, names = oracle_decode_sample(host_for_cpu, args.cpu_seconds)
+        cpu = {"value": 2 * w / sec / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"{w} weights ({len(names)} whole tensors from blocks 0-2, {names[0]} ... {names[-1]}), "
+                         f"single-threaded bit-by-bit oracle decode + field merge, {sec:.1f} s"}
+
+    if rank != 0:
+        return
+    ms_per_step = elapsed_ms / args.steps
+    value = world * out_bytes_total * args.steps / (elapsed_ms / 1e3) / 1e9
+    per_launch = np.array(launch_ms)  # steps x groups
+    tot_launch_s = per_launch.sum() / 1e3
+    algo_step = float(sum(algo))
+    achieved = algo_step * args.steps / tot_launch_s / 1e9
+    peak, peak_src = hbm_peak()
+    tpw, tsrc = traffic_per_weight()
+    n_w = cfg["n_weights"]
+    traffic = tpw * n_w / len(groups) if tpw is not None else None
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u32", "data": "synthetic (seeded N(0,1/sqrt(fan_in)) / N(0,0.02) weights, "
+                                                     "random init, no trained checkpoint)",
+        "config": full_config(args, world),
+        "weights_per_s": world * n_w * args.steps / (elapsed_ms / 1e3),
+        "compression_ratio": ser_total / uncompressed_total,
+        "bits_per_weight": 8 * ser_total / n_w,
+        "max_code_len": max_len,
+        "hbm_roofline_frac": achieved / peak,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": peak_src,
+                     "kernel": f"decode_kernel<{'bf16' if cfg['dtype_in'] == 'bf16' else 'e4m3'},"
+                               f"{args.chunk_bits},{args.tile_threads}>",
+                     "algorithmic_bytes_per_launch": algo_step / len(groups),
+                     "launch_ms_mean": float(per_launch.mean()),
+                     "launch_ms_by_group": {"first": float(per_launch[:, 0].mean()),
+                                            "block_mean": float(per_launch[:, 1:-1].mean()) if len(groups) > 2
+                                            else None,
+                                            "last": float(per_launch[:, -1].mean())},
+                     "traffic_source": tsrc},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": len(groups) * args.steps,
+        "clocks": clk,
+        "setup_s": setup_s,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -6,7 +6,7 @@
 #include <cstring>
 #include <new>
 
-#include "../../include/df11.h"
+#include "df11.h"
 #include "codec.h"
 #include "launch.h"
 
@@ -226,16 +226,27 @@ df11_status df11_blob_upload(df11_blob *blob, void *dev_dst, uint64_t cap, df11_
     return DF11_OK;
 }
 
-df11_status df11_decode(const df11_blob *const *blobs, void *const *dst_dev, int n_blobs, int *dev_err_flag,
-                        df11_stream stream) {
+df11_status df11_decode_ex(const df11_blob *const *blobs, void *const *dst_dev, int n_blobs, int *dev_err_flag,
+                           df11_stream stream, const df11_decode_opts *opts) {
     if (!blobs || !dst_dev || n_blobs < 1 || n_blobs > df11::kMaxTensorsPerLaunch) return DF11_EINVAL;
     const df11::Blob *bs[df11::kMaxTensorsPerLaunch];
     for (int i = 0; i < n_blobs; ++i) {
         if (!blobs[i]) return DF11_EINVAL;
         bs[i] = &blobs[i]->b;
     }
-    return from_launch(df11::launch_decode(bs, dst_dev, n_blobs, dev_err_flag,
+    df11::DecodeOptions o;
+    if (opts) {
+        o.chunks_per_thread = opts->chunks_per_thread;
+        o.ctas_per_sm = opts->ctas_per_sm;
+        if (o.chunks_per_thread < 0 || o.ctas_per_sm < 0) return DF11_EINVAL;
+    }
+    return from_launch(df11::launch_decode(bs, dst_dev, n_blobs, dev_err_flag, o,
                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
+df11_status df11_decode(const df11_blob *const *blobs, void *const *dst_dev, int n_blobs, int *dev_err_flag,
+                        df11_stream stream) {
+    return df11_decode_ex(blobs, dst_dev, n_blobs, dev_err_flag, stream, nullptr);
 }
 
 df11_status df11_decode_host(df11_blob *const *blobs, const void *const *host_images, void *const *dev_images,
@@ -268,6 +279,11 @@ df11_status df11_decode_host(df11_blob *const *blobs, const void *const *host_im
 
 df11_status df11_decode_launch_shape(const df11_blob *const *blobs, int n_blobs, int *grid, int *block,
                                      int *smem_bytes) {
+    return df11_decode_launch_shape_ex(blobs, n_blobs, nullptr, grid, block, smem_bytes);
+}
+
+df11_status df11_decode_launch_shape_ex(const df11_blob *const *blobs, int n_blobs, const df11_decode_opts *opts,
+                                        int *grid, int *block, int *smem_bytes) {
     if (!blobs || n_blobs < 1 || n_blobs > df11::kMaxTensorsPerLaunch) return DF11_EINVAL;
     const df11::Blob *bs[df11::kMaxTensorsPerLaunch];
     for (int i = 0; i < n_blobs; ++i) {
@@ -275,7 +291,12 @@ df11_status df11_decode_launch_shape(const df11_blob *const *blobs, int n_blobs,
         bs[i] = &blobs[i]->b;
     }
     df11::LaunchShape sh;
-    df11::LaunchStatus st = df11::decode_launch_shape(bs, n_blobs, &sh);
+    df11::DecodeOptions o;
+    if (opts) {
+        o.chunks_per_thread = opts->chunks_per_thread;
+        o.ctas_per_sm = opts->ctas_per_sm;
+    }
+    df11::LaunchStatus st = df11::decode_launch_shape(bs, n_blobs, o, &sh);
     if (st != df11::LaunchStatus::kOk) return from_launch(st);
     if (grid) *grid = sh.grid;
     if (block) *block = sh.block;

@@ -220,7 +220,7 @@ bool build_lut(const uint8_t *lengths, const uint32_t *codes, int nsym, std::vec
 // Multi-symbol table over 12-bit windows, from a length-indexed canonical
 // decoder: a code of length l matches when the next l bits fall in the range
 // of length-l codes.
-void build_multi(const uint8_t *lengths, const uint32_t *codes, int nsym, std::vector<uint16_t> &meta,
+void build_multi(const uint8_t *lengths, const uint32_t *codes, int nsym, std::vector<uint32_t> &meta,
                  std::vector<uint32_t> &syms) {
     int lo_sym[kMaxCodeLen + 1];
     uint32_t first[kMaxCodeLen + 1], cnt[kMaxCodeLen + 1] = {};
@@ -245,7 +245,7 @@ void build_multi(const uint8_t *lengths, const uint32_t *codes, int nsym, std::v
     syms.assign(kMultiEntries, 0);
     for (uint32_t v = 0; v < static_cast<uint32_t>(kMultiEntries); ++v) {
         int pos = 0, k = 0;
-        uint32_t packed = 0;
+        uint32_t packed = 0, starts = 0;
         while (k < kMultiMaxSyms) {
             int found = -1, flen = 0;
             for (int l = 1; l <= kMultiBits - pos; ++l) {
@@ -258,12 +258,13 @@ void build_multi(const uint8_t *lengths, const uint32_t *codes, int nsym, std::v
                 }
             }
             if (found < 0) break;
+            starts |= 1u << pos;
             packed |= static_cast<uint32_t>(found) << (8 * k);
             pos += flen;
             ++k;
         }
         if (k) {
-            meta[v] = static_cast<uint16_t>(pos | (k << 8));
+            meta[v] = static_cast<uint32_t>(pos) | (static_cast<uint32_t>(k) << 8) | (starts << kMetaMaskShift);
             syms[v] = packed;
         }
     }
@@ -591,7 +592,7 @@ ImageLayout image_layout(const Blob &b) {
     ImageLayout L;
     uint64_t o = align_up(sizeof(ImageHeader), kImageAlign);
     L.meta = o;
-    o = align_up(o + kMultiEntries * 2, kImageAlign);
+    o = align_up(o + kMultiEntries * 4, kImageAlign);
     L.syms = o;
     o = align_up(o + kMultiEntries * 4, kImageAlign);
     L.lut = o;
@@ -623,7 +624,7 @@ void write_image(const Blob &b, uint8_t *dst) {
     h.max_span = b.max_span;
     h.layout = L;
     std::memcpy(dst, &h, sizeof h);
-    std::memcpy(dst + L.meta, b.cb->meta.data(), kMultiEntries * 2);
+    std::memcpy(dst + L.meta, b.cb->meta.data(), kMultiEntries * 4);
     std::memcpy(dst + L.syms, b.cb->syms.data(), kMultiEntries * 4);
     std::memcpy(dst + L.lut, b.cb->lut.data(), b.cb->lut.size() * 2);
     if (!b.gaps.empty()) std::memcpy(dst + L.gaps, b.gaps.data(), b.gaps.size());

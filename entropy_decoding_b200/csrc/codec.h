@@ -22,7 +22,7 @@ struct Codebook {
     uint32_t codes[256] = {};
     int max_len_used = 0;
     int min_len_used = 0;
-    std::vector<uint16_t> meta;  // kMultiEntries
+    std::vector<uint32_t> meta;  // kMultiEntries
     std::vector<uint32_t> syms;  // kMultiEntries
     std::vector<uint16_t> lut;   // n_luts * kLutEntries
     int n_luts() const { return static_cast<int>(lut.size() / kLutEntries); }

@@ -34,7 +34,7 @@
 #include <cstdint>
 #include <mutex>
 
-#include "../../include/df11.h"
+#include "df11.h"
 #include "launch.h"
 
 namespace df11 {
@@ -126,94 +126,223 @@ struct StageMeta {
 static_assert(sizeof(StageMeta) == 32, "stage meta");
 
 constexpr uint32_t kCtrlBytes = 1024;
+constexpr uint32_t kSmemBudget = 227u * 1024u;  // opt-in dynamic shared memory per CTA on sm_100
+constexpr int kStreamStages = 2;
 
+// Shared memory of one CTA:
+//   control (barriers, per-stage tile metadata, warp totals)
+//   decode tables: 12-bit multi-symbol meta (u32) and symbols (u32), the
+//   first hierarchical 256-entry tables (u16)
+//   kStreamStages x (tile stream slice + 16 look-ahead bytes), x (gaps)
+//   the tile's exponents in output order (all zero between tiles)
 struct Plan {
-    uint32_t stream_bytes;  // per stage: tile stream + 16 look-ahead bytes
-    uint32_t gaps_bytes;    // per stage
-    uint32_t plane_bytes;   // per stage
-    uint32_t stage_bytes;
-    uint32_t off_meta, off_syms, off_lut, off_stage, off_exps, exps_bytes, total;
+    uint32_t stream_bytes, gaps_bytes, exps_bytes;
+    uint32_t off_meta, off_syms, off_lut, off_stream, off_gaps, off_exps, total;
 };
 
 __host__ __device__ inline uint32_t up128(uint32_t x) { return (x + 127u) & ~127u; }
 
-__host__ __device__ inline Plan make_plan(int dtype, int chunk_bits, int nt, int stages, uint32_t max_span,
-                                          int n_lut_smem) {
+__host__ __device__ inline Plan make_plan(int chunk_bits, int chunks, uint32_t max_span, int n_lut_smem) {
     Plan p;
-    p.stream_bytes = static_cast<uint32_t>(nt * chunk_bits / 8) + 16u;
-    p.gaps_bytes = static_cast<uint32_t>(nt);
-    // plane span of a tile: BF16 16-element groups (16 plane bytes), E4M3
-    // 32-element groups (16 plane bytes)
-    p.plane_bytes = dtype == 0 ? ((max_span + 32u + 15u) & ~15u) : (((max_span + 1u) / 2u + 48u + 15u) & ~15u);
-    p.stage_bytes = up128(p.stream_bytes) + up128(p.gaps_bytes) + up128(p.plane_bytes);
-    p.off_meta = kCtrlBytes;
-    p.off_syms = p.off_meta + kMultiEntries * 2;
-    p.off_lut = p.off_syms + kMultiEntries * 4;
-    p.off_stage = up128(p.off_lut + static_cast<uint32_t>(n_lut_smem) * kLutEntries * 2);
-    p.off_exps = p.off_stage + static_cast<uint32_t>(stages) * p.stage_bytes;
+    p.stream_bytes = static_cast<uint32_t>(chunks * chunk_bits / 8) + 16u;
+    p.gaps_bytes = static_cast<uint32_t>(chunks);
     p.exps_bytes = up128(max_span + 2u * 32u + 16u);
+    p.off_meta = kCtrlBytes;
+    p.off_syms = p.off_meta + kMultiEntries * 4;
+    p.off_lut = p.off_syms + kMultiEntries * 4;
+    p.off_stream = up128(p.off_lut + static_cast<uint32_t>(n_lut_smem) * kLutEntries * 2);
+    p.off_gaps = p.off_stream + kStreamStages * up128(p.stream_bytes);
+    p.off_exps = p.off_gaps + kStreamStages * up128(p.gaps_bytes);
     p.total = p.off_exps + p.exps_bytes;
     return p;
 }
 
-// ------------------------------------------------------------------ the two walks
+// ------------------------------------------------------------------ decoding a chunk
 
-// Walks the codes that start in one thread's chunk.  w[0..CW] hold the chunk
-// (CW 32-bit words, most significant bit first) plus one look-ahead word;
-// decoding starts at bit p = gap and stops before bit E (chunk_bits, or the
-// stream end inside the last chunk).  EMIT = false counts (phase 1); EMIT =
-// true also writes each symbol to out[0..count) (phase 2).  Both passes take
-// the identical path through the same tables, so they visit the same codes.
-template <bool EMIT, int CW>
-__device__ __forceinline__ uint32_t walk(const uint32_t (&w)[CW + 1], int p, const int E,
-                                         const uint16_t *__restrict__ meta, const uint32_t *__restrict__ syms,
-                                         const uint16_t *__restrict__ lut_s, const uint16_t *__restrict__ lut_g,
-                                         const int n_lut_smem, uint8_t *__restrict__ out, uint32_t &err) {
-    uint32_t cnt = 0;
+struct Tables {
+    const uint32_t *meta;   // shared
+    const uint32_t *syms;   // shared
+    const uint16_t *lut_s;  // shared: hierarchical tables [0, n_lut_smem)
+    const uint16_t *lut_g;  // global: all hierarchical tables
+    int n_lut_smem;
+    int n_luts;
+};
+
+// One code through the hierarchical 256-entry tables; `win` holds the next 32
+// stream bits, most significant first.  Returns symbol | length << 8.  A bit
+// pattern that is no codeword (possible only for a one-symbol code or a
+// damaged stream), a pointer past the last table or a zero length (damaged
+// tables) is flagged and consumed as one 1-bit code, so every step advances.
+__device__ __forceinline__ uint32_t lut_decode(uint32_t win, const Tables &T, uint32_t &err) {
+    uint32_t e = T.lut_s[win >> 24];
+#pragma unroll 1
+    for (int lvl = 1; (e & kLutPointer) && lvl < 4; ++lvl) {
+        const int tbl = static_cast<int>(e & 0x7FFFu);
+        if (tbl >= T.n_luts) break;
+        const uint32_t ix = static_cast<uint32_t>(tbl) * kLutEntries + ((win >> (24 - 8 * lvl)) & 0xFFu);
+        e = tbl < T.n_lut_smem ? T.lut_s[ix] : __ldg(T.lut_g + ix);
+    }
+    if ((e & (kLutPointer | 0x4000u)) || !(e & 0x3F00u)) {
+        err |= DF11_DEV_ERR_CODE;
+        e = 1u << 8;
+    }
+    return e;
+}
+
+// A multi-symbol entry is used only when it consumes 1..12 bits, yields 1..4
+// symbols and its start mask has one bit per symbol starting at offset 0;
+// anything else (a damaged table) becomes the long-code sentinel, whose codes
+// the hierarchical tables then decode one at a time.
+__device__ __forceinline__ uint32_t sane_meta(uint32_t e) {
+    const uint32_t used = e & 0xFFu, n = (e >> 8) & 0xFFFu, mask = e >> kMetaMaskShift;
+    const bool ok = used >= 1 && used <= kMultiBits && n >= 1 && n <= kMultiMaxSyms && (mask & 1u) &&
+                    static_cast<uint32_t>(__popc(mask)) == n && mask < (1u << used);
+    return ok ? e : kMetaLong;
+}
+
+// Number of an entry's codes that start before bit `room` of its window.
+__device__ __forceinline__ uint32_t starts_before(uint32_t mm, int room) {
+    return static_cast<uint32_t>(__popc((mm >> kMetaMaskShift) & ((1u << room) - 1u)));
+}
+
+// Phase 1: count the codes that start in each of this thread's CPT chunks.
+// Chunk c occupies w[c*CW .. c*CW+CW-1] (most significant bit first) and
+// w[c*CW+CW] is its look-ahead word (the next chunk's first word).  Its walk
+// starts at bit gap[c] and counts codes that start before bit E[c].  The walk
+// moves through the chunk 32 bits at a time ("stage" k reads the word pair
+// w[k], w[k+1]).  While a whole 12-bit window lies before E, one lookup in
+// the multi-symbol table consumes up to 4 codes; in the last 11 bits before
+// E the entry's start mask counts only the codes that start before E; codes
+// longer than 12 bits (the sentinel entry) go through the hierarchical tables.
+// acc = p | count << 8 and an entry is consumed | count << 8 | mask << 20, so
+// one add advances both (the mask bits land above the 12-bit count field);
+// the sentinel adds 64 to p, which ends the loop.  The CPT chunks advance in
+// lockstep so their table lookups overlap.
+template <int CW, int CPT>
+__device__ __forceinline__ void count_codes(const uint32_t (&w)[CPT * CW + 1], const int (&gap)[CPT],
+                                            const int (&E)[CPT], const Tables &T, uint32_t (&cnt)[CPT],
+                                            uint32_t &err) {
+    uint32_t acc[CPT];
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) acc[c] = static_cast<uint32_t>(gap[c]);
 #pragma unroll
     for (int k = 0; k < CW; ++k) {
-        const int base = 32 * k;
-        const int ls = min(32, E - base);                     // a code may start here
-        const int lm = min(32, E - base - (kMultiBits - 1));  // a whole 12-bit window lies before E
-        const uint32_t hi = w[k], lo = w[k + 1];
-        while (p < ls) {
-            const uint32_t win = __funnelshift_l(lo, hi, p);  // stream bits [p, p + 32) of this word pair
-            if (p < lm) {
-                const uint32_t idx = win >> (32 - kMultiBits);
-                const uint32_t mm = meta[idx];
-                if (!(mm & kMetaLong)) {
-                    const uint32_t c = mm >> 8;
-                    if (EMIT) {
-                        const uint32_t sy = syms[idx];
-                        out[cnt] = static_cast<uint8_t>(sy);
-                        if (c > 1) out[cnt + 1] = static_cast<uint8_t>(sy >> 8);
-                        if (c > 2) out[cnt + 2] = static_cast<uint8_t>(sy >> 16);
-                        if (c > 3) out[cnt + 3] = static_cast<uint8_t>(sy >> 24);
+        int lm[CPT], ls[CPT], er[CPT];
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) {
+            er[c] = E[c] - 32 * k;
+            lm[c] = min(32, er[c] - (kMultiBits - 1));
+            ls[c] = min(32, er[c]);
+        }
+        for (;;) {
+            for (;;) {
+                bool act[CPT], any = false;
+#pragma unroll
+                for (int c = 0; c < CPT; ++c) {
+                    act[c] = static_cast<int>(acc[c] & 0xFFu) < lm[c];
+                    any |= act[c];
+                }
+                if (!any) break;
+#pragma unroll
+                for (int c = 0; c < CPT; ++c) {
+                    if (act[c]) {
+                        const uint32_t win = __funnelshift_l(w[c * CW + k + 1], w[c * CW + k], acc[c]);
+                        acc[c] += T.meta[win >> (32 - kMultiBits)];
                     }
-                    p += static_cast<int>(mm & 0x3Fu);
-                    cnt += c;
-                    continue;
                 }
             }
-            // one code through the hierarchical 256-entry tables
-            uint32_t e = lut_s[win >> 24];
-#pragma unroll 1
-            for (int lvl = 1; (e & kLutPointer) && lvl < 4; ++lvl) {
-                const uint32_t tbl = e & 0x7FFFu;
-                const uint32_t ix = tbl * kLutEntries + ((win >> (24 - 8 * lvl)) & 0xFFu);
-                e = static_cast<int>(tbl) < n_lut_smem ? lut_s[ix] : __ldg(lut_g + ix);
+            bool more = false;
+#pragma unroll
+            for (int c = 0; c < CPT; ++c) {
+                int p = static_cast<int>(acc[c] & 0xFFu);
+                bool single = false;
+                if (p >= 64) {  // sentinel: the first code is longer than 12 bits
+                    acc[c] -= 64;
+                    p -= 64;
+                    single = true;
+                } else if (p >= ls[c]) {
+                    continue;
+                }
+                const uint32_t win = __funnelshift_l(w[c * CW + k + 1], w[c * CW + k], p);
+                const uint32_t mm = single ? kMetaLong : T.meta[win >> (32 - kMultiBits)];
+                if (mm & kMetaLong) {
+                    const uint32_t e = lut_decode(win, T, err);
+                    acc[c] += ((e >> 8) & 0x3Fu) + 256u;
+                } else {  // last bits before E: count only the codes that start before it
+                    acc[c] += (mm & 0x3Fu) + (starts_before(mm, er[c] - p) << 8);
+                }
+                more = true;
             }
-            if (e & (kLutPointer | 0x4000u)) {  // no codeword: count one bit so the walk still ends
-                err |= DF11_DEV_ERR_CODE;
-                e = 1u << 8;
-            }
-            if (EMIT) out[cnt] = static_cast<uint8_t>(e);
-            p += static_cast<int>((e >> 8) & 0x3Fu);
-            cnt += 1;
+            if (!more) break;
         }
-        p -= 32;
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) acc[c] -= min(acc[c] & 0xFFu, 32u);
     }
-    return cnt;
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) cnt[c] = (acc[c] >> 8) & 0xFFFu;
+}
+
+// Appends nbits (a multiple of 8, <= 32) of packed symbols `sy` to the
+// pending word lo (fill bits used); every completed 32-bit word is ORed into
+// shared memory at `out`, which then advances.  The exponent buffer is zero
+// before phase 2, so neighbouring chunks can OR into a word they share.
+__device__ __forceinline__ void append(uint32_t sy, uint32_t nbits, uint32_t &lo, uint32_t &fill, uint32_t &out) {
+    const uint32_t vhi = __funnelshift_l(sy, 0u, fill);  // bytes of sy that spill past this word
+    lo |= sy << fill;
+    fill += nbits;
+    if (fill >= 32) {
+        asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(out), "r"(lo) : "memory");
+        out += 4;
+        lo = vhi;
+        fill -= 32;
+    }
+}
+
+// Phase 2: decode chunk C again along the same path as phase 1 and write its
+// symbols, packed four to a word, from shared-memory byte address q on.
+template <int CW, int CPT, int C>
+__device__ __forceinline__ void emit_codes(const uint32_t (&w)[CPT * CW + 1], int p, const int E, const Tables &T,
+                                           uint32_t q, uint32_t &err) {
+    uint32_t out = q & ~3u, fill = 8u * (q & 3u), lo = 0;
+#pragma unroll
+    for (int k = 0; k < CW; ++k) {
+        const int er = E - 32 * k;
+        const int lm = min(32, er - (kMultiBits - 1));
+        const int ls = min(32, er);
+        const uint32_t hi = w[C * CW + k], lw = w[C * CW + k + 1];
+        for (;;) {
+            while (p < lm) {
+                const uint32_t win = __funnelshift_l(lw, hi, p);
+                const uint32_t idx = win >> (32 - kMultiBits);
+                const uint32_t mm = T.meta[idx];
+                p += static_cast<int>(mm & 0x7Fu);
+                append(T.syms[idx], (mm >> 5) & 0x38u, lo, fill, out);
+            }
+            bool single = false;
+            if (p >= 64) {
+                p -= 64;
+                single = true;
+            } else if (p >= ls) {
+                break;
+            }
+            const uint32_t win = __funnelshift_l(lw, hi, p);
+            const uint32_t idx = win >> (32 - kMultiBits);
+            const uint32_t mm = single ? kMetaLong : T.meta[idx];
+            if (mm & kMetaLong) {
+                const uint32_t e = lut_decode(win, T, err);
+                p += static_cast<int>((e >> 8) & 0x3Fu);
+                append(e & 0xFFu, 8u, lo, fill, out);
+            } else {
+                const uint32_t nv = starts_before(mm, er - p);
+                const uint32_t nb = 8u * nv;
+                const uint32_t sy = nb >= 32 ? T.syms[idx] : (T.syms[idx] & ((1u << nb) - 1u));
+                p += static_cast<int>(mm & 0x3Fu);
+                if (nb) append(sy, nb, lo, fill, out);
+            }
+        }
+        p -= min(p, 32);
+    }
+    if (fill) asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(out), "r"(lo) : "memory");
 }
 
 // ------------------------------------------------------------------ field merges
@@ -241,22 +370,39 @@ __device__ __forceinline__ void st_global_v4(void *p, uint4 v) {
                  : "memory");
 }
 
+__device__ __forceinline__ uint4 ld_global_stream_v4(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // ------------------------------------------------------------------ kernel
 
-template <int DT, int CB, int NT, int STAGES>
-__global__ void __launch_bounds__(NT + 32, 1)
+// DT: 0 = BF16, 1 = E4M3.  CB: stream bits per chunk.  CPT: chunks per
+// decoding thread.  NTH: decoding threads per CTA; a tile has NTH * CPT chunks.
+// The CTA has NTH / 32 consumer warps and one producer warp.
+template <int DT, int CB, int CPT, int NTH>
+__global__ void __launch_bounds__(NTH + 32, 1)
     decode_kernel(const __grid_constant__ DecodeParams P, const uint32_t max_span, const int n_lut_smem) {
     constexpr int CW = CB / 32;
-    constexpr int NW = NT / 32;
+    constexpr int NW = NTH / 32;
+    constexpr int CHUNKS = NTH * CPT;
+    constexpr uint32_t TILE_BYTES = CHUNKS * CB / 8;
     constexpr uint32_t GROUP = DT == 0 ? 16u : 32u;  // elements per 16 plane bytes
     extern __shared__ __align__(128) uint8_t smem[];
-    const Plan plan = make_plan(DT, CB, NT, STAGES, max_span, n_lut_smem);
+    const Plan plan = make_plan(CB, CHUNKS, max_span, n_lut_smem);
 
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem);
-    uint64_t *empty = full + STAGES;
+    uint64_t *full_s = reinterpret_cast<uint64_t *>(smem);  // stream + gaps landed
+    uint64_t *empty_s = full_s + kStreamStages;             // stream slot free again
     StageMeta *smeta = reinterpret_cast<StageMeta *>(smem + 128);
-    uint32_t *warp_tot = reinterpret_cast<uint32_t *>(smem + 128 + 32 * 8);
-    uint16_t *s_meta = reinterpret_cast<uint16_t *>(smem + plan.off_meta);
+    uint32_t *warp_tot = reinterpret_cast<uint32_t *>(smem + 384);
+    uint32_t *s_meta = reinterpret_cast<uint32_t *>(smem + plan.off_meta);
     uint32_t *s_syms = reinterpret_cast<uint32_t *>(smem + plan.off_syms);
     uint16_t *s_lut = reinterpret_cast<uint16_t *>(smem + plan.off_lut);
     uint8_t *s_exps = smem + plan.off_exps;
@@ -264,42 +410,51 @@ __global__ void __launch_bounds__(NT + 32, 1)
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
 
-    // stage the decode tables (all warps), initialise the pipeline barriers
+    // stage the decode tables (all warps), zero the exponent buffer,
+    // initialise the pipeline barriers
     {
         const uint4 *g = reinterpret_cast<const uint4 *>(P.meta);
         uint4 *s = reinterpret_cast<uint4 *>(s_meta);
-        for (int i = tid; i < kMultiEntries * 2 / 16; i += NT + 32) s[i] = __ldg(g + i);
+        for (int i = tid; i < kMultiEntries * 4 / 16; i += NTH + 32) {
+            uint4 v = __ldg(g + i);
+            v.x = sane_meta(v.x);
+            v.y = sane_meta(v.y);
+            v.z = sane_meta(v.z);
+            v.w = sane_meta(v.w);
+            s[i] = v;
+        }
         g = reinterpret_cast<const uint4 *>(P.syms);
         s = reinterpret_cast<uint4 *>(s_syms);
-        for (int i = tid; i < kMultiEntries * 4 / 16; i += NT + 32) s[i] = __ldg(g + i);
+        for (int i = tid; i < kMultiEntries * 4 / 16; i += NTH + 32) s[i] = __ldg(g + i);
         g = reinterpret_cast<const uint4 *>(P.lut);
         s = reinterpret_cast<uint4 *>(s_lut);
-        for (int i = tid; i < n_lut_smem * kLutEntries * 2 / 16; i += NT + 32) s[i] = __ldg(g + i);
+        for (int i = tid; i < n_lut_smem * kLutEntries * 2 / 16; i += NTH + 32) s[i] = __ldg(g + i);
+        s = reinterpret_cast<uint4 *>(s_exps);
+        for (uint32_t i = tid; i < plan.exps_bytes / 16; i += NTH + 32) s[i] = make_uint4(0, 0, 0, 0);
     }
     if (tid == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], NW);
+        for (int s = 0; s < kStreamStages; ++s) {
+            mbar_init(&full_s[s], 1);
+            mbar_init(&empty_s[s], NW);
         }
         warp_tot[NW] = 0;  // abort marker
         fence_mbar_init();
     }
     __syncthreads();
 
-    auto stage_stream = [&](int s) { return smem + plan.off_stage + s * plan.stage_bytes; };
-    auto stage_gaps = [&](int s) { return stage_stream(s) + up128(plan.stream_bytes); };
-    auto stage_plane = [&](int s) { return stage_gaps(s) + up128(plan.gaps_bytes); };
+    uint8_t *const s_stream0 = smem + plan.off_stream;
+    uint8_t *const s_gaps0 = smem + plan.off_gaps;
+    const uint32_t stream_stride = up128(plan.stream_bytes);
+    const uint32_t gaps_stride = up128(plan.gaps_bytes);
 
     if (warp == NW) {
         // ---------------- producer warp: one lane issues every copy
         if (lane != 0) return;
-        uint32_t k = 0;
-        uint32_t armed = 0;          // bit s: stage s has been armed at least once
-        uint32_t last_parity = 0;    // bit s: parity of its last armed phase
+        uint32_t k = 0, armed = 0, last_parity = 0;
         for (uint32_t t = blockIdx.x; t < P.total_tiles; t += gridDim.x, ++k) {
-            const int s = static_cast<int>(k % STAGES);
-            const uint32_t ph = (k / STAGES) & 1u;
-            if (!mbar_wait(&empty[s], ph ^ 1u)) {
+            const int s = static_cast<int>(k % kStreamStages);
+            const uint32_t ph = (k / kStreamStages) & 1u;
+            if (!mbar_wait(&empty_s[s], ph ^ 1u)) {
                 report(P.err, DF11_DEV_ERR_TIMEOUT);
                 break;
             }
@@ -322,77 +477,89 @@ __global__ void __launch_bounds__(NT + 32, 1)
             m.tensor = static_cast<uint32_t>(ti);
             m.local_tile = lt;
             m.bad = bad;
-            uint64_t a0 = 0, a1 = 0;
+            mbar_arrive_expect_tx(&full_s[s], plan.stream_bytes + plan.gaps_bytes);
+            bulk_load(s_stream0 + s * stream_stride, d.stream + static_cast<uint64_t>(lt) * TILE_BYTES,
+                      plan.stream_bytes, &full_s[s]);
+            bulk_load(s_gaps0 + s * gaps_stride, d.gaps + static_cast<uint64_t>(lt) * CHUNKS, plan.gaps_bytes,
+                      &full_s[s]);
+            // the merge reads this tile's plane span from global memory: pull it into L2 now
             if (span) {
-                a0 = (S / GROUP) * 16u;
-                a1 = ((S + span + GROUP - 1) / GROUP) * 16u;
+                const uint64_t a0 = (S / GROUP) * 16u, a1 = ((S + span + GROUP - 1) / GROUP) * 16u;
+                prefetch_l2(d.plane + a0, static_cast<uint32_t>(a1 - a0));
             }
-            const uint32_t pbytes = static_cast<uint32_t>(a1 - a0);
-            mbar_arrive_expect_tx(&full[s], plan.stream_bytes + plan.gaps_bytes + pbytes);
-            bulk_load(stage_stream(s), d.stream + static_cast<uint64_t>(lt) * (NT * CB / 8), plan.stream_bytes,
-                      &full[s]);
-            bulk_load(stage_gaps(s), d.gaps + static_cast<uint64_t>(lt) * NT, plan.gaps_bytes, &full[s]);
-            if (pbytes) bulk_load(stage_plane(s), d.plane + a0, pbytes, &full[s]);
             armed |= 1u << s;
             last_parity = (last_parity & ~(1u << s)) | (ph << s);
         }
         // keep the CTA alive until every copy it issued has landed
-        for (int s = 0; s < STAGES; ++s)
+        for (int s = 0; s < kStreamStages; ++s)
             if (armed & (1u << s))
-                if (!mbar_wait(&full[s], (last_parity >> s) & 1u)) report(P.err, DF11_DEV_ERR_TIMEOUT);
+                if (!mbar_wait(&full_s[s], (last_parity >> s) & 1u)) report(P.err, DF11_DEV_ERR_TIMEOUT);
         return;
     }
 
     // ---------------- consumer warps
+    const Tables T{s_meta, s_syms, s_lut, P.lut, n_lut_smem, P.n_luts};
     uint32_t err = 0;
     uint32_t k = 0;
     for (uint32_t t = blockIdx.x; t < P.total_tiles; t += gridDim.x, ++k) {
-        const int s = static_cast<int>(k % STAGES);
-        const uint32_t ph = (k / STAGES) & 1u;
-        const bool landed = mbar_wait(&full[s], ph);
+        const int s = static_cast<int>(k % kStreamStages);
+        const uint32_t ph = (k / kStreamStages) & 1u;
+        const bool landed = mbar_wait(&full_s[s], ph);
         const StageMeta m = smeta[s];
         const int ti = landed && m.tensor < static_cast<uint32_t>(P.n_tensors) ? static_cast<int>(m.tensor) : 0;
         const TensorDesc &d = P.t[ti];
 
-        // ---- phase 1: load this thread's chunk, count the codes starting in it
-        const uint8_t *sst = stage_stream(s);
-        uint32_t w[CW + 1];
-        if constexpr (CW % 4 == 0) {
+        // ---- this thread's CPT consecutive chunks + one look-ahead word
+        const uint8_t *sst = s_stream0 + s * stream_stride + tid * (CPT * CB / 8);
+        uint32_t w[CPT * CW + 1];
+        if constexpr ((CPT * CW) % 4 == 0) {
 #pragma unroll
-            for (int j = 0; j < CW / 4; ++j) {
-                const uint4 v = *reinterpret_cast<const uint4 *>(sst + tid * (CB / 8) + 16 * j);
+            for (int j = 0; j < CPT * CW / 4; ++j) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(sst + 16 * j);
                 w[4 * j + 0] = bswap32(v.x);
                 w[4 * j + 1] = bswap32(v.y);
                 w[4 * j + 2] = bswap32(v.z);
                 w[4 * j + 3] = bswap32(v.w);
             }
         } else {
-            const uint2 v = *reinterpret_cast<const uint2 *>(sst + tid * (CB / 8));
+            const uint2 v = *reinterpret_cast<const uint2 *>(sst);
             w[0] = bswap32(v.x);
             w[1] = bswap32(v.y);
         }
         {
-            // look-ahead word: the next thread's first word (lane 31 reads it)
             const uint32_t nxt = __shfl_down_sync(0xFFFFFFFFu, w[0], 1);
-            w[CW] = lane == 31 ? bswap32(*reinterpret_cast<const uint32_t *>(sst + (tid + 1) * (CB / 8))) : nxt;
+            w[CPT * CW] =
+                lane == 31 ? bswap32(*reinterpret_cast<const uint32_t *>(sst + CPT * CB / 8)) : nxt;
         }
-        const int gap = stage_gaps(s)[tid];
-        const int64_t chunk_start = (static_cast<int64_t>(m.local_tile) * NT + tid) * CB;
-        const int64_t rem = static_cast<int64_t>(d.total_bits) - chunk_start;
-        const int E = rem >= CB ? CB : (rem <= 0 ? 0 : static_cast<int>(rem));
-        const uint32_t cnt =
-            walk<false, CW>(w, gap, E, s_meta, s_syms, s_lut, P.lut, n_lut_smem, nullptr, err);
+        int gap[CPT], E[CPT];
+        const uint8_t *sg = s_gaps0 + s * gaps_stride + tid * CPT;
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) {
+            const int g = sg[c];
+            if (g >= 32) err |= DF11_DEV_ERR_AUX;
+            gap[c] = min(g, 63);
+            const int64_t chunk_start = (static_cast<int64_t>(m.local_tile) * CHUNKS + tid * CPT + c) * CB;
+            const int64_t rem = static_cast<int64_t>(d.total_bits) - chunk_start;
+            E[c] = rem >= CB ? CB : (rem <= 0 ? 0 : static_cast<int>(rem));
+        }
+
+        // ---- phase 1: count
+        uint32_t cnt[CPT];
+        count_codes<CW, CPT>(w, gap, E, T, cnt, err);
+        uint32_t mine = 0;
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) mine += cnt[c];
 
         // ---- scan: warp shuffles, then the warp totals
-        uint32_t incl = cnt;
+        uint32_t incl = mine;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
             if (lane >= o) incl += v;
         }
         if (lane == 31) warp_tot[warp] = incl;
-        if (!landed) warp_tot[NW] = 1;  // abort marker, read after the barrier
-        consumer_sync(NT);
+        if (!landed) warp_tot[NW] = 1;
+        consumer_sync(NTH);
         if (warp_tot[NW]) {
             err |= DF11_DEV_ERR_TIMEOUT;
             break;
@@ -404,35 +571,44 @@ __global__ void __launch_bounds__(NT + 32, 1)
             total += v;
             prefix += i < warp ? v : 0u;
         }
-        const uint32_t q0 = prefix + incl - cnt;
         const bool good = !m.bad && total == m.span;
         if (!good && !m.bad && tid == 0) err |= DF11_DEV_ERR_SPAN;
 
-        // ---- phase 2: decode again, exponents into shared memory
-        if (good && m.span)
-            walk<true, CW>(w, gap, E, s_meta, s_syms, s_lut, P.lut, n_lut_smem,
-                           s_exps + (m.S % GROUP) + q0, err);
-        consumer_sync(NT);
+        // ---- phase 2: decode again, exponents into shared memory in output order
+        if (good && m.span) {
+            const uint32_t q = smem_addr(s_exps) + static_cast<uint32_t>(m.S % GROUP) + prefix + incl - mine;
+            emit_codes<CW, CPT, 0>(w, gap[0], E[0], T, q, err);
+            if constexpr (CPT > 1) emit_codes<CW, CPT, 1>(w, gap[1], E[1], T, q + cnt[0], err);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_s[s]);
+        consumer_sync(NTH);
 
-        // ---- merge with the raw plane, 16-byte stores
+        // ---- merge with the raw plane (read from global/L2), 16-byte stores;
+        // each group's exponents are cleared for the next tile once read
         if (good && m.span) {
             const uint64_t g0 = m.S / GROUP;
             const uint32_t ng = static_cast<uint32_t>((m.S + m.span + GROUP - 1) / GROUP - g0);
-            const uint8_t *spl = stage_plane(s);
             uint8_t *dst = static_cast<uint8_t *>(d.dst);
+            const uint8_t *plane = d.plane + g0 * 16u;
             const uint64_t lo = m.S, hi = m.S + m.span;
-            for (uint32_t i = tid; i < ng; i += NT) {
-                const uint4 p4 = *reinterpret_cast<const uint4 *>(spl + 16 * i);
+            for (uint32_t i = tid; i < ng; i += NTH) {
+                const uint4 p4 = ld_global_stream_v4(plane + 16u * i);
                 uint4 a, b;
                 if constexpr (DT == 0) {
-                    const uint4 x4 = *reinterpret_cast<const uint4 *>(s_exps + 16 * i);
+                    uint4 *xp = reinterpret_cast<uint4 *>(s_exps + 16 * i);
+                    const uint4 x4 = *xp;
+                    *xp = make_uint4(0, 0, 0, 0);
                     merge_bf16x4(p4.x, x4.x, a.x, a.y);
                     merge_bf16x4(p4.y, x4.y, a.z, a.w);
                     merge_bf16x4(p4.z, x4.z, b.x, b.y);
                     merge_bf16x4(p4.w, x4.w, b.z, b.w);
                 } else {
-                    const uint4 x0 = *reinterpret_cast<const uint4 *>(s_exps + 32 * i);
-                    const uint4 x1 = *reinterpret_cast<const uint4 *>(s_exps + 32 * i + 16);
+                    uint4 *xp = reinterpret_cast<uint4 *>(s_exps + 32 * i);
+                    const uint4 x0 = xp[0];
+                    const uint4 x1 = xp[1];
+                    xp[0] = make_uint4(0, 0, 0, 0);
+                    xp[1] = make_uint4(0, 0, 0, 0);
                     merge_e4m3x8(p4.x, x0.x, x0.y, a.x, a.y);
                     merge_e4m3x8(p4.y, x0.z, x0.w, a.z, a.w);
                     merge_e4m3x8(p4.z, x1.x, x1.y, b.x, b.y);
@@ -464,25 +640,21 @@ __global__ void __launch_bounds__(NT + 32, 1)
                 }
             }
         }
-        // ---- release the stage (every warp is done reading it)
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
     }
     report(P.err, err);
 }
 
 // ------------------------------------------------------------------ host side
 
-constexpr int kStages = 2;
-
 using KernelFn = void (*)(DecodeParams, uint32_t, int);
 
 struct KernelEntry {
-    int dtype, chunk_bits, nt;
+    int dtype, chunk_bits, chunks, cpt;
     KernelFn fn;
 };
 
-#define DF11_KERNEL(DT, CB, NT) {DT, CB, NT, &decode_kernel<DT, CB, NT, kStages>}
+#define DF11_KERNEL(DT, CB, CH) \
+    {DT, CB, CH, 1, &decode_kernel<DT, CB, 1, CH>}, { DT, CB, CH, 2, &decode_kernel<DT, CB, 2, CH / 2> }
 
 const KernelEntry kKernels[] = {
     DF11_KERNEL(0, 128, 256), DF11_KERNEL(1, 128, 256), DF11_KERNEL(0, 256, 128), DF11_KERNEL(1, 256, 128),
@@ -490,9 +662,9 @@ const KernelEntry kKernels[] = {
     DF11_KERNEL(0, 128, 512), DF11_KERNEL(1, 128, 512), DF11_KERNEL(0, 256, 256), DF11_KERNEL(1, 256, 256),
 };
 
-const KernelEntry *find_kernel(int dtype, int chunk_bits, int nt) {
+const KernelEntry *find_kernel(int dtype, int chunk_bits, int chunks, int cpt) {
     for (const auto &e : kKernels)
-        if (e.dtype == dtype && e.chunk_bits == chunk_bits && e.nt == nt) return &e;
+        if (e.dtype == dtype && e.chunk_bits == chunk_bits && e.chunks == chunks && e.cpt == cpt) return &e;
     return nullptr;
 }
 
@@ -529,19 +701,24 @@ struct Prepared {
     const KernelEntry *ke = nullptr;
     uint32_t max_span = 0;
     int n_lut_smem = 0;
+    int ctas_per_sm = 0;
     Plan plan;
 };
 
-LaunchStatus build_params(const Blob *const *blobs, void *const *dst, int n, int *err, Prepared *out) {
+LaunchStatus build_params(const Blob *const *blobs, void *const *dst, int n, int *err, const DecodeOptions &opt,
+                          Prepared *out) {
     if (n < 1 || n > kMaxTensorsPerLaunch || !blobs[0]) return LaunchStatus::kInvalid;
     const Blob &b0 = *blobs[0];
-    const KernelEntry *ke = find_kernel(b0.dtype, b0.chunk_bits, b0.tile_threads);
+    const int cpt = opt.chunks_per_thread ? opt.chunks_per_thread : kDefaultChunksPerThread;
+    if (cpt != 1 && cpt != 2) return LaunchStatus::kInvalid;
+    const KernelEntry *ke = find_kernel(b0.dtype, b0.chunk_bits, b0.tile_threads, cpt);
     if (!ke) return LaunchStatus::kUnsupported;
     DecodeParams &P = out->params;
     P = DecodeParams{};
     uint64_t tiles = 0, max_span = 0;
     int nt = 0;
     for (int i = 0; i < n; ++i) {
+        if (!blobs[i]) return LaunchStatus::kInvalid;
         const Blob &b = *blobs[i];
         if (!b.dev_image || b.dtype != b0.dtype || b.chunk_bits != b0.chunk_bits ||
             b.tile_threads != b0.tile_threads)
@@ -567,7 +744,7 @@ LaunchStatus build_params(const Blob *const *blobs, void *const *dst, int n, int
     }
     if (tiles >= (uint64_t{1} << 31)) return LaunchStatus::kInvalid;
     const ImageLayout L0 = image_layout(b0);
-    P.meta = reinterpret_cast<const uint16_t *>(b0.dev_image + L0.meta);
+    P.meta = reinterpret_cast<const uint32_t *>(b0.dev_image + L0.meta);
     P.syms = reinterpret_cast<const uint32_t *>(b0.dev_image + L0.syms);
     P.lut = reinterpret_cast<const uint16_t *>(b0.dev_image + L0.lut);
     P.err = err;
@@ -578,7 +755,9 @@ LaunchStatus build_params(const Blob *const *blobs, void *const *dst, int n, int
     out->ke = ke;
     out->max_span = static_cast<uint32_t>(max_span);
     out->n_lut_smem = P.n_luts < kSmemLutTables ? P.n_luts : kSmemLutTables;
-    out->plan = make_plan(b0.dtype, b0.chunk_bits, b0.tile_threads, kStages, out->max_span, out->n_lut_smem);
+    out->ctas_per_sm = opt.ctas_per_sm;
+    out->plan = make_plan(b0.chunk_bits, b0.tile_threads, out->max_span, out->n_lut_smem);
+    if (out->plan.total > kSmemBudget) return LaunchStatus::kUnsupported;
     return LaunchStatus::kOk;
 }
 
@@ -587,11 +766,12 @@ LaunchStatus shape_for(const Prepared &pp, LaunchShape *sh) {
     if (cudaGetDevice(&dev) != cudaSuccess) return LaunchStatus::kCuda;
     if (!prepare(pp.ke, dev)) return LaunchStatus::kCuda;
     if (static_cast<int>(pp.plan.total) > g_smem_optin[dev]) return LaunchStatus::kUnsupported;
-    const int block = pp.ke->nt + 32;
+    const int block = pp.ke->chunks / pp.ke->cpt + 32;
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pp.ke->fn, block, pp.plan.total) != cudaSuccess)
         return LaunchStatus::kCuda;
     if (per_sm < 1) return LaunchStatus::kUnsupported;
+    if (pp.ctas_per_sm > 0 && pp.ctas_per_sm < per_sm) per_sm = pp.ctas_per_sm;
     const uint64_t want = static_cast<uint64_t>(per_sm) * static_cast<uint64_t>(g_sm_count[dev]);
     sh->grid = static_cast<int>(want < pp.params.total_tiles ? want : pp.params.total_tiles);
     sh->block = block;
@@ -602,15 +782,15 @@ LaunchStatus shape_for(const Prepared &pp, LaunchShape *sh) {
 }  // namespace
 
 bool kernel_available(int dtype, int chunk_bits, int tile_threads) {
-    return find_kernel(dtype, chunk_bits, tile_threads) != nullptr;
+    return find_kernel(dtype, chunk_bits, tile_threads, 1) != nullptr;
 }
 
-LaunchStatus decode_launch_shape(const Blob *const *blobs, int n, LaunchShape *out) {
+LaunchStatus decode_launch_shape(const Blob *const *blobs, int n, const DecodeOptions &opt, LaunchShape *out) {
     Prepared pp;
-    // shape does not depend on the destinations: use 16-byte aligned stand-ins
+    // the shape does not depend on the destinations: use 16-byte aligned stand-ins
     void *fake[kMaxTensorsPerLaunch];
     for (int i = 0; i < n && i < kMaxTensorsPerLaunch; ++i) fake[i] = reinterpret_cast<void *>(uintptr_t{256});
-    LaunchStatus st = build_params(blobs, fake, n, nullptr, &pp);
+    LaunchStatus st = build_params(blobs, fake, n, nullptr, opt, &pp);
     if (st != LaunchStatus::kOk) return st;
     if (!pp.params.total_tiles) {
         *out = LaunchShape{};
@@ -619,9 +799,10 @@ LaunchStatus decode_launch_shape(const Blob *const *blobs, int n, LaunchShape *o
     return shape_for(pp, out);
 }
 
-LaunchStatus launch_decode(const Blob *const *blobs, void *const *dst, int n, int *err, cudaStream_t s) {
+LaunchStatus launch_decode(const Blob *const *blobs, void *const *dst, int n, int *err, const DecodeOptions &opt,
+                           cudaStream_t s) {
     Prepared pp;
-    LaunchStatus st = build_params(blobs, dst, n, err, &pp);
+    LaunchStatus st = build_params(blobs, dst, n, err, opt, &pp);
     if (st != LaunchStatus::kOk) return st;
     if (!pp.params.total_tiles) return LaunchStatus::kOk;
     LaunchShape sh;

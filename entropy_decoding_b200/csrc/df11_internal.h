@@ -10,11 +10,12 @@
 //       invalid  bit14 = 1 (leaf form, length 1): no codeword has this prefix
 //     A 32-bit code needs at most 4 levels.
 //   * multi-symbol table (an addition for sm_100a's instruction budget): 4096
-//     entries indexed by the next 12 stream bits.  meta[v] = consumed bits
-//     (bits 0..5) | symbols decoded (bits 8..10), for the longest run of up
-//     to 4 whole codes inside the 12-bit window; meta[v] = kMetaLong when the
-//     first code is longer than 12 bits.  syms[v] holds those symbols, first
-//     in the low byte.
+//     entries indexed by the next 12 stream bits, for the longest run of up
+//     to 4 whole codes inside the 12-bit window.  meta[v] (u32) = consumed
+//     bits (bits 0..5) | symbols decoded (bits 8..10) | start mask (bit 20+j
+//     set when one of those codes starts at window offset j); meta[v] =
+//     kMetaLong when the first code is longer than 12 bits.  syms[v] holds
+//     the symbols, first in the low byte, unused bytes zero.
 #pragma once
 
 #include <cstdint>
@@ -24,7 +25,8 @@ namespace df11 {
 constexpr int kMultiBits = 12;
 constexpr int kMultiEntries = 1 << kMultiBits;
 constexpr int kMultiMaxSyms = 4;
-constexpr uint16_t kMetaLong = 0x0040;
+constexpr uint32_t kMetaLong = 0x0040;
+constexpr int kMetaMaskShift = 20;
 
 constexpr int kLutEntries = 256;
 constexpr uint16_t kLutPointer = 0x8000;
@@ -69,7 +71,7 @@ struct TensorDesc {
 };
 
 struct DecodeParams {
-    const uint16_t *meta;
+    const uint32_t *meta;
     const uint32_t *syms;
     const uint16_t *lut;
     int *err;

@@ -9,6 +9,13 @@ namespace df11 {
 
 enum class LaunchStatus { kOk, kInvalid, kUnsupported, kCuda };
 
+struct DecodeOptions {
+    int chunks_per_thread = 0;  // 0 = kDefaultChunksPerThread
+    int ctas_per_sm = 0;        // 0 = as many as fit
+};
+
+constexpr int kDefaultChunksPerThread = 1;
+
 struct LaunchShape {
     int grid = 0;
     int block = 0;
@@ -17,9 +24,10 @@ struct LaunchShape {
 
 bool kernel_available(int dtype, int chunk_bits, int tile_threads);
 
-LaunchStatus decode_launch_shape(const Blob *const *blobs, int n, LaunchShape *out);
+LaunchStatus decode_launch_shape(const Blob *const *blobs, int n, const DecodeOptions &opt, LaunchShape *out);
 
 // One launch decoding every blob into dst[i] on stream s.
-LaunchStatus launch_decode(const Blob *const *blobs, void *const *dst, int n, int *err, cudaStream_t s);
+LaunchStatus launch_decode(const Blob *const *blobs, void *const *dst, int n, int *err, const DecodeOptions &opt,
+                           cudaStream_t s);
 
 }  // namespace df11

@@ -50,6 +50,10 @@ class BlobInfo(ctypes.Structure):
         return {k: getattr(self, k) for k, _ in self._fields_}
 
 
+class DecodeOpts(ctypes.Structure):
+    _fields_ = [("chunks_per_thread", ctypes.c_int32), ("ctas_per_sm", ctypes.c_int32)]
+
+
 _P = ctypes.c_void_p
 _PP = ctypes.POINTER(ctypes.c_void_p)
 _U64 = ctypes.c_uint64
@@ -76,6 +80,9 @@ _SIGS = {
     "df11_blob_bind": ([_P, _P, _U64], _S),
     "df11_blob_upload": ([_P, _P, _U64, _P], _S),
     "df11_decode": ([_PP, _PP, _I, _P, _P], _S),
+    "df11_decode_ex": ([_PP, _PP, _I, _P, _P, ctypes.POINTER(DecodeOpts)], _S),
+    "df11_decode_launch_shape_ex": ([_PP, _I, ctypes.POINTER(DecodeOpts), ctypes.POINTER(_I), ctypes.POINTER(_I),
+                                     ctypes.POINTER(_I)], _S),
     "df11_decode_host": ([_PP, _PP, _PP, _PP, _PP, _I, _P, _P], _S),
     "df11_decode_launch_shape": ([_PP, _I, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I)], _S),
 }
@@ -117,9 +124,9 @@ class Codebook:
         _check(_lib.df11_codebook_lengths(self._h, out.ctypes.data), "df11_codebook_lengths")
         return out[: 256 if self.dtype == "bf16" else 16]
 
-    def __del__(self):
+    def __del__(self, _free=_lib.df11_codebook_free):
         if getattr(self, "_h", None) and self._h.value:
-            _lib.df11_codebook_free(self._h)
+            _free(self._h)
             self._h = ctypes.c_void_p(0)
 
 
@@ -162,9 +169,9 @@ class Blob:
         _check(_lib.df11_blob_lengths(self._h, out.ctypes.data), "df11_blob_lengths")
         return out
 
-    def __del__(self):
+    def __del__(self, _free=_lib.df11_blob_free):
         if getattr(self, "_h", None) and self._h.value:
-            _lib.df11_blob_free(self._h)
+            _free(self._h)
             self._h = ctypes.c_void_p(0)
 
 
@@ -245,6 +252,13 @@ def df11_decode(blobs, dst_ptrs, err_ptr: int | None = None, stream: int = 0):
     _check(_lib.df11_decode(hs, ds, len(blobs), err_ptr or None, stream or None), "df11_decode")
 
 
+def df11_decode_ex(blobs, dst_ptrs, err_ptr: int | None = None, stream: int = 0, chunks_per_thread: int = 0,
+                   ctas_per_sm: int = 0):
+    o = DecodeOpts(chunks_per_thread, ctas_per_sm)
+    _check(_lib.df11_decode_ex(_ptr_array([b.handle.value for b in blobs]), _ptr_array(dst_ptrs), len(blobs),
+                               err_ptr or None, stream or None, ctypes.byref(o)), "df11_decode_ex")
+
+
 def df11_decode_host(blobs, host_image_ptrs, dev_image_ptrs, dst_dev_ptrs, dst_host_ptrs,
                      err_ptr: int | None = None, stream: int = 0):
     _check(_lib.df11_decode_host(_ptr_array([b.handle.value for b in blobs]), _ptr_array(host_image_ptrs),
@@ -252,10 +266,11 @@ def df11_decode_host(blobs, host_image_ptrs, dev_image_ptrs, dst_dev_ptrs, dst_h
                                  len(blobs), err_ptr or None, stream or None), "df11_decode_host")
 
 
-def df11_decode_launch_shape(blobs) -> tuple[int, int, int]:
+def df11_decode_launch_shape(blobs, chunks_per_thread: int = 0, ctas_per_sm: int = 0) -> tuple[int, int, int]:
     g, b, s = _I(), _I(), _I()
-    _check(_lib.df11_decode_launch_shape(_ptr_array([x.handle.value for x in blobs]), len(blobs),
-                                         ctypes.byref(g), ctypes.byref(b), ctypes.byref(s)),
+    o = DecodeOpts(chunks_per_thread, ctas_per_sm)
+    _check(_lib.df11_decode_launch_shape_ex(_ptr_array([x.handle.value for x in blobs]), len(blobs), ctypes.byref(o),
+                                            ctypes.byref(g), ctypes.byref(b), ctypes.byref(s)),
            "df11_decode_launch_shape")
     return g.value, b.value, s.value
 

@@ -221,6 +221,17 @@ df11_status df11_blob_upload(df11_blob *blob, void *dev_dst, uint64_t cap, df11_
 df11_status df11_decode(const df11_blob *const *blobs, void *const *dst_dev, int n_blobs,
                         int *dev_err_flag, df11_stream stream);
 
+/* Tuning knobs of the decode launch; zero-initialise for the defaults. */
+typedef struct {
+    int32_t chunks_per_thread; /* stream chunks each decoding thread walks: 1 or 2 (0 = default, 2) */
+    int32_t ctas_per_sm;       /* persistent CTAs per SM, capped by occupancy (0 = as many as fit) */
+} df11_decode_opts;
+
+/* df11_decode with explicit launch options (opts may be NULL).  The result is
+ * identical for every option value; only the speed changes. */
+df11_status df11_decode_ex(const df11_blob *const *blobs, void *const *dst_dev, int n_blobs,
+                           int *dev_err_flag, df11_stream stream, const df11_decode_opts *opts);
+
 /* End-to-end decode from host memory to host memory, all on `stream` and
  * asynchronous (the caller synchronises the stream before reading dst_host):
  * for each blob, cudaMemcpyAsync host_images[i] (its device image, e.g. from
@@ -236,6 +247,11 @@ df11_status df11_decode_host(df11_blob *const *blobs, const void *const *host_im
  * Any output pointer may be NULL. */
 df11_status df11_decode_launch_shape(const df11_blob *const *blobs, int n_blobs, int *grid,
                                      int *block, int *smem_bytes);
+
+/* As df11_decode_launch_shape, for the given options (opts may be NULL). */
+df11_status df11_decode_launch_shape_ex(const df11_blob *const *blobs, int n_blobs,
+                                        const df11_decode_opts *opts, int *grid, int *block,
+                                        int *smem_bytes);
 
 #ifdef __cplusplus
 }

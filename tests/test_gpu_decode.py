@@ -20,10 +20,11 @@ def df11():
     return mod
 
 
-def _roundtrip(df11, oracle_mod, x, dt, chunk_bits=128, tile_threads=256, max_len=0, check_oracle=True):
+def _roundtrip(df11, oracle_mod, x, dt, chunk_bits=128, tile_threads=256, max_len=0, check_oracle=True, cpt=0,
+               ctas=0):
     cb = df11.df11_build_codebook(dt, [x], max_len)
     blob = df11.df11_encode(cb, x, chunk_bits, tile_threads)
-    (out,), err, guards = decode_gpu(df11, [blob])
+    (out,), err, guards = decode_gpu(df11, [blob], chunks_per_thread=cpt, ctas_per_sm=ctas)
     assert err == 0
     assert guards
     assert out.shape == x.shape
@@ -65,11 +66,21 @@ def test_parity_ragged_sizes(df11, oracle_mod, dt, n):
 LAYOUTS = [(128, 256), (256, 128), (64, 512), (128, 128), (128, 512), (256, 256)]
 
 
+@pytest.mark.parametrize("cpt", [1, 2])
 @pytest.mark.parametrize("layout", LAYOUTS)
 @pytest.mark.parametrize("case", ["heavy_2m", "e4m3_normal", "single_symbol", "uniform_random"])
-def test_parity_layouts(df11, oracle_mod, layout, case):
+def test_parity_layouts(df11, oracle_mod, layout, case, cpt):
+    """Every layout the kernel is built for, with one and with two chunks per
+    decoding thread (same output, different launch shape)."""
     dt, make = SMALL[case]
-    _roundtrip(df11, oracle_mod, make(), dt, *layout)
+    _roundtrip(df11, oracle_mod, make(), dt, *layout, cpt=cpt)
+
+
+@pytest.mark.parametrize("ctas", [1, 2])
+@pytest.mark.parametrize("cpt", [1, 2])
+def test_parity_launch_options(df11, oracle_mod, cpt, ctas):
+    dt, make = SMALL["heavy_2m"]
+    _roundtrip(df11, oracle_mod, make(), dt, cpt=cpt, ctas=ctas)
 
 
 def test_parity_32_bit_codes(df11, oracle_mod):
@@ -204,6 +215,8 @@ def test_launch_shape_is_persistent(df11):
     df11.upload(blob)
     grid, block, smem = df11.df11_decode_launch_shape([blob])
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    assert block == 256 + 32
+    assert block == 256 + 32  # default: one chunk per decoding thread, plus the producer warp
+    g2, b2, _ = df11.df11_decode_launch_shape([blob], chunks_per_thread=2, ctas_per_sm=1)
+    assert b2 == 256 // 2 + 32 and g2 == min(sms, blob.info().n_tiles)
     assert grid == min(blob.info().n_tiles, grid) and grid % sms == 0 or grid == blob.info().n_tiles
     assert 0 < smem <= 227 * 1024

@@ -138,20 +138,21 @@ def test_decode_tables_match_independent_prefix_decode(df11, oracle_mod, case):
     lengths = oracle_mod.build_lengths([x], dt)
     codes = oracle_mod.canonical_codes(lengths)
     table = _prefix_decoder(lengths, codes)
-    meta = img[lay["meta"]:lay["meta"] + 8192].view(np.uint16)
+    meta = img[lay["meta"]:lay["meta"] + 16384].view(np.uint32)
     syms = img[lay["syms"]:lay["syms"] + 16384].view(np.uint32)
     for v in range(4096):
-        pos, got = 0, []
+        pos, got, starts = 0, [], 0
         while len(got) < 4:
             r = _first_code(table, v & ((1 << (12 - pos)) - 1), 12 - pos) if pos < 12 else None
             if r is None:
                 break
+            starts |= 1 << pos
             got.append(r[0])
             pos += r[1]
         if not got:
             assert meta[v] == 0x40, v
         else:
-            assert meta[v] == pos | (len(got) << 8), v
+            assert meta[v] == pos | (len(got) << 8) | (starts << 20), v
             assert [(int(syms[v]) >> (8 * i)) & 0xFF for i in range(len(got))] == got
     lut = img[lay["lut"]:lay["lut"] + lay["n_luts"] * 512].view(np.uint16)
     rng = np.random.default_rng(0)
