@@ -128,6 +128,7 @@ static_assert(sizeof(StageMeta) == 32, "stage meta");
 constexpr uint32_t kCtrlBytes = 1024;
 constexpr uint32_t kSmemBudget = 227u * 1024u;  // opt-in dynamic shared memory per CTA on sm_100
 constexpr int kStreamStages = 2;
+constexpr int kPrefetchGroups = 4;  // plane groups per thread loaded at tile start
 
 // Shared memory of one CTA:
 //   control (barriers, per-stage tile metadata, warp totals)
@@ -382,13 +383,68 @@ __device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
+// Stores the elements of a 32-byte output group that fall in [lo, hi) (tile-local
+// element indices); the rest of the group belongs to a neighbouring tile or
+// lies past the end of the tensor.  Rare: at most two groups per tile.
+template <int DT>
+__device__ __noinline__ void store_partial(uint8_t *out, uint4 a, uint4 b, uint32_t e0, uint32_t lo, uint32_t hi) {
+    const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    if constexpr (DT == 0) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (e0 + j >= lo && e0 + j < hi)
+                reinterpret_cast<uint16_t *>(out)[j] = static_cast<uint16_t>(wv[j >> 1] >> (16 * (j & 1)));
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (e0 + j >= lo && e0 + j < hi) out[j] = static_cast<uint8_t>(wv[j >> 2] >> (8 * (j & 3)));
+    }
+}
+
+// Merges group i of a tile: 16 plane bytes p4 with its exponents from shared
+// memory (which are then cleared for the next tile) into 32 output bytes.
+// [lo, hi) are the tile's elements relative to the first group's first element.
+template <int DT>
+__device__ __forceinline__ void merge_group(uint4 p4, uint32_t i, uint8_t *s_exps, uint8_t *dst_tile, uint32_t lo,
+                                            uint32_t hi) {
+    constexpr uint32_t GROUP = DT == 0 ? 16u : 32u;
+    uint4 a, b;
+    if constexpr (DT == 0) {
+        uint4 *xp = reinterpret_cast<uint4 *>(s_exps + 16 * i);
+        const uint4 x4 = *xp;
+        *xp = make_uint4(0, 0, 0, 0);
+        merge_bf16x4(p4.x, x4.x, a.x, a.y);
+        merge_bf16x4(p4.y, x4.y, a.z, a.w);
+        merge_bf16x4(p4.z, x4.z, b.x, b.y);
+        merge_bf16x4(p4.w, x4.w, b.z, b.w);
+    } else {
+        uint4 *xp = reinterpret_cast<uint4 *>(s_exps + 32 * i);
+        const uint4 x0 = xp[0];
+        const uint4 x1 = xp[1];
+        xp[0] = make_uint4(0, 0, 0, 0);
+        xp[1] = make_uint4(0, 0, 0, 0);
+        merge_e4m3x8(p4.x, x0.x, x0.y, a.x, a.y);
+        merge_e4m3x8(p4.y, x0.z, x0.w, a.z, a.w);
+        merge_e4m3x8(p4.z, x1.x, x1.y, b.x, b.y);
+        merge_e4m3x8(p4.w, x1.z, x1.w, b.z, b.w);
+    }
+    const uint32_t e0 = i * GROUP;
+    uint8_t *out = dst_tile + 32u * i;
+    if (e0 >= lo && e0 + GROUP <= hi) {
+        st_global_v4(out, a);
+        st_global_v4(out + 16, b);
+    } else {
+        store_partial<DT>(out, a, b, e0, lo, hi);
+    }
+}
+
 // ------------------------------------------------------------------ kernel
 
 // DT: 0 = BF16, 1 = E4M3.  CB: stream bits per chunk.  CPT: chunks per
 // decoding thread.  NTH: decoding threads per CTA; a tile has NTH * CPT chunks.
 // The CTA has NTH / 32 consumer warps and one producer warp.
 template <int DT, int CB, int CPT, int NTH>
-__global__ void __launch_bounds__(NTH + 32, 1)
+__global__ void __launch_bounds__(NTH + 32, (NTH + 32) * 3 <= 1024 ? 3 : 1)
     decode_kernel(const __grid_constant__ DecodeParams P, const uint32_t max_span, const int n_lut_smem) {
     constexpr int CW = CB / 32;
     constexpr int NW = NTH / 32;
@@ -509,6 +565,20 @@ __global__ void __launch_bounds__(NTH + 32, 1)
         const int ti = landed && m.tensor < static_cast<uint32_t>(P.n_tensors) ? static_cast<int>(m.tensor) : 0;
         const TensorDesc &d = P.t[ti];
 
+        // ---- the tile's plane span (16 bytes per group of GROUP elements): the
+        // first kPrefetchGroups groups of this thread are loaded now, so they
+        // arrive while the chunk is decoded; the merge loads any others itself
+        const uint64_t g0 = m.S / GROUP;
+        const uint32_t ng =
+            landed && !m.bad && m.span ? static_cast<uint32_t>((m.S + m.span + GROUP - 1) / GROUP - g0) : 0u;
+        const uint8_t *plane = d.plane + g0 * 16u;
+        uint4 pre[kPrefetchGroups];
+#pragma unroll
+        for (int u = 0; u < kPrefetchGroups; ++u) {
+            const uint32_t i = tid + u * NTH;
+            if (i < ng) pre[u] = ld_global_stream_v4(plane + 16u * i);
+        }
+
         // ---- this thread's CPT consecutive chunks + one look-ahead word
         const uint8_t *sst = s_stream0 + s * stream_stride + tid * (CPT * CB / 8);
         uint32_t w[CPT * CW + 1];
@@ -533,14 +603,17 @@ __global__ void __launch_bounds__(NTH + 32, 1)
         }
         int gap[CPT], E[CPT];
         const uint8_t *sg = s_gaps0 + s * gaps_stride + tid * CPT;
+        // stream bits of this tile from this thread's first chunk on (clamped)
+        const int64_t rem64 = static_cast<int64_t>(d.total_bits) -
+                              static_cast<int64_t>(m.local_tile) * (static_cast<int64_t>(CHUNKS) * CB) -
+                              static_cast<int64_t>(tid * CPT * CB);
+        const int rem = rem64 > CPT * CB ? CPT * CB : (rem64 < 0 ? 0 : static_cast<int>(rem64));
 #pragma unroll
         for (int c = 0; c < CPT; ++c) {
             const int g = sg[c];
             if (g >= 32) err |= DF11_DEV_ERR_AUX;
             gap[c] = min(g, 63);
-            const int64_t chunk_start = (static_cast<int64_t>(m.local_tile) * CHUNKS + tid * CPT + c) * CB;
-            const int64_t rem = static_cast<int64_t>(d.total_bits) - chunk_start;
-            E[c] = rem >= CB ? CB : (rem <= 0 ? 0 : static_cast<int>(rem));
+            E[c] = min(max(rem - c * CB, 0), CB);
         }
 
         // ---- phase 1: count
@@ -566,10 +639,14 @@ __global__ void __launch_bounds__(NTH + 32, 1)
         }
         uint32_t prefix = 0, total = 0;
 #pragma unroll
-        for (int i = 0; i < NW; ++i) {
-            const uint32_t v = warp_tot[i];
-            total += v;
-            prefix += i < warp ? v : 0u;
+        for (int i = 0; i < NW; i += 4) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(warp_tot + i);
+            const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4 && i + j < NW; ++j) {
+                total += vv[j];
+                prefix += i + j < warp ? vv[j] : 0u;
+            }
         }
         const bool good = !m.bad && total == m.span;
         if (!good && !m.bad && tid == 0) err |= DF11_DEV_ERR_SPAN;
@@ -587,58 +664,15 @@ __global__ void __launch_bounds__(NTH + 32, 1)
         // ---- merge with the raw plane (read from global/L2), 16-byte stores;
         // each group's exponents are cleared for the next tile once read
         if (good && m.span) {
-            const uint64_t g0 = m.S / GROUP;
-            const uint32_t ng = static_cast<uint32_t>((m.S + m.span + GROUP - 1) / GROUP - g0);
-            uint8_t *dst = static_cast<uint8_t *>(d.dst);
-            const uint8_t *plane = d.plane + g0 * 16u;
-            const uint64_t lo = m.S, hi = m.S + m.span;
-            for (uint32_t i = tid; i < ng; i += NTH) {
-                const uint4 p4 = ld_global_stream_v4(plane + 16u * i);
-                uint4 a, b;
-                if constexpr (DT == 0) {
-                    uint4 *xp = reinterpret_cast<uint4 *>(s_exps + 16 * i);
-                    const uint4 x4 = *xp;
-                    *xp = make_uint4(0, 0, 0, 0);
-                    merge_bf16x4(p4.x, x4.x, a.x, a.y);
-                    merge_bf16x4(p4.y, x4.y, a.z, a.w);
-                    merge_bf16x4(p4.z, x4.z, b.x, b.y);
-                    merge_bf16x4(p4.w, x4.w, b.z, b.w);
-                } else {
-                    uint4 *xp = reinterpret_cast<uint4 *>(s_exps + 32 * i);
-                    const uint4 x0 = xp[0];
-                    const uint4 x1 = xp[1];
-                    xp[0] = make_uint4(0, 0, 0, 0);
-                    xp[1] = make_uint4(0, 0, 0, 0);
-                    merge_e4m3x8(p4.x, x0.x, x0.y, a.x, a.y);
-                    merge_e4m3x8(p4.y, x0.z, x0.w, a.z, a.w);
-                    merge_e4m3x8(p4.z, x1.x, x1.y, b.x, b.y);
-                    merge_e4m3x8(p4.w, x1.z, x1.w, b.z, b.w);
-                }
-                const uint64_t e0 = (g0 + i) * GROUP;
-                uint8_t *out = dst + e0 * (DT == 0 ? 2 : 1);
-                if (e0 >= lo && e0 + GROUP <= hi) {
-                    st_global_v4(out, a);
-                    st_global_v4(out + 16, b);
-                } else {
-                    // group shared with a neighbouring tile or past the tensor end
-                    const uint32_t wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-                    if constexpr (DT == 0) {
+            uint8_t *dst_tile = static_cast<uint8_t *>(d.dst) + g0 * 32u;
+            const uint32_t lo = static_cast<uint32_t>(m.S % GROUP), hi = lo + m.span;
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            const uint64_t pos = e0 + j;
-                            if (pos >= lo && pos < hi)
-                                reinterpret_cast<uint16_t *>(out)[j] =
-                                    static_cast<uint16_t>(wv[j >> 1] >> (16 * (j & 1)));
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const uint64_t pos = e0 + j;
-                            if (pos >= lo && pos < hi) out[j] = static_cast<uint8_t>(wv[j >> 2] >> (8 * (j & 3)));
-                        }
-                    }
-                }
+            for (int u = 0; u < kPrefetchGroups; ++u) {
+                const uint32_t i = tid + u * NTH;
+                if (i < ng) merge_group<DT>(pre[u], i, s_exps, dst_tile, lo, hi);
             }
+            for (uint32_t i = tid + kPrefetchGroups * NTH; i < ng; i += NTH)
+                merge_group<DT>(ld_global_stream_v4(plane + 16u * i), i, s_exps, dst_tile, lo, hi);
         }
     }
     report(P.err, err);
