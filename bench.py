@@ -55,9 +55,10 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
     p.add_argument("--chunk-bits", type=int, default=128)
-    p.add_argument("--tile-threads", type=int, default=256)
+    p.add_argument("--tile-threads", type=int, default=32)
     p.add_argument("--chunks-per-thread", type=int, default=0, help="decode launch option (0 = library default)")
     p.add_argument("--ctas-per-sm", type=int, default=0, help="decode launch option (0 = as many as fit)")
+    p.add_argument("--warps-per-cta", type=int, default=0, help="decode launch option, warp tiles (0 = 8)")
     return p.parse_args()
 
 
@@ -82,7 +83,8 @@ def full_config(args, world: int) -> dict:
     cfg = workload_config(args.workload)
     out_gb = cfg["n_weights"] * (2 if cfg["dtype_in"] == "bf16" else 1) / 1e9
     return {**cfg, "seed": args.seed, "chunk_bits": args.chunk_bits, "tile_threads": args.tile_threads,
-            "chunks_per_thread": args.chunks_per_thread or 2, "ctas_per_sm": args.ctas_per_sm or "max",
+            "chunks_per_thread": args.chunks_per_thread or 1, "ctas_per_sm": args.ctas_per_sm or "max",
+            "warps_per_cta": (args.warps_per_cta or 16) if args.tile_threads == 32 else None,
             "l2": f"no flush: inputs larger than L2 (decoded output {out_gb:.1f} GB, compressed images "
                   f"about 0.68x that, vs 126 MB L2)",
             "parallelism": f"replicas x{world} (each GPU decodes its own copy)"}
@@ -339,7 +341,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             if events is not None:
                 events[gi][0].record(stream)
             df11.df11_decode_ex(blobs, [d[0] for d in dsts], err.data_ptr(), stream.cuda_stream,
-                                args.chunks_per_thread, args.ctas_per_sm)
+                                args.chunks_per_thread, args.ctas_per_sm, args.warps_per_cta)
             if events is not None:
                 events[gi][1].record(stream)
 
@@ -474,8 +476,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": peak_src,
-                     "kernel": f"decode_kernel<{'bf16' if cfg['dtype_in'] == 'bf16' else 'e4m3'},"
-                               f"{args.chunk_bits},{args.tile_threads}>",
+                     "kernel": (f"decode_warp_kernel<{cfg["dtype_in"]},{args.chunk_bits},{args.warps_per_cta or 16}>"
+                                if args.tile_threads == 32 else
+                                f"decode_kernel<{cfg['dtype_in']},{args.chunk_bits},{args.chunks_per_thread or 1},"
+                                f"{args.tile_threads // (args.chunks_per_thread or 1)}>"),
                      "algorithmic_bytes_per_launch": algo_step / len(groups),
                      "launch_ms_mean": float(per_launch.mean()),
                      "launch_ms_by_group": {"first": float(per_launch[:, 0].mean()),

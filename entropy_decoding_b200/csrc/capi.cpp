@@ -117,7 +117,7 @@ df11_status df11_encode_ex(const df11_codebook *cb, const void *host_src, uint64
 }
 
 df11_status df11_encode(const df11_codebook *cb, const void *host_src, uint64_t n_elems, df11_blob **out) {
-    return df11_encode_ex(cb, host_src, n_elems, 128, 256, 0, out);
+    return df11_encode_ex(cb, host_src, n_elems, 128, 32, 0, out);
 }
 
 int df11_layout_supported(df11_dtype dtype, int chunk_bits, int tile_threads) {
@@ -238,7 +238,8 @@ df11_status df11_decode_ex(const df11_blob *const *blobs, void *const *dst_dev, 
     if (opts) {
         o.chunks_per_thread = opts->chunks_per_thread;
         o.ctas_per_sm = opts->ctas_per_sm;
-        if (o.chunks_per_thread < 0 || o.ctas_per_sm < 0) return DF11_EINVAL;
+        o.warps_per_cta = opts->warps_per_cta;
+        if (o.chunks_per_thread < 0 || o.ctas_per_sm < 0 || o.warps_per_cta < 0) return DF11_EINVAL;
     }
     return from_launch(df11::launch_decode(bs, dst_dev, n_blobs, dev_err_flag, o,
                                            reinterpret_cast<cudaStream_t>(stream)));
@@ -295,6 +296,7 @@ df11_status df11_decode_launch_shape_ex(const df11_blob *const *blobs, int n_blo
     if (opts) {
         o.chunks_per_thread = opts->chunks_per_thread;
         o.ctas_per_sm = opts->ctas_per_sm;
+        o.warps_per_cta = opts->warps_per_cta;
     }
     df11::LaunchStatus st = df11::decode_launch_shape(bs, n_blobs, o, &sh);
     if (st != df11::LaunchStatus::kOk) return from_launch(st);

@@ -309,7 +309,7 @@ void histogram(int dtype, const void *src, uint64_t n, uint64_t *counts, int n_t
 
 bool valid_layout(int chunk_bits, int tile_threads) {
     return (chunk_bits == 64 || chunk_bits == 128 || chunk_bits == 256) &&
-           (tile_threads == 128 || tile_threads == 256 || tile_threads == 512);
+           (tile_threads == 32 || tile_threads == 128 || tile_threads == 256 || tile_threads == 512);
 }
 
 uint64_t plane_bytes(int dtype, uint64_t n) { return dtype == kBF16 ? n : (n + 1) / 2; }

@@ -678,27 +678,252 @@ __global__ void __launch_bounds__(NTH + 32, (NTH + 32) * 3 <= 1024 ? 3 : 1)
     report(P.err, err);
 }
 
+// ------------------------------------------------------------------ warp-tile kernel
+
+// Shared memory of the warp-tile kernel: the decode tables once per CTA, then
+// per warp two stream stages (the tile's 32 chunks + 16 look-ahead bytes,
+// then its 32 gaps), two mbarriers and the warp's exponent buffer.
+struct WarpPlan {
+    uint32_t stage_bytes, exps_bytes, warp_bytes;
+    uint32_t off_meta, off_syms, off_lut, off_warps, total;
+};
+
+__host__ __device__ inline WarpPlan make_warp_plan(int chunk_bits, int nwarp, uint32_t max_span, int n_lut_smem) {
+    WarpPlan p;
+    p.stage_bytes = static_cast<uint32_t>(32 * chunk_bits / 8) + 16u + 32u;  // stream + look-ahead, gaps
+    p.exps_bytes = (max_span + 2u * 32u + 16u + 15u) & ~15u;
+    p.warp_bytes = (16u + 2u * p.stage_bytes + p.exps_bytes + 127u) & ~127u;
+    p.off_meta = 0;
+    p.off_syms = p.off_meta + kMultiEntries * 4;
+    p.off_lut = p.off_syms + kMultiEntries * 4;
+    p.off_warps = up128(p.off_lut + static_cast<uint32_t>(n_lut_smem) * kLutEntries * 2);
+    p.total = p.off_warps + static_cast<uint32_t>(nwarp) * p.warp_bytes;
+    return p;
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Tile t's descriptor index (tiles of all tensors are numbered consecutively).
+__device__ __forceinline__ int tensor_of(const DecodeParams &P, uint32_t t) {
+    int ti = 0;
+    while (ti + 1 < P.n_tensors && t >= P.t[ti + 1].tile_begin) ++ti;
+    return ti;
+}
+
+// One tile = 32 chunks = one warp.  The per-tile output offsets of the
+// container (out_off) are per warp here, so a warp's tiles are decoded with a
+// warp-shuffle scan only and the warps of a CTA never wait for each other:
+// each warp streams its own tiles through two shared-memory stages with 1-D
+// TMA bulk copies (issued by its lane 0 two tiles ahead, completing on the
+// warp's own mbarriers), runs phase 1, the scan, phase 2 and the merge.  The
+// decode tables are staged once per CTA.
+template <int DT, int CB, int NWARP>
+__global__ void __launch_bounds__(NWARP * 32, NWARP <= 8 ? 4 : 2)
+    decode_warp_kernel(const __grid_constant__ DecodeParams P, const uint32_t max_span, const int n_lut_smem) {
+    constexpr int CW = CB / 32;
+    constexpr uint32_t TILE_BYTES = 32 * CB / 8;
+    constexpr uint32_t GROUP = DT == 0 ? 16u : 32u;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const WarpPlan plan = make_warp_plan(CB, NWARP, max_span, n_lut_smem);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    uint32_t *s_meta = reinterpret_cast<uint32_t *>(smem + plan.off_meta);
+    uint32_t *s_syms = reinterpret_cast<uint32_t *>(smem + plan.off_syms);
+    uint16_t *s_lut = reinterpret_cast<uint16_t *>(smem + plan.off_lut);
+    uint8_t *wbase = smem + plan.off_warps + warp * plan.warp_bytes;
+    uint64_t *full = reinterpret_cast<uint64_t *>(wbase);  // [2]
+    uint8_t *stage0 = wbase + 16;
+    uint8_t *s_exps = wbase + 16 + 2 * plan.stage_bytes;
+
+    {
+        const uint4 *g = reinterpret_cast<const uint4 *>(P.meta);
+        uint4 *s = reinterpret_cast<uint4 *>(s_meta);
+        for (int i = tid; i < kMultiEntries * 4 / 16; i += NWARP * 32) {
+            uint4 v = __ldg(g + i);
+            v.x = sane_meta(v.x);
+            v.y = sane_meta(v.y);
+            v.z = sane_meta(v.z);
+            v.w = sane_meta(v.w);
+            s[i] = v;
+        }
+        g = reinterpret_cast<const uint4 *>(P.syms);
+        s = reinterpret_cast<uint4 *>(s_syms);
+        for (int i = tid; i < kMultiEntries * 4 / 16; i += NWARP * 32) s[i] = __ldg(g + i);
+        g = reinterpret_cast<const uint4 *>(P.lut);
+        s = reinterpret_cast<uint4 *>(s_lut);
+        for (int i = tid; i < n_lut_smem * kLutEntries * 2 / 16; i += NWARP * 32) s[i] = __ldg(g + i);
+        s = reinterpret_cast<uint4 *>(s_exps);
+        for (uint32_t i = lane; i < plan.exps_bytes / 16; i += 32) s[i] = make_uint4(0, 0, 0, 0);
+    }
+    if (lane == 0) {
+        mbar_init(&full[0], 1);
+        mbar_init(&full[1], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    const uint32_t stride = gridDim.x * NWARP;
+    const uint32_t first = blockIdx.x * NWARP + warp;
+    uint32_t issued = 0;  // bit s: stage s holds a copy not yet waited for
+    uint32_t par = 0;     // bit s: phase parity of that copy
+    // lane 0: copy tile t's stream slice and gaps into stage s
+    auto issue = [&](uint32_t t, int s) {
+        const TensorDesc &d = P.t[tensor_of(P, t)];
+        const uint32_t lt = t - d.tile_begin;
+        uint8_t *st = stage0 + s * plan.stage_bytes;
+        mbar_arrive_expect_tx(&full[s], TILE_BYTES + 16u + 32u);
+        bulk_load(st, d.stream + static_cast<uint64_t>(lt) * TILE_BYTES, TILE_BYTES + 16u, &full[s]);
+        bulk_load(st + TILE_BYTES + 16u, d.gaps + static_cast<uint64_t>(lt) * 32u, 32u, &full[s]);
+    };
+    if (lane == 0) {
+        if (first < P.total_tiles) issue(first, 0);
+        if (first + stride < P.total_tiles) issue(first + stride, 1);
+    }
+    if (first < P.total_tiles) issued |= 1u;
+    if (first + stride < P.total_tiles) issued |= 2u;
+
+    const Tables T{s_meta, s_syms, s_lut, P.lut, n_lut_smem, P.n_luts};
+    uint32_t err = 0;
+    uint32_t k = 0;
+    for (uint32_t t = first; t < P.total_tiles; t += stride, ++k) {
+        const int s = static_cast<int>(k & 1u);
+        const uint32_t ph = (k >> 1) & 1u;
+        const TensorDesc &d = P.t[tensor_of(P, t)];
+        const uint32_t lt = t - d.tile_begin;
+        uint64_t S = __ldg(d.out_off + lt);
+        const uint64_t Eo = __ldg(d.out_off + lt + 1);
+        const bool bad = Eo < S || Eo > d.n || Eo - S > max_span;
+        if (bad) S = 0;
+        const uint32_t span = bad ? 0u : static_cast<uint32_t>(Eo - S);
+
+        // the tile's plane span: the first kPrefetchGroups groups of each lane now
+        const uint64_t g0 = S / GROUP;
+        const uint32_t ng = span ? static_cast<uint32_t>((S + span + GROUP - 1) / GROUP - g0) : 0u;
+        const uint8_t *plane = d.plane + g0 * 16u;
+        uint4 pre[kPrefetchGroups];
+#pragma unroll
+        for (int u = 0; u < kPrefetchGroups; ++u) {
+            const uint32_t i = lane + 32u * u;
+            if (i < ng) pre[u] = ld_global_stream_v4(plane + 16u * i);
+        }
+
+        const bool landed = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], ph));
+        if (!landed) {
+            err |= DF11_DEV_ERR_TIMEOUT;
+            break;
+        }
+        issued &= ~(1u << s);
+        const uint8_t *st = stage0 + s * plan.stage_bytes;
+        uint32_t w[CW + 1];
+        if constexpr (CW % 4 == 0) {
+#pragma unroll
+            for (int j = 0; j < CW / 4; ++j) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(st + lane * (CB / 8) + 16 * j);
+                w[4 * j + 0] = bswap32(v.x);
+                w[4 * j + 1] = bswap32(v.y);
+                w[4 * j + 2] = bswap32(v.z);
+                w[4 * j + 3] = bswap32(v.w);
+            }
+        } else {
+            const uint2 v = *reinterpret_cast<const uint2 *>(st + lane * (CB / 8));
+            w[0] = bswap32(v.x);
+            w[1] = bswap32(v.y);
+        }
+        {
+            const uint32_t nxt = __shfl_down_sync(0xFFFFFFFFu, w[0], 1);
+            w[CW] = lane == 31 ? bswap32(*reinterpret_cast<const uint32_t *>(st + TILE_BYTES)) : nxt;
+        }
+        int gap[1], E[1];
+        {
+            const int g = st[TILE_BYTES + 16u + lane];
+            if (g >= 32) err |= DF11_DEV_ERR_AUX;
+            gap[0] = min(g, 63);
+            const int64_t rem64 = static_cast<int64_t>(d.total_bits) -
+                                  static_cast<int64_t>(lt) * (32 * CB) - static_cast<int64_t>(lane * CB);
+            E[0] = rem64 >= CB ? CB : (rem64 <= 0 ? 0 : static_cast<int>(rem64));
+        }
+        // the stage's words are in registers: refill it with tile t + 2 * stride
+        __syncwarp();
+        if (t + 2 * stride < P.total_tiles) {
+            if (lane == 0) {
+                fence_proxy_async_smem();
+                issue(t + 2 * stride, s);
+            }
+            issued |= 1u << s;
+            par = (par & ~(1u << s)) | ((((k + 2) >> 1) & 1u) << s);
+        }
+
+        // ---- phase 1, warp scan
+        uint32_t cnt[1];
+        count_codes<CW, 1>(w, gap, E, T, cnt, err);
+        uint32_t incl = cnt[0];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const uint32_t total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+        const bool good = !bad && total == span;
+        if (bad) err |= DF11_DEV_ERR_AUX;
+        else if (!good) err |= DF11_DEV_ERR_SPAN;
+
+        // ---- phase 2, then the merge
+        if (good && span) {
+            emit_codes<CW, 1, 0>(w, gap[0], E[0], T, smem_addr(s_exps) + static_cast<uint32_t>(S % GROUP) + incl - cnt[0],
+                                 err);
+            __syncwarp();
+            uint8_t *dst_tile = static_cast<uint8_t *>(d.dst) + g0 * 32u;
+            const uint32_t lo = static_cast<uint32_t>(S % GROUP), hi = lo + span;
+#pragma unroll
+            for (int u = 0; u < kPrefetchGroups; ++u) {
+                const uint32_t i = lane + 32u * u;
+                if (i < ng) merge_group<DT>(pre[u], i, s_exps, dst_tile, lo, hi);
+            }
+            for (uint32_t i = lane + 32u * kPrefetchGroups; i < ng; i += 32)
+                merge_group<DT>(ld_global_stream_v4(plane + 16u * i), i, s_exps, dst_tile, lo, hi);
+            __syncwarp();
+        }
+    }
+    // after an abort: wait (bounded) for copies that were issued but never consumed
+    for (int s = 0; s < 2; ++s)
+        if (issued & (1u << s))
+            if (!mbar_wait(&full[s], (par >> s) & 1u)) err |= DF11_DEV_ERR_TIMEOUT;
+    err = __reduce_or_sync(0xFFFFFFFFu, err);
+    if (lane == 0) report(P.err, err);
+}
+
 // ------------------------------------------------------------------ host side
 
 using KernelFn = void (*)(DecodeParams, uint32_t, int);
 
+// chunks = chunks per tile (the container's tile_threads).  chunks == 32: the
+// warp-tile kernel with nwarp warps per CTA; otherwise the CTA-tile kernel
+// with chunks / cpt decoding threads and a producer warp.
 struct KernelEntry {
-    int dtype, chunk_bits, chunks, cpt;
+    int dtype, chunk_bits, chunks, cpt, nwarp;
     KernelFn fn;
 };
 
 #define DF11_KERNEL(DT, CB, CH) \
-    {DT, CB, CH, 1, &decode_kernel<DT, CB, 1, CH>}, { DT, CB, CH, 2, &decode_kernel<DT, CB, 2, CH / 2> }
+    {DT, CB, CH, 1, 0, &decode_kernel<DT, CB, 1, CH>}, { DT, CB, CH, 2, 0, &decode_kernel<DT, CB, 2, CH / 2> }
+#define DF11_WARP_KERNEL(DT, CB) \
+    {DT, CB, 32, 1, 8, &decode_warp_kernel<DT, CB, 8>}, { DT, CB, 32, 1, 16, &decode_warp_kernel<DT, CB, 16> }
 
 const KernelEntry kKernels[] = {
+    DF11_WARP_KERNEL(0, 128), DF11_WARP_KERNEL(1, 128), DF11_WARP_KERNEL(0, 256), DF11_WARP_KERNEL(1, 256),
+    DF11_WARP_KERNEL(0, 64),  DF11_WARP_KERNEL(1, 64),
     DF11_KERNEL(0, 128, 256), DF11_KERNEL(1, 128, 256), DF11_KERNEL(0, 256, 128), DF11_KERNEL(1, 256, 128),
     DF11_KERNEL(0, 64, 512),  DF11_KERNEL(1, 64, 512),  DF11_KERNEL(0, 128, 128), DF11_KERNEL(1, 128, 128),
     DF11_KERNEL(0, 128, 512), DF11_KERNEL(1, 128, 512), DF11_KERNEL(0, 256, 256), DF11_KERNEL(1, 256, 256),
 };
 
-const KernelEntry *find_kernel(int dtype, int chunk_bits, int chunks, int cpt) {
+const KernelEntry *find_kernel(int dtype, int chunk_bits, int chunks, int cpt, int nwarp) {
     for (const auto &e : kKernels)
-        if (e.dtype == dtype && e.chunk_bits == chunk_bits && e.chunks == chunks && e.cpt == cpt) return &e;
+        if (e.dtype == dtype && e.chunk_bits == chunk_bits && e.chunks == chunks && e.cpt == cpt &&
+            e.nwarp == nwarp)
+            return &e;
     return nullptr;
 }
 
@@ -736,16 +961,19 @@ struct Prepared {
     uint32_t max_span = 0;
     int n_lut_smem = 0;
     int ctas_per_sm = 0;
-    Plan plan;
+    uint32_t smem = 0;
 };
 
 LaunchStatus build_params(const Blob *const *blobs, void *const *dst, int n, int *err, const DecodeOptions &opt,
                           Prepared *out) {
     if (n < 1 || n > kMaxTensorsPerLaunch || !blobs[0]) return LaunchStatus::kInvalid;
     const Blob &b0 = *blobs[0];
+    const bool warp_tiles = b0.tile_threads == 32;
     const int cpt = opt.chunks_per_thread ? opt.chunks_per_thread : kDefaultChunksPerThread;
     if (cpt != 1 && cpt != 2) return LaunchStatus::kInvalid;
-    const KernelEntry *ke = find_kernel(b0.dtype, b0.chunk_bits, b0.tile_threads, cpt);
+    const int nwarp = warp_tiles ? (opt.warps_per_cta ? opt.warps_per_cta : kDefaultWarpsPerCta) : 0;
+    if (warp_tiles && cpt != 1) return LaunchStatus::kInvalid;
+    const KernelEntry *ke = find_kernel(b0.dtype, b0.chunk_bits, b0.tile_threads, cpt, nwarp);
     if (!ke) return LaunchStatus::kUnsupported;
     DecodeParams &P = out->params;
     P = DecodeParams{};
@@ -790,8 +1018,9 @@ LaunchStatus build_params(const Blob *const *blobs, void *const *dst, int n, int
     out->max_span = static_cast<uint32_t>(max_span);
     out->n_lut_smem = P.n_luts < kSmemLutTables ? P.n_luts : kSmemLutTables;
     out->ctas_per_sm = opt.ctas_per_sm;
-    out->plan = make_plan(b0.chunk_bits, b0.tile_threads, out->max_span, out->n_lut_smem);
-    if (out->plan.total > kSmemBudget) return LaunchStatus::kUnsupported;
+    out->smem = warp_tiles ? make_warp_plan(b0.chunk_bits, nwarp, out->max_span, out->n_lut_smem).total
+                           : make_plan(b0.chunk_bits, b0.tile_threads, out->max_span, out->n_lut_smem).total;
+    if (out->smem > kSmemBudget) return LaunchStatus::kUnsupported;
     return LaunchStatus::kOk;
 }
 
@@ -799,24 +1028,27 @@ LaunchStatus shape_for(const Prepared &pp, LaunchShape *sh) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return LaunchStatus::kCuda;
     if (!prepare(pp.ke, dev)) return LaunchStatus::kCuda;
-    if (static_cast<int>(pp.plan.total) > g_smem_optin[dev]) return LaunchStatus::kUnsupported;
-    const int block = pp.ke->chunks / pp.ke->cpt + 32;
+    if (static_cast<int>(pp.smem) > g_smem_optin[dev]) return LaunchStatus::kUnsupported;
+    const int block = pp.ke->nwarp ? pp.ke->nwarp * 32 : pp.ke->chunks / pp.ke->cpt + 32;
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pp.ke->fn, block, pp.plan.total) != cudaSuccess)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pp.ke->fn, block, pp.smem) != cudaSuccess)
         return LaunchStatus::kCuda;
     if (per_sm < 1) return LaunchStatus::kUnsupported;
     if (pp.ctas_per_sm > 0 && pp.ctas_per_sm < per_sm) per_sm = pp.ctas_per_sm;
     const uint64_t want = static_cast<uint64_t>(per_sm) * static_cast<uint64_t>(g_sm_count[dev]);
-    sh->grid = static_cast<int>(want < pp.params.total_tiles ? want : pp.params.total_tiles);
+    // one CTA per tile (CTA kernel) or per nwarp tiles (warp kernel) at most
+    const uint64_t tiles_per_cta = pp.ke->nwarp ? static_cast<uint64_t>(pp.ke->nwarp) : 1u;
+    const uint64_t need = (pp.params.total_tiles + tiles_per_cta - 1) / tiles_per_cta;
+    sh->grid = static_cast<int>(want < need ? want : need);
     sh->block = block;
-    sh->smem = static_cast<int>(pp.plan.total);
+    sh->smem = static_cast<int>(pp.smem);
     return LaunchStatus::kOk;
 }
 
 }  // namespace
 
 bool kernel_available(int dtype, int chunk_bits, int tile_threads) {
-    return find_kernel(dtype, chunk_bits, tile_threads, 1) != nullptr;
+    return find_kernel(dtype, chunk_bits, tile_threads, 1, tile_threads == 32 ? kDefaultWarpsPerCta : 0) != nullptr;
 }
 
 LaunchStatus decode_launch_shape(const Blob *const *blobs, int n, const DecodeOptions &opt, LaunchShape *out) {

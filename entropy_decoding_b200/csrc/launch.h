@@ -12,9 +12,11 @@ enum class LaunchStatus { kOk, kInvalid, kUnsupported, kCuda };
 struct DecodeOptions {
     int chunks_per_thread = 0;  // 0 = kDefaultChunksPerThread
     int ctas_per_sm = 0;        // 0 = as many as fit
+    int warps_per_cta = 0;      // warp-tile layouts: 0 = kDefaultWarpsPerCta
 };
 
 constexpr int kDefaultChunksPerThread = 1;
+constexpr int kDefaultWarpsPerCta = 16;
 
 struct LaunchShape {
     int grid = 0;

@@ -51,7 +51,8 @@ class BlobInfo(ctypes.Structure):
 
 
 class DecodeOpts(ctypes.Structure):
-    _fields_ = [("chunks_per_thread", ctypes.c_int32), ("ctas_per_sm", ctypes.c_int32)]
+    _fields_ = [("chunks_per_thread", ctypes.c_int32), ("ctas_per_sm", ctypes.c_int32),
+                ("warps_per_cta", ctypes.c_int32)]
 
 
 _P = ctypes.c_void_p
@@ -199,7 +200,7 @@ def df11_codebook_from_lengths(dtype: str, lengths) -> Codebook:
     return Codebook(out.value, dtype)
 
 
-def df11_encode(cb: Codebook, x: np.ndarray, chunk_bits: int = 128, tile_threads: int = 256,
+def df11_encode(cb: Codebook, x: np.ndarray, chunk_bits: int = 128, tile_threads: int = 32,
                 n_threads: int = 0) -> Blob:
     a = np.ascontiguousarray(x).reshape(-1)
     out = ctypes.c_void_p()
@@ -253,8 +254,8 @@ def df11_decode(blobs, dst_ptrs, err_ptr: int | None = None, stream: int = 0):
 
 
 def df11_decode_ex(blobs, dst_ptrs, err_ptr: int | None = None, stream: int = 0, chunks_per_thread: int = 0,
-                   ctas_per_sm: int = 0):
-    o = DecodeOpts(chunks_per_thread, ctas_per_sm)
+                   ctas_per_sm: int = 0, warps_per_cta: int = 0):
+    o = DecodeOpts(chunks_per_thread, ctas_per_sm, warps_per_cta)
     _check(_lib.df11_decode_ex(_ptr_array([b.handle.value for b in blobs]), _ptr_array(dst_ptrs), len(blobs),
                                err_ptr or None, stream or None, ctypes.byref(o)), "df11_decode_ex")
 
@@ -266,9 +267,10 @@ def df11_decode_host(blobs, host_image_ptrs, dev_image_ptrs, dst_dev_ptrs, dst_h
                                  len(blobs), err_ptr or None, stream or None), "df11_decode_host")
 
 
-def df11_decode_launch_shape(blobs, chunks_per_thread: int = 0, ctas_per_sm: int = 0) -> tuple[int, int, int]:
+def df11_decode_launch_shape(blobs, chunks_per_thread: int = 0, ctas_per_sm: int = 0,
+                             warps_per_cta: int = 0) -> tuple[int, int, int]:
     g, b, s = _I(), _I(), _I()
-    o = DecodeOpts(chunks_per_thread, ctas_per_sm)
+    o = DecodeOpts(chunks_per_thread, ctas_per_sm, warps_per_cta)
     _check(_lib.df11_decode_launch_shape_ex(_ptr_array([x.handle.value for x in blobs]), len(blobs), ctypes.byref(o),
                                             ctypes.byref(g), ctypes.byref(b), ctypes.byref(s)),
            "df11_decode_launch_shape")

@@ -116,7 +116,8 @@ void df11_codebook_free(df11_codebook *cb);
 
 /* Compresses one tensor with a codebook (whose code must cover every exponent
  * the tensor holds).  Default layout: chunk_bits = 128 stream bits per decode
- * thread, tile_threads = 256 threads per tile; all host cores are used.
+ * thread, tile_threads = 32 chunks per tile (one warp: out_off is kept per
+ * warp-sized block of threads); all host cores are used.
  * The blob holds, in host memory:
  *   plane    n bytes (BF16: sign << 7 | mantissa) or ceil(n/2) bytes (E4M3:
  *            nibble sign << 3 | mantissa, element 2i in the low nibble)
@@ -131,7 +132,8 @@ df11_status df11_encode(const df11_codebook *cb, const void *host_src, uint64_t 
                         df11_blob **out);
 
 /* df11_encode with an explicit layout: chunk_bits in {64, 128, 256},
- * tile_threads in {128, 256, 512}; n_threads host threads (0 = all cores).
+ * tile_threads (chunks per tile, one out_off entry each) in {32, 128, 256,
+ * 512}; n_threads host threads (0 = all cores).
  * df11_decode supports the layouts listed by df11_layout_supported. */
 df11_status df11_encode_ex(const df11_codebook *cb, const void *host_src, uint64_t n_elems,
                            int chunk_bits, int tile_threads, int n_threads, df11_blob **out);
@@ -223,8 +225,9 @@ df11_status df11_decode(const df11_blob *const *blobs, void *const *dst_dev, int
 
 /* Tuning knobs of the decode launch; zero-initialise for the defaults. */
 typedef struct {
-    int32_t chunks_per_thread; /* stream chunks each decoding thread walks: 1 or 2 (0 = default, 2) */
+    int32_t chunks_per_thread; /* CTA-tile layouts: chunks each decoding thread walks, 1 or 2 (0 = 1) */
     int32_t ctas_per_sm;       /* persistent CTAs per SM, capped by occupancy (0 = as many as fit) */
+    int32_t warps_per_cta;     /* warp-tile layout (tile_threads 32): 8 or 16 (0 = 16) */
 } df11_decode_opts;
 
 /* df11_decode with explicit launch options (opts may be NULL).  The result is

@@ -20,11 +20,11 @@ def df11():
     return mod
 
 
-def _roundtrip(df11, oracle_mod, x, dt, chunk_bits=128, tile_threads=256, max_len=0, check_oracle=True, cpt=0,
-               ctas=0):
+def _roundtrip(df11, oracle_mod, x, dt, chunk_bits=128, tile_threads=32, max_len=0, check_oracle=True, cpt=0,
+               ctas=0, wpc=0):
     cb = df11.df11_build_codebook(dt, [x], max_len)
     blob = df11.df11_encode(cb, x, chunk_bits, tile_threads)
-    (out,), err, guards = decode_gpu(df11, [blob], chunks_per_thread=cpt, ctas_per_sm=ctas)
+    (out,), err, guards = decode_gpu(df11, [blob], chunks_per_thread=cpt, ctas_per_sm=ctas, warps_per_cta=wpc)
     assert err == 0
     assert guards
     assert out.shape == x.shape
@@ -63,24 +63,36 @@ def test_parity_ragged_sizes(df11, oracle_mod, dt, n):
     _roundtrip(df11, oracle_mod, x, dt)
 
 
-LAYOUTS = [(128, 256), (256, 128), (64, 512), (128, 128), (128, 512), (256, 256)]
+CTA_LAYOUTS = [(128, 256), (256, 128), (64, 512), (128, 128), (128, 512), (256, 256)]
+WARP_LAYOUTS = [(128, 32), (256, 32), (64, 32)]
 
 
 @pytest.mark.parametrize("cpt", [1, 2])
-@pytest.mark.parametrize("layout", LAYOUTS)
+@pytest.mark.parametrize("layout", CTA_LAYOUTS)
 @pytest.mark.parametrize("case", ["heavy_2m", "e4m3_normal", "single_symbol", "uniform_random"])
-def test_parity_layouts(df11, oracle_mod, layout, case, cpt):
-    """Every layout the kernel is built for, with one and with two chunks per
-    decoding thread (same output, different launch shape)."""
+def test_parity_cta_layouts(df11, oracle_mod, layout, case, cpt):
+    """CTA-tile layouts (one out_off per tile of 128-512 chunks, block-wide
+    scan), with one and with two chunks per decoding thread."""
     dt, make = SMALL[case]
     _roundtrip(df11, oracle_mod, make(), dt, *layout, cpt=cpt)
 
 
+@pytest.mark.parametrize("wpc", [8, 16])
+@pytest.mark.parametrize("layout", WARP_LAYOUTS)
+@pytest.mark.parametrize("case", ["heavy_2m", "e4m3_normal", "single_symbol", "uniform_random", "fib26"])
+def test_parity_warp_layouts(df11, oracle_mod, layout, case, wpc):
+    """Warp-tile layouts (one out_off per 32 chunks, warp-shuffle scan), with
+    8 and 16 warps per CTA."""
+    dt, make = SMALL[case]
+    _roundtrip(df11, oracle_mod, make(), dt, *layout, wpc=wpc)
+
+
 @pytest.mark.parametrize("ctas", [1, 2])
-@pytest.mark.parametrize("cpt", [1, 2])
-def test_parity_launch_options(df11, oracle_mod, cpt, ctas):
+@pytest.mark.parametrize("layout_cpt", [((128, 256), 1), ((128, 256), 2), ((128, 32), 1)])
+def test_parity_launch_options(df11, oracle_mod, layout_cpt, ctas):
+    (cb, tt), cpt = layout_cpt
     dt, make = SMALL["heavy_2m"]
-    _roundtrip(df11, oracle_mod, make(), dt, cpt=cpt, ctas=ctas)
+    _roundtrip(df11, oracle_mod, make(), dt, cb, tt, cpt=cpt, ctas=ctas)
 
 
 def test_parity_32_bit_codes(df11, oracle_mod):
@@ -215,8 +227,14 @@ def test_launch_shape_is_persistent(df11):
     df11.upload(blob)
     grid, block, smem = df11.df11_decode_launch_shape([blob])
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    assert block == 256 + 32  # default: one chunk per decoding thread, plus the producer warp
-    g2, b2, _ = df11.df11_decode_launch_shape([blob], chunks_per_thread=2, ctas_per_sm=1)
-    assert b2 == 256 // 2 + 32 and g2 == min(sms, blob.info().n_tiles)
-    assert grid == min(blob.info().n_tiles, grid) and grid % sms == 0 or grid == blob.info().n_tiles
+    assert block == 16 * 32  # default layout: warp tiles, 16 warps per CTA
+    assert grid % sms == 0 or grid * 16 >= blob.info().n_tiles
+    g8, b8, _ = df11.df11_decode_launch_shape([blob], warps_per_cta=8, ctas_per_sm=1)
+    assert b8 == 8 * 32 and g8 == sms
+    cta = df11.df11_encode(df11.df11_build_codebook("bf16", [x]), x, 128, 256)
+    df11.upload(cta)
+    g1, b1, _ = df11.df11_decode_launch_shape([cta])
+    assert b1 == 256 + 32  # CTA tiles: one chunk per decoding thread plus the producer warp
+    g2, b2, _ = df11.df11_decode_launch_shape([cta], chunks_per_thread=2, ctas_per_sm=1)
+    assert b2 == 256 // 2 + 32 and g2 == min(sms, cta.info().n_tiles)
     assert 0 < smem <= 227 * 1024

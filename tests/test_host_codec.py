@@ -48,7 +48,7 @@ def test_lengths_and_sections_match_oracle(df11, oracle_mod, case):
     cb = df11.df11_build_codebook(dt, [x])
     want = oracle_mod.build_lengths([x], dt)
     assert np.array_equal(cb.lengths(), want)
-    for chunk_bits, tile_threads in [(128, 256), (64, 512), (256, 128)]:
+    for chunk_bits, tile_threads in [(128, 32), (128, 256), (64, 512), (256, 128)]:
         blob = df11.df11_encode(cb, x, chunk_bits, tile_threads)
         o = oracle_mod.compress(x, dt, lengths=want, chunk_bits=chunk_bits, tile_threads=tile_threads)
         info = blob.info()
