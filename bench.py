@@ -179,6 +179,28 @@ def traffic_per_weight():
     return float(t["dram_bytes_per_weight"]), t.get("source")
 
 
+def rank_env() -> tuple[int, int, int]:
+    """(rank, world size, local rank) from the torchrun environment."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(x: float, device) -> float:
+    """Max of a per-rank number over all ranks (identity for one rank)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_rank: float, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job GB/s: bytes decoded by all ranks over the slowest rank's time."""
+    return world * bytes_per_rank * steps / (max_ms / 1e3) / 1e9
+
+
 def host_threads(world: int) -> int:
     try:
         c = len(os.sched_getaffinity(0))
@@ -369,12 +391,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
-    elapsed_ms = start.elapsed_time(end)
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), dev)
     launch_ms = [[e[0].elapsed_time(e[1]) for e in step] for step in ev]
-    if world > 1:
-        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
 
     # ---- correctness outside the timed region: error word + sampled positions
     e = int(err.item())
@@ -431,13 +449,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             e2e_step()
         s1.record(stream)
         s1.synchronize()
-        e2e_ms = s0.elapsed_time(s1) / args.e2e_steps
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(s0.elapsed_time(s1) / args.e2e_steps, dev)
         assert int(err.item()) == 0
-        e2e = {"value": world * out_bytes_total / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
+        e2e = {"value": job_throughput(out_bytes_total, world, 1, e2e_ms), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                "path": "df11_decode_host: pinned host image -> H2D -> decode launch -> D2H of every output"}
         del himgs, hout
@@ -453,7 +467,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if rank != 0:
         return
     ms_per_step = elapsed_ms / args.steps
-    value = world * out_bytes_total * args.steps / (elapsed_ms / 1e3) / 1e9
+    value = job_throughput(out_bytes_total, world, args.steps, elapsed_ms)
     per_launch = np.array(launch_ms)  # steps x groups
     tot_launch_s = per_launch.sum() / 1e3
     algo_step = float(sum(algo))
@@ -498,9 +512,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
 def main():
     args = parse_args()
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local_rank = rank_env()
     if args.impl == "reference":
         run_reference(args, rank, world)
         return
