@@ -404,10 +404,13 @@ __device__ __noinline__ void store_partial(uint8_t *out, uint4 a, uint4 b, uint3
 // Merges group i of a tile: 16 plane bytes p4 with its exponents from shared
 // memory (which are then cleared for the next tile) into 32 output bytes.
 // [lo, hi) are the tile's elements relative to the first group's first element.
-template <int DT>
+template <int DT, bool PARTIAL = true>
 __device__ __forceinline__ void merge_group(uint4 p4, uint32_t i, uint8_t *s_exps, uint8_t *dst_tile, uint32_t lo,
                                             uint32_t hi) {
     constexpr uint32_t GROUP = DT == 0 ? 16u : 32u;
+    if constexpr (!PARTIAL) {
+        if (i * GROUP < lo || i * GROUP + GROUP > hi) return;  // edge group: stored by edge_groups()
+    }
     uint4 a, b;
     if constexpr (DT == 0) {
         uint4 *xp = reinterpret_cast<uint4 *>(s_exps + 16 * i);
@@ -430,11 +433,66 @@ __device__ __forceinline__ void merge_group(uint4 p4, uint32_t i, uint8_t *s_exp
     }
     const uint32_t e0 = i * GROUP;
     uint8_t *out = dst_tile + 32u * i;
-    if (e0 >= lo && e0 + GROUP <= hi) {
+    if (!PARTIAL || (e0 >= lo && e0 + GROUP <= hi)) {
         st_global_v4(out, a);
         st_global_v4(out + 16, b);
     } else {
         store_partial<DT>(out, a, b, e0, lo, hi);
+    }
+}
+
+// The first and last group of a warp tile can be shared with the neighbouring
+// tile.  The whole warp stores them element by element, one element per lane
+// per pass: the group's 16 plane bytes come from the lane that loaded them
+// (shuffled), its exponents from shared memory, which are then cleared.
+template <int DT>
+__device__ __forceinline__ void edge_groups(const uint4 (&pre)[kPrefetchGroups], const uint8_t *plane, uint32_t ng,
+                                            uint8_t *s_exps, uint8_t *dst_tile, uint32_t lo, uint32_t hi, int lane) {
+    constexpr uint32_t GROUP = DT == 0 ? 16u : 32u;
+    const uint32_t last = ng - 1;
+    const bool head = lo != 0, tail = (hi % GROUP) != 0 && !(head && last == 0);
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+        const bool on = which == 0 ? head : tail;
+        if (!on) continue;  // warp-uniform
+        const uint32_t g = which == 0 ? 0u : last;
+        // plane bytes of group g: held by lane g % 32 in pre[g / 32] when g < 32 * kPrefetchGroups
+        uint4 v;
+        const uint32_t u = g / 32u;
+        if (u < kPrefetchGroups) {
+            uint4 mine = pre[0];
+#pragma unroll
+            for (int k = 1; k < kPrefetchGroups; ++k)
+                if (u == static_cast<uint32_t>(k)) mine = pre[k];
+            const int src = static_cast<int>(g % 32u);
+            v.x = __shfl_sync(0xFFFFFFFFu, mine.x, src);
+            v.y = __shfl_sync(0xFFFFFFFFu, mine.y, src);
+            v.z = __shfl_sync(0xFFFFFFFFu, mine.z, src);
+            v.w = __shfl_sync(0xFFFFFFFFu, mine.w, src);
+        } else {
+            v = ld_global_stream_v4(plane + 16u * g);
+        }
+#pragma unroll
+        for (uint32_t j0 = 0; j0 < GROUP; j0 += 32) {
+            const uint32_t j = j0 + static_cast<uint32_t>(lane);
+            if (j < GROUP) {
+                const uint32_t e = g * GROUP + j;
+                const uint32_t x = s_exps[e];
+                s_exps[e] = 0;
+                if (e >= lo && e < hi) {
+                    const uint32_t wi = DT == 0 ? (j >> 2) : (j >> 3);
+                    const uint32_t word = wi == 0 ? v.x : (wi == 1 ? v.y : (wi == 2 ? v.z : v.w));
+                    if constexpr (DT == 0) {
+                        const uint32_t pb = (word >> (8 * (j & 3))) & 0xFFu;
+                        const uint32_t val = ((pb & 0x80u) << 8) | (x << 7) | (pb & 0x7Fu);
+                        reinterpret_cast<uint16_t *>(dst_tile)[e] = static_cast<uint16_t>(val);
+                    } else {
+                        const uint32_t nib = (word >> (4 * (j & 7))) & 0xFu;
+                        dst_tile[e] = static_cast<uint8_t>(((nib & 8u) << 4) | (x << 3) | (nib & 7u));
+                    }
+                }
+            }
+        }
     }
 }
 
@@ -705,9 +763,10 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Tile t's descriptor index (tiles of all tensors are numbered consecutively).
-__device__ __forceinline__ int tensor_of(const DecodeParams &P, uint32_t t) {
-    int ti = 0;
+// Descriptor index of tile t (tiles of all tensors are numbered consecutively),
+// searching forward from `from`: a warp's tiles only increase.
+__device__ __forceinline__ int tensor_of(const DecodeParams &P, uint32_t t, int from = 0) {
+    int ti = from;
     while (ti + 1 < P.n_tensors && t >= P.t[ti + 1].tile_begin) ++ti;
     return ti;
 }
@@ -769,8 +828,10 @@ __global__ void __launch_bounds__(NWARP * 32, NWARP <= 8 ? 4 : 2)
     uint32_t issued = 0;  // bit s: stage s holds a copy not yet waited for
     uint32_t par = 0;     // bit s: phase parity of that copy
     // lane 0: copy tile t's stream slice and gaps into stage s
+    int ti_issue = 0, ti_cur = 0;
     auto issue = [&](uint32_t t, int s) {
-        const TensorDesc &d = P.t[tensor_of(P, t)];
+        ti_issue = tensor_of(P, t, ti_issue);
+        const TensorDesc &d = P.t[ti_issue];
         const uint32_t lt = t - d.tile_begin;
         uint8_t *st = stage0 + s * plan.stage_bytes;
         mbar_arrive_expect_tx(&full[s], TILE_BYTES + 16u + 32u);
@@ -790,7 +851,8 @@ __global__ void __launch_bounds__(NWARP * 32, NWARP <= 8 ? 4 : 2)
     for (uint32_t t = first; t < P.total_tiles; t += stride, ++k) {
         const int s = static_cast<int>(k & 1u);
         const uint32_t ph = (k >> 1) & 1u;
-        const TensorDesc &d = P.t[tensor_of(P, t)];
+        ti_cur = tensor_of(P, t, ti_cur);
+        const TensorDesc &d = P.t[ti_cur];
         const uint32_t lt = t - d.tile_begin;
         uint64_t S = __ldg(d.out_off + lt);
         const uint64_t Eo = __ldg(d.out_off + lt + 1);
@@ -879,10 +941,11 @@ __global__ void __launch_bounds__(NWARP * 32, NWARP <= 8 ? 4 : 2)
 #pragma unroll
             for (int u = 0; u < kPrefetchGroups; ++u) {
                 const uint32_t i = lane + 32u * u;
-                if (i < ng) merge_group<DT>(pre[u], i, s_exps, dst_tile, lo, hi);
+                if (i < ng) merge_group<DT, false>(pre[u], i, s_exps, dst_tile, lo, hi);
             }
             for (uint32_t i = lane + 32u * kPrefetchGroups; i < ng; i += 32)
-                merge_group<DT>(ld_global_stream_v4(plane + 16u * i), i, s_exps, dst_tile, lo, hi);
+                merge_group<DT, false>(ld_global_stream_v4(plane + 16u * i), i, s_exps, dst_tile, lo, hi);
+            edge_groups<DT>(pre, plane, ng, s_exps, dst_tile, lo, hi, lane);
             __syncwarp();
         }
     }
