@@ -283,28 +283,22 @@ __device__ __forceinline__ void count_codes(const uint32_t (&w)[CPT * CW + 1], c
     for (int c = 0; c < CPT; ++c) cnt[c] = (acc[c] >> 8) & 0xFFFu;
 }
 
-// Appends nbits (a multiple of 8, <= 32) of packed symbols `sy` to the
-// pending word lo (fill bits used); every completed 32-bit word is ORed into
-// shared memory at `out`, which then advances.  The exponent buffer is zero
-// before phase 2, so neighbouring chunks can OR into a word they share.
-__device__ __forceinline__ void append(uint32_t sy, uint32_t nbits, uint32_t &lo, uint32_t &fill, uint32_t &out) {
-    const uint32_t vhi = __funnelshift_l(sy, 0u, fill);  // bytes of sy that spill past this word
-    lo |= sy << fill;
-    fill += nbits;
-    if (fill >= 32) {
-        asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(out), "r"(lo) : "memory");
-        out += 4;
-        lo = vhi;
-        fill -= 32;
-    }
+// ORs up to 4 symbol bytes `sy` (unused high bytes zero) into shared memory at
+// byte address out: the one or two 32-bit words they touch.  The exponent
+// buffer is zero before phase 2, so neighbouring chunks can OR into a word
+// they share and the zero high bytes leave other symbols intact.
+__device__ __forceinline__ void put_symbols(uint32_t sy, uint32_t out) {
+    const uint32_t a = out & ~3u, sh = (out & 3u) << 3;
+    asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(a), "r"(sy << sh) : "memory");
+    if (sh) asm volatile("red.shared.or.b32 [%0+4], %1;" ::"r"(a), "r"(__funnelshift_l(sy, 0u, sh)) : "memory");
 }
 
 // Phase 2: decode chunk C again along the same path as phase 1 and write its
-// symbols, packed four to a word, from shared-memory byte address q on.
+// symbols from shared-memory byte address q on.
 template <int CW, int CPT, int C>
 __device__ __forceinline__ void emit_codes(const uint32_t (&w)[CPT * CW + 1], int p, const int E, const Tables &T,
                                            uint32_t q, uint32_t &err) {
-    uint32_t out = q & ~3u, fill = 8u * (q & 3u), lo = 0;
+    uint32_t out = q;
 #pragma unroll
     for (int k = 0; k < CW; ++k) {
         const int er = E - 32 * k;
@@ -317,7 +311,8 @@ __device__ __forceinline__ void emit_codes(const uint32_t (&w)[CPT * CW + 1], in
                 const uint32_t idx = win >> (32 - kMultiBits);
                 const uint32_t mm = T.meta[idx];
                 p += static_cast<int>(mm & 0x7Fu);
-                append(T.syms[idx], (mm >> 5) & 0x38u, lo, fill, out);
+                put_symbols(T.syms[idx], out);
+                out += (mm >> 8) & 7u;
             }
             bool single = false;
             if (p >= 64) {
@@ -332,18 +327,19 @@ __device__ __forceinline__ void emit_codes(const uint32_t (&w)[CPT * CW + 1], in
             if (mm & kMetaLong) {
                 const uint32_t e = lut_decode(win, T, err);
                 p += static_cast<int>((e >> 8) & 0x3Fu);
-                append(e & 0xFFu, 8u, lo, fill, out);
+                put_symbols(e & 0xFFu, out);
+                out += 1;
             } else {
                 const uint32_t nv = starts_before(mm, er - p);
                 const uint32_t nb = 8u * nv;
                 const uint32_t sy = nb >= 32 ? T.syms[idx] : (T.syms[idx] & ((1u << nb) - 1u));
                 p += static_cast<int>(mm & 0x3Fu);
-                if (nb) append(sy, nb, lo, fill, out);
+                if (nv) put_symbols(sy, out);
+                out += nv;
             }
         }
         p -= min(p, 32);
     }
-    if (fill) asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(out), "r"(lo) : "memory");
 }
 
 // ------------------------------------------------------------------ field merges
