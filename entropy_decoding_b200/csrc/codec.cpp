@@ -264,7 +264,8 @@ void build_multi(const uint8_t *lengths, const uint32_t *codes, int nsym, std::v
             ++k;
         }
         if (k) {
-            meta[v] = static_cast<uint32_t>(pos) | (static_cast<uint32_t>(k) << 8) | (starts << kMetaMaskShift);
+            meta[v] = static_cast<uint32_t>(pos) | (static_cast<uint32_t>(k) << kMetaCountShift) |
+                      (starts << kMetaMaskShift);
             syms[v] = packed;
         }
     }
@@ -629,7 +630,8 @@ void write_image(const Blob &b, uint8_t *dst) {
     std::memcpy(dst + L.lut, b.cb->lut.data(), b.cb->lut.size() * 2);
     if (!b.gaps.empty()) std::memcpy(dst + L.gaps, b.gaps.data(), b.gaps.size());
     std::memcpy(dst + L.out_off, b.out_off.data(), b.out_off.size() * 8);
-    if (!b.stream.empty()) std::memcpy(dst + L.stream, b.stream.data(), b.stream.size());
+    // stream as 32-bit words, earliest bit in bit 31 (little-endian storage)
+    for (uint64_t i = 0; i < b.stream.size(); ++i) dst[L.stream + (i ^ 3)] = b.stream[i];
     if (!b.plane.empty()) std::memcpy(dst + L.plane, b.plane.data(), b.plane.size());
 }
 

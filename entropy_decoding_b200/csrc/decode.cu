@@ -107,8 +107,6 @@ __device__ __forceinline__ void consumer_sync(int nthreads) {
     asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }
 
-__device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
-
 __device__ __forceinline__ void report(int *err, uint32_t bits) {
     if (err && bits) atomicOr(err, static_cast<int>(bits));
 }
@@ -195,7 +193,7 @@ __device__ __forceinline__ uint32_t lut_decode(uint32_t win, const Tables &T, ui
 // anything else (a damaged table) becomes the long-code sentinel, whose codes
 // the hierarchical tables then decode one at a time.
 __device__ __forceinline__ uint32_t sane_meta(uint32_t e) {
-    const uint32_t used = e & 0xFFu, n = (e >> 8) & 0xFFFu, mask = e >> kMetaMaskShift;
+    const uint32_t used = e & 0x7FFu, n = (e >> kMetaCountShift) & 0x1FFu, mask = e >> kMetaMaskShift;
     const bool ok = used >= 1 && used <= kMultiBits && n >= 1 && n <= kMultiMaxSyms && (mask & 1u) &&
                     static_cast<uint32_t>(__popc(mask)) == n && mask < (1u << used);
     return ok ? e : kMetaLong;
@@ -206,19 +204,23 @@ __device__ __forceinline__ uint32_t starts_before(uint32_t mm, int room) {
     return static_cast<uint32_t>(__popc((mm >> kMetaMaskShift) & ((1u << room) - 1u)));
 }
 
-// Phase 1: count the codes that start in each of this thread's CPT chunks.
-// Chunk c occupies w[c*CW .. c*CW+CW-1] (most significant bit first) and
-// w[c*CW+CW] is its look-ahead word (the next chunk's first word).  Its walk
-// starts at bit gap[c] and counts codes that start before bit E[c].  The walk
-// moves through the chunk 32 bits at a time ("stage" k reads the word pair
-// w[k], w[k+1]).  While a whole 12-bit window lies before E, one lookup in
-// the multi-symbol table consumes up to 4 codes; in the last 11 bits before
-// E the entry's start mask counts only the codes that start before E; codes
-// longer than 12 bits (the sentinel entry) go through the hierarchical tables.
-// acc = p | count << 8 and an entry is consumed | count << 8 | mask << 20, so
-// one add advances both (the mask bits land above the 12-bit count field);
-// the sentinel adds 64 to p, which ends the loop.  The CPT chunks advance in
-// lockstep so their table lookups overlap.
+// Field masks of a walker's accumulator acc = p | count << kMetaCountShift.
+constexpr uint32_t kPosMask = (1u << kMetaCountShift) - 1u;
+constexpr uint32_t kCountOne = 1u << kMetaCountShift;
+
+// Phase 1 (CTA-tile kernel): count the codes that start in each of this
+// thread's CPT chunks, with the chunk in registers.  Chunk c occupies
+// w[c*CW .. c*CW+CW-1] (earliest bit first) and w[c*CW+CW] is its look-ahead
+// word (the next chunk's first word).  Its walk starts at bit gap[c] and
+// counts codes that start before bit E[c].  The walk moves through the chunk
+// 32 bits at a time ("stage" k reads the word pair w[k], w[k+1]).  While a
+// whole 12-bit window lies before E, one lookup in the multi-symbol table
+// consumes up to 4 codes; in the last 11 bits before E the entry's start mask
+// counts only the codes that start before E; codes longer than 12 bits (the
+// sentinel entry) go through the hierarchical tables.  acc = p | count << 11
+// and an entry is consumed | count << 11 | mask << 20, so one add advances
+// both (the mask lands above the count field); the sentinel adds 1024 to p,
+// which ends the loop.  The CPT chunks advance in lockstep.
 template <int CW, int CPT>
 __device__ __forceinline__ void count_codes(const uint32_t (&w)[CPT * CW + 1], const int (&gap)[CPT],
                                             const int (&E)[CPT], const Tables &T, uint32_t (&cnt)[CPT],
@@ -240,7 +242,7 @@ __device__ __forceinline__ void count_codes(const uint32_t (&w)[CPT * CW + 1], c
                 bool act[CPT], any = false;
 #pragma unroll
                 for (int c = 0; c < CPT; ++c) {
-                    act[c] = static_cast<int>(acc[c] & 0xFFu) < lm[c];
+                    act[c] = static_cast<int>(acc[c] & kPosMask) < lm[c];
                     any |= act[c];
                 }
                 if (!any) break;
@@ -255,11 +257,11 @@ __device__ __forceinline__ void count_codes(const uint32_t (&w)[CPT * CW + 1], c
             bool more = false;
 #pragma unroll
             for (int c = 0; c < CPT; ++c) {
-                int p = static_cast<int>(acc[c] & 0xFFu);
+                int p = static_cast<int>(acc[c] & kPosMask);
                 bool single = false;
-                if (p >= 64) {  // sentinel: the first code is longer than 12 bits
-                    acc[c] -= 64;
-                    p -= 64;
+                if (p >= static_cast<int>(kMetaLong)) {  // sentinel: the first code is longer than 12 bits
+                    acc[c] -= kMetaLong;
+                    p -= kMetaLong;
                     single = true;
                 } else if (p >= ls[c]) {
                     continue;
@@ -268,19 +270,19 @@ __device__ __forceinline__ void count_codes(const uint32_t (&w)[CPT * CW + 1], c
                 const uint32_t mm = single ? kMetaLong : T.meta[win >> (32 - kMultiBits)];
                 if (mm & kMetaLong) {
                     const uint32_t e = lut_decode(win, T, err);
-                    acc[c] += ((e >> 8) & 0x3Fu) + 256u;
+                    acc[c] += ((e >> 8) & 0x3Fu) + kCountOne;
                 } else {  // last bits before E: count only the codes that start before it
-                    acc[c] += (mm & 0x3Fu) + (starts_before(mm, er[c] - p) << 8);
+                    acc[c] += (mm & 0xFu) + (starts_before(mm, er[c] - p) << kMetaCountShift);
                 }
                 more = true;
             }
             if (!more) break;
         }
 #pragma unroll
-        for (int c = 0; c < CPT; ++c) acc[c] -= min(acc[c] & 0xFFu, 32u);
+        for (int c = 0; c < CPT; ++c) acc[c] -= min(acc[c] & kPosMask, 32u);
     }
 #pragma unroll
-    for (int c = 0; c < CPT; ++c) cnt[c] = (acc[c] >> 8) & 0xFFFu;
+    for (int c = 0; c < CPT; ++c) cnt[c] = (acc[c] >> kMetaCountShift) & 0x1FFu;
 }
 
 // ORs up to 4 symbol bytes `sy` (unused high bytes zero) into shared memory at
@@ -293,8 +295,8 @@ __device__ __forceinline__ void put_symbols(uint32_t sy, uint32_t out) {
     if (sh) asm volatile("red.shared.or.b32 [%0+4], %1;" ::"r"(a), "r"(__funnelshift_l(sy, 0u, sh)) : "memory");
 }
 
-// Phase 2: decode chunk C again along the same path as phase 1 and write its
-// symbols from shared-memory byte address q on.
+// Phase 2 (CTA-tile kernel): decode chunk C again along the same path as
+// phase 1 and write its symbols from shared-memory byte address q on.
 template <int CW, int CPT, int C>
 __device__ __forceinline__ void emit_codes(const uint32_t (&w)[CPT * CW + 1], int p, const int E, const Tables &T,
                                            uint32_t q, uint32_t &err) {
@@ -310,13 +312,13 @@ __device__ __forceinline__ void emit_codes(const uint32_t (&w)[CPT * CW + 1], in
                 const uint32_t win = __funnelshift_l(lw, hi, p);
                 const uint32_t idx = win >> (32 - kMultiBits);
                 const uint32_t mm = T.meta[idx];
-                p += static_cast<int>(mm & 0x7Fu);
+                p += static_cast<int>(mm & kPosMask);
                 put_symbols(T.syms[idx], out);
-                out += (mm >> 8) & 7u;
+                out += (mm >> kMetaCountShift) & 7u;
             }
             bool single = false;
-            if (p >= 64) {
-                p -= 64;
+            if (p >= static_cast<int>(kMetaLong)) {
+                p -= kMetaLong;
                 single = true;
             } else if (p >= ls) {
                 break;
@@ -333,7 +335,7 @@ __device__ __forceinline__ void emit_codes(const uint32_t (&w)[CPT * CW + 1], in
                 const uint32_t nv = starts_before(mm, er - p);
                 const uint32_t nb = 8u * nv;
                 const uint32_t sy = nb >= 32 ? T.syms[idx] : (T.syms[idx] & ((1u << nb) - 1u));
-                p += static_cast<int>(mm & 0x3Fu);
+                p += static_cast<int>(mm & 0xFu);
                 if (nv) put_symbols(sy, out);
                 out += nv;
             }
@@ -640,20 +642,20 @@ __global__ void __launch_bounds__(NTH + 32, (NTH + 32) * 3 <= 1024 ? 3 : 1)
 #pragma unroll
             for (int j = 0; j < CPT * CW / 4; ++j) {
                 const uint4 v = *reinterpret_cast<const uint4 *>(sst + 16 * j);
-                w[4 * j + 0] = bswap32(v.x);
-                w[4 * j + 1] = bswap32(v.y);
-                w[4 * j + 2] = bswap32(v.z);
-                w[4 * j + 3] = bswap32(v.w);
+                w[4 * j + 0] = v.x;
+                w[4 * j + 1] = v.y;
+                w[4 * j + 2] = v.z;
+                w[4 * j + 3] = v.w;
             }
         } else {
             const uint2 v = *reinterpret_cast<const uint2 *>(sst);
-            w[0] = bswap32(v.x);
-            w[1] = bswap32(v.y);
+            w[0] = v.x;
+            w[1] = v.y;
         }
         {
             const uint32_t nxt = __shfl_down_sync(0xFFFFFFFFu, w[0], 1);
             w[CPT * CW] =
-                lane == 31 ? bswap32(*reinterpret_cast<const uint32_t *>(sst + CPT * CB / 8)) : nxt;
+                lane == 31 ? *reinterpret_cast<const uint32_t *>(sst + CPT * CB / 8) : nxt;
         }
         int gap[CPT], E[CPT];
         const uint8_t *sg = s_gaps0 + s * gaps_stride + tid * CPT;
@@ -879,19 +881,19 @@ __global__ void __launch_bounds__(NWARP * 32, NWARP <= 8 ? 4 : 2)
 #pragma unroll
             for (int j = 0; j < CW / 4; ++j) {
                 const uint4 v = *reinterpret_cast<const uint4 *>(st + lane * (CB / 8) + 16 * j);
-                w[4 * j + 0] = bswap32(v.x);
-                w[4 * j + 1] = bswap32(v.y);
-                w[4 * j + 2] = bswap32(v.z);
-                w[4 * j + 3] = bswap32(v.w);
+                w[4 * j + 0] = v.x;
+                w[4 * j + 1] = v.y;
+                w[4 * j + 2] = v.z;
+                w[4 * j + 3] = v.w;
             }
         } else {
             const uint2 v = *reinterpret_cast<const uint2 *>(st + lane * (CB / 8));
-            w[0] = bswap32(v.x);
-            w[1] = bswap32(v.y);
+            w[0] = v.x;
+            w[1] = v.y;
         }
         {
             const uint32_t nxt = __shfl_down_sync(0xFFFFFFFFu, w[0], 1);
-            w[CW] = lane == 31 ? bswap32(*reinterpret_cast<const uint32_t *>(st + TILE_BYTES)) : nxt;
+            w[CW] = lane == 31 ? *reinterpret_cast<const uint32_t *>(st + TILE_BYTES) : nxt;
         }
         int gap[1], E[1];
         {

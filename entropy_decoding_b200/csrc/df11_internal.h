@@ -12,10 +12,15 @@
 //   * multi-symbol table (an addition for sm_100a's instruction budget): 4096
 //     entries indexed by the next 12 stream bits, for the longest run of up
 //     to 4 whole codes inside the 12-bit window.  meta[v] (u32) = consumed
-//     bits (bits 0..5) | symbols decoded (bits 8..10) | start mask (bit 20+j
-//     set when one of those codes starts at window offset j); meta[v] =
-//     kMetaLong when the first code is longer than 12 bits.  syms[v] holds
+//     bits (bits 0..3) | symbols decoded (bits 11..13) | start mask (bit 20+j
+//     set when one of those codes starts at window offset j).  Bits 0..10
+//     and 11..19 line up with a walker's accumulator (bit position | count
+//     << 11), so one add advances both.  meta[v] = kMetaLong (consumed 1024,
+//     no symbol) when the first code is longer than 12 bits.  syms[v] holds
 //     the symbols, first in the low byte, unused bytes zero.
+//   * in the device image the stream is stored as 32-bit words whose bit 31
+//     is the earliest stream bit (each 4-byte group of the MSB-first byte
+//     stream reversed), so a word load needs no byte swap.
 #pragma once
 
 #include <cstdint>
@@ -25,7 +30,8 @@ namespace df11 {
 constexpr int kMultiBits = 12;
 constexpr int kMultiEntries = 1 << kMultiBits;
 constexpr int kMultiMaxSyms = 4;
-constexpr uint32_t kMetaLong = 0x0040;
+constexpr uint32_t kMetaLong = 0x0400;
+constexpr int kMetaCountShift = 11;
 constexpr int kMetaMaskShift = 20;
 
 constexpr int kLutEntries = 256;

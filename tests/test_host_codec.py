@@ -150,9 +150,9 @@ def test_decode_tables_match_independent_prefix_decode(df11, oracle_mod, case):
             got.append(r[0])
             pos += r[1]
         if not got:
-            assert meta[v] == 0x40, v
+            assert meta[v] == 0x400, v
         else:
-            assert meta[v] == pos | (len(got) << 8) | (starts << 20), v
+            assert meta[v] == pos | (len(got) << 11) | (starts << 20), v
             assert [(int(syms[v]) >> (8 * i)) & 0xFF for i in range(len(got))] == got
     lut = img[lay["lut"]:lay["lut"] + lay["n_luts"] * 512].view(np.uint16)
     rng = np.random.default_rng(0)
@@ -255,8 +255,9 @@ def test_device_image_layout(df11):
     s = blob.sections()
     tile_bytes = info.chunk_bits // 8 * info.tile_threads
     stream = img[lay["stream"]:lay["plane"]]
-    assert np.array_equal(stream[: s["stream"].size], s["stream"])
+    words = stream[: (stream.size // 4) * 4].reshape(-1, 4)[:, ::-1].reshape(-1)  # back to MSB-first bytes
+    assert np.array_equal(words[: s["stream"].size], s["stream"])
     assert stream.size >= info.n_tiles * tile_bytes + 16
-    assert not stream[s["stream"].size:].any()
+    assert not words[s["stream"].size:].any()
     assert np.array_equal(img[lay["plane"]:lay["plane"] + info.plane_bytes], s["plane"])
     assert lay["total"] - lay["plane"] >= info.plane_bytes + 32
