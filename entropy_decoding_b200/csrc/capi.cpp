@@ -8,6 +8,7 @@
 
 #include "df11.h"
 #include "codec.h"
+#include "encode.h"
 #include "launch.h"
 
 struct df11_codebook {
@@ -16,6 +17,15 @@ struct df11_codebook {
 
 struct df11_blob {
     df11::Blob b;
+};
+
+struct df11_encoding {
+    df11::EncodeJob job;
+    uint64_t *scratch = nullptr;
+    cudaStream_t stream = nullptr;
+    uint64_t total_bits = 0;
+    uint64_t image_bytes = 0;
+    bool packed = false;
 };
 
 namespace {
@@ -139,10 +149,10 @@ df11_status df11_blob_get_info(const df11_blob *blob, df11_blob_info *info) {
     info->total_bits = b.total_bits;
     info->n_tiles = b.n_tiles;
     info->max_span = b.max_span;
-    info->stream_bytes = b.stream.size();
-    info->plane_bytes = b.plane.size();
-    info->gaps_bytes = b.gaps.size();
-    info->out_off_bytes = b.out_off.size() * 8;
+    info->stream_bytes = (b.total_bits + 7) / 8;
+    info->plane_bytes = df11::plane_bytes(b.dtype, b.n);
+    info->gaps_bytes = b.n_tiles * static_cast<uint64_t>(b.tile_threads);
+    info->out_off_bytes = (b.n_tiles + 1) * 8;
     info->serialized_bytes = df11::serialized_bytes(b);
     info->device_bytes = df11::image_layout(b).total;
     info->uncompressed_bytes = b.dtype == df11::kBF16 ? 2 * b.n : b.n;
@@ -151,7 +161,7 @@ df11_status df11_blob_get_info(const df11_blob *blob, df11_blob_info *info) {
 
 df11_status df11_blob_sections(const df11_blob *blob, const uint8_t **stream, const uint8_t **plane,
                                const uint8_t **gaps, const uint64_t **out_off) {
-    if (!blob) return DF11_EINVAL;
+    if (!blob || blob->b.device_only) return DF11_EINVAL;
     if (stream) *stream = blob->b.stream.data();
     if (plane) *plane = blob->b.plane.data();
     if (gaps) *gaps = blob->b.gaps.data();
@@ -166,7 +176,7 @@ df11_status df11_blob_lengths(const df11_blob *blob, uint8_t *lengths) {
 }
 
 df11_status df11_serialize(const df11_blob *blob, void *buf, uint64_t cap, uint64_t *used) {
-    if (!blob) return DF11_EINVAL;
+    if (!blob || blob->b.device_only) return DF11_EINVAL;
     uint64_t need = df11::serialized_bytes(blob->b);
     if (used) *used = need;
     if (!buf || cap < need) return DF11_ENOMEM;
@@ -192,7 +202,7 @@ df11_status df11_deserialize(const void *buf, uint64_t len, df11_blob **out) {
 }
 
 df11_status df11_blob_device_image(const df11_blob *blob, void *host_dst, uint64_t cap) {
-    if (!blob || !host_dst) return DF11_EINVAL;
+    if (!blob || !host_dst || blob->b.device_only) return DF11_EINVAL;
     if (cap < df11::image_layout(blob->b).total) return DF11_ENOMEM;
     df11::write_image(blob->b, static_cast<uint8_t *>(host_dst));
     return DF11_OK;
@@ -208,7 +218,7 @@ df11_status df11_blob_bind(df11_blob *blob, const void *dev_image, uint64_t cap)
 }
 
 df11_status df11_blob_upload(df11_blob *blob, void *dev_dst, uint64_t cap, df11_stream stream) {
-    if (!blob || !dev_dst) return DF11_EINVAL;
+    if (!blob || !dev_dst || blob->b.device_only) return DF11_EINVAL;
     if (reinterpret_cast<uintptr_t>(dev_dst) % df11::kImageAlign) return DF11_EINVAL;
     const uint64_t need = df11::image_layout(blob->b).total;
     if (cap < need) return DF11_ENOMEM;
@@ -304,6 +314,143 @@ df11_status df11_decode_launch_shape_ex(const df11_blob *const *blobs, int n_blo
     if (block) *block = sh.block;
     if (smem_bytes) *smem_bytes = sh.smem;
     return DF11_OK;
+}
+
+// ---------------------------------------------------------------- GPU encoder
+
+df11_status df11_histogram_device(df11_dtype dtype, const void *src_dev, uint64_t n_elems, uint64_t *counts_dev,
+                                  df11_stream stream) {
+    if (!valid_dtype(dtype) || !counts_dev || (n_elems && !src_dev)) return DF11_EINVAL;
+    if (reinterpret_cast<uintptr_t>(src_dev) % 16) return DF11_EINVAL;
+    return df11::launch_histogram(dtype, src_dev, n_elems, counts_dev, reinterpret_cast<cudaStream_t>(stream))
+               ? DF11_OK
+               : DF11_ECUDA;
+}
+
+df11_status df11_codebook_from_counts(df11_dtype dtype, const uint64_t *counts, int n_counts, int max_code_len,
+                                      df11_codebook **out) {
+    if (!out || !counts || !valid_dtype(dtype) || n_counts != df11::nsym_of(dtype)) return DF11_EINVAL;
+    if (max_code_len == 0) max_code_len = df11::kMaxCodeLen;
+    if (max_code_len < 1 || max_code_len > df11::kMaxCodeLen) return DF11_EINVAL;
+    *out = nullptr;
+    try {
+        uint64_t c[256] = {};
+        std::memcpy(c, counts, static_cast<size_t>(n_counts) * 8);
+        uint8_t lengths[256] = {};
+        if (!df11::code_lengths(c, n_counts, max_code_len, lengths)) return DF11_EINVAL;
+        auto cb = df11::make_codebook(dtype, lengths);
+        if (!cb) return DF11_EINVAL;
+        *out = new df11_codebook{cb};
+        return DF11_OK;
+    } catch (const std::bad_alloc &) {
+        return DF11_ENOMEM;
+    }
+}
+
+uint64_t df11_encode_device_scratch_bytes(uint64_t n_elems) { return df11::encode_scratch_bytes(n_elems); }
+
+df11_status df11_encode_device_begin(const df11_codebook *cb, const void *src_dev, uint64_t n_elems, int chunk_bits,
+                                     int tile_threads, void *scratch_dev, uint64_t scratch_cap, df11_stream stream,
+                                     uint64_t *image_bytes, df11_encoding **out) {
+    if (!cb || !out || !image_bytes || !scratch_dev || (n_elems && !src_dev)) return DF11_EINVAL;
+    if (!df11::valid_layout(chunk_bits, tile_threads)) return DF11_EINVAL;
+    if (reinterpret_cast<uintptr_t>(src_dev) % 16 || reinterpret_cast<uintptr_t>(scratch_dev) % 16) return DF11_EINVAL;
+    if (scratch_cap < df11::encode_scratch_bytes(n_elems)) return DF11_ENOMEM;
+    *out = nullptr;
+    try {
+        auto *enc = new df11_encoding;
+        enc->job.cb = cb->cb;
+        enc->job.src = src_dev;
+        enc->job.n = n_elems;
+        enc->job.chunk_bits = chunk_bits;
+        enc->job.tile_threads = tile_threads;
+        enc->scratch = static_cast<uint64_t *>(scratch_dev);
+        enc->stream = reinterpret_cast<cudaStream_t>(stream);
+        std::string err = df11::encode_device_bits(enc->job, enc->scratch, enc->stream, &enc->total_bits);
+        if (!err.empty()) {
+            delete enc;
+            return err.find("cover") != std::string::npos ? DF11_EINVAL : DF11_ECUDA;
+        }
+        df11::Blob meta;
+        meta.dtype = cb->cb->dtype;
+        meta.chunk_bits = chunk_bits;
+        meta.tile_threads = tile_threads;
+        meta.n = n_elems;
+        meta.total_bits = enc->total_bits;
+        const uint64_t cbits = static_cast<uint64_t>(chunk_bits);
+        meta.n_tiles = ((enc->total_bits + cbits - 1) / cbits + tile_threads - 1) / tile_threads;
+        meta.cb = cb->cb;
+        enc->image_bytes = df11::image_layout(meta).total;
+        *image_bytes = enc->image_bytes;
+        *out = enc;
+        return DF11_OK;
+    } catch (const std::bad_alloc &) {
+        return DF11_ENOMEM;
+    }
+}
+
+df11_status df11_encode_device_end(df11_encoding *enc, void *image_dev, uint64_t image_cap, df11_blob **out) {
+    if (!enc || !image_dev || !out || enc->packed) return DF11_EINVAL;
+    if (reinterpret_cast<uintptr_t>(image_dev) % df11::kImageAlign) return DF11_EINVAL;
+    if (image_cap < enc->image_bytes) return DF11_ENOMEM;
+    *out = nullptr;
+    try {
+        auto *blob = new df11_blob;
+        df11::Blob &b = blob->b;
+        b.dtype = enc->job.cb->dtype;
+        b.chunk_bits = enc->job.chunk_bits;
+        b.tile_threads = enc->job.tile_threads;
+        b.n = enc->job.n;
+        b.total_bits = enc->total_bits;
+        const uint64_t cbits = static_cast<uint64_t>(b.chunk_bits);
+        b.n_tiles = ((b.total_bits + cbits - 1) / cbits + b.tile_threads - 1) / b.tile_threads;
+        b.cb = enc->job.cb;
+        b.device_only = true;
+        const df11::ImageLayout L = df11::image_layout(b);
+        if (b.n) {
+            std::string err = df11::encode_device_pack(enc->job, enc->scratch, b.total_bits, L,
+                                                       static_cast<uint8_t *>(image_dev), enc->stream, &b.max_span);
+            if (!err.empty()) {
+                delete blob;
+                return DF11_ECUDA;
+            }
+        } else {
+            std::vector<uint8_t> img(L.total, 0);
+            df11::write_image_head(b, L, img.data());
+            if (cudaMemcpyAsync(image_dev, img.data(), img.size(), cudaMemcpyHostToDevice, enc->stream) !=
+                    cudaSuccess ||
+                cudaStreamSynchronize(enc->stream) != cudaSuccess) {
+                delete blob;
+                return DF11_ECUDA;
+            }
+        }
+        b.dev_image = static_cast<const uint8_t *>(image_dev);
+        b.dev_cap = image_cap;
+        enc->packed = true;
+        *out = blob;
+        return DF11_OK;
+    } catch (const std::bad_alloc &) {
+        return DF11_ENOMEM;
+    }
+}
+
+void df11_encoding_free(df11_encoding *enc) { delete enc; }
+
+df11_status df11_blob_fetch(df11_blob *blob, df11_stream stream) {
+    if (!blob || !blob->b.dev_image) return DF11_EINVAL;
+    if (!blob->b.device_only) return DF11_OK;
+    try {
+        const df11::ImageLayout L = df11::image_layout(blob->b);
+        std::vector<uint8_t> img(L.total);
+        cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+        if (cudaMemcpyAsync(img.data(), blob->b.dev_image, L.total, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+            cudaStreamSynchronize(s) != cudaSuccess)
+            return DF11_ECUDA;
+        df11::read_image_sections(blob->b, img.data());
+        return DF11_OK;
+    } catch (const std::bad_alloc &) {
+        return DF11_ENOMEM;
+    }
 }
 
 }  // extern "C"

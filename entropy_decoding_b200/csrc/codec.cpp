@@ -599,20 +599,19 @@ ImageLayout image_layout(const Blob &b) {
     L.lut = o;
     o = align_up(o + b.cb->lut.size() * 2, kImageAlign);
     L.gaps = o;
-    o = align_up(o + b.gaps.size(), kImageAlign);
+    o = align_up(o + b.n_tiles * static_cast<uint64_t>(b.tile_threads), kImageAlign);
     L.out_off = o;
-    o = align_up(o + b.out_off.size() * 8, kImageAlign);
+    o = align_up(o + (b.n_tiles + 1) * 8, kImageAlign);
     L.stream = o;
     o = align_up(o + b.n_tiles * (static_cast<uint64_t>(b.chunk_bits) / 8) * b.tile_threads + kStreamTail, kImageAlign);
     L.plane = o;
-    o = align_up(o + align_up(b.plane.size(), 16) + kPlaneTail, kImageAlign);
+    o = align_up(o + align_up(plane_bytes(b.dtype, b.n), 16) + kPlaneTail, kImageAlign);
     L.total = o;
     return L;
 }
 
-void write_image(const Blob &b, uint8_t *dst) {
-    ImageLayout L = image_layout(b);
-    std::memset(dst, 0, L.total);
+void write_image_head(const Blob &b, const ImageLayout &L, uint8_t *dst) {
+    std::memset(dst, 0, L.gaps);
     ImageHeader h{};
     std::memcpy(h.magic, "DF11IMG1", 8);
     h.dtype = static_cast<uint32_t>(b.dtype);
@@ -628,11 +627,28 @@ void write_image(const Blob &b, uint8_t *dst) {
     std::memcpy(dst + L.meta, b.cb->meta.data(), kMultiEntries * 4);
     std::memcpy(dst + L.syms, b.cb->syms.data(), kMultiEntries * 4);
     std::memcpy(dst + L.lut, b.cb->lut.data(), b.cb->lut.size() * 2);
+}
+
+void write_image(const Blob &b, uint8_t *dst) {
+    ImageLayout L = image_layout(b);
+    std::memset(dst, 0, L.total);
+    write_image_head(b, L, dst);
     if (!b.gaps.empty()) std::memcpy(dst + L.gaps, b.gaps.data(), b.gaps.size());
     std::memcpy(dst + L.out_off, b.out_off.data(), b.out_off.size() * 8);
     // stream as 32-bit words, earliest bit in bit 31 (little-endian storage)
     for (uint64_t i = 0; i < b.stream.size(); ++i) dst[L.stream + (i ^ 3)] = b.stream[i];
     if (!b.plane.empty()) std::memcpy(dst + L.plane, b.plane.data(), b.plane.size());
+}
+
+void read_image_sections(Blob &b, const uint8_t *img) {
+    const ImageLayout L = image_layout(b);
+    b.gaps.assign(img + L.gaps, img + L.gaps + b.n_tiles * b.tile_threads);
+    b.out_off.resize(b.n_tiles + 1);
+    std::memcpy(b.out_off.data(), img + L.out_off, (b.n_tiles + 1) * 8);
+    b.stream.resize((b.total_bits + 7) / 8);
+    for (uint64_t i = 0; i < b.stream.size(); ++i) b.stream[i] = img[L.stream + (i ^ 3)];
+    b.plane.assign(img + L.plane, img + L.plane + plane_bytes(b.dtype, b.n));
+    b.device_only = false;
 }
 
 }  // namespace df11

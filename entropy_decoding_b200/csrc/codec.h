@@ -41,6 +41,7 @@ struct Blob {
     std::vector<uint8_t> plane;     // n (BF16) or ceil(n / 2) (E4M3)
     std::vector<uint8_t> gaps;      // n_tiles * tile_threads
     std::vector<uint64_t> out_off;  // n_tiles + 1
+    bool device_only = false;  // encoded on the GPU: host sections empty until fetched
     const uint8_t *dev_image = nullptr;
     uint64_t dev_cap = 0;
     std::vector<uint8_t> host_image;  // staging copy kept alive for df11_blob_upload
@@ -65,6 +66,10 @@ std::string deserialize(const uint8_t *src, uint64_t len, Blob *out);
 
 ImageLayout image_layout(const Blob &b);
 void write_image(const Blob &b, uint8_t *dst);
+// The image's header and decode tables: bytes [0, L.gaps).
+void write_image_head(const Blob &b, const ImageLayout &L, uint8_t *dst);
+// Host sections of a blob back from its device image (inverse of write_image).
+void read_image_sections(Blob &b, const uint8_t *img);
 
 bool valid_layout(int chunk_bits, int tile_threads);
 

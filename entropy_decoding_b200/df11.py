@@ -84,6 +84,13 @@ _SIGS = {
     "df11_decode_ex": ([_PP, _PP, _I, _P, _P, ctypes.POINTER(DecodeOpts)], _S),
     "df11_decode_launch_shape_ex": ([_PP, _I, ctypes.POINTER(DecodeOpts), ctypes.POINTER(_I), ctypes.POINTER(_I),
                                      ctypes.POINTER(_I)], _S),
+    "df11_histogram_device": ([_I, _P, _U64, _P, _P], _S),
+    "df11_codebook_from_counts": ([_I, _P, _I, _I, _PP], _S),
+    "df11_encode_device_scratch_bytes": ([_U64], _U64),
+    "df11_encode_device_begin": ([_P, _P, _U64, _I, _I, _P, _U64, _P, ctypes.POINTER(_U64), _PP], _S),
+    "df11_encode_device_end": ([_P, _P, _U64, _PP], _S),
+    "df11_encoding_free": ([_P], None),
+    "df11_blob_fetch": ([_P, _P], _S),
     "df11_decode_host": ([_PP, _PP, _PP, _PP, _PP, _I, _P, _P], _S),
     "df11_decode_launch_shape": ([_PP, _I, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I)], _S),
 }
@@ -277,6 +284,56 @@ def df11_decode_launch_shape(blobs, chunks_per_thread: int = 0, ctas_per_sm: int
     return g.value, b.value, s.value
 
 
+def df11_histogram_device(dtype: str, src_ptr: int, n: int, counts_ptr: int, stream: int = 0):
+    _check(_lib.df11_histogram_device(DTYPES[dtype], src_ptr or None, n, counts_ptr, stream or None),
+           "df11_histogram_device")
+
+
+def df11_codebook_from_counts(dtype: str, counts, max_code_len: int = 0) -> Codebook:
+    c = np.ascontiguousarray(counts, np.uint64)
+    out = ctypes.c_void_p()
+    _check(_lib.df11_codebook_from_counts(DTYPES[dtype], c.ctypes.data, c.size, max_code_len, ctypes.byref(out)),
+           "df11_codebook_from_counts")
+    return Codebook(out.value, dtype)
+
+
+def df11_encode_device_scratch_bytes(n: int) -> int:
+    return int(_lib.df11_encode_device_scratch_bytes(n))
+
+
+class Encoding:
+    def __init__(self, handle: int, image_bytes: int):
+        self._h = ctypes.c_void_p(handle)
+        self.image_bytes = image_bytes
+
+    def __del__(self, _free=_lib.df11_encoding_free):
+        if getattr(self, "_h", None) and self._h.value:
+            _free(self._h)
+            self._h = ctypes.c_void_p(0)
+
+
+def df11_encode_device_begin(cb: Codebook, src_ptr: int, n: int, chunk_bits: int = 128, tile_threads: int = 32,
+                             scratch_ptr: int = 0, scratch_cap: int = 0, stream: int = 0) -> Encoding:
+    nbytes = _U64()
+    out = ctypes.c_void_p()
+    _check(_lib.df11_encode_device_begin(cb.handle, src_ptr or None, n, chunk_bits, tile_threads, scratch_ptr or None,
+                                         scratch_cap, stream or None, ctypes.byref(nbytes), ctypes.byref(out)),
+           "df11_encode_device_begin")
+    return Encoding(out.value, nbytes.value)
+
+
+def df11_encode_device_end(enc: Encoding, image_ptr: int, image_cap: int, keep=None) -> Blob:
+    out = ctypes.c_void_p()
+    _check(_lib.df11_encode_device_end(enc._h, image_ptr, image_cap, ctypes.byref(out)), "df11_encode_device_end")
+    b = Blob(out.value)
+    b._keep = keep
+    return b
+
+
+def df11_blob_fetch(blob: Blob, stream: int = 0):
+    _check(_lib.df11_blob_fetch(blob.handle, stream or None), "df11_blob_fetch")
+
+
 # ----------------------------------------------------------------- torch-side helpers (device memory only)
 
 def upload(blob: Blob, stream=None):
@@ -290,6 +347,20 @@ def upload(blob: Blob, stream=None):
     s = stream.cuda_stream if stream is not None else torch.cuda.current_stream().cuda_stream
     df11_blob_upload(blob, base + off, n, s, keep=dev)
     return dev
+
+
+def encode_on_device(cb: Codebook, x_dev, chunk_bits: int = 128, tile_threads: int = 32, stream=None) -> Blob:
+    """GPU encode of a torch device tensor (raw uint16 / uint8 bits); scratch
+    and the image are allocated with torch.  Returns a blob bound to its image."""
+    import torch
+    s = stream.cuda_stream if stream is not None else torch.cuda.current_stream().cuda_stream
+    n = x_dev.numel()
+    scratch = torch.empty(df11_encode_device_scratch_bytes(n), dtype=torch.uint8, device=x_dev.device)
+    enc = df11_encode_device_begin(cb, x_dev.data_ptr(), n, chunk_bits, tile_threads, scratch.data_ptr(),
+                                   scratch.numel(), s)
+    img = torch.empty(enc.image_bytes + 256, dtype=torch.uint8, device=x_dev.device)
+    base = img.data_ptr() + (-img.data_ptr()) % 256
+    return df11_encode_device_end(enc, base, enc.image_bytes, keep=img)
 
 
 def elem_bytes(dtype: str) -> int:

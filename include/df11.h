@@ -67,6 +67,7 @@ typedef struct CUstream_st *df11_stream;
 
 typedef struct df11_codebook df11_codebook; /* host object: code lengths + decode tables */
 typedef struct df11_blob df11_blob;         /* host object: one compressed tensor */
+typedef struct df11_encoding df11_encoding; /* host object: a GPU encode between its two steps */
 
 /* Library version: major * 10000 + minor * 100 + patch. */
 int df11_version(void);
@@ -164,7 +165,8 @@ typedef struct {
 df11_status df11_blob_get_info(const df11_blob *blob, df11_blob_info *info);
 
 /* Read-only host views of the blob's sections (valid until the blob is freed);
- * any output pointer may be NULL. */
+ * any output pointer may be NULL.  DF11_EINVAL for a GPU-encoded blob that
+ * was not fetched (df11_blob_fetch). */
 df11_status df11_blob_sections(const df11_blob *blob, const uint8_t **stream, const uint8_t **plane,
                                const uint8_t **gaps, const uint64_t **out_off);
 
@@ -255,6 +257,57 @@ df11_status df11_decode_launch_shape(const df11_blob *const *blobs, int n_blobs,
 df11_status df11_decode_launch_shape_ex(const df11_blob *const *blobs, int n_blobs,
                                         const df11_decode_opts *opts, int *grid, int *block,
                                         int *smem_bytes);
+
+/* ---------------------------------------------------------------------
+ * GPU encoder (the offline half, run on the device)
+ * ------------------------------------------------------------------ */
+
+/* Adds the exponent histogram of a device tensor into counts_dev (device
+ * array of 256 uint64 for BF16, 16 for E4M3; the caller zeroes it), on
+ * `stream`, asynchronously.  src_dev must be 16-byte aligned.  Errors:
+ * DF11_EINVAL, DF11_ECUDA. */
+df11_status df11_histogram_device(df11_dtype dtype, const void *src_dev, uint64_t n_elems,
+                                  uint64_t *counts_dev, df11_stream stream);
+
+/* Builds a codebook from exponent counts (host array of 256 / 16 uint64, e.g.
+ * copied back from df11_histogram_device): the same code construction as
+ * df11_build_codebook.  Errors: DF11_EINVAL, DF11_ENOMEM. */
+df11_status df11_codebook_from_counts(df11_dtype dtype, const uint64_t *counts, int n_counts,
+                                      int max_code_len, df11_codebook **out);
+
+/* Device scratch bytes df11_encode_device_begin needs for n_elems weights
+ * (8 bytes per 4096 weights plus 1.3 KB). */
+uint64_t df11_encode_device_scratch_bytes(uint64_t n_elems);
+
+/* GPU encode, step 1: computes every code length on the device, scans them
+ * and returns the exact device-image size in *image_bytes.  Synchronises
+ * `stream` once (to read the stream length back).  src_dev (the raw weights,
+ * 16-byte aligned) and scratch_dev (>= df11_encode_device_scratch_bytes,
+ * 16-byte aligned) must stay valid until df11_encode_device_end.  Errors:
+ * DF11_EINVAL (bad arguments, or an exponent the code does not cover),
+ * DF11_ENOMEM (scratch too small), DF11_ECUDA. */
+df11_status df11_encode_device_begin(const df11_codebook *cb, const void *src_dev, uint64_t n_elems,
+                                     int chunk_bits, int tile_threads, void *scratch_dev,
+                                     uint64_t scratch_cap, df11_stream stream, uint64_t *image_bytes,
+                                     df11_encoding **out);
+
+/* GPU encode, step 2: writes the device image (byte-identical to the one
+ * df11_blob_device_image produces for the same tensor and codebook) into
+ * image_dev (256-byte aligned, >= *image_bytes of step 1) and returns a blob
+ * bound to it, ready for df11_decode.  Synchronises the stream once (to read
+ * the largest tile span).  The blob's host sections are empty until
+ * df11_blob_fetch.  Errors: DF11_EINVAL, DF11_ENOMEM, DF11_ECUDA. */
+df11_status df11_encode_device_end(df11_encoding *enc, void *image_dev, uint64_t image_cap,
+                                   df11_blob **out);
+
+void df11_encoding_free(df11_encoding *enc);
+
+/* Copies a GPU-encoded blob's sections back from its device image into host
+ * memory (synchronises `stream`), after which df11_serialize,
+ * df11_blob_sections and df11_blob_device_image work on it.  A no-op for
+ * host-encoded blobs.  Errors: DF11_EINVAL (unbound), DF11_ENOMEM,
+ * DF11_ECUDA. */
+df11_status df11_blob_fetch(df11_blob *blob, df11_stream stream);
 
 #ifdef __cplusplus
 }
