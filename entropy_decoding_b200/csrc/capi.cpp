@@ -453,4 +453,31 @@ df11_status df11_blob_fetch(df11_blob *blob, df11_stream stream) {
     }
 }
 
+df11_status df11_encode_device_noalloc(const df11_codebook *cb, const void *src_dev, uint64_t n_elems,
+                                       int chunk_bits, int tile_threads, void *image_dev, uint64_t image_cap,
+                                       df11_stream stream, df11_encode_result *result) {
+    if (!cb || !result || !image_dev || (n_elems && !src_dev)) return DF11_EINVAL;
+    if (!df11::valid_layout(chunk_bits, tile_threads)) return DF11_EINVAL;
+    if (n_elems > df11::noalloc_max_elems()) return DF11_EINVAL;
+    if (reinterpret_cast<uintptr_t>(src_dev) % 16 || reinterpret_cast<uintptr_t>(image_dev) % df11::kImageAlign)
+        return DF11_EINVAL;
+    df11::EncodeJob job;
+    job.cb = cb->cb;
+    job.src = src_dev;
+    job.n = n_elems;
+    job.chunk_bits = chunk_bits;
+    job.tile_threads = tile_threads;
+    df11::NoallocResult r{};
+    const std::string err = df11::encode_device_noalloc(job, static_cast<uint8_t *>(image_dev), image_cap,
+                                                        reinterpret_cast<cudaStream_t>(stream), &r);
+    result->image_bytes = r.image_bytes;
+    result->total_bits = r.total_bits;
+    result->n_tiles = r.n_tiles;
+    result->max_span = r.max_span;
+    if (err.empty()) return DF11_OK;
+    if (err.find("too small") != std::string::npos) return DF11_ENOMEM;
+    if (err.find("cover") != std::string::npos) return DF11_EINVAL;
+    return DF11_ECUDA;
+}
+
 }  // extern "C"

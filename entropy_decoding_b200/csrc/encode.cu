@@ -16,6 +16,7 @@
 #include <cstddef>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "df11.h"
@@ -422,6 +423,124 @@ std::string encode_device_pack(const EncodeJob &J, uint64_t *scratch, uint64_t t
         cudaStreamSynchronize(s) != cudaSuccess)
         return "header update failed";
     *max_span = ms;
+    return "";
+}
+
+// ---------------------------------------------------------------- encoding without allocation
+//
+// For callers that cannot allocate device memory when they encode (see
+// df11_encode_device_noalloc in df11.h): the encoder's scratch lives in one
+// static device array per GPU instead of a caller buffer.
+
+namespace {
+
+constexpr uint64_t kNoallocScratchWords = 65536;  // 512 KB on every GPU that loads the library
+__device__ __align__(256) uint64_t g_noalloc_scratch[kNoallocScratchWords];
+
+std::mutex g_noalloc_mu;
+constexpr int kNoallocDevices = 64;
+uint64_t *g_noalloc_addr[kNoallocDevices] = {};
+
+}  // namespace
+
+uint64_t noalloc_max_elems() { return (kNoallocScratchWords - (2 + 32 + 128 + 1)) * kSegElems; }
+
+std::string encode_device_noalloc(const EncodeJob &J, uint8_t *image, uint64_t image_cap, cudaStream_t s,
+                                  NoallocResult *r) {
+    // device address of the static scratch on the current device, looked up
+    // once per device (host code cannot use the symbol itself)
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocDevices) return "no current device";
+    uint64_t *scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_noalloc_mu);
+        if (!g_noalloc_addr[dev]) {
+            void *p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return "scratch lookup failed";
+            g_noalloc_addr[dev] = static_cast<uint64_t *>(p);
+        }
+        scratch = g_noalloc_addr[dev];
+    }
+    // pass 1: every slot it reads is written first (sums, total, flag)
+    uint64_t total = 0;
+    std::string err = encode_device_bits(J, scratch, s, &total);
+    if (!err.empty()) return err;
+    Blob meta;  // metadata only: its sections stay empty
+    meta.dtype = J.cb->dtype;
+    meta.chunk_bits = J.chunk_bits;
+    meta.tile_threads = J.tile_threads;
+    meta.n = J.n;
+    meta.total_bits = total;
+    const uint64_t cbits = static_cast<uint64_t>(J.chunk_bits);
+    const uint64_t n_chunks = (total + cbits - 1) / cbits;
+    meta.n_tiles = (n_chunks + J.tile_threads - 1) / J.tile_threads;
+    meta.cb = J.cb;
+    const ImageLayout L = image_layout(meta);
+    r->image_bytes = L.total;
+    r->total_bits = total;
+    r->n_tiles = meta.n_tiles;
+    r->max_span = 0;
+    if (image_cap < L.total) return "image buffer too small";
+    // header and decode tables, copied from the codebook without a staging buffer
+    ImageHeader h{};
+    std::memcpy(h.magic, "DF11IMG1", 8);
+    h.dtype = static_cast<uint32_t>(meta.dtype);
+    h.chunk_bits = static_cast<uint32_t>(meta.chunk_bits);
+    h.tile_threads = static_cast<uint32_t>(meta.tile_threads);
+    h.n_luts = static_cast<uint32_t>(J.cb->n_luts());
+    h.n_elems = meta.n;
+    h.total_bits = total;
+    h.n_tiles = meta.n_tiles;
+    h.layout = L;
+    if (cudaMemsetAsync(image, 0, L.total, s) != cudaSuccess ||
+        cudaMemcpyAsync(image, &h, sizeof h, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(image + L.meta, J.cb->meta.data(), kMultiEntries * 4, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(image + L.syms, J.cb->syms.data(), kMultiEntries * 4, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(image + L.lut, J.cb->lut.data(), J.cb->lut.size() * 2, cudaMemcpyHostToDevice, s) !=
+            cudaSuccess)
+        return "table upload failed";
+    if (!J.n) return cudaStreamSynchronize(s) == cudaSuccess ? "" : "synchronise failed";
+    // pass 2, as in encode_device_pack
+    const uint64_t n_seg = segments_of(J.n);
+    uint64_t *out_off = reinterpret_cast<uint64_t *>(image + L.out_off);
+    fill_u64_kernel<<<grid_for((meta.n_tiles + 1 + 255) / 256), 256, 0, s>>>(out_off, meta.n_tiles + 1, J.n);
+    uint8_t *dev_len = reinterpret_cast<uint8_t *>(scratch + n_seg + 2);
+    uint32_t *dev_codes = reinterpret_cast<uint32_t *>(scratch + n_seg + 2 + 32);
+    if (cudaMemcpyAsync(dev_codes, J.cb->codes, 1024, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return "copy of codes failed";
+    PackArgs A;
+    A.src = J.src;
+    A.n = J.n;
+    A.lengths = dev_len;
+    A.codes = dev_codes;
+    A.seg_off = scratch;
+    A.n_seg = n_seg;
+    A.stream = reinterpret_cast<uint32_t *>(image + L.stream);
+    A.plane = image + L.plane;
+    A.gaps = image + L.gaps;
+    A.out_off = out_off;
+    A.chunk_bits = static_cast<uint32_t>(J.chunk_bits);
+    A.tile_bits = cbits * static_cast<uint64_t>(J.tile_threads);
+    if (J.cb->dtype == kBF16) {
+        pack_kernel<0><<<grid_for(n_seg), kEncThreads, 0, s>>>(A);
+        tail_gaps_kernel<0><<<1, 128, 0, s>>>(J.src, J.n, dev_len, A.gaps, n_chunks, total, A.chunk_bits);
+    } else {
+        pack_kernel<1><<<grid_for(n_seg), kEncThreads, 0, s>>>(A);
+        tail_gaps_kernel<1><<<1, 128, 0, s>>>(J.src, J.n, dev_len, A.gaps, n_chunks, total, A.chunk_bits);
+    }
+    // the span accumulator keeps the previous call's value: clear it
+    unsigned long long *dev_max = reinterpret_cast<unsigned long long *>(scratch + n_seg + 1);
+    if (cudaMemsetAsync(dev_max, 0, 8, s) != cudaSuccess) return "memset failed";
+    max_span_kernel<<<grid_for((meta.n_tiles + 255) / 256), 256, 0, s>>>(out_off, meta.n_tiles, dev_max);
+    uint64_t ms = 0;
+    if (cudaMemcpyAsync(&ms, dev_max, 8, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return "max span read-back failed";
+    if (cudaGetLastError() != cudaSuccess) return "kernel launch failed";
+    if (cudaMemcpyAsync(image + offsetof(ImageHeader, max_span), &ms, 8, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return "header update failed";
+    r->max_span = ms;
     return "";
 }
 

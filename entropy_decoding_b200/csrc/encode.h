@@ -34,4 +34,14 @@ std::string encode_device_bits(const EncodeJob &J, uint64_t *scratch, cudaStream
 std::string encode_device_pack(const EncodeJob &J, uint64_t *scratch, uint64_t total_bits, const ImageLayout &L,
                                uint8_t *image, cudaStream_t s, uint64_t *max_span);
 
+// Encoding without any allocation: the scratch is a static device array of
+// 512 KB per GPU, so n must not exceed noalloc_max_elems().  Calls that
+// overlap on the GPU share that array and race.
+struct NoallocResult {
+    uint64_t image_bytes, total_bits, n_tiles, max_span;
+};
+uint64_t noalloc_max_elems();
+std::string encode_device_noalloc(const EncodeJob &J, uint8_t *image, uint64_t image_cap, cudaStream_t s,
+                                  NoallocResult *r);
+
 }  // namespace df11

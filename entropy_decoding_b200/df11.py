@@ -50,6 +50,11 @@ class BlobInfo(ctypes.Structure):
         return {k: getattr(self, k) for k, _ in self._fields_}
 
 
+class EncodeResult(ctypes.Structure):
+    _fields_ = [("image_bytes", ctypes.c_uint64), ("total_bits", ctypes.c_uint64), ("n_tiles", ctypes.c_uint64),
+                ("max_span", ctypes.c_uint64)]
+
+
 class DecodeOpts(ctypes.Structure):
     _fields_ = [("chunks_per_thread", ctypes.c_int32), ("ctas_per_sm", ctypes.c_int32),
                 ("warps_per_cta", ctypes.c_int32)]
@@ -91,6 +96,7 @@ _SIGS = {
     "df11_encode_device_end": ([_P, _P, _U64, _PP], _S),
     "df11_encoding_free": ([_P], None),
     "df11_blob_fetch": ([_P, _P], _S),
+    "df11_encode_device_noalloc": ([_P, _P, _U64, _I, _I, _P, _U64, _P, ctypes.POINTER(EncodeResult)], _S),
     "df11_decode_host": ([_PP, _PP, _PP, _PP, _PP, _I, _P, _P], _S),
     "df11_decode_launch_shape": ([_PP, _I, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I)], _S),
 }
@@ -332,6 +338,26 @@ def df11_encode_device_end(enc: Encoding, image_ptr: int, image_cap: int, keep=N
 
 def df11_blob_fetch(blob: Blob, stream: int = 0):
     _check(_lib.df11_blob_fetch(blob.handle, stream or None), "df11_blob_fetch")
+
+
+NOALLOC_SCRATCH_BYTES = 65536 * 8
+NOALLOC_MAX_ELEMS = (65536 - 163) * 4096
+
+
+def df11_encode_device_noalloc(cb: Codebook, src_ptr: int, n: int, chunk_bits: int, tile_threads: int,
+                               image_ptr: int, image_cap: int, stream: int = 0) -> EncodeResult:
+    """GPU encode for callers that cannot allocate device memory: scratch is a
+    static device array of the library, so n is limited to NOALLOC_MAX_ELEMS.
+    Raises Df11Error (status DF11_ENOMEM with .result.image_bytes set when
+    the image buffer is too small)."""
+    r = EncodeResult()
+    st = _lib.df11_encode_device_noalloc(cb.handle, src_ptr or None, n, chunk_bits, tile_threads, image_ptr or None,
+                                         image_cap, stream or None, ctypes.byref(r))
+    if st != DF11_OK:
+        e = Df11Error(st, "df11_encode_device_noalloc")
+        e.result = r
+        raise e
+    return r
 
 
 # ----------------------------------------------------------------- torch-side helpers (device memory only)

@@ -309,6 +309,60 @@ void df11_encoding_free(df11_encoding *enc);
  * DF11_ECUDA. */
 df11_status df11_blob_fetch(df11_blob *blob, df11_stream stream);
 
+/* ---------------------------------------------------------------------
+ * GPU encoding that allocates nothing
+ * ------------------------------------------------------------------ */
+
+/* The paper has no counterpart to this call: it exists for programs that
+ * cannot allocate device memory at the moment they encode.  Examples are
+ * inference servers that reserve nearly all HBM for weights and KV cache at
+ * start-up (a cudaMalloc would fail or fragment that pool), and loops that
+ * must not pay cudaMalloc/cudaFree's implicit device synchronisation.
+ *
+ * df11_encode_device_noalloc does what df11_encode_device_begin + _end do and
+ * writes the same device image, byte for byte, into the caller's image_dev.
+ * It calls no cudaMalloc, cudaFree or other allocating routine, on the device
+ * or the host.  The caller passes the raw weights (src_dev, 16-byte aligned)
+ * and the image buffer (image_dev, 256-byte aligned, image_cap bytes).
+ *
+ * Scratch.  Its scratch is one static device array of
+ * DF11_NOALLOC_SCRATCH_BYTES, which every GPU that loads the library holds
+ * until the process exits.  That bounds n_elems at DF11_NOALLOC_MAX_ELEMS;
+ * larger tensors are rejected with DF11_EINVAL before any GPU work.
+ *
+ * First call per device.  It looks up the array's device address with
+ * cudaGetSymbolAddress, with that device current.  Make this first call
+ * before any stream capture.
+ *
+ * Overlapping calls.  Every call shares the array, and the array keeps the
+ * last call's contents (each call clears what must start at zero). Calls
+ * that overlap on the GPU, from other threads or on other streams of the
+ * same device, race and must be serialised by the caller.
+ *
+ * Synchronisation.  The call synchronises `stream` (it reads the stream
+ * length and the largest tile span back).
+ *
+ * Result.  *result receives image_bytes, total_bits, n_tiles and max_span.
+ * When image_cap < image_bytes the call returns DF11_ENOMEM with
+ * result->image_bytes set and the image untouched.
+ *
+ * Errors: DF11_EINVAL (arguments, size limit, or an exponent the code does
+ * not cover), DF11_ENOMEM, DF11_ECUDA. */
+#define DF11_NOALLOC_SCRATCH_BYTES (65536ull * 8ull)
+#define DF11_NOALLOC_MAX_ELEMS ((65536ull - 163ull) * 4096ull)
+
+typedef struct {
+    uint64_t image_bytes; /* device image size this tensor needs */
+    uint64_t total_bits;  /* stream length in bits */
+    uint64_t n_tiles;
+    uint64_t max_span;    /* most codes that start in one tile */
+} df11_encode_result;
+
+df11_status df11_encode_device_noalloc(const df11_codebook *cb, const void *src_dev, uint64_t n_elems,
+                                       int chunk_bits, int tile_threads, void *image_dev,
+                                       uint64_t image_cap, df11_stream stream,
+                                       df11_encode_result *result);
+
 #ifdef __cplusplus
 }
 #endif
