@@ -58,7 +58,10 @@ def parse_args():
     p.add_argument("--tile-threads", type=int, default=32)
     p.add_argument("--chunks-per-thread", type=int, default=0, help="decode launch option (0 = library default)")
     p.add_argument("--ctas-per-sm", type=int, default=0, help="decode launch option (0 = as many as fit)")
-    p.add_argument("--warps-per-cta", type=int, default=0, help="decode launch option, warp tiles (0 = 8)")
+    p.add_argument("--warps-per-cta", type=int, default=0,
+                   help="decode launch option, warp tiles (0 = library default for the walker)")
+    p.add_argument("--walker", choices=["auto", "window", "byte_step"], default="auto",
+                   help="decode launch option, warp tiles: how a thread walks its chunk")
     return p.parse_args()
 
 
@@ -84,7 +87,8 @@ def full_config(args, world: int) -> dict:
     out_gb = cfg["n_weights"] * (2 if cfg["dtype_in"] == "bf16" else 1) / 1e9
     return {**cfg, "seed": args.seed, "chunk_bits": args.chunk_bits, "tile_threads": args.tile_threads,
             "chunks_per_thread": args.chunks_per_thread or 1, "ctas_per_sm": args.ctas_per_sm or "max",
-            "warps_per_cta": (args.warps_per_cta or 16) if args.tile_threads == 32 else None,
+            "warps_per_cta": (args.warps_per_cta or "library default") if args.tile_threads == 32 else None,
+            "walker": args.walker if args.tile_threads == 32 else "window",
             "l2": f"no flush: inputs larger than L2 (decoded output {out_gb:.1f} GB, compressed images "
                   f"about 0.68x that, vs 126 MB L2)",
             "parallelism": f"replicas x{world} (each GPU decodes its own copy)"}
@@ -278,6 +282,18 @@ def run_reference(args, rank: int, world: int):
 
 # ------------------------------------------------------------------ our arm
 
+def kernel_name(args, cfg: dict, shape) -> str:
+    """Name of the decode kernel the library launched for these options."""
+    dt = cfg["dtype_in"]
+    if args.tile_threads != 32:
+        cpt = args.chunks_per_thread or 1
+        return f"decode_kernel<{dt},{args.chunk_bits},{cpt},{args.tile_threads // cpt}>"
+    nw = shape[1] // 32
+    if shape[3] == 2:  # DF11_WALKER_BYTE_STEP
+        return f"decode_fsm_kernel<{dt},{args.chunk_bits},{nw}>"
+    return f"decode_warp_kernel<{dt},{args.chunk_bits},{nw}>"
+
+
 def run_ours(args, rank: int, world: int, local_rank: int):
     import torch
     import torch.distributed as dist
@@ -358,12 +374,18 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             a += i.stream_bytes + i.plane_bytes + i.gaps_bytes + i.out_off_bytes + i.uncompressed_bytes
         algo.append(a)
 
+    walker = {"auto": 0, "window": 1, "byte_step": 2}[args.walker]
+    # the launch shape of the largest group (what the library picked for these options)
+    big = max(range(len(groups)), key=lambda gi: sum(b.info().n_elems for b in groups[gi][1]))
+    shape = df11.df11_decode_launch_shape(groups[big][1], args.chunks_per_thread, args.ctas_per_sm,
+                                          args.warps_per_cta, walker, with_walker=True)
+
     def one_step(events=None):
         for gi, (name, blobs, dt, dsts) in enumerate(groups):
             if events is not None:
                 events[gi][0].record(stream)
             df11.df11_decode_ex(blobs, [d[0] for d in dsts], err.data_ptr(), stream.cuda_stream,
-                                args.chunks_per_thread, args.ctas_per_sm, args.warps_per_cta)
+                                args.chunks_per_thread, args.ctas_per_sm, args.warps_per_cta, walker)
             if events is not None:
                 events[gi][1].record(stream)
 
@@ -490,10 +512,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": peak_src,
-                     "kernel": (f"decode_warp_kernel<{cfg["dtype_in"]},{args.chunk_bits},{args.warps_per_cta or 16}>"
-                                if args.tile_threads == 32 else
-                                f"decode_kernel<{cfg['dtype_in']},{args.chunk_bits},{args.chunks_per_thread or 1},"
-                                f"{args.tile_threads // (args.chunks_per_thread or 1)}>"),
+                     "kernel": kernel_name(args, cfg, shape),
+                     "launch": {"grid": shape[0], "block": shape[1], "smem_bytes": shape[2],
+                                "walker": {1: "window", 2: "byte_step"}.get(shape[3], shape[3])},
                      "algorithmic_bytes_per_launch": algo_step / len(groups),
                      "launch_ms_mean": float(per_launch.mean()),
                      "launch_ms_by_group": {"first": float(per_launch[:, 0].mean()),

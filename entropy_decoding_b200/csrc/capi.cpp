@@ -249,7 +249,10 @@ df11_status df11_decode_ex(const df11_blob *const *blobs, void *const *dst_dev, 
         o.chunks_per_thread = opts->chunks_per_thread;
         o.ctas_per_sm = opts->ctas_per_sm;
         o.warps_per_cta = opts->warps_per_cta;
-        if (o.chunks_per_thread < 0 || o.ctas_per_sm < 0 || o.warps_per_cta < 0) return DF11_EINVAL;
+        o.walker = opts->walker;
+        if (o.chunks_per_thread < 0 || o.ctas_per_sm < 0 || o.warps_per_cta < 0 || o.walker < 0 ||
+            o.walker > DF11_WALKER_BYTE_STEP)
+            return DF11_EINVAL;
     }
     return from_launch(df11::launch_decode(bs, dst_dev, n_blobs, dev_err_flag, o,
                                            reinterpret_cast<cudaStream_t>(stream)));
@@ -290,11 +293,11 @@ df11_status df11_decode_host(df11_blob *const *blobs, const void *const *host_im
 
 df11_status df11_decode_launch_shape(const df11_blob *const *blobs, int n_blobs, int *grid, int *block,
                                      int *smem_bytes) {
-    return df11_decode_launch_shape_ex(blobs, n_blobs, nullptr, grid, block, smem_bytes);
+    return df11_decode_launch_shape_ex(blobs, n_blobs, nullptr, grid, block, smem_bytes, nullptr);
 }
 
 df11_status df11_decode_launch_shape_ex(const df11_blob *const *blobs, int n_blobs, const df11_decode_opts *opts,
-                                        int *grid, int *block, int *smem_bytes) {
+                                        int *grid, int *block, int *smem_bytes, int *walker) {
     if (!blobs || n_blobs < 1 || n_blobs > df11::kMaxTensorsPerLaunch) return DF11_EINVAL;
     const df11::Blob *bs[df11::kMaxTensorsPerLaunch];
     for (int i = 0; i < n_blobs; ++i) {
@@ -307,12 +310,17 @@ df11_status df11_decode_launch_shape_ex(const df11_blob *const *blobs, int n_blo
         o.chunks_per_thread = opts->chunks_per_thread;
         o.ctas_per_sm = opts->ctas_per_sm;
         o.warps_per_cta = opts->warps_per_cta;
+        o.walker = opts->walker;
+        if (o.chunks_per_thread < 0 || o.ctas_per_sm < 0 || o.warps_per_cta < 0 || o.walker < 0 ||
+            o.walker > DF11_WALKER_BYTE_STEP)
+            return DF11_EINVAL;
     }
     df11::LaunchStatus st = df11::decode_launch_shape(bs, n_blobs, o, &sh);
     if (st != df11::LaunchStatus::kOk) return from_launch(st);
     if (grid) *grid = sh.grid;
     if (block) *block = sh.block;
     if (smem_bytes) *smem_bytes = sh.smem;
+    if (walker) *walker = sh.walker;
     return DF11_OK;
 }
 

@@ -10,6 +10,7 @@
 #include "codec.h"
 
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <cstring>
 #include <thread>
@@ -271,6 +272,92 @@ void build_multi(const uint8_t *lengths, const uint32_t *codes, int nsym, std::v
     }
 }
 
+// Byte-step transition tables over the code tree (layout in df11_internal.h).
+// The tree is built from the canonical codes; the rows go to the internal
+// nodes with the most probability mass below them, taking 2^-length as a
+// code's probability (a byte boundary falls on node v with a probability
+// proportional to that mass), so the dead row is rarely reached.
+void build_fsm(const uint8_t *lengths, const uint32_t *codes, int nsym, std::vector<uint32_t> &fsm,
+               int &rows) {
+    struct Node {
+        int child[2] = {-1, -1};
+        int sym = -1;
+        int depth = 0;
+        uint64_t prefix = 0;
+        double mass = 0.0;
+    };
+    std::vector<Node> nodes(1);
+    for (int s = 0; s < nsym; ++s) {
+        const int L = lengths[s];
+        if (!L) continue;
+        int v = 0;
+        for (int i = L - 1; i >= 0; --i) {
+            const int bit = static_cast<int>((codes[s] >> i) & 1u);
+            if (nodes[v].child[bit] < 0) {
+                Node n;
+                n.depth = nodes[v].depth + 1;
+                n.prefix = (nodes[v].prefix << 1) | static_cast<uint64_t>(bit);
+                nodes.push_back(n);
+                nodes[v].child[bit] = static_cast<int>(nodes.size()) - 1;
+            }
+            v = nodes[v].child[bit];
+        }
+        nodes[v].sym = s;
+        nodes[v].mass = std::ldexp(1.0, -L);
+    }
+    // children are created after their parent: one backward pass sums the masses
+    for (int v = static_cast<int>(nodes.size()) - 1; v > 0; --v) {
+        for (int c : nodes[v].child)
+            if (c >= 0) nodes[v].mass += nodes[c].mass;
+    }
+    for (int c : nodes[0].child)
+        if (c >= 0) nodes[0].mass += nodes[c].mass;
+    std::vector<int> internal;
+    for (int v = 0; v < static_cast<int>(nodes.size()); ++v)
+        if (nodes[v].sym < 0) internal.push_back(v);
+    std::stable_sort(internal.begin() + 1, internal.end(), [&](int a, int b) {
+        if (nodes[a].mass != nodes[b].mass) return nodes[a].mass > nodes[b].mass;
+        if (nodes[a].depth != nodes[b].depth) return nodes[a].depth < nodes[b].depth;
+        return nodes[a].prefix < nodes[b].prefix;
+    });
+    const int live = std::min<int>(static_cast<int>(internal.size()), kFsmMaxRows - 1);
+    rows = live + 1;
+    const uint32_t dead = static_cast<uint32_t>(live);
+    std::vector<int> row_of(nodes.size(), -1);
+    for (int r = 0; r < live; ++r) row_of[internal[r]] = r;
+    fsm.assign(static_cast<size_t>(rows) * kLutEntries * 2, 0);
+    for (int r = 0; r < rows; ++r) {
+        for (uint32_t b = 0; b < static_cast<uint32_t>(kLutEntries); ++b) {
+            uint32_t ctl = dead << kFsmRowShift, packed = 0;
+            if (r < live) {
+                int v = internal[r], k = 0;
+                uint32_t ends = 0;
+                bool bad = false;
+                for (int i = 0; i < 8; ++i) {
+                    const int c = nodes[v].child[(b >> (7 - i)) & 1u];
+                    if (c < 0) {
+                        bad = true;
+                        break;
+                    }
+                    if (nodes[c].sym >= 0) {
+                        if (k < 4) packed |= static_cast<uint32_t>(nodes[c].sym) << (8 * k);
+                        ++k;
+                        ends |= 1u << i;
+                        v = 0;
+                    } else {
+                        v = c;
+                    }
+                }
+                const uint32_t next = (bad || k > 4 || row_of[v] < 0) ? dead : static_cast<uint32_t>(row_of[v]);
+                ctl = ends | (next << kFsmRowShift) | (static_cast<uint32_t>(std::min(k, 7)) << kFsmCountShift);
+            }
+            const size_t e = (static_cast<size_t>(r) * kLutEntries + b) * 2;
+            fsm[e] = ctl;
+            fsm[e + 1] = packed;
+        }
+    }
+}
+
 }  // namespace
 
 std::shared_ptr<Codebook> make_codebook(int dtype, const uint8_t *lengths) {
@@ -290,6 +377,7 @@ std::shared_ptr<Codebook> make_codebook(int dtype, const uint8_t *lengths) {
     if (!canonical_codes(cb->lengths, cb->nsym, cb->codes)) return nullptr;
     if (!build_lut(cb->lengths, cb->codes, cb->nsym, cb->lut)) return nullptr;
     build_multi(cb->lengths, cb->codes, cb->nsym, cb->meta, cb->syms);
+    build_fsm(cb->lengths, cb->codes, cb->nsym, cb->fsm, cb->fsm_rows);
     return cb;
 }
 
@@ -598,8 +686,10 @@ ImageLayout image_layout(const Blob &b) {
     o = align_up(o + kMultiEntries * 4, kImageAlign);
     L.lut = o;
     o = align_up(o + b.cb->lut.size() * 2, kImageAlign);
+    L.fsm = o;
+    o = align_up(o + b.cb->fsm.size() * 4, kImageAlign);
     L.gaps = o;
-    o = align_up(o + b.n_tiles * static_cast<uint64_t>(b.tile_threads), kImageAlign);
+    o = align_up(o + b.n_tiles * static_cast<uint64_t>(b.tile_threads) + kGapsTail, kImageAlign);
     L.out_off = o;
     o = align_up(o + (b.n_tiles + 1) * 8, kImageAlign);
     L.stream = o;
@@ -618,6 +708,7 @@ void write_image_head(const Blob &b, const ImageLayout &L, uint8_t *dst) {
     h.chunk_bits = static_cast<uint32_t>(b.chunk_bits);
     h.tile_threads = static_cast<uint32_t>(b.tile_threads);
     h.n_luts = static_cast<uint32_t>(b.cb->n_luts());
+    h.fsm_rows = static_cast<uint32_t>(b.cb->fsm_rows);
     h.n_elems = b.n;
     h.total_bits = b.total_bits;
     h.n_tiles = b.n_tiles;
@@ -627,6 +718,7 @@ void write_image_head(const Blob &b, const ImageLayout &L, uint8_t *dst) {
     std::memcpy(dst + L.meta, b.cb->meta.data(), kMultiEntries * 4);
     std::memcpy(dst + L.syms, b.cb->syms.data(), kMultiEntries * 4);
     std::memcpy(dst + L.lut, b.cb->lut.data(), b.cb->lut.size() * 2);
+    std::memcpy(dst + L.fsm, b.cb->fsm.data(), b.cb->fsm.size() * 4);
 }
 
 void write_image(const Blob &b, uint8_t *dst) {

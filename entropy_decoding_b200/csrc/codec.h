@@ -25,6 +25,8 @@ struct Codebook {
     std::vector<uint32_t> meta;  // kMultiEntries
     std::vector<uint32_t> syms;  // kMultiEntries
     std::vector<uint16_t> lut;   // n_luts * kLutEntries
+    std::vector<uint32_t> fsm;   // fsm_rows * kLutEntries * 2: {ctl, syms} per entry
+    int fsm_rows = 0;            // including the dead row (the last one)
     int n_luts() const { return static_cast<int>(lut.size() / kLutEntries); }
 };
 

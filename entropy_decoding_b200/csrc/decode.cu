@@ -199,6 +199,20 @@ __device__ __forceinline__ uint32_t sane_meta(uint32_t e) {
     return ok ? e : kMetaLong;
 }
 
+// Multi-symbol table reads: shared-memory copies were checked when staged;
+// GM = true reads the image in global memory and checks each entry.
+template <bool GM>
+__device__ __forceinline__ uint32_t meta_at(const Tables &T, uint32_t idx) {
+    if constexpr (GM) return sane_meta(__ldg(T.meta + idx));
+    else return T.meta[idx];
+}
+
+template <bool GM>
+__device__ __forceinline__ uint32_t syms_at(const Tables &T, uint32_t idx) {
+    if constexpr (GM) return __ldg(T.syms + idx);
+    else return T.syms[idx];
+}
+
 // Number of an entry's codes that start before bit `room` of its window.
 __device__ __forceinline__ uint32_t starts_before(uint32_t mm, int room) {
     return static_cast<uint32_t>(__popc((mm >> kMetaMaskShift) & ((1u << room) - 1u)));
@@ -221,7 +235,7 @@ constexpr uint32_t kCountOne = 1u << kMetaCountShift;
 // and an entry is consumed | count << 11 | mask << 20, so one add advances
 // both (the mask lands above the count field); the sentinel adds 1024 to p,
 // which ends the loop.  The CPT chunks advance in lockstep.
-template <int CW, int CPT>
+template <int CW, int CPT, bool GM = false>
 __device__ __forceinline__ void count_codes(const uint32_t (&w)[CPT * CW + 1], const int (&gap)[CPT],
                                             const int (&E)[CPT], const Tables &T, uint32_t (&cnt)[CPT],
                                             uint32_t &err) {
@@ -250,7 +264,7 @@ __device__ __forceinline__ void count_codes(const uint32_t (&w)[CPT * CW + 1], c
                 for (int c = 0; c < CPT; ++c) {
                     if (act[c]) {
                         const uint32_t win = __funnelshift_l(w[c * CW + k + 1], w[c * CW + k], acc[c]);
-                        acc[c] += T.meta[win >> (32 - kMultiBits)];
+                        acc[c] += meta_at<GM>(T, win >> (32 - kMultiBits));
                     }
                 }
             }
@@ -267,7 +281,7 @@ __device__ __forceinline__ void count_codes(const uint32_t (&w)[CPT * CW + 1], c
                     continue;
                 }
                 const uint32_t win = __funnelshift_l(w[c * CW + k + 1], w[c * CW + k], p);
-                const uint32_t mm = single ? kMetaLong : T.meta[win >> (32 - kMultiBits)];
+                const uint32_t mm = single ? kMetaLong : meta_at<GM>(T, win >> (32 - kMultiBits));
                 if (mm & kMetaLong) {
                     const uint32_t e = lut_decode(win, T, err);
                     acc[c] += ((e >> 8) & 0x3Fu) + kCountOne;
@@ -297,7 +311,7 @@ __device__ __forceinline__ void put_symbols(uint32_t sy, uint32_t out) {
 
 // Phase 2 (CTA-tile kernel): decode chunk C again along the same path as
 // phase 1 and write its symbols from shared-memory byte address q on.
-template <int CW, int CPT, int C>
+template <int CW, int CPT, int C, bool GM = false>
 __device__ __forceinline__ void emit_codes(const uint32_t (&w)[CPT * CW + 1], int p, const int E, const Tables &T,
                                            uint32_t q, uint32_t &err) {
     uint32_t out = q;
@@ -311,9 +325,9 @@ __device__ __forceinline__ void emit_codes(const uint32_t (&w)[CPT * CW + 1], in
             while (p < lm) {
                 const uint32_t win = __funnelshift_l(lw, hi, p);
                 const uint32_t idx = win >> (32 - kMultiBits);
-                const uint32_t mm = T.meta[idx];
+                const uint32_t mm = meta_at<GM>(T, idx);
                 p += static_cast<int>(mm & kPosMask);
-                put_symbols(T.syms[idx], out);
+                put_symbols(syms_at<GM>(T, idx), out);
                 out += (mm >> kMetaCountShift) & 7u;
             }
             bool single = false;
@@ -325,7 +339,7 @@ __device__ __forceinline__ void emit_codes(const uint32_t (&w)[CPT * CW + 1], in
             }
             const uint32_t win = __funnelshift_l(lw, hi, p);
             const uint32_t idx = win >> (32 - kMultiBits);
-            const uint32_t mm = single ? kMetaLong : T.meta[idx];
+            const uint32_t mm = single ? kMetaLong : meta_at<GM>(T, idx);
             if (mm & kMetaLong) {
                 const uint32_t e = lut_decode(win, T, err);
                 p += static_cast<int>((e >> 8) & 0x3Fu);
@@ -334,7 +348,7 @@ __device__ __forceinline__ void emit_codes(const uint32_t (&w)[CPT * CW + 1], in
             } else {
                 const uint32_t nv = starts_before(mm, er - p);
                 const uint32_t nb = 8u * nv;
-                const uint32_t sy = nb >= 32 ? T.syms[idx] : (T.syms[idx] & ((1u << nb) - 1u));
+                const uint32_t sy = nb >= 32 ? syms_at<GM>(T, idx) : (syms_at<GM>(T, idx) & ((1u << nb) - 1u));
                 p += static_cast<int>(mm & 0xFu);
                 if (nv) put_symbols(sy, out);
                 out += nv;
@@ -955,22 +969,313 @@ __global__ void __launch_bounds__(NWARP * 32, NWARP <= 8 ? 4 : 2)
     if (lane == 0) report(P.err, err);
 }
 
+// ------------------------------------------------------------------ byte-step kernel
+
+// Entry offset within a transition-table row of byte k (0 = earliest) of the
+// 32 stream bits x (earliest bit in bit 31): byte * 8.
+__device__ __forceinline__ uint32_t step_off(uint32_t x, int k) {
+    return k == 3 ? (x << 3) & 0x7F8u : (x >> (21 - 8 * k)) & 0x7F8u;
+}
+
+// The byte-step walk of one chunk.  The thread's codes occupy bits [g, g +
+// 8 * nfull + r) of the words w[0..CW] followed by w2 (earliest bit first):
+// from the first code start in the chunk to the first code start in the next
+// chunk (or the end of the stream).  Step j looks up byte j of that range in
+// the row of the tree node the previous step stopped on (the root first): the
+// entry lists the codes that end in the byte and the next row.  Steps below
+// NFIX are taken by every thread with a whole chunk (its range is at least
+// CB - 31 bits); the others are predicated on nfull, and the warp stops after
+// its longest range (jmax steps).  A last partial byte (r bits) counts only
+// the codes whose end mask bit falls in its first r bits; those end exactly
+// at the range's end, so the codes of the next chunk are never counted.
+// Phase 1 (EMIT = false) returns the number of codes and, in ctl_out, the
+// last entry, whose row is the dead row (`dead`) when the walk left the
+// tables or the partial byte ends more than the 4 codes an entry holds
+// (possible only with a 1-bit codeword).  Phase 2 (EMIT = true) writes the
+// symbols from shared-memory address out on.
+template <int CB, bool EMIT>
+__device__ __forceinline__ uint32_t byte_step_walk(const uint32_t (&w)[CB / 32 + 1], uint32_t w2, int g, int nfull,
+                                                   int r, int jmax, const uint8_t *tab, uint32_t out, uint32_t dead,
+                                                   uint32_t &ctl_out) {
+    constexpr int CW = CB / 32, NFIX = (CB - 32) / 8;
+    uint32_t ctl = 0, cnt = 0;
+#pragma unroll
+    for (int m = 0; m <= CW; ++m) {
+        if (4 * m >= NFIX && 4 * m >= jmax) break;  // warp-uniform
+        const uint32_t x = __funnelshift_l(m < CW ? w[m + 1] : w2, w[m], static_cast<uint32_t>(g));
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int j = 4 * m + k;
+            if (j >= NFIX && j >= jmax) break;
+            const uint32_t a = (ctl & kFsmRowMask) | step_off(x, k);
+            if constexpr (!EMIT) {
+                const uint32_t e = *reinterpret_cast<const uint32_t *>(tab + a);
+                if (j < NFIX || j < nfull) {
+                    ctl = e;
+                    cnt += e >> kFsmCountShift;
+                } else if (j == nfull) {
+                    const uint32_t c = static_cast<uint32_t>(__popc(e & ((1u << r) - 1u)));
+                    cnt += c;
+                    if (c > 4) ctl = dead;
+                }
+            } else {
+                const uint2 e = *reinterpret_cast<const uint2 *>(tab + a);
+                if (j < NFIX || j < nfull) {
+                    ctl = e.x;
+                    put_symbols(e.y, out);
+                    out += e.x >> kFsmCountShift;
+                } else if (j == nfull) {
+                    const uint32_t c = min(static_cast<uint32_t>(__popc(e.x & ((1u << r) - 1u))), 4u);
+                    if (c) put_symbols(e.y & (0xFFFFFFFFu >> (32u - 8u * c)), out);
+                }
+            }
+        }
+    }
+    ctl_out = ctl;
+    return cnt;
+}
+
+// Shared memory of the byte-step kernel: the transition table (fsm_rows rows
+// of kFsmRowBytes) at offset 0, the root hierarchical table, then per warp
+// its mbarrier, one stage (the tile's 32 chunks + 16 look-ahead bytes, then
+// 48 gap bytes: its own 32 and the next tile's first 16) and its exponent
+// buffer.
+struct FsmPlan {
+    uint32_t stage_bytes, exps_bytes, warp_bytes, off_lut, off_warps, total;
+};
+
+__host__ __device__ inline FsmPlan make_fsm_plan(int chunk_bits, int nwarp, uint32_t max_span, int fsm_rows) {
+    FsmPlan p;
+    p.stage_bytes = static_cast<uint32_t>(32 * chunk_bits / 8) + 16u + 48u;
+    p.exps_bytes = (max_span + 2u * 32u + 16u + 15u) & ~15u;
+    p.warp_bytes = (16u + p.stage_bytes + p.exps_bytes + 127u) & ~127u;
+    p.off_lut = static_cast<uint32_t>(fsm_rows) * kFsmRowBytes;
+    p.off_warps = up128(p.off_lut + kLutEntries * 2);
+    p.total = p.off_warps + static_cast<uint32_t>(nwarp) * p.warp_bytes;
+    return p;
+}
+
+// Warp tiles (32 chunks) decoded with the byte-step walk, one CTA of NWARP
+// warps per SM sharing the transition table.  Each warp streams its tiles
+// through one shared-memory stage (lane 0 refills it with the warp's next
+// tile as soon as the current one is in registers, so the copy has a whole
+// tile's decode to land), then runs phase 1, the warp scan, phase 2 and the
+// merge as the window kernel does.  Threads whose walk reaches the dead row,
+// or whose range is cut short by the end of the stream, take the window walk
+// instead (12-bit table read from global memory through L1).
+template <int DT, int CB, int NWARP>
+__global__ void __launch_bounds__(NWARP * 32, 1)
+    decode_fsm_kernel(const __grid_constant__ DecodeParams P, const uint32_t max_span, const int) {
+    constexpr int CW = CB / 32;
+    constexpr int NFIX = (CB - 32) / 8;
+    constexpr uint32_t TILE_BYTES = 32 * CB / 8;
+    constexpr uint32_t GROUP = DT == 0 ? 16u : 32u;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int rows = P.fsm_rows;
+    const FsmPlan plan = make_fsm_plan(CB, NWARP, max_span, rows);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint16_t *s_lut = reinterpret_cast<uint16_t *>(smem + plan.off_lut);
+    uint8_t *wbase = smem + plan.off_warps + warp * plan.warp_bytes;
+    uint64_t *full = reinterpret_cast<uint64_t *>(wbase);
+    uint8_t *stage = wbase + 16;
+    uint8_t *s_exps = wbase + 16 + plan.stage_bytes;
+    const uint32_t dead = static_cast<uint32_t>(rows - 1) << kFsmRowShift;
+
+    {
+        // the transition table; a row index past the last row (damaged
+        // tables) is redirected to the dead row so every lookup stays inside
+        const uint4 *g = reinterpret_cast<const uint4 *>(P.fsm);
+        uint4 *s = reinterpret_cast<uint4 *>(smem);
+        const uint32_t lim = static_cast<uint32_t>(rows) << kFsmRowShift;
+        for (int i = tid; i < rows * kFsmRowBytes / 16; i += NWARP * 32) {
+            uint4 v = __ldg(g + i);
+            if ((v.x & kFsmRowMask) >= lim) v.x = (v.x & ~kFsmRowMask) | dead;
+            if ((v.z & kFsmRowMask) >= lim) v.z = (v.z & ~kFsmRowMask) | dead;
+            s[i] = v;
+        }
+        const uint4 *gl = reinterpret_cast<const uint4 *>(P.lut);
+        uint4 *sl = reinterpret_cast<uint4 *>(s_lut);
+        for (int i = tid; i < kLutEntries * 2 / 16; i += NWARP * 32) sl[i] = __ldg(gl + i);
+        uint4 *se = reinterpret_cast<uint4 *>(s_exps);
+        for (uint32_t i = lane; i < plan.exps_bytes / 16; i += 32) se[i] = make_uint4(0, 0, 0, 0);
+    }
+    if (lane == 0) {
+        mbar_init(&full[0], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    const uint32_t stride = gridDim.x * NWARP;
+    const uint32_t first = blockIdx.x * NWARP + warp;
+    int ti_issue = 0, ti_cur = 0;
+    // lane 0: copy tile t's stream slice and gaps into the stage
+    auto issue = [&](uint32_t t) {
+        ti_issue = tensor_of(P, t, ti_issue);
+        const TensorDesc &d = P.t[ti_issue];
+        const uint32_t lt = t - d.tile_begin;
+        mbar_arrive_expect_tx(&full[0], TILE_BYTES + 16u + 48u);
+        bulk_load(stage, d.stream + static_cast<uint64_t>(lt) * TILE_BYTES, TILE_BYTES + 16u, &full[0]);
+        bulk_load(stage + TILE_BYTES + 16u, d.gaps + static_cast<uint64_t>(lt) * 32u, 48u, &full[0]);
+    };
+    if (lane == 0 && first < P.total_tiles) issue(first);
+    bool pending = first < P.total_tiles;
+
+    // the window walk of the fallback: 12-bit table in global memory, root
+    // hierarchical table in shared memory
+    const Tables T{P.meta, P.syms, s_lut, P.lut, 1, P.n_luts};
+    uint32_t err = 0;
+    uint32_t k = 0;
+    for (uint32_t t = first; t < P.total_tiles; t += stride, ++k) {
+        ti_cur = tensor_of(P, t, ti_cur);
+        const TensorDesc &d = P.t[ti_cur];
+        const uint32_t lt = t - d.tile_begin;
+        uint64_t S = __ldg(d.out_off + lt);
+        const uint64_t Eo = __ldg(d.out_off + lt + 1);
+        const bool bad = Eo < S || Eo > d.n || Eo - S > max_span;
+        if (bad) S = 0;
+        const uint32_t span = bad ? 0u : static_cast<uint32_t>(Eo - S);
+
+        // the tile's plane span: the first kPrefetchGroups groups of each lane now
+        const uint64_t g0 = S / GROUP;
+        const uint32_t ng = span ? static_cast<uint32_t>((S + span + GROUP - 1) / GROUP - g0) : 0u;
+        const uint8_t *plane = d.plane + g0 * 16u;
+        uint4 pre[kPrefetchGroups];
+#pragma unroll
+        for (int u = 0; u < kPrefetchGroups; ++u) {
+            const uint32_t i = lane + 32u * u;
+            if (i < ng) pre[u] = ld_global_stream_v4(plane + 16u * i);
+        }
+
+        const bool landed = __all_sync(0xFFFFFFFFu, mbar_wait(&full[0], k & 1u));
+        if (!landed) {
+            err |= DF11_DEV_ERR_TIMEOUT;
+            break;
+        }
+        pending = false;
+        uint32_t w[CW + 1], w2;
+        if constexpr (CW % 4 == 0) {
+#pragma unroll
+            for (int j = 0; j < CW / 4; ++j) {
+                const uint4 v = *reinterpret_cast<const uint4 *>(stage + lane * (CB / 8) + 16 * j);
+                w[4 * j + 0] = v.x;
+                w[4 * j + 1] = v.y;
+                w[4 * j + 2] = v.z;
+                w[4 * j + 3] = v.w;
+            }
+        } else {
+            const uint2 v = *reinterpret_cast<const uint2 *>(stage + lane * (CB / 8));
+            w[0] = v.x;
+            w[1] = v.y;
+        }
+        {
+            const uint32_t n0 = __shfl_down_sync(0xFFFFFFFFu, w[0], 1);
+            const uint32_t n1 = __shfl_down_sync(0xFFFFFFFFu, w[1], 1);
+            const uint32_t *la = reinterpret_cast<const uint32_t *>(stage + TILE_BYTES);
+            w[CW] = lane == 31 ? la[0] : n0;
+            w2 = lane == 31 ? la[1] : n1;
+        }
+        const int graw = stage[TILE_BYTES + 16u + lane];
+        const int gnext = stage[TILE_BYTES + 16u + lane + 1];
+        // the stage is in registers: refill it with the warp's next tile
+        __syncwarp();
+        if (t + stride < P.total_tiles) {
+            if (lane == 0) {
+                fence_proxy_async_smem();
+                issue(t + stride);
+            }
+            pending = true;
+        }
+
+        // ---- this thread's range of codes
+        const int64_t rem64 = static_cast<int64_t>(d.total_bits) - static_cast<int64_t>(lt) * (32 * CB) -
+                              static_cast<int64_t>(lane * CB);
+        const int E = rem64 >= CB ? CB : (rem64 <= 0 ? 0 : static_cast<int>(rem64));
+        if (graw >= 32) err |= DF11_DEV_ERR_AUX;
+        const int g = min(graw, 63);
+        const int64_t end64 = rem64 < CB + gnext ? rem64 : static_cast<int64_t>(CB + gnext);
+        const int nbits = static_cast<int>(max(end64 - g, static_cast<int64_t>(-1)));
+        const bool whole = graw < 32 && gnext < 32 && nbits >= 8 * NFIX;
+        const int nfull = nbits >> 3, r = nbits & 7;
+        const int jmax = static_cast<int>(__reduce_max_sync(0xFFFFFFFFu, whole ? nfull + (r != 0) : 0));
+
+        // ---- phase 1: count
+        uint32_t ctl;
+        uint32_t cnt = byte_step_walk<CB, false>(w, w2, g & 31, nfull, r, jmax, smem, 0u, dead, ctl);
+        const bool slow = !whole || (ctl & kFsmRowMask) == dead;
+        if (__any_sync(0xFFFFFFFFu, slow)) {
+            if (slow) {
+                const int gg[1] = {g}, ee[1] = {E};
+                uint32_t c1[1];
+                count_codes<CW, 1, true>(w, gg, ee, T, c1, err);
+                cnt = c1[0];
+            }
+        }
+        uint32_t incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const uint32_t total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+        const bool good = !bad && total == span;
+        if (bad) err |= DF11_DEV_ERR_AUX;
+        else if (!good) err |= DF11_DEV_ERR_SPAN;
+
+        // ---- phase 2, then the merge
+        if (good && span) {
+            const uint32_t q = smem_addr(s_exps) + static_cast<uint32_t>(S % GROUP) + incl - cnt;
+            if (!slow) byte_step_walk<CB, true>(w, w2, g, nfull, r, jmax, smem, q, dead, ctl);
+            if (__any_sync(0xFFFFFFFFu, slow)) {
+                if (slow) emit_codes<CW, 1, 0, true>(w, g, E, T, q, err);
+            }
+            __syncwarp();
+            uint8_t *dst_tile = static_cast<uint8_t *>(d.dst) + g0 * 32u;
+            const uint32_t lo = static_cast<uint32_t>(S % GROUP), hi = lo + span;
+#pragma unroll
+            for (int u = 0; u < kPrefetchGroups; ++u) {
+                const uint32_t i = lane + 32u * u;
+                if (i < ng) merge_group<DT, false>(pre[u], i, s_exps, dst_tile, lo, hi);
+            }
+            for (uint32_t i = lane + 32u * kPrefetchGroups; i < ng; i += 32)
+                merge_group<DT, false>(ld_global_stream_v4(plane + 16u * i), i, s_exps, dst_tile, lo, hi);
+            edge_groups<DT>(pre, plane, ng, s_exps, dst_tile, lo, hi, lane);
+            __syncwarp();
+        }
+    }
+    // after an abort: wait (bounded) for a copy that was issued but never consumed
+    if (pending)
+        if (!mbar_wait(&full[0], k & 1u)) err |= DF11_DEV_ERR_TIMEOUT;
+    err = __reduce_or_sync(0xFFFFFFFFu, err);
+    if (lane == 0) report(P.err, err);
+}
+
 // ------------------------------------------------------------------ host side
 
 using KernelFn = void (*)(DecodeParams, uint32_t, int);
 
-// chunks = chunks per tile (the container's tile_threads).  chunks == 32: the
-// warp-tile kernel with nwarp warps per CTA; otherwise the CTA-tile kernel
-// with chunks / cpt decoding threads and a producer warp.
+// chunks = chunks per tile (the container's tile_threads).  chunks == 32: a
+// warp-tile kernel with nwarp warps per CTA, walking with the 12-bit window
+// (walker DF11_WALKER_WINDOW) or the byte-step tables (DF11_WALKER_BYTE_STEP);
+// otherwise the CTA-tile kernel with chunks / cpt decoding threads and a
+// producer warp.
 struct KernelEntry {
-    int dtype, chunk_bits, chunks, cpt, nwarp;
+    int dtype, chunk_bits, chunks, cpt, nwarp, walker;
     KernelFn fn;
 };
 
-#define DF11_KERNEL(DT, CB, CH) \
-    {DT, CB, CH, 1, 0, &decode_kernel<DT, CB, 1, CH>}, { DT, CB, CH, 2, 0, &decode_kernel<DT, CB, 2, CH / 2> }
-#define DF11_WARP_KERNEL(DT, CB) \
-    {DT, CB, 32, 1, 8, &decode_warp_kernel<DT, CB, 8>}, { DT, CB, 32, 1, 16, &decode_warp_kernel<DT, CB, 16> }
+#define DF11_KERNEL(DT, CB, CH)                                          \
+    {DT, CB, CH, 1, 0, DF11_WALKER_WINDOW, &decode_kernel<DT, CB, 1, CH>}, \
+    {                                                                    \
+        DT, CB, CH, 2, 0, DF11_WALKER_WINDOW, &decode_kernel<DT, CB, 2, CH / 2> \
+    }
+#define DF11_WARP_KERNEL(DT, CB)                                             \
+    {DT, CB, 32, 1, 8, DF11_WALKER_WINDOW, &decode_warp_kernel<DT, CB, 8>},   \
+        {DT, CB, 32, 1, 16, DF11_WALKER_WINDOW, &decode_warp_kernel<DT, CB, 16>}, \
+        {DT, CB, 32, 1, 16, DF11_WALKER_BYTE_STEP, &decode_fsm_kernel<DT, CB, 16>}, \
+        {DT, CB, 32, 1, 24, DF11_WALKER_BYTE_STEP, &decode_fsm_kernel<DT, CB, 24>}, \
+    {                                                                        \
+        DT, CB, 32, 1, 32, DF11_WALKER_BYTE_STEP, &decode_fsm_kernel<DT, CB, 32>  \
+    }
 
 const KernelEntry kKernels[] = {
     DF11_WARP_KERNEL(0, 128), DF11_WARP_KERNEL(1, 128), DF11_WARP_KERNEL(0, 256), DF11_WARP_KERNEL(1, 256),
@@ -980,10 +1285,10 @@ const KernelEntry kKernels[] = {
     DF11_KERNEL(0, 128, 512), DF11_KERNEL(1, 128, 512), DF11_KERNEL(0, 256, 256), DF11_KERNEL(1, 256, 256),
 };
 
-const KernelEntry *find_kernel(int dtype, int chunk_bits, int chunks, int cpt, int nwarp) {
+const KernelEntry *find_kernel(int dtype, int chunk_bits, int chunks, int cpt, int nwarp, int walker) {
     for (const auto &e : kKernels)
         if (e.dtype == dtype && e.chunk_bits == chunk_bits && e.chunks == chunks && e.cpt == cpt &&
-            e.nwarp == nwarp)
+            e.nwarp == nwarp && e.walker == walker)
             return &e;
     return nullptr;
 }
@@ -1032,10 +1337,9 @@ LaunchStatus build_params(const Blob *const *blobs, void *const *dst, int n, int
     const bool warp_tiles = b0.tile_threads == 32;
     const int cpt = opt.chunks_per_thread ? opt.chunks_per_thread : kDefaultChunksPerThread;
     if (cpt != 1 && cpt != 2) return LaunchStatus::kInvalid;
-    const int nwarp = warp_tiles ? (opt.warps_per_cta ? opt.warps_per_cta : kDefaultWarpsPerCta) : 0;
     if (warp_tiles && cpt != 1) return LaunchStatus::kInvalid;
-    const KernelEntry *ke = find_kernel(b0.dtype, b0.chunk_bits, b0.tile_threads, cpt, nwarp);
-    if (!ke) return LaunchStatus::kUnsupported;
+    if (opt.walker < DF11_WALKER_AUTO || opt.walker > DF11_WALKER_BYTE_STEP) return LaunchStatus::kInvalid;
+    if (!warp_tiles && opt.walker == DF11_WALKER_BYTE_STEP) return LaunchStatus::kUnsupported;
     DecodeParams &P = out->params;
     P = DecodeParams{};
     uint64_t tiles = 0, max_span = 0;
@@ -1066,10 +1370,34 @@ LaunchStatus build_params(const Blob *const *blobs, void *const *dst, int n, int
         if (b.max_span > max_span) max_span = b.max_span;
     }
     if (tiles >= (uint64_t{1} << 31)) return LaunchStatus::kInvalid;
+    // kernel: the byte-step walk for warp tiles unless the window walk is asked
+    // for, the code has a 1-bit codeword (a byte would end up to 8 codes) or
+    // its tables and the warps' buffers do not fit in shared memory
+    const int rows = b0.cb->fsm_rows;
+    const KernelEntry *ke = nullptr;
+    if (warp_tiles && opt.walker != DF11_WALKER_WINDOW && rows >= 2 && rows <= kFsmMaxRows &&
+        (opt.walker == DF11_WALKER_BYTE_STEP || b0.cb->min_len_used >= 2)) {
+        const int tries[3] = {32, 24, 16};
+        for (int nw : tries) {
+            if (opt.warps_per_cta && opt.warps_per_cta != nw) continue;
+            if (make_fsm_plan(b0.chunk_bits, nw, static_cast<uint32_t>(max_span), rows).total > kSmemBudget)
+                continue;
+            ke = find_kernel(b0.dtype, b0.chunk_bits, 32, 1, nw, DF11_WALKER_BYTE_STEP);
+            if (ke) break;
+        }
+        if (!ke && opt.walker == DF11_WALKER_BYTE_STEP) return LaunchStatus::kUnsupported;
+    }
+    if (!ke) {
+        const int nwarp = warp_tiles ? (opt.warps_per_cta ? opt.warps_per_cta : kDefaultWarpsPerCta) : 0;
+        ke = find_kernel(b0.dtype, b0.chunk_bits, b0.tile_threads, cpt, nwarp, DF11_WALKER_WINDOW);
+        if (!ke) return LaunchStatus::kUnsupported;
+    }
     const ImageLayout L0 = image_layout(b0);
     P.meta = reinterpret_cast<const uint32_t *>(b0.dev_image + L0.meta);
     P.syms = reinterpret_cast<const uint32_t *>(b0.dev_image + L0.syms);
     P.lut = reinterpret_cast<const uint16_t *>(b0.dev_image + L0.lut);
+    P.fsm = reinterpret_cast<const uint32_t *>(b0.dev_image + L0.fsm);
+    P.fsm_rows = rows;
     P.err = err;
     P.n_luts = b0.cb->n_luts();
     P.n_tensors = nt;
@@ -1079,8 +1407,12 @@ LaunchStatus build_params(const Blob *const *blobs, void *const *dst, int n, int
     out->max_span = static_cast<uint32_t>(max_span);
     out->n_lut_smem = P.n_luts < kSmemLutTables ? P.n_luts : kSmemLutTables;
     out->ctas_per_sm = opt.ctas_per_sm;
-    out->smem = warp_tiles ? make_warp_plan(b0.chunk_bits, nwarp, out->max_span, out->n_lut_smem).total
-                           : make_plan(b0.chunk_bits, b0.tile_threads, out->max_span, out->n_lut_smem).total;
+    if (ke->walker == DF11_WALKER_BYTE_STEP)
+        out->smem = make_fsm_plan(b0.chunk_bits, ke->nwarp, out->max_span, rows).total;
+    else if (warp_tiles)
+        out->smem = make_warp_plan(b0.chunk_bits, ke->nwarp, out->max_span, out->n_lut_smem).total;
+    else
+        out->smem = make_plan(b0.chunk_bits, b0.tile_threads, out->max_span, out->n_lut_smem).total;
     if (out->smem > kSmemBudget) return LaunchStatus::kUnsupported;
     return LaunchStatus::kOk;
 }
@@ -1103,13 +1435,15 @@ LaunchStatus shape_for(const Prepared &pp, LaunchShape *sh) {
     sh->grid = static_cast<int>(want < need ? want : need);
     sh->block = block;
     sh->smem = static_cast<int>(pp.smem);
+    sh->walker = pp.ke->walker;
     return LaunchStatus::kOk;
 }
 
 }  // namespace
 
 bool kernel_available(int dtype, int chunk_bits, int tile_threads) {
-    return find_kernel(dtype, chunk_bits, tile_threads, 1, tile_threads == 32 ? kDefaultWarpsPerCta : 0) != nullptr;
+    return find_kernel(dtype, chunk_bits, tile_threads, 1, tile_threads == 32 ? kDefaultWarpsPerCta : 0,
+                       DF11_WALKER_WINDOW) != nullptr;
 }
 
 LaunchStatus decode_launch_shape(const Blob *const *blobs, int n, const DecodeOptions &opt, LaunchShape *out) {

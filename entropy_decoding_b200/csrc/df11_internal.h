@@ -18,6 +18,21 @@
 //     << 11), so one add advances both.  meta[v] = kMetaLong (consumed 1024,
 //     no symbol) when the first code is longer than 12 bits.  syms[v] holds
 //     the symbols, first in the low byte, unused bytes zero.
+//   * byte-step transition tables ("fsm"): one row of 256 entries per node of
+//     the code tree that a byte boundary can fall on (the root, then the
+//     other internal nodes in decreasing order of the probability mass below
+//     them, up to kFsmMaxRows - 1 rows), plus a dead row.  Entry (row v,
+//     byte b) is what walking the 8 bits of b from node v produces: ctl (u32)
+//     = end mask (bit i set when a code ends at bit i of b, bit 0 = the first
+//     bit) | next row << kFsmRowShift | codes ended << kFsmCountShift, and
+//     syms (u32) = the first up to 4 symbols ended, first in the low byte.
+//     A byte that ends more than 4 codes, leads to a node without a row or
+//     meets a prefix that is no codeword leads to the dead row, whose
+//     entries lead back to it and end no code.  The walk of a byte is thus
+//     one lookup that does not depend on where the codes start: the
+//     hierarchical tables generalised to every node at a byte boundary.
+//     Row v occupies bytes [v * kFsmRowBytes, (v + 1) * kFsmRowBytes), entry
+//     b the 8 bytes {ctl, syms} at b * 8 within it.
 //   * in the device image the stream is stored as 32-bit words whose bit 31
 //     is the earliest stream bit (each 4-byte group of the MSB-first byte
 //     stream reversed), so a word load needs no byte swap.
@@ -40,24 +55,31 @@ constexpr uint16_t kLutInvalid = 0x4000 | (1u << 8);
 constexpr int kMaxLutTables = 0x7FFF;
 constexpr int kSmemLutTables = 16;  // hierarchical tables staged in shared memory; the rest stay in global
 
+constexpr int kFsmMaxRows = 64;  // including the dead row
+constexpr int kFsmRowBytes = kLutEntries * 8;
+constexpr int kFsmRowShift = 11;  // row index << 11 = the row's byte offset
+constexpr uint32_t kFsmRowMask = static_cast<uint32_t>(kFsmMaxRows - 1) << kFsmRowShift;
+constexpr int kFsmCountShift = 29;
+
 constexpr int kMaxCodeLen = 32;
 constexpr int kMaxTensorsPerLaunch = 64;
 constexpr uint64_t kImageAlign = 256;
 constexpr uint64_t kStreamTail = 16;  // zero bytes after the last tile: look-ahead of the last thread
 constexpr uint64_t kPlaneTail = 32;
+constexpr uint64_t kGapsTail = 16;  // readable bytes after the last tile's gaps: the next chunk's gap
 
 inline uint64_t align_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
 
 // Offsets of the sections inside one blob's device image.
 struct ImageLayout {
-    uint64_t meta, syms, lut, gaps, out_off, stream, plane, total;
+    uint64_t meta, syms, lut, fsm, gaps, out_off, stream, plane, total;
 };
 
 // Header at offset 0 of every device image (kept for inspection; the kernel
 // takes everything it needs from its launch parameters).
 struct ImageHeader {
     char magic[8];  // "DF11IMG1"
-    uint32_t dtype, chunk_bits, tile_threads, n_luts;
+    uint32_t dtype, chunk_bits, tile_threads, n_luts, fsm_rows, reserved;
     uint64_t n_elems, total_bits, n_tiles, max_span;
     ImageLayout layout;
 };
@@ -80,6 +102,9 @@ struct DecodeParams {
     const uint32_t *meta;
     const uint32_t *syms;
     const uint16_t *lut;
+    const uint32_t *fsm;  // fsm_rows * kFsmRowBytes bytes
+    int32_t fsm_rows;
+    int32_t pad;
     int *err;
     int32_t n_luts;
     int32_t n_tensors;

@@ -488,6 +488,7 @@ std::string encode_device_noalloc(const EncodeJob &J, uint8_t *image, uint64_t i
     h.chunk_bits = static_cast<uint32_t>(meta.chunk_bits);
     h.tile_threads = static_cast<uint32_t>(meta.tile_threads);
     h.n_luts = static_cast<uint32_t>(J.cb->n_luts());
+    h.fsm_rows = static_cast<uint32_t>(J.cb->fsm_rows);
     h.n_elems = meta.n;
     h.total_bits = total;
     h.n_tiles = meta.n_tiles;
@@ -497,6 +498,8 @@ std::string encode_device_noalloc(const EncodeJob &J, uint8_t *image, uint64_t i
         cudaMemcpyAsync(image + L.meta, J.cb->meta.data(), kMultiEntries * 4, cudaMemcpyHostToDevice, s) != cudaSuccess ||
         cudaMemcpyAsync(image + L.syms, J.cb->syms.data(), kMultiEntries * 4, cudaMemcpyHostToDevice, s) != cudaSuccess ||
         cudaMemcpyAsync(image + L.lut, J.cb->lut.data(), J.cb->lut.size() * 2, cudaMemcpyHostToDevice, s) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(image + L.fsm, J.cb->fsm.data(), J.cb->fsm.size() * 4, cudaMemcpyHostToDevice, s) !=
             cudaSuccess)
         return "table upload failed";
     if (!J.n) return cudaStreamSynchronize(s) == cudaSuccess ? "" : "synchronise failed";

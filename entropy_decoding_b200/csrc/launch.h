@@ -12,7 +12,8 @@ enum class LaunchStatus { kOk, kInvalid, kUnsupported, kCuda };
 struct DecodeOptions {
     int chunks_per_thread = 0;  // 0 = kDefaultChunksPerThread
     int ctas_per_sm = 0;        // 0 = as many as fit
-    int warps_per_cta = 0;      // warp-tile layouts: 0 = kDefaultWarpsPerCta
+    int warps_per_cta = 0;      // warp-tile layouts: 0 = kDefaultWarpsPerCta (window) / most that fit (byte step)
+    int walker = 0;             // DF11_WALKER_*: 0 = auto
 };
 
 constexpr int kDefaultChunksPerThread = 1;
@@ -22,6 +23,7 @@ struct LaunchShape {
     int grid = 0;
     int block = 0;
     int smem = 0;
+    int walker = 0;  // DF11_WALKER_WINDOW or DF11_WALKER_BYTE_STEP
 };
 
 bool kernel_available(int dtype, int chunk_bits, int tile_threads);

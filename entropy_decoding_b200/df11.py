@@ -57,7 +57,10 @@ class EncodeResult(ctypes.Structure):
 
 class DecodeOpts(ctypes.Structure):
     _fields_ = [("chunks_per_thread", ctypes.c_int32), ("ctas_per_sm", ctypes.c_int32),
-                ("warps_per_cta", ctypes.c_int32)]
+                ("warps_per_cta", ctypes.c_int32), ("walker", ctypes.c_int32)]
+
+
+WALKER_AUTO, WALKER_WINDOW, WALKER_BYTE_STEP = 0, 1, 2
 
 
 _P = ctypes.c_void_p
@@ -88,7 +91,7 @@ _SIGS = {
     "df11_decode": ([_PP, _PP, _I, _P, _P], _S),
     "df11_decode_ex": ([_PP, _PP, _I, _P, _P, ctypes.POINTER(DecodeOpts)], _S),
     "df11_decode_launch_shape_ex": ([_PP, _I, ctypes.POINTER(DecodeOpts), ctypes.POINTER(_I), ctypes.POINTER(_I),
-                                     ctypes.POINTER(_I)], _S),
+                                     ctypes.POINTER(_I), ctypes.POINTER(_I)], _S),
     "df11_histogram_device": ([_I, _P, _U64, _P, _P], _S),
     "df11_codebook_from_counts": ([_I, _P, _I, _I, _PP], _S),
     "df11_encode_device_scratch_bytes": ([_U64], _U64),
@@ -267,8 +270,8 @@ def df11_decode(blobs, dst_ptrs, err_ptr: int | None = None, stream: int = 0):
 
 
 def df11_decode_ex(blobs, dst_ptrs, err_ptr: int | None = None, stream: int = 0, chunks_per_thread: int = 0,
-                   ctas_per_sm: int = 0, warps_per_cta: int = 0):
-    o = DecodeOpts(chunks_per_thread, ctas_per_sm, warps_per_cta)
+                   ctas_per_sm: int = 0, warps_per_cta: int = 0, walker: int = 0):
+    o = DecodeOpts(chunks_per_thread, ctas_per_sm, warps_per_cta, walker)
     _check(_lib.df11_decode_ex(_ptr_array([b.handle.value for b in blobs]), _ptr_array(dst_ptrs), len(blobs),
                                err_ptr or None, stream or None, ctypes.byref(o)), "df11_decode_ex")
 
@@ -281,13 +284,15 @@ def df11_decode_host(blobs, host_image_ptrs, dev_image_ptrs, dst_dev_ptrs, dst_h
 
 
 def df11_decode_launch_shape(blobs, chunks_per_thread: int = 0, ctas_per_sm: int = 0,
-                             warps_per_cta: int = 0) -> tuple[int, int, int]:
-    g, b, s = _I(), _I(), _I()
-    o = DecodeOpts(chunks_per_thread, ctas_per_sm, warps_per_cta)
+                             warps_per_cta: int = 0, walker: int = 0, with_walker: bool = False):
+    """(grid, block, shared-memory bytes) of the launch df11_decode_ex would
+    make with these options, plus the walk it would use when with_walker."""
+    g, b, s, w = _I(), _I(), _I(), _I()
+    o = DecodeOpts(chunks_per_thread, ctas_per_sm, warps_per_cta, walker)
     _check(_lib.df11_decode_launch_shape_ex(_ptr_array([x.handle.value for x in blobs]), len(blobs), ctypes.byref(o),
-                                            ctypes.byref(g), ctypes.byref(b), ctypes.byref(s)),
+                                            ctypes.byref(g), ctypes.byref(b), ctypes.byref(s), ctypes.byref(w)),
            "df11_decode_launch_shape")
-    return g.value, b.value, s.value
+    return (g.value, b.value, s.value, w.value) if with_walker else (g.value, b.value, s.value)
 
 
 def df11_histogram_device(dtype: str, src_ptr: int, n: int, counts_ptr: int, stream: int = 0):

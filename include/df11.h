@@ -229,8 +229,24 @@ df11_status df11_decode(const df11_blob *const *blobs, void *const *dst_dev, int
 typedef struct {
     int32_t chunks_per_thread; /* CTA-tile layouts: chunks each decoding thread walks, 1 or 2 (0 = 1) */
     int32_t ctas_per_sm;       /* persistent CTAs per SM, capped by occupancy (0 = as many as fit) */
-    int32_t warps_per_cta;     /* warp-tile layout (tile_threads 32): 8 or 16 (0 = 16) */
+    int32_t warps_per_cta;     /* warp-tile layout (tile_threads 32): warps per CTA; window walker 8 or
+                                  16 (0 = 16), byte-step walker 16, 24 or 32 (0 = the most that fit) */
+    int32_t walker;            /* warp-tile layout: DF11_WALKER_AUTO (0), DF11_WALKER_WINDOW or
+                                  DF11_WALKER_BYTE_STEP; CTA-tile layouts take 0 or WINDOW only */
 } df11_decode_opts;
+
+/* How a decoding thread walks its chunk (both give the same output).
+ * WINDOW: lookups in the 12-bit multi-symbol table, each consuming the
+ * whole codes in the next 12 bits (a variable number of bits).
+ * BYTE_STEP: lookups in the byte-step transition tables, one per 8 stream
+ * bits whatever the code boundaries, so every thread of a warp takes the
+ * same number of steps; a thread whose walk reaches the dead row falls back
+ * to the window walk.  One CTA per SM holds the tables (up to 128 KB of
+ * shared memory).  AUTO picks BYTE_STEP for warp tiles when the code has no
+ * 1-bit codeword and the tables fit, else WINDOW. */
+#define DF11_WALKER_AUTO 0
+#define DF11_WALKER_WINDOW 1
+#define DF11_WALKER_BYTE_STEP 2
 
 /* df11_decode with explicit launch options (opts may be NULL).  The result is
  * identical for every option value; only the speed changes. */
@@ -253,10 +269,12 @@ df11_status df11_decode_host(df11_blob *const *blobs, const void *const *host_im
 df11_status df11_decode_launch_shape(const df11_blob *const *blobs, int n_blobs, int *grid,
                                      int *block, int *smem_bytes);
 
-/* As df11_decode_launch_shape, for the given options (opts may be NULL). */
+/* As df11_decode_launch_shape, for the given options (opts may be NULL);
+ * *walker (nullable) receives the walk the launch would use,
+ * DF11_WALKER_WINDOW or DF11_WALKER_BYTE_STEP. */
 df11_status df11_decode_launch_shape_ex(const df11_blob *const *blobs, int n_blobs,
                                         const df11_decode_opts *opts, int *grid, int *block,
-                                        int *smem_bytes);
+                                        int *smem_bytes, int *walker);
 
 /* ---------------------------------------------------------------------
  * GPU encoder (the offline half, run on the device)

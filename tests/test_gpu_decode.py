@@ -21,10 +21,11 @@ def df11():
 
 
 def _roundtrip(df11, oracle_mod, x, dt, chunk_bits=128, tile_threads=32, max_len=0, check_oracle=True, cpt=0,
-               ctas=0, wpc=0):
+               ctas=0, wpc=0, walker=0):
     cb = df11.df11_build_codebook(dt, [x], max_len)
     blob = df11.df11_encode(cb, x, chunk_bits, tile_threads)
-    (out,), err, guards = decode_gpu(df11, [blob], chunks_per_thread=cpt, ctas_per_sm=ctas, warps_per_cta=wpc)
+    (out,), err, guards = decode_gpu(df11, [blob], chunks_per_thread=cpt, ctas_per_sm=ctas, warps_per_cta=wpc,
+                                     walker=walker)
     assert err == 0
     assert guards
     assert out.shape == x.shape
@@ -77,14 +78,29 @@ def test_parity_cta_layouts(df11, oracle_mod, layout, case, cpt):
     _roundtrip(df11, oracle_mod, make(), dt, *layout, cpt=cpt)
 
 
-@pytest.mark.parametrize("wpc", [8, 16])
+WALKS = [(1, 8), (1, 16), (2, 16), (2, 24), (2, 32)]  # (walker, warps per CTA)
+
+
+@pytest.mark.parametrize("walk", WALKS)
 @pytest.mark.parametrize("layout", WARP_LAYOUTS)
-@pytest.mark.parametrize("case", ["heavy_2m", "e4m3_normal", "single_symbol", "uniform_random", "fib26"])
-def test_parity_warp_layouts(df11, oracle_mod, layout, case, wpc):
+@pytest.mark.parametrize("case", ["heavy_2m", "e4m3_normal", "single_symbol", "uniform_random", "fib26",
+                                  "normal_1m", "all_bf16"])
+def test_parity_warp_layouts(df11, oracle_mod, layout, case, walk):
     """Warp-tile layouts (one out_off per 32 chunks, warp-shuffle scan), with
-    8 and 16 warps per CTA."""
+    the 12-bit window walk (8 and 16 warps per CTA) and the byte-step walk (16,
+    24 and 32 warps in one CTA per SM).  A 1-bit code (single_symbol) sends
+    every thread of the byte-step walk to the window fallback, random bits
+    send many; both must still be exact."""
     dt, make = SMALL[case]
-    _roundtrip(df11, oracle_mod, make(), dt, *layout, wpc=wpc)
+    walker, wpc = walk
+    try:
+        _roundtrip(df11, oracle_mod, make(), dt, *layout, wpc=wpc, walker=walker)
+    except df11.Df11Error as e:
+        # 1-bit codes in 256-bit chunks: a tile spans 8192 codes and 32 warps'
+        # exponent buffers no longer fit in shared memory beside the tables
+        if not (walker == 2 and e.status == df11.DF11_EUNSUPPORTED and case == "single_symbol"):
+            raise
+        pytest.skip("tile span too large for this many warps")
 
 
 @pytest.mark.parametrize("ctas", [1, 2])
@@ -177,14 +193,19 @@ def test_corrupted_device_data_sets_error_flag(df11):
     n = blob.info().device_bytes
     img = np.zeros(n, np.uint8)
     df11.df11_blob_device_image(blob, img.ctypes.data, n)
-    out_off_at = struct.unpack_from("<Q", img.tobytes(), 56 + 8 * 4)[0]
-    gaps_at = struct.unpack_from("<Q", img.tobytes(), 56 + 8 * 3)[0]
-    for what in ("out_off", "gap"):
+    # layout offsets in the header: meta, syms, lut, fsm, gaps, out_off, ...
+    fsm_at = struct.unpack_from("<Q", img.tobytes(), 64 + 8 * 3)[0]
+    gaps_at = struct.unpack_from("<Q", img.tobytes(), 64 + 8 * 4)[0]
+    out_off_at = struct.unpack_from("<Q", img.tobytes(), 64 + 8 * 5)[0]
+    rng = np.random.default_rng(7)
+    for what in ("out_off", "gap", "fsm"):
         bad = img.copy()
         if what == "out_off":
             bad[out_off_at + 8 * 3: out_off_at + 8 * 4] = np.frombuffer(struct.pack("<Q", 10 ** 12), np.uint8)
-        else:
+        elif what == "gap":
             bad[gaps_at + 5] = (int(bad[gaps_at + 5]) + 3) % 32
+        else:  # random counts, masks, symbols and rows in the first two transition rows
+            bad[fsm_at: fsm_at + 4096] = rng.integers(0, 256, 4096, dtype=np.uint8)
         dev = torch.from_numpy(bad).cuda()
         df11.df11_blob_bind(blob, dev.data_ptr(), n, keep=dev)
         guard = 64
@@ -198,9 +219,37 @@ def test_corrupted_device_data_sets_error_flag(df11):
         assert (g[:guard] == 0xA5).all() and (g[guard + nbytes:] == 0xA5).all()
         if what == "out_off":
             assert e & df11.DEV_ERR_AUX
+        if what == "fsm":
+            assert e & df11.DEV_ERR_SPAN
         # a shifted gap is caught when it changes the tile's code count; when
         # the parse resynchronises to the same count the output is wrong but
         # still inside the destination, which is what is checked above
+
+
+def test_transition_rows_past_the_table_are_dead(df11):
+    """An E4M3 code has at most 16 transition rows; root entries whose next
+    row lies past the last one are sent to the dead row when the table is
+    staged, so every thread falls back to the window walk and the output is
+    still exact."""
+    import struct
+    x = synth.normal_e4m3(np.random.SeedSequence(9), 400003)
+    blob = df11.df11_encode(df11.df11_build_codebook("e4m3", [x]), x)
+    n = blob.info().device_bytes
+    img = np.zeros(n, np.uint8)
+    df11.df11_blob_device_image(blob, img.ctypes.data, n)
+    rows = struct.unpack_from("<I", img.tobytes(), 24)[0]
+    assert 2 <= rows <= 16
+    fsm_at = struct.unpack_from("<Q", img.tobytes(), 64 + 8 * 3)[0]
+    ent = img[fsm_at: fsm_at + 2048].view(np.uint32)
+    ent[0::2] |= np.uint32(63 << 11)
+    dev = torch.from_numpy(img).cuda()
+    df11.df11_blob_bind(blob, dev.data_ptr(), n, keep=dev)
+    out = torch.empty(x.size, dtype=torch.uint8, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    df11.df11_decode_ex([blob], [out.data_ptr()], err.data_ptr(), walker=df11.WALKER_BYTE_STEP)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert np.array_equal(out.cpu().numpy(), x)
 
 
 def test_decode_host_end_to_end(df11):
@@ -227,14 +276,28 @@ def test_launch_shape_is_persistent(df11):
     df11.upload(blob)
     grid, block, smem = df11.df11_decode_launch_shape([blob])
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    assert block == 16 * 32  # default layout: warp tiles, 16 warps per CTA
-    assert grid % sms == 0 or grid * 16 >= blob.info().n_tiles
-    g8, b8, _ = df11.df11_decode_launch_shape([blob], warps_per_cta=8, ctas_per_sm=1)
+    # default layout: warp tiles, byte-step walk, one CTA per SM of as many warps as fit
+    assert block in (16 * 32, 24 * 32, 32 * 32)
+    assert grid == sms or grid * (block // 32) >= blob.info().n_tiles
+    gw, bw, _ = df11.df11_decode_launch_shape([blob], walker=df11.WALKER_WINDOW)
+    assert bw == 16 * 32 and (gw % sms == 0 or gw * 16 >= blob.info().n_tiles)
+    g8, b8, _ = df11.df11_decode_launch_shape([blob], warps_per_cta=8, ctas_per_sm=1, walker=df11.WALKER_WINDOW)
     assert b8 == 8 * 32 and g8 == sms
+    g24, b24, s24 = df11.df11_decode_launch_shape([blob], warps_per_cta=24, walker=df11.WALKER_BYTE_STEP)
+    assert b24 == 24 * 32 and g24 == sms and s24 >= 2 * 2048  # at least the root and the dead row
+    assert df11.df11_decode_launch_shape([blob], with_walker=True)[3] == df11.WALKER_BYTE_STEP
+    # a 1-bit codeword: automatic choice is the window walk
+    one = synth.constant_bf16(5000, 0.5)
+    b1bit = df11.df11_encode(df11.df11_build_codebook("bf16", [one]), one)
+    df11.upload(b1bit)
+    assert df11.df11_decode_launch_shape([b1bit], with_walker=True)[3] == df11.WALKER_WINDOW
     cta = df11.df11_encode(df11.df11_build_codebook("bf16", [x]), x, 128, 256)
     df11.upload(cta)
     g1, b1, _ = df11.df11_decode_launch_shape([cta])
     assert b1 == 256 + 32  # CTA tiles: one chunk per decoding thread plus the producer warp
     g2, b2, _ = df11.df11_decode_launch_shape([cta], chunks_per_thread=2, ctas_per_sm=1)
     assert b2 == 256 // 2 + 32 and g2 == min(sms, cta.info().n_tiles)
+    assert df11.df11_decode_launch_shape([cta], with_walker=True)[3] == df11.WALKER_WINDOW
+    with pytest.raises(df11.Df11Error):
+        df11.df11_decode_launch_shape([cta], walker=df11.WALKER_BYTE_STEP)
     assert 0 < smem <= 227 * 1024

@@ -92,12 +92,12 @@ def test_fibonacci_34_reaches_32_bit_codes(df11, oracle_mod):
 def _image_layout(img: bytes):
     magic = img[:8]
     assert magic == b"DF11IMG1"
-    dtype, chunk, tile, n_luts = struct.unpack_from("<4I", img, 8)
-    n, total, n_tiles, max_span = struct.unpack_from("<4Q", img, 24)
-    keys = ["meta", "syms", "lut", "gaps", "out_off", "stream", "plane", "total"]
-    lay = dict(zip(keys, struct.unpack_from("<8Q", img, 56)))
-    return dict(dtype=dtype, chunk=chunk, tile=tile, n_luts=n_luts, n=n, total_bits=total, n_tiles=n_tiles,
-                max_span=max_span, **lay)
+    dtype, chunk, tile, n_luts, fsm_rows, _ = struct.unpack_from("<6I", img, 8)
+    n, total, n_tiles, max_span = struct.unpack_from("<4Q", img, 32)
+    keys = ["meta", "syms", "lut", "fsm", "gaps", "out_off", "stream", "plane", "total"]
+    lay = dict(zip(keys, struct.unpack_from("<9Q", img, 64)))
+    return dict(dtype=dtype, chunk=chunk, tile=tile, n_luts=n_luts, fsm_rows=fsm_rows, n=n, total_bits=total,
+                n_tiles=n_tiles, max_span=max_span, **lay)
 
 
 def _image(df11, blob):
@@ -134,7 +134,7 @@ def test_decode_tables_match_independent_prefix_decode(df11, oracle_mod, case):
     cb = df11.df11_build_codebook(dt, [x])
     blob = df11.df11_encode(cb, x)
     img = _image(df11, blob)
-    lay = _image_layout(img.tobytes()[:128])
+    lay = _image_layout(img.tobytes()[:256])
     lengths = oracle_mod.build_lengths([x], dt)
     codes = oracle_mod.canonical_codes(lengths)
     table = _prefix_decoder(lengths, codes)
@@ -173,6 +173,73 @@ def test_decode_tables_match_independent_prefix_decode(df11, oracle_mod, case):
         else:
             assert not e & 0xC000
             assert (e & 0xFF, (e >> 8) & 0x3F) == r
+
+
+def _tree_rows(lengths, codes, max_rows=64):
+    """Internal nodes of the code tree as (depth, prefix) in the row order the
+    transition tables use: the root first, then decreasing probability mass
+    below the node (a code of length l weighs 2^-l), then depth, then prefix.
+    The last row is the dead row; returns (nodes of the live rows, rows)."""
+    mass = {}
+    for s, l in enumerate(lengths):
+        l = int(l)
+        for d in range(l):
+            key = (d, int(codes[s]) >> (l - d))
+            mass[key] = mass.get(key, 0.0) + 2.0 ** -l
+    nodes = sorted(mass, key=lambda k: (k != (0, 0), -mass[k], k[0], k[1]))
+    live = nodes[:max_rows - 1]
+    return live, len(live) + 1
+
+
+@pytest.mark.parametrize("case", ["normal", "heavy", "fib", "single", "e4m3", "random"])
+def test_transition_tables_match_independent_prefix_decode(df11, oracle_mod, case):
+    """Every entry of the byte-step transition tables in the device image:
+    starting from the row's tree node, the 8 bits of the byte are decoded with
+    a dictionary prefix decoder over the oracle's canonical codes; the entry
+    must list the codes that end in the byte (end mask, count, first four
+    symbols) and lead to the row of the node the byte stops on, or to the dead
+    row when that node has no row, more than four codes end or a prefix is no
+    codeword."""
+    dt, make = _cases()[case]
+    x = make()
+    cb = df11.df11_build_codebook(dt, [x])
+    img = _image(df11, df11.df11_encode(cb, x))
+    lay = _image_layout(img.tobytes()[:256])
+    lengths = oracle_mod.build_lengths([x], dt)
+    codes = oracle_mod.canonical_codes(lengths)
+    table = _prefix_decoder(lengths, codes)
+    live, rows = _tree_rows(lengths, codes)
+    assert lay["fsm_rows"] == rows
+    row_of = {node: r for r, node in enumerate(live)}
+    dead = rows - 1
+    fsm = img[lay["fsm"]:lay["fsm"] + rows * 2048].view(np.uint32).reshape(rows, 256, 2)
+    assert np.all(fsm[dead, :, 0] == dead << 11) and np.all(fsm[dead, :, 1] == 0)
+    for r, (depth, prefix) in enumerate(live):
+        for b in range(256):
+            bits, nbits = (prefix << 8) | b, depth + 8
+            pos, ends, got = 0, 0, []
+            while pos < nbits:
+                hit = None
+                for l in range(1, nbits - pos + 1):
+                    if (l, (bits >> (nbits - pos - l)) & ((1 << l) - 1)) in table:
+                        hit = l
+                        break
+                if hit is None:
+                    break
+                got.append(table[(hit, (bits >> (nbits - pos - hit)) & ((1 << hit) - 1))])
+                pos += hit
+                ends |= 1 << (pos - depth - 1)
+            # the leftover bits: a node with a row, a node without one, or a
+            # prefix of no codeword (the last two lead to the dead row)
+            rest = nbits - pos
+            node = (rest, bits & ((1 << rest) - 1))
+            nxt = dead if (len(got) > 4 or node not in row_of) else row_of[node]
+            ctl, sy = int(fsm[r, b, 0]), int(fsm[r, b, 1])
+            assert ctl & 0xFF == ends, (r, b)
+            assert (ctl >> 11) & 0x3F == nxt, (r, b)
+            assert ctl >> 29 == min(len(got), 7), (r, b)
+            assert ctl & 0x1FFE0700 == 0, (r, b)
+            assert sy == sum(s << (8 * i) for i, s in enumerate(got[:4])), (r, b)
 
 
 def test_serialize_roundtrip_and_size(df11, oracle_mod):
@@ -247,7 +314,7 @@ def test_device_image_layout(df11):
     cb = df11.df11_build_codebook("bf16", [x])
     blob = df11.df11_encode(cb, x)
     img = _image(df11, blob)
-    lay = _image_layout(img.tobytes()[:128])
+    lay = _image_layout(img.tobytes()[:256])
     info = blob.info()
     assert lay["total"] == info.device_bytes == img.size
     for k in ("meta", "syms", "lut", "gaps", "out_off", "stream", "plane"):
