@@ -977,6 +977,14 @@ __device__ __forceinline__ uint32_t step_off(uint32_t x, int k) {
     return k == 3 ? (x << 3) & 0x7F8u : (x >> (21 - 8 * k)) & 0x7F8u;
 }
 
+// Entry offset of byte k of x in a row of the compact control array: byte * 4.
+__device__ __forceinline__ uint32_t step_off4(uint32_t x, int k) {
+    return k == 3 ? (x << 2) & 0x3FCu : (x >> (22 - 8 * k)) & 0x3FCu;
+}
+
+// Row field of the compact control words (row << 10: rows of 1 KB).
+constexpr uint32_t kCtlRowMask = kFsmRowMask >> 1;
+
 // The byte-step walk of one chunk.  The thread's codes occupy bits [g, g +
 // 8 * nfull + r) of the words w[0..CW] followed by w2 (earliest bit first):
 // from the first code start in the chunk to the first code start in the next
@@ -988,15 +996,17 @@ __device__ __forceinline__ uint32_t step_off(uint32_t x, int k) {
 // its longest range (jmax steps).  A last partial byte (r bits) counts only
 // the codes whose end mask bit falls in its first r bits; those end exactly
 // at the range's end, so the codes of the next chunk are never counted.
-// Phase 1 (EMIT = false) returns the number of codes and, in ctl_out, the
-// last entry, whose row is the dead row (`dead`) when the walk left the
-// tables or the partial byte ends more than the 4 codes an entry holds
-// (possible only with a 1-bit codeword).  Phase 2 (EMIT = true) writes the
-// symbols from shared-memory address out on.
-template <int CB, bool EMIT>
-__device__ __forceinline__ uint32_t byte_step_walk(const uint32_t (&w)[CB / 32 + 1], uint32_t w2, int g, int nfull,
-                                                   int r, int jmax, const uint8_t *tab, uint32_t out, uint32_t dead,
-                                                   uint32_t &ctl_out) {
+//
+// Phase 1 (byte_step_count) walks the compact control words (4 bytes per
+// entry, so a warp's random lookups spread over all 32 banks) and returns the
+// number of codes; ctl_out receives the last control word, whose row is the
+// dead row (`dead`, in control-word form) when the walk left the tables or the
+// partial byte ends more than the 4 codes an entry holds (possible only with
+// a 1-bit codeword).
+template <int CB>
+__device__ __forceinline__ uint32_t byte_step_count(const uint32_t (&w)[CB / 32 + 1], uint32_t w2, int g, int nfull,
+                                                    int r, int jmax, const uint8_t *ctl_tab, uint32_t dead,
+                                                    uint32_t &ctl_out) {
     constexpr int CW = CB / 32, NFIX = (CB - 32) / 8;
     uint32_t ctl = 0, cnt = 0;
 #pragma unroll
@@ -1007,27 +1017,14 @@ __device__ __forceinline__ uint32_t byte_step_walk(const uint32_t (&w)[CB / 32 +
         for (int k = 0; k < 4; ++k) {
             const int j = 4 * m + k;
             if (j >= NFIX && j >= jmax) break;
-            const uint32_t a = (ctl & kFsmRowMask) | step_off(x, k);
-            if constexpr (!EMIT) {
-                const uint32_t e = *reinterpret_cast<const uint32_t *>(tab + a);
-                if (j < NFIX || j < nfull) {
-                    ctl = e;
-                    cnt += e >> kFsmCountShift;
-                } else if (j == nfull) {
-                    const uint32_t c = static_cast<uint32_t>(__popc(e & ((1u << r) - 1u)));
-                    cnt += c;
-                    if (c > 4) ctl = dead;
-                }
-            } else {
-                const uint2 e = *reinterpret_cast<const uint2 *>(tab + a);
-                if (j < NFIX || j < nfull) {
-                    ctl = e.x;
-                    put_symbols(e.y, out);
-                    out += e.x >> kFsmCountShift;
-                } else if (j == nfull) {
-                    const uint32_t c = min(static_cast<uint32_t>(__popc(e.x & ((1u << r) - 1u))), 4u);
-                    if (c) put_symbols(e.y & (0xFFFFFFFFu >> (32u - 8u * c)), out);
-                }
+            const uint32_t e = *reinterpret_cast<const uint32_t *>(ctl_tab + ((ctl & kCtlRowMask) | step_off4(x, k)));
+            if (j < NFIX || j < nfull) {
+                ctl = e;
+                cnt += e >> kFsmCountShift;
+            } else if (j == nfull) {
+                const uint32_t c = static_cast<uint32_t>(__popc(e & ((1u << r) - 1u)));
+                cnt += c;
+                if (c > 4) ctl = dead;
             }
         }
     }
@@ -1035,13 +1032,68 @@ __device__ __forceinline__ uint32_t byte_step_walk(const uint32_t (&w)[CB / 32 +
     return cnt;
 }
 
+// Phase 2: the same walk on the full entries {ctl, syms}, writing the symbols
+// in order from shared-memory byte address `out` on.  Symbols are assembled
+// in a register (acc holds f8 / 8 pending bytes, unused bytes zero) and every
+// completed 32-bit word is stored with one plain store.  The word the range
+// starts in may hold earlier threads' bytes (stored as zeros here) and the
+// word it ends in later threads' bytes: that last, partial word is returned
+// in acc / wp / f8 and OR-ed in by the caller after a __syncwarp, so it
+// lands after every plain store of the warp and no store clears another
+// thread's bytes.  The buffer is zero outside the words written.
+template <int CB>
+__device__ __forceinline__ void byte_step_emit(const uint32_t (&w)[CB / 32 + 1], uint32_t w2, int g, int nfull,
+                                               int r, int jmax, const uint8_t *tab, uint32_t out, uint32_t &acc,
+                                               uint32_t &wp, uint32_t &f8) {
+    constexpr int CW = CB / 32, NFIX = (CB - 32) / 8;
+    uint32_t ctl = 0;
+    acc = 0;
+    wp = out & ~3u;
+    f8 = (out & 3u) << 3;
+#pragma unroll
+    for (int m = 0; m <= CW; ++m) {
+        if (4 * m >= NFIX && 4 * m >= jmax) break;  // warp-uniform
+        const uint32_t x = __funnelshift_l(m < CW ? w[m + 1] : w2, w[m], static_cast<uint32_t>(g));
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int j = 4 * m + k;
+            if (j >= NFIX && j >= jmax) break;
+            const uint2 e = *reinterpret_cast<const uint2 *>(tab + ((ctl & kFsmRowMask) | step_off(x, k)));
+            uint32_t sy, c8;
+            if (j < NFIX || j < nfull) {
+                ctl = e.x;
+                sy = e.y;
+                c8 = e.x >> (kFsmCountShift - 3);  // 8 x codes ended
+            } else if (j == nfull) {
+                const uint32_t c = min(static_cast<uint32_t>(__popc(e.x & ((1u << r) - 1u))), 4u);
+                sy = c ? e.y & (0xFFFFFFFFu >> (32u - 8u * c)) : 0u;
+                c8 = 8u * c;
+            } else {
+                continue;
+            }
+            const uint32_t lo = acc | (sy << f8);
+            const uint32_t hi = __funnelshift_l(sy, 0u, f8);  // bytes pushed past the word
+            f8 += c8;
+            if (f8 >= 32u) {
+                asm volatile("st.shared.u32 [%0], %1;" ::"r"(wp), "r"(lo) : "memory");
+                wp += 4u;
+                f8 -= 32u;
+                acc = hi;
+            } else {
+                acc = lo;
+            }
+        }
+    }
+}
+
 // Shared memory of the byte-step kernel: the transition table (fsm_rows rows
-// of kFsmRowBytes) at offset 0, the root hierarchical table, then per warp
+// of kFsmRowBytes) at offset 0, its control words alone (rows of 1 KB, row
+// field at bit 10), the root hierarchical table, then per warp
 // its mbarrier, one stage (the tile's 32 chunks + 16 look-ahead bytes, then
 // 48 gap bytes: its own 32 and the next tile's first 16) and its exponent
 // buffer.
 struct FsmPlan {
-    uint32_t stage_bytes, exps_bytes, warp_bytes, off_lut, off_warps, total;
+    uint32_t stage_bytes, exps_bytes, warp_bytes, off_ctl, off_lut, off_warps, total;
 };
 
 __host__ __device__ inline FsmPlan make_fsm_plan(int chunk_bits, int nwarp, uint32_t max_span, int fsm_rows) {
@@ -1049,7 +1101,8 @@ __host__ __device__ inline FsmPlan make_fsm_plan(int chunk_bits, int nwarp, uint
     p.stage_bytes = static_cast<uint32_t>(32 * chunk_bits / 8) + 16u + 48u;
     p.exps_bytes = (max_span + 2u * 32u + 16u + 15u) & ~15u;
     p.warp_bytes = (16u + p.stage_bytes + p.exps_bytes + 127u) & ~127u;
-    p.off_lut = static_cast<uint32_t>(fsm_rows) * kFsmRowBytes;
+    p.off_ctl = static_cast<uint32_t>(fsm_rows) * kFsmRowBytes;
+    p.off_lut = p.off_ctl + static_cast<uint32_t>(fsm_rows) * (kFsmRowBytes / 2);
     p.off_warps = up128(p.off_lut + kLutEntries * 2);
     p.total = p.off_warps + static_cast<uint32_t>(nwarp) * p.warp_bytes;
     return p;
@@ -1086,12 +1139,15 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         // tables) is redirected to the dead row so every lookup stays inside
         const uint4 *g = reinterpret_cast<const uint4 *>(P.fsm);
         uint4 *s = reinterpret_cast<uint4 *>(smem);
+        uint2 *sc = reinterpret_cast<uint2 *>(smem + plan.off_ctl);
         const uint32_t lim = static_cast<uint32_t>(rows) << kFsmRowShift;
         for (int i = tid; i < rows * kFsmRowBytes / 16; i += NWARP * 32) {
             uint4 v = __ldg(g + i);
             if ((v.x & kFsmRowMask) >= lim) v.x = (v.x & ~kFsmRowMask) | dead;
             if ((v.z & kFsmRowMask) >= lim) v.z = (v.z & ~kFsmRowMask) | dead;
             s[i] = v;
+            sc[i] = make_uint2((v.x & ~kFsmRowMask) | ((v.x & kFsmRowMask) >> 1),
+                               (v.z & ~kFsmRowMask) | ((v.z & kFsmRowMask) >> 1));
         }
         const uint4 *gl = reinterpret_cast<const uint4 *>(P.lut);
         uint4 *sl = reinterpret_cast<uint4 *>(s_lut);
@@ -1200,8 +1256,9 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
 
         // ---- phase 1: count
         uint32_t ctl;
-        uint32_t cnt = byte_step_walk<CB, false>(w, w2, g & 31, nfull, r, jmax, smem, 0u, dead, ctl);
-        const bool slow = !whole || (ctl & kFsmRowMask) == dead;
+        const uint32_t dead_c = dead >> 1;
+        uint32_t cnt = byte_step_count<CB>(w, w2, g & 31, nfull, r, jmax, smem + plan.off_ctl, dead_c, ctl);
+        const bool slow = !whole || (ctl & kCtlRowMask) == dead_c;
         if (__any_sync(0xFFFFFFFFu, slow)) {
             if (slow) {
                 const int gg[1] = {g}, ee[1] = {E};
@@ -1224,7 +1281,10 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         // ---- phase 2, then the merge
         if (good && span) {
             const uint32_t q = smem_addr(s_exps) + static_cast<uint32_t>(S % GROUP) + incl - cnt;
-            if (!slow) byte_step_walk<CB, true>(w, w2, g, nfull, r, jmax, smem, q, dead, ctl);
+            uint32_t acc = 0, wp = 0, f8 = 0;
+            if (!slow) byte_step_emit<CB>(w, w2, g, nfull, r, jmax, smem, q, acc, wp, f8);
+            __syncwarp();  // every plain store of phase 2 before the OR-ed words
+            if (!slow && f8) asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(wp), "r"(acc) : "memory");
             if (__any_sync(0xFFFFFFFFu, slow)) {
                 if (slow) emit_codes<CW, 1, 0, true>(w, g, E, T, q, err);
             }
