@@ -250,8 +250,9 @@ df11_status df11_decode_ex(const df11_blob *const *blobs, void *const *dst_dev, 
         o.ctas_per_sm = opts->ctas_per_sm;
         o.warps_per_cta = opts->warps_per_cta;
         o.walker = opts->walker;
+        o.max_ctas = opts->max_ctas;
         if (o.chunks_per_thread < 0 || o.ctas_per_sm < 0 || o.warps_per_cta < 0 || o.walker < 0 ||
-            o.walker > DF11_WALKER_BYTE_STEP)
+            o.walker > DF11_WALKER_BYTE_STEP || o.max_ctas < 0)
             return DF11_EINVAL;
     }
     return from_launch(df11::launch_decode(bs, dst_dev, n_blobs, dev_err_flag, o,
@@ -311,8 +312,9 @@ df11_status df11_decode_launch_shape_ex(const df11_blob *const *blobs, int n_blo
         o.ctas_per_sm = opts->ctas_per_sm;
         o.warps_per_cta = opts->warps_per_cta;
         o.walker = opts->walker;
+        o.max_ctas = opts->max_ctas;
         if (o.chunks_per_thread < 0 || o.ctas_per_sm < 0 || o.warps_per_cta < 0 || o.walker < 0 ||
-            o.walker > DF11_WALKER_BYTE_STEP)
+            o.walker > DF11_WALKER_BYTE_STEP || o.max_ctas < 0)
             return DF11_EINVAL;
     }
     df11::LaunchStatus st = df11::decode_launch_shape(bs, n_blobs, o, &sh);

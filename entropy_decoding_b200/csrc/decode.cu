@@ -1034,7 +1034,8 @@ __device__ __forceinline__ uint32_t byte_step_count(const uint32_t (&w)[CB / 32 
 
 // Phase 2: the same walk on the full entries {ctl, syms}, writing the symbols
 // in order from shared-memory byte address `out` on.  Symbols are assembled
-// in a register (acc holds f8 / 8 pending bytes, unused bytes zero) and every
+// in a register (acc holds f8 / 8 pending bytes, starting from acc0, the
+// current content of the word `out` falls in; unused bytes zero) and every
 // completed 32-bit word is stored with one plain store.  The word the range
 // starts in may hold earlier threads' bytes (stored as zeros here) and the
 // word it ends in later threads' bytes: that last, partial word is returned
@@ -1043,11 +1044,11 @@ __device__ __forceinline__ uint32_t byte_step_count(const uint32_t (&w)[CB / 32 
 // thread's bytes.  The buffer is zero outside the words written.
 template <int CB>
 __device__ __forceinline__ void byte_step_emit(const uint32_t (&w)[CB / 32 + 1], uint32_t w2, int g, int nfull,
-                                               int r, int jmax, const uint8_t *tab, uint32_t out, uint32_t &acc,
-                                               uint32_t &wp, uint32_t &f8) {
+                                               int r, int jmax, const uint8_t *tab, uint32_t out, uint32_t acc0,
+                                               uint32_t &acc, uint32_t &wp, uint32_t &f8) {
     constexpr int CW = CB / 32, NFIX = (CB - 32) / 8;
     uint32_t ctl = 0;
-    acc = 0;
+    acc = acc0;
     wp = out & ~3u;
     f8 = (out & 3u) << 3;
 #pragma unroll
@@ -1109,13 +1110,19 @@ __host__ __device__ inline FsmPlan make_fsm_plan(int chunk_bits, int nwarp, uint
 }
 
 // Warp tiles (32 chunks) decoded with the byte-step walk, one CTA of NWARP
-// warps per SM sharing the transition table.  Each warp streams its tiles
-// through one shared-memory stage (lane 0 refills it with the warp's next
-// tile as soon as the current one is in registers, so the copy has a whole
-// tile's decode to land), then runs phase 1, the warp scan, phase 2 and the
-// merge as the window kernel does.  Threads whose walk reaches the dead row,
-// or whose range is cut short by the end of the stream, take the window walk
-// instead (12-bit table read from global memory through L1).
+// warps per SM sharing the transition table.  Each warp decodes a contiguous
+// run of tiles, streaming them through one shared-memory stage (lane 0
+// refills it with the next tile as soon as the current one is in registers,
+// so the copy has a whole tile's decode to land), and runs phase 1, the warp
+// scan, phase 2 and the merge per tile.  Threads whose walk reaches the dead
+// row, or whose range is cut short by the end of the stream, take the window
+// walk instead (12-bit table read from global memory through L1).
+//
+// A tile's last output group usually continues in the next tile.  Its
+// exponents stay at the start of the buffer ("carried") and the next tile of
+// the run, which decodes the rest of the group right after them, merges it
+// as a whole group; a group is stored piecewise only where a run or a tensor
+// begins or ends.
 template <int DT, int CB, int NWARP>
 __global__ void __launch_bounds__(NWARP * 32, 1)
     decode_fsm_kernel(const __grid_constant__ DecodeParams P, const uint32_t max_span, const int) {
@@ -1135,8 +1142,9 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
     const uint32_t dead = static_cast<uint32_t>(rows - 1) << kFsmRowShift;
 
     {
-        // the transition table; a row index past the last row (damaged
-        // tables) is redirected to the dead row so every lookup stays inside
+        // the transition table and its control words; a row index past the
+        // last row (damaged tables) is redirected to the dead row so every
+        // lookup stays inside
         const uint4 *g = reinterpret_cast<const uint4 *>(P.fsm);
         uint4 *s = reinterpret_cast<uint4 *>(smem);
         uint2 *sc = reinterpret_cast<uint2 *>(smem + plan.off_ctl);
@@ -1161,9 +1169,12 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
     }
     __syncthreads();
 
-    const uint32_t stride = gridDim.x * NWARP;
-    const uint32_t first = blockIdx.x * NWARP + warp;
-    int ti_issue = 0, ti_cur = 0;
+    // this warp's run of tiles
+    const uint32_t nwt = gridDim.x * NWARP;
+    const uint32_t per = (P.total_tiles + nwt - 1) / nwt;
+    const uint32_t t_begin = min((blockIdx.x * NWARP + warp) * per, P.total_tiles);
+    const uint32_t t_end = min(t_begin + per, P.total_tiles);
+    int ti_issue = tensor_of(P, t_begin), ti_cur = ti_issue;
     // lane 0: copy tile t's stream slice and gaps into the stage
     auto issue = [&](uint32_t t) {
         ti_issue = tensor_of(P, t, ti_issue);
@@ -1173,15 +1184,30 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         bulk_load(stage, d.stream + static_cast<uint64_t>(lt) * TILE_BYTES, TILE_BYTES + 16u, &full[0]);
         bulk_load(stage + TILE_BYTES + 16u, d.gaps + static_cast<uint64_t>(lt) * 32u, 48u, &full[0]);
     };
-    if (lane == 0 && first < P.total_tiles) issue(first);
-    bool pending = first < P.total_tiles;
+    if (lane == 0 && t_begin < t_end) issue(t_begin);
+    bool pending = t_begin < t_end;
 
     // the window walk of the fallback: 12-bit table in global memory, root
     // hierarchical table in shared memory
     const Tables T{P.meta, P.syms, s_lut, P.lut, 1, P.n_luts};
     uint32_t err = 0;
     uint32_t k = 0;
-    for (uint32_t t = first; t < P.total_tiles; t += stride, ++k) {
+    // carried group: exponents of its elements [0, carry_n) at the buffer start
+    uint32_t carry_n = 0;
+    uint64_t carry_g = 0;
+    int carry_ti = 0;
+    // stores the carried elements alone (lane 0) and clears their exponents
+    auto flush_carry = [&]() {
+        if (lane == 0) {
+            const TensorDesc &dc = P.t[carry_ti];
+            merge_group<DT, true>(ld_global_stream_v4(dc.plane + carry_g * 16u), 0u, s_exps,
+                                  static_cast<uint8_t *>(dc.dst) + carry_g * 32u, 0u, carry_n);
+        }
+        carry_n = 0;
+        __syncwarp();
+    };
+
+    for (uint32_t t = t_begin; t < t_end; ++t, ++k) {
         ti_cur = tensor_of(P, t, ti_cur);
         const TensorDesc &d = P.t[ti_cur];
         const uint32_t lt = t - d.tile_begin;
@@ -1190,10 +1216,14 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         const bool bad = Eo < S || Eo > d.n || Eo - S > max_span;
         if (bad) S = 0;
         const uint32_t span = bad ? 0u : static_cast<uint32_t>(Eo - S);
+        const uint64_t g0 = S / GROUP;
+        const uint32_t s0 = static_cast<uint32_t>(S % GROUP);
+        const uint32_t ng = span ? static_cast<uint32_t>((S + span + GROUP - 1) / GROUP - g0) : 0u;
+        // the carried group goes on in this tile only if the tile starts right after it
+        if (carry_n && !(span && ti_cur == carry_ti && g0 == carry_g && s0 == carry_n)) flush_carry();
+        const bool joined = carry_n != 0;
 
         // the tile's plane span: the first kPrefetchGroups groups of each lane now
-        const uint64_t g0 = S / GROUP;
-        const uint32_t ng = span ? static_cast<uint32_t>((S + span + GROUP - 1) / GROUP - g0) : 0u;
         const uint8_t *plane = d.plane + g0 * 16u;
         uint4 pre[kPrefetchGroups];
 #pragma unroll
@@ -1232,12 +1262,12 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         }
         const int graw = stage[TILE_BYTES + 16u + lane];
         const int gnext = stage[TILE_BYTES + 16u + lane + 1];
-        // the stage is in registers: refill it with the warp's next tile
+        // the stage is in registers: refill it with the run's next tile
         __syncwarp();
-        if (t + stride < P.total_tiles) {
+        if (t + 1 < t_end) {
             if (lane == 0) {
                 fence_proxy_async_smem();
-                issue(t + stride);
+                issue(t + 1);
             }
             pending = true;
         }
@@ -1280,28 +1310,50 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
 
         // ---- phase 2, then the merge
         if (good && span) {
-            const uint32_t q = smem_addr(s_exps) + static_cast<uint32_t>(S % GROUP) + incl - cnt;
+            const uint32_t qrel = s0 + incl - cnt;
+            const uint32_t q = smem_addr(s_exps) + qrel;
+            // the word a range starts in may hold carried exponents: start from it
+            const uint32_t acc0 = joined ? *reinterpret_cast<const uint32_t *>(s_exps + (qrel & ~3u)) : 0u;
+            __syncwarp();
             uint32_t acc = 0, wp = 0, f8 = 0;
-            if (!slow) byte_step_emit<CB>(w, w2, g, nfull, r, jmax, smem, q, acc, wp, f8);
+            if (!slow) byte_step_emit<CB>(w, w2, g, nfull, r, jmax, smem, q, acc0, acc, wp, f8);
             __syncwarp();  // every plain store of phase 2 before the OR-ed words
             if (!slow && f8) asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(wp), "r"(acc) : "memory");
             if (__any_sync(0xFFFFFFFFu, slow)) {
                 if (slow) emit_codes<CW, 1, 0, true>(w, g, E, T, q, err);
             }
             __syncwarp();
+            // groups [0, nmerge): group 0 is whole when it continues the carry
+            // or starts on a group boundary; an unfinished last group becomes
+            // the next carry (unless it is also the unfinished first group)
             uint8_t *dst_tile = static_cast<uint8_t *>(d.dst) + g0 * 32u;
-            const uint32_t lo = static_cast<uint32_t>(S % GROUP), hi = lo + span;
+            const uint32_t lo = joined ? 0u : s0, hi = s0 + span;
+            const bool keep = (hi % GROUP) != 0 && !(ng == 1 && lo != 0);
+            const uint32_t nmerge = keep ? ng - 1 : ng;
 #pragma unroll
             for (int u = 0; u < kPrefetchGroups; ++u) {
                 const uint32_t i = lane + 32u * u;
-                if (i < ng) merge_group<DT, false>(pre[u], i, s_exps, dst_tile, lo, hi);
+                if (i < nmerge) merge_group<DT, true>(pre[u], i, s_exps, dst_tile, lo, hi);
             }
-            for (uint32_t i = lane + 32u * kPrefetchGroups; i < ng; i += 32)
-                merge_group<DT, false>(ld_global_stream_v4(plane + 16u * i), i, s_exps, dst_tile, lo, hi);
-            edge_groups<DT>(pre, plane, ng, s_exps, dst_tile, lo, hi, lane);
+            for (uint32_t i = lane + 32u * kPrefetchGroups; i < nmerge; i += 32)
+                merge_group<DT, true>(ld_global_stream_v4(plane + 16u * i), i, s_exps, dst_tile, lo, hi);
             __syncwarp();
+            if (keep) {
+                if (ng > 1 && lane < static_cast<int>(GROUP / 16u)) {  // move the group's exponents to the start
+                    uint4 *src = reinterpret_cast<uint4 *>(s_exps + GROUP * (ng - 1)) + lane;
+                    reinterpret_cast<uint4 *>(s_exps)[lane] = *src;
+                    *src = make_uint4(0, 0, 0, 0);
+                }
+                carry_n = hi % GROUP;
+                carry_g = g0 + ng - 1;
+                carry_ti = ti_cur;
+                __syncwarp();
+            } else {
+                carry_n = 0;  // a carried group was merged above
+            }
         }
     }
+    if (carry_n) flush_carry();
     // after an abort: wait (bounded) for a copy that was issued but never consumed
     if (pending)
         if (!mbar_wait(&full[0], k & 1u)) err |= DF11_DEV_ERR_TIMEOUT;
@@ -1387,6 +1439,7 @@ struct Prepared {
     uint32_t max_span = 0;
     int n_lut_smem = 0;
     int ctas_per_sm = 0;
+    int max_ctas = 0;
     uint32_t smem = 0;
 };
 
@@ -1467,6 +1520,7 @@ LaunchStatus build_params(const Blob *const *blobs, void *const *dst, int n, int
     out->max_span = static_cast<uint32_t>(max_span);
     out->n_lut_smem = P.n_luts < kSmemLutTables ? P.n_luts : kSmemLutTables;
     out->ctas_per_sm = opt.ctas_per_sm;
+    out->max_ctas = opt.max_ctas;
     if (ke->walker == DF11_WALKER_BYTE_STEP)
         out->smem = make_fsm_plan(b0.chunk_bits, ke->nwarp, out->max_span, rows).total;
     else if (warp_tiles)
@@ -1492,7 +1546,9 @@ LaunchStatus shape_for(const Prepared &pp, LaunchShape *sh) {
     // one CTA per tile (CTA kernel) or per nwarp tiles (warp kernel) at most
     const uint64_t tiles_per_cta = pp.ke->nwarp ? static_cast<uint64_t>(pp.ke->nwarp) : 1u;
     const uint64_t need = (pp.params.total_tiles + tiles_per_cta - 1) / tiles_per_cta;
-    sh->grid = static_cast<int>(want < need ? want : need);
+    uint64_t grid = want < need ? want : need;
+    if (pp.max_ctas > 0 && grid > static_cast<uint64_t>(pp.max_ctas)) grid = static_cast<uint64_t>(pp.max_ctas);
+    sh->grid = static_cast<int>(grid);
     sh->block = block;
     sh->smem = static_cast<int>(pp.smem);
     sh->walker = pp.ke->walker;

@@ -14,6 +14,7 @@ struct DecodeOptions {
     int ctas_per_sm = 0;        // 0 = as many as fit
     int warps_per_cta = 0;      // warp-tile layouts: 0 = kDefaultWarpsPerCta (window) / most that fit (byte step)
     int walker = 0;             // DF11_WALKER_*: 0 = auto
+    int max_ctas = 0;           // grid cap, 0 = none
 };
 
 constexpr int kDefaultChunksPerThread = 1;

@@ -233,6 +233,8 @@ typedef struct {
                                   16 (0 = 16), byte-step walker 16, 24 or 32 (0 = the most that fit) */
     int32_t walker;            /* warp-tile layout: DF11_WALKER_AUTO (0), DF11_WALKER_WINDOW or
                                   DF11_WALKER_BYTE_STEP; CTA-tile layouts take 0 or WINDOW only */
+    int32_t max_ctas;          /* upper bound on the grid (0 = none): fewer persistent CTAs leave
+                                  SMs free for work running beside the decode */
 } df11_decode_opts;
 
 /* How a decoding thread walks its chunk (both give the same output).

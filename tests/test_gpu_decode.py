@@ -153,6 +153,29 @@ def test_batched_block_launch_scaled(df11, oracle_mod):
         assert np.array_equal(out, oracle_mod.decompress(oracle_mod.compress(x, "bf16", lengths=lengths)))
 
 
+@pytest.mark.parametrize("max_ctas", [1, 3])
+@pytest.mark.parametrize("chunk_bits", [64, 128, 256])
+@pytest.mark.parametrize("walker", [1, 2])
+def test_long_runs_across_tensors(df11, oracle_mod, walker, chunk_bits, max_ctas):
+    """A capped grid: every warp of the byte-step kernel decodes a long run of
+    consecutive tiles that crosses tensor boundaries, so unfinished output
+    groups are carried from tile to tile and stored at the ends of runs and
+    tensors.  Tensor sizes are ragged on purpose."""
+    g = synth.transformer_block(1)[0]
+    xs = [t.bits[: t.bits.size // 64 + 13 * i + 5] for i, t in enumerate(g.tensors)]
+    xs.append(synth.random_bits(1, "bf16", 3) & 0x3FFF)  # one weight: a run that ends at once
+    xs.insert(2, g.tensors[0].bits[:31])
+    cb = df11.df11_build_codebook("bf16", xs)
+    blobs = [df11.df11_encode(cb, x, chunk_bits, 32) for x in xs]
+    outs, err, guards = decode_gpu(df11, blobs, walker=walker, warps_per_cta=16, max_ctas=max_ctas)
+    assert err == 0 and guards
+    lengths = cb.lengths()
+    for x, out in zip(xs, outs):
+        assert np.array_equal(out, x)
+    assert np.array_equal(outs[0], oracle_mod.decompress(oracle_mod.compress(xs[0], "bf16", lengths=lengths,
+                                                                             chunk_bits=chunk_bits, tile_threads=32)))
+
+
 def test_mixed_codes_rejected(df11):
     a = synth.single_matrix(0)[0].tensors[0].bits[:5000]
     b = synth.heavy_tail_matrix(0)[0].tensors[0].bits[:5000]
