@@ -453,6 +453,35 @@ __device__ __forceinline__ void merge_group(uint4 p4, uint32_t i, uint8_t *s_exp
     }
 }
 
+// Merges group i of a tile that lies wholly inside it: as merge_group without
+// the piecewise store.
+template <int DT>
+__device__ __forceinline__ void merge_whole(uint4 p4, uint32_t i, uint8_t *s_exps, uint8_t *dst_tile) {
+    uint4 a, b;
+    if constexpr (DT == 0) {
+        uint4 *xp = reinterpret_cast<uint4 *>(s_exps + 16 * i);
+        const uint4 x4 = *xp;
+        *xp = make_uint4(0, 0, 0, 0);
+        merge_bf16x4(p4.x, x4.x, a.x, a.y);
+        merge_bf16x4(p4.y, x4.y, a.z, a.w);
+        merge_bf16x4(p4.z, x4.z, b.x, b.y);
+        merge_bf16x4(p4.w, x4.w, b.z, b.w);
+    } else {
+        uint4 *xp = reinterpret_cast<uint4 *>(s_exps + 32 * i);
+        const uint4 x0 = xp[0];
+        const uint4 x1 = xp[1];
+        xp[0] = make_uint4(0, 0, 0, 0);
+        xp[1] = make_uint4(0, 0, 0, 0);
+        merge_e4m3x8(p4.x, x0.x, x0.y, a.x, a.y);
+        merge_e4m3x8(p4.y, x0.z, x0.w, a.z, a.w);
+        merge_e4m3x8(p4.z, x1.x, x1.y, b.x, b.y);
+        merge_e4m3x8(p4.w, x1.z, x1.w, b.z, b.w);
+    }
+    uint8_t *out = dst_tile + 32u * i;
+    st_global_v4(out, a);
+    st_global_v4(out + 16, b);
+}
+
 // The first and last group of a warp tile can be shared with the neighbouring
 // tile.  The whole warp stores them element by element, one element per lane
 // per pass: the group's 16 plane bytes come from the lane that loaded them
@@ -977,6 +1006,13 @@ __device__ __forceinline__ uint32_t step_off(uint32_t x, int k) {
     return k == 3 ? (x << 3) & 0x7F8u : (x >> (21 - 8 * k)) & 0x7F8u;
 }
 
+// Steps of the byte-step walk taken unconditionally by a chunk: its range is
+// CB + (next gap) - (gap) bits, at least CB - 31 (a gap is below 32), so every
+// chunk with a whole range takes its first (CB - 32) / 8 steps without
+// per-step checks.
+template <int CB>
+constexpr int kFixedSteps = (CB - 32) / 8;
+
 // Entry offset of byte k of x in a row of the compact control array: byte * 4.
 __device__ __forceinline__ uint32_t step_off4(uint32_t x, int k) {
     return k == 3 ? (x << 2) & 0x3FCu : (x >> (22 - 8 * k)) & 0x3FCu;
@@ -991,9 +1027,9 @@ constexpr uint32_t kCtlRowMask = kFsmRowMask >> 1;
 // chunk (or the end of the stream).  Step j looks up byte j of that range in
 // the row of the tree node the previous step stopped on (the root first): the
 // entry lists the codes that end in the byte and the next row.  Steps below
-// NFIX are taken by every thread with a whole chunk (its range is at least
-// CB - 31 bits); the others are predicated on nfull, and the warp stops after
-// its longest range (jmax steps).  A last partial byte (r bits) counts only
+// NFIX are taken by every thread on the byte-step walk (kFixedSteps); the
+// others are predicated on nfull, and the warp stops after its longest range
+// (jmax steps).  A last partial byte (r bits) counts only
 // the codes whose end mask bit falls in its first r bits; those end exactly
 // at the range's end, so the codes of the next chunk are never counted.
 //
@@ -1007,7 +1043,7 @@ template <int CB>
 __device__ __forceinline__ uint32_t byte_step_count(const uint32_t (&w)[CB / 32 + 1], uint32_t w2, int g, int nfull,
                                                     int r, int jmax, const uint8_t *ctl_tab, uint32_t dead,
                                                     uint32_t &ctl_out) {
-    constexpr int CW = CB / 32, NFIX = (CB - 32) / 8;
+    constexpr int CW = CB / 32, NFIX = kFixedSteps<CB>;
     uint32_t ctl = 0, cnt = 0;
 #pragma unroll
     for (int m = 0; m <= CW; ++m) {
@@ -1046,7 +1082,7 @@ template <int CB>
 __device__ __forceinline__ void byte_step_emit(const uint32_t (&w)[CB / 32 + 1], uint32_t w2, int g, int nfull,
                                                int r, int jmax, const uint8_t *tab, uint32_t out, uint32_t acc0,
                                                uint32_t &acc, uint32_t &wp, uint32_t &f8) {
-    constexpr int CW = CB / 32, NFIX = (CB - 32) / 8;
+    constexpr int CW = CB / 32, NFIX = kFixedSteps<CB>;
     uint32_t ctl = 0;
     acc = acc0;
     wp = out & ~3u;
@@ -1127,7 +1163,7 @@ template <int DT, int CB, int NWARP>
 __global__ void __launch_bounds__(NWARP * 32, 1)
     decode_fsm_kernel(const __grid_constant__ DecodeParams P, const uint32_t max_span, const int) {
     constexpr int CW = CB / 32;
-    constexpr int NFIX = (CB - 32) / 8;
+    constexpr int NFIX = kFixedSteps<CB>;
     constexpr uint32_t TILE_BYTES = 32 * CB / 8;
     constexpr uint32_t GROUP = DT == 0 ? 16u : 32u;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -1325,18 +1361,20 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
             __syncwarp();
             // groups [0, nmerge): group 0 is whole when it continues the carry
             // or starts on a group boundary; an unfinished last group becomes
-            // the next carry (unless it is also the unfinished first group)
+            // the next carry (unless it is also the unfinished first group,
+            // the one group that may be stored piecewise)
             uint8_t *dst_tile = static_cast<uint8_t *>(d.dst) + g0 * 32u;
             const uint32_t lo = joined ? 0u : s0, hi = s0 + span;
             const bool keep = (hi % GROUP) != 0 && !(ng == 1 && lo != 0);
             const uint32_t nmerge = keep ? ng - 1 : ng;
+            if (lane < nmerge) merge_group<DT, true>(pre[0], lane, s_exps, dst_tile, lo, hi);
 #pragma unroll
-            for (int u = 0; u < kPrefetchGroups; ++u) {
+            for (int u = 1; u < kPrefetchGroups; ++u) {
                 const uint32_t i = lane + 32u * u;
-                if (i < nmerge) merge_group<DT, true>(pre[u], i, s_exps, dst_tile, lo, hi);
+                if (i < nmerge) merge_whole<DT>(pre[u], i, s_exps, dst_tile);
             }
             for (uint32_t i = lane + 32u * kPrefetchGroups; i < nmerge; i += 32)
-                merge_group<DT, true>(ld_global_stream_v4(plane + 16u * i), i, s_exps, dst_tile, lo, hi);
+                merge_whole<DT>(ld_global_stream_v4(plane + 16u * i), i, s_exps, dst_tile);
             __syncwarp();
             if (keep) {
                 if (ng > 1 && lane < static_cast<int>(GROUP / 16u)) {  // move the group's exponents to the start

@@ -93,17 +93,22 @@ def test_parity_warp_layouts(df11, oracle_mod, layout, case, walk):
     send many; both must still be exact."""
     dt, make = SMALL[case]
     walker, wpc = walk
+    x = make()
     try:
-        _roundtrip(df11, oracle_mod, make(), dt, *layout, wpc=wpc, walker=walker)
+        _roundtrip(df11, oracle_mod, x, dt, *layout, wpc=wpc, walker=walker)
     except df11.Df11Error as e:
-        # the byte-step walk asked for explicitly with a warp count whose
-        # buffers do not fit beside the tables (64-row tables of codes over
-        # all 256 exponents, or 8192-code tiles of 1-bit codes in 256-bit
-        # chunks); the default options fall back to the window walk there
-        if not (walker == 2 and e.status == df11.DF11_EUNSUPPORTED and case in ("single_symbol", "uniform_random",
-                                                                              "all_bf16")):
+        # the byte-step walk asked for with a warp count whose buffers do not
+        # fit beside the tables (64-row tables of codes over all 256
+        # exponents, long tiles of short codes, 256-bit chunks): refused, and
+        # then the library's own warp count, or the automatic walk, must work
+        if not (walker == 2 and e.status == df11.DF11_EUNSUPPORTED):
             raise
-        pytest.skip("shared memory too small for this many warps")
+        try:
+            _roundtrip(df11, oracle_mod, x, dt, *layout, walker=walker)
+        except df11.Df11Error as e2:
+            if e2.status != df11.DF11_EUNSUPPORTED:
+                raise
+            _roundtrip(df11, oracle_mod, x, dt, *layout)
 
 
 @pytest.mark.parametrize("ctas", [1, 2])
@@ -246,7 +251,9 @@ def test_corrupted_device_data_sets_error_flag(df11):
         if what == "out_off":
             assert e & df11.DEV_ERR_AUX
         if what == "fsm":
-            assert e & df11.DEV_ERR_SPAN
+            # a walk that meets a damaged row either falls back to the window
+            # walk (exact output) or miscounts (flagged): never silent
+            assert e & df11.DEV_ERR_SPAN or np.array_equal(g[guard:guard + nbytes].view(np.uint16), x)
         # a shifted gap is caught when it changes the tile's code count; when
         # the parse resynchronises to the same count the output is wrong but
         # still inside the destination, which is what is checked above
