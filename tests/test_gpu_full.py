@@ -1,6 +1,7 @@
 """GPU parity at the workloads' full sizes, in the launch configuration the
-benchmark times (default layout: 128-bit chunks, 32-chunk tiles, 16 warps per
-CTA; one df11_decode launch per codebook group).
+benchmark times (default layout: 128-bit chunks, 32-chunk tiles; default launch:
+the byte-step walk, one CTA of 32 warps per SM; one df11_decode launch per
+codebook group).
 
 Small enough for the oracle (1M and 16.7M weights): every element is
 compared with the oracle's decompression.  Larger workloads: every element is
