@@ -251,8 +251,9 @@ df11_status df11_decode_ex(const df11_blob *const *blobs, void *const *dst_dev, 
         o.warps_per_cta = opts->warps_per_cta;
         o.walker = opts->walker;
         o.max_ctas = opts->max_ctas;
+        o.overlap = opts->overlap;
         if (o.chunks_per_thread < 0 || o.ctas_per_sm < 0 || o.warps_per_cta < 0 || o.walker < 0 ||
-            o.walker > DF11_WALKER_BYTE_STEP || o.max_ctas < 0)
+            o.walker > DF11_WALKER_BYTE_STEP || o.max_ctas < 0 || o.overlap < 0 || o.overlap > 1)
             return DF11_EINVAL;
     }
     return from_launch(df11::launch_decode(bs, dst_dev, n_blobs, dev_err_flag, o,

@@ -107,6 +107,13 @@ __device__ __forceinline__ void consumer_sync(int nthreads) {
     asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }
 
+// Lets a kernel launched after this one with programmatic stream
+// serialization start as soon as SMs free up (no effect otherwise).  Decode
+// launches never consume a previous decode's output, so they trigger at once.
+__device__ __forceinline__ void allow_dependent_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void report(int *err, uint32_t bits) {
     if (err && bits) atomicOr(err, static_cast<int>(bits));
 }
@@ -596,6 +603,7 @@ __global__ void __launch_bounds__(NTH + 32, (NTH + 32) * 3 <= 1024 ? 3 : 1)
         fence_mbar_init();
     }
     __syncthreads();
+    allow_dependent_launch();
 
     uint8_t *const s_stream0 = smem + plan.off_stream;
     uint8_t *const s_gaps0 = smem + plan.off_gaps;
@@ -863,6 +871,7 @@ __global__ void __launch_bounds__(NWARP * 32, NWARP <= 8 ? 4 : 2)
         fence_mbar_init();
     }
     __syncthreads();
+    allow_dependent_launch();
 
     const uint32_t stride = gridDim.x * NWARP;
     const uint32_t first = blockIdx.x * NWARP + warp;
@@ -1204,6 +1213,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         fence_mbar_init();
     }
     __syncthreads();
+    allow_dependent_launch();
 
     // this warp's run of tiles
     const uint32_t nwt = gridDim.x * NWARP;
@@ -1623,7 +1633,22 @@ LaunchStatus launch_decode(const Blob *const *blobs, void *const *dst, int n, in
     LaunchShape sh;
     st = shape_for(pp, &sh);
     if (st != LaunchStatus::kOk) return st;
-    pp.ke->fn<<<sh.grid, sh.block, sh.smem, s>>>(pp.params, pp.max_span, pp.n_lut_smem);
+    if (opt.overlap) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(sh.grid));
+        cfg.blockDim = dim3(static_cast<unsigned>(sh.block));
+        cfg.dynamicSmemBytes = static_cast<size_t>(sh.smem);
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, pp.ke->fn, pp.params, pp.max_span, pp.n_lut_smem) != cudaSuccess)
+            return LaunchStatus::kCuda;
+    } else {
+        pp.ke->fn<<<sh.grid, sh.block, sh.smem, s>>>(pp.params, pp.max_span, pp.n_lut_smem);
+    }
     if (cudaGetLastError() != cudaSuccess) return LaunchStatus::kCuda;
     return LaunchStatus::kOk;
 }

@@ -15,6 +15,7 @@ struct DecodeOptions {
     int warps_per_cta = 0;      // warp-tile layouts: 0 = kDefaultWarpsPerCta (window) / most that fit (byte step)
     int walker = 0;             // DF11_WALKER_*: 0 = auto
     int max_ctas = 0;           // grid cap, 0 = none
+    int overlap = 0;            // 1: programmatic dependent launch (no dependency on earlier stream work)
 };
 
 constexpr int kDefaultChunksPerThread = 1;

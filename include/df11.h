@@ -235,6 +235,10 @@ typedef struct {
                                   DF11_WALKER_BYTE_STEP; CTA-tile layouts take 0 or WINDOW only */
     int32_t max_ctas;          /* upper bound on the grid (0 = none): fewer persistent CTAs leave
                                   SMs free for work running beside the decode */
+    int32_t overlap;           /* 1: the launch reads nothing that the work before it on the
+                                  stream writes, so it may start while the previous kernel is
+                                  still finishing (programmatic dependent launch); 0: ordinary
+                                  stream order */
 } df11_decode_opts;
 
 /* How a decoding thread walks its chunk (both give the same output).

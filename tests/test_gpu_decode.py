@@ -181,6 +181,35 @@ def test_long_runs_across_tensors(df11, oracle_mod, walker, chunk_bits, max_ctas
                                                                              chunk_bits=chunk_bits, tile_threads=32)))
 
 
+def test_overlapped_launches(df11, oracle_mod):
+    """Independent decodes launched back to back with overlap = 1 (each may
+    start while the previous one finishes, programmatic dependent launch) on
+    one stream, both walks and a capped grid among them: every output exact,
+    no error."""
+    s = torch.cuda.Stream()
+    jobs = []
+    for seed, (walker, max_ctas) in enumerate([(0, 0), (1, 0), (2, 5), (0, 2), (2, 0)]):
+        xs = [synth.single_matrix(seed)[0].tensors[0].bits[: 300000 + 7 * seed],
+              synth.heavy_tail_matrix(seed)[0].tensors[0].bits[: 200001]]
+        cb = df11.df11_build_codebook("bf16", xs)
+        blobs = [df11.df11_encode(cb, x) for x in xs]
+        with torch.cuda.stream(s):
+            for b in blobs:
+                df11.upload(b, s)
+        outs = [torch.empty(2 * x.size, dtype=torch.uint8, device="cuda") for x in xs]
+        jobs.append((xs, blobs, outs, walker, max_ctas))
+    s.synchronize()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for xs, blobs, outs, walker, max_ctas in jobs:
+        df11.df11_decode_ex(blobs, [o.data_ptr() for o in outs], err.data_ptr(), s.cuda_stream, walker=walker,
+                            max_ctas=max_ctas, overlap=1)
+    s.synchronize()
+    assert int(err.item()) == 0
+    for xs, blobs, outs, walker, max_ctas in jobs:
+        for x, o in zip(xs, outs):
+            assert np.array_equal(o.cpu().numpy().view(np.uint16), x)
+
+
 def test_mixed_codes_rejected(df11):
     a = synth.single_matrix(0)[0].tensors[0].bits[:5000]
     b = synth.heavy_tail_matrix(0)[0].tensors[0].bits[:5000]
