@@ -56,6 +56,7 @@ def parse_args():
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
+    p.add_argument("--no-encode", action="store_true", help="skip the GPU encoder measurement")
     p.add_argument("--chunk-bits", type=int, default=128)
     p.add_argument("--tile-threads", type=int, default=32)
     p.add_argument("--chunks-per-thread", type=int, default=0, help="decode launch option (0 = library default)")
@@ -243,6 +244,37 @@ def oracle_decode_sample(groups_host, seconds: float):
     return done_w, spent, names
 
 
+def _oracle_decode_task(task):
+    """Worker of oracle_decode_parallel: one whole tensor through the oracle."""
+    import oracle
+    stream, total_bits, lengths, n, plane, dt = task
+    t0 = time.perf_counter()
+    exps = oracle.decode(stream, total_bits, lengths, 0, n)
+    oracle.merge(exps, plane, n, dt)
+    return n, time.perf_counter() - t0
+
+
+def oracle_decode_parallel(groups_host, cores: int):
+    """The same oracle decode on every host core at once: whole tensors, one
+    per task, in a pool of `cores` processes started with spawn.  Returns
+    (weights, wall seconds around the whole map, tensors)."""
+    import multiprocessing as mp
+    import oracle
+    oracle.build()
+    tasks = []
+    for gname, tensors in groups_host:
+        for tname, dt, n, lengths, sec in tensors:
+            nsym = 256 if dt == "bf16" else 16
+            tasks.append((sec["stream"], int(sec["total_bits"]), lengths[:nsym], n, sec["plane"], dt))
+    tasks.sort(key=lambda t: -t[3])  # longest first
+    with mp.get_context("spawn").Pool(cores) as pool:
+        pool.map(_oracle_decode_task, tasks[-1:])  # workers up before the clock starts
+        t0 = time.perf_counter()
+        done = pool.map(_oracle_decode_task, tasks, chunksize=1)
+        wall = time.perf_counter() - t0
+    return sum(d[0] for d in done), wall, len(tasks)
+
+
 # ------------------------------------------------------------------ reference arm
 
 def run_reference(args, rank: int, world: int):
@@ -428,23 +460,26 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         launch_ms = [[e[0].elapsed_time(e[1]) for e in step] for step in ev]
 
     # ---- correctness outside the timed region: error word + sampled positions
-    e = int(err.item())
-    host_out = {}
-    bad = 0
-    for gi, ti, pos, vals in samples:
-        name, blobs, dt, dsts = groups[gi]
-        ptr, o, s = dsts[ti]
-        if dt == "bf16":
-            v = out[o:o + s].view(torch.int16)
-            got = v[torch.from_numpy(pos).to(dev)].cpu().numpy().view(np.uint16)
-        else:
-            got = out[o:o + s][torch.from_numpy(pos).to(dev)].cpu().numpy()
-        bad += int((got != vals).sum())
-    assert e == 0, f"device error word {e}"
-    assert bad == 0, f"{bad} sampled outputs differ from the source weights"
+    def check_samples(what: str):
+        e = int(err.item())
+        bad = 0
+        for gi, ti, pos, vals in samples:
+            name, blobs, dt, dsts = groups[gi]
+            ptr, o, s_ = dsts[ti]
+            if dt == "bf16":
+                v = out[o:o + s_].view(torch.int16)
+                got = v[torch.from_numpy(pos).to(dev)].cpu().numpy().view(np.uint16)
+            else:
+                got = out[o:o + s_][torch.from_numpy(pos).to(dev)].cpu().numpy()
+            bad += int((got != vals).sum())
+        assert e == 0, f"{what}: device error word {e}"
+        assert bad == 0, f"{what}: {bad} sampled outputs differ from the source weights"
+
+    check_samples("decode")
 
     # ---- end to end through the C-ABI with host buffers (pinned)
     e2e = None
+    streamed = None
     if not args.no_e2e:
         himgs = []
         for name, blobs, dt, dsts in groups:
@@ -487,7 +522,47 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         e2e = {"value": job_throughput(out_bytes_total, world, 1, e2e_ms), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                "path": "df11_decode_host: pinned host image -> H2D -> decode launch -> D2H of every output"}
-        del himgs, hout
+        check_samples("e2e")
+
+        # ---- decode of weights kept in host memory (offloaded): images stay in
+        # pinned host memory and stream through device staging slots, each
+        # group's copy overlapping earlier groups' decodes; outputs stay on the
+        # device (where the layers would consume them)
+        slot_cap = max(sum(((b.info().device_bytes + 255) // 256) * 256 for b in blobs) for _, blobs, _, _ in groups)
+        slot_bufs = [torch.empty(slot_cap + 256, dtype=torch.uint8, device=dev) for _ in range(2)]
+        slot_ptrs = [x.data_ptr() + (-x.data_ptr()) % 256 for x in slot_bufs]
+        cstream = torch.cuda.Stream(device=dev)
+        flat_imgs = [h.data_ptr() for hs in himgs for h in hs]
+        flat_dst = [d[0] for _, _, _, dsts in groups for d in dsts]
+        glist = [blobs for _, blobs, _, _ in groups]
+        st_ms = {}
+        for nslots in (2, 1):
+            def streamed_step():
+                df11.df11_decode_streamed(glist, flat_imgs, slot_ptrs[:nslots], slot_cap, flat_dst, err.data_ptr(),
+                                          cstream.cuda_stream, stream.cuda_stream)
+            streamed_step()
+            stream.synchronize()
+            cstream.synchronize()
+            if world > 1:
+                dist.barrier()
+            a0 = torch.cuda.Event(enable_timing=True)
+            a1 = torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            cstream.wait_event(a0)
+            for _ in range(args.e2e_steps):
+                streamed_step()
+            a1.record(stream)
+            a1.synchronize()
+            cstream.synchronize()
+            st_ms[nslots] = max_over_ranks(a0.elapsed_time(a1) / args.e2e_steps, dev)
+        check_samples("streamed")
+        streamed = {"value": job_throughput(out_bytes_total, world, 1, st_ms[2]), "unit": "GB/s",
+                    "ms_per_step": st_ms[2], "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 0, "slots": 2,
+                    "one_slot": {"value": job_throughput(out_bytes_total, world, 1, st_ms[1]), "ms_per_step": st_ms[1]},
+                    "path": "df11_decode_streamed: pinned host images -> device staging slots on a copy stream, "
+                            "decodes on the bench stream, outputs on the device; one_slot = copy and decode "
+                            "in turn"}
+        del himgs, hout, slot_bufs
 
     # ---- CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
@@ -496,6 +571,46 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         cpu = {"value": 2 * w / sec / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
                "sample": f"{w} weights ({len(names)} whole tensors from blocks 0-2, {names[0]} ... {names[-1]}), "
                          f"single-threaded bit-by-bit oracle decode + field merge, {sec:.1f} s"}
+        cores = host_threads(1)
+        if cores > 1:
+            wa, wall, nt = oracle_decode_parallel(host_for_cpu, cores)
+            cpu["all_cores"] = {"value": 2 * wa / wall / 1e9, "unit": "GB/s", "cores": cores,
+                                "weights_per_s": wa / wall,
+                                "sample": f"{wa} weights ({nt} whole tensors of blocks 0-2), one tensor per "
+                                          f"task on {cores} spawned processes, {wall:.1f} s wall"}
+
+    # ---- the GPU encoder on the largest group (histogram, code, packing, aux),
+    # its source being the decoded output (bit-identical to the weights)
+    enc = None
+    if rank == 0 and not args.no_encode:
+        ge = 1 if len(groups) > 2 else big  # a transformer block for the whole model
+        _, blobs_b, dt_b, dsts_b = groups[ge]
+        srcs = [out[o:o + s_].view(torch.int16 if dt_b == "bf16" else torch.uint8) for _, o, s_ in dsts_b]
+        n_b = sum(x.numel() for x in srcs)
+
+        def encode_group():
+            counts = torch.zeros(256, dtype=torch.int64, device=dev)
+            with torch.cuda.stream(stream):
+                for x in srcs:
+                    df11.df11_histogram_device(dt_b, x.data_ptr(), x.numel(), counts.data_ptr(), stream.cuda_stream)
+                nsym = 256 if dt_b == "bf16" else 16
+                cb_g = df11.df11_codebook_from_counts(dt_b, counts.cpu().numpy().view(np.uint64)[:nsym])
+                return [df11.encode_on_device(cb_g, x, args.chunk_bits, args.tile_threads, stream) for x in srcs]
+
+        encode_group()
+        stream.synchronize()
+        t0 = time.perf_counter()
+        reps = 5
+        for _ in range(reps):
+            res = encode_group()
+        stream.synchronize()
+        enc_s = (time.perf_counter() - t0) / reps
+        same = all(r.info().device_bytes == b.info().device_bytes for r, b in zip(res, blobs_b))
+        enc = {"value": n_b * (2 if dt_b == "bf16" else 1) / enc_s / 1e9, "unit": "GB/s of source",
+               "ms": enc_s * 1e3, "weights": n_b, "same_size_as_host_encoding": same,
+               "sample": f"group {groups[ge][0]}: device histogram, host code from the 256 counts, device "
+                         f"bit packing and gap/out_off, one image per tensor; wall clock over {reps} repetitions"}
+        del res
 
     if rank != 0:
         return
@@ -523,6 +638,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": peak_src,
+                     "peak_datasheet": 8000.0, "frac_datasheet": achieved / 8000.0,
                      "kernel": kernel_name(args, cfg, shape),
                      "launch": {"grid": shape[0], "block": shape[1], "smem_bytes": shape[2],
                                 "walker": {1: "window", 2: "byte_step"}.get(shape[3], shape[3])},
@@ -534,7 +650,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                                             "last": float(per_launch[:, -1].mean())},
                      "traffic_source": tsrc},
         "cpu_baseline": cpu,
+        "encode_gpu": enc,
         "e2e": e2e,
+        "streamed_from_host": streamed,
         "gpu_launches": len(groups) * args.steps,
         "clocks": clk,
         "setup_s": setup_s,

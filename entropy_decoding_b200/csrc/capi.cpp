@@ -4,6 +4,7 @@
 #include <cuda_runtime_api.h>
 
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include "df11.h"
@@ -39,6 +40,25 @@ df11_status from_launch(df11::LaunchStatus s) {
         case df11::LaunchStatus::kUnsupported: return DF11_EUNSUPPORTED;
         default: return DF11_ECUDA;
     }
+}
+
+// Events of df11_decode_streamed, created once per device: per slot, "copy
+// done" (recorded on the copy stream) and "slot free" (recorded on the decode
+// stream after the decode that read the slot).
+constexpr int kStreamSlots = 8;
+constexpr int kEventDevices = 64;
+std::mutex g_event_mu;
+cudaEvent_t g_events[kEventDevices][2 * kStreamSlots] = {};
+
+cudaEvent_t *stream_events() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kEventDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(g_event_mu);
+    if (!g_events[dev][0]) {
+        for (int i = 0; i < 2 * kStreamSlots; ++i)
+            if (cudaEventCreateWithFlags(&g_events[dev][i], cudaEventDisableTiming) != cudaSuccess) return nullptr;
+    }
+    return g_events[dev];
 }
 
 }  // namespace
@@ -289,6 +309,59 @@ df11_status df11_decode_host(df11_blob *const *blobs, const void *const *host_im
         const uint64_t bytes = b.dtype == df11::kBF16 ? 2 * b.n : b.n;
         if (bytes && cudaMemcpyAsync(dst_host[i], dst_dev[i], bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
             return DF11_ECUDA;
+    }
+    return DF11_OK;
+}
+
+df11_status df11_decode_streamed(df11_blob *const *blobs, const int32_t *group_sizes, int n_groups,
+                                 const void *const *host_images, void *const *slots, int n_slots,
+                                 uint64_t slot_bytes, void *const *dst_dev, int *dev_err_flag,
+                                 df11_stream copy_stream, df11_stream decode_stream) {
+    if (!blobs || !group_sizes || n_groups < 1 || !host_images || !slots || n_slots < 1 ||
+        n_slots > kStreamSlots || !dst_dev)
+        return DF11_EINVAL;
+    // check every group before enqueueing anything
+    int at = 0;
+    for (int g = 0; g < n_groups; ++g) {
+        const int k = group_sizes[g];
+        if (k < 1 || k > df11::kMaxTensorsPerLaunch) return DF11_EINVAL;
+        uint64_t need = 0;
+        for (int i = at; i < at + k; ++i) {
+            if (!blobs[i] || !host_images[i]) return DF11_EINVAL;
+            need += df11::align_up(df11::image_layout(blobs[i]->b).total, df11::kImageAlign);
+        }
+        if (need > slot_bytes) return DF11_ENOMEM;
+        at += k;
+    }
+    for (int s = 0; s < n_slots; ++s)
+        if (!slots[s] || reinterpret_cast<uintptr_t>(slots[s]) % df11::kImageAlign) return DF11_EINVAL;
+    cudaEvent_t *ev = stream_events();
+    if (!ev) return DF11_ECUDA;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(copy_stream);
+    cudaStream_t ds = reinterpret_cast<cudaStream_t>(decode_stream);
+    at = 0;
+    for (int g = 0; g < n_groups; ++g) {
+        const int s = g % n_slots, k = group_sizes[g];
+        cudaEvent_t copied = ev[2 * s], freed = ev[2 * s + 1];
+        // the slot's previous group has been decoded
+        if (cudaStreamWaitEvent(cs, freed, 0) != cudaSuccess) return DF11_ECUDA;
+        uint8_t *dst = static_cast<uint8_t *>(slots[s]);
+        for (int i = at; i < at + k; ++i) {
+            df11::Blob &b = blobs[i]->b;
+            const uint64_t bytes = df11::image_layout(b).total;
+            if (cudaMemcpyAsync(dst, host_images[i], bytes, cudaMemcpyHostToDevice, cs) != cudaSuccess)
+                return DF11_ECUDA;
+            b.dev_image = dst;
+            b.dev_cap = bytes;
+            dst += df11::align_up(bytes, df11::kImageAlign);
+        }
+        if (cudaEventRecord(copied, cs) != cudaSuccess || cudaStreamWaitEvent(ds, copied, 0) != cudaSuccess)
+            return DF11_ECUDA;
+        const df11_status st = df11_decode(reinterpret_cast<const df11_blob *const *>(blobs + at), dst_dev + at, k,
+                                           dev_err_flag, decode_stream);
+        if (st != DF11_OK) return st;
+        if (cudaEventRecord(freed, ds) != cudaSuccess) return DF11_ECUDA;
+        at += k;
     }
     return DF11_OK;
 }

@@ -94,6 +94,7 @@ _SIGS = {
     "df11_decode_launch_shape_ex": ([_PP, _I, ctypes.POINTER(DecodeOpts), ctypes.POINTER(_I), ctypes.POINTER(_I),
                                      ctypes.POINTER(_I), ctypes.POINTER(_I)], _S),
     "df11_histogram_device": ([_I, _P, _U64, _P, _P], _S),
+    "df11_decode_streamed": ([_PP, _P, _I, _PP, _PP, _I, _U64, _PP, _P, _P, _P], _S),
     "df11_codebook_from_counts": ([_I, _P, _I, _I, _PP], _S),
     "df11_encode_device_scratch_bytes": ([_U64], _U64),
     "df11_encode_device_begin": ([_P, _P, _U64, _I, _I, _P, _U64, _P, ctypes.POINTER(_U64), _PP], _S),
@@ -296,6 +297,18 @@ def df11_decode_launch_shape(blobs, chunks_per_thread: int = 0, ctas_per_sm: int
                                             ctypes.byref(g), ctypes.byref(b), ctypes.byref(s), ctypes.byref(w)),
            "df11_decode_launch_shape")
     return (g.value, b.value, s.value, w.value) if with_walker else (g.value, b.value, s.value)
+
+
+def df11_decode_streamed(groups, host_image_ptrs, slot_ptrs, slot_bytes: int, dst_ptrs,
+                         err_ptr: int | None = None, copy_stream: int = 0, decode_stream: int = 0):
+    """groups: list of lists of blobs (one code per group); host_image_ptrs and
+    dst_ptrs flat, in the same order as the blobs."""
+    blobs = [b for g in groups for b in g]
+    sizes = (ctypes.c_int32 * len(groups))(*[len(g) for g in groups])
+    _check(_lib.df11_decode_streamed(_ptr_array([b.handle.value for b in blobs]), ctypes.cast(sizes, _P), len(groups),
+                                     _ptr_array(host_image_ptrs), _ptr_array(slot_ptrs), len(slot_ptrs), slot_bytes,
+                                     _ptr_array(dst_ptrs), err_ptr or None, copy_stream or None, decode_stream or None),
+           "df11_decode_streamed")
 
 
 def df11_histogram_device(dtype: str, src_ptr: int, n: int, counts_ptr: int, stream: int = 0):

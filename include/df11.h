@@ -269,6 +269,34 @@ df11_status df11_decode_host(df11_blob *const *blobs, const void *const *host_im
                              void *const *dev_images, void *const *dst_dev, void *const *dst_host,
                              int n_blobs, int *dev_err_flag, df11_stream stream);
 
+/* Decode of weights kept in host memory, streamed group by group: the
+ * offloaded-weights case of "70% Size, 100% Accuracy ... (DFloat11)",
+ * Abstract (decompression on the GPU of compressed weights), with the
+ * transfer of the next group overlapping the decode of the current one.
+ *   blobs        n_blobs = sum(group_sizes) blobs, group after group; the
+ *                blobs of one group share one code (as in one df11_decode)
+ *   group_sizes  n_groups counts, each 1..64
+ *   host_images  per blob, its device image (df11_blob_device_image) in
+ *                pinned host memory, unchanged until decode_stream completes
+ *   slots        n_slots (1..8) device staging buffers of slot_bytes each,
+ *                256-byte aligned; group g is copied into slot g % n_slots,
+ *                its images packed at 256-byte boundaries
+ *   dst_dev      per blob, output as in df11_decode
+ *   copy_stream  the host-to-device copies; decode_stream the launches.
+ * Group g's copy waits for the decode that last used its slot; its decode
+ * waits for its copy, so with 2 slots the copy of group g + 1 overlaps the
+ * decode of group g.  Asynchronous; the caller synchronises decode_stream.
+ * On return every blob is bound to its place in its slot (rebind before
+ * decoding it again: the slot is reused).  Allocates no device memory; the
+ * first call on a device creates 2 x 8 CUDA events that live until exit.
+ * Errors: DF11_EINVAL (arguments, group size, mixed codes in a group),
+ * DF11_ENOMEM (a group's images exceed slot_bytes; nothing is enqueued),
+ * DF11_EUNSUPPORTED, DF11_ECUDA (copy, event or launch failure). */
+df11_status df11_decode_streamed(df11_blob *const *blobs, const int32_t *group_sizes, int n_groups,
+                                 const void *const *host_images, void *const *slots, int n_slots,
+                                 uint64_t slot_bytes, void *const *dst_dev, int *dev_err_flag,
+                                 df11_stream copy_stream, df11_stream decode_stream);
+
 /* Launch shape df11_decode would use for these blobs on the current device:
  * grid (persistent CTAs), threads per CTA and dynamic shared memory bytes.
  * Any output pointer may be NULL. */
