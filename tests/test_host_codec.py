@@ -309,6 +309,33 @@ def test_invalid_arguments(df11):
     assert not df11.df11_layout_supported("bf16", 96, 256)
 
 
+def test_decode_argument_checks_need_no_gpu(df11):
+    """Bad launch options and bad streamed-decode arguments are refused
+    before any CUDA call (these run without a GPU)."""
+    x = synth.random_bits(5000, "bf16", 3)
+    cb = df11.df11_build_codebook("bf16", [x])
+    blob = df11.df11_encode(cb, x)
+    for kw in ({"walker": 3}, {"walker": -1}, {"overlap": 2}, {"max_ctas": -1}, {"warps_per_cta": -4},
+               {"chunks_per_thread": -1}):
+        with pytest.raises(df11.Df11Error) as e:
+            df11.df11_decode_ex([blob], [0x1000], None, 0, **kw)
+        assert e.value.status == df11.DF11_EINVAL, kw
+    need = (blob.info().device_bytes + 255) // 256 * 256
+    fake = 0x10000  # never dereferenced: every check below fails first
+    with pytest.raises(df11.Df11Error) as e:  # a group's images do not fit the slot
+        df11.df11_decode_streamed([[blob]], [fake], [fake], need - 256, [fake])
+    assert e.value.status == df11.DF11_ENOMEM
+    with pytest.raises(df11.Df11Error) as e:  # more than 8 slots
+        df11.df11_decode_streamed([[blob]], [fake], [fake] * 9, need, [fake])
+    assert e.value.status == df11.DF11_EINVAL
+    with pytest.raises(df11.Df11Error) as e:  # misaligned slot
+        df11.df11_decode_streamed([[blob]], [fake], [fake + 16], need, [fake])
+    assert e.value.status == df11.DF11_EINVAL
+    with pytest.raises(df11.Df11Error) as e:  # more than 64 blobs in a group
+        df11.df11_decode_streamed([[blob] * 65], [fake] * 65, [fake], need * 65, [fake] * 65)
+    assert e.value.status == df11.DF11_EINVAL
+
+
 def test_device_image_layout(df11):
     x = synth.random_bits(300000, "bf16", 9)
     cb = df11.df11_build_codebook("bf16", [x])
@@ -317,8 +344,13 @@ def test_device_image_layout(df11):
     lay = _image_layout(img.tobytes()[:256])
     info = blob.info()
     assert lay["total"] == info.device_bytes == img.size
-    for k in ("meta", "syms", "lut", "gaps", "out_off", "stream", "plane"):
+    for k in ("meta", "syms", "lut", "fsm", "gaps", "out_off", "stream", "plane"):
         assert lay[k] % 256 == 0
+    assert lay["gaps"] - lay["fsm"] >= lay["fsm_rows"] * 2048
+    # the gaps section keeps 16 zero bytes after the last tile's gaps
+    ng = info.n_tiles * info.tile_threads
+    assert lay["out_off"] - lay["gaps"] >= ng + 16
+    assert not img[lay["gaps"] + ng: lay["gaps"] + ng + 16].any()
     s = blob.sections()
     tile_bytes = info.chunk_bits // 8 * info.tile_threads
     stream = img[lay["stream"]:lay["plane"]]
