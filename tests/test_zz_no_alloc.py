@@ -152,6 +152,8 @@ def test_uncovered_symbol_then_clean_call(df11):
 def test_empty_input(df11):
     cb = df11.df11_build_codebook("bf16", [synth.random_bits(100, "bf16")])
     src = torch.zeros(8, dtype=torch.int16, device="cuda")
-    buf, ptr, _ = _aligned(1 << 16)
-    r = df11.df11_encode_device_noalloc(cb, src.data_ptr(), 0, 128, 32, ptr, 1 << 16)
+    need = df11.df11_encode(cb, np.zeros(0, np.uint16)).info().device_bytes  # header and decode tables
+    buf, ptr, _ = _aligned(need)
+    r = df11.df11_encode_device_noalloc(cb, src.data_ptr(), 0, 128, 32, ptr, need)
     assert r.n_tiles == 0 and r.total_bits == 0 and r.max_span == 0
+    assert r.image_bytes == need
