@@ -460,35 +460,6 @@ __device__ __forceinline__ void merge_group(uint4 p4, uint32_t i, uint8_t *s_exp
     }
 }
 
-// Merges group i of a tile that lies wholly inside it: as merge_group without
-// the piecewise store.
-template <int DT>
-__device__ __forceinline__ void merge_whole(uint4 p4, uint32_t i, uint8_t *s_exps, uint8_t *dst_tile) {
-    uint4 a, b;
-    if constexpr (DT == 0) {
-        uint4 *xp = reinterpret_cast<uint4 *>(s_exps + 16 * i);
-        const uint4 x4 = *xp;
-        *xp = make_uint4(0, 0, 0, 0);
-        merge_bf16x4(p4.x, x4.x, a.x, a.y);
-        merge_bf16x4(p4.y, x4.y, a.z, a.w);
-        merge_bf16x4(p4.z, x4.z, b.x, b.y);
-        merge_bf16x4(p4.w, x4.w, b.z, b.w);
-    } else {
-        uint4 *xp = reinterpret_cast<uint4 *>(s_exps + 32 * i);
-        const uint4 x0 = xp[0];
-        const uint4 x1 = xp[1];
-        xp[0] = make_uint4(0, 0, 0, 0);
-        xp[1] = make_uint4(0, 0, 0, 0);
-        merge_e4m3x8(p4.x, x0.x, x0.y, a.x, a.y);
-        merge_e4m3x8(p4.y, x0.z, x0.w, a.z, a.w);
-        merge_e4m3x8(p4.z, x1.x, x1.y, b.x, b.y);
-        merge_e4m3x8(p4.w, x1.z, x1.w, b.z, b.w);
-    }
-    uint8_t *out = dst_tile + 32u * i;
-    st_global_v4(out, a);
-    st_global_v4(out + 16, b);
-}
-
 // The first and last group of a warp tile can be shared with the neighbouring
 // tile.  The whole warp stores them element by element, one element per lane
 // per pass: the group's 16 plane bytes come from the lane that loaded them
@@ -542,6 +513,57 @@ __device__ __forceinline__ void edge_groups(const uint4 (&pre)[kPrefetchGroups],
             }
         }
     }
+}
+
+// Output half-groups: half j of a tile covers output bytes [16j, 16j + 16),
+// plane bytes [8j, 8j + 8) and 8 (BF16) or 16 (E4M3) exponents.  Lane L of
+// store round r takes half 32r + L, so each 16-byte store instruction of the
+// warp writes 512 contiguous bytes.
+__device__ __forceinline__ uint2 ld_global_stream_v2(const void *p) {
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return v;
+}
+
+template <int DT>
+__device__ __noinline__ void store_partial_half(uint8_t *out, uint4 a, uint32_t e0, uint32_t lo, uint32_t hi) {
+    const uint32_t wv[4] = {a.x, a.y, a.z, a.w};
+    if constexpr (DT == 0) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (e0 + j >= lo && e0 + j < hi)
+                reinterpret_cast<uint16_t *>(out)[j] = static_cast<uint16_t>(wv[j >> 1] >> (16 * (j & 1)));
+    } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (e0 + j >= lo && e0 + j < hi) out[j] = static_cast<uint8_t>(wv[j >> 2] >> (8 * (j & 3)));
+    }
+}
+
+template <int DT, bool PARTIAL>
+__device__ __forceinline__ void merge_half(uint2 p2, uint32_t j, uint8_t *s_exps, uint8_t *dst_tile, uint32_t lo,
+                                           uint32_t hi) {
+    uint4 a;
+    uint32_t e0;
+    if constexpr (DT == 0) {
+        uint2 *xp = reinterpret_cast<uint2 *>(s_exps + 8 * j);
+        const uint2 x2 = *xp;
+        *xp = make_uint2(0, 0);
+        merge_bf16x4(p2.x, x2.x, a.x, a.y);
+        merge_bf16x4(p2.y, x2.y, a.z, a.w);
+        e0 = 8u * j;
+    } else {
+        uint4 *xp = reinterpret_cast<uint4 *>(s_exps + 16 * j);
+        const uint4 x4 = *xp;
+        *xp = make_uint4(0, 0, 0, 0);
+        merge_e4m3x8(p2.x, x4.x, x4.y, a.x, a.y);
+        merge_e4m3x8(p2.y, x4.z, x4.w, a.z, a.w);
+        e0 = 16u * j;
+    }
+    uint8_t *out = dst_tile + 16u * j;
+    constexpr uint32_t HALF = DT == 0 ? 8u : 16u;
+    if (!PARTIAL || (e0 >= lo && e0 + HALF <= hi)) st_global_v4(out, a);
+    else store_partial_half<DT>(out, a, e0, lo, hi);
 }
 
 // ------------------------------------------------------------------ kernel
@@ -1271,11 +1293,11 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
 
         // the tile's plane span: the first kPrefetchGroups groups of each lane now
         const uint8_t *plane = d.plane + g0 * 16u;
-        uint4 pre[kPrefetchGroups];
+        uint2 pre[2 * kPrefetchGroups];
 #pragma unroll
-        for (int u = 0; u < kPrefetchGroups; ++u) {
-            const uint32_t i = lane + 32u * u;
-            if (i < ng) pre[u] = ld_global_stream_v4(plane + 16u * i);
+        for (int u = 0; u < 2 * kPrefetchGroups; ++u) {
+            const uint32_t j = lane + 32u * u;
+            if (j < 2 * ng) pre[u] = ld_global_stream_v2(plane + 8u * j);
         }
 
         const bool landed = __all_sync(0xFFFFFFFFu, mbar_wait(&full[0], k & 1u));
@@ -1377,14 +1399,15 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
             const uint32_t lo = joined ? 0u : s0, hi = s0 + span;
             const bool keep = (hi % GROUP) != 0 && !(ng == 1 && lo != 0);
             const uint32_t nmerge = keep ? ng - 1 : ng;
-            if (lane < nmerge) merge_group<DT, true>(pre[0], lane, s_exps, dst_tile, lo, hi);
+            const uint32_t nh = 2u * nmerge;
+            if (static_cast<uint32_t>(lane) < nh) merge_half<DT, true>(pre[0], lane, s_exps, dst_tile, lo, hi);
 #pragma unroll
-            for (int u = 1; u < kPrefetchGroups; ++u) {
-                const uint32_t i = lane + 32u * u;
-                if (i < nmerge) merge_whole<DT>(pre[u], i, s_exps, dst_tile);
+            for (int u = 1; u < 2 * kPrefetchGroups; ++u) {
+                const uint32_t j = lane + 32u * u;
+                if (j < nh) merge_half<DT, false>(pre[u], j, s_exps, dst_tile, lo, hi);
             }
-            for (uint32_t i = lane + 32u * kPrefetchGroups; i < nmerge; i += 32)
-                merge_whole<DT>(ld_global_stream_v4(plane + 16u * i), i, s_exps, dst_tile);
+            for (uint32_t j = lane + 64u * kPrefetchGroups; j < nh; j += 32)
+                merge_half<DT, false>(ld_global_stream_v2(plane + 8u * j), j, s_exps, dst_tile, lo, hi);
             __syncwarp();
             if (keep) {
                 if (ng > 1 && lane < static_cast<int>(GROUP / 16u)) {  // move the group's exponents to the start
