@@ -81,14 +81,14 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
-
-// Waits for the phase of `parity` to complete; false after kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+// Waits for the phase of `parity` to complete; false after limit_ns (the
+// launch's DecodeParams::wait_ns: 2 s, or 10 ms when its waits are made to
+// run out on purpose).
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     while (!mbar_try_wait(bar, parity)) {
-        if (global_ns() - t0 > kWaitLimitNs) return false;
+        if (global_ns() - t0 > limit_ns) return false;
     }
     return true;
 }
@@ -634,12 +634,12 @@ __global__ void __launch_bounds__(NTH + 32, (NTH + 32) * 3 <= 1024 ? 3 : 1)
 
     if (warp == NW) {
         // ---------------- producer warp: one lane issues every copy
-        if (lane != 0) return;
+        if (lane != 0 || P.expire) return;
         uint32_t k = 0, armed = 0, last_parity = 0;
         for (uint32_t t = blockIdx.x; t < P.total_tiles; t += gridDim.x, ++k) {
             const int s = static_cast<int>(k % kStreamStages);
             const uint32_t ph = (k / kStreamStages) & 1u;
-            if (!mbar_wait(&empty_s[s], ph ^ 1u)) {
+            if (!mbar_wait(&empty_s[s], ph ^ 1u, P.wait_ns)) {
                 report(P.err, DF11_DEV_ERR_TIMEOUT);
                 break;
             }
@@ -678,7 +678,7 @@ __global__ void __launch_bounds__(NTH + 32, (NTH + 32) * 3 <= 1024 ? 3 : 1)
         // keep the CTA alive until every copy it issued has landed
         for (int s = 0; s < kStreamStages; ++s)
             if (armed & (1u << s))
-                if (!mbar_wait(&full_s[s], (last_parity >> s) & 1u)) report(P.err, DF11_DEV_ERR_TIMEOUT);
+                if (!mbar_wait(&full_s[s], (last_parity >> s) & 1u, P.wait_ns)) report(P.err, DF11_DEV_ERR_TIMEOUT);
         return;
     }
 
@@ -689,7 +689,7 @@ __global__ void __launch_bounds__(NTH + 32, (NTH + 32) * 3 <= 1024 ? 3 : 1)
     for (uint32_t t = blockIdx.x; t < P.total_tiles; t += gridDim.x, ++k) {
         const int s = static_cast<int>(k % kStreamStages);
         const uint32_t ph = (k / kStreamStages) & 1u;
-        const bool landed = mbar_wait(&full_s[s], ph);
+        const bool landed = mbar_wait(&full_s[s], ph, P.wait_ns);
         const StageMeta m = smeta[s];
         const int ti = landed && m.tensor < static_cast<uint32_t>(P.n_tensors) ? static_cast<int>(m.tensor) : 0;
         const TensorDesc &d = P.t[ti];
@@ -910,12 +910,14 @@ __global__ void __launch_bounds__(NWARP * 32, NWARP <= 8 ? 4 : 2)
         bulk_load(st, d.stream + static_cast<uint64_t>(lt) * TILE_BYTES, TILE_BYTES + 16u, &full[s]);
         bulk_load(st + TILE_BYTES + 16u, d.gaps + static_cast<uint64_t>(lt) * 32u, 32u, &full[s]);
     };
-    if (lane == 0) {
-        if (first < P.total_tiles) issue(first, 0);
-        if (first + stride < P.total_tiles) issue(first + stride, 1);
+    if (!P.expire) {
+        if (lane == 0) {
+            if (first < P.total_tiles) issue(first, 0);
+            if (first + stride < P.total_tiles) issue(first + stride, 1);
+        }
+        if (first < P.total_tiles) issued |= 1u;
+        if (first + stride < P.total_tiles) issued |= 2u;
     }
-    if (first < P.total_tiles) issued |= 1u;
-    if (first + stride < P.total_tiles) issued |= 2u;
 
     const Tables T{s_meta, s_syms, s_lut, P.lut, n_lut_smem, P.n_luts};
     uint32_t err = 0;
@@ -943,7 +945,7 @@ __global__ void __launch_bounds__(NWARP * 32, NWARP <= 8 ? 4 : 2)
             if (i < ng) pre[u] = ld_global_stream_v4(plane + 16u * i);
         }
 
-        const bool landed = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], ph));
+        const bool landed = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], ph, P.wait_ns));
         if (!landed) {
             err |= DF11_DEV_ERR_TIMEOUT;
             break;
@@ -1024,7 +1026,7 @@ __global__ void __launch_bounds__(NWARP * 32, NWARP <= 8 ? 4 : 2)
     // after an abort: wait (bounded) for copies that were issued but never consumed
     for (int s = 0; s < 2; ++s)
         if (issued & (1u << s))
-            if (!mbar_wait(&full[s], (par >> s) & 1u)) err |= DF11_DEV_ERR_TIMEOUT;
+            if (!mbar_wait(&full[s], (par >> s) & 1u, P.wait_ns)) err |= DF11_DEV_ERR_TIMEOUT;
     err = __reduce_or_sync(0xFFFFFFFFu, err);
     if (lane == 0) report(P.err, err);
 }
@@ -1252,8 +1254,8 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         bulk_load(stage, d.stream + static_cast<uint64_t>(lt) * TILE_BYTES, TILE_BYTES + 16u, &full[0]);
         bulk_load(stage + TILE_BYTES + 16u, d.gaps + static_cast<uint64_t>(lt) * 32u, 48u, &full[0]);
     };
-    if (lane == 0 && t_begin < t_end) issue(t_begin);
-    bool pending = t_begin < t_end;
+    if (lane == 0 && t_begin < t_end && !P.expire) issue(t_begin);
+    bool pending = t_begin < t_end && !P.expire;
 
     // the window walk of the fallback: 12-bit table in global memory, root
     // hierarchical table in shared memory
@@ -1300,7 +1302,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
             if (j < 2 * ng) pre[u] = ld_global_stream_v2(plane + 8u * j);
         }
 
-        const bool landed = __all_sync(0xFFFFFFFFu, mbar_wait(&full[0], k & 1u));
+        const bool landed = __all_sync(0xFFFFFFFFu, mbar_wait(&full[0], k & 1u, P.wait_ns));
         if (!landed) {
             err |= DF11_DEV_ERR_TIMEOUT;
             break;
@@ -1427,7 +1429,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
     if (carry_n) flush_carry();
     // after an abort: wait (bounded) for a copy that was issued but never consumed
     if (pending)
-        if (!mbar_wait(&full[0], k & 1u)) err |= DF11_DEV_ERR_TIMEOUT;
+        if (!mbar_wait(&full[0], k & 1u, P.wait_ns)) err |= DF11_DEV_ERR_TIMEOUT;
     err = __reduce_or_sync(0xFFFFFFFFu, err);
     if (lane == 0) report(P.err, err);
 }
@@ -1582,6 +1584,8 @@ LaunchStatus build_params(const Blob *const *blobs, void *const *dst, int n, int
     P.lut = reinterpret_cast<const uint16_t *>(b0.dev_image + L0.lut);
     P.fsm = reinterpret_cast<const uint32_t *>(b0.dev_image + L0.fsm);
     P.fsm_rows = rows;
+    P.expire = opt.diag_expire_waits ? 1 : 0;
+    P.wait_ns = opt.diag_expire_waits ? 10000000ull : 2000000000ull;
     P.err = err;
     P.n_luts = b0.cb->n_luts();
     P.n_tensors = nt;

@@ -104,7 +104,8 @@ struct DecodeParams {
     const uint16_t *lut;
     const uint32_t *fsm;  // fsm_rows * kFsmRowBytes bytes
     int32_t fsm_rows;
-    int32_t pad;
+    int32_t expire;    // diagnostics: issue no copies, so every wait runs out after wait_ns
+    uint64_t wait_ns;  // limit of every mbarrier wait
     int *err;
     int32_t n_luts;
     int32_t n_tensors;

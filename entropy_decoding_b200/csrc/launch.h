@@ -16,6 +16,7 @@ struct DecodeOptions {
     int walker = 0;             // DF11_WALKER_*: 0 = auto
     int max_ctas = 0;           // grid cap, 0 = none
     int overlap = 0;            // 1: programmatic dependent launch (no dependency on earlier stream work)
+    int diag_expire_waits = 0;  // diagnostics: no copies, every wait runs out after 10 ms
 };
 
 constexpr int kDefaultChunksPerThread = 1;

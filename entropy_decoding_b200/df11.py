@@ -58,7 +58,7 @@ class EncodeResult(ctypes.Structure):
 class DecodeOpts(ctypes.Structure):
     _fields_ = [("chunks_per_thread", ctypes.c_int32), ("ctas_per_sm", ctypes.c_int32),
                 ("warps_per_cta", ctypes.c_int32), ("walker", ctypes.c_int32), ("max_ctas", ctypes.c_int32),
-                ("overlap", ctypes.c_int32)]
+                ("overlap", ctypes.c_int32), ("diag_expire_waits", ctypes.c_int32)]
 
 
 WALKER_AUTO, WALKER_WINDOW, WALKER_BYTE_STEP = 0, 1, 2
@@ -273,8 +273,8 @@ def df11_decode(blobs, dst_ptrs, err_ptr: int | None = None, stream: int = 0):
 
 def df11_decode_ex(blobs, dst_ptrs, err_ptr: int | None = None, stream: int = 0, chunks_per_thread: int = 0,
                    ctas_per_sm: int = 0, warps_per_cta: int = 0, walker: int = 0, max_ctas: int = 0,
-                   overlap: int = 0):
-    o = DecodeOpts(chunks_per_thread, ctas_per_sm, warps_per_cta, walker, max_ctas, overlap)
+                   overlap: int = 0, diag_expire_waits: int = 0):
+    o = DecodeOpts(chunks_per_thread, ctas_per_sm, warps_per_cta, walker, max_ctas, overlap, diag_expire_waits)
     _check(_lib.df11_decode_ex(_ptr_array([b.handle.value for b in blobs]), _ptr_array(dst_ptrs), len(blobs),
                                err_ptr or None, stream or None, ctypes.byref(o)), "df11_decode_ex")
 
@@ -292,7 +292,7 @@ def df11_decode_launch_shape(blobs, chunks_per_thread: int = 0, ctas_per_sm: int
     """(grid, block, shared-memory bytes) of the launch df11_decode_ex would
     make with these options, plus the walk it would use when with_walker."""
     g, b, s, w = _I(), _I(), _I(), _I()
-    o = DecodeOpts(chunks_per_thread, ctas_per_sm, warps_per_cta, walker, max_ctas, 0)
+    o = DecodeOpts(chunks_per_thread, ctas_per_sm, warps_per_cta, walker, max_ctas, 0, 0)
     _check(_lib.df11_decode_launch_shape_ex(_ptr_array([x.handle.value for x in blobs]), len(blobs), ctypes.byref(o),
                                             ctypes.byref(g), ctypes.byref(b), ctypes.byref(s), ctypes.byref(w)),
            "df11_decode_launch_shape")

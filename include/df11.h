@@ -239,6 +239,11 @@ typedef struct {
                                   stream writes, so it may start while the previous kernel is
                                   still finishing (programmatic dependent launch); 0: ordinary
                                   stream order */
+    int32_t diag_expire_waits; /* diagnostics, 0 in normal use.  1: the kernel issues no copies
+                                  and gives each of its bounded waits 10 ms instead of 2 s, so
+                                  the first wait runs out: the launch decodes nothing, sets
+                                  DF11_DEV_ERR_TIMEOUT in dev_err_flag and ends (how a stalled
+                                  copy is reported, exercised without a fault) */
 } df11_decode_opts;
 
 /* How a decoding thread walks its chunk (both give the same output).

@@ -210,6 +210,33 @@ def test_overlapped_launches(df11, oracle_mod):
             assert np.array_equal(o.cpu().numpy().view(np.uint16), x)
 
 
+@pytest.mark.parametrize("layout_walker", [((128, 32), 2), ((128, 32), 1), ((128, 256), 0)])
+def test_bounded_wait_runs_out_and_reports(df11, layout_walker):
+    """With diag_expire_waits the kernel issues no copy and each bounded
+    wait gets 10 ms: the first one runs out, the launch writes nothing and
+    reports DF11_DEV_ERR_TIMEOUT, and the context stays usable (the next,
+    normal decode is exact).  Byte-step, window and CTA-tile kernels."""
+    import time
+    (chunk_bits, tile_threads), walker = layout_walker
+    x = synth.single_matrix(3)[0].tensors[0].bits
+    blob = df11.df11_encode(df11.df11_build_codebook("bf16", [x]), x, chunk_bits, tile_threads)
+    df11.upload(blob)
+    torch.cuda.synchronize()
+    out = torch.full((2 * x.size,), 0xA5, dtype=torch.uint8, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t0 = time.time()
+    df11.df11_decode_ex([blob], [out.data_ptr()], err.data_ptr(), walker=walker, diag_expire_waits=1)
+    torch.cuda.synchronize()
+    assert time.time() - t0 < 5.0
+    assert int(err.item()) & df11.DEV_ERR_TIMEOUT
+    assert (out.cpu().numpy() == 0xA5).all()
+    err.zero_()
+    df11.df11_decode_ex([blob], [out.data_ptr()], err.data_ptr(), walker=walker)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert np.array_equal(out.cpu().numpy().view(np.uint16), x)
+
+
 def test_mixed_codes_rejected(df11):
     a = synth.single_matrix(0)[0].tensors[0].bits[:5000]
     b = synth.heavy_tail_matrix(0)[0].tensors[0].bits[:5000]

@@ -316,7 +316,7 @@ def test_decode_argument_checks_need_no_gpu(df11):
     cb = df11.df11_build_codebook("bf16", [x])
     blob = df11.df11_encode(cb, x)
     for kw in ({"walker": 3}, {"walker": -1}, {"overlap": 2}, {"max_ctas": -1}, {"warps_per_cta": -4},
-               {"chunks_per_thread": -1}):
+               {"chunks_per_thread": -1}, {"diag_expire_waits": 2}):
         with pytest.raises(df11.Df11Error) as e:
             df11.df11_decode_ex([blob], [0x1000], None, 0, **kw)
         assert e.value.status == df11.DF11_EINVAL, kw
