@@ -1067,8 +1067,10 @@ constexpr uint32_t kCtlRowMask = kFsmRowMask >> 1;
 // at the range's end, so the codes of the next chunk are never counted.
 //
 // Phase 1 (byte_step_count) walks the compact control words (4 bytes per
-// entry, so a warp's random lookups spread over all 32 banks) and returns the
-// number of codes; ctl_out receives the last control word, whose row is the
+// entry, so a warp's random lookups spread over all 32 banks: end mask in
+// bits 0..7, row << 10, codes ended << 24, so adding whole words counts the
+// codes while the lower fields of at most 20 steps stay below bit 24) and
+// returns the number of codes; ctl_out receives the last control word, whose row is the
 // dead row (`dead`, in control-word form) when the walk left the tables or the
 // partial byte ends more than the 4 codes an entry holds (possible only with
 // a 1-bit codeword).
@@ -1089,16 +1091,16 @@ __device__ __forceinline__ uint32_t byte_step_count(const uint32_t (&w)[CB / 32 
             const uint32_t e = *reinterpret_cast<const uint32_t *>(ctl_tab + ((ctl & kCtlRowMask) | step_off4(x, k)));
             if (j < NFIX || j < nfull) {
                 ctl = e;
-                cnt += e >> kFsmCountShift;
+                cnt += e;  // the count field at bit 24 gathers the codes; the fields below it never carry into it
             } else if (j == nfull) {
                 const uint32_t c = static_cast<uint32_t>(__popc(e & ((1u << r) - 1u)));
-                cnt += c;
+                cnt += c << 24;
                 if (c > 4) ctl = dead;
             }
         }
     }
     ctl_out = ctl;
-    return cnt;
+    return cnt >> 24;
 }
 
 // Phase 2: the same walk on the full entries {ctl, syms}, writing the symbols
@@ -1157,8 +1159,8 @@ __device__ __forceinline__ void byte_step_emit(const uint32_t (&w)[CB / 32 + 1],
 }
 
 // Shared memory of the byte-step kernel: the transition table (fsm_rows rows
-// of kFsmRowBytes) at offset 0, its control words alone (rows of 1 KB, row
-// field at bit 10), the root hierarchical table, then per warp
+// of kFsmRowBytes) at offset 0, its control words alone (rows of 1 KB: end
+// mask, row << 10, count << 24), the root hierarchical table, then per warp
 // its mbarrier, one stage (the tile's 32 chunks + 16 look-ahead bytes, then
 // 48 gap bytes: its own 32 and the next tile's first 16) and its exponent
 // buffer.
@@ -1223,8 +1225,8 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
             if ((v.x & kFsmRowMask) >= lim) v.x = (v.x & ~kFsmRowMask) | dead;
             if ((v.z & kFsmRowMask) >= lim) v.z = (v.z & ~kFsmRowMask) | dead;
             s[i] = v;
-            sc[i] = make_uint2((v.x & ~kFsmRowMask) | ((v.x & kFsmRowMask) >> 1),
-                               (v.z & ~kFsmRowMask) | ((v.z & kFsmRowMask) >> 1));
+            sc[i] = make_uint2((v.x & 0xFFu) | ((v.x & kFsmRowMask) >> 1) | ((v.x >> kFsmCountShift) << 24),
+                               (v.z & 0xFFu) | ((v.z & kFsmRowMask) >> 1) | ((v.z >> kFsmCountShift) << 24));
         }
         const uint4 *gl = reinterpret_cast<const uint4 *>(P.lut);
         uint4 *sl = reinterpret_cast<uint4 *>(s_lut);
