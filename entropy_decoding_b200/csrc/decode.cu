@@ -1033,12 +1033,6 @@ __global__ void __launch_bounds__(NWARP * 32, NWARP <= 8 ? 4 : 2)
 
 // ------------------------------------------------------------------ byte-step kernel
 
-// Entry offset within a transition-table row of byte k (0 = earliest) of the
-// 32 stream bits x (earliest bit in bit 31): byte * 8.
-__device__ __forceinline__ uint32_t step_off(uint32_t x, int k) {
-    return k == 3 ? (x << 3) & 0x7F8u : (x >> (21 - 8 * k)) & 0x7F8u;
-}
-
 // Steps of the byte-step walk taken unconditionally by a chunk: its range is
 // CB + (next gap) - (gap) bits, at least CB - 31 (a gap is below 32), so every
 // chunk with a whole range takes its first (CB - 32) / 8 steps without
@@ -1046,9 +1040,14 @@ __device__ __forceinline__ uint32_t step_off(uint32_t x, int k) {
 template <int CB>
 constexpr int kFixedSteps = (CB - 32) / 8;
 
-// Entry offset of byte k of x in a row of the compact control array: byte * 4.
-__device__ __forceinline__ uint32_t step_off4(uint32_t x, int k) {
-    return k == 3 ? (x << 2) & 0x3FCu : (x >> (22 - 8 * k)) & 0x3FCu;
+// Row base + byte k of x times the entry size, as a byte permute and a
+// multiply-add (the multiply-add issues on the FMA pipe).
+template <uint32_t ENTRY>
+__device__ __forceinline__ uint32_t step_addr(uint32_t x, int k, uint32_t base) {
+    const uint32_t b = __byte_perm(x, 0u, 0x4440u + static_cast<uint32_t>(3 - k));
+    uint32_t a;
+    asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(a) : "r"(b), "n"(ENTRY), "r"(base));
+    return a;
 }
 
 // Row field of the compact control words (row << 10: rows of 1 KB).
@@ -1088,7 +1087,7 @@ __device__ __forceinline__ uint32_t byte_step_count(const uint32_t (&w)[CB / 32 
         for (int k = 0; k < 4; ++k) {
             const int j = 4 * m + k;
             if (j >= NFIX && j >= jmax) break;
-            const uint32_t e = *reinterpret_cast<const uint32_t *>(ctl_tab + ((ctl & kCtlRowMask) | step_off4(x, k)));
+            const uint32_t e = *reinterpret_cast<const uint32_t *>(ctl_tab + step_addr<4>(x, k, ctl & kCtlRowMask));
             if (j < NFIX || j < nfull) {
                 ctl = e;
                 cnt += e;  // the count field at bit 24 gathers the codes; the fields below it never carry into it
@@ -1130,7 +1129,7 @@ __device__ __forceinline__ void byte_step_emit(const uint32_t (&w)[CB / 32 + 1],
         for (int k = 0; k < 4; ++k) {
             const int j = 4 * m + k;
             if (j >= NFIX && j >= jmax) break;
-            const uint2 e = *reinterpret_cast<const uint2 *>(tab + ((ctl & kFsmRowMask) | step_off(x, k)));
+            const uint2 e = *reinterpret_cast<const uint2 *>(tab + step_addr<8>(x, k, ctl & kFsmRowMask));
             uint32_t sy, c8;
             if (j < NFIX || j < nfull) {
                 ctl = e.x;
