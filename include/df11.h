@@ -295,8 +295,10 @@ df11_status df11_decode_host(df11_blob *const *blobs, const void *const *host_im
  * decoding it again: the slot is reused).  Allocates no device memory; the
  * first call on a device creates 2 x 8 CUDA events that live until exit.
  * Errors: DF11_EINVAL (arguments, group size, mixed codes in a group),
- * DF11_ENOMEM (a group's images exceed slot_bytes; nothing is enqueued),
- * DF11_EUNSUPPORTED, DF11_ECUDA (copy, event or launch failure). */
+ * DF11_ENOMEM (a group's images exceed slot_bytes), both found before
+ * anything is enqueued; DF11_EUNSUPPORTED and DF11_ECUDA (copy, event or
+ * launch failure) stop at the failing group, the groups before it staying
+ * enqueued (synchronise both streams before reusing the slots). */
 df11_status df11_decode_streamed(df11_blob *const *blobs, const int32_t *group_sizes, int n_groups,
                                  const void *const *host_images, void *const *slots, int n_slots,
                                  uint64_t slot_bytes, void *const *dst_dev, int *dev_err_flag,
