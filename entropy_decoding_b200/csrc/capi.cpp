@@ -330,7 +330,12 @@ df11_status df11_decode_streamed(df11_blob *const *blobs, const int32_t *group_s
         uint64_t need = 0;
         for (int i = at; i < at + k; ++i) {
             if (!blobs[i] || !host_images[i]) return DF11_EINVAL;
-            need += df11::align_up(df11::image_layout(blobs[i]->b).total, df11::kImageAlign);
+            // one launch per group: one code and one layout in it
+            const df11::Blob &b = blobs[i]->b, &f = blobs[at]->b;
+            if (b.dtype != f.dtype || b.chunk_bits != f.chunk_bits || b.tile_threads != f.tile_threads ||
+                std::memcmp(b.cb->lengths, f.cb->lengths, sizeof b.cb->lengths) != 0)
+                return DF11_EINVAL;
+            need += df11::align_up(df11::image_layout(b).total, df11::kImageAlign);
         }
         if (need > slot_bytes) return DF11_ENOMEM;
         at += k;

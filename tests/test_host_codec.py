@@ -331,6 +331,11 @@ def test_decode_argument_checks_need_no_gpu(df11):
     with pytest.raises(df11.Df11Error) as e:  # misaligned slot
         df11.df11_decode_streamed([[blob]], [fake], [fake + 16], need, [fake])
     assert e.value.status == df11.DF11_EINVAL
+    other = df11.df11_encode(df11.df11_build_codebook("bf16", [synth.random_bits(5000, "bf16", 4)]),
+                             synth.random_bits(5000, "bf16", 4))
+    with pytest.raises(df11.Df11Error) as e:  # two codes in one group
+        df11.df11_decode_streamed([[blob, other]], [fake, fake], [fake], 4 * need, [fake, fake])
+    assert e.value.status == df11.DF11_EINVAL
     with pytest.raises(df11.Df11Error) as e:  # more than 64 blobs in a group
         df11.df11_decode_streamed([[blob] * 65], [fake] * 65, [fake], need * 65, [fake] * 65)
     assert e.value.status == df11.DF11_EINVAL
