@@ -28,10 +28,13 @@ def df11():
 
 
 def _decode_group(df11, blobs):
+    """One launch over the blobs with the benchmark's options (default walk,
+    overlapped launch)."""
     imgs = [df11.upload(b) for b in blobs]
     outs = [df11.empty_output(b) for b in blobs]
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    df11.df11_decode(blobs, [o.data_ptr() for o in outs], err.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    df11.df11_decode_ex(blobs, [o.data_ptr() for o in outs], err.data_ptr(), torch.cuda.current_stream().cuda_stream,
+                        overlap=1)
     torch.cuda.synchronize()
     del imgs
     return outs, int(err.item())
