@@ -65,6 +65,12 @@ def parse_args():
                    help="decode launch option, warp tiles (0 = library default for the walker)")
     p.add_argument("--walker", choices=["auto", "window", "byte_step"], default="auto",
                    help="decode launch option, warp tiles: how a thread walks its chunk")
+    p.add_argument("--no-chunk-counts", dest="chunk_counts", action="store_false",
+                   help="encode without the chunk-counts section (the pages' sections only): the decode "
+                        "counts each chunk's codes with a first walk")
+    p.add_argument("--count-walk", action="store_true",
+                   help="decode launch option: count each chunk's codes with a first walk even though the "
+                        "images store chunk counts")
     p.add_argument("--no-overlap", dest="overlap", action="store_false",
                    help="launch the groups in plain stream order (default: each group's decode may start "
                         "while the previous one finishes, the groups being independent; the roofline then "
@@ -96,6 +102,8 @@ def full_config(args, world: int) -> dict:
             "chunks_per_thread": args.chunks_per_thread or 1, "ctas_per_sm": args.ctas_per_sm or "max",
             "warps_per_cta": (args.warps_per_cta or "library default") if args.tile_threads == 32 else None,
             "walker": args.walker if args.tile_threads == 32 else "window",
+            "chunk_counts": bool(args.chunk_counts) and args.chunk_bits <= 128,
+            "count_walk": bool(args.count_walk),  # the device-resident decode's launch option
             "overlap_launches": bool(args.overlap),
             "l2": f"no flush: inputs larger than L2 (decoded output {out_gb:.1f} GB, compressed images "
                   f"about 0.68x that, vs 126 MB L2)",
@@ -328,8 +336,8 @@ def kernel_name(args, cfg: dict, shape) -> str:
         cpt = args.chunks_per_thread or 1
         return f"decode_kernel<{dt},{args.chunk_bits},{cpt},{args.tile_threads // cpt}>"
     nw = shape[1] // 32
-    if shape[3] == 2:  # DF11_WALKER_BYTE_STEP
-        return f"decode_fsm_kernel<{dt},{args.chunk_bits},{nw}>"
+    if shape[3] == 2:  # DF11_WALKER_BYTE_STEP; shape[4]: reads the stored chunk counts
+        return f"decode_fsm_kernel<{dt},{args.chunk_bits},{nw},{'true' if shape[4] else 'false'}>"
     return f"decode_warp_kernel<{dt},{args.chunk_bits},{nw}>"
 
 
@@ -360,7 +368,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         g = make_group(args.workload, args.seed, gi)
         dt = "bf16" if g.tensors[0].bits.dtype == np.uint16 else "e4m3"
         cb = df11.df11_build_codebook(dt, [t.bits for t in g.tensors])
-        blobs = [df11.df11_encode(cb, t.bits, args.chunk_bits, args.tile_threads, threads) for t in g.tensors]
+        blobs = [df11.df11_encode(cb, t.bits, args.chunk_bits, args.tile_threads, threads,
+                                  chunk_counts=args.chunk_counts) for t in g.tensors]
         for ti, (t, b) in enumerate(zip(g.tensors, blobs)):
             pos = np.unique(np.concatenate([np.arange(min(4096, t.bits.size)),
                                             np.arange(max(0, t.bits.size - 4096), t.bits.size),
@@ -402,7 +411,15 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     stream.synchronize()
     out_bytes_total = sum(sum(ss) for ss in sizes)
 
-    # algorithmic bytes per launch: compressed sections read + output written
+    walker = {"auto": 0, "window": 1, "byte_step": 2}[args.walker]
+    # the launch shape of the largest group (what the library picked for these options)
+    big = max(range(len(groups)), key=lambda gi: sum(b.info().n_elems for b in groups[gi][1]))
+    shape = df11.df11_decode_launch_shape(groups[big][1], args.chunks_per_thread, args.ctas_per_sm,
+                                          args.warps_per_cta, walker, with_walk=True,
+                                          count_walk=int(args.count_walk))
+
+    # algorithmic bytes per launch: compressed sections read (the chunk counts
+    # when the kernel reads them) + output written
     algo = []
     k = 0
     for name, blobs, dt, dsts in groups:
@@ -411,13 +428,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             i = tensors_meta[k]
             k += 1
             a += i.stream_bytes + i.plane_bytes + i.gaps_bytes + i.out_off_bytes + i.uncompressed_bytes
+            if shape[4]:
+                a += i.counts_bytes
         algo.append(a)
-
-    walker = {"auto": 0, "window": 1, "byte_step": 2}[args.walker]
-    # the launch shape of the largest group (what the library picked for these options)
-    big = max(range(len(groups)), key=lambda gi: sum(b.info().n_elems for b in groups[gi][1]))
-    shape = df11.df11_decode_launch_shape(groups[big][1], args.chunks_per_thread, args.ctas_per_sm,
-                                          args.warps_per_cta, walker, with_walker=True)
 
     def one_step(events=None):
         for gi, (name, blobs, dt, dsts) in enumerate(groups):
@@ -425,7 +438,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                 events[gi][0].record(stream)
             df11.df11_decode_ex(blobs, [d[0] for d in dsts], err.data_ptr(), stream.cuda_stream,
                                 args.chunks_per_thread, args.ctas_per_sm, args.warps_per_cta, walker, 0,
-                                int(args.overlap))
+                                int(args.overlap), count_walk=int(args.count_walk))
             if events is not None and not args.overlap:
                 events[gi][1].record(stream)
 
@@ -595,7 +608,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                     df11.df11_histogram_device(dt_b, x.data_ptr(), x.numel(), counts.data_ptr(), stream.cuda_stream)
                 nsym = 256 if dt_b == "bf16" else 16
                 cb_g = df11.df11_codebook_from_counts(dt_b, counts.cpu().numpy().view(np.uint64)[:nsym])
-                return [df11.encode_on_device(cb_g, x, args.chunk_bits, args.tile_threads, stream) for x in srcs]
+                return [df11.encode_on_device(cb_g, x, args.chunk_bits, args.tile_threads, stream,
+                                              chunk_counts=args.chunk_counts) for x in srcs]
 
         encode_group()
         stream.synchronize()
@@ -641,7 +655,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                      "peak_datasheet": 8000.0, "frac_datasheet": achieved / 8000.0,
                      "kernel": kernel_name(args, cfg, shape),
                      "launch": {"grid": shape[0], "block": shape[1], "smem_bytes": shape[2],
-                                "walker": {1: "window", 2: "byte_step"}.get(shape[3], shape[3])},
+                                "walker": {1: "window", 2: "byte_step"}.get(shape[3], shape[3]),
+                                "stored_counts": bool(shape[4])},
                      "algorithmic_bytes_per_launch": algo_step / len(groups),
                      "launch_ms_mean": float(per_launch.mean()),
                      "launch_ms_by_group": {"first": float(per_launch[:, 0].mean()),

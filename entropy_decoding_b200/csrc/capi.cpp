@@ -32,6 +32,7 @@ struct df11_encoding {
 namespace {
 
 bool valid_dtype(df11_dtype d) { return d == DF11_BF16 || d == DF11_FP8_E4M3; }
+bool valid_encode_flags(int flags) { return (flags & ~DF11_ENCODE_NO_CHUNK_COUNTS) == 0; }
 
 df11_status from_launch(df11::LaunchStatus s) {
     switch (s) {
@@ -128,13 +129,14 @@ df11_status df11_codebook_lengths(const df11_codebook *cb, uint8_t *lengths) {
 void df11_codebook_free(df11_codebook *cb) { delete cb; }
 
 df11_status df11_encode_ex(const df11_codebook *cb, const void *host_src, uint64_t n_elems, int chunk_bits,
-                           int tile_threads, int n_threads, df11_blob **out) {
+                           int tile_threads, int flags, int n_threads, df11_blob **out) {
     if (!cb || !out || (n_elems && !host_src) || n_threads < 0) return DF11_EINVAL;
-    if (!df11::valid_layout(chunk_bits, tile_threads)) return DF11_EINVAL;
+    if (!df11::valid_layout(chunk_bits, tile_threads) || !valid_encode_flags(flags)) return DF11_EINVAL;
     *out = nullptr;
     try {
         auto *blob = new df11_blob;
-        std::string err = df11::encode(cb->cb, host_src, n_elems, chunk_bits, tile_threads, n_threads, &blob->b);
+        std::string err = df11::encode(cb->cb, host_src, n_elems, chunk_bits, tile_threads, n_threads,
+                                       !(flags & DF11_ENCODE_NO_CHUNK_COUNTS), &blob->b);
         if (!err.empty()) {
             delete blob;
             return DF11_EINVAL;
@@ -147,7 +149,7 @@ df11_status df11_encode_ex(const df11_codebook *cb, const void *host_src, uint64
 }
 
 df11_status df11_encode(const df11_codebook *cb, const void *host_src, uint64_t n_elems, df11_blob **out) {
-    return df11_encode_ex(cb, host_src, n_elems, 128, 32, 0, out);
+    return df11_encode_ex(cb, host_src, n_elems, 128, 32, 0, 0, out);
 }
 
 int df11_layout_supported(df11_dtype dtype, int chunk_bits, int tile_threads) {
@@ -176,6 +178,7 @@ df11_status df11_blob_get_info(const df11_blob *blob, df11_blob_info *info) {
     info->serialized_bytes = df11::serialized_bytes(b);
     info->device_bytes = df11::image_layout(b).total;
     info->uncompressed_bytes = b.dtype == df11::kBF16 ? 2 * b.n : b.n;
+    info->counts_bytes = b.chunk_counts ? b.n_tiles * static_cast<uint64_t>(b.tile_threads) : 0;
     return DF11_OK;
 }
 
@@ -186,6 +189,12 @@ df11_status df11_blob_sections(const df11_blob *blob, const uint8_t **stream, co
     if (plane) *plane = blob->b.plane.data();
     if (gaps) *gaps = blob->b.gaps.data();
     if (out_off) *out_off = blob->b.out_off.data();
+    return DF11_OK;
+}
+
+df11_status df11_blob_chunk_counts(const df11_blob *blob, const uint8_t **counts) {
+    if (!blob || !counts || blob->b.device_only) return DF11_EINVAL;
+    *counts = blob->b.chunk_counts ? blob->b.counts.data() : nullptr;
     return DF11_OK;
 }
 
@@ -273,9 +282,10 @@ df11_status df11_decode_ex(const df11_blob *const *blobs, void *const *dst_dev, 
         o.max_ctas = opts->max_ctas;
         o.overlap = opts->overlap;
         o.diag_expire_waits = opts->diag_expire_waits;
+        o.count_walk = opts->count_walk;
         if (o.chunks_per_thread < 0 || o.ctas_per_sm < 0 || o.warps_per_cta < 0 || o.walker < 0 ||
             o.walker > DF11_WALKER_BYTE_STEP || o.max_ctas < 0 || o.overlap < 0 || o.overlap > 1 ||
-            o.diag_expire_waits < 0 || o.diag_expire_waits > 1)
+            o.diag_expire_waits < 0 || o.diag_expire_waits > 1 || o.count_walk < 0 || o.count_walk > 1)
             return DF11_EINVAL;
     }
     return from_launch(df11::launch_decode(bs, dst_dev, n_blobs, dev_err_flag, o,
@@ -375,11 +385,12 @@ df11_status df11_decode_streamed(df11_blob *const *blobs, const int32_t *group_s
 
 df11_status df11_decode_launch_shape(const df11_blob *const *blobs, int n_blobs, int *grid, int *block,
                                      int *smem_bytes) {
-    return df11_decode_launch_shape_ex(blobs, n_blobs, nullptr, grid, block, smem_bytes, nullptr);
+    return df11_decode_launch_shape_ex(blobs, n_blobs, nullptr, grid, block, smem_bytes, nullptr, nullptr);
 }
 
 df11_status df11_decode_launch_shape_ex(const df11_blob *const *blobs, int n_blobs, const df11_decode_opts *opts,
-                                        int *grid, int *block, int *smem_bytes, int *walker) {
+                                        int *grid, int *block, int *smem_bytes, int *walker,
+                                        int *stored_counts) {
     if (!blobs || n_blobs < 1 || n_blobs > df11::kMaxTensorsPerLaunch) return DF11_EINVAL;
     const df11::Blob *bs[df11::kMaxTensorsPerLaunch];
     for (int i = 0; i < n_blobs; ++i) {
@@ -394,8 +405,9 @@ df11_status df11_decode_launch_shape_ex(const df11_blob *const *blobs, int n_blo
         o.warps_per_cta = opts->warps_per_cta;
         o.walker = opts->walker;
         o.max_ctas = opts->max_ctas;
+        o.count_walk = opts->count_walk;
         if (o.chunks_per_thread < 0 || o.ctas_per_sm < 0 || o.warps_per_cta < 0 || o.walker < 0 ||
-            o.walker > DF11_WALKER_BYTE_STEP || o.max_ctas < 0)
+            o.walker > DF11_WALKER_BYTE_STEP || o.max_ctas < 0 || o.count_walk < 0 || o.count_walk > 1)
             return DF11_EINVAL;
     }
     df11::LaunchStatus st = df11::decode_launch_shape(bs, n_blobs, o, &sh);
@@ -404,6 +416,7 @@ df11_status df11_decode_launch_shape_ex(const df11_blob *const *blobs, int n_blo
     if (block) *block = sh.block;
     if (smem_bytes) *smem_bytes = sh.smem;
     if (walker) *walker = sh.walker;
+    if (stored_counts) *stored_counts = sh.stored_counts;
     return DF11_OK;
 }
 
@@ -441,10 +454,10 @@ df11_status df11_codebook_from_counts(df11_dtype dtype, const uint64_t *counts, 
 uint64_t df11_encode_device_scratch_bytes(uint64_t n_elems) { return df11::encode_scratch_bytes(n_elems); }
 
 df11_status df11_encode_device_begin(const df11_codebook *cb, const void *src_dev, uint64_t n_elems, int chunk_bits,
-                                     int tile_threads, void *scratch_dev, uint64_t scratch_cap, df11_stream stream,
-                                     uint64_t *image_bytes, df11_encoding **out) {
+                                     int tile_threads, int flags, void *scratch_dev, uint64_t scratch_cap,
+                                     df11_stream stream, uint64_t *image_bytes, df11_encoding **out) {
     if (!cb || !out || !image_bytes || !scratch_dev || (n_elems && !src_dev)) return DF11_EINVAL;
-    if (!df11::valid_layout(chunk_bits, tile_threads)) return DF11_EINVAL;
+    if (!df11::valid_layout(chunk_bits, tile_threads) || !valid_encode_flags(flags)) return DF11_EINVAL;
     if (reinterpret_cast<uintptr_t>(src_dev) % 16 || reinterpret_cast<uintptr_t>(scratch_dev) % 16) return DF11_EINVAL;
     if (scratch_cap < df11::encode_scratch_bytes(n_elems)) return DF11_ENOMEM;
     *out = nullptr;
@@ -455,6 +468,7 @@ df11_status df11_encode_device_begin(const df11_codebook *cb, const void *src_de
         enc->job.n = n_elems;
         enc->job.chunk_bits = chunk_bits;
         enc->job.tile_threads = tile_threads;
+        enc->job.chunk_counts = !(flags & DF11_ENCODE_NO_CHUNK_COUNTS) && df11::counts_fit(chunk_bits);
         enc->scratch = static_cast<uint64_t *>(scratch_dev);
         enc->stream = reinterpret_cast<cudaStream_t>(stream);
         std::string err = df11::encode_device_bits(enc->job, enc->scratch, enc->stream, &enc->total_bits);
@@ -471,6 +485,7 @@ df11_status df11_encode_device_begin(const df11_codebook *cb, const void *src_de
         const uint64_t cbits = static_cast<uint64_t>(chunk_bits);
         meta.n_tiles = ((enc->total_bits + cbits - 1) / cbits + tile_threads - 1) / tile_threads;
         meta.cb = cb->cb;
+        meta.chunk_counts = enc->job.chunk_counts;
         enc->image_bytes = df11::image_layout(meta).total;
         *image_bytes = enc->image_bytes;
         *out = enc;
@@ -496,6 +511,7 @@ df11_status df11_encode_device_end(df11_encoding *enc, void *image_dev, uint64_t
         const uint64_t cbits = static_cast<uint64_t>(b.chunk_bits);
         b.n_tiles = ((b.total_bits + cbits - 1) / cbits + b.tile_threads - 1) / b.tile_threads;
         b.cb = enc->job.cb;
+        b.chunk_counts = enc->job.chunk_counts;
         b.device_only = true;
         const df11::ImageLayout L = df11::image_layout(b);
         if (b.n) {
@@ -545,10 +561,10 @@ df11_status df11_blob_fetch(df11_blob *blob, df11_stream stream) {
 }
 
 df11_status df11_encode_device_noalloc(const df11_codebook *cb, const void *src_dev, uint64_t n_elems,
-                                       int chunk_bits, int tile_threads, void *image_dev, uint64_t image_cap,
-                                       df11_stream stream, df11_encode_result *result) {
+                                       int chunk_bits, int tile_threads, int flags, void *image_dev,
+                                       uint64_t image_cap, df11_stream stream, df11_encode_result *result) {
     if (!cb || !result || !image_dev || (n_elems && !src_dev)) return DF11_EINVAL;
-    if (!df11::valid_layout(chunk_bits, tile_threads)) return DF11_EINVAL;
+    if (!df11::valid_layout(chunk_bits, tile_threads) || !valid_encode_flags(flags)) return DF11_EINVAL;
     if (n_elems > df11::noalloc_max_elems()) return DF11_EINVAL;
     if (reinterpret_cast<uintptr_t>(src_dev) % 16 || reinterpret_cast<uintptr_t>(image_dev) % df11::kImageAlign)
         return DF11_EINVAL;
@@ -558,6 +574,7 @@ df11_status df11_encode_device_noalloc(const df11_codebook *cb, const void *src_
     job.n = n_elems;
     job.chunk_bits = chunk_bits;
     job.tile_threads = tile_threads;
+    job.chunk_counts = !(flags & DF11_ENCODE_NO_CHUNK_COUNTS) && df11::counts_fit(chunk_bits);
     df11::NoallocResult r{};
     const std::string err = df11::encode_device_noalloc(job, static_cast<uint8_t *>(image_dev), image_cap,
                                                         reinterpret_cast<cudaStream_t>(stream), &r);

@@ -410,7 +410,7 @@ inline void or_byte(uint8_t *p, uint8_t v) { __atomic_fetch_or(p, v, __ATOMIC_RE
 }  // namespace
 
 std::string encode(std::shared_ptr<const Codebook> cb, const void *src, uint64_t n, int chunk_bits,
-                   int tile_threads, int n_threads, Blob *out) {
+                   int tile_threads, int n_threads, bool chunk_counts, Blob *out) {
     if (!valid_layout(chunk_bits, tile_threads)) return "unsupported layout";
     if (n && !src) return "null source";
     const int dtype = cb->dtype;
@@ -421,6 +421,7 @@ std::string encode(std::shared_ptr<const Codebook> cb, const void *src, uint64_t
     b.tile_threads = tile_threads;
     b.n = n;
     b.cb = cb;
+    b.chunk_counts = chunk_counts && counts_fit(chunk_bits);
     b.plane.assign(plane_bytes(dtype, n), 0);
 
     // segments of an even number of elements (E4M3 packs pairs into a byte)
@@ -543,6 +544,32 @@ std::string encode(std::shared_ptr<const Codebook> cb, const void *src, uint64_t
     uint64_t ms = 0;
     for (uint64_t t = 0; t < b.n_tiles; ++t) ms = std::max(ms, b.out_off[t + 1] - b.out_off[t]);
     b.max_span = ms;
+
+    // pass 3 (chunk counts): codes starting in each chunk.  A segment counts
+    // the chunk its first code starts in locally (an earlier segment may
+    // count codes of that chunk too) and every later chunk in place, which
+    // no other segment touches; the local counts are added afterwards.
+    if (b.chunk_counts) {
+        b.counts.assign(b.n_tiles * tile_threads, 0);
+        std::vector<uint32_t> first_count(n_seg, 0);
+        parallel_for(n_seg, n_threads, [&](uint64_t s0, uint64_t s1) {
+            for (uint64_t s = s0; s < s1; ++s) {
+                const uint64_t i0 = s * seg_elems, i1 = std::min(n, i0 + seg_elems);
+                uint64_t start = seg_bits[s];
+                const uint64_t c_first = start / cbits;
+                uint32_t local = 0;
+                for (uint64_t i = i0; i < i1; ++i) {
+                    const uint64_t c = start / cbits;
+                    if (c == c_first) ++local;
+                    else ++b.counts[c];
+                    start += len[exps[i]];
+                }
+                first_count[s] = local;
+            }
+        });
+        for (uint64_t s = 0; s < n_seg; ++s)
+            b.counts[seg_bits[s] / cbits] = static_cast<uint8_t>(b.counts[seg_bits[s] / cbits] + first_count[s]);
+    }
     return "";
 }
 
@@ -561,21 +588,24 @@ struct FileHeader {
     uint64_t n_tiles;
     uint64_t max_span;
     uint32_t nsym;
-    uint32_t reserved;
+    uint32_t flags;  // version 2: bit 0 = the chunk-counts section follows the gaps
 };
 static_assert(sizeof(FileHeader) == 64, "header layout");
+constexpr uint32_t kFileFlagCounts = 1;
 
 const char kMagic[8] = {'D', 'F', '1', '1', 'B', '2', '0', '0'};
 
 struct FileLayout {
-    uint64_t lengths, gaps, out_off, stream, plane, total;
+    uint64_t lengths, gaps, counts, out_off, stream, plane, total;
 };
 
-FileLayout file_layout(int dtype, uint64_t n, uint64_t total_bits, uint64_t n_tiles, int tile_threads) {
+FileLayout file_layout(int dtype, uint64_t n, uint64_t total_bits, uint64_t n_tiles, int tile_threads,
+                       bool counts) {
     FileLayout f;
     f.lengths = sizeof(FileHeader);
     f.gaps = align_up(f.lengths + 256, 16);
-    f.out_off = align_up(f.gaps + n_tiles * tile_threads, 16);
+    f.counts = align_up(f.gaps + n_tiles * tile_threads, 16);
+    f.out_off = align_up(f.counts + (counts ? n_tiles * tile_threads : 0), 16);
     f.stream = align_up(f.out_off + (n_tiles + 1) * 8, 16);
     f.plane = align_up(f.stream + (total_bits + 7) / 8, 16);
     f.total = align_up(f.plane + plane_bytes(dtype, n), 16);
@@ -585,15 +615,17 @@ FileLayout file_layout(int dtype, uint64_t n, uint64_t total_bits, uint64_t n_ti
 }  // namespace
 
 uint64_t serialized_bytes(const Blob &b) {
-    return file_layout(b.dtype, b.n, b.total_bits, b.n_tiles, b.tile_threads).total;
+    return file_layout(b.dtype, b.n, b.total_bits, b.n_tiles, b.tile_threads, b.chunk_counts).total;
 }
 
 void serialize(const Blob &b, uint8_t *dst) {
-    FileLayout f = file_layout(b.dtype, b.n, b.total_bits, b.n_tiles, b.tile_threads);
+    FileLayout f = file_layout(b.dtype, b.n, b.total_bits, b.n_tiles, b.tile_threads, b.chunk_counts);
     std::memset(dst, 0, f.total);
     FileHeader h{};
     std::memcpy(h.magic, kMagic, 8);
-    h.version = 1;
+    // version 1 (no flags) unless the counts section is present
+    h.version = b.chunk_counts ? 2 : 1;
+    h.flags = b.chunk_counts ? kFileFlagCounts : 0;
     h.dtype = static_cast<uint32_t>(b.dtype);
     h.n_elems = b.n;
     h.total_bits = b.total_bits;
@@ -605,6 +637,7 @@ void serialize(const Blob &b, uint8_t *dst) {
     std::memcpy(dst, &h, sizeof h);
     std::memcpy(dst + f.lengths, b.cb->lengths, 256);
     if (!b.gaps.empty()) std::memcpy(dst + f.gaps, b.gaps.data(), b.gaps.size());
+    if (b.chunk_counts && !b.counts.empty()) std::memcpy(dst + f.counts, b.counts.data(), b.counts.size());
     std::memcpy(dst + f.out_off, b.out_off.data(), b.out_off.size() * 8);
     if (!b.stream.empty()) std::memcpy(dst + f.stream, b.stream.data(), b.stream.size());
     if (!b.plane.empty()) std::memcpy(dst + f.plane, b.plane.data(), b.plane.size());
@@ -615,17 +648,22 @@ std::string deserialize(const uint8_t *src, uint64_t len, Blob *out) {
     FileHeader h;
     std::memcpy(&h, src, sizeof h);
     if (std::memcmp(h.magic, kMagic, 8) != 0) return "bad magic";
-    if (h.version != 1) return "unknown version";
+    if (h.version != 1 && h.version != 2) return "unknown version";
+    if (h.version == 1 && h.flags) return "flags in a version 1 container";
+    if (h.flags & ~kFileFlagCounts) return "unknown flags";
+    const bool has_counts = (h.flags & kFileFlagCounts) != 0;
     if (h.dtype != kBF16 && h.dtype != kE4M3) return "bad dtype";
     const int dtype = static_cast<int>(h.dtype);
     if (h.nsym != static_cast<uint32_t>(nsym_of(dtype))) return "bad symbol count";
     if (!valid_layout(static_cast<int>(h.chunk_bits), static_cast<int>(h.tile_threads))) return "bad layout";
+    if (has_counts && !counts_fit(static_cast<int>(h.chunk_bits))) return "chunk counts with chunks over 128 bits";
     if (h.n_elems > (uint64_t{1} << 48)) return "element count out of range";
     const uint64_t cbits = h.chunk_bits, tbits = cbits * h.tile_threads;
     const uint64_t n_chunks = (h.total_bits + cbits - 1) / cbits;
     if (h.n_tiles != (n_chunks + h.tile_threads - 1) / h.tile_threads) return "tile count mismatch";
     if (h.total_bits > h.n_elems * kMaxCodeLen || h.total_bits < h.n_elems) return "stream length out of range";
-    FileLayout f = file_layout(dtype, h.n_elems, h.total_bits, h.n_tiles, static_cast<int>(h.tile_threads));
+    FileLayout f = file_layout(dtype, h.n_elems, h.total_bits, h.n_tiles, static_cast<int>(h.tile_threads),
+                               has_counts);
     if (f.total != len) return "container size mismatch";
     uint8_t lengths[256];
     std::memcpy(lengths, src + f.lengths, 256);
@@ -645,6 +683,8 @@ std::string deserialize(const uint8_t *src, uint64_t len, Blob *out) {
     b.max_span = h.max_span;
     b.cb = cb;
     b.gaps.assign(src + f.gaps, src + f.gaps + h.n_tiles * h.tile_threads);
+    b.chunk_counts = has_counts;
+    if (has_counts) b.counts.assign(src + f.counts, src + f.counts + h.n_tiles * h.tile_threads);
     b.out_off.resize(h.n_tiles + 1);
     std::memcpy(b.out_off.data(), src + f.out_off, (h.n_tiles + 1) * 8);
     b.stream.assign(src + f.stream, src + f.stream + (h.total_bits + 7) / 8);
@@ -665,6 +705,19 @@ std::string deserialize(const uint8_t *src, uint64_t len, Blob *out) {
             if (c * cbits + b.gaps[c] > h.total_bits) return "gap beyond the stream";
         } else if (b.gaps[c]) {
             return "nonzero padding gap";
+        }
+    }
+    if (has_counts) {
+        // each tile's counts add up to its span; padding chunks start no code
+        for (uint64_t t = 0; t < h.n_tiles; ++t) {
+            uint64_t sum = 0;
+            for (uint64_t j = 0; j < h.tile_threads; ++j) {
+                const uint64_t c = t * h.tile_threads + j;
+                if (c >= n_chunks && b.counts[c]) return "nonzero padding count";
+                if (b.counts[c] > cbits) return "chunk count above its bits";
+                sum += b.counts[c];
+            }
+            if (sum != b.out_off[t + 1] - b.out_off[t]) return "chunk counts do not add up to the tile span";
         }
     }
     if (h.total_bits & 7) {
@@ -690,6 +743,8 @@ ImageLayout image_layout(const Blob &b) {
     o = align_up(o + b.cb->fsm.size() * 4, kImageAlign);
     L.gaps = o;
     o = align_up(o + b.n_tiles * static_cast<uint64_t>(b.tile_threads) + kGapsTail, kImageAlign);
+    L.counts = o;
+    if (b.chunk_counts) o = align_up(o + b.n_tiles * static_cast<uint64_t>(b.tile_threads), kImageAlign);
     L.out_off = o;
     o = align_up(o + (b.n_tiles + 1) * 8, kImageAlign);
     L.stream = o;
@@ -709,6 +764,7 @@ void write_image_head(const Blob &b, const ImageLayout &L, uint8_t *dst) {
     h.tile_threads = static_cast<uint32_t>(b.tile_threads);
     h.n_luts = static_cast<uint32_t>(b.cb->n_luts());
     h.fsm_rows = static_cast<uint32_t>(b.cb->fsm_rows);
+    h.flags = b.chunk_counts ? kImageFlagCounts : 0u;
     h.n_elems = b.n;
     h.total_bits = b.total_bits;
     h.n_tiles = b.n_tiles;
@@ -726,6 +782,7 @@ void write_image(const Blob &b, uint8_t *dst) {
     std::memset(dst, 0, L.total);
     write_image_head(b, L, dst);
     if (!b.gaps.empty()) std::memcpy(dst + L.gaps, b.gaps.data(), b.gaps.size());
+    if (b.chunk_counts && !b.counts.empty()) std::memcpy(dst + L.counts, b.counts.data(), b.counts.size());
     std::memcpy(dst + L.out_off, b.out_off.data(), b.out_off.size() * 8);
     // stream as 32-bit words, earliest bit in bit 31 (little-endian storage)
     for (uint64_t i = 0; i < b.stream.size(); ++i) dst[L.stream + (i ^ 3)] = b.stream[i];
@@ -735,6 +792,8 @@ void write_image(const Blob &b, uint8_t *dst) {
 void read_image_sections(Blob &b, const uint8_t *img) {
     const ImageLayout L = image_layout(b);
     b.gaps.assign(img + L.gaps, img + L.gaps + b.n_tiles * b.tile_threads);
+    if (b.chunk_counts) b.counts.assign(img + L.counts, img + L.counts + b.n_tiles * b.tile_threads);
+    else b.counts.clear();
     b.out_off.resize(b.n_tiles + 1);
     std::memcpy(b.out_off.data(), img + L.out_off, (b.n_tiles + 1) * 8);
     b.stream.resize((b.total_bits + 7) / 8);

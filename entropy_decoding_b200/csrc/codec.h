@@ -42,6 +42,8 @@ struct Blob {
     std::vector<uint8_t> stream;    // ceil(total_bits / 8)
     std::vector<uint8_t> plane;     // n (BF16) or ceil(n / 2) (E4M3)
     std::vector<uint8_t> gaps;      // n_tiles * tile_threads
+    bool chunk_counts = false;      // the counts section is part of the container
+    std::vector<uint8_t> counts;    // n_tiles * tile_threads when chunk_counts (codes starting per chunk)
     std::vector<uint64_t> out_off;  // n_tiles + 1
     bool device_only = false;  // encoded on the GPU: host sections empty until fetched
     const uint8_t *dev_image = nullptr;
@@ -57,9 +59,13 @@ std::shared_ptr<Codebook> make_codebook(int dtype, const uint8_t *lengths);  // 
 // Histogram of the exponent field, added into counts[256].
 void histogram(int dtype, const void *src, uint64_t n, uint64_t *counts, int n_threads);
 
-// Encoder: returns an empty string on success, else the reason.
+// Encoder: returns an empty string on success, else the reason.  chunk_counts
+// asks for the chunk-counts section (stored only when chunk_bits <= 128).
 std::string encode(std::shared_ptr<const Codebook> cb, const void *src, uint64_t n, int chunk_bits,
-                   int tile_threads, int n_threads, Blob *out);
+                   int tile_threads, int n_threads, bool chunk_counts, Blob *out);
+
+// Whether a layout stores chunk counts when they are asked for.
+inline bool counts_fit(int chunk_bits) { return chunk_bits <= kCountsMaxChunkBits; }
 
 uint64_t plane_bytes(int dtype, uint64_t n);
 uint64_t serialized_bytes(const Blob &b);

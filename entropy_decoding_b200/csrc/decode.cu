@@ -1111,11 +1111,14 @@ __device__ __forceinline__ uint32_t byte_step_count(const uint32_t (&w)[CB / 32 
 // word it ends in later threads' bytes: that last, partial word is returned
 // in acc / wp / f8 and OR-ed in by the caller after a __syncwarp, so it
 // lands after every plain store of the warp and no store clears another
-// thread's bytes.  The buffer is zero outside the words written.
+// thread's bytes.  The buffer is zero outside the words written.  ctl_out
+// receives the last control word, whose row is the dead row (`dead`) when
+// the walk left the tables or the partial byte ends more than 4 codes.
 template <int CB>
 __device__ __forceinline__ void byte_step_emit(const uint32_t (&w)[CB / 32 + 1], uint32_t w2, int g, int nfull,
                                                int r, int jmax, const uint8_t *tab, uint32_t out, uint32_t acc0,
-                                               uint32_t &acc, uint32_t &wp, uint32_t &f8) {
+                                               uint32_t dead, uint32_t &acc, uint32_t &wp, uint32_t &f8,
+                                               uint32_t &ctl_out) {
     constexpr int CW = CB / 32, NFIX = kFixedSteps<CB>;
     uint32_t ctl = 0;
     acc = acc0;
@@ -1136,9 +1139,11 @@ __device__ __forceinline__ void byte_step_emit(const uint32_t (&w)[CB / 32 + 1],
                 sy = e.y;
                 c8 = e.x >> (kFsmCountShift - 3);  // 8 x codes ended
             } else if (j == nfull) {
-                const uint32_t c = min(static_cast<uint32_t>(__popc(e.x & ((1u << r) - 1u))), 4u);
+                const uint32_t ce = static_cast<uint32_t>(__popc(e.x & ((1u << r) - 1u)));
+                const uint32_t c = min(ce, 4u);
                 sy = c ? e.y & (0xFFFFFFFFu >> (32u - 8u * c)) : 0u;
                 c8 = 8u * c;
+                if (ce > 4) ctl = dead;
             } else {
                 continue;
             }
@@ -1155,25 +1160,34 @@ __device__ __forceinline__ void byte_step_emit(const uint32_t (&w)[CB / 32 + 1],
             }
         }
     }
+    ctl_out = ctl;
 }
 
 // Shared memory of the byte-step kernel: the transition table (fsm_rows rows
 // of kFsmRowBytes) at offset 0, its control words alone (rows of 1 KB: end
-// mask, row << 10, count << 24), the root hierarchical table, then per warp
-// its mbarrier, one stage (the tile's 32 chunks + 16 look-ahead bytes, then
-// 48 gap bytes: its own 32 and the next tile's first 16) and its exponent
-// buffer.
+// mask, row << 10, count << 24; only when the kernel counts with a walk),
+// the root hierarchical table, then per warp its mbarrier, one stage (the
+// tile's 32 chunks + 16 look-ahead bytes, then 48 gap bytes: its own 32 and
+// the next tile's first 16, then with stored counts the tile's 32 chunk
+// counts) and its exponent buffer.
 struct FsmPlan {
     uint32_t stage_bytes, exps_bytes, warp_bytes, off_ctl, off_lut, off_warps, total;
 };
 
-__host__ __device__ inline FsmPlan make_fsm_plan(int chunk_bits, int nwarp, uint32_t max_span, int fsm_rows) {
+__host__ __device__ inline FsmPlan make_fsm_plan(int chunk_bits, int nwarp, uint32_t max_span, int fsm_rows,
+                                                 bool counts) {
     FsmPlan p;
-    p.stage_bytes = static_cast<uint32_t>(32 * chunk_bits / 8) + 16u + 48u;
-    p.exps_bytes = (max_span + 2u * 32u + 16u + 15u) & ~15u;
+    p.stage_bytes = static_cast<uint32_t>(32 * chunk_bits / 8) + 16u + 48u + (counts ? 32u : 0u);
+    // the tile's span after its offset in the first group (< 32), plus room for
+    // the last group's rounding; with stored counts, plus what one thread's
+    // walk can write past the range its stored count gives it (4 symbols a
+    // step, chunk_bits / 8 + 4 steps at most, and the word it ends in) when
+    // the stream disagrees with the count
+    const uint32_t slack = counts ? 32u + 4u * static_cast<uint32_t>(chunk_bits / 8 + 6) : 2u * 32u + 16u;
+    p.exps_bytes = (max_span + slack + 15u) & ~15u;
     p.warp_bytes = (16u + p.stage_bytes + p.exps_bytes + 127u) & ~127u;
     p.off_ctl = static_cast<uint32_t>(fsm_rows) * kFsmRowBytes;
-    p.off_lut = p.off_ctl + static_cast<uint32_t>(fsm_rows) * (kFsmRowBytes / 2);
+    p.off_lut = p.off_ctl + (counts ? 0u : static_cast<uint32_t>(fsm_rows) * (kFsmRowBytes / 2));
     p.off_warps = up128(p.off_lut + kLutEntries * 2);
     p.total = p.off_warps + static_cast<uint32_t>(nwarp) * p.warp_bytes;
     return p;
@@ -1193,16 +1207,24 @@ __host__ __device__ inline FsmPlan make_fsm_plan(int chunk_bits, int nwarp, uint
 // the run, which decodes the rest of the group right after them, merges it
 // as a whole group; a group is stored piecewise only where a run or a tensor
 // begins or ends.
-template <int DT, int CB, int NWARP>
+//
+// CNT: the images store chunk counts, copied with the tile, and the scan of
+// those bytes places each thread's output: no count walk (phase 1).  Each
+// thread's walk is then checked against its stored count; a walk that ends a
+// different number of codes flags DF11_DEV_ERR_SPAN, its tile's exponent
+// buffer is cleared afterwards, and the carried group is dropped.
+template <int DT, int CB, int NWARP, bool CNT>
 __global__ void __launch_bounds__(NWARP * 32, 1)
     decode_fsm_kernel(const __grid_constant__ DecodeParams P, const uint32_t max_span, const int) {
     constexpr int CW = CB / 32;
     constexpr int NFIX = kFixedSteps<CB>;
     constexpr uint32_t TILE_BYTES = 32 * CB / 8;
     constexpr uint32_t GROUP = DT == 0 ? 16u : 32u;
+    constexpr uint32_t STAGE_TX = TILE_BYTES + 16u + 48u + (CNT ? 32u : 0u);
+    static_assert(!CNT || CB <= kCountsMaxChunkBits, "chunk counts need chunks of at most 128 bits");
     extern __shared__ __align__(128) uint8_t smem[];
     const int rows = P.fsm_rows;
-    const FsmPlan plan = make_fsm_plan(CB, NWARP, max_span, rows);
+    const FsmPlan plan = make_fsm_plan(CB, NWARP, max_span, rows, CNT);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint16_t *s_lut = reinterpret_cast<uint16_t *>(smem + plan.off_lut);
     uint8_t *wbase = smem + plan.off_warps + warp * plan.warp_bytes;
@@ -1224,8 +1246,9 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
             if ((v.x & kFsmRowMask) >= lim) v.x = (v.x & ~kFsmRowMask) | dead;
             if ((v.z & kFsmRowMask) >= lim) v.z = (v.z & ~kFsmRowMask) | dead;
             s[i] = v;
-            sc[i] = make_uint2((v.x & 0xFFu) | ((v.x & kFsmRowMask) >> 1) | ((v.x >> kFsmCountShift) << 24),
-                               (v.z & 0xFFu) | ((v.z & kFsmRowMask) >> 1) | ((v.z >> kFsmCountShift) << 24));
+            if constexpr (!CNT)
+                sc[i] = make_uint2((v.x & 0xFFu) | ((v.x & kFsmRowMask) >> 1) | ((v.x >> kFsmCountShift) << 24),
+                                   (v.z & 0xFFu) | ((v.z & kFsmRowMask) >> 1) | ((v.z >> kFsmCountShift) << 24));
         }
         const uint4 *gl = reinterpret_cast<const uint4 *>(P.lut);
         uint4 *sl = reinterpret_cast<uint4 *>(s_lut);
@@ -1251,9 +1274,10 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         ti_issue = tensor_of(P, t, ti_issue);
         const TensorDesc &d = P.t[ti_issue];
         const uint32_t lt = t - d.tile_begin;
-        mbar_arrive_expect_tx(&full[0], TILE_BYTES + 16u + 48u);
+        mbar_arrive_expect_tx(&full[0], STAGE_TX);
         bulk_load(stage, d.stream + static_cast<uint64_t>(lt) * TILE_BYTES, TILE_BYTES + 16u, &full[0]);
         bulk_load(stage + TILE_BYTES + 16u, d.gaps + static_cast<uint64_t>(lt) * 32u, 48u, &full[0]);
+        if constexpr (CNT) bulk_load(stage + TILE_BYTES + 64u, d.counts + static_cast<uint64_t>(lt) * 32u, 32u, &full[0]);
     };
     if (lane == 0 && t_begin < t_end && !P.expire) issue(t_begin);
     bool pending = t_begin < t_end && !P.expire;
@@ -1333,6 +1357,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         }
         const int graw = stage[TILE_BYTES + 16u + lane];
         const int gnext = stage[TILE_BYTES + 16u + lane + 1];
+        uint32_t cnt = CNT ? static_cast<uint32_t>(stage[TILE_BYTES + 64u + lane]) : 0u;
         // the stage is in registers: refill it with the run's next tile
         __syncwarp();
         if (t + 1 < t_end) {
@@ -1355,17 +1380,25 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         const int nfull = nbits >> 3, r = nbits & 7;
         const int jmax = static_cast<int>(__reduce_max_sync(0xFFFFFFFFu, whole ? nfull + (r != 0) : 0));
 
-        // ---- phase 1: count
-        uint32_t ctl;
-        const uint32_t dead_c = dead >> 1;
-        uint32_t cnt = byte_step_count<CB>(w, w2, g & 31, nfull, r, jmax, smem + plan.off_ctl, dead_c, ctl);
-        const bool slow = !whole || (ctl & kCtlRowMask) == dead_c;
+        // ---- the thread's number of codes: stored, or counted by phase 1
+        // (threads without a whole range count with the window walk; with
+        // stored counts that count checks the stored one)
+        bool slow, mism = false;
+        if constexpr (CNT) {
+            slow = !whole;
+        } else {
+            uint32_t ctl;
+            const uint32_t dead_c = dead >> 1;
+            cnt = byte_step_count<CB>(w, w2, g & 31, nfull, r, jmax, smem + plan.off_ctl, dead_c, ctl);
+            slow = !whole || (ctl & kCtlRowMask) == dead_c;
+        }
         if (__any_sync(0xFFFFFFFFu, slow)) {
             if (slow) {
                 const int gg[1] = {g}, ee[1] = {E};
                 uint32_t c1[1];
                 count_codes<CW, 1, true>(w, gg, ee, T, c1, err);
-                cnt = c1[0];
+                if (CNT) mism = c1[0] != cnt;
+                else cnt = c1[0];
             }
         }
         uint32_t incl = cnt;
@@ -1386,10 +1419,29 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
             // the word a range starts in may hold carried exponents: start from it
             const uint32_t acc0 = joined ? *reinterpret_cast<const uint32_t *>(s_exps + (qrel & ~3u)) : 0u;
             __syncwarp();
-            uint32_t acc = 0, wp = 0, f8 = 0;
-            if (!slow) byte_step_emit<CB>(w, w2, g, nfull, r, jmax, smem, q, acc0, acc, wp, f8);
+            uint32_t acc = 0, wp = 0, f8 = 0, last = 0;
+            if (!slow) byte_step_emit<CB>(w, w2, g, nfull, r, jmax, smem, q, acc0, dead, acc, wp, f8, last);
+            // with stored counts: a walk that left the tables is redone with the
+            // window walk below; a whole walk must end the stored number of codes
+            // (8 bits of f8 per code: wp * 8 + f8 advanced by 8 per symbol from q * 8)
+            bool redo = false;
+            if constexpr (CNT) {
+                redo = !slow && (last & kFsmRowMask) == dead;
+                if (!slow && !redo && (wp - q) * 8u + f8 != 8u * cnt) mism = true;
+            }
             __syncwarp();  // every plain store of phase 2 before the OR-ed words
-            if (!slow && f8) asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(wp), "r"(acc) : "memory");
+            if (!slow && !redo && f8) asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(wp), "r"(acc) : "memory");
+            if constexpr (CNT) {
+                if (__any_sync(0xFFFFFFFFu, redo)) {
+                    if (redo) {
+                        const int gg[1] = {g}, ee[1] = {E};
+                        uint32_t c1[1];
+                        count_codes<CW, 1, true>(w, gg, ee, T, c1, err);
+                        if (c1[0] != cnt) mism = true;
+                    }
+                }
+                slow = (slow || redo) && !mism;  // a thread whose count disagrees writes nothing more
+            }
             if (__any_sync(0xFFFFFFFFu, slow)) {
                 if (slow) emit_codes<CW, 1, 0, true>(w, g, E, T, q, err);
             }
@@ -1425,7 +1477,16 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
             } else {
                 carry_n = 0;  // a carried group was merged above
             }
+            if (CNT && __any_sync(0xFFFFFFFFu, mism)) {
+                // a walk wrote past its stored range: clear the whole buffer
+                // (the tile's output is flagged) and drop the carried group
+                uint4 *se = reinterpret_cast<uint4 *>(s_exps);
+                for (uint32_t i = lane; i < plan.exps_bytes / 16; i += 32) se[i] = make_uint4(0, 0, 0, 0);
+                carry_n = 0;
+                __syncwarp();
+            }
         }
+        if (mism) err |= DF11_DEV_ERR_SPAN;
     }
     if (carry_n) flush_carry();
     // after an abort: wait (bounded) for a copy that was issued but never consumed
@@ -1443,27 +1504,35 @@ using KernelFn = void (*)(DecodeParams, uint32_t, int);
 // warp-tile kernel with nwarp warps per CTA, walking with the 12-bit window
 // (walker DF11_WALKER_WINDOW) or the byte-step tables (DF11_WALKER_BYTE_STEP);
 // otherwise the CTA-tile kernel with chunks / cpt decoding threads and a
-// producer warp.
+// producer warp.  counts: the byte-step kernel that reads stored chunk
+// counts instead of counting with a walk.
 struct KernelEntry {
-    int dtype, chunk_bits, chunks, cpt, nwarp, walker;
+    int dtype, chunk_bits, chunks, cpt, nwarp, walker, counts;
     KernelFn fn;
 };
 
-#define DF11_KERNEL(DT, CB, CH)                                          \
-    {DT, CB, CH, 1, 0, DF11_WALKER_WINDOW, &decode_kernel<DT, CB, 1, CH>}, \
-    {                                                                    \
-        DT, CB, CH, 2, 0, DF11_WALKER_WINDOW, &decode_kernel<DT, CB, 2, CH / 2> \
+#define DF11_KERNEL(DT, CB, CH)                                             \
+    {DT, CB, CH, 1, 0, DF11_WALKER_WINDOW, 0, &decode_kernel<DT, CB, 1, CH>}, \
+    {                                                                       \
+        DT, CB, CH, 2, 0, DF11_WALKER_WINDOW, 0, &decode_kernel<DT, CB, 2, CH / 2> \
     }
-#define DF11_WARP_KERNEL(DT, CB)                                             \
-    {DT, CB, 32, 1, 8, DF11_WALKER_WINDOW, &decode_warp_kernel<DT, CB, 8>},   \
-        {DT, CB, 32, 1, 16, DF11_WALKER_WINDOW, &decode_warp_kernel<DT, CB, 16>}, \
-        {DT, CB, 32, 1, 16, DF11_WALKER_BYTE_STEP, &decode_fsm_kernel<DT, CB, 16>}, \
-        {DT, CB, 32, 1, 24, DF11_WALKER_BYTE_STEP, &decode_fsm_kernel<DT, CB, 24>}, \
-    {                                                                        \
-        DT, CB, 32, 1, 32, DF11_WALKER_BYTE_STEP, &decode_fsm_kernel<DT, CB, 32>  \
+#define DF11_WARP_KERNEL(DT, CB)                                                      \
+    {DT, CB, 32, 1, 8, DF11_WALKER_WINDOW, 0, &decode_warp_kernel<DT, CB, 8>},         \
+        {DT, CB, 32, 1, 16, DF11_WALKER_WINDOW, 0, &decode_warp_kernel<DT, CB, 16>},   \
+        {DT, CB, 32, 1, 16, DF11_WALKER_BYTE_STEP, 0, &decode_fsm_kernel<DT, CB, 16, false>}, \
+        {DT, CB, 32, 1, 24, DF11_WALKER_BYTE_STEP, 0, &decode_fsm_kernel<DT, CB, 24, false>}, \
+    {                                                                                 \
+        DT, CB, 32, 1, 32, DF11_WALKER_BYTE_STEP, 0, &decode_fsm_kernel<DT, CB, 32, false>  \
+    }
+#define DF11_COUNTS_KERNEL(DT, CB)                                                   \
+    {DT, CB, 32, 1, 16, DF11_WALKER_BYTE_STEP, 1, &decode_fsm_kernel<DT, CB, 16, true>}, \
+        {DT, CB, 32, 1, 24, DF11_WALKER_BYTE_STEP, 1, &decode_fsm_kernel<DT, CB, 24, true>}, \
+    {                                                                                \
+        DT, CB, 32, 1, 32, DF11_WALKER_BYTE_STEP, 1, &decode_fsm_kernel<DT, CB, 32, true>  \
     }
 
 const KernelEntry kKernels[] = {
+    DF11_COUNTS_KERNEL(0, 128), DF11_COUNTS_KERNEL(1, 128), DF11_COUNTS_KERNEL(0, 64), DF11_COUNTS_KERNEL(1, 64),
     DF11_WARP_KERNEL(0, 128), DF11_WARP_KERNEL(1, 128), DF11_WARP_KERNEL(0, 256), DF11_WARP_KERNEL(1, 256),
     DF11_WARP_KERNEL(0, 64),  DF11_WARP_KERNEL(1, 64),
     DF11_KERNEL(0, 128, 256), DF11_KERNEL(1, 128, 256), DF11_KERNEL(0, 256, 128), DF11_KERNEL(1, 256, 128),
@@ -1471,10 +1540,11 @@ const KernelEntry kKernels[] = {
     DF11_KERNEL(0, 128, 512), DF11_KERNEL(1, 128, 512), DF11_KERNEL(0, 256, 256), DF11_KERNEL(1, 256, 256),
 };
 
-const KernelEntry *find_kernel(int dtype, int chunk_bits, int chunks, int cpt, int nwarp, int walker) {
+const KernelEntry *find_kernel(int dtype, int chunk_bits, int chunks, int cpt, int nwarp, int walker,
+                               int counts = 0) {
     for (const auto &e : kKernels)
         if (e.dtype == dtype && e.chunk_bits == chunk_bits && e.chunks == chunks && e.cpt == cpt &&
-            e.nwarp == nwarp && e.walker == walker)
+            e.nwarp == nwarp && e.walker == walker && e.counts == counts)
             return &e;
     return nullptr;
 }
@@ -1531,6 +1601,7 @@ LaunchStatus build_params(const Blob *const *blobs, void *const *dst, int n, int
     P = DecodeParams{};
     uint64_t tiles = 0, max_span = 0;
     int nt = 0;
+    bool all_counts = true;  // every non-empty image of the launch stores chunk counts
     for (int i = 0; i < n; ++i) {
         if (!blobs[i]) return LaunchStatus::kInvalid;
         const Blob &b = *blobs[i];
@@ -1547,6 +1618,8 @@ LaunchStatus build_params(const Blob *const *blobs, void *const *dst, int n, int
         d.stream = b.dev_image + L.stream;
         d.plane = b.dev_image + L.plane;
         d.gaps = b.dev_image + L.gaps;
+        d.counts = b.chunk_counts ? b.dev_image + L.counts : nullptr;
+        all_counts = all_counts && b.chunk_counts;
         d.out_off = reinterpret_cast<const uint64_t *>(b.dev_image + L.out_off);
         d.dst = dst[i];
         d.n = b.n;
@@ -1559,17 +1632,21 @@ LaunchStatus build_params(const Blob *const *blobs, void *const *dst, int n, int
     if (tiles >= (uint64_t{1} << 31)) return LaunchStatus::kInvalid;
     // kernel: the byte-step walk for warp tiles unless the window walk is asked
     // for, the code has a 1-bit codeword (a byte would end up to 8 codes) or
-    // its tables and the warps' buffers do not fit in shared memory
+    // its tables and the warps' buffers do not fit in shared memory; it reads
+    // the stored chunk counts when every image has them and no count walk is
+    // asked for
     const int rows = b0.cb->fsm_rows;
+    const int use_counts = all_counts && nt > 0 && !opt.count_walk && counts_fit(b0.chunk_bits) ? 1 : 0;
     const KernelEntry *ke = nullptr;
     if (warp_tiles && opt.walker != DF11_WALKER_WINDOW && rows >= 2 && rows <= kFsmMaxRows &&
         (opt.walker == DF11_WALKER_BYTE_STEP || b0.cb->min_len_used >= 2)) {
         const int tries[3] = {32, 24, 16};
         for (int nw : tries) {
             if (opt.warps_per_cta && opt.warps_per_cta != nw) continue;
-            if (make_fsm_plan(b0.chunk_bits, nw, static_cast<uint32_t>(max_span), rows).total > kSmemBudget)
+            if (make_fsm_plan(b0.chunk_bits, nw, static_cast<uint32_t>(max_span), rows, use_counts).total >
+                kSmemBudget)
                 continue;
-            ke = find_kernel(b0.dtype, b0.chunk_bits, 32, 1, nw, DF11_WALKER_BYTE_STEP);
+            ke = find_kernel(b0.dtype, b0.chunk_bits, 32, 1, nw, DF11_WALKER_BYTE_STEP, use_counts);
             if (ke) break;
         }
         if (!ke && opt.walker == DF11_WALKER_BYTE_STEP) return LaunchStatus::kUnsupported;
@@ -1598,7 +1675,7 @@ LaunchStatus build_params(const Blob *const *blobs, void *const *dst, int n, int
     out->ctas_per_sm = opt.ctas_per_sm;
     out->max_ctas = opt.max_ctas;
     if (ke->walker == DF11_WALKER_BYTE_STEP)
-        out->smem = make_fsm_plan(b0.chunk_bits, ke->nwarp, out->max_span, rows).total;
+        out->smem = make_fsm_plan(b0.chunk_bits, ke->nwarp, out->max_span, rows, ke->counts != 0).total;
     else if (warp_tiles)
         out->smem = make_warp_plan(b0.chunk_bits, ke->nwarp, out->max_span, out->n_lut_smem).total;
     else
@@ -1628,6 +1705,7 @@ LaunchStatus shape_for(const Prepared &pp, LaunchShape *sh) {
     sh->block = block;
     sh->smem = static_cast<int>(pp.smem);
     sh->walker = pp.ke->walker;
+    sh->stored_counts = pp.ke->counts;
     return LaunchStatus::kOk;
 }
 

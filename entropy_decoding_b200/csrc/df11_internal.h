@@ -33,6 +33,12 @@
 //     hierarchical tables generalised to every node at a byte boundary.
 //     Row v occupies bytes [v * kFsmRowBytes, (v + 1) * kFsmRowBytes), entry
 //     b the 8 bytes {ctl, syms} at b * 8 within it.
+//   * chunk counts (optional, chunk_bits <= 128): one byte per chunk, the
+//     number of codes that start in its chunk_bits stream bits.  With them a
+//     decoding thread's output position is a warp scan of stored bytes, and
+//     the count walk of the first phase (the two-phase kernel of the DFloat11
+//     Abstract, item (ii)) is not needed.  A chunk of at most 128 bits holds
+//     at most 128 code starts, so the byte never overflows.
 //   * in the device image the stream is stored as 32-bit words whose bit 31
 //     is the earliest stream bit (each 4-byte group of the MSB-first byte
 //     stream reversed), so a word load needs no byte swap.
@@ -67,19 +73,22 @@ constexpr uint64_t kImageAlign = 256;
 constexpr uint64_t kStreamTail = 16;  // zero bytes after the last tile: look-ahead of the last thread
 constexpr uint64_t kPlaneTail = 32;
 constexpr uint64_t kGapsTail = 16;  // readable bytes after the last tile's gaps: the next chunk's gap
+constexpr int kCountsMaxChunkBits = 128;  // chunk counts are stored for chunk_bits up to this
+constexpr uint32_t kImageFlagCounts = 1;  // ImageHeader::flags: the chunk-counts section is present
 
 inline uint64_t align_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
 
 // Offsets of the sections inside one blob's device image.
+// counts == out_off when the image has no chunk counts.
 struct ImageLayout {
-    uint64_t meta, syms, lut, fsm, gaps, out_off, stream, plane, total;
+    uint64_t meta, syms, lut, fsm, gaps, counts, out_off, stream, plane, total;
 };
 
 // Header at offset 0 of every device image (kept for inspection; the kernel
 // takes everything it needs from its launch parameters).
 struct ImageHeader {
     char magic[8];  // "DF11IMG1"
-    uint32_t dtype, chunk_bits, tile_threads, n_luts, fsm_rows, reserved;
+    uint32_t dtype, chunk_bits, tile_threads, n_luts, fsm_rows, flags;  // flags: kImageFlagCounts
     uint64_t n_elems, total_bits, n_tiles, max_span;
     ImageLayout layout;
 };
@@ -90,6 +99,7 @@ struct TensorDesc {
     const uint8_t *stream;
     const uint8_t *plane;
     const uint8_t *gaps;
+    const uint8_t *counts;  // nullptr: the image has no chunk counts
     const uint64_t *out_off;
     void *dst;
     uint64_t n;

@@ -198,6 +198,7 @@ struct PackArgs {
     uint32_t *stream;  // words, earliest bit in bit 31; zeroed
     uint8_t *plane;
     uint8_t *gaps;      // zeroed
+    uint32_t *counts;   // chunk counts as words (byte c at bits 8 * (c % 4) of word c / 4), zeroed; or nullptr
     uint64_t *out_off;  // filled with n
     uint32_t chunk_bits;
     uint64_t tile_bits;
@@ -238,18 +239,32 @@ __global__ void __launch_bounds__(kEncThreads) pack_kernel(const PackArgs A) {
         // previous element's start: from its code length
         uint64_t prev = ~uint64_t{0};
         if (i0 > 0 && c > 0) prev = start - s_len[exponent_at<DT>(A.src, i0 - 1)];
+        // chunk counts: this thread's codes fall in one or two chunks mostly;
+        // one add per run of codes in the same chunk (a chunk of at most 128
+        // bits has at most 128 starts, so the byte never carries into the next)
+        uint64_t run_c = ~uint64_t{0};
+        uint32_t run_n = 0;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             if (j >= c) break;
             const uint32_t len = s_len[e[j]];
             or_code(A.stream, start, s_code[e[j]], len);
             const uint64_t ck = start / cb, pk = prev == ~uint64_t{0} ? ~uint64_t{0} : prev / cb;
+            if (A.counts) {
+                if (ck != run_c) {
+                    if (run_n) atomicAdd(A.counts + (run_c >> 2), run_n << (8u * static_cast<uint32_t>(run_c & 3u)));
+                    run_c = ck;
+                    run_n = 0;
+                }
+                ++run_n;
+            }
             for (uint64_t q = pk + 1; q <= ck; ++q) A.gaps[q] = static_cast<uint8_t>(start - q * cb);
             const uint64_t tk = start / A.tile_bits, ptk = prev == ~uint64_t{0} ? ~uint64_t{0} : prev / A.tile_bits;
             for (uint64_t q = ptk + 1; q <= tk; ++q) A.out_off[q] = i0 + j;
             prev = start;
             start += len;
         }
+        if (A.counts && run_n) atomicAdd(A.counts + (run_c >> 2), run_n << (8u * static_cast<uint32_t>(run_c & 3u)));
         // raw fields
         if constexpr (DT == 0) {
             if (c == 16) {
@@ -378,6 +393,7 @@ std::string encode_device_pack(const EncodeJob &J, uint64_t *scratch, uint64_t t
     meta_only.total_bits = total_bits;
     meta_only.n_tiles = n_tiles;
     meta_only.cb = J.cb;
+    meta_only.chunk_counts = J.chunk_counts && counts_fit(J.chunk_bits);
     write_image_head(meta_only, L, head.data());
     if (cudaMemcpyAsync(image, head.data(), head.size(), cudaMemcpyHostToDevice, s) != cudaSuccess)
         return "table upload failed";
@@ -398,6 +414,7 @@ std::string encode_device_pack(const EncodeJob &J, uint64_t *scratch, uint64_t t
     A.stream = reinterpret_cast<uint32_t *>(image + L.stream);
     A.plane = image + L.plane;
     A.gaps = image + L.gaps;
+    A.counts = meta_only.chunk_counts ? reinterpret_cast<uint32_t *>(image + L.counts) : nullptr;
     A.out_off = out_off;
     A.chunk_bits = static_cast<uint32_t>(J.chunk_bits);
     A.tile_bits = tbits;
@@ -475,6 +492,7 @@ std::string encode_device_noalloc(const EncodeJob &J, uint8_t *image, uint64_t i
     const uint64_t n_chunks = (total + cbits - 1) / cbits;
     meta.n_tiles = (n_chunks + J.tile_threads - 1) / J.tile_threads;
     meta.cb = J.cb;
+    meta.chunk_counts = J.chunk_counts && counts_fit(J.chunk_bits);
     const ImageLayout L = image_layout(meta);
     r->image_bytes = L.total;
     r->total_bits = total;
@@ -489,6 +507,7 @@ std::string encode_device_noalloc(const EncodeJob &J, uint8_t *image, uint64_t i
     h.tile_threads = static_cast<uint32_t>(meta.tile_threads);
     h.n_luts = static_cast<uint32_t>(J.cb->n_luts());
     h.fsm_rows = static_cast<uint32_t>(J.cb->fsm_rows);
+    h.flags = meta.chunk_counts ? kImageFlagCounts : 0u;
     h.n_elems = meta.n;
     h.total_bits = total;
     h.n_tiles = meta.n_tiles;
@@ -521,6 +540,7 @@ std::string encode_device_noalloc(const EncodeJob &J, uint8_t *image, uint64_t i
     A.stream = reinterpret_cast<uint32_t *>(image + L.stream);
     A.plane = image + L.plane;
     A.gaps = image + L.gaps;
+    A.counts = meta.chunk_counts ? reinterpret_cast<uint32_t *>(image + L.counts) : nullptr;
     A.out_off = out_off;
     A.chunk_bits = static_cast<uint32_t>(J.chunk_bits);
     A.tile_bits = cbits * static_cast<uint64_t>(J.tile_threads);

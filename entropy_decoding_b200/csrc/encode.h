@@ -16,6 +16,7 @@ struct EncodeJob {
     uint64_t n = 0;
     int chunk_bits = 128;
     int tile_threads = 32;
+    bool chunk_counts = true;  // write the chunk-counts section (chunk_bits <= 128 only)
 };
 
 uint64_t segments_of(uint64_t n);

@@ -17,6 +17,7 @@ struct DecodeOptions {
     int max_ctas = 0;           // grid cap, 0 = none
     int overlap = 0;            // 1: programmatic dependent launch (no dependency on earlier stream work)
     int diag_expire_waits = 0;  // diagnostics: no copies, every wait runs out after 10 ms
+    int count_walk = 0;         // 1: byte-step walker counts with a walk even when chunk counts are stored
 };
 
 constexpr int kDefaultChunksPerThread = 1;
@@ -26,7 +27,8 @@ struct LaunchShape {
     int grid = 0;
     int block = 0;
     int smem = 0;
-    int walker = 0;  // DF11_WALKER_WINDOW or DF11_WALKER_BYTE_STEP
+    int walker = 0;         // DF11_WALKER_WINDOW or DF11_WALKER_BYTE_STEP
+    int stored_counts = 0;  // 1: output positions from the stored chunk counts
 };
 
 bool kernel_available(int dtype, int chunk_bits, int tile_threads);

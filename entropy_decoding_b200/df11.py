@@ -44,7 +44,8 @@ class BlobInfo(ctypes.Structure):
                 ("n_tiles", ctypes.c_uint64), ("max_span", ctypes.c_uint64), ("stream_bytes", ctypes.c_uint64),
                 ("plane_bytes", ctypes.c_uint64), ("gaps_bytes", ctypes.c_uint64),
                 ("out_off_bytes", ctypes.c_uint64), ("serialized_bytes", ctypes.c_uint64),
-                ("device_bytes", ctypes.c_uint64), ("uncompressed_bytes", ctypes.c_uint64)]
+                ("device_bytes", ctypes.c_uint64), ("uncompressed_bytes", ctypes.c_uint64),
+                ("counts_bytes", ctypes.c_uint64)]
 
     def as_dict(self) -> dict:
         return {k: getattr(self, k) for k, _ in self._fields_}
@@ -58,10 +59,11 @@ class EncodeResult(ctypes.Structure):
 class DecodeOpts(ctypes.Structure):
     _fields_ = [("chunks_per_thread", ctypes.c_int32), ("ctas_per_sm", ctypes.c_int32),
                 ("warps_per_cta", ctypes.c_int32), ("walker", ctypes.c_int32), ("max_ctas", ctypes.c_int32),
-                ("overlap", ctypes.c_int32), ("diag_expire_waits", ctypes.c_int32)]
+                ("overlap", ctypes.c_int32), ("diag_expire_waits", ctypes.c_int32), ("count_walk", ctypes.c_int32)]
 
 
 WALKER_AUTO, WALKER_WINDOW, WALKER_BYTE_STEP = 0, 1, 2
+ENCODE_NO_CHUNK_COUNTS = 1  # encoder flag: leave out the chunk-counts section
 
 
 _P = ctypes.c_void_p
@@ -78,11 +80,12 @@ _SIGS = {
     "df11_codebook_lengths": ([_P, _P], _S),
     "df11_codebook_free": ([_P], None),
     "df11_encode": ([_P, _P, _U64, _PP], _S),
-    "df11_encode_ex": ([_P, _P, _U64, _I, _I, _I, _PP], _S),
+    "df11_encode_ex": ([_P, _P, _U64, _I, _I, _I, _I, _PP], _S),
     "df11_layout_supported": ([_I, _I, _I], _I),
     "df11_blob_free": ([_P], None),
     "df11_blob_get_info": ([_P, ctypes.POINTER(BlobInfo)], _S),
     "df11_blob_sections": ([_P, _PP, _PP, _PP, _PP], _S),
+    "df11_blob_chunk_counts": ([_P, _PP], _S),
     "df11_blob_lengths": ([_P, _P], _S),
     "df11_serialize": ([_P, _P, _U64, ctypes.POINTER(_U64)], _S),
     "df11_deserialize": ([_P, _U64, _PP], _S),
@@ -92,16 +95,16 @@ _SIGS = {
     "df11_decode": ([_PP, _PP, _I, _P, _P], _S),
     "df11_decode_ex": ([_PP, _PP, _I, _P, _P, ctypes.POINTER(DecodeOpts)], _S),
     "df11_decode_launch_shape_ex": ([_PP, _I, ctypes.POINTER(DecodeOpts), ctypes.POINTER(_I), ctypes.POINTER(_I),
-                                     ctypes.POINTER(_I), ctypes.POINTER(_I)], _S),
+                                     ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I)], _S),
     "df11_histogram_device": ([_I, _P, _U64, _P, _P], _S),
     "df11_decode_streamed": ([_PP, _P, _I, _PP, _PP, _I, _U64, _PP, _P, _P, _P], _S),
     "df11_codebook_from_counts": ([_I, _P, _I, _I, _PP], _S),
     "df11_encode_device_scratch_bytes": ([_U64], _U64),
-    "df11_encode_device_begin": ([_P, _P, _U64, _I, _I, _P, _U64, _P, ctypes.POINTER(_U64), _PP], _S),
+    "df11_encode_device_begin": ([_P, _P, _U64, _I, _I, _I, _P, _U64, _P, ctypes.POINTER(_U64), _PP], _S),
     "df11_encode_device_end": ([_P, _P, _U64, _PP], _S),
     "df11_encoding_free": ([_P], None),
     "df11_blob_fetch": ([_P, _P], _S),
-    "df11_encode_device_noalloc": ([_P, _P, _U64, _I, _I, _P, _U64, _P, ctypes.POINTER(EncodeResult)], _S),
+    "df11_encode_device_noalloc": ([_P, _P, _U64, _I, _I, _I, _P, _U64, _P, ctypes.POINTER(EncodeResult)], _S),
     "df11_decode_host": ([_PP, _PP, _PP, _PP, _PP, _I, _P, _P], _S),
     "df11_decode_launch_shape": ([_PP, _I, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I)], _S),
 }
@@ -168,7 +171,8 @@ class Blob:
         return "bf16" if self.info().dtype == DF11_BF16 else "e4m3"
 
     def sections(self) -> dict:
-        """Copies of the host sections: stream, plane, gaps, out_off."""
+        """Copies of the host sections: stream, plane, gaps, out_off, and counts
+        (None when the blob has no chunk counts)."""
         i = self.info()
         ptrs = [ctypes.c_void_p() for _ in range(4)]
         _check(_lib.df11_blob_sections(self._h, *[ctypes.byref(p) for p in ptrs]), "df11_blob_sections")
@@ -181,7 +185,19 @@ class Blob:
         return {"stream": grab(ptrs[0], i.stream_bytes, np.uint8),
                 "plane": grab(ptrs[1], i.plane_bytes, np.uint8),
                 "gaps": grab(ptrs[2], i.gaps_bytes, np.uint8),
-                "out_off": grab(ptrs[3], i.out_off_bytes, np.uint64)}
+                "out_off": grab(ptrs[3], i.out_off_bytes, np.uint64),
+                "counts": self.chunk_counts()}
+
+    def chunk_counts(self):
+        """Copy of the chunk counts, or None when the blob has none."""
+        p = ctypes.c_void_p()
+        _check(_lib.df11_blob_chunk_counts(self._h, ctypes.byref(p)), "df11_blob_chunk_counts")
+        if not p.value:
+            return None
+        n = self.info().counts_bytes
+        if n == 0:
+            return np.zeros(0, np.uint8)
+        return np.ctypeslib.as_array(ctypes.cast(p, ctypes.POINTER(ctypes.c_uint8)), (n,)).copy()
 
     def lengths(self) -> np.ndarray:
         out = np.zeros(256, np.uint8)
@@ -218,12 +234,16 @@ def df11_codebook_from_lengths(dtype: str, lengths) -> Codebook:
     return Codebook(out.value, dtype)
 
 
+def _encode_flags(chunk_counts: bool) -> int:
+    return 0 if chunk_counts else ENCODE_NO_CHUNK_COUNTS
+
+
 def df11_encode(cb: Codebook, x: np.ndarray, chunk_bits: int = 128, tile_threads: int = 32,
-                n_threads: int = 0) -> Blob:
+                n_threads: int = 0, chunk_counts: bool = True) -> Blob:
     a = np.ascontiguousarray(x).reshape(-1)
     out = ctypes.c_void_p()
     _check(_lib.df11_encode_ex(cb.handle, a.ctypes.data if a.size else None, a.size, chunk_bits, tile_threads,
-                               n_threads, ctypes.byref(out)), "df11_encode")
+                               _encode_flags(chunk_counts), n_threads, ctypes.byref(out)), "df11_encode")
     return Blob(out.value)
 
 
@@ -273,8 +293,9 @@ def df11_decode(blobs, dst_ptrs, err_ptr: int | None = None, stream: int = 0):
 
 def df11_decode_ex(blobs, dst_ptrs, err_ptr: int | None = None, stream: int = 0, chunks_per_thread: int = 0,
                    ctas_per_sm: int = 0, warps_per_cta: int = 0, walker: int = 0, max_ctas: int = 0,
-                   overlap: int = 0, diag_expire_waits: int = 0):
-    o = DecodeOpts(chunks_per_thread, ctas_per_sm, warps_per_cta, walker, max_ctas, overlap, diag_expire_waits)
+                   overlap: int = 0, diag_expire_waits: int = 0, count_walk: int = 0):
+    o = DecodeOpts(chunks_per_thread, ctas_per_sm, warps_per_cta, walker, max_ctas, overlap, diag_expire_waits,
+                   count_walk)
     _check(_lib.df11_decode_ex(_ptr_array([b.handle.value for b in blobs]), _ptr_array(dst_ptrs), len(blobs),
                                err_ptr or None, stream or None, ctypes.byref(o)), "df11_decode_ex")
 
@@ -287,16 +308,18 @@ def df11_decode_host(blobs, host_image_ptrs, dev_image_ptrs, dst_dev_ptrs, dst_h
 
 
 def df11_decode_launch_shape(blobs, chunks_per_thread: int = 0, ctas_per_sm: int = 0,
-                             warps_per_cta: int = 0, walker: int = 0, with_walker: bool = False,
-                             max_ctas: int = 0):
+                             warps_per_cta: int = 0, walker: int = 0, with_walk: bool = False,
+                             max_ctas: int = 0, count_walk: int = 0):
     """(grid, block, shared-memory bytes) of the launch df11_decode_ex would
-    make with these options, plus the walk it would use when with_walker."""
-    g, b, s, w = _I(), _I(), _I(), _I()
-    o = DecodeOpts(chunks_per_thread, ctas_per_sm, warps_per_cta, walker, max_ctas, 0, 0)
+    make with these options; with_walk adds the walk it would use and whether
+    it reads the stored chunk counts (0 / 1)."""
+    g, b, s, w, c = _I(), _I(), _I(), _I(), _I()
+    o = DecodeOpts(chunks_per_thread, ctas_per_sm, warps_per_cta, walker, max_ctas, 0, 0, count_walk)
     _check(_lib.df11_decode_launch_shape_ex(_ptr_array([x.handle.value for x in blobs]), len(blobs), ctypes.byref(o),
-                                            ctypes.byref(g), ctypes.byref(b), ctypes.byref(s), ctypes.byref(w)),
+                                            ctypes.byref(g), ctypes.byref(b), ctypes.byref(s), ctypes.byref(w),
+                                            ctypes.byref(c)),
            "df11_decode_launch_shape")
-    return (g.value, b.value, s.value, w.value) if with_walker else (g.value, b.value, s.value)
+    return (g.value, b.value, s.value, w.value, c.value) if with_walk else (g.value, b.value, s.value)
 
 
 def df11_decode_streamed(groups, host_image_ptrs, slot_ptrs, slot_bytes: int, dst_ptrs,
@@ -340,11 +363,13 @@ class Encoding:
 
 
 def df11_encode_device_begin(cb: Codebook, src_ptr: int, n: int, chunk_bits: int = 128, tile_threads: int = 32,
-                             scratch_ptr: int = 0, scratch_cap: int = 0, stream: int = 0) -> Encoding:
+                             scratch_ptr: int = 0, scratch_cap: int = 0, stream: int = 0,
+                             chunk_counts: bool = True) -> Encoding:
     nbytes = _U64()
     out = ctypes.c_void_p()
-    _check(_lib.df11_encode_device_begin(cb.handle, src_ptr or None, n, chunk_bits, tile_threads, scratch_ptr or None,
-                                         scratch_cap, stream or None, ctypes.byref(nbytes), ctypes.byref(out)),
+    _check(_lib.df11_encode_device_begin(cb.handle, src_ptr or None, n, chunk_bits, tile_threads,
+                                         _encode_flags(chunk_counts), scratch_ptr or None, scratch_cap,
+                                         stream or None, ctypes.byref(nbytes), ctypes.byref(out)),
            "df11_encode_device_begin")
     return Encoding(out.value, nbytes.value)
 
@@ -366,14 +391,16 @@ NOALLOC_MAX_ELEMS = (65536 - 163) * 4096
 
 
 def df11_encode_device_noalloc(cb: Codebook, src_ptr: int, n: int, chunk_bits: int, tile_threads: int,
-                               image_ptr: int, image_cap: int, stream: int = 0) -> EncodeResult:
+                               image_ptr: int, image_cap: int, stream: int = 0,
+                               chunk_counts: bool = True) -> EncodeResult:
     """GPU encode for callers that cannot allocate device memory: scratch is a
     static device array of the library, so n is limited to NOALLOC_MAX_ELEMS.
     Raises Df11Error (status DF11_ENOMEM with .result.image_bytes set when
     the image buffer is too small)."""
     r = EncodeResult()
-    st = _lib.df11_encode_device_noalloc(cb.handle, src_ptr or None, n, chunk_bits, tile_threads, image_ptr or None,
-                                         image_cap, stream or None, ctypes.byref(r))
+    st = _lib.df11_encode_device_noalloc(cb.handle, src_ptr or None, n, chunk_bits, tile_threads,
+                                         _encode_flags(chunk_counts), image_ptr or None, image_cap, stream or None,
+                                         ctypes.byref(r))
     if st != DF11_OK:
         e = Df11Error(st, "df11_encode_device_noalloc")
         e.result = r
@@ -396,7 +423,8 @@ def upload(blob: Blob, stream=None):
     return dev
 
 
-def encode_on_device(cb: Codebook, x_dev, chunk_bits: int = 128, tile_threads: int = 32, stream=None) -> Blob:
+def encode_on_device(cb: Codebook, x_dev, chunk_bits: int = 128, tile_threads: int = 32, stream=None,
+                     chunk_counts: bool = True) -> Blob:
     """GPU encode of a torch device tensor (raw uint16 / uint8 bits); scratch
     and the image are allocated with torch.  Returns a blob bound to its image."""
     import torch
@@ -404,7 +432,7 @@ def encode_on_device(cb: Codebook, x_dev, chunk_bits: int = 128, tile_threads: i
     n = x_dev.numel()
     scratch = torch.empty(df11_encode_device_scratch_bytes(n), dtype=torch.uint8, device=x_dev.device)
     enc = df11_encode_device_begin(cb, x_dev.data_ptr(), n, chunk_bits, tile_threads, scratch.data_ptr(),
-                                   scratch.numel(), s)
+                                   scratch.numel(), s, chunk_counts)
     img = torch.empty(enc.image_bytes + 256, dtype=torch.uint8, device=x_dev.device)
     base = img.data_ptr() + (-img.data_ptr()) % 256
     return df11_encode_device_end(enc, base, enc.image_bytes, keep=img)

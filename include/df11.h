@@ -126,18 +126,31 @@ void df11_codebook_free(df11_codebook *cb);
  *            significant bit first (stream bit k = bit 7 - k%8 of byte k/8)
  *   gaps     one byte per chunk: offset of the first code that starts in the
  *            chunk (padded with 0 to whole tiles)
+ *   counts   one byte per chunk: the number of codes that start in the chunk
+ *            (padded with 0 to whole tiles).  Not in the pages' format: it
+ *            lets the decoder place each thread's output with a scan of
+ *            stored bytes instead of a first walk over the codes that only
+ *            counts them (the first of the two phases of the DFloat11
+ *            Abstract, item (ii)).  Costs chunk_bits / 8 : 1 of the stream
+ *            (about 0.17 bits per weight at 128-bit chunks); left out with
+ *            DF11_ENCODE_NO_CHUNK_COUNTS and for 256-bit chunks.
  *   out_off  n_tiles + 1 uint64 values: codes starting before each tile
  * Errors: DF11_EINVAL (bad layout, or a symbol the code does not cover),
  * DF11_ENOMEM. */
 df11_status df11_encode(const df11_codebook *cb, const void *host_src, uint64_t n_elems,
                         df11_blob **out);
 
+/* Flags of df11_encode_ex, df11_encode_device_begin and
+ * df11_encode_device_noalloc (0 = the default layout's sections). */
+#define DF11_ENCODE_NO_CHUNK_COUNTS 1 /* leave out the counts section: the pages' format, smallest size */
+
 /* df11_encode with an explicit layout: chunk_bits in {64, 128, 256},
  * tile_threads (chunks per tile, one out_off entry each) in {32, 128, 256,
- * 512}; n_threads host threads (0 = all cores).
- * df11_decode supports the layouts listed by df11_layout_supported. */
+ * 512}; flags from DF11_ENCODE_*; n_threads host threads (0 = all cores).
+ * df11_decode supports the layouts listed by df11_layout_supported.  Errors
+ * as df11_encode, and DF11_EINVAL for an unknown flag. */
 df11_status df11_encode_ex(const df11_codebook *cb, const void *host_src, uint64_t n_elems,
-                           int chunk_bits, int tile_threads, int n_threads, df11_blob **out);
+                           int chunk_bits, int tile_threads, int flags, int n_threads, df11_blob **out);
 
 /* 1 when df11_decode has a kernel for this (dtype, chunk_bits, tile_threads). */
 int df11_layout_supported(df11_dtype dtype, int chunk_bits, int tile_threads);
@@ -160,6 +173,7 @@ typedef struct {
     uint64_t serialized_bytes;/* size of df11_serialize's output: the container */
     uint64_t device_bytes;    /* size of the device image (df11_blob_device_image) */
     uint64_t uncompressed_bytes;
+    uint64_t counts_bytes;    /* chunk counts: n_tiles * tile_threads, 0 when the blob has none */
 } df11_blob_info;
 
 df11_status df11_blob_get_info(const df11_blob *blob, df11_blob_info *info);
@@ -170,6 +184,11 @@ df11_status df11_blob_get_info(const df11_blob *blob, df11_blob_info *info);
 df11_status df11_blob_sections(const df11_blob *blob, const uint8_t **stream, const uint8_t **plane,
                                const uint8_t **gaps, const uint64_t **out_off);
 
+/* *counts receives a read-only host view of the chunk counts
+ * (info.counts_bytes bytes), or NULL when the blob has none.  DF11_EINVAL as
+ * df11_blob_sections. */
+df11_status df11_blob_chunk_counts(const df11_blob *blob, const uint8_t **counts);
+
 /* Copies the code lengths the blob was encoded with into lengths[0..255]. */
 df11_status df11_blob_lengths(const df11_blob *blob, uint8_t *lengths);
 
@@ -177,8 +196,9 @@ df11_status df11_blob_lengths(const df11_blob *blob, uint8_t *lengths);
  * Container (the offline, on-disk form)
  * ------------------------------------------------------------------ */
 
-/* Writes the container (header with code lengths, gaps, out_off, stream,
- * plane; sections 16-byte aligned) into buf[0..cap).  *used receives
+/* Writes the container (header with code lengths, gaps, chunk counts when
+ * the blob has them, out_off, stream, plane; sections 16-byte aligned) into
+ * buf[0..cap): format version 2 with counts, else version 1.  *used receives
  * info.serialized_bytes.  Errors: DF11_ENOMEM when cap is too small. */
 df11_status df11_serialize(const df11_blob *blob, void *buf, uint64_t cap, uint64_t *used);
 
@@ -195,8 +215,9 @@ df11_status df11_deserialize(const void *buf, uint64_t len, df11_blob **out);
 /* Writes the blob's device image into host memory host_dst[0..cap) (cap >=
  * info.device_bytes; pinned memory makes the later copy asynchronous).  The
  * image is one buffer with 256-byte aligned sections: the decode tables
- * built from the code lengths, gaps, out_off, the stream padded with zeros
- * to whole tiles plus 16 bytes, and the plane padded to 16 bytes plus 32. */
+ * built from the code lengths, gaps, chunk counts (when the blob has them),
+ * out_off, the stream padded with zeros to whole tiles plus 16 bytes, and the
+ * plane padded to 16 bytes plus 32. */
 df11_status df11_blob_device_image(const df11_blob *blob, void *host_dst, uint64_t cap);
 
 /* Records that the blob's device image is at device address dev_image
@@ -232,7 +253,8 @@ typedef struct {
     int32_t warps_per_cta;     /* warp-tile layout (tile_threads 32): warps per CTA; window walker 8 or
                                   16 (0 = 16), byte-step walker 16, 24 or 32 (0 = the most that fit) */
     int32_t walker;            /* warp-tile layout: DF11_WALKER_AUTO (0), DF11_WALKER_WINDOW or
-                                  DF11_WALKER_BYTE_STEP; CTA-tile layouts take 0 or WINDOW only */
+                                  DF11_WALKER_BYTE_STEP; CTA-tile layouts take 0 or WINDOW only.
+                                  The window walk always counts with a first walk */
     int32_t max_ctas;          /* upper bound on the grid (0 = none): fewer persistent CTAs leave
                                   SMs free for work running beside the decode */
     int32_t overlap;           /* 1: the launch reads nothing that the work before it on the
@@ -244,6 +266,10 @@ typedef struct {
                                   the first wait runs out: the launch decodes nothing, sets
                                   DF11_DEV_ERR_TIMEOUT in dev_err_flag and ends (how a stalled
                                   copy is reported, exercised without a fault) */
+    int32_t count_walk;        /* byte-step walker: 0 = place each thread's output with the chunk
+                                  counts when every image of the launch stores them, else walk;
+                                  1 = always walk each chunk once to count its codes first (the
+                                  first phase of the two-phase kernel), ignoring stored counts */
 } df11_decode_opts;
 
 /* How a decoding thread walks its chunk (both give the same output).
@@ -312,10 +338,12 @@ df11_status df11_decode_launch_shape(const df11_blob *const *blobs, int n_blobs,
 
 /* As df11_decode_launch_shape, for the given options (opts may be NULL);
  * *walker (nullable) receives the walk the launch would use,
- * DF11_WALKER_WINDOW or DF11_WALKER_BYTE_STEP. */
+ * DF11_WALKER_WINDOW or DF11_WALKER_BYTE_STEP, and *stored_counts (nullable)
+ * 1 when it places the threads' output with the stored chunk counts, 0 when
+ * it walks to count. */
 df11_status df11_decode_launch_shape_ex(const df11_blob *const *blobs, int n_blobs,
                                         const df11_decode_opts *opts, int *grid, int *block,
-                                        int *smem_bytes, int *walker);
+                                        int *smem_bytes, int *walker, int *stored_counts);
 
 /* ---------------------------------------------------------------------
  * GPU encoder (the offline half, run on the device)
@@ -342,11 +370,11 @@ uint64_t df11_encode_device_scratch_bytes(uint64_t n_elems);
  * and returns the exact device-image size in *image_bytes.  Synchronises
  * `stream` once (to read the stream length back).  src_dev (the raw weights,
  * 16-byte aligned) and scratch_dev (>= df11_encode_device_scratch_bytes,
- * 16-byte aligned) must stay valid until df11_encode_device_end.  Errors:
- * DF11_EINVAL (bad arguments, or an exponent the code does not cover),
- * DF11_ENOMEM (scratch too small), DF11_ECUDA. */
+ * 16-byte aligned) must stay valid until df11_encode_device_end.  flags as
+ * df11_encode_ex.  Errors: DF11_EINVAL (bad arguments, or an exponent the
+ * code does not cover), DF11_ENOMEM (scratch too small), DF11_ECUDA. */
 df11_status df11_encode_device_begin(const df11_codebook *cb, const void *src_dev, uint64_t n_elems,
-                                     int chunk_bits, int tile_threads, void *scratch_dev,
+                                     int chunk_bits, int tile_threads, int flags, void *scratch_dev,
                                      uint64_t scratch_cap, df11_stream stream, uint64_t *image_bytes,
                                      df11_encoding **out);
 
@@ -382,7 +410,8 @@ df11_status df11_blob_fetch(df11_blob *blob, df11_stream stream);
  * writes the same device image, byte for byte, into the caller's image_dev.
  * It calls no cudaMalloc, cudaFree or other allocating routine, on the device
  * or the host.  The caller passes the raw weights (src_dev, 16-byte aligned)
- * and the image buffer (image_dev, 256-byte aligned, image_cap bytes).
+ * and the image buffer (image_dev, 256-byte aligned, image_cap bytes); flags
+ * as df11_encode_ex.
  *
  * Scratch.  Its scratch is one static device array of
  * DF11_NOALLOC_SCRATCH_BYTES, which every GPU that loads the library holds
@@ -418,7 +447,7 @@ typedef struct {
 } df11_encode_result;
 
 df11_status df11_encode_device_noalloc(const df11_codebook *cb, const void *src_dev, uint64_t n_elems,
-                                       int chunk_bits, int tile_threads, void *image_dev,
+                                       int chunk_bits, int tile_threads, int flags, void *image_dev,
                                        uint64_t image_cap, df11_stream stream,
                                        df11_encode_result *result);
 

@@ -75,6 +75,8 @@ def _load():
         lib.oracle_layout.argtypes = [U64, I, I, P, P]
         lib.oracle_aux.argtypes = [P, U64, P, I, I, P, P, P]
         lib.oracle_aux.restype = I
+        lib.oracle_chunk_counts.argtypes = [P, U64, P, I, I, P]
+        lib.oracle_chunk_counts.restype = I
         lib.oracle_decode.argtypes = [P, U64, P, I, U64, U64, P]
         lib.oracle_decode.restype = I
         _lib = lib
@@ -207,6 +209,19 @@ def aux(exps: np.ndarray, lengths: np.ndarray, chunk_bits: int, tile_threads: in
     _check(lib.oracle_aux(_p(exps), exps.size, _p(ln), chunk_bits, tile_threads,
                           _p(gaps), _p(out_off), ctypes.byref(ms)), "aux")
     return gaps[: nt * tile_threads].copy(), out_off, int(ms.value)
+
+
+def chunk_counts(exps: np.ndarray, lengths: np.ndarray, chunk_bits: int, tile_threads: int) -> np.ndarray:
+    """Codes starting in each chunk (n_tiles * tile_threads bytes, 0 past the
+    last chunk): what the first phase of the two-phase kernel counts."""
+    lib = _load()
+    ln = np.zeros(256, np.uint8)
+    ln[: len(lengths)] = lengths
+    exps = np.ascontiguousarray(exps, np.uint8)
+    _, nt = layout(total_bits(exps, ln), chunk_bits, tile_threads)
+    out = np.zeros(max(nt * tile_threads, 1), np.uint8)
+    _check(lib.oracle_chunk_counts(_p(exps), exps.size, _p(ln), chunk_bits, tile_threads, _p(out)), "chunk_counts")
+    return out[: nt * tile_threads].copy()
 
 
 def decode(stream: np.ndarray, total: int, lengths: np.ndarray, start_bit: int, count: int) -> np.ndarray:

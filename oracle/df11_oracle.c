@@ -41,6 +41,8 @@
  *    total_bits) - c*chunk_bits.  Threads are grouped into tiles of
  *    tile_threads chunks; out_off[b] = number of codes starting before bit
  *    b*tile_threads*chunk_bits, for b = 0..n_tiles (out_off[n_tiles] = n).
+ *  - Chunk counts (this implementation's optional container section):
+ *    counts[c] = number of codes whose first bit lies in chunk c.
  *  - Raw fields: BF16 keeps one byte (sign << 7 | 7-bit mantissa) per weight;
  *    E4M3 keeps one nibble (sign << 3 | 3-bit mantissa) per weight, element
  *    2i in the low nibble of byte i.
@@ -443,6 +445,35 @@ int oracle_aux(const uint8_t *exps, uint64_t n, const uint8_t *lengths,
         if (out_off[b + 1] - out_off[b] > ms) ms = out_off[b + 1] - out_off[b];
     *max_span = ms;
     return ORACLE_OK;
+}
+
+/* Chunk counts (a container section of this implementation, not of the
+ * pages' format; it stores what the first of the two phases computes, the
+ * number of codes each thread's chunk holds, so that the decoder needs only
+ * the second): counts[c] = the number of codes whose first bit lies in
+ * [c * chunk_bits, (c + 1) * chunk_bits).  n_tiles * tile_threads entries,
+ * 0 past the last chunk.  Fails when a count does not fit a byte. */
+int oracle_chunk_counts(const uint8_t *exps, uint64_t n, const uint8_t *lengths,
+                        int chunk_bits, int tile_threads, uint8_t *counts)
+{
+    uint64_t total = oracle_total_bits(exps, n, lengths);
+    uint64_t n_chunks, n_tiles;
+    oracle_layout(total, chunk_bits, tile_threads, &n_chunks, &n_tiles);
+    uint64_t *tally = (uint64_t *)calloc(n_chunks ? n_chunks : 1, sizeof(uint64_t));
+    if (!tally) return ORACLE_EINVAL;
+    uint64_t start = 0;
+    for (uint64_t i = 0; i < n; i++) {
+        tally[start / (uint64_t)chunk_bits]++;
+        start += lengths[exps[i]];
+    }
+    int rc = ORACLE_OK;
+    for (uint64_t c = 0; c < n_tiles * (uint64_t)tile_threads; c++) {
+        uint64_t v = c < n_chunks ? tally[c] : 0;
+        if (v > 255) rc = ORACLE_EINVAL;
+        counts[c] = (uint8_t)v;
+    }
+    free(tally);
+    return rc;
 }
 
 /* ------------------------------------------------------------------ */

@@ -21,13 +21,21 @@ def df11():
 
 
 def _roundtrip(df11, oracle_mod, x, dt, chunk_bits=128, tile_threads=32, max_len=0, check_oracle=True, cpt=0,
-               ctas=0, wpc=0, walker=0):
+               ctas=0, wpc=0, walker=0, counts="stored"):
+    """counts: "stored" (default encoding and decode), "walk" (counts stored,
+    the decode told to count with a walk) or "absent" (encoded without)."""
     cb = df11.df11_build_codebook(dt, [x], max_len)
-    blob = df11.df11_encode(cb, x, chunk_bits, tile_threads)
+    blob = df11.df11_encode(cb, x, chunk_bits, tile_threads, chunk_counts=counts != "absent")
+    cw = 1 if counts == "walk" else 0
     (out,), err, guards = decode_gpu(df11, [blob], chunks_per_thread=cpt, ctas_per_sm=ctas, warps_per_cta=wpc,
-                                     walker=walker)
+                                     walker=walker, count_walk=cw)
     assert err == 0
     assert guards
+    if x.size:
+        # the byte-step walk reads the stored counts exactly when they are there and not declined
+        shape = df11.df11_decode_launch_shape([blob], cpt, ctas, wpc, walker, with_walk=True, count_walk=cw)
+        stored = counts == "stored" and chunk_bits <= 128 and shape[3] == df11.WALKER_BYTE_STEP
+        assert shape[4] == int(stored)
     assert out.shape == x.shape
     assert np.array_equal(out, x)
     if check_oracle:
@@ -78,7 +86,10 @@ def test_parity_cta_layouts(df11, oracle_mod, layout, case, cpt):
     _roundtrip(df11, oracle_mod, make(), dt, *layout, cpt=cpt)
 
 
-WALKS = [(1, 8), (1, 16), (2, 16), (2, 24), (2, 32)]  # (walker, warps per CTA)
+# (walker, warps per CTA, chunk counts): the byte-step walk with stored
+# counts, with the count walk asked for, and on images without counts
+WALKS = [(1, 8, "stored"), (1, 16, "stored"), (2, 16, "stored"), (2, 24, "stored"), (2, 32, "stored"),
+         (2, 32, "walk"), (2, 16, "walk"), (2, 32, "absent")]
 
 
 @pytest.mark.parametrize("walk", WALKS)
@@ -88,14 +99,15 @@ WALKS = [(1, 8), (1, 16), (2, 16), (2, 24), (2, 32)]  # (walker, warps per CTA)
 def test_parity_warp_layouts(df11, oracle_mod, layout, case, walk):
     """Warp-tile layouts (one out_off per 32 chunks, warp-shuffle scan), with
     the 12-bit window walk (8 and 16 warps per CTA) and the byte-step walk (16,
-    24 and 32 warps in one CTA per SM).  A 1-bit code (single_symbol) sends
-    every thread of the byte-step walk to the window fallback, random bits
-    send many; both must still be exact."""
+    24 and 32 warps in one CTA per SM), placing the threads' output with the
+    stored chunk counts or with the count walk.  A 1-bit code (single_symbol)
+    sends every thread of the byte-step walk to the window fallback, random
+    bits send many; both must still be exact."""
     dt, make = SMALL[case]
-    walker, wpc = walk
+    walker, wpc, counts = walk
     x = make()
     try:
-        _roundtrip(df11, oracle_mod, x, dt, *layout, wpc=wpc, walker=walker)
+        _roundtrip(df11, oracle_mod, x, dt, *layout, wpc=wpc, walker=walker, counts=counts)
     except df11.Df11Error as e:
         # the byte-step walk asked for with a warp count whose buffers do not
         # fit beside the tables (64-row tables of codes over all 256
@@ -104,11 +116,11 @@ def test_parity_warp_layouts(df11, oracle_mod, layout, case, walk):
         if not (walker == 2 and e.status == df11.DF11_EUNSUPPORTED):
             raise
         try:
-            _roundtrip(df11, oracle_mod, x, dt, *layout, walker=walker)
+            _roundtrip(df11, oracle_mod, x, dt, *layout, walker=walker, counts=counts)
         except df11.Df11Error as e2:
             if e2.status != df11.DF11_EUNSUPPORTED:
                 raise
-            _roundtrip(df11, oracle_mod, x, dt, *layout)
+            _roundtrip(df11, oracle_mod, x, dt, *layout, counts=counts)
 
 
 @pytest.mark.parametrize("ctas", [1, 2])
@@ -160,7 +172,7 @@ def test_batched_block_launch_scaled(df11, oracle_mod):
 
 @pytest.mark.parametrize("max_ctas", [1, 3])
 @pytest.mark.parametrize("chunk_bits", [64, 128, 256])
-@pytest.mark.parametrize("walker", [1, 2])
+@pytest.mark.parametrize("walker", [1, 2, "2_walk"])
 def test_long_runs_across_tensors(df11, oracle_mod, walker, chunk_bits, max_ctas):
     """A capped grid: every warp of the byte-step kernel decodes a long run of
     consecutive tiles that crosses tensor boundaries, so unfinished output
@@ -172,7 +184,10 @@ def test_long_runs_across_tensors(df11, oracle_mod, walker, chunk_bits, max_ctas
     xs.insert(2, g.tensors[0].bits[:31])
     cb = df11.df11_build_codebook("bf16", xs)
     blobs = [df11.df11_encode(cb, x, chunk_bits, 32) for x in xs]
-    outs, err, guards = decode_gpu(df11, blobs, walker=walker, warps_per_cta=16, max_ctas=max_ctas)
+    count_walk = 1 if walker == "2_walk" else 0
+    walker = 2 if walker == "2_walk" else walker
+    outs, err, guards = decode_gpu(df11, blobs, walker=walker, warps_per_cta=16, max_ctas=max_ctas,
+                                   count_walk=count_walk)
     assert err == 0 and guards
     lengths = cb.lengths()
     for x, out in zip(xs, outs):
@@ -280,17 +295,22 @@ def test_corrupted_device_data_sets_error_flag(df11):
     n = blob.info().device_bytes
     img = np.zeros(n, np.uint8)
     df11.df11_blob_device_image(blob, img.ctypes.data, n)
-    # layout offsets in the header: meta, syms, lut, fsm, gaps, out_off, ...
+    # layout offsets in the header: meta, syms, lut, fsm, gaps, counts, out_off, ...
     fsm_at = struct.unpack_from("<Q", img.tobytes(), 64 + 8 * 3)[0]
     gaps_at = struct.unpack_from("<Q", img.tobytes(), 64 + 8 * 4)[0]
-    out_off_at = struct.unpack_from("<Q", img.tobytes(), 64 + 8 * 5)[0]
+    counts_at = struct.unpack_from("<Q", img.tobytes(), 64 + 8 * 5)[0]
+    out_off_at = struct.unpack_from("<Q", img.tobytes(), 64 + 8 * 6)[0]
     rng = np.random.default_rng(7)
-    for what in ("out_off", "gap", "fsm"):
+    for what in ("out_off", "gap", "fsm", "count_sum", "count_big"):
         bad = img.copy()
         if what == "out_off":
             bad[out_off_at + 8 * 3: out_off_at + 8 * 4] = np.frombuffer(struct.pack("<Q", 10 ** 12), np.uint8)
         elif what == "gap":
             bad[gaps_at + 5] = (int(bad[gaps_at + 5]) + 3) % 32
+        elif what == "count_sum":  # a tile's counts no longer add up to its span
+            bad[counts_at + 40] += 1
+        elif what == "count_big":  # far more codes than the chunk holds, and a wrong sum
+            bad[counts_at + 70] = 255
         else:  # random counts, masks, symbols and rows in the first two transition rows
             bad[fsm_at: fsm_at + 4096] = rng.integers(0, 256, 4096, dtype=np.uint8)
         dev = torch.from_numpy(bad).cuda()
@@ -306,6 +326,8 @@ def test_corrupted_device_data_sets_error_flag(df11):
         assert (g[:guard] == 0xA5).all() and (g[guard + nbytes:] == 0xA5).all()
         if what == "out_off":
             assert e & df11.DEV_ERR_AUX
+        if what.startswith("count"):
+            assert e & df11.DEV_ERR_SPAN
         if what == "fsm":
             # a walk that meets a damaged row either falls back to the window
             # walk (exact output) or miscounts (flagged): never silent
@@ -313,6 +335,67 @@ def test_corrupted_device_data_sets_error_flag(df11):
         # a shifted gap is caught when it changes the tile's code count; when
         # the parse resynchronises to the same count the output is wrong but
         # still inside the destination, which is what is checked above
+
+
+def _decode_bound_image(df11, blob, img, guard=64, **opts):
+    """Binds the blob to a device copy of img (no re-upload) and decodes it
+    into a buffer with guard bytes: (output bits, error word, guards intact)."""
+    dev = torch.from_numpy(img).cuda()
+    df11.df11_blob_bind(blob, dev.data_ptr(), img.size, keep=dev)
+    nbytes = 2 * blob.info().n_elems
+    buf = torch.full((nbytes + 2 * guard,), 0xA5, dtype=torch.uint8, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    df11.df11_decode_ex([blob], [buf.data_ptr() + guard], err.data_ptr(), **opts)
+    torch.cuda.synchronize()
+    g = buf.cpu().numpy()
+    ok = bool((g[:guard] == 0xA5).all() and (g[guard + nbytes:] == 0xA5).all())
+    return g[guard:guard + nbytes].view(np.uint16), int(err.item()), ok
+
+
+@pytest.mark.parametrize("count_walk", [0, 1])
+def test_moved_chunk_count_is_caught_and_contained(df11, oracle_mod, count_walk):
+    """One code moved between two chunk counts of tile 3 (the tile's sum, and
+    so every other thread's position, unchanged): with stored counts the two
+    threads' walks disagree with their counts, the launch flags
+    DF11_DEV_ERR_SPAN, and every weight outside tile 3's range is still exact
+    (the damaged tile's buffer is cleared, nothing carries over).  With the
+    count walk the stored counts are not read: exact, no flag."""
+    import struct
+    x = synth.single_matrix(6)[0].tensors[0].bits
+    blob = df11.df11_encode(df11.df11_build_codebook("bf16", [x]), x)
+    n = blob.info().device_bytes
+    img = np.zeros(n, np.uint8)
+    df11.df11_blob_device_image(blob, img.ctypes.data, n)
+    counts_at = struct.unpack_from("<Q", img.tobytes(), 64 + 8 * 5)[0]
+    t, j = 3, 5
+    c = counts_at + 32 * t + j
+    assert img[c] > 0
+    img[c] -= 1
+    img[c + 1] += 1
+    out, err, guards = _decode_bound_image(df11, blob, img, count_walk=count_walk)
+    assert guards
+    if count_walk:
+        assert err == 0 and np.array_equal(out, x)
+        return
+    assert err & df11.DEV_ERR_SPAN
+    oo = blob.sections()["out_off"].astype(np.int64)
+    assert np.array_equal(out[: oo[t]], x[: oo[t]])
+    assert np.array_equal(out[oo[t + 1]:], x[oo[t + 1]:])
+
+
+def test_launch_mixing_images_with_and_without_counts(df11, oracle_mod):
+    """One launch over images with and without chunk counts: the byte-step
+    kernel counts with a walk for all of them; exact output."""
+    g = synth.transformer_block(2)[0]
+    xs = [t.bits[: 200000 + 17 * i] for i, t in enumerate(g.tensors[:4])]
+    cb = df11.df11_build_codebook("bf16", xs)
+    blobs = [df11.df11_encode(cb, x, chunk_counts=i % 2 == 0) for i, x in enumerate(xs)]
+    outs, err, guards = decode_gpu(df11, blobs)
+    assert err == 0 and guards
+    for x, o in zip(xs, outs):
+        assert np.array_equal(o, x)
+    assert df11.df11_decode_launch_shape(blobs, with_walk=True)[3:] == (df11.WALKER_BYTE_STEP, 0)
+    assert df11.df11_decode_launch_shape(blobs[::2], with_walk=True)[3:] == (df11.WALKER_BYTE_STEP, 1)
 
 
 def test_transition_rows_past_the_table_are_dead(df11):
@@ -374,19 +457,22 @@ def test_launch_shape_is_persistent(df11):
     assert b8 == 8 * 32 and g8 == sms
     g24, b24, s24 = df11.df11_decode_launch_shape([blob], warps_per_cta=24, walker=df11.WALKER_BYTE_STEP)
     assert b24 == 24 * 32 and g24 == sms and s24 >= 2 * 2048  # at least the root and the dead row
-    assert df11.df11_decode_launch_shape([blob], with_walker=True)[3] == df11.WALKER_BYTE_STEP
+    assert df11.df11_decode_launch_shape([blob], with_walk=True)[3:] == (df11.WALKER_BYTE_STEP, 1)
+    assert df11.df11_decode_launch_shape([blob], with_walk=True, count_walk=1)[3:] == (df11.WALKER_BYTE_STEP, 0)
+    # stored counts leave out the control-word copy of the tables: less shared memory
+    assert df11.df11_decode_launch_shape([blob], count_walk=1)[2] > smem
     # a 1-bit codeword: automatic choice is the window walk
     one = synth.constant_bf16(5000, 0.5)
     b1bit = df11.df11_encode(df11.df11_build_codebook("bf16", [one]), one)
     df11.upload(b1bit)
-    assert df11.df11_decode_launch_shape([b1bit], with_walker=True)[3] == df11.WALKER_WINDOW
+    assert df11.df11_decode_launch_shape([b1bit], with_walk=True)[3:] == (df11.WALKER_WINDOW, 0)
     cta = df11.df11_encode(df11.df11_build_codebook("bf16", [x]), x, 128, 256)
     df11.upload(cta)
     g1, b1, _ = df11.df11_decode_launch_shape([cta])
     assert b1 == 256 + 32  # CTA tiles: one chunk per decoding thread plus the producer warp
     g2, b2, _ = df11.df11_decode_launch_shape([cta], chunks_per_thread=2, ctas_per_sm=1)
     assert b2 == 256 // 2 + 32 and g2 == min(sms, cta.info().n_tiles)
-    assert df11.df11_decode_launch_shape([cta], with_walker=True)[3] == df11.WALKER_WINDOW
+    assert df11.df11_decode_launch_shape([cta], with_walk=True)[3:] == (df11.WALKER_WINDOW, 0)
     with pytest.raises(df11.Df11Error):
         df11.df11_decode_launch_shape([cta], walker=df11.WALKER_BYTE_STEP)
     assert 0 < smem <= 227 * 1024

@@ -62,17 +62,21 @@ def test_histogram_matches_oracle(df11, oracle_mod, case):
     assert np.array_equal(cb.lengths(), oracle_mod.build_lengths([x], dt))
 
 
+@pytest.mark.parametrize("counts", [True, False])
 @pytest.mark.parametrize("layout", [(128, 32), (128, 256), (64, 512), (256, 128)])
 @pytest.mark.parametrize("case", list(CASES))
-def test_device_image_equals_host_image(df11, case, layout):
+def test_device_image_equals_host_image(df11, case, layout, counts):
+    """Byte-identical images from the GPU and host encoders, with and without
+    the chunk-counts section (the GPU adds each thread's run of code starts
+    per chunk into the section with atomics)."""
     dt, make = CASES[case]
     x = make()
     cb = df11.df11_build_codebook(dt, [x])
-    host = df11.df11_encode(cb, x, *layout)
+    host = df11.df11_encode(cb, x, *layout, chunk_counts=counts)
     n = host.info().device_bytes
     want = np.zeros(n, np.uint8)
     df11.df11_blob_device_image(host, want.ctypes.data, n)
-    dev = df11.encode_on_device(cb, _dev(x), *layout)
+    dev = df11.encode_on_device(cb, _dev(x), *layout, chunk_counts=counts)
     torch.cuda.synchronize()
     assert dev.info().device_bytes == n
     assert dev.info().max_span == host.info().max_span
@@ -102,6 +106,8 @@ def test_device_encoded_blob_decodes_and_fetches(df11, oracle_mod, case):
     assert np.array_equal(sec["plane"], o.plane)
     assert np.array_equal(sec["gaps"], o.gaps)
     assert np.array_equal(sec["out_off"], o.out_off)
+    exps, _ = oracle_mod.split(x, dt)
+    assert np.array_equal(sec["counts"], oracle_mod.chunk_counts(exps, cb.lengths(), 128, 32))
     assert df11.df11_serialize(blob) == df11.df11_serialize(df11.df11_encode(cb, x))
 
 

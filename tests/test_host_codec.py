@@ -60,6 +60,12 @@ def test_lengths_and_sections_match_oracle(df11, oracle_mod, case):
         assert np.array_equal(s["plane"], o.plane)
         assert np.array_equal(s["gaps"], o.gaps)
         assert np.array_equal(s["out_off"], o.out_off)
+        exps, _ = oracle_mod.split(x, dt)
+        if chunk_bits <= 128:  # counts are stored up to 128-bit chunks
+            assert np.array_equal(s["counts"], oracle_mod.chunk_counts(exps, want, chunk_bits, tile_threads))
+        else:
+            assert s["counts"] is None
+        assert df11.df11_encode(cb, x, chunk_bits, tile_threads, chunk_counts=False).sections()["counts"] is None
 
 
 def test_shared_codebook_over_a_group(df11, oracle_mod):
@@ -92,12 +98,12 @@ def test_fibonacci_34_reaches_32_bit_codes(df11, oracle_mod):
 def _image_layout(img: bytes):
     magic = img[:8]
     assert magic == b"DF11IMG1"
-    dtype, chunk, tile, n_luts, fsm_rows, _ = struct.unpack_from("<6I", img, 8)
+    dtype, chunk, tile, n_luts, fsm_rows, flags = struct.unpack_from("<6I", img, 8)
     n, total, n_tiles, max_span = struct.unpack_from("<4Q", img, 32)
-    keys = ["meta", "syms", "lut", "fsm", "gaps", "out_off", "stream", "plane", "total"]
-    lay = dict(zip(keys, struct.unpack_from("<9Q", img, 64)))
-    return dict(dtype=dtype, chunk=chunk, tile=tile, n_luts=n_luts, fsm_rows=fsm_rows, n=n, total_bits=total,
-                n_tiles=n_tiles, max_span=max_span, **lay)
+    keys = ["meta", "syms", "lut", "fsm", "gaps", "counts", "out_off", "stream", "plane", "total"]
+    lay = dict(zip(keys, struct.unpack_from("<10Q", img, 64)))
+    return dict(dtype=dtype, chunk=chunk, tile=tile, n_luts=n_luts, fsm_rows=fsm_rows, flags=flags, n=n,
+                total_bits=total, n_tiles=n_tiles, max_span=max_span, **lay)
 
 
 def _image(df11, blob):
@@ -257,6 +263,25 @@ def test_serialize_roundtrip_and_size(df11, oracle_mod):
         assert np.array_equal(s1[k], s2[k])
     assert np.array_equal(b2.lengths(), blob.lengths())
     assert df11.df11_serialize(b2) == data
+    assert struct.unpack_from("<I", data, 8)[0] == 2  # version 2: with chunk counts
+    # without counts: version 1, the pages' sections only, smaller by the counts
+    bare = df11.df11_encode(cb, x, chunk_counts=False)
+    d1 = df11.df11_serialize(bare)
+    assert struct.unpack_from("<II", d1, 8)[0] == 1 and struct.unpack_from("<I", d1, 60)[0] == 0
+    assert 0 < len(data) - len(d1) <= info.counts_bytes + 16
+    b1 = df11.df11_deserialize(d1)
+    assert b1.sections()["counts"] is None and b1.info().counts_bytes == 0
+    assert df11.df11_serialize(b1) == d1
+
+
+def _container_offsets(info, counts: bool):
+    """Section offsets of a serialized blob: 64-byte header, 256 code lengths,
+    then gaps, counts (version 2), out_off, each 16-byte aligned."""
+    up = lambda v: (v + 15) // 16 * 16
+    gaps = up(64 + 256)
+    cnt = up(gaps + info.gaps_bytes)
+    oo = up(cnt + (info.gaps_bytes if counts else 0))
+    return gaps, cnt, oo
 
 
 def test_deserialize_rejects_corruption(df11):
@@ -277,11 +302,31 @@ def test_deserialize_rejects_corruption(df11):
     bad = bytearray(good); bad[16] ^= 1; rejected(bad)         # element count
     lengths_off = 64
     bad = bytearray(good); bad[lengths_off + 120] = 1; rejected(bad)  # Kraft sum > 1
-    gaps_off = (64 + 256 + 15) // 16 * 16
+    gaps_off, cnt_off, oo = _container_offsets(info, True)
     bad = bytearray(good); bad[gaps_off + 3] = 200; rejected(bad)     # gap out of range
-    oo = (gaps_off + info.gaps_bytes + 15) // 16 * 16
     bad = bytearray(good); struct.pack_into("<Q", bad, oo + 8 * 2, 0); rejected(bad)  # out_off not monotone
     bad = bytearray(good); struct.pack_into("<Q", bad, oo, 5); rejected(bad)          # out_off[0] != 0
+    # chunk counts: a tile whose counts no longer add up to its span, a count
+    # above the chunk's bits, a count in a padding chunk
+    bad = bytearray(good); bad[cnt_off + 5] += 1; rejected(bad)
+    bad = bytearray(good)
+    excess = 200 - bad[cnt_off + 5]
+    bad[cnt_off + 5] = 200  # keep the tile's sum: take the excess from the chunks after it
+    for j in range(6, 32):
+        take = min(excess, bad[cnt_off + j])
+        bad[cnt_off + j] -= take
+        excess -= take
+    assert excess == 0
+    rejected(bad)
+    n_chunks = -(-info.total_bits // info.chunk_bits)
+    if n_chunks < info.gaps_bytes:
+        bad = bytearray(good); bad[cnt_off + info.gaps_bytes - 1] = 1; rejected(bad)
+    # flags: none allowed in version 1, no unknown ones in version 2
+    bad = bytearray(good); struct.pack_into("<I", bad, 60, 3); rejected(bad)
+    bare = bytearray(df11.df11_serialize(df11.df11_encode(cb, x, chunk_counts=False)))
+    bad = bytearray(bare); struct.pack_into("<I", bad, 60, 1); rejected(bad)
+    _, _, oo1 = _container_offsets(info, False)
+    bad = bytearray(bare); struct.pack_into("<Q", bad, oo1, 5); rejected(bad)
     with pytest.raises(df11.Df11Error):
         df11.df11_deserialize(b"")
 
@@ -349,14 +394,24 @@ def test_device_image_layout(df11):
     lay = _image_layout(img.tobytes()[:256])
     info = blob.info()
     assert lay["total"] == info.device_bytes == img.size
-    for k in ("meta", "syms", "lut", "fsm", "gaps", "out_off", "stream", "plane"):
+    for k in ("meta", "syms", "lut", "fsm", "gaps", "counts", "out_off", "stream", "plane"):
         assert lay[k] % 256 == 0
     assert lay["gaps"] - lay["fsm"] >= lay["fsm_rows"] * 2048
     # the gaps section keeps 16 zero bytes after the last tile's gaps
     ng = info.n_tiles * info.tile_threads
-    assert lay["out_off"] - lay["gaps"] >= ng + 16
+    assert lay["counts"] - lay["gaps"] >= ng + 16
     assert not img[lay["gaps"] + ng: lay["gaps"] + ng + 16].any()
+    # chunk counts (default layout): one byte per chunk, as the blob holds them
     s = blob.sections()
+    assert lay["flags"] == 1 and info.counts_bytes == ng
+    assert lay["out_off"] - lay["counts"] >= ng
+    assert np.array_equal(img[lay["counts"]:lay["counts"] + ng], s["counts"])
+    # without them the section is empty and the flag clear
+    bare = df11.df11_encode(cb, x, chunk_counts=False)
+    lay0 = _image_layout(_image(df11, bare).tobytes()[:256])
+    assert lay0["flags"] == 0 and lay0["counts"] == lay0["out_off"] and bare.info().counts_bytes == 0
+    assert bare.sections()["counts"] is None
+    assert bare.info().device_bytes < info.device_bytes
     tile_bytes = info.chunk_bits // 8 * info.tile_threads
     stream = img[lay["stream"]:lay["plane"]]
     words = stream[: (stream.size // 4) * 4].reshape(-1, 4)[:, ::-1].reshape(-1)  # back to MSB-first bytes

@@ -318,6 +318,46 @@ def test_aux_matches_independent_walk(oracle_mod, chunk_bits, tile_threads):
     assert c.max_span == int(np.diff(c.out_off.astype(np.int64)).max())
 
 
+@pytest.mark.parametrize("chunk_bits,tile_threads", [(128, 32), (64, 128), (32, 8), (128, 256)])
+def test_chunk_counts_match_independent_tally(oracle_mod, chunk_bits, tile_threads):
+    """Codes per chunk against a tally of the code start positions by chunk
+    (np.bincount over start // chunk_bits), and each tile's sum against
+    out_off's difference (a second walk of the oracle, over tile bounds)."""
+    x = synth.heavy_tail_matrix(0)[0].tensors[0].bits[:300000]
+    c = oracle_mod.compress(x, "bf16", chunk_bits=chunk_bits, tile_threads=tile_threads)
+    exps, _ = oracle_mod.split(x, "bf16")
+    got = oracle_mod.chunk_counts(exps, c.lengths, chunk_bits, tile_threads)
+    assert len(got) == c.n_tiles * tile_threads
+    lens = c.lengths[exps].astype(np.int64)
+    starts = np.concatenate([[0], np.cumsum(lens)[:-1]])
+    want = np.bincount(starts // chunk_bits, minlength=len(got))
+    assert np.array_equal(got.astype(np.int64), want)
+    sums = got.astype(np.int64).reshape(-1, tile_threads).sum(axis=1)
+    assert np.array_equal(sums, np.diff(c.out_off.astype(np.int64)))
+    n_chunks = -(-c.total_bits // chunk_bits)
+    assert np.all(got[n_chunks:] == 0) and np.all(got[: n_chunks - 1] > 0)
+
+
+def test_chunk_counts_closed_form_one_bit_codes(oracle_mod):
+    """A constant tensor has one symbol, coded with 1 bit: chunk c holds
+    min(chunk_bits, n - c * chunk_bits) codes.  At 256-bit chunks a full chunk
+    holds 256 codes, more than a byte: the oracle refuses."""
+    n = 1000
+    x = synth.constant_bf16(n, 1.0)
+    exps, _ = oracle_mod.split(x, "bf16")
+    lengths = oracle_mod.build_lengths([x], "bf16")
+    assert int(lengths.max()) == 1
+    for cb_bits, tt in [(64, 4), (128, 32), (32, 8)]:
+        got = oracle_mod.chunk_counts(exps, lengths, cb_bits, tt).astype(np.int64)
+        n_chunks = -(-n // cb_bits)
+        want = np.zeros(len(got), np.int64)
+        want[:n_chunks] = cb_bits
+        want[n_chunks - 1] = n - (n_chunks - 1) * cb_bits
+        assert np.array_equal(got, want)
+    with pytest.raises(oracle_mod.OracleError):
+        oracle_mod.chunk_counts(exps, lengths, 256, 4)
+
+
 def test_decode_at_sampled_positions(oracle_mod):
     x = synth.single_matrix(3)[0].tensors[0].bits[:100000]
     c = oracle_mod.compress(x, "bf16")

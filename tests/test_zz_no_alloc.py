@@ -33,9 +33,9 @@ def _aligned(nbytes):
     return buf, buf.data_ptr() + off, off
 
 
-def _reference_image(df11, cb, xd, chunk_bits, tile_threads):
+def _reference_image(df11, cb, xd, chunk_bits, tile_threads, counts=True):
     """Image and info from the allocating GPU encoder."""
-    blob = df11.encode_on_device(cb, xd, chunk_bits, tile_threads)
+    blob = df11.encode_on_device(cb, xd, chunk_bits, tile_threads, chunk_counts=counts)
     torch.cuda.synchronize()
     info = blob.info()
     keep = blob._keep
@@ -43,17 +43,18 @@ def _reference_image(df11, cb, xd, chunk_bits, tile_threads):
     return blob, info, keep[off:off + info.device_bytes].cpu().numpy()
 
 
-def _noalloc_image(df11, cb, xd, chunk_bits, tile_threads, cap):
+def _noalloc_image(df11, cb, xd, chunk_bits, tile_threads, cap, counts=True):
     buf, ptr, off = _aligned(cap)
-    r = df11.df11_encode_device_noalloc(cb, xd.data_ptr(), xd.numel(), chunk_bits, tile_threads, ptr, cap)
+    r = df11.df11_encode_device_noalloc(cb, xd.data_ptr(), xd.numel(), chunk_bits, tile_threads, ptr, cap,
+                                        chunk_counts=counts)
     return buf, ptr, r, buf[off:off + r.image_bytes].cpu().numpy()
 
 
-def _check_against_reference(df11, dt, x, chunk_bits=128, tile_threads=32):
+def _check_against_reference(df11, dt, x, chunk_bits=128, tile_threads=32, counts=True):
     cb = df11.df11_build_codebook(dt, [x])
     xd = _dev(x)
-    blob, info, want = _reference_image(df11, cb, xd, chunk_bits, tile_threads)
-    buf, ptr, r, got = _noalloc_image(df11, cb, xd, chunk_bits, tile_threads, info.device_bytes + 4096)
+    blob, info, want = _reference_image(df11, cb, xd, chunk_bits, tile_threads, counts)
+    buf, ptr, r, got = _noalloc_image(df11, cb, xd, chunk_bits, tile_threads, info.device_bytes + 4096, counts)
     assert r.image_bytes == info.device_bytes
     assert r.total_bits == info.total_bits
     assert r.n_tiles == info.n_tiles
@@ -82,6 +83,13 @@ def test_two_calls_in_a_row_match_allocating_encoder(df11):
 def test_every_call_in_sequence_matches(df11):
     for dt, make, cbits, tt in CALLS + CALLS[::-1]:
         _check_against_reference(df11, dt, make(), cbits, tt)
+
+
+def test_without_chunk_counts_matches(df11):
+    """The layout without the chunk-counts section, after a call with it."""
+    x = synth.heavy_tail_matrix(3)[0].tensors[0].bits[: 2 * 10 ** 6 + 9]
+    _check_against_reference(df11, "bf16", x)
+    _check_against_reference(df11, "bf16", x, counts=False)
 
 
 def test_same_input_twice_gives_same_image(df11):
