@@ -33,6 +33,7 @@
 
 #include <cstdint>
 #include <mutex>
+#include <utility>
 
 #include "df11.h"
 #include "launch.h"
@@ -525,6 +526,22 @@ __device__ __forceinline__ uint2 ld_global_stream_v2(const void *p) {
     return v;
 }
 
+// The same load and the 16-byte store at a constant offset OFF from p (the
+// offset is part of the instruction: one address register serves every round).
+template <int OFF>
+__device__ __forceinline__ uint2 ld_global_stream_v2_at(const void *p) {
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2+%3];" : "=r"(v.x), "=r"(v.y) : "l"(p), "n"(OFF));
+    return v;
+}
+
+template <int OFF>
+__device__ __forceinline__ void st_global_v4_at(void *p, uint4 v) {
+    asm volatile("st.global.v4.u32 [%0+%1], {%2, %3, %4, %5};" ::"l"(p), "n"(OFF), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w)
+                 : "memory");
+}
+
 template <int DT>
 __device__ __noinline__ void store_partial_half(uint8_t *out, uint4 a, uint32_t e0, uint32_t lo, uint32_t hi) {
     const uint32_t wv[4] = {a.x, a.y, a.z, a.w};
@@ -564,6 +581,40 @@ __device__ __forceinline__ void merge_half(uint2 p2, uint32_t j, uint8_t *s_exps
     constexpr uint32_t HALF = DT == 0 ? 8u : 16u;
     if (!PARTIAL || (e0 >= lo && e0 + HALF <= hi)) st_global_v4(out, a);
     else store_partial_half<DT>(out, a, e0, lo, hi);
+}
+
+// Round U (>= 1) of the merge for a lane: half j = lane + 32 U, whole (no
+// piecewise store).  x_l and out_l are the lane's round-0 addresses in the
+// exponent buffer and the tile's output.
+template <int DT, int U>
+__device__ __forceinline__ void merge_half_round(uint2 p2, uint8_t *x_l, uint8_t *out_l) {
+    uint4 a;
+    if constexpr (DT == 0) {
+        uint2 *xp = reinterpret_cast<uint2 *>(x_l + 256 * U);
+        const uint2 x2 = *xp;
+        *xp = make_uint2(0, 0);
+        merge_bf16x4(p2.x, x2.x, a.x, a.y);
+        merge_bf16x4(p2.y, x2.y, a.z, a.w);
+    } else {
+        uint4 *xp = reinterpret_cast<uint4 *>(x_l + 512 * U);
+        const uint4 x4 = *xp;
+        *xp = make_uint4(0, 0, 0, 0);
+        merge_e4m3x8(p2.x, x4.x, x4.y, a.x, a.y);
+        merge_e4m3x8(p2.y, x4.z, x4.w, a.z, a.w);
+    }
+    st_global_v4_at<512 * U>(out_l, a);
+}
+
+template <int DT, int... U>
+__device__ __forceinline__ void merge_rounds(const uint2 *pre, uint32_t lane, uint32_t nh, uint8_t *x_l, uint8_t *out_l,
+                                             std::integer_sequence<int, U...>) {
+    ((lane + 32u * (U + 1) < nh ? merge_half_round<DT, U + 1>(pre[U + 1], x_l, out_l) : (void)0), ...);
+}
+
+template <int... U>
+__device__ __forceinline__ void prefetch_halves(uint2 *pre, const uint8_t *pl, uint32_t lane, uint32_t nhalf,
+                                                std::integer_sequence<int, U...>) {
+    ((lane + 32u * U < nhalf ? (void)(pre[U] = ld_global_stream_v2_at<256 * U>(pl)) : (void)0), ...);
 }
 
 // ------------------------------------------------------------------ kernel
@@ -1102,6 +1153,22 @@ __device__ __forceinline__ uint32_t byte_step_count(const uint32_t (&w)[CB / 32 
     return cnt >> 24;
 }
 
+// Puts symbol bytes sy (c8 / 8 of them, unused bytes zero) after the f8 / 8
+// pending bytes of acc; a completed word goes to byte address wp.
+__device__ __forceinline__ void emit_word(uint32_t sy, uint32_t c8, uint32_t &acc, uint32_t &wp, uint32_t &f8) {
+    const uint32_t lo = acc | (sy << f8);
+    const uint32_t hi = __funnelshift_l(sy, 0u, f8);  // bytes pushed past the word
+    f8 += c8;
+    if (f8 >= 32u) {
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(wp), "r"(lo) : "memory");
+        wp += 4u;
+        f8 -= 32u;
+        acc = hi;
+    } else {
+        acc = lo;
+    }
+}
+
 // Phase 2: the same walk on the full entries {ctl, syms}, writing the symbols
 // in order from shared-memory byte address `out` on.  Symbols are assembled
 // in a register (acc holds f8 / 8 pending bytes, starting from acc0, the
@@ -1111,7 +1178,9 @@ __device__ __forceinline__ uint32_t byte_step_count(const uint32_t (&w)[CB / 32 
 // word it ends in later threads' bytes: that last, partial word is returned
 // in acc / wp / f8 and OR-ed in by the caller after a __syncwarp, so it
 // lands after every plain store of the warp and no store clears another
-// thread's bytes.  The buffer is zero outside the words written.  ctl_out
+// thread's bytes.  The buffer is zero outside the words written.  The
+// steps after the whole bytes only keep the entry of the last, partial byte
+// (j == nfull), whose codes are emitted once after the loop.  ctl_out
 // receives the last control word, whose row is the dead row (`dead`) when
 // the walk left the tables or the partial byte ends more than 4 codes.
 template <int CB>
@@ -1124,6 +1193,7 @@ __device__ __forceinline__ void byte_step_emit(const uint32_t (&w)[CB / 32 + 1],
     acc = acc0;
     wp = out & ~3u;
     f8 = (out & 3u) << 3;
+    uint2 ep = make_uint2(0u, 0u);
 #pragma unroll
     for (int m = 0; m <= CW; ++m) {
         if (4 * m >= NFIX && 4 * m >= jmax) break;  // warp-uniform
@@ -1133,32 +1203,19 @@ __device__ __forceinline__ void byte_step_emit(const uint32_t (&w)[CB / 32 + 1],
             const int j = 4 * m + k;
             if (j >= NFIX && j >= jmax) break;
             const uint2 e = *reinterpret_cast<const uint2 *>(tab + step_addr<8>(x, k, ctl & kFsmRowMask));
-            uint32_t sy, c8;
             if (j < NFIX || j < nfull) {
                 ctl = e.x;
-                sy = e.y;
-                c8 = e.x >> (kFsmCountShift - 3);  // 8 x codes ended
+                emit_word(e.y, e.x >> (kFsmCountShift - 3), acc, wp, f8);
             } else if (j == nfull) {
-                const uint32_t ce = static_cast<uint32_t>(__popc(e.x & ((1u << r) - 1u)));
-                const uint32_t c = min(ce, 4u);
-                sy = c ? e.y & (0xFFFFFFFFu >> (32u - 8u * c)) : 0u;
-                c8 = 8u * c;
-                if (ce > 4) ctl = dead;
-            } else {
-                continue;
-            }
-            const uint32_t lo = acc | (sy << f8);
-            const uint32_t hi = __funnelshift_l(sy, 0u, f8);  // bytes pushed past the word
-            f8 += c8;
-            if (f8 >= 32u) {
-                asm volatile("st.shared.u32 [%0], %1;" ::"r"(wp), "r"(lo) : "memory");
-                wp += 4u;
-                f8 -= 32u;
-                acc = hi;
-            } else {
-                acc = lo;
+                ep = e;  // the partial byte: emitted once after the loop
             }
         }
+    }
+    if (r) {
+        const uint32_t ce = static_cast<uint32_t>(__popc(ep.x & ((1u << r) - 1u)));
+        const uint32_t c = min(ce, 4u);
+        emit_word(c ? ep.y & (0xFFFFFFFFu >> (32u - 8u * c)) : 0u, 8u * c, acc, wp, f8);
+        if (ce > 4) ctl = dead;
     }
     ctl_out = ctl;
 }
@@ -1321,11 +1378,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         // the tile's plane span: the first kPrefetchGroups groups of each lane now
         const uint8_t *plane = d.plane + g0 * 16u;
         uint2 pre[2 * kPrefetchGroups];
-#pragma unroll
-        for (int u = 0; u < 2 * kPrefetchGroups; ++u) {
-            const uint32_t j = lane + 32u * u;
-            if (j < 2 * ng) pre[u] = ld_global_stream_v2(plane + 8u * j);
-        }
+        prefetch_halves(pre, plane + 8u * lane, lane, 2 * ng, std::make_integer_sequence<int, 2 * kPrefetchGroups>{});
 
         const bool landed = __all_sync(0xFFFFFFFFu, mbar_wait(&full[0], k & 1u, P.wait_ns));
         if (!landed) {
@@ -1456,11 +1509,8 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
             const uint32_t nmerge = keep ? ng - 1 : ng;
             const uint32_t nh = 2u * nmerge;
             if (static_cast<uint32_t>(lane) < nh) merge_half<DT, true>(pre[0], lane, s_exps, dst_tile, lo, hi);
-#pragma unroll
-            for (int u = 1; u < 2 * kPrefetchGroups; ++u) {
-                const uint32_t j = lane + 32u * u;
-                if (j < nh) merge_half<DT, false>(pre[u], j, s_exps, dst_tile, lo, hi);
-            }
+            merge_rounds<DT>(pre, lane, nh, s_exps + (DT == 0 ? 8u : 16u) * lane, dst_tile + 16u * lane,
+                             std::make_integer_sequence<int, 2 * kPrefetchGroups - 1>{});
             for (uint32_t j = lane + 64u * kPrefetchGroups; j < nh; j += 32)
                 merge_half<DT, false>(ld_global_stream_v2(plane + 8u * j), j, s_exps, dst_tile, lo, hi);
             __syncwarp();

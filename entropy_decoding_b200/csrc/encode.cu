@@ -28,6 +28,9 @@ namespace {
 constexpr int kEncThreads = 256;
 constexpr int kElemsPerThread = 16;
 constexpr uint32_t kSegElems = kEncThreads * kElemsPerThread;  // 4096 elements per segment
+// chunks a segment's codes can start in: its bits (at most 32 per element)
+// over the smallest chunk that stores counts (64 bits), plus both ends
+constexpr uint32_t kSegChunks = kSegElems * kMaxCodeLen / 64 + 2;
 
 template <int DT>
 __device__ __forceinline__ uint32_t exponent_at(const void *src, uint64_t i) {
@@ -216,13 +219,20 @@ __device__ __forceinline__ void or_code(uint32_t *stream, uint64_t o, uint32_t c
     }
 }
 
+// Chunk counts are tallied per segment in shared memory (s_cnt[c - c_lo] for
+// the segment's chunks [c_lo, c_hi]) and written out by words of 4 chunks: a
+// word whose chunks all lie strictly inside the range belongs to this segment
+// alone (a neighbouring segment's codes start at or before c_lo, or at or
+// after c_hi) and is stored; the words at the ends are added atomically.
 template <int DT>
 __global__ void __launch_bounds__(kEncThreads) pack_kernel(const PackArgs A) {
     __shared__ uint8_t s_len[256];
     __shared__ uint32_t s_code[256];
     __shared__ uint32_t s_warp[kEncThreads / 32];
+    __shared__ uint32_t s_cnt[kSegChunks];
     s_len[threadIdx.x] = A.lengths[threadIdx.x];
     s_code[threadIdx.x] = A.codes[threadIdx.x];
+    for (uint32_t i = threadIdx.x; i < kSegChunks; i += kEncThreads) s_cnt[i] = 0;
     __syncthreads();
     const uint64_t cb = A.chunk_bits;
     for (uint64_t seg = blockIdx.x; seg < A.n_seg; seg += gridDim.x) {
@@ -236,12 +246,13 @@ __global__ void __launch_bounds__(kEncThreads) pack_kernel(const PackArgs A) {
         uint32_t total;
         const uint32_t incl = block_inclusive_scan(bits, s_warp, total);
         uint64_t start = A.seg_off[seg] + (incl - bits);
+        // the segment's chunks (its codes start in [seg_off, seg_off + total))
+        const uint64_t c_lo = A.seg_off[seg] / cb, c_hi = (A.seg_off[seg] + total - 1) / cb;
         // previous element's start: from its code length
         uint64_t prev = ~uint64_t{0};
         if (i0 > 0 && c > 0) prev = start - s_len[exponent_at<DT>(A.src, i0 - 1)];
         // chunk counts: this thread's codes fall in one or two chunks mostly;
-        // one add per run of codes in the same chunk (a chunk of at most 128
-        // bits has at most 128 starts, so the byte never carries into the next)
+        // one shared-memory add per run of codes in the same chunk
         uint64_t run_c = ~uint64_t{0};
         uint32_t run_n = 0;
 #pragma unroll
@@ -252,7 +263,7 @@ __global__ void __launch_bounds__(kEncThreads) pack_kernel(const PackArgs A) {
             const uint64_t ck = start / cb, pk = prev == ~uint64_t{0} ? ~uint64_t{0} : prev / cb;
             if (A.counts) {
                 if (ck != run_c) {
-                    if (run_n) atomicAdd(A.counts + (run_c >> 2), run_n << (8u * static_cast<uint32_t>(run_c & 3u)));
+                    if (run_n) atomicAdd(&s_cnt[run_c - c_lo], run_n);
                     run_c = ck;
                     run_n = 0;
                 }
@@ -264,7 +275,25 @@ __global__ void __launch_bounds__(kEncThreads) pack_kernel(const PackArgs A) {
             prev = start;
             start += len;
         }
-        if (A.counts && run_n) atomicAdd(A.counts + (run_c >> 2), run_n << (8u * static_cast<uint32_t>(run_c & 3u)));
+        if (A.counts) {
+            if (run_n) atomicAdd(&s_cnt[run_c - c_lo], run_n);
+            __syncthreads();
+            // a chunk of at most 128 bits holds at most 128 starts: bytes never carry
+            for (uint64_t wd = c_lo / 4 + threadIdx.x; wd <= c_hi / 4; wd += kEncThreads) {
+                uint32_t packed = 0;
+#pragma unroll
+                for (uint32_t k = 0; k < 4; ++k) {
+                    const uint64_t ch = 4 * wd + k;
+                    if (ch >= c_lo && ch <= c_hi) {
+                        packed |= s_cnt[ch - c_lo] << (8u * k);
+                        s_cnt[ch - c_lo] = 0;  // zero again for the next segment
+                    }
+                }
+                if (4 * wd > c_lo && 4 * wd + 3 < c_hi) A.counts[wd] = packed;
+                else if (packed) atomicAdd(A.counts + wd, packed);
+            }
+            // the next segment's adds come after the block scan's barriers
+        }
         // raw fields
         if constexpr (DT == 0) {
             if (c == 16) {
