@@ -1365,7 +1365,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         const uint32_t lt = t - d.tile_begin;
         uint64_t S = __ldg(d.out_off + lt);
         const uint64_t Eo = __ldg(d.out_off + lt + 1);
-        const bool bad = Eo < S || Eo > d.n || Eo - S > max_span;
+        const bool bad = Eo - S > max_span || Eo > d.n;  // Eo < S wraps above max_span
         if (bad) S = 0;
         const uint32_t span = bad ? 0u : static_cast<uint32_t>(Eo - S);
         const uint64_t g0 = S / GROUP;
@@ -1422,13 +1422,16 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         }
 
         // ---- this thread's range of codes
-        const int64_t rem64 = static_cast<int64_t>(d.total_bits) - static_cast<int64_t>(lt) * (32 * CB) -
-                              static_cast<int64_t>(lane * CB);
-        const int E = rem64 >= CB ? CB : (rem64 <= 0 ? 0 : static_cast<int>(rem64));
+        // stream bits from this thread's chunk on: the tile's remainder (64-bit,
+        // warp-uniform) clamped to [-1, 32 CB + 256], then 32-bit per thread
+        // (no range reaches past CB + 255 bits of its chunk)
+        const int64_t trem = static_cast<int64_t>(d.total_bits) - static_cast<int64_t>(lt) * (32 * CB);
+        const int rem = static_cast<int>(max(min(trem, static_cast<int64_t>(32 * CB + 256)), static_cast<int64_t>(-1))) -
+                        lane * CB;
+        const int E = min(max(rem, 0), CB);
         if (graw >= 32) err |= DF11_DEV_ERR_AUX;
         const int g = min(graw, 63);
-        const int64_t end64 = rem64 < CB + gnext ? rem64 : static_cast<int64_t>(CB + gnext);
-        const int nbits = static_cast<int>(max(end64 - g, static_cast<int64_t>(-1)));
+        const int nbits = max(min(rem, CB + gnext) - g, -1);
         const bool whole = graw < 32 && gnext < 32 && nbits >= 8 * NFIX;
         const int nfull = nbits >> 3, r = nbits & 7;
         const int jmax = static_cast<int>(__reduce_max_sync(0xFFFFFFFFu, whole ? nfull + (r != 0) : 0));
