@@ -57,7 +57,8 @@ typedef enum {
 /* Bits the decode kernel ORs into the caller's device error word.  Any
  * non-zero value means some output of that call is not valid; the kernel
  * still never writes outside the destination buffers it was given. */
-#define DF11_DEV_ERR_SPAN 1u     /* a tile decoded a different number of codes than its out_off span */
+#define DF11_DEV_ERR_SPAN 1u     /* a tile decoded a different number of codes than its out_off span,
+                                    or a chunk a different number than its stored count */
 #define DF11_DEV_ERR_CODE 2u     /* the stream held a bit pattern that is no codeword */
 #define DF11_DEV_ERR_AUX 4u      /* an auxiliary value (gap, out_off) out of its valid range */
 #define DF11_DEV_ERR_TIMEOUT 8u  /* a bounded wait on an on-chip barrier gave up */
