@@ -252,6 +252,40 @@ def test_bounded_wait_runs_out_and_reports(df11, layout_walker):
     assert np.array_equal(out.cpu().numpy().view(np.uint16), x)
 
 
+def test_decode_captured_in_a_cuda_graph(df11):
+    """df11_decode_ex launched inside CUDA stream capture (plain and
+    overlapped launch) and replayed: every replay exact, no error.  The call
+    allocates and synchronises nothing, so it can be captured."""
+    g = synth.transformer_block(3)[0]
+    xs = [t.bits[: 150000 + 11 * i] for i, t in enumerate(g.tensors[:3])]
+    cb = df11.df11_build_codebook("bf16", xs)
+    blobs = [df11.df11_encode(cb, x) for x in xs]
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        for b in blobs:
+            df11.upload(b, s)
+    s.synchronize()
+    outs = [torch.zeros(2 * x.size, dtype=torch.uint8, device="cuda") for x in xs]
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    # one plain launch first: the library's one-time set-up per kernel and
+    # device (shared-memory attribute) happens outside the capture
+    df11.df11_decode_ex(blobs, [o.data_ptr() for o in outs], err.data_ptr(), s.cuda_stream)
+    s.synchronize()
+    for overlap in (0, 1):
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=s):
+            df11.df11_decode_ex(blobs, [o.data_ptr() for o in outs], err.data_ptr(), s.cuda_stream, overlap=overlap)
+        for _ in range(3):
+            for o in outs:
+                o.zero_()
+            graph.replay()
+            torch.cuda.synchronize()
+            assert int(err.item()) == 0
+            for x, o in zip(xs, outs):
+                assert np.array_equal(o.cpu().numpy().view(np.uint16), x)
+        del graph
+
+
 def test_mixed_codes_rejected(df11):
     a = synth.single_matrix(0)[0].tensors[0].bits[:5000]
     b = synth.heavy_tail_matrix(0)[0].tensors[0].bits[:5000]

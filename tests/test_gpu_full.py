@@ -27,14 +27,14 @@ def df11():
     return mod
 
 
-def _decode_group(df11, blobs):
+def _decode_group(df11, blobs, count_walk=0):
     """One launch over the blobs with the benchmark's options (default walk,
-    overlapped launch)."""
+    overlapped launch); count_walk = 1 counts with the first-phase walk."""
     imgs = [df11.upload(b) for b in blobs]
     outs = [df11.empty_output(b) for b in blobs]
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     df11.df11_decode_ex(blobs, [o.data_ptr() for o in outs], err.data_ptr(), torch.cuda.current_stream().cuda_stream,
-                        overlap=1)
+                        overlap=1, count_walk=count_walk)
     torch.cuda.synchronize()
     del imgs
     return outs, int(err.item())
@@ -78,7 +78,10 @@ def test_full_size_small_configs(df11, oracle_mod, cfg):
         assert blob.info().max_code_len >= 20  # the long tail reaches the deep table levels
 
 
-def test_full_size_transformer_block_one_launch(df11, oracle_mod):
+@pytest.mark.parametrize("count_walk", [0, 1])
+def test_full_size_transformer_block_one_launch(df11, oracle_mod, count_walk):
+    """The block in one launch, placing each thread's output with the stored
+    chunk counts (the benchmark's default) and with the first-phase count walk."""
     g = synth.transformer_block(0)[0]
     xs = [t.bits for t in g.tensors]
     cb = df11.df11_build_codebook("bf16", xs)
@@ -86,7 +89,7 @@ def test_full_size_transformer_block_one_launch(df11, oracle_mod):
     assert np.array_equal(lengths, oracle_mod.build_lengths(xs, "bf16"))
     blobs = [df11.df11_encode(cb, x) for x in xs]
     assert sum(b.info().n_elems for b in blobs) == 218103808
-    outs, err = _decode_group(df11, blobs)
+    outs, err = _decode_group(df11, blobs, count_walk)
     assert err == 0
     for x, out in zip(xs, outs):
         assert _device_equal(out, x)
