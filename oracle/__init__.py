@@ -77,6 +77,14 @@ def _load():
         lib.oracle_aux.restype = I
         lib.oracle_chunk_counts.argtypes = [P, U64, P, I, I, P]
         lib.oracle_chunk_counts.restype = I
+        lib.oracle_rans_freqs.argtypes = [P, I, P]
+        lib.oracle_rans_freqs.restype = I
+        lib.oracle_rans_encode.argtypes = [P, U64, P, I, ctypes.c_uint32, P, U64, P, P]
+        lib.oracle_rans_encode.restype = I
+        lib.oracle_rans_words_bound.argtypes = [U64, ctypes.c_uint32]
+        lib.oracle_rans_words_bound.restype = U64
+        lib.oracle_rans_decode.argtypes = [P, P, P, U64, P, I, ctypes.c_uint32, P]
+        lib.oracle_rans_decode.restype = I
         lib.oracle_decode.argtypes = [P, U64, P, I, U64, U64, P]
         lib.oracle_decode.restype = I
         _lib = lib
@@ -290,3 +298,81 @@ def decode_at(c: Compressed, start_bit: int, count: int) -> np.ndarray:
     """Exponent symbols of `count` consecutive weights whose first code starts
     at `start_bit` (a sampled slice, decoded one symbol at a time)."""
     return decode(c.stream, c.total_bits, c.lengths, start_bit, count)
+
+
+# ---------------------------------------------------------------- rANS variant
+# ("Approaching Shannon Bound with Lossless LLM Weight Compression", Abstract:
+# ANS decoding by tiles; coder details are the readings of df11_oracle.c
+# section 9)
+
+RANS_BITS = 12
+RANS_M = 1 << RANS_BITS
+RANS_L = 1 << 16
+RANS_LANES = 32
+
+
+def rans_freqs(counts: np.ndarray, nsym: int) -> np.ndarray:
+    """Quantized frequencies (sum 2^12) from exponent counts."""
+    lib = _load()
+    c = np.zeros(256, np.uint64)
+    c[:nsym] = np.asarray(counts, np.uint64)[:nsym]
+    f = np.zeros(256, np.uint32)
+    _check(lib.oracle_rans_freqs(_p(c), nsym, _p(f)), "rans_freqs")
+    return f[:nsym].copy()
+
+
+def rans_encode(exps: np.ndarray, freqs: np.ndarray, tile_symbols: int):
+    """(words u16, states u32 [n_tiles * 32], tile_words u64 [n_tiles + 1])."""
+    lib = _load()
+    exps = np.ascontiguousarray(exps, np.uint8)
+    fr = np.ascontiguousarray(freqs, np.uint32)
+    n = exps.size
+    n_tiles = -(-n // tile_symbols)
+    cap = int(lib.oracle_rans_words_bound(n, tile_symbols))
+    words = np.zeros(max(cap, 1), np.uint16)
+    states = np.zeros(max(n_tiles * RANS_LANES, 1), np.uint32)
+    tile_words = np.zeros(n_tiles + 1, np.uint64)
+    src = exps if n else np.zeros(1, np.uint8)
+    _check(lib.oracle_rans_encode(_p(src), n, _p(fr), fr.size, tile_symbols, _p(words), cap, _p(states),
+                                  _p(tile_words)), "rans_encode")
+    return words[: int(tile_words[-1])].copy(), states[: n_tiles * RANS_LANES].copy(), tile_words
+
+
+def rans_decode(words: np.ndarray, states: np.ndarray, tile_words: np.ndarray, n: int, freqs: np.ndarray,
+                tile_symbols: int) -> np.ndarray:
+    lib = _load()
+    w = np.ascontiguousarray(words, np.uint16) if words.size else np.zeros(1, np.uint16)
+    st = np.ascontiguousarray(states, np.uint32) if states.size else np.zeros(1, np.uint32)
+    tw = np.ascontiguousarray(tile_words, np.uint64)
+    fr = np.ascontiguousarray(freqs, np.uint32)
+    out = np.zeros(max(n, 1), np.uint8)
+    _check(lib.oracle_rans_decode(_p(w), _p(st), _p(tw), n, _p(fr), fr.size, tile_symbols, _p(out)),
+           "rans_decode")
+    return out[:n]
+
+
+@dataclass
+class RansCompressed:
+    dtype: str
+    n: int
+    freqs: np.ndarray       # quantized frequencies, sum 2^12
+    words: np.ndarray       # u16 words, tiles 8-word aligned
+    states: np.ndarray      # u32, 32 per tile
+    tile_words: np.ndarray  # u64, n_tiles + 1
+    plane: np.ndarray       # raw sign+mantissa field, as the Huffman container's
+    tile_symbols: int
+
+
+def rans_compress(x: np.ndarray, dtype: str, freqs: np.ndarray | None = None,
+                  tile_symbols: int = 16384) -> RansCompressed:
+    x = np.ascontiguousarray(x).reshape(-1)
+    exps, plane = split(x, dtype)
+    if freqs is None:
+        freqs = rans_freqs(histogram(exps)[: NSYM[dtype]], NSYM[dtype])
+    words, states, tile_words = rans_encode(exps, freqs, tile_symbols)
+    return RansCompressed(dtype, x.size, freqs, words, states, tile_words, plane, tile_symbols)
+
+
+def rans_decompress(c: RansCompressed) -> np.ndarray:
+    exps = rans_decode(c.words, c.states, c.tile_words, c.n, c.freqs, c.tile_symbols)
+    return merge(exps, c.plane, c.n, c.dtype)

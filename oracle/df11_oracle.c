@@ -544,3 +544,187 @@ int oracle_decode(const uint8_t *stream, uint64_t total_bits,
     free(t);
     return ORACLE_OK;
 }
+
+/* ------------------------------------------------------------------ */
+/* 9. rANS variant of the exponent coder.                               */
+/*    [SHANNON] "Approaching Shannon Bound with Lossless LLM Weight     */
+/*    Compression", Abstract: tile-level decoding with Asymmetric       */
+/*    Numeral Systems, within 0.01-0.1 bits of the Shannon limit.       */
+/*    The page gives no coder details.  This is the range variant of    */
+/*    ANS (rANS, Duda) in its textbook form: a state x; a symbol s      */
+/*    with quantized frequency f_s and cumulative frequency c_s over a  */
+/*    total M = 2^12 is coded as                                        */
+/*        x' = floor(x / f_s) * M + (x mod f_s) + c_s                   */
+/*    and decoded from x' as the s with c_s <= x' mod M < c_s + f_s,    */
+/*        x = f_s * floor(x' / M) + (x' mod M) - c_s,                   */
+/*    the state kept in [2^16, 2^32) by moving 16-bit words.            */
+/*    Readings (the page is silent; all listed in the design notes):   */
+/*    frequencies by the rule of oracle_rans_freqs; 32 interleaved      */
+/*    coders per tile in the order of oracle_rans_encode; tiles of      */
+/*    tile_symbols symbols.                                             */
+/* ------------------------------------------------------------------ */
+
+#define ORACLE_RANS_BITS 12
+#define ORACLE_RANS_M (1u << ORACLE_RANS_BITS)
+#define ORACLE_RANS_L 65536u
+#define ORACLE_RANS_LANES 32
+
+/* Quantized frequencies summing to M = 2^12: a present symbol s gets
+ * max(1, floor(count_s * M / total)); the shortfall is then given one unit
+ * at a time to the present symbols in order of decreasing count (smaller
+ * symbol first on ties), cycling, and an excess taken one unit at a time in
+ * the same order from symbols above 1.  Absent symbols get 0. */
+int oracle_rans_freqs(const uint64_t *counts, int nsym, uint32_t *freqs)
+{
+    uint64_t total = 0;
+    int order[256], present = 0;
+    for (int s = 0; s < nsym; s++) {
+        freqs[s] = 0;
+        total += counts[s];
+        if (counts[s]) order[present++] = s;
+    }
+    if (present == 0) return ORACLE_OK;
+    /* order: count descending, symbol ascending (insertion sort) */
+    for (int i = 1; i < present; i++) {
+        int s = order[i], j = i - 1;
+        while (j >= 0 && (counts[order[j]] < counts[s] ||
+                          (counts[order[j]] == counts[s] && order[j] > s))) {
+            order[j + 1] = order[j];
+            j--;
+        }
+        order[j + 1] = s;
+    }
+    long long sum = 0;
+    for (int i = 0; i < present; i++) {
+        int s = order[i];
+        uint64_t f = counts[s] * (uint64_t)ORACLE_RANS_M / total;
+        if (f < 1) f = 1;
+        freqs[s] = (uint32_t)f;
+        sum += (long long)f;
+    }
+    long long d = (long long)ORACLE_RANS_M - sum;
+    for (int i = 0; d > 0; i++, d--) freqs[order[i % present]]++;
+    for (int i = 0; d < 0; i++) {
+        int s = order[i % present];
+        if (freqs[s] > 1) {
+            freqs[s]--;
+            d++;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* Tiles of tile_symbols symbols (the last one shorter), each coded by 32
+ * interleaved coders: coder j takes the tile's symbols j, j + 32, j + 64, ...
+ * Decoding runs steps k = 0, 1, ... and in each step coders j = 0..31 in
+ * turn: coder j decodes symbol 32k + j (when the tile has it), then, if its
+ * state fell below 2^16, appends the tile's next 16-bit word below it.  The
+ * encoder runs that order backwards from states 2^16, moving a word out
+ * before a symbol whenever the state would leave [2^16, 2^32), and reverses
+ * the words it wrote.  Each tile's words start at a multiple of 8 words
+ * (zero padding between tiles).  Outputs: words; states[t * 32 + j] =
+ * coder j's final encoder state (its initial decoder state); tile_words
+ * (n_tiles + 1 offsets in words, the last one the padded total). */
+int oracle_rans_encode(const uint8_t *exps, uint64_t n, const uint32_t *freqs, int nsym,
+                       uint32_t tile_symbols, uint16_t *words, uint64_t words_cap,
+                       uint32_t *states, uint64_t *tile_words)
+{
+    uint32_t cum[257];
+    if (n == 0) { /* no symbol: no table needed */
+        tile_words[0] = 0;
+        return ORACLE_OK;
+    }
+    cum[0] = 0;
+    for (int s = 0; s < nsym; s++) cum[s + 1] = cum[s] + freqs[s];
+    if (nsym < 1 || cum[nsym] != ORACLE_RANS_M || tile_symbols == 0 || tile_symbols % ORACLE_RANS_LANES)
+        return ORACLE_EINVAL;
+    uint64_t n_tiles = (n + tile_symbols - 1) / tile_symbols;
+    uint16_t *tmp = (uint16_t *)malloc((size_t)tile_symbols * sizeof(uint16_t));
+    if (!tmp) return ORACLE_ENOMEM;
+    uint64_t pos = 0;
+    for (uint64_t t = 0; t < n_tiles; t++) {
+        uint64_t base = t * tile_symbols;
+        uint64_t m = n - base < tile_symbols ? n - base : tile_symbols;
+        uint32_t x[ORACLE_RANS_LANES];
+        for (int j = 0; j < ORACLE_RANS_LANES; j++) x[j] = ORACLE_RANS_L;
+        uint64_t nw = 0;
+        uint64_t steps = (m + ORACLE_RANS_LANES - 1) / ORACLE_RANS_LANES;
+        for (uint64_t k = steps; k-- > 0;) {
+            for (int j = ORACLE_RANS_LANES - 1; j >= 0; j--) {
+                uint64_t p = k * ORACLE_RANS_LANES + (uint64_t)j;
+                if (p >= m) continue;
+                int s = exps[base + p];
+                if (s >= nsym || freqs[s] == 0) { free(tmp); return ORACLE_EINVAL; }
+                uint32_t f = freqs[s];
+                /* after coding, x' < 2^32 needs x < f * 2^20 */
+                if ((uint64_t)x[j] >= ((uint64_t)f << (32 - ORACLE_RANS_BITS))) {
+                    tmp[nw++] = (uint16_t)(x[j] & 0xFFFFu);
+                    x[j] >>= 16;
+                }
+                x[j] = (x[j] / f) * ORACLE_RANS_M + (x[j] % f) + cum[s];
+            }
+        }
+        tile_words[t] = pos;
+        if (pos + nw + 8 > words_cap) { free(tmp); return ORACLE_EINVAL; }
+        for (uint64_t i = 0; i < nw; i++) words[pos + i] = tmp[nw - 1 - i];
+        pos += nw;
+        while (pos % 8) words[pos++] = 0;
+        for (int j = 0; j < ORACLE_RANS_LANES; j++) states[t * ORACLE_RANS_LANES + (uint64_t)j] = x[j];
+    }
+    tile_words[n_tiles] = pos;
+    free(tmp);
+    return ORACLE_OK;
+}
+
+/* Words a tile of tile_symbols symbols can need at most: one per symbol,
+ * plus the padding. */
+uint64_t oracle_rans_words_bound(uint64_t n, uint32_t tile_symbols)
+{
+    uint64_t n_tiles = (n + tile_symbols - 1) / tile_symbols;
+    return n + 8 * n_tiles + 8;
+}
+
+/* The decoder in the order the encoder defines (steps, then coders).  Every
+ * coder must end in state 2^16 having read only its tile's words (the rest
+ * of the tile's range being padding): ORACLE_ECORRUPT otherwise. */
+int oracle_rans_decode(const uint16_t *words, const uint32_t *states, const uint64_t *tile_words,
+                       uint64_t n, const uint32_t *freqs, int nsym, uint32_t tile_symbols,
+                       uint8_t *exps_out)
+{
+    uint32_t cum[257];
+    uint8_t sym[ORACLE_RANS_M];
+    if (n == 0) return ORACLE_OK;
+    cum[0] = 0;
+    for (int s = 0; s < nsym; s++) cum[s + 1] = cum[s] + freqs[s];
+    if (nsym < 1 || cum[nsym] != ORACLE_RANS_M || tile_symbols == 0 || tile_symbols % ORACLE_RANS_LANES)
+        return ORACLE_EINVAL;
+    for (int s = 0; s < nsym; s++)
+        for (uint32_t v = cum[s]; v < cum[s + 1]; v++) sym[v] = (uint8_t)s;
+    uint64_t n_tiles = (n + tile_symbols - 1) / tile_symbols;
+    for (uint64_t t = 0; t < n_tiles; t++) {
+        uint64_t base = t * tile_symbols;
+        uint64_t m = n - base < tile_symbols ? n - base : tile_symbols;
+        uint32_t x[ORACLE_RANS_LANES];
+        for (int j = 0; j < ORACLE_RANS_LANES; j++) x[j] = states[t * ORACLE_RANS_LANES + (uint64_t)j];
+        uint64_t ptr = tile_words[t], end = tile_words[t + 1];
+        uint64_t steps = (m + ORACLE_RANS_LANES - 1) / ORACLE_RANS_LANES;
+        for (uint64_t k = 0; k < steps; k++) {
+            for (int j = 0; j < ORACLE_RANS_LANES; j++) {
+                uint64_t p = k * ORACLE_RANS_LANES + (uint64_t)j;
+                if (p >= m) continue;
+                uint32_t slot = x[j] & (ORACLE_RANS_M - 1);
+                int s = sym[slot];
+                x[j] = freqs[s] * (x[j] >> ORACLE_RANS_BITS) + slot - cum[s];
+                if (x[j] < ORACLE_RANS_L) {
+                    if (ptr >= end) return ORACLE_ECORRUPT;
+                    x[j] = (x[j] << 16) | words[ptr++];
+                }
+                exps_out[base + p] = (uint8_t)s;
+            }
+        }
+        for (int j = 0; j < ORACLE_RANS_LANES; j++)
+            if (x[j] != ORACLE_RANS_L) return ORACLE_ECORRUPT;
+        if (end - ptr >= 8) return ORACLE_ECORRUPT;
+    }
+    return ORACLE_OK;
+}
