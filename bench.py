@@ -71,6 +71,10 @@ def parse_args():
     p.add_argument("--count-walk", action="store_true",
                    help="decode launch option: count each chunk's codes with a first walk even though the "
                         "images store chunk counts")
+    p.add_argument("--coder", choices=["huffman", "rans"], default="huffman",
+                   help="exponent coder: the Huffman container (default) or the rANS variant (decode from HBM "
+                        "only; no end-to-end, streaming, encoder or CPU measurements)")
+    p.add_argument("--rans-tile", type=int, default=0, help="rANS symbols per tile (0 = library default)")
     p.add_argument("--no-overlap", dest="overlap", action="store_false",
                    help="launch the groups in plain stream order (default: each group's decode may start "
                         "while the previous one finishes, the groups being independent; the roofline then "
@@ -675,6 +679,123 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     print(json.dumps(line), flush=True)
 
 
+def run_rans(args, rank: int, world: int, local_rank: int):
+    """The rANS variant of the exponent coder on the same workload: every
+    group encoded with one frequency table on the host, then per step one
+    decode launch per group from HBM, timed and checked as the Huffman arm."""
+    import torch
+    import torch.distributed as dist
+    from entropy_decoding_b200 import df11
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    threads = host_threads(world)
+    t_setup = time.time()
+    groups, samples = [], []
+    rng = np.random.default_rng(12345)
+    coded = plane = uncompressed = 0
+    n_w = 0
+    for gi in range(group_count(args.workload)):
+        g = make_group(args.workload, args.seed, gi)
+        dt = "bf16" if g.tensors[0].bits.dtype == np.uint16 else "e4m3"
+        xs = [t.bits for t in g.tensors]
+        rg = df11.df11_rans_encode_group(dt, xs, args.rans_tile, threads)
+        for ti, x in enumerate(xs):
+            pos = np.unique(np.concatenate([np.arange(min(4096, x.size)), np.arange(max(0, x.size - 4096), x.size),
+                                            rng.integers(0, x.size, 32768)]))
+            samples.append((gi, ti, pos, x[pos].copy()))
+            inf = rg.info(ti)
+            coded += inf.coded_bytes
+            plane += inf.plane_bytes
+            uncompressed += inf.uncompressed_bytes
+            n_w += x.size
+        with torch.cuda.stream(stream):
+            df11.rans_upload(rg, stream)
+        groups.append([g.name, rg, dt, [x.size * x.itemsize for x in xs]])
+        del g, xs
+    setup_s = time.time() - t_setup
+    total_out = sum(((s_ + 255) // 256) * 256 for grp in groups for s_ in grp[3])
+    out = torch.empty(total_out, dtype=torch.uint8, device=dev)
+    off = 0
+    for grp in groups:
+        dsts = []
+        for s_ in grp[3]:
+            dsts.append((out.data_ptr() + off, off, s_))
+            off += ((s_ + 255) // 256) * 256
+        grp.append(dsts)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream.synchronize()
+    out_bytes = sum(sum(grp[3]) for grp in groups)
+
+    def one_step():
+        for name, rg, dt, sizes, dsts in groups:
+            df11.df11_rans_decode(rg, [d[0] for d in dsts], err.data_ptr(), stream.cuda_stream)
+
+    for _ in range(args.warmup):
+        one_step()
+    stream.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    start.record(stream)
+    for _ in range(args.steps):
+        one_step()
+    end.record(stream)
+    end.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    elapsed_ms = max_over_ranks(start.elapsed_time(end), dev)
+    e = int(err.item())
+    bad = 0
+    for gi, ti, pos, vals in samples:
+        ptr, o, s_ = groups[gi][4][ti]
+        v = out[o:o + s_]
+        if groups[gi][2] == "bf16":
+            got = v.view(torch.int16)[torch.from_numpy(pos).to(dev)].cpu().numpy().view(np.uint16)
+        else:
+            got = v[torch.from_numpy(pos).to(dev)].cpu().numpy()
+        bad += int((got != vals).sum())
+    assert e == 0, f"rans decode: device error word {e}"
+    assert bad == 0, f"rans decode: {bad} sampled outputs differ from the source weights"
+    if rank != 0:
+        return
+    value = job_throughput(out_bytes, world, args.steps, elapsed_ms)
+    algo = coded + plane + out_bytes
+    achieved = algo * args.steps / (elapsed_ms / 1e3) / 1e9
+    peak, peak_src = hbm_peak()
+    freq_bytes = 2 * (256 if groups[0][2] == "bf16" else 16) * len(groups)  # the stored form of each table
+    shape = df11.df11_rans_decode_launch_shape(groups[0][1])
+    dtn = groups[0][2]
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u32", "data": "synthetic (seeded N(0,1/sqrt(fan_in)) / N(0,0.02) weights, "
+                                                     "random init, no trained checkpoint)",
+        "config": {**full_config(args, world), "coder": "rans",
+                   "rans_tile_symbols": args.rans_tile or df11.RANS_TILE_DEFAULT},
+        "weights_per_s": world * n_w * args.steps / (elapsed_ms / 1e3),
+        "compression_ratio": (coded + plane + freq_bytes) / uncompressed,
+        "bits_per_weight": 8 * (coded + plane + freq_bytes) / n_w,
+        "hbm_roofline_frac": achieved / peak,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "peak_source": peak_src, "peak_datasheet": 8000.0,
+                     "frac_datasheet": achieved / 8000.0,
+                     "kernel": f"rans_decode_kernel<{dtn},32>",
+                     "launch": {"grid": shape[0], "block": shape[1], "smem_bytes": shape[2]},
+                     "algorithmic_bytes_per_step": algo, "traffic_source": "not captured for this kernel"},
+        "cpu_baseline": None, "e2e": None, "gpu_launches": len(groups) * args.steps, "clocks": clk,
+        "setup_s": setup_s,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     rank, world, local_rank = rank_env()
@@ -688,7 +809,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        run_ours(args, rank, world, local_rank)
+        if args.coder == "rans":
+            run_rans(args, rank, world, local_rank)
+        else:
+            run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -21,9 +21,9 @@ CUDA_HOME = os.environ.get("CUDA_HOME", "/usr/local/cuda")
 NVCC = os.path.join(CUDA_HOME, "bin", "nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
-SOURCES_CU = ["decode.cu", "encode.cu"]
-SOURCES_CPP = ["codec.cpp", "capi.cpp"]
-HEADERS = ["df11_internal.h", "codec.h", "launch.h", "encode.h"]
+SOURCES_CU = ["decode.cu", "encode.cu", "rans_decode.cu"]
+SOURCES_CPP = ["codec.cpp", "capi.cpp", "rans.cpp"]
+HEADERS = ["df11_internal.h", "codec.h", "launch.h", "encode.h", "rans.h"]
 
 
 def _newer(target: str, deps: list[str]) -> bool:

@@ -11,6 +11,7 @@
 #include "codec.h"
 #include "encode.h"
 #include "launch.h"
+#include "rans.h"
 
 struct df11_codebook {
     std::shared_ptr<df11::Codebook> cb;
@@ -586,6 +587,108 @@ df11_status df11_encode_device_noalloc(const df11_codebook *cb, const void *src_
     if (err.find("too small") != std::string::npos) return DF11_ENOMEM;
     if (err.find("cover") != std::string::npos) return DF11_EINVAL;
     return DF11_ECUDA;
+}
+
+// ---------------------------------------------------------------- rANS coder
+
+struct df11_rans_group {
+    df11::RansGroup g;
+};
+
+df11_status df11_rans_encode_group(df11_dtype dtype, const void *const *host_tensors, const uint64_t *n_elems,
+                                   int n_tensors, int tile_symbols, int n_threads, df11_rans_group **out) {
+    if (!out || !valid_dtype(dtype) || n_tensors < 1 || n_tensors > 64 || !host_tensors || !n_elems ||
+        n_threads < 0 || tile_symbols < 0)
+        return DF11_EINVAL;
+    *out = nullptr;
+    try {
+        auto *g = new df11_rans_group;
+        const uint32_t ts = tile_symbols ? static_cast<uint32_t>(tile_symbols) : DF11_RANS_TILE_DEFAULT;
+        const std::string err = df11::rans_encode_group(dtype, host_tensors, n_elems, n_tensors, ts, n_threads, &g->g);
+        if (!err.empty()) {
+            delete g;
+            return DF11_EINVAL;
+        }
+        *out = g;
+        return DF11_OK;
+    } catch (const std::bad_alloc &) {
+        return DF11_ENOMEM;
+    }
+}
+
+void df11_rans_group_free(df11_rans_group *g) { delete g; }
+
+df11_status df11_rans_group_freqs(const df11_rans_group *g, uint32_t *freqs) {
+    if (!g || !freqs) return DF11_EINVAL;
+    std::memcpy(freqs, g->g.freqs, sizeof g->g.freqs);
+    return DF11_OK;
+}
+
+df11_status df11_rans_group_info(const df11_rans_group *g, int tensor, df11_rans_tensor_info *info) {
+    if (!g || !info || tensor < 0 || tensor >= static_cast<int>(g->g.tensors.size())) return DF11_EINVAL;
+    const df11::RansTensor &t = g->g.tensors[tensor];
+    info->n_elems = t.n;
+    info->n_tiles = t.n_tiles;
+    info->words = t.words.size();
+    info->coded_bytes = t.words.size() * 2 + t.states.size() * 4 + t.tile_words.size() * 8;
+    info->plane_bytes = t.plane.size();
+    info->uncompressed_bytes = g->g.dtype == df11::kBF16 ? 2 * t.n : t.n;
+    return DF11_OK;
+}
+
+df11_status df11_rans_group_sections(const df11_rans_group *g, int tensor, const uint16_t **words,
+                                     const uint32_t **states, const uint64_t **tile_words, const uint8_t **plane) {
+    if (!g || tensor < 0 || tensor >= static_cast<int>(g->g.tensors.size())) return DF11_EINVAL;
+    const df11::RansTensor &t = g->g.tensors[tensor];
+    if (words) *words = t.words.data();
+    if (states) *states = t.states.data();
+    if (tile_words) *tile_words = t.tile_words.data();
+    if (plane) *plane = t.plane.data();
+    return DF11_OK;
+}
+
+uint64_t df11_rans_group_device_bytes(const df11_rans_group *g) {
+    if (!g) return 0;
+    uint64_t total = 0;
+    df11::rans_layout(g->g, &total);
+    return total;
+}
+
+df11_status df11_rans_group_upload(df11_rans_group *g, void *dev_dst, uint64_t cap, df11_stream stream) {
+    if (!g || !dev_dst || reinterpret_cast<uintptr_t>(dev_dst) % df11::kImageAlign) return DF11_EINVAL;
+    const uint64_t need = df11_rans_group_device_bytes(g);
+    if (cap < need) return DF11_ENOMEM;
+    try {
+        g->g.host_image.resize(need);
+    } catch (const std::bad_alloc &) {
+        return DF11_ENOMEM;
+    }
+    df11::rans_write_image(g->g, g->g.host_image.data());
+    if (cudaMemcpyAsync(dev_dst, g->g.host_image.data(), need, cudaMemcpyHostToDevice,
+                        reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return DF11_ECUDA;
+    g->g.dev_image = static_cast<const uint8_t *>(dev_dst);
+    g->g.dev_cap = cap;
+    return DF11_OK;
+}
+
+df11_status df11_rans_decode(const df11_rans_group *g, void *const *dst_dev, int *dev_err_flag, df11_stream stream) {
+    if (!g || !dst_dev) return DF11_EINVAL;
+    switch (df11::rans_launch_decode(g->g, dst_dev, dev_err_flag, reinterpret_cast<cudaStream_t>(stream), nullptr,
+                                     nullptr, nullptr)) {
+    case df11::RansLaunch::kOk: return DF11_OK;
+    case df11::RansLaunch::kInvalid: return DF11_EINVAL;
+    default: return DF11_ECUDA;
+    }
+}
+
+df11_status df11_rans_decode_launch_shape(const df11_rans_group *g, int *grid, int *block, int *smem_bytes) {
+    if (!g) return DF11_EINVAL;
+    switch (df11::rans_launch_decode(g->g, nullptr, nullptr, nullptr, grid, block, smem_bytes)) {
+    case df11::RansLaunch::kOk: return DF11_OK;
+    case df11::RansLaunch::kInvalid: return DF11_EINVAL;
+    default: return DF11_ECUDA;
+    }
 }
 
 }  // extern "C"

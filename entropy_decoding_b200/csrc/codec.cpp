@@ -19,25 +19,6 @@ namespace df11 {
 
 namespace {
 
-template <class F>
-void parallel_for(uint64_t n_items, int n_threads, F fn) {
-    if (n_items == 0) return;
-    unsigned hw = std::thread::hardware_concurrency();
-    int t = n_threads > 0 ? n_threads : static_cast<int>(hw ? hw : 1);
-    if (static_cast<uint64_t>(t) > n_items) t = static_cast<int>(n_items);
-    if (t <= 1) {
-        fn(uint64_t{0}, n_items);
-        return;
-    }
-    std::vector<std::thread> pool;
-    pool.reserve(t);
-    for (int k = 0; k < t; ++k) {
-        uint64_t b = n_items * k / t, e = n_items * (k + 1) / t;
-        pool.emplace_back([=, &fn] { fn(b, e); });
-    }
-    for (auto &th : pool) th.join();
-}
-
 inline uint8_t exponent_of(int dtype, const void *src, uint64_t i) {
     if (dtype == kBF16) return static_cast<uint8_t>((static_cast<const uint16_t *>(src)[i] >> 7) & 0xFF);
     return static_cast<uint8_t>((static_cast<const uint8_t *>(src)[i] >> 3) & 0xF);

@@ -5,6 +5,7 @@
 #include <cstdint>
 #include <memory>
 #include <string>
+#include <thread>
 #include <vector>
 
 #include "df11_internal.h"
@@ -50,6 +51,27 @@ struct Blob {
     uint64_t dev_cap = 0;
     std::vector<uint8_t> host_image;  // staging copy kept alive for df11_blob_upload
 };
+
+// Runs fn(begin, end) over [0, n_items) split evenly across n_threads host
+// threads (0 = all cores).
+template <class F>
+void parallel_for(uint64_t n_items, int n_threads, F fn) {
+    if (n_items == 0) return;
+    unsigned hw = std::thread::hardware_concurrency();
+    int t = n_threads > 0 ? n_threads : static_cast<int>(hw ? hw : 1);
+    if (static_cast<uint64_t>(t) > n_items) t = static_cast<int>(n_items);
+    if (t <= 1) {
+        fn(uint64_t{0}, n_items);
+        return;
+    }
+    std::vector<std::thread> pool;
+    pool.reserve(t);
+    for (int k = 0; k < t; ++k) {
+        uint64_t b = n_items * k / t, e = n_items * (k + 1) / t;
+        pool.emplace_back([=, &fn] { fn(b, e); });
+    }
+    for (auto &th : pool) th.join();
+}
 
 // Code construction.  Returns false when the arguments admit no code.
 bool code_lengths(const uint64_t *counts, int nsym, int max_len, uint8_t *lengths);

@@ -56,6 +56,12 @@ class EncodeResult(ctypes.Structure):
                 ("max_span", ctypes.c_uint64)]
 
 
+class RansTensorInfo(ctypes.Structure):
+    _fields_ = [("n_elems", ctypes.c_uint64), ("n_tiles", ctypes.c_uint64), ("words", ctypes.c_uint64),
+                ("coded_bytes", ctypes.c_uint64), ("plane_bytes", ctypes.c_uint64),
+                ("uncompressed_bytes", ctypes.c_uint64)]
+
+
 class DecodeOpts(ctypes.Structure):
     _fields_ = [("chunks_per_thread", ctypes.c_int32), ("ctas_per_sm", ctypes.c_int32),
                 ("warps_per_cta", ctypes.c_int32), ("walker", ctypes.c_int32), ("max_ctas", ctypes.c_int32),
@@ -107,6 +113,15 @@ _SIGS = {
     "df11_encode_device_noalloc": ([_P, _P, _U64, _I, _I, _I, _P, _U64, _P, ctypes.POINTER(EncodeResult)], _S),
     "df11_decode_host": ([_PP, _PP, _PP, _PP, _PP, _I, _P, _P], _S),
     "df11_decode_launch_shape": ([_PP, _I, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I)], _S),
+    "df11_rans_encode_group": ([_I, _PP, ctypes.POINTER(_U64), _I, _I, _I, _PP], _S),
+    "df11_rans_group_free": ([_P], None),
+    "df11_rans_group_freqs": ([_P, _P], _S),
+    "df11_rans_group_info": ([_P, _I, ctypes.POINTER(RansTensorInfo)], _S),
+    "df11_rans_group_sections": ([_P, _I, _PP, _PP, _PP, _PP], _S),
+    "df11_rans_group_device_bytes": ([_P], _U64),
+    "df11_rans_group_upload": ([_P, _P, _U64, _P], _S),
+    "df11_rans_decode": ([_P, _PP, _P, _P], _S),
+    "df11_rans_decode_launch_shape": ([_P, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I)], _S),
 }
 for _name, (_args, _res) in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -448,3 +463,94 @@ def empty_output(blob: Blob):
     i = blob.info()
     nbytes = i.n_elems * (2 if i.dtype == DF11_BF16 else 1)
     return torch.empty(max(nbytes, 16), dtype=torch.uint8, device="cuda")
+
+
+# ----------------------------------------------------------------- rANS coder (same names as the C-ABI)
+
+RANS_TILE_DEFAULT = 16384
+
+
+class RansGroup:
+    """Tensors coded with one rANS frequency table (df11_rans_group)."""
+
+    def __init__(self, handle: int, dtype: str, n_tensors: int):
+        self._h = ctypes.c_void_p(handle)
+        self.dtype = dtype
+        self.n_tensors = n_tensors
+        self._keep = None
+
+    @property
+    def handle(self):
+        return self._h
+
+    def freqs(self) -> np.ndarray:
+        f = np.zeros(256, np.uint32)
+        _check(_lib.df11_rans_group_freqs(self._h, f.ctypes.data), "df11_rans_group_freqs")
+        return f[: 256 if self.dtype == "bf16" else 16]
+
+    def info(self, i: int) -> RansTensorInfo:
+        r = RansTensorInfo()
+        _check(_lib.df11_rans_group_info(self._h, i, ctypes.byref(r)), "df11_rans_group_info")
+        return r
+
+    def sections(self, i: int) -> dict:
+        """Copies of tensor i's words, states, tile_words and plane."""
+        inf = self.info(i)
+        ptrs = [ctypes.c_void_p() for _ in range(4)]
+        _check(_lib.df11_rans_group_sections(self._h, i, *[ctypes.byref(p) for p in ptrs]), "df11_rans_group_sections")
+
+        def grab(p, n, dt):
+            if n == 0:
+                return np.zeros(0, dt)
+            nb = n * np.dtype(dt).itemsize
+            return np.ctypeslib.as_array(ctypes.cast(p, ctypes.POINTER(ctypes.c_uint8)), (nb,)).view(dt).copy()
+
+        return {"words": grab(ptrs[0], inf.words, np.uint16), "states": grab(ptrs[1], inf.n_tiles * 32, np.uint32),
+                "tile_words": grab(ptrs[2], inf.n_tiles + 1, np.uint64),
+                "plane": grab(ptrs[3], inf.plane_bytes, np.uint8)}
+
+    def device_bytes(self) -> int:
+        return int(_lib.df11_rans_group_device_bytes(self._h))
+
+    def __del__(self, _free=_lib.df11_rans_group_free):
+        if getattr(self, "_h", None) and self._h.value:
+            _free(self._h)
+            self._h = ctypes.c_void_p(0)
+
+
+def df11_rans_encode_group(dtype: str, tensors, tile_symbols: int = 0, n_threads: int = 0) -> RansGroup:
+    arrs = [np.ascontiguousarray(t).reshape(-1) for t in tensors]
+    ptrs = _ptr_array([a.ctypes.data if a.size else None for a in arrs])
+    ns = (_U64 * len(arrs))(*[a.size for a in arrs])
+    out = ctypes.c_void_p()
+    _check(_lib.df11_rans_encode_group(DTYPES[dtype], ptrs, ns, len(arrs), tile_symbols, n_threads,
+                                       ctypes.byref(out)), "df11_rans_encode_group")
+    return RansGroup(out.value, dtype, len(arrs))
+
+
+def df11_rans_group_upload(g: RansGroup, dev_ptr: int, cap: int, stream: int = 0, keep=None):
+    _check(_lib.df11_rans_group_upload(g.handle, dev_ptr, cap, stream or None), "df11_rans_group_upload")
+    g._keep = keep
+
+
+def df11_rans_decode(g: RansGroup, dst_ptrs, err_ptr: int | None = None, stream: int = 0):
+    _check(_lib.df11_rans_decode(g.handle, _ptr_array(dst_ptrs), err_ptr or None, stream or None), "df11_rans_decode")
+
+
+def df11_rans_decode_launch_shape(g: RansGroup):
+    a, b, c = _I(), _I(), _I()
+    _check(_lib.df11_rans_decode_launch_shape(g.handle, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)),
+           "df11_rans_decode_launch_shape")
+    return a.value, b.value, c.value
+
+
+def rans_upload(g: RansGroup, stream=None):
+    """Allocates the group's device image with torch, copies it and binds it."""
+    import torch
+    n = g.device_bytes()
+    dev = torch.empty(n + 256, dtype=torch.uint8, device="cuda")
+    base = dev.data_ptr()
+    off = (-base) % 256
+    s = stream.cuda_stream if stream is not None else torch.cuda.current_stream().cuda_stream
+    df11_rans_group_upload(g, base + off, n, s, keep=dev)
+    return dev

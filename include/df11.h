@@ -452,6 +452,83 @@ df11_status df11_encode_device_noalloc(const df11_codebook *cb, const void *src_
                                        uint64_t image_cap, df11_stream stream,
                                        df11_encode_result *result);
 
+/* ---------------------------------------------------------------------
+ * rANS variant of the exponent coder
+ * ------------------------------------------------------------------ */
+
+/* The same exponent symbols and raw plane as the Huffman container, coded
+ * with range asymmetric numeral systems instead of a prefix code: the
+ * tile-level ANS decoding of "Approaching Shannon Bound with Lossless LLM
+ * Weight Compression", Abstract (which gives no coder details; the format
+ * below is this library's).
+ *   frequencies  quantized to a total of 2^12 over the group's exponent
+ *                histogram (every present symbol at least 1)
+ *   state        32 bits in [2^16, 2^32); 16-bit words move in and out
+ *   tiles        tile_symbols symbols (a multiple of 32), coded by 32
+ *                interleaved coders: coder j takes symbols j, j+32, ...
+ *                Decoding runs steps, and in each step coders 0..31 in
+ *                order; a coder whose state fell below 2^16 after its symbol
+ *                reads the tile's next word.
+ *   per tile     32 initial states (u32) and its words' offset (u64, a
+ *                multiple of 8 words)
+ * One group = the tensors of one launch, sharing one frequency table (a
+ * transformer block).  Decoding is exact: the output equals the source bits. */
+typedef struct df11_rans_group df11_rans_group;
+
+#define DF11_RANS_TILE_DEFAULT 16384
+
+typedef struct {
+    uint64_t n_elems;
+    uint64_t n_tiles;
+    uint64_t words;        /* 16-bit words, with the padding between tiles */
+    uint64_t coded_bytes;  /* words * 2 + states (n_tiles * 128) + offsets ((n_tiles + 1) * 8) */
+    uint64_t plane_bytes;
+    uint64_t uncompressed_bytes;
+} df11_rans_tensor_info;
+
+/* Encodes n_tensors host tensors (dtype's raw bits) with one frequency table
+ * built from all of them; tile_symbols a multiple of 32 in [32, 2^20] (0 =
+ * DF11_RANS_TILE_DEFAULT); n_threads host threads (0 = all cores).
+ * Errors: DF11_EINVAL, DF11_ENOMEM. */
+df11_status df11_rans_encode_group(df11_dtype dtype, const void *const *host_tensors, const uint64_t *n_elems,
+                                   int n_tensors, int tile_symbols, int n_threads, df11_rans_group **out);
+
+void df11_rans_group_free(df11_rans_group *g);
+
+/* The quantized frequencies (freqs[0..255]; E4M3 uses 16). */
+df11_status df11_rans_group_freqs(const df11_rans_group *g, uint32_t *freqs);
+
+df11_status df11_rans_group_info(const df11_rans_group *g, int tensor, df11_rans_tensor_info *info);
+
+/* Read-only host views of one tensor's sections (valid until the group is
+ * freed); any output may be NULL. */
+df11_status df11_rans_group_sections(const df11_rans_group *g, int tensor, const uint16_t **words,
+                                     const uint32_t **states, const uint64_t **tile_words,
+                                     const uint8_t **plane);
+
+/* Bytes of the group's device image: the 4096-entry decode table, then per
+ * tensor its states, offsets, words (plus 1024 zero words) and plane (plus
+ * 512 bytes), each section 256-byte aligned. */
+uint64_t df11_rans_group_device_bytes(const df11_rans_group *g);
+
+/* Builds the image in host memory held by the group, copies it to dev_dst
+ * (256-byte aligned, cap >= device bytes) on `stream` and binds it.  The
+ * caller owns dev_dst.  Errors: DF11_EINVAL, DF11_ENOMEM, DF11_ECUDA. */
+df11_status df11_rans_group_upload(df11_rans_group *g, void *dev_dst, uint64_t cap, df11_stream stream);
+
+/* Decodes every tensor of the bound group in one launch on `stream`,
+ * asynchronously; dst_dev[i] as in df11_decode (16-byte aligned).  Damaged
+ * data ORs DF11_DEV_ERR_SPAN (a tile's coders do not end in their initial
+ * state, or took other than its words) or DF11_DEV_ERR_AUX (offsets out of
+ * range) into dev_err_flag; nothing is written outside the destinations.
+ * Errors: DF11_EINVAL (unbound group, bad pointer), DF11_ECUDA. */
+df11_status df11_rans_decode(const df11_rans_group *g, void *const *dst_dev, int *dev_err_flag,
+                             df11_stream stream);
+
+/* Grid, threads per CTA and dynamic shared memory of that launch (any output
+ * may be NULL; the group must be bound). */
+df11_status df11_rans_decode_launch_shape(const df11_rans_group *g, int *grid, int *block, int *smem_bytes);
+
 #ifdef __cplusplus
 }
 #endif

@@ -18,7 +18,8 @@ def df11():
     return mod
 
 
-STRUCTS = {"df11_blob_info": "BlobInfo", "df11_decode_opts": "DecodeOpts", "df11_encode_result": "EncodeResult"}
+STRUCTS = {"df11_blob_info": "BlobInfo", "df11_decode_opts": "DecodeOpts", "df11_encode_result": "EncodeResult",
+           "df11_rans_tensor_info": "RansTensorInfo"}
 CONSTANTS = {
     "DF11_OK": "DF11_OK", "DF11_EINVAL": "DF11_EINVAL", "DF11_ENOMEM": "DF11_ENOMEM", "DF11_ECUDA": "DF11_ECUDA",
     "DF11_ECORRUPT": "DF11_ECORRUPT", "DF11_EUNSUPPORTED": "DF11_EUNSUPPORTED",
@@ -29,6 +30,7 @@ CONSTANTS = {
     "DF11_WALKER_BYTE_STEP": "WALKER_BYTE_STEP",
     "DF11_ENCODE_NO_CHUNK_COUNTS": "ENCODE_NO_CHUNK_COUNTS",
     "DF11_NOALLOC_SCRATCH_BYTES": "NOALLOC_SCRATCH_BYTES", "DF11_NOALLOC_MAX_ELEMS": "NOALLOC_MAX_ELEMS",
+    "DF11_RANS_TILE_DEFAULT": "RANS_TILE_DEFAULT",
 }
 
 
