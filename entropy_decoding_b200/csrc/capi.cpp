@@ -647,6 +647,31 @@ df11_status df11_rans_group_sections(const df11_rans_group *g, int tensor, const
     return DF11_OK;
 }
 
+df11_status df11_rans_group_serialize(const df11_rans_group *g, void *buf, uint64_t cap, uint64_t *used) {
+    if (!g) return DF11_EINVAL;
+    const uint64_t need = df11::rans_serialized_bytes(g->g);
+    if (used) *used = need;
+    if (!buf || cap < need) return DF11_ENOMEM;
+    df11::rans_serialize(g->g, static_cast<uint8_t *>(buf));
+    return DF11_OK;
+}
+
+df11_status df11_rans_group_deserialize(const void *buf, uint64_t len, df11_rans_group **out) {
+    if (!buf || !out) return DF11_EINVAL;
+    *out = nullptr;
+    try {
+        auto *g = new df11_rans_group;
+        if (!df11::rans_deserialize(static_cast<const uint8_t *>(buf), len, &g->g).empty()) {
+            delete g;
+            return DF11_ECORRUPT;
+        }
+        *out = g;
+        return DF11_OK;
+    } catch (const std::bad_alloc &) {
+        return DF11_ENOMEM;
+    }
+}
+
 uint64_t df11_rans_group_device_bytes(const df11_rans_group *g) {
     if (!g) return 0;
     uint64_t total = 0;

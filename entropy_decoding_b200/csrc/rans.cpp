@@ -183,3 +183,157 @@ void rans_write_image(const RansGroup &g, uint8_t *dst) {
 }
 
 }  // namespace df11
+
+// ---------------------------------------------------------------- container
+//
+// One file per group: a 64-byte header, the frequencies (u16 per symbol),
+// then per tensor a 32-byte record (n, n_tiles, words, reserved) followed by
+// its states, tile word offsets, words and plane, every section 16-byte
+// aligned.  The decode table is derived from the frequencies.
+
+namespace df11 {
+namespace {
+
+struct RansFileHeader {
+    char magic[8];  // "DF11RANS"
+    uint32_t version;
+    uint32_t dtype;
+    uint32_t nsym;
+    uint32_t tile_symbols;
+    uint32_t n_tensors;
+    uint32_t reserved[9];
+};
+static_assert(sizeof(RansFileHeader) == 64, "header layout");
+
+struct RansFileTensor {
+    uint64_t n, n_tiles, words, reserved;
+};
+
+const char kRansMagic[8] = {'D', 'F', '1', '1', 'R', 'A', 'N', 'S'};
+
+inline uint64_t up16(uint64_t x) { return (x + 15) / 16 * 16; }
+
+// Bytes of a tensor's sections after its record.
+uint64_t tensor_bytes(int dtype, uint64_t n, uint64_t n_tiles, uint64_t words) {
+    uint64_t o = up16(n_tiles * kRansLanes * 4);
+    o += up16((n_tiles + 1) * 8);
+    o += up16(words * 2);
+    o += up16(plane_bytes(dtype, n));
+    return o;
+}
+
+}  // namespace
+
+uint64_t rans_serialized_bytes(const RansGroup &g) {
+    uint64_t o = sizeof(RansFileHeader) + up16(static_cast<uint64_t>(g.nsym) * 2);
+    for (const RansTensor &t : g.tensors)
+        o += sizeof(RansFileTensor) + tensor_bytes(g.dtype, t.n, t.n_tiles, t.words.size());
+    return o;
+}
+
+void rans_serialize(const RansGroup &g, uint8_t *dst) {
+    const uint64_t total = rans_serialized_bytes(g);
+    std::memset(dst, 0, total);
+    RansFileHeader h{};
+    std::memcpy(h.magic, kRansMagic, 8);
+    h.version = 1;
+    h.dtype = static_cast<uint32_t>(g.dtype);
+    h.nsym = static_cast<uint32_t>(g.nsym);
+    h.tile_symbols = g.tile_symbols;
+    h.n_tensors = static_cast<uint32_t>(g.tensors.size());
+    std::memcpy(dst, &h, sizeof h);
+    uint64_t o = sizeof h;
+    for (int s = 0; s < g.nsym; ++s) {
+        const uint16_t f = static_cast<uint16_t>(g.freqs[s]);
+        std::memcpy(dst + o + 2 * s, &f, 2);
+    }
+    o += up16(static_cast<uint64_t>(g.nsym) * 2);
+    for (const RansTensor &t : g.tensors) {
+        const RansFileTensor r{t.n, t.n_tiles, t.words.size(), 0};
+        std::memcpy(dst + o, &r, sizeof r);
+        o += sizeof r;
+        if (!t.states.empty()) std::memcpy(dst + o, t.states.data(), t.states.size() * 4);
+        o += up16(t.states.size() * 4);
+        std::memcpy(dst + o, t.tile_words.data(), t.tile_words.size() * 8);
+        o += up16(t.tile_words.size() * 8);
+        if (!t.words.empty()) std::memcpy(dst + o, t.words.data(), t.words.size() * 2);
+        o += up16(t.words.size() * 2);
+        if (!t.plane.empty()) std::memcpy(dst + o, t.plane.data(), t.plane.size());
+        o += up16(t.plane.size());
+    }
+}
+
+std::string rans_deserialize(const uint8_t *src, uint64_t len, RansGroup *out) {
+    if (len < sizeof(RansFileHeader)) return "truncated header";
+    RansFileHeader h;
+    std::memcpy(&h, src, sizeof h);
+    if (std::memcmp(h.magic, kRansMagic, 8) != 0) return "bad magic";
+    if (h.version != 1) return "unknown version";
+    if (h.dtype != kBF16 && h.dtype != kE4M3) return "bad dtype";
+    const int dtype = static_cast<int>(h.dtype);
+    if (h.nsym != static_cast<uint32_t>(nsym_of(dtype))) return "bad symbol count";
+    if (h.tile_symbols < kRansLanes || h.tile_symbols % kRansLanes || h.tile_symbols > (1u << 20))
+        return "bad tile size";
+    if (h.n_tensors < 1 || h.n_tensors > 64) return "bad tensor count";
+    RansGroup &g = *out;
+    g = RansGroup();
+    g.dtype = dtype;
+    g.nsym = static_cast<int>(h.nsym);
+    g.tile_symbols = h.tile_symbols;
+    uint64_t o = sizeof h;
+    if (len < o + up16(static_cast<uint64_t>(g.nsym) * 2)) return "truncated frequencies";
+    uint32_t sum = 0;
+    for (int s = 0; s < g.nsym; ++s) {
+        uint16_t f;
+        std::memcpy(&f, src + o + 2 * s, 2);
+        if (f > kRansM) return "frequency out of range";
+        g.freqs[s] = f;
+        sum += f;
+    }
+    o += up16(static_cast<uint64_t>(g.nsym) * 2);
+    bool any_symbols = false;
+    g.tensors.resize(h.n_tensors);
+    for (uint32_t i = 0; i < h.n_tensors; ++i) {
+        if (len < o + sizeof(RansFileTensor)) return "truncated tensor record";
+        RansFileTensor r;
+        std::memcpy(&r, src + o, sizeof r);
+        o += sizeof r;
+        if (r.n > (uint64_t{1} << 40) || r.reserved) return "bad tensor record";
+        if (r.n_tiles != (r.n + h.tile_symbols - 1) / h.tile_symbols) return "tile count mismatch";
+        if (r.words > r.n + 8 * r.n_tiles) return "word count out of range";
+        const uint64_t need = tensor_bytes(dtype, r.n, r.n_tiles, r.words);
+        if (len < o + need) return "truncated tensor sections";
+        RansTensor &t = g.tensors[i];
+        t.n = r.n;
+        t.n_tiles = r.n_tiles;
+        any_symbols |= r.n != 0;
+        t.states.resize(r.n_tiles * kRansLanes);
+        if (!t.states.empty()) std::memcpy(t.states.data(), src + o, t.states.size() * 4);
+        o += up16(t.states.size() * 4);
+        t.tile_words.resize(r.n_tiles + 1);
+        std::memcpy(t.tile_words.data(), src + o, t.tile_words.size() * 8);
+        o += up16(t.tile_words.size() * 8);
+        t.words.resize(r.words);
+        if (r.words) std::memcpy(t.words.data(), src + o, r.words * 2);
+        o += up16(r.words * 2);
+        t.plane.assign(src + o, src + o + plane_bytes(dtype, r.n));
+        o += up16(t.plane.size());
+        if (t.tile_words[0] != 0 || t.tile_words[r.n_tiles] != r.words) return "tile offsets endpoints";
+        for (uint64_t k = 0; k < r.n_tiles; ++k) {
+            if (t.tile_words[k + 1] < t.tile_words[k] || t.tile_words[k + 1] % 8) return "tile offsets";
+            // a tile of m symbols takes at most one word per symbol, plus padding
+            const uint64_t m = std::min<uint64_t>(h.tile_symbols, r.n - k * h.tile_symbols);
+            if (t.tile_words[k + 1] - t.tile_words[k] > m + 7) return "tile word count out of range";
+        }
+        for (uint32_t x : t.states)
+            if (x < kRansL) return "state below 2^16";
+        if (dtype == kE4M3 && (r.n & 1) && (t.plane.back() & 0xF0)) return "nonzero plane padding";
+    }
+    if (o != len) return "container size mismatch";
+    // the table: frequencies summing to 2^12 (all zero only for a group without symbols)
+    if (sum != kRansM && (any_symbols || sum != 0)) return "frequencies do not sum to 4096";
+    if (sum == kRansM) rans_build_table(g.freqs, g.nsym, g.table);
+    return "";
+}
+
+}  // namespace df11

@@ -70,6 +70,12 @@ std::string rans_encode_group(int dtype, const void *const *src, const uint64_t 
 std::vector<RansTensorLayout> rans_layout(const RansGroup &g, uint64_t *total);
 void rans_write_image(const RansGroup &g, uint8_t *dst);
 
+// The group's container (the offline form) and its reader, which checks the
+// header, the frequencies, every size and tile offset and the states' range.
+uint64_t rans_serialized_bytes(const RansGroup &g);
+void rans_serialize(const RansGroup &g, uint8_t *dst);
+std::string rans_deserialize(const uint8_t *src, uint64_t len, RansGroup *out);
+
 enum class RansLaunch { kOk, kInvalid, kCuda };
 // One launch decoding every tensor of the bound group into dst[i].
 RansLaunch rans_launch_decode(const RansGroup &g, void *const *dst, int *err, cudaStream_t s, int *grid_out,

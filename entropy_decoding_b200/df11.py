@@ -12,6 +12,7 @@ pointers are plain integers (``tensor.data_ptr()``), streams are
 from __future__ import annotations
 
 import ctypes
+import struct
 import os
 import re
 
@@ -119,6 +120,8 @@ _SIGS = {
     "df11_rans_group_info": ([_P, _I, ctypes.POINTER(RansTensorInfo)], _S),
     "df11_rans_group_sections": ([_P, _I, _PP, _PP, _PP, _PP], _S),
     "df11_rans_group_device_bytes": ([_P], _U64),
+    "df11_rans_group_serialize": ([_P, _P, _U64, ctypes.POINTER(_U64)], _S),
+    "df11_rans_group_deserialize": ([_P, _U64, _PP], _S),
     "df11_rans_group_upload": ([_P, _P, _U64, _P], _S),
     "df11_rans_decode": ([_P, _PP, _P, _P], _S),
     "df11_rans_decode_launch_shape": ([_P, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I)], _S),
@@ -526,6 +529,22 @@ def df11_rans_encode_group(dtype: str, tensors, tile_symbols: int = 0, n_threads
     _check(_lib.df11_rans_encode_group(DTYPES[dtype], ptrs, ns, len(arrs), tile_symbols, n_threads,
                                        ctypes.byref(out)), "df11_rans_encode_group")
     return RansGroup(out.value, dtype, len(arrs))
+
+
+def df11_rans_group_serialize(g: RansGroup) -> bytes:
+    need = _U64()
+    _lib.df11_rans_group_serialize(g.handle, None, 0, ctypes.byref(need))
+    buf = ctypes.create_string_buffer(need.value)
+    _check(_lib.df11_rans_group_serialize(g.handle, buf, need.value, ctypes.byref(need)), "df11_rans_group_serialize")
+    return buf.raw[: need.value]
+
+
+def df11_rans_group_deserialize(data) -> RansGroup:
+    b = bytes(data)
+    out = ctypes.c_void_p()
+    _check(_lib.df11_rans_group_deserialize(b, len(b), ctypes.byref(out)), "df11_rans_group_deserialize")
+    dt = "bf16" if struct.unpack_from("<I", b, 12)[0] == DF11_BF16 else "e4m3"
+    return RansGroup(out.value, dt, struct.unpack_from("<I", b, 24)[0])
 
 
 def df11_rans_group_upload(g: RansGroup, dev_ptr: int, cap: int, stream: int = 0, keep=None):

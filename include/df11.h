@@ -506,6 +506,19 @@ df11_status df11_rans_group_sections(const df11_rans_group *g, int tensor, const
                                      const uint32_t **states, const uint64_t **tile_words,
                                      const uint8_t **plane);
 
+/* The group's container (offline form): a 64-byte header ("DF11RANS",
+ * version 1, dtype, symbols, tile size, tensor count), the frequencies (u16
+ * per symbol), then per tensor a 32-byte record (n, n_tiles, words) and its
+ * states, tile offsets, words and plane, each section 16-byte aligned.
+ * *used receives the size; DF11_ENOMEM when cap is too small. */
+df11_status df11_rans_group_serialize(const df11_rans_group *g, void *buf, uint64_t cap, uint64_t *used);
+
+/* Reads a container; checks the header, that the frequencies sum to 2^12,
+ * every size, the tile offsets (monotone, multiples of 8, at most one word
+ * per symbol plus padding) and that every state is at least 2^16.  Errors:
+ * DF11_ECORRUPT, DF11_ENOMEM. */
+df11_status df11_rans_group_deserialize(const void *buf, uint64_t len, df11_rans_group **out);
+
 /* Bytes of the group's device image: the 4096-entry decode table, then per
  * tensor its states, offsets, words (plus 1024 zero words) and plane (plus
  * 512 bytes), each section 256-byte aligned. */

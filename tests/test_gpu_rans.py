@@ -139,3 +139,15 @@ def test_launch_shape(df11):
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     assert block == 1024 and 0 < smem <= 227 * 1024
     assert grid == min(sms, -(-g.info(0).n_tiles // 32))
+
+
+def test_group_from_its_container_decodes(df11):
+    """Serialize, read back, upload, decode: the container is enough."""
+    g0 = synth.transformer_block(5)[0]
+    xs = [g0.tensors[1].bits[:300001], g0.tensors[5].bits[:200003]]
+    g = df11.df11_rans_encode_group("bf16", xs, 4096)
+    g2 = df11.df11_rans_group_deserialize(df11.df11_rans_group_serialize(g))
+    outs, err, ok = _decode(df11, g2, xs)
+    assert err == 0 and ok
+    for x, o in zip(xs, outs):
+        assert np.array_equal(o, x)

@@ -79,3 +79,65 @@ def test_invalid_arguments(df11):
         df11.df11_rans_encode_group("bf16", [x], 16)   # below 32
     with pytest.raises(df11.Df11Error):
         df11.df11_rans_encode_group("bf16", [])
+
+
+def _group_for_container(df11):
+    g0 = synth.transformer_block(4)[0]
+    xs = [g0.tensors[0].bits[:70001], np.zeros(0, np.uint16), g0.tensors[4].bits[:50003]]
+    return xs, df11.df11_rans_encode_group("bf16", xs, 4096)
+
+
+def test_container_roundtrip(df11):
+    xs, g = _group_for_container(df11)
+    data = df11.df11_rans_group_serialize(g)
+    g2 = df11.df11_rans_group_deserialize(data)
+    assert g2.n_tensors == 3 and g2.dtype == "bf16"
+    assert np.array_equal(g2.freqs(), g.freqs())
+    for i in range(3):
+        a, b = g.sections(i), g2.sections(i)
+        for k in a:
+            assert np.array_equal(a[k], b[k]), (i, k)
+    assert df11.df11_rans_group_serialize(g2) == data
+    # header, frequencies, and per tensor a record plus its 16-byte aligned sections
+    up = lambda v: (v + 15) // 16 * 16
+    want = 64 + up(2 * 256)
+    for i in range(3):
+        inf = g.info(i)
+        want += 32 + up(inf.n_tiles * 128) + up((inf.n_tiles + 1) * 8) + up(2 * inf.words) + up(inf.plane_bytes)
+    assert len(data) == want
+
+
+def test_container_e4m3_and_one_symbol(df11):
+    for dt, x in [("e4m3", synth.normal_e4m3(np.random.SeedSequence(8), 30001)),
+                  ("bf16", synth.constant_bf16(9000, 2.0))]:
+        g = df11.df11_rans_encode_group(dt, [x], 1024)
+        data = df11.df11_rans_group_serialize(g)
+        g2 = df11.df11_rans_group_deserialize(data)
+        assert np.array_equal(g2.freqs(), g.freqs())
+        assert df11.df11_rans_group_serialize(g2) == data
+
+
+def test_container_rejects_damage(df11):
+    import struct
+    xs, g = _group_for_container(df11)
+    good = bytearray(df11.df11_rans_group_serialize(g))
+    inf0 = g.info(0)
+    rec0 = 64 + 512                         # first tensor's record
+    states0 = rec0 + 32
+    tw0 = states0 + (inf0.n_tiles * 128 + 15) // 16 * 16
+
+    def rejected(buf):
+        with pytest.raises(df11.Df11Error) as e:
+            df11.df11_rans_group_deserialize(bytes(buf))
+        assert e.value.status == df11.DF11_ECORRUPT
+
+    rejected(good[:-16])                                                      # truncated
+    rejected(good + b"\0" * 16)                                               # trailing bytes
+    bad = bytearray(good); bad[0] ^= 1; rejected(bad)                         # magic
+    bad = bytearray(good); struct.pack_into("<I", bad, 8, 2); rejected(bad)   # version
+    f = g.freqs()
+    s = int(np.flatnonzero(f)[0])
+    bad = bytearray(good); struct.pack_into("<H", bad, 64 + 2 * s, int(f[s]) + 1); rejected(bad)  # sum 4097
+    bad = bytearray(good); struct.pack_into("<I", bad, states0 + 4 * 3, 1000); rejected(bad)      # state < 2^16
+    bad = bytearray(good); struct.pack_into("<Q", bad, tw0 + 8, 3); rejected(bad)                 # offset not a multiple of 8
+    bad = bytearray(good); struct.pack_into("<Q", bad, rec0, inf0.n_elems + 5000); rejected(bad)  # tile count mismatch
