@@ -2,7 +2,6 @@
 #include "rans.h"
 
 #include <algorithm>
-#include <atomic>
 #include <cstring>
 
 #include "codec.h"
