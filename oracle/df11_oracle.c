@@ -22,6 +22,10 @@
  *          offline and replaces the 8 bits by shorter lookup keys.
  *  [ECF8]  "To Compress or Not? ... Exponent Concentration", Abstract: the same
  *          exponent coding applied to FP8 weights.
+ *  [SHANNON] "Approaching Shannon Bound with Lossless LLM Weight
+ *          Compression", Abstract: tile-level decoding with Asymmetric
+ *          Numeral Systems, within 0.01-0.1 bits of the Shannon limit
+ *          (section 9, the rANS variant).
  *
  * Where the sources are silent the oracle takes these readings (all listed
  * in the repository's design notes):
@@ -50,7 +54,10 @@
  * Parity status: every function here is pinned by tests that do not reuse
  * it (round-trip identity, Kraft equality, entropy bounds, brute-force
  * optimality, closed forms, hand-derived golden streams, an independent
- * dynamic program for length-limited optimality, independent aux walks).
+ * dynamic program for length-limited optimality, independent aux walks, a
+ * tally of code starts for the chunk counts; for section 9 hand-derived
+ * frequencies, states and words, closed forms, the information bound and
+ * the distance to the Shannon limit).
  */
 #include <stdint.h>
 #include <stdlib.h>
