@@ -24,6 +24,7 @@ import argparse
 import datetime
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -53,10 +54,13 @@ def parse_args():
     p.add_argument("--workload", choices=["whole_model", "block", "e4m3"], default="whole_model")
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--e2e-steps", type=int, default=3)
-    p.add_argument("--cpu-seconds", type=float, default=10.0)
+    p.add_argument("--cpu-seconds", type=float, default=6.0)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
     p.add_argument("--no-encode", action="store_true", help="skip the GPU encoder measurement")
+    p.add_argument("--no-extra", action="store_true",
+                   help="skip the extra measurements of the default line (sustained, two-phase, block, single "
+                        "matrices with an L2 flush, E4M3, rANS)")
     p.add_argument("--chunk-bits", type=int, default=128)
     p.add_argument("--tile-threads", type=int, default=32)
     p.add_argument("--chunks-per-thread", type=int, default=0, help="decode launch option (0 = library default)")
@@ -235,50 +239,54 @@ def host_threads(world: int) -> int:
 
 # ------------------------------------------------------------------ CPU oracle
 
-def oracle_decode_sample(groups_host, seconds: float):
-    """Times the CPU oracle decoder (single-threaded) on whole tensors of the
-    workload, in order, until `seconds` of decode time have accumulated.
-    The oracle decodes the same compressed stream the GPU decodes."""
+def oracle_prepare(groups_host, chunk_bits: int, tile_threads: int, budget: int):
+    """Compresses whole tensors of the workload with the oracle itself (its
+    own code lengths, one code per group), in order, until `budget` weights:
+    the oracle decodes streams it wrote, so no library code is involved."""
     import oracle
     oracle.build()
+    out = []
+    for gname, dt, lengths, tensors in groups_host:
+        for tname, bits in tensors:
+            out.append((f"{gname}.{tname}", oracle.compress(bits, dt, lengths=lengths, chunk_bits=chunk_bits,
+                                                            tile_threads=tile_threads), bits))
+            if sum(c.n for _, c, _ in out) >= budget:
+                return out
+    return out
+
+
+def oracle_decode_sample(prepared, seconds: float):
+    """Times the CPU oracle decoder (single-threaded) on whole tensors, in
+    order, until `seconds` of decode time have accumulated; each result is
+    checked against the source weights outside the timed part."""
+    import oracle
     done_w, spent, names = 0, 0.0, []
-    for gname, tensors in groups_host:
-        for tname, dt, n, lengths, sec in tensors:
-            nsym = 256 if dt == "bf16" else 16
-            t0 = time.perf_counter()
-            exps = oracle.decode(sec["stream"], int(sec["total_bits"]), lengths[:nsym], 0, n)
-            oracle.merge(exps, sec["plane"], n, dt)
-            spent += time.perf_counter() - t0
-            done_w += n
-            names.append(f"{gname}.{tname}")
-            if spent >= seconds:
-                return done_w, spent, names
+    for name, c, bits in prepared:
+        t0 = time.perf_counter()
+        got = oracle.decompress(c)
+        spent += time.perf_counter() - t0
+        assert np.array_equal(got, bits), name
+        done_w += c.n
+        names.append(name)
+        if spent >= seconds:
+            break
     return done_w, spent, names
 
 
-def _oracle_decode_task(task):
+def _oracle_decode_task(c):
     """Worker of oracle_decode_parallel: one whole tensor through the oracle."""
     import oracle
-    stream, total_bits, lengths, n, plane, dt = task
     t0 = time.perf_counter()
-    exps = oracle.decode(stream, total_bits, lengths, 0, n)
-    oracle.merge(exps, plane, n, dt)
-    return n, time.perf_counter() - t0
+    oracle.decompress(c)
+    return c.n, time.perf_counter() - t0
 
 
-def oracle_decode_parallel(groups_host, cores: int):
+def oracle_decode_parallel(prepared, cores: int):
     """The same oracle decode on every host core at once: whole tensors, one
     per task, in a pool of `cores` processes started with spawn.  Returns
     (weights, wall seconds around the whole map, tensors)."""
     import multiprocessing as mp
-    import oracle
-    oracle.build()
-    tasks = []
-    for gname, tensors in groups_host:
-        for tname, dt, n, lengths, sec in tensors:
-            nsym = 256 if dt == "bf16" else 16
-            tasks.append((sec["stream"], int(sec["total_bits"]), lengths[:nsym], n, sec["plane"], dt))
-    tasks.sort(key=lambda t: -t[3])  # longest first
+    tasks = sorted((c for _, c, _ in prepared), key=lambda c: -c.n)  # longest first
     with mp.get_context("spawn").Pool(cores) as pool:
         pool.map(_oracle_decode_task, tasks[-1:])  # workers up before the clock starts
         t0 = time.perf_counter()
@@ -290,38 +298,32 @@ def oracle_decode_parallel(groups_host, cores: int):
 # ------------------------------------------------------------------ reference arm
 
 def run_reference(args, rank: int, world: int):
+    """The oracle end to end: it builds its own code for the group, compresses
+    the group's first tensor and, per step, decodes it on one host core.  The
+    library is not loaded."""
     if rank != 0:
         return
     cfg = full_config(args, world)
     gi = 1 if args.workload == "whole_model" else 0
     g = make_group(args.workload, args.seed, gi)
-    from entropy_decoding_b200 import df11
     import oracle
     oracle.build()
     t = g.tensors[0]
     dt = "bf16" if t.bits.dtype == np.uint16 else "e4m3"
-    cb = df11.df11_build_codebook(dt, [x.bits for x in g.tensors])
-    blob = df11.df11_encode(cb, t.bits)
-    sec = blob.sections()
-    info = blob.info()
-    lengths = cb.lengths()
+    lengths = oracle.build_lengths([x.bits for x in g.tensors], dt)
+    c = oracle.compress(t.bits, dt, lengths=lengths, chunk_bits=args.chunk_bits, tile_threads=args.tile_threads)
     n = t.bits.size
-
-    def step():
-        exps = oracle.decode(sec["stream"], int(info.total_bits), lengths, 0, n)
-        return oracle.merge(exps, sec["plane"], n, dt)
-
     for _ in range(args.warmup):
-        step()
+        oracle.decompress(c)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        out = step()
+        out = oracle.decompress(c)
     el = time.perf_counter() - t0
     assert np.array_equal(out, t.bits)
     out_bytes = n * (2 if dt == "bf16" else 1)
     value = out_bytes * args.steps / el / 1e9
-    sample = (f"{g.name}.{t.name} ({n} weights) per step, decoded by the single-threaded CPU oracle "
-              f"from the library's compressed stream")
+    sample = (f"{g.name}.{t.name} ({n} weights) per step: compressed by the oracle with its own code for the "
+              f"group, decoded by the single-threaded CPU oracle (bit-by-bit code walk + field merge)")
     line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "u32", "data": "synthetic",
@@ -329,6 +331,122 @@ def run_reference(args, rank: int, world: int):
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ single-launch measurements
+
+L2_FLUSH_BYTES = 256 << 20  # written between timed launches: more than 2 x the 126 MB L2
+
+
+def timed_launches(torch, stream, launch, flush, smi_index: int, min_s: float = 0.3, min_reps: int = 20,
+                   max_reps: int = 5000):
+    """CUDA-event times of single launches on `stream`, each preceded by an
+    L2 flush outside its events; at least min_reps launches and about min_s
+    seconds, with the SM clocks sampled meanwhile.  Returns (median ms, min
+    ms, reps, clocks)."""
+    for _ in range(3):
+        flush()
+        launch()
+    stream.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(3)]
+    for a, b in ev:
+        flush()
+        a.record(stream)
+        launch()
+        b.record(stream)
+    stream.synchronize()
+    est = statistics.median(a.elapsed_time(b) for a, b in ev)
+    reps = int(min(max_reps, max(min_reps, min_s * 1e3 / (est + 0.06))))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    clocks = ClockSampler(smi_index)
+    clocks.start()
+    time.sleep(0.3)
+    for a, b in ev:
+        flush()
+        a.record(stream)
+        launch()
+        b.record(stream)
+    stream.synchronize()
+    clk = clocks.stop()
+    ms = [a.elapsed_time(b) for a, b in ev]
+    return statistics.median(ms), min(ms), reps, clk
+
+
+def huffman_single(df11, torch, stream, dev, xs, dt, flush, smi_index, peak, label, threads, count_walk=0):
+    """One group (one codebook, one launch) encoded on the host, decoded from
+    HBM: median launch time with an L2 flush between launches, the roofline
+    fraction of the algorithmic bytes, and a full comparison with the source."""
+    cb = df11.df11_build_codebook(dt, xs)
+    blobs = [df11.df11_encode(cb, x, 128, 32, threads) for x in xs]
+    with torch.cuda.stream(stream):
+        for b in blobs:
+            df11.upload(b, stream)
+        outs = [torch.empty(max(16, x.size * x.itemsize + 64), dtype=torch.uint8, device=dev) for x in xs]
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream.synchronize()
+    shape = df11.df11_decode_launch_shape(blobs, with_walk=True, count_walk=count_walk)
+    algo = 0
+    for b in blobs:
+        i = b.info()
+        algo += i.stream_bytes + i.plane_bytes + i.gaps_bytes + i.out_off_bytes + i.uncompressed_bytes
+        algo += i.counts_bytes if shape[4] else 0
+    out_bytes = sum(x.size * x.itemsize for x in xs)
+
+    def launch():
+        df11.df11_decode_ex(blobs, [o.data_ptr() for o in outs], err.data_ptr(), stream.cuda_stream,
+                            count_walk=count_walk)
+
+    med, mn, reps, clk = timed_launches(torch, stream, launch, flush, smi_index)
+    assert int(err.item()) == 0, f"{label}: device error word {int(err.item())}"
+    for x, o in zip(xs, outs):
+        src = torch.from_numpy(x.view(np.int16) if x.dtype == np.uint16 else x).to(dev)
+        got = o[: x.size * x.itemsize].view(torch.int16 if x.dtype == np.uint16 else torch.uint8)
+        assert torch.equal(got, src), f"{label}: output differs from the source"
+    ser = sum(b.info().serialized_bytes for b in blobs)
+    nw = sum(x.size for x in xs)
+    nwarp = shape[1] // 32
+    kern = (f"decode_fsm_kernel<{dt},128,{nwarp},{'true' if shape[4] else 'false'}>" if shape[3] == 2
+            else f"decode_warp_kernel<{dt},128,{nwarp}>")
+    return {"value": out_bytes / (med / 1e3) / 1e9, "unit": "GB/s", "ms": med, "ms_min": mn, "reps": reps,
+            "weights_per_s": nw / (med / 1e3), "weights": nw, "compression_ratio": ser / out_bytes,
+            "roofline": {"bound": "hbm", "achieved": algo / (med / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                         "frac": algo / (med / 1e3) / 1e9 / peak, "algorithmic_bytes": algo, "kernel": kern,
+                         "stored_counts": bool(shape[4])},
+            "l2": f"flushed: {L2_FLUSH_BYTES >> 20} MB written between launches", "clocks": clk,
+            "workload": label, "checked": "every output equal to the source"}
+
+
+def rans_single(df11, torch, stream, dev, xs, dt, flush, smi_index, peak, label, threads):
+    """The rANS variant on one group: one launch, timed and checked as huffman_single."""
+    rg = df11.df11_rans_encode_group(dt, xs, 0, threads)
+    with torch.cuda.stream(stream):
+        df11.rans_upload(rg, stream)
+        outs = [torch.empty(max(16, x.size * x.itemsize + 64), dtype=torch.uint8, device=dev) for x in xs]
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream.synchronize()
+    coded = sum(rg.info(i).coded_bytes + rg.info(i).plane_bytes for i in range(len(xs)))
+    out_bytes = sum(x.size * x.itemsize for x in xs)
+    algo = coded + out_bytes
+
+    def launch():
+        df11.df11_rans_decode(rg, [o.data_ptr() for o in outs], err.data_ptr(), stream.cuda_stream)
+
+    med, mn, reps, clk = timed_launches(torch, stream, launch, flush, smi_index)
+    assert int(err.item()) == 0, f"{label}: device error word {int(err.item())}"
+    for x, o in zip(xs, outs):
+        src = torch.from_numpy(x.view(np.int16) if x.dtype == np.uint16 else x).to(dev)
+        got = o[: x.size * x.itemsize].view(torch.int16 if x.dtype == np.uint16 else torch.uint8)
+        assert torch.equal(got, src), f"{label}: output differs from the source"
+    nw = sum(x.size for x in xs)
+    freq_bytes = 2 * (256 if dt == "bf16" else 16)
+    return {"value": out_bytes / (med / 1e3) / 1e9, "unit": "GB/s", "ms": med, "ms_min": mn, "reps": reps,
+            "weights_per_s": nw / (med / 1e3), "weights": nw,
+            "bits_per_weight": 8 * (coded + freq_bytes) / nw,
+            "roofline": {"bound": "hbm", "achieved": algo / (med / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                         "frac": algo / (med / 1e3) / 1e9 / peak, "algorithmic_bytes": algo,
+                         "kernel": f"rans_decode_kernel<{dt},32>"},
+            "l2": f"flushed: {L2_FLUSH_BYTES >> 20} MB written between launches", "clocks": clk,
+            "workload": label, "checked": "every output equal to the source"}
 
 
 # ------------------------------------------------------------------ our arm
@@ -385,10 +503,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             uncompressed_total += i.uncompressed_bytes
             max_len = max(max_len, i.max_code_len)
             tensors_meta.append(i)
-        if rank == 0 and not args.no_cpu and gi in (1, 2, 3):
-            lengths = cb.lengths()
-            host_for_cpu.append((g.name, [(t.name, dt, t.bits.size, lengths, {**b.sections(),
-                                 "total_bits": b.info().total_bits}) for t, b in zip(g.tensors, blobs)]))
+        if rank == 0 and world == 1 and not args.no_cpu and gi in (1, 2, 3):
+            # raw weights for the oracle baseline, which compresses them itself
+            host_for_cpu.append((g.name, dt, [(t.name, t.bits) for t in g.tensors]))
         groups.append([g.name, blobs, dt])
         del g
     setup_s = time.time() - t_setup
@@ -493,6 +610,91 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         assert bad == 0, f"{what}: {bad} sampled outputs differ from the source weights"
 
     check_samples("decode")
+    smi_index = torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank
+    peak, peak_src = hbm_peak()
+    extras = world == 1 and not args.no_extra
+
+    # ---- the same step held for seconds (clocks settle under the power cap),
+    # and the pages' two phases: each chunk's codes counted by a first walk
+    def whole_run(nsteps: int, count_walk: int):
+        def step():
+            for name, blobs, dt, dsts in groups:
+                df11.df11_decode_ex(blobs, [d[0] for d in dsts], err.data_ptr(), stream.cuda_stream,
+                                    args.chunks_per_thread, args.ctas_per_sm, args.warps_per_cta, walker, 0,
+                                    int(args.overlap), count_walk=count_walk)
+        for _ in range(3):
+            step()
+        stream.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        cs = ClockSampler(smi_index)
+        cs.start()
+        time.sleep(0.3)
+        a.record(stream)
+        for _ in range(nsteps):
+            step()
+        b.record(stream)
+        b.synchronize()
+        c = cs.stop()
+        ms = a.elapsed_time(b) / nsteps
+        counts_read = df11.df11_decode_launch_shape(groups[big][1], args.chunks_per_thread, args.ctas_per_sm,
+                                                    args.warps_per_cta, walker, with_walk=True,
+                                                    count_walk=count_walk)[4]
+        algo_b = 0
+        for i in tensors_meta:
+            algo_b += i.stream_bytes + i.plane_bytes + i.gaps_bytes + i.out_off_bytes + i.uncompressed_bytes
+            algo_b += i.counts_bytes if counts_read else 0
+        return {"value": out_bytes_total / (ms / 1e3) / 1e9, "unit": "GB/s", "ms_per_step": ms, "steps": nsteps,
+                "seconds": ms * nsteps / 1e3,
+                "roofline": {"bound": "hbm", "achieved": algo_b / (ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                             "frac": algo_b / (ms / 1e3) / 1e9 / peak, "algorithmic_bytes_per_step": algo_b,
+                             "stored_counts": bool(counts_read)},
+                "clocks": c}
+
+    sub = {}
+    if extras:
+        n_sus = max(args.steps, int(math.ceil(2.0 / (elapsed_ms / args.steps / 1e3))))
+        sub["sustained"] = {**whole_run(n_sus, int(args.count_walk)),
+                            "what": "the headline step repeated for about 2 s (steady state under the power cap)"}
+        check_samples("sustained")
+        if not args.count_walk and shape[3] == 2:
+            tp = whole_run(args.steps, 1)
+            tp_s = whole_run(n_sus, 1)
+            check_samples("two_phase")
+            sub["two_phase"] = {**tp, "sustained": tp_s,
+                                "what": "whole model, each chunk's codes counted by a first walk (phase 1), "
+                                        "warp scan, then the decoding walk (phase 2): the two-phase kernel of "
+                                        "the DFloat11 Abstract, item (ii); the images keep their stored counts "
+                                        "but the launches do not read them"}
+        # the block workload: one launch of the first transformer block alone
+        gb = 1 if len(groups) > 2 else big
+        _, blobs_b, dt_b, dsts_b = groups[gb]
+        flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+        def flush():
+            with torch.cuda.stream(stream):
+                flush_buf.fill_(1)
+
+        for cw in (0, 1):
+            def launch_b(cw=cw):
+                df11.df11_decode_ex(blobs_b, [d[0] for d in dsts_b], err.data_ptr(), stream.cuda_stream,
+                                    count_walk=cw)
+            med, mn, reps, clk_b = timed_launches(torch, stream, launch_b, flush, smi_index)
+            cr = df11.df11_decode_launch_shape(blobs_b, with_walk=True, count_walk=cw)[4]
+            ab = 0
+            for b in blobs_b:
+                i = b.info()
+                ab += i.stream_bytes + i.plane_bytes + i.gaps_bytes + i.out_off_bytes + i.uncompressed_bytes
+                ab += i.counts_bytes if cr else 0
+            ob = sum(d[2] for d in dsts_b)
+            sub["block" if cw == 0 else "block_two_phase"] = {
+                "value": ob / (med / 1e3) / 1e9, "unit": "GB/s", "ms": med, "ms_min": mn, "reps": reps,
+                "weights_per_s": sum(b.info().n_elems for b in blobs_b) / (med / 1e3),
+                "roofline": {"bound": "hbm", "achieved": ab / (med / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                             "frac": ab / (med / 1e3) / 1e9 / peak, "algorithmic_bytes": ab,
+                             "stored_counts": bool(cr)},
+                "l2": f"flushed: {L2_FLUSH_BYTES >> 20} MB written between launches", "clocks": clk_b,
+                "workload": f"one Llama-3-8B-shaped transformer block ({groups[gb][0]}), shared code, 1 launch"}
+        check_samples("block")
 
     # ---- end to end through the C-ABI with host buffers (pinned)
     e2e = None
@@ -584,13 +786,20 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     # ---- CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu and host_for_cpu:
-        w, sec, names = oracle_decode_sample(host_for_cpu, args.cpu_seconds)
+        import oracle
+        oracle.build()
+        ghost = [(gname, dt, oracle.build_lengths([b for _, b in ts], dt), ts) for gname, dt, ts in host_for_cpu]
+        prepared = oracle_prepare(ghost, args.chunk_bits, args.tile_threads, int(args.cpu_seconds * 1.2e8))
+        del ghost, host_for_cpu
+        w, sec, names = oracle_decode_sample(prepared, args.cpu_seconds)
         cpu = {"value": 2 * w / sec / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
                "sample": f"{w} weights ({len(names)} whole tensors from blocks 0-2, {names[0]} ... {names[-1]}), "
-                         f"single-threaded bit-by-bit oracle decode + field merge, {sec:.1f} s"}
+                         f"compressed by the oracle with its own per-block code, then single-threaded "
+                         f"bit-by-bit oracle decode + field merge, {sec:.1f} s"}
         cores = host_threads(1)
         if cores > 1:
-            wa, wall, nt = oracle_decode_parallel(host_for_cpu, cores)
+            prepared = [p_ for p_ in prepared if p_[0] in names]
+            wa, wall, nt = oracle_decode_parallel(prepared, cores)
             cpu["all_cores"] = {"value": 2 * wa / wall / 1e9, "unit": "GB/s", "cores": cores,
                                 "weights_per_s": wa / wall,
                                 "sample": f"{wa} weights ({nt} whole tensors of blocks 0-2), one tensor per "
@@ -630,6 +839,30 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                          f"bit packing and gap/out_off, one image per tensor; wall clock over {reps} repetitions"}
         del res
 
+    # ---- the other workloads, one launch each, with an L2 flush between
+    # launches (the whole model's memory is released first)
+    if extras:
+        for _, blobs, _, _ in groups:
+            for b in blobs:
+                b._keep = None
+        del out
+        torch.cuda.empty_cache()
+        wl = [("c1_l2_flushed", "bf16", lambda: synth.single_matrix(args.seed)[0],
+               "single 1024x1024 BF16 matrix, N(0, 0.02)"),
+              ("c2_l2_flushed", "bf16", lambda: synth.heavy_tail_matrix(args.seed)[0],
+               "4096x4096 BF16, 0.02 t(3) with 0.1% N(0,1) outliers"),
+              ("e4m3", "e4m3", lambda: synth.e4m3_matrix(args.seed)[0],
+               "8192x28672 FP8 E4M3, N(0, 0.02) scaled to the E4M3 range")]
+        for key, dt_w, make, label in wl:
+            xs = [t.bits for t in make().tensors]
+            sub[key] = huffman_single(df11, torch, stream, dev, xs, dt_w, flush, smi_index, peak, label, threads)
+            del xs
+        xs = [t.bits for t in synth.transformer_block(args.seed)[0].tensors]
+        sub["rans"] = rans_single(df11, torch, stream, dev, xs, "bf16", flush, smi_index, peak,
+                                  "the transformer block, rANS-coded exponents (16,384-symbol tiles, 32 "
+                                  "interleaved coders)", threads)
+        del xs
+
     if rank != 0:
         return
     ms_per_step = elapsed_ms / args.steps
@@ -638,7 +871,6 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     tot_launch_s = per_launch.sum() / 1e3
     algo_step = float(sum(algo))
     achieved = algo_step * args.steps / tot_launch_s / 1e9
-    peak, peak_src = hbm_peak()
     tpw, tsrc = traffic_per_weight()
     n_w = cfg["n_weights"]
     traffic = tpw * n_w / len(groups) if tpw is not None else None
@@ -672,6 +904,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "encode_gpu": enc,
         "e2e": e2e,
         "streamed_from_host": streamed,
+        **sub,
         "gpu_launches": len(groups) * args.steps,
         "clocks": clk,
         "setup_s": setup_s,

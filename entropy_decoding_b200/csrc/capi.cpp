@@ -46,11 +46,16 @@ df11_status from_launch(df11::LaunchStatus s) {
 
 // Events of df11_decode_streamed, created once per device: per slot, "copy
 // done" (recorded on the copy stream) and "slot free" (recorded on the decode
-// stream after the decode that read the slot).
+// stream after the decode that read the slot).  Every call re-records them,
+// so one call's enqueue loop runs under its device's g_enqueue_mu: a wait
+// then always refers to a record made earlier by the same call (or by a call
+// that finished enqueueing before it started, which only adds an ordering),
+// never to a record another thread makes between this call's record and wait.
 constexpr int kStreamSlots = 8;
 constexpr int kEventDevices = 64;
 std::mutex g_event_mu;
 cudaEvent_t g_events[kEventDevices][2 * kStreamSlots] = {};
+std::mutex g_enqueue_mu[kEventDevices];
 
 cudaEvent_t *stream_events() {
     int dev = 0;
@@ -182,6 +187,8 @@ df11_status df11_blob_get_info(const df11_blob *blob, df11_blob_info *info) {
     info->counts_bytes = b.chunk_counts ? b.n_tiles * static_cast<uint64_t>(b.tile_threads) : 0;
     return DF11_OK;
 }
+
+uint64_t df11_blob_compressed_bytes(const df11_blob *blob) { return blob ? df11::serialized_bytes(blob->b) : 0; }
 
 df11_status df11_blob_sections(const df11_blob *blob, const uint8_t **stream, const uint8_t **plane,
                                const uint8_t **gaps, const uint64_t **out_off) {
@@ -355,6 +362,9 @@ df11_status df11_decode_streamed(df11_blob *const *blobs, const int32_t *group_s
         if (!slots[s] || reinterpret_cast<uintptr_t>(slots[s]) % df11::kImageAlign) return DF11_EINVAL;
     cudaEvent_t *ev = stream_events();
     if (!ev) return DF11_ECUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DF11_ECUDA;
+    std::lock_guard<std::mutex> enqueue_lock(g_enqueue_mu[dev]);  // dev < kEventDevices: stream_events checked
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(copy_stream);
     cudaStream_t ds = reinterpret_cast<cudaStream_t>(decode_stream);
     at = 0;
@@ -472,10 +482,10 @@ df11_status df11_encode_device_begin(const df11_codebook *cb, const void *src_de
         enc->job.chunk_counts = !(flags & DF11_ENCODE_NO_CHUNK_COUNTS) && df11::counts_fit(chunk_bits);
         enc->scratch = static_cast<uint64_t *>(scratch_dev);
         enc->stream = reinterpret_cast<cudaStream_t>(stream);
-        std::string err = df11::encode_device_bits(enc->job, enc->scratch, enc->stream, &enc->total_bits);
-        if (!err.empty()) {
+        const df11::EncodeError err = df11::encode_device_bits(enc->job, enc->scratch, enc->stream, &enc->total_bits);
+        if (err != df11::EncodeError::kOk) {
             delete enc;
-            return err.find("cover") != std::string::npos ? DF11_EINVAL : DF11_ECUDA;
+            return err == df11::EncodeError::kUncovered ? DF11_EINVAL : DF11_ECUDA;
         }
         df11::Blob meta;
         meta.dtype = cb->cb->dtype;
@@ -516,9 +526,10 @@ df11_status df11_encode_device_end(df11_encoding *enc, void *image_dev, uint64_t
         b.device_only = true;
         const df11::ImageLayout L = df11::image_layout(b);
         if (b.n) {
-            std::string err = df11::encode_device_pack(enc->job, enc->scratch, b.total_bits, L,
-                                                       static_cast<uint8_t *>(image_dev), enc->stream, &b.max_span);
-            if (!err.empty()) {
+            const df11::EncodeError err = df11::encode_device_pack(enc->job, enc->scratch, b.total_bits, L,
+                                                                   static_cast<uint8_t *>(image_dev), enc->stream,
+                                                                   &b.max_span);
+            if (err != df11::EncodeError::kOk) {
                 delete blob;
                 return DF11_ECUDA;
             }
@@ -577,16 +588,18 @@ df11_status df11_encode_device_noalloc(const df11_codebook *cb, const void *src_
     job.tile_threads = tile_threads;
     job.chunk_counts = !(flags & DF11_ENCODE_NO_CHUNK_COUNTS) && df11::counts_fit(chunk_bits);
     df11::NoallocResult r{};
-    const std::string err = df11::encode_device_noalloc(job, static_cast<uint8_t *>(image_dev), image_cap,
-                                                        reinterpret_cast<cudaStream_t>(stream), &r);
+    const df11::EncodeError err = df11::encode_device_noalloc(job, static_cast<uint8_t *>(image_dev), image_cap,
+                                                              reinterpret_cast<cudaStream_t>(stream), &r);
     result->image_bytes = r.image_bytes;
     result->total_bits = r.total_bits;
     result->n_tiles = r.n_tiles;
     result->max_span = r.max_span;
-    if (err.empty()) return DF11_OK;
-    if (err.find("too small") != std::string::npos) return DF11_ENOMEM;
-    if (err.find("cover") != std::string::npos) return DF11_EINVAL;
-    return DF11_ECUDA;
+    switch (err) {
+        case df11::EncodeError::kOk: return DF11_OK;
+        case df11::EncodeError::kTooSmall: return DF11_ENOMEM;
+        case df11::EncodeError::kUncovered: return DF11_EINVAL;
+        default: return DF11_ECUDA;
+    }
 }
 
 // ---------------------------------------------------------------- rANS coder

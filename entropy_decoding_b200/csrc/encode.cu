@@ -378,15 +378,15 @@ bool launch_histogram(int dtype, const void *src, uint64_t n, uint64_t *counts, 
     return cudaGetLastError() == cudaSuccess;
 }
 
-std::string encode_device_bits(const EncodeJob &J, uint64_t *scratch, cudaStream_t s, uint64_t *total_bits) {
+EncodeError encode_device_bits(const EncodeJob &J, uint64_t *scratch, cudaStream_t s, uint64_t *total_bits) {
     const uint64_t n_seg = segments_of(J.n);
     *total_bits = 0;
-    if (!J.n) return "";
+    if (!J.n) return EncodeError::kOk;
     uint8_t *dev_len = reinterpret_cast<uint8_t *>(scratch + n_seg + 2);  // 256 bytes after the sums
     unsigned long long *uncovered = reinterpret_cast<unsigned long long *>(scratch + n_seg + 2 + 32 + 128);
     if (cudaMemcpyAsync(dev_len, J.cb->lengths, 256, cudaMemcpyHostToDevice, s) != cudaSuccess ||
         cudaMemsetAsync(uncovered, 0, 8, s) != cudaSuccess)
-        return "copy of code lengths failed";
+        return EncodeError::kCuda;
     const int grid = grid_for(n_seg);
     if (J.cb->dtype == kBF16)
         seg_bits_kernel<0><<<grid, kEncThreads, 0, s>>>(J.src, J.n, dev_len, n_seg, scratch, uncovered);
@@ -397,14 +397,14 @@ std::string encode_device_bits(const EncodeJob &J, uint64_t *scratch, cudaStream
     if (cudaMemcpyAsync(&tb, scratch + n_seg, 8, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
         cudaMemcpyAsync(&miss, uncovered, 8, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
         cudaStreamSynchronize(s) != cudaSuccess)
-        return "stream length read-back failed";
-    if (cudaGetLastError() != cudaSuccess) return "kernel launch failed";
-    if (miss) return "tensor holds an exponent the code does not cover";
+        return EncodeError::kCuda;
+    if (cudaGetLastError() != cudaSuccess) return EncodeError::kCuda;
+    if (miss) return EncodeError::kUncovered;
     *total_bits = tb;
-    return "";
+    return EncodeError::kOk;
 }
 
-std::string encode_device_pack(const EncodeJob &J, uint64_t *scratch, uint64_t total_bits, const ImageLayout &L,
+EncodeError encode_device_pack(const EncodeJob &J, uint64_t *scratch, uint64_t total_bits, const ImageLayout &L,
                                uint8_t *image, cudaStream_t s, uint64_t *max_span) {
     const uint64_t n_seg = segments_of(J.n);
     const uint64_t cbits = static_cast<uint64_t>(J.chunk_bits);
@@ -425,14 +425,14 @@ std::string encode_device_pack(const EncodeJob &J, uint64_t *scratch, uint64_t t
     meta_only.chunk_counts = J.chunk_counts && counts_fit(J.chunk_bits);
     write_image_head(meta_only, L, head.data());
     if (cudaMemcpyAsync(image, head.data(), head.size(), cudaMemcpyHostToDevice, s) != cudaSuccess)
-        return "table upload failed";
-    if (cudaMemsetAsync(image + L.gaps, 0, L.total - L.gaps, s) != cudaSuccess) return "memset failed";
+        return EncodeError::kCuda;
+    if (cudaMemsetAsync(image + L.gaps, 0, L.total - L.gaps, s) != cudaSuccess) return EncodeError::kCuda;
     uint64_t *out_off = reinterpret_cast<uint64_t *>(image + L.out_off);
     fill_u64_kernel<<<grid_for((n_tiles + 1 + 255) / 256), 256, 0, s>>>(out_off, n_tiles + 1, J.n);
     uint8_t *dev_len = reinterpret_cast<uint8_t *>(scratch + n_seg + 2);
     uint32_t *dev_codes = reinterpret_cast<uint32_t *>(scratch + n_seg + 2 + 32);  // 1 KB after the lengths
     if (cudaMemcpyAsync(dev_codes, J.cb->codes, 1024, cudaMemcpyHostToDevice, s) != cudaSuccess)
-        return "copy of codes failed";
+        return EncodeError::kCuda;
     PackArgs A;
     A.src = J.src;
     A.n = J.n;
@@ -457,19 +457,19 @@ std::string encode_device_pack(const EncodeJob &J, uint64_t *scratch, uint64_t t
     else
         tail_gaps_kernel<1><<<1, 128, 0, s>>>(J.src, J.n, dev_len, A.gaps, n_chunks, total_bits, A.chunk_bits);
     unsigned long long *dev_max = reinterpret_cast<unsigned long long *>(scratch + n_seg + 1);
-    if (cudaMemsetAsync(dev_max, 0, 8, s) != cudaSuccess) return "memset failed";
+    if (cudaMemsetAsync(dev_max, 0, 8, s) != cudaSuccess) return EncodeError::kCuda;
     max_span_kernel<<<grid_for((n_tiles + 255) / 256), 256, 0, s>>>(out_off, n_tiles, dev_max);
     uint64_t ms = 0;
     if (cudaMemcpyAsync(&ms, dev_max, 8, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
         cudaStreamSynchronize(s) != cudaSuccess)
-        return "max span read-back failed";
-    if (cudaGetLastError() != cudaSuccess) return "kernel launch failed";
+        return EncodeError::kCuda;
+    if (cudaGetLastError() != cudaSuccess) return EncodeError::kCuda;
     // the header was written before the span was known
     if (cudaMemcpyAsync(image + offsetof(ImageHeader, max_span), &ms, 8, cudaMemcpyHostToDevice, s) != cudaSuccess ||
         cudaStreamSynchronize(s) != cudaSuccess)
-        return "header update failed";
+        return EncodeError::kCuda;
     *max_span = ms;
-    return "";
+    return EncodeError::kOk;
 }
 
 // ---------------------------------------------------------------- encoding without allocation
@@ -491,26 +491,26 @@ uint64_t *g_noalloc_addr[kNoallocDevices] = {};
 
 uint64_t noalloc_max_elems() { return (kNoallocScratchWords - (2 + 32 + 128 + 1)) * kSegElems; }
 
-std::string encode_device_noalloc(const EncodeJob &J, uint8_t *image, uint64_t image_cap, cudaStream_t s,
+EncodeError encode_device_noalloc(const EncodeJob &J, uint8_t *image, uint64_t image_cap, cudaStream_t s,
                                   NoallocResult *r) {
     // device address of the static scratch on the current device, looked up
     // once per device (host code cannot use the symbol itself)
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocDevices) return "no current device";
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocDevices) return EncodeError::kCuda;
     uint64_t *scratch = nullptr;
     {
         std::lock_guard<std::mutex> lk(g_noalloc_mu);
         if (!g_noalloc_addr[dev]) {
             void *p = nullptr;
-            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return "scratch lookup failed";
+            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return EncodeError::kCuda;
             g_noalloc_addr[dev] = static_cast<uint64_t *>(p);
         }
         scratch = g_noalloc_addr[dev];
     }
     // pass 1: every slot it reads is written first (sums, total, flag)
     uint64_t total = 0;
-    std::string err = encode_device_bits(J, scratch, s, &total);
-    if (!err.empty()) return err;
+    const EncodeError err = encode_device_bits(J, scratch, s, &total);
+    if (err != EncodeError::kOk) return err;
     Blob meta;  // metadata only: its sections stay empty
     meta.dtype = J.cb->dtype;
     meta.chunk_bits = J.chunk_bits;
@@ -527,7 +527,7 @@ std::string encode_device_noalloc(const EncodeJob &J, uint8_t *image, uint64_t i
     r->total_bits = total;
     r->n_tiles = meta.n_tiles;
     r->max_span = 0;
-    if (image_cap < L.total) return "image buffer too small";
+    if (image_cap < L.total) return EncodeError::kTooSmall;
     // header and decode tables, copied from the codebook without a staging buffer
     ImageHeader h{};
     std::memcpy(h.magic, "DF11IMG1", 8);
@@ -549,8 +549,8 @@ std::string encode_device_noalloc(const EncodeJob &J, uint8_t *image, uint64_t i
             cudaSuccess ||
         cudaMemcpyAsync(image + L.fsm, J.cb->fsm.data(), J.cb->fsm.size() * 4, cudaMemcpyHostToDevice, s) !=
             cudaSuccess)
-        return "table upload failed";
-    if (!J.n) return cudaStreamSynchronize(s) == cudaSuccess ? "" : "synchronise failed";
+        return EncodeError::kCuda;
+    if (!J.n) return cudaStreamSynchronize(s) == cudaSuccess ? EncodeError::kOk : EncodeError::kCuda;
     // pass 2, as in encode_device_pack
     const uint64_t n_seg = segments_of(J.n);
     uint64_t *out_off = reinterpret_cast<uint64_t *>(image + L.out_off);
@@ -558,7 +558,7 @@ std::string encode_device_noalloc(const EncodeJob &J, uint8_t *image, uint64_t i
     uint8_t *dev_len = reinterpret_cast<uint8_t *>(scratch + n_seg + 2);
     uint32_t *dev_codes = reinterpret_cast<uint32_t *>(scratch + n_seg + 2 + 32);
     if (cudaMemcpyAsync(dev_codes, J.cb->codes, 1024, cudaMemcpyHostToDevice, s) != cudaSuccess)
-        return "copy of codes failed";
+        return EncodeError::kCuda;
     PackArgs A;
     A.src = J.src;
     A.n = J.n;
@@ -582,18 +582,18 @@ std::string encode_device_noalloc(const EncodeJob &J, uint8_t *image, uint64_t i
     }
     // the span accumulator keeps the previous call's value: clear it
     unsigned long long *dev_max = reinterpret_cast<unsigned long long *>(scratch + n_seg + 1);
-    if (cudaMemsetAsync(dev_max, 0, 8, s) != cudaSuccess) return "memset failed";
+    if (cudaMemsetAsync(dev_max, 0, 8, s) != cudaSuccess) return EncodeError::kCuda;
     max_span_kernel<<<grid_for((meta.n_tiles + 255) / 256), 256, 0, s>>>(out_off, meta.n_tiles, dev_max);
     uint64_t ms = 0;
     if (cudaMemcpyAsync(&ms, dev_max, 8, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
         cudaStreamSynchronize(s) != cudaSuccess)
-        return "max span read-back failed";
-    if (cudaGetLastError() != cudaSuccess) return "kernel launch failed";
+        return EncodeError::kCuda;
+    if (cudaGetLastError() != cudaSuccess) return EncodeError::kCuda;
     if (cudaMemcpyAsync(image + offsetof(ImageHeader, max_span), &ms, 8, cudaMemcpyHostToDevice, s) != cudaSuccess ||
         cudaStreamSynchronize(s) != cudaSuccess)
-        return "header update failed";
+        return EncodeError::kCuda;
     r->max_span = ms;
-    return "";
+    return EncodeError::kOk;
 }
 
 }  // namespace df11

@@ -26,13 +26,17 @@ uint64_t encode_scratch_bytes(uint64_t n);
 
 bool launch_histogram(int dtype, const void *src, uint64_t n, uint64_t *counts, cudaStream_t s);
 
+// Outcome of a device encode step (no strings: the allocation-free path
+// touches no host heap either).
+enum class EncodeError { kOk, kUncovered, kTooSmall, kCuda };
+
 // Pass 1: bits per segment, their exclusive scan (left in scratch) and the
 // total, read back to the host (synchronises s).
-std::string encode_device_bits(const EncodeJob &J, uint64_t *scratch, cudaStream_t s, uint64_t *total_bits);
+EncodeError encode_device_bits(const EncodeJob &J, uint64_t *scratch, cudaStream_t s, uint64_t *total_bits);
 
 // Pass 2: the device image at `image` (layout L), from the scan in scratch;
 // reads back the largest tile span (synchronises s).
-std::string encode_device_pack(const EncodeJob &J, uint64_t *scratch, uint64_t total_bits, const ImageLayout &L,
+EncodeError encode_device_pack(const EncodeJob &J, uint64_t *scratch, uint64_t total_bits, const ImageLayout &L,
                                uint8_t *image, cudaStream_t s, uint64_t *max_span);
 
 // Encoding without any allocation: the scratch is a static device array of
@@ -42,7 +46,7 @@ struct NoallocResult {
     uint64_t image_bytes, total_bits, n_tiles, max_span;
 };
 uint64_t noalloc_max_elems();
-std::string encode_device_noalloc(const EncodeJob &J, uint8_t *image, uint64_t image_cap, cudaStream_t s,
+EncodeError encode_device_noalloc(const EncodeJob &J, uint8_t *image, uint64_t image_cap, cudaStream_t s,
                                   NoallocResult *r);
 
 }  // namespace df11

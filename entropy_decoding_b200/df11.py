@@ -91,6 +91,7 @@ _SIGS = {
     "df11_layout_supported": ([_I, _I, _I], _I),
     "df11_blob_free": ([_P], None),
     "df11_blob_get_info": ([_P, ctypes.POINTER(BlobInfo)], _S),
+    "df11_blob_compressed_bytes": ([_P], _U64),
     "df11_blob_sections": ([_P, _PP, _PP, _PP, _PP], _S),
     "df11_blob_chunk_counts": ([_P, _PP], _S),
     "df11_blob_lengths": ([_P, _P], _S),
@@ -167,7 +168,7 @@ class Codebook:
     def __del__(self, _free=_lib.df11_codebook_free):
         if getattr(self, "_h", None) and self._h.value:
             _free(self._h)
-            self._h = ctypes.c_void_p(0)
+            self._h = None
 
 
 class Blob:
@@ -183,6 +184,9 @@ class Blob:
         i = BlobInfo()
         _check(_lib.df11_blob_get_info(self._h, ctypes.byref(i)), "df11_blob_get_info")
         return i
+
+    def compressed_bytes(self) -> int:
+        return int(_lib.df11_blob_compressed_bytes(self._h))
 
     @property
     def dtype(self) -> str:
@@ -225,7 +229,7 @@ class Blob:
     def __del__(self, _free=_lib.df11_blob_free):
         if getattr(self, "_h", None) and self._h.value:
             _free(self._h)
-            self._h = ctypes.c_void_p(0)
+            self._h = None
 
 
 # ----------------------------------------------------------------- functions (same names as the C-ABI)
@@ -377,7 +381,7 @@ class Encoding:
     def __del__(self, _free=_lib.df11_encoding_free):
         if getattr(self, "_h", None) and self._h.value:
             _free(self._h)
-            self._h = ctypes.c_void_p(0)
+            self._h = None
 
 
 def df11_encode_device_begin(cb: Codebook, src_ptr: int, n: int, chunk_bits: int = 128, tile_threads: int = 32,
@@ -518,7 +522,7 @@ class RansGroup:
     def __del__(self, _free=_lib.df11_rans_group_free):
         if getattr(self, "_h", None) and self._h.value:
             _free(self._h)
-            self._h = ctypes.c_void_p(0)
+            self._h = None
 
 
 def df11_rans_encode_group(dtype: str, tensors, tile_symbols: int = 0, n_threads: int = 0) -> RansGroup:

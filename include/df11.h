@@ -179,6 +179,12 @@ typedef struct {
 
 df11_status df11_blob_get_info(const df11_blob *blob, df11_blob_info *info);
 
+/* Size in bytes of the blob's container (df11_serialize's output: header,
+ * code lengths, gaps, chunk counts when present, out_off, stream and plane),
+ * the numerator of the compression ratio; equal to info.serialized_bytes.
+ * 0 for a NULL blob. */
+uint64_t df11_blob_compressed_bytes(const df11_blob *blob);
+
 /* Read-only host views of the blob's sections (valid until the blob is freed);
  * any output pointer may be NULL.  DF11_EINVAL for a GPU-encoded blob that
  * was not fetched (df11_blob_fetch). */
@@ -321,6 +327,11 @@ df11_status df11_decode_host(df11_blob *const *blobs, const void *const *host_im
  * On return every blob is bound to its place in its slot (rebind before
  * decoding it again: the slot is reused).  Allocates no device memory; the
  * first call on a device creates 2 x 8 CUDA events that live until exit.
+ * Calls from several host threads (each with its own streams, slots and
+ * blobs) are safe: the library enqueues one call at a time per device, so
+ * each copy waits for the right decode.  A call may then also wait for the
+ * decodes of a call enqueued before it on other streams (the events are
+ * shared); that orders the two calls but never changes an output.
  * Errors: DF11_EINVAL (arguments, group size, mixed codes in a group),
  * DF11_ENOMEM (a group's images exceed slot_bytes), both found before
  * anything is enqueued; DF11_EUNSUPPORTED and DF11_ECUDA (copy, event or
@@ -421,7 +432,12 @@ df11_status df11_blob_fetch(df11_blob *blob, df11_stream stream);
  *
  * First call per device.  It looks up the array's device address with
  * cudaGetSymbolAddress, with that device current.  Make this first call
- * before any stream capture.
+ * before any stream capture.  With lazy module loading (the CUDA 12
+ * default) that lookup is also when the driver loads the encoder's code and
+ * places the array in device memory, so a program that later reserves
+ * nearly all HBM should make the first call at start-up, before reserving
+ * it (a call with n_elems = 0 and an image buffer of the empty tensor's
+ * size is enough).
  *
  * Overlapping calls.  Every call shares the array, and the array keeps the
  * last call's contents (each call clears what must start at zero). Calls

@@ -467,7 +467,7 @@ int oracle_chunk_counts(const uint8_t *exps, uint64_t n, const uint8_t *lengths,
     uint64_t n_chunks, n_tiles;
     oracle_layout(total, chunk_bits, tile_threads, &n_chunks, &n_tiles);
     uint64_t *tally = (uint64_t *)calloc(n_chunks ? n_chunks : 1, sizeof(uint64_t));
-    if (!tally) return ORACLE_EINVAL;
+    if (!tally) return ORACLE_ENOMEM;
     uint64_t start = 0;
     for (uint64_t i = 0; i < n; i++) {
         tally[start / (uint64_t)chunk_bits]++;

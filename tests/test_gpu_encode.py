@@ -100,14 +100,16 @@ def test_device_encoded_blob_decodes_and_fetches(df11, oracle_mod, case):
     with pytest.raises(df11.Df11Error):
         df11.df11_serialize(blob)  # host sections are not there before the fetch
     df11.df11_blob_fetch(blob)
-    o = oracle_mod.compress(x, dt, lengths=cb.lengths(), chunk_bits=128, tile_threads=32)
+    lengths = oracle_mod.build_lengths([x], dt)
+    assert np.array_equal(cb.lengths(), lengths)
+    o = oracle_mod.compress(x, dt, lengths=lengths, chunk_bits=128, tile_threads=32)
     sec = blob.sections()
     assert np.array_equal(sec["stream"], o.stream)
     assert np.array_equal(sec["plane"], o.plane)
     assert np.array_equal(sec["gaps"], o.gaps)
     assert np.array_equal(sec["out_off"], o.out_off)
     exps, _ = oracle_mod.split(x, dt)
-    assert np.array_equal(sec["counts"], oracle_mod.chunk_counts(exps, cb.lengths(), 128, 32))
+    assert np.array_equal(sec["counts"], oracle_mod.chunk_counts(exps, lengths, 128, 32))
     assert df11.df11_serialize(blob) == df11.df11_serialize(df11.df11_encode(cb, x))
 
 

@@ -71,7 +71,7 @@ def test_full_size_small_configs(df11, oracle_mod, cfg):
     (out,), err = _decode_group(df11, [blob])
     assert err == 0
     host = out[: 2 * x.size].cpu().numpy().view(np.uint16)
-    want = oracle_mod.decompress(oracle_mod.compress(x, "bf16", lengths=cb.lengths()))
+    want = oracle_mod.decompress(oracle_mod.compress(x, "bf16"))
     assert np.array_equal(host, want)
     assert np.array_equal(host, x)
     if cfg.startswith("heavy"):
@@ -85,8 +85,8 @@ def test_full_size_transformer_block_one_launch(df11, oracle_mod, count_walk):
     g = synth.transformer_block(0)[0]
     xs = [t.bits for t in g.tensors]
     cb = df11.df11_build_codebook("bf16", xs)
-    lengths = cb.lengths()
-    assert np.array_equal(lengths, oracle_mod.build_lengths(xs, "bf16"))
+    lengths = oracle_mod.build_lengths(xs, "bf16")
+    assert np.array_equal(cb.lengths(), lengths)
     blobs = [df11.df11_encode(cb, x) for x in xs]
     assert sum(b.info().n_elems for b in blobs) == 218103808
     outs, err = _decode_group(df11, blobs, count_walk)
@@ -105,7 +105,7 @@ def test_full_size_e4m3(df11, oracle_mod):
     (out,), err = _decode_group(df11, [blob])
     assert err == 0
     assert _device_equal(out, x)
-    _sampled_oracle(oracle_mod, df11, x, "e4m3", cb.lengths(), out, seed=3)
+    _sampled_oracle(oracle_mod, df11, x, "e4m3", oracle_mod.build_lengths([x], "e4m3"), out, seed=3)
 
 
 @pytest.mark.slow
@@ -125,7 +125,7 @@ def test_full_size_whole_model(df11, oracle_mod):
             assert _device_equal(out, x), g.name
             total += x.size
         if gi in (0, 1, n_groups - 1):
-            _sampled_oracle(oracle_mod, df11, xs[-1][: 50_000_000], "bf16", cb.lengths(),
+            _sampled_oracle(oracle_mod, df11, xs[-1][: 50_000_000], "bf16", oracle_mod.build_lengths(xs, "bf16"),
                             _decode_group(df11, [df11.df11_encode(cb, xs[-1][: 50_000_000])])[0][0],
                             n_samples=64, seed=gi)
         del outs, blobs, xs, g

@@ -90,3 +90,57 @@ def test_streamed_decode_rejects_small_slot(df11):
         df11.df11_decode_streamed([g[2] for g in groups], [h.data_ptr() for h in imgs], [ptr] * 9, cap,
                                   [o.data_ptr() for o in outs])
     assert e.value.status == df11.DF11_EINVAL
+
+
+def test_streamed_decode_from_two_host_threads(df11):
+    """Two host threads call df11_decode_streamed at the same time, each with
+    its own blobs, staging slots and stream pair, four times in a row.  The
+    library shares one set of events per device between calls, so it must
+    enqueue one call at a time; every output is compared with the oracle's
+    decompression of the same tensor."""
+    import threading
+
+    import oracle
+    oracle.build()
+    work = []
+    for t in range(2):
+        groups = _groups(df11)  # fresh blob objects: each call rebinds its own
+        blobs = [b for g in groups for b in g[2]]
+        xs = [x for g in groups for x in g[1]]
+        dts = [g[0] for g in groups for _ in g[1]]
+        imgs = _host_images(df11, blobs)
+        cap = _slot_bytes(groups)
+        slots = [torch.empty(cap + 256, dtype=torch.uint8, device="cuda") for _ in range(2)]
+        outs = [torch.full((x.size * x.itemsize + 64,), 0xA5, dtype=torch.uint8, device="cuda") for x in xs]
+        work.append(dict(groups=groups, xs=xs, dts=dts, imgs=imgs, cap=cap, slots=slots, outs=outs,
+                         err=torch.zeros(1, dtype=torch.int32, device="cuda"),
+                         cs=torch.cuda.Stream(), ds=torch.cuda.Stream()))
+    torch.cuda.synchronize()
+    start = threading.Barrier(2)
+    failures = []
+
+    def run(w):
+        try:
+            start.wait()
+            for _ in range(4):
+                df11.df11_decode_streamed([g[2] for g in w["groups"]], [h.data_ptr() for h in w["imgs"]],
+                                          [s.data_ptr() + (-s.data_ptr()) % 256 for s in w["slots"]], w["cap"],
+                                          [o.data_ptr() for o in w["outs"]], w["err"].data_ptr(),
+                                          w["cs"].cuda_stream, w["ds"].cuda_stream)
+        except Exception as e:  # reported below, on the main thread
+            failures.append(e)
+
+    threads = [threading.Thread(target=run, args=(w,)) for w in work]
+    for th in threads:
+        th.start()
+    for th in threads:
+        th.join()
+    assert not failures, failures
+    torch.cuda.synchronize()
+    for w in work:
+        assert int(w["err"].item()) == 0
+        for x, dt, o in zip(w["xs"], w["dts"], w["outs"]):
+            got = o.cpu().numpy()
+            want = oracle.decompress(oracle.compress(x, dt))
+            assert np.array_equal(got[: x.size * x.itemsize].view(x.dtype), want)
+            assert (got[x.size * x.itemsize:] == 0xA5).all()

@@ -254,7 +254,7 @@ def test_serialize_roundtrip_and_size(df11, oracle_mod):
     blob = df11.df11_encode(cb, x)
     data = df11.df11_serialize(blob)
     info = blob.info()
-    assert len(data) == info.serialized_bytes
+    assert len(data) == info.serialized_bytes == blob.compressed_bytes()
     # near the pages' ~70% of BF16 ("70% Size", DFloat11 title / Abstract)
     assert 0.62 < info.serialized_bytes / info.uncompressed_bytes < 0.72
     b2 = df11.df11_deserialize(data)
@@ -272,6 +272,7 @@ def test_serialize_roundtrip_and_size(df11, oracle_mod):
     b1 = df11.df11_deserialize(d1)
     assert b1.sections()["counts"] is None and b1.info().counts_bytes == 0
     assert df11.df11_serialize(b1) == d1
+    assert b1.compressed_bytes() == len(d1)
 
 
 def _container_offsets(info, counts: bool):

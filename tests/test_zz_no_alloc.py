@@ -165,3 +165,27 @@ def test_empty_input(df11):
     r = df11.df11_encode_device_noalloc(cb, src.data_ptr(), 0, 128, 32, ptr, need)
     assert r.n_tiles == 0 and r.total_bits == 0 and r.max_span == 0
     assert r.image_bytes == need
+
+
+def test_call_takes_no_device_memory(df11):
+    """The defining property: once the first call on the device has looked up
+    the static scratch, a further call of several MB changes neither the
+    device's free memory nor torch's allocation counters (every buffer it
+    uses is allocated, and counted, before the measurement)."""
+    x = synth.heavy_tail_matrix(5)[0].tensors[0].bits[: 6 * 10 ** 6 + 3]
+    cb = df11.df11_build_codebook("bf16", [x])
+    xd = _dev(x)
+    need = df11.df11_encode(cb, x).info().device_bytes
+    buf, ptr, _ = _aligned(need)
+    r0 = df11.df11_encode_device_noalloc(cb, xd.data_ptr(), x.size, 128, 32, ptr, need)  # warm-up
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    stats0 = torch.cuda.memory_stats()
+    r1 = df11.df11_encode_device_noalloc(cb, xd.data_ptr(), x.size, 128, 32, ptr, need)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    stats1 = torch.cuda.memory_stats()
+    assert free1 == free0
+    for k in ("allocation.all.allocated", "segment.all.allocated", "reserved_bytes.all.current"):
+        assert stats1.get(k) == stats0.get(k), k
+    assert (r1.image_bytes, r1.total_bits, r1.max_span) == (r0.image_bytes, r0.total_bits, r0.max_span)
