@@ -12,6 +12,7 @@ the order the method states them:
   split fields -> histogram -> code lengths -> canonical codes -> pack
   -> auxiliary variables          (compression, done offline)
   bit-by-bit tree walk -> merge fields                           (decompression)
+  decompression -> operand-tile order undone -> y = x W          (the fused GEMM)
 
 Sources: "70% Size, 100% Accuracy: Lossless LLM Compression for Efficient GPU
 Inference via Dynamic-Length Float (DFloat11)", Abstract; "Compressing LLMs
@@ -376,3 +377,51 @@ def rans_compress(x: np.ndarray, dtype: str, freqs: np.ndarray | None = None,
 def rans_decompress(c: RansCompressed) -> np.ndarray:
     exps = rans_decode(c.words, c.states, c.tile_words, c.n, c.freqs, c.tile_symbols)
     return merge(exps, c.plane, c.n, c.dtype)
+
+
+# ---------------------------------------------------------------- decode fused into the consuming GEMM
+# ("Compressing LLMs without Compromise" summary page, ZipServ paragraph:
+# decompression fused into the matrix multiply; "Approaching Shannon Bound
+# with Lossless LLM Weight Compression", Abstract: decoding aligned with the
+# GEMM's tiling).  Fusing changes where the decoded weights go, not what is
+# computed: the result is the plain product y = x W of the exactly decoded
+# weights.  The pages give no tile shape; the reading here is one tcgen05
+# MMA's operand tile of 128 output rows x 16 reduction columns, each tile a
+# contiguous run of the encoded weights.
+
+GEMM_TILE_N, GEMM_TILE_K = 128, 16
+
+
+def gemm_tile(w: np.ndarray, k: int, n: int) -> np.ndarray:
+    """Operand-tile order of a K x N matrix (row-major, element (k, n) at
+    k * N + n): tile t = nb * (K / 16) + kb holds W[16 kb + c][128 nb + r] at
+    position 2048 t + 16 r + c."""
+    w = np.asarray(w).reshape(k, n)
+    return w.reshape(k // GEMM_TILE_K, GEMM_TILE_K, n // GEMM_TILE_N, GEMM_TILE_N).transpose(2, 0, 3, 1).reshape(-1)
+
+
+def gemm_untile(t: np.ndarray, k: int, n: int) -> np.ndarray:
+    """Inverse of gemm_tile: the K x N row-major matrix."""
+    t = np.asarray(t).reshape(n // GEMM_TILE_N, k // GEMM_TILE_K, GEMM_TILE_N, GEMM_TILE_K)
+    return t.transpose(1, 3, 0, 2).reshape(k, n)
+
+
+def bf16_to_float(bits: np.ndarray) -> np.ndarray:
+    """BF16 bit patterns -> float64 values (BF16 is the high half of FP32)."""
+    return (np.asarray(bits, np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def gemm(x_bits: np.ndarray, w_bits: np.ndarray, m: int, k: int, n: int) -> np.ndarray:
+    """y = x W in float64 from BF16 bit patterns: x is m x k, W is k x n."""
+    return bf16_to_float(x_bits).reshape(m, k) @ bf16_to_float(w_bits).reshape(k, n)
+
+
+def gemm_abs(x_bits: np.ndarray, w_bits: np.ndarray, m: int, k: int, n: int) -> np.ndarray:
+    """sum_k |x_mk w_kn|, the scale of a float32 accumulation's rounding error."""
+    return np.abs(bf16_to_float(x_bits).reshape(m, k)) @ np.abs(bf16_to_float(w_bits).reshape(k, n))
+
+
+def decode_gemm(c: Compressed, x_bits: np.ndarray, m: int, k: int, n: int) -> np.ndarray:
+    """What the fused path computes from a tiled container: decompress,
+    restore the K x N order, multiply (float64)."""
+    return gemm(x_bits, gemm_untile(decompress(c), k, n), m, k, n)
