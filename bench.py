@@ -449,6 +449,88 @@ def rans_single(df11, torch, stream, dev, xs, dt, flush, smi_index, peak, label,
             "workload": label, "checked": "every output equal to the source"}
 
 
+def fused_gemm_block(df11, torch, stream, dev, tensors, flush, smi_index, peak, threads, m=16):
+    """The decode fused into the consuming GEMM (y += x W) on the block's
+    seven matrices, one launch at batch M = m, against the unfused path on
+    the same weights: the decode launch of the row-major block followed by
+    one cuBLAS BF16 GEMM per matrix (torch.matmul).  Both timed with CUDA
+    events, an L2 flush before every timed launch sequence."""
+    shapes = [tuple(t.shape) for t in tensors]
+    ws = [t.bits for t in tensors]
+    g = np.random.default_rng(2024)
+    xs = [synth.to_bf16_bits(g.standard_normal(m * k).astype(np.float32)) for k, _ in shapes]
+    tiled = [df11.df11_gemm_tile_weights(w, k, n) for w, (k, n) in zip(ws, shapes)]
+    cbt = df11.df11_build_codebook("bf16", tiled)
+    blobs_t = [df11.df11_encode(cbt, t, 128, 32, threads) for t in tiled]
+    del tiled
+    cb = df11.df11_build_codebook("bf16", ws)
+    blobs = [df11.df11_encode(cb, w, 128, 32, threads) for w in ws]
+    with torch.cuda.stream(stream):
+        for b in blobs_t + blobs:
+            df11.upload(b, stream)
+        xd = [torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16).reshape(m, k)
+              for x, (k, _) in zip(xs, shapes)]
+        ys = [torch.zeros(m * n, dtype=torch.float32, device=dev) for _, n in shapes]
+        wout = [torch.empty(2 * k * n, dtype=torch.uint8, device=dev) for k, n in shapes]
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream.synchronize()
+    mats = [(b, k, n, x.data_ptr(), y.data_ptr()) for b, (k, n), x, y in zip(blobs_t, shapes, xd, ys)]
+    wviews = [o.view(torch.bfloat16).reshape(k, n) for o, (k, n) in zip(wout, shapes)]
+
+    def fused():
+        for y in ys:
+            y.zero_()
+        df11.df11_decode_gemm(mats, m, err.data_ptr(), stream.cuda_stream)
+
+    def unfused():
+        df11.df11_decode(blobs, [o.data_ptr() for o in wout], err.data_ptr(), stream.cuda_stream)
+        for x, wv in zip(xd, wviews):
+            torch.matmul(x, wv)
+
+    def gemm_only():
+        for x, wv in zip(xd, wviews):
+            torch.matmul(x, wv)
+
+    with torch.cuda.stream(stream):
+        f_ms, f_min, f_reps, f_clk = timed_launches(torch, stream, fused, flush, smi_index)
+        u_ms, u_min, u_reps, u_clk = timed_launches(torch, stream, unfused, flush, smi_index)
+        g_ms, _, _, _ = timed_launches(torch, stream, gemm_only, flush, smi_index)
+        # correctness outside the timed region: one clean launch against float32 matmuls
+        fused()
+        stream.synchronize()
+        assert int(err.item()) == 0, f"fused gemm: device error word {int(err.item())}"
+        for y, x, wv, (k, n) in zip(ys, xd, wviews, shapes):
+            ref = x.float() @ wv.float()
+            scale = x.float().abs() @ wv.float().abs()
+            assert bool((( y.reshape(m, n) - ref).abs() <= 2 * (k + 16) * 2.0 ** -24 * scale).all()), "fused gemm"
+    nw = sum(k * n for k, n in shapes)
+    comp = 0
+    for b in blobs_t:
+        i = b.info()
+        comp += i.stream_bytes + i.plane_bytes + i.gaps_bytes + i.out_off_bytes + i.counts_bytes
+    act = sum(2 * m * k + 8 * m * n for k, n in shapes)  # x read; y read and written (fp32)
+    algo = comp + act
+    dec_algo = 0
+    for b in blobs:
+        i = b.info()
+        dec_algo += i.stream_bytes + i.plane_bytes + i.gaps_bytes + i.out_off_bytes + i.counts_bytes + 2 * i.n_elems
+    unfused_bytes = dec_algo + 2 * nw + sum(2 * m * k + 2 * m * n for k, n in shapes)
+    shape = df11.df11_decode_gemm_launch_shape([(b, k, n, 0, 0) for b, (k, n) in zip(blobs_t, shapes)], m)
+    return {"value": nw / (f_ms / 1e3), "unit": "weights/s", "ms": f_ms, "ms_min": f_min, "reps": f_reps,
+            "batch_m": m, "weights": nw,
+            "unfused_ms": u_ms, "unfused_gemm_ms": g_ms, "speedup_vs_unfused": u_ms / f_ms,
+            "bytes_per_weight": algo / nw, "unfused_bytes_per_weight": unfused_bytes / nw,
+            "roofline": {"bound": "hbm", "achieved": algo / (f_ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                         "frac": algo / (f_ms / 1e3) / 1e9 / peak, "algorithmic_bytes": algo,
+                         "kernel": "decode_gemm_kernel", "launch": {"grid": shape[0], "block": shape[1],
+                                                                    "smem_bytes": shape[2]}},
+            "clocks": f_clk, "unfused_clocks": u_clk,
+            "l2": f"flushed: {L2_FLUSH_BYTES >> 20} MB written before every timed launch sequence",
+            "workload": f"one Llama-3-8B-shaped transformer block, 7 matrices [in, out], y += x W at M = {m}, "
+                        f"one fused launch; unfused = one decode launch + 7 cuBLAS BF16 GEMMs (torch.matmul)",
+            "checked": "every output within (K + 16) 2^-24 sum|x w| of float32 matmuls of the decoded weights"}
+
+
 # ------------------------------------------------------------------ our arm
 
 def kernel_name(args, cfg: dict, shape) -> str:
@@ -857,11 +939,15 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             xs = [t.bits for t in make().tensors]
             sub[key] = huffman_single(df11, torch, stream, dev, xs, dt_w, flush, smi_index, peak, label, threads)
             del xs
-        xs = [t.bits for t in synth.transformer_block(args.seed)[0].tensors]
+        blk = synth.transformer_block(args.seed)[0]
+        xs = [t.bits for t in blk.tensors]
         sub["rans"] = rans_single(df11, torch, stream, dev, xs, "bf16", flush, smi_index, peak,
                                   "the transformer block, rANS-coded exponents (16,384-symbol tiles, 32 "
                                   "interleaved coders)", threads)
         del xs
+        torch.cuda.empty_cache()
+        sub["fused_gemm"] = fused_gemm_block(df11, torch, stream, dev, blk.tensors, flush, smi_index, peak, threads)
+        del blk
 
     if rank != 0:
         return

@@ -21,9 +21,9 @@ CUDA_HOME = os.environ.get("CUDA_HOME", "/usr/local/cuda")
 NVCC = os.path.join(CUDA_HOME, "bin", "nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
-SOURCES_CU = ["decode.cu", "encode.cu", "rans_decode.cu"]
+SOURCES_CU = ["decode.cu", "encode.cu", "rans_decode.cu", "gemm.cu"]
 SOURCES_CPP = ["codec.cpp", "capi.cpp", "rans.cpp"]
-HEADERS = ["df11_internal.h", "codec.h", "launch.h", "encode.h", "rans.h"]
+HEADERS = ["df11_internal.h", "codec.h", "launch.h", "encode.h", "rans.h", "walk.cuh", "gemm.h"]
 
 
 def _newer(target: str, deps: list[str]) -> bool:

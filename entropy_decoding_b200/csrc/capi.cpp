@@ -10,6 +10,7 @@
 #include "df11.h"
 #include "codec.h"
 #include "encode.h"
+#include "gemm.h"
 #include "launch.h"
 #include "rans.h"
 
@@ -66,6 +67,20 @@ cudaEvent_t *stream_events() {
             if (cudaEventCreateWithFlags(&g_events[dev][i], cudaEventDisableTiming) != cudaSuccess) return nullptr;
     }
     return g_events[dev];
+}
+
+df11_status gemm_jobs(const df11_gemm_matrix *mats, int n_mats, bool stand_ins, df11::GemmJob *jobs) {
+    if (!mats || n_mats < 1 || n_mats > DF11_GEMM_MAX_MATS) return DF11_EINVAL;
+    for (int i = 0; i < n_mats; ++i) {
+        if (!mats[i].weights) return DF11_EINVAL;
+        jobs[i].w = &mats[i].weights->b;
+        jobs[i].k = mats[i].k;
+        jobs[i].n = mats[i].n;
+        // the shape does not depend on x and y: 16-byte aligned stand-ins when absent
+        jobs[i].x = stand_ins && !mats[i].x ? reinterpret_cast<const void *>(uintptr_t{256}) : mats[i].x;
+        jobs[i].y = stand_ins && !mats[i].y ? reinterpret_cast<float *>(uintptr_t{256}) : mats[i].y;
+    }
+    return DF11_OK;
 }
 
 }  // namespace
@@ -391,6 +406,37 @@ df11_status df11_decode_streamed(df11_blob *const *blobs, const int32_t *group_s
         if (cudaEventRecord(freed, ds) != cudaSuccess) return DF11_ECUDA;
         at += k;
     }
+    return DF11_OK;
+}
+
+df11_status df11_gemm_tile_weights(const uint16_t *host_w, uint64_t k, uint64_t n, uint16_t *host_tiled) {
+    if (!host_w || !host_tiled || k == 0 || n == 0 || k % DF11_GEMM_TILE_K || n % DF11_GEMM_TILE_N) return DF11_EINVAL;
+    if (k > (uint64_t{1} << 40) / n) return DF11_EINVAL;
+    const uint8_t *a = reinterpret_cast<const uint8_t *>(host_w), *b = reinterpret_cast<const uint8_t *>(host_tiled);
+    if (a < b + 2 * k * n && b < a + 2 * k * n) return DF11_EINVAL;  // the buffers overlap
+    df11::gemm_tile_weights(host_w, k, n, host_tiled, 0);
+    return DF11_OK;
+}
+
+df11_status df11_decode_gemm(const df11_gemm_matrix *mats, int n_mats, int m, int *dev_err_flag,
+                             df11_stream stream) {
+    df11::GemmJob jobs[df11::kGemmMaxMats];
+    const df11_status st = gemm_jobs(mats, n_mats, false, jobs);
+    if (st != DF11_OK) return st;
+    return from_launch(df11::launch_decode_gemm(jobs, n_mats, m, dev_err_flag, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+df11_status df11_decode_gemm_launch_shape(const df11_gemm_matrix *mats, int n_mats, int m, int *grid, int *block,
+                                          int *smem_bytes) {
+    df11::GemmJob jobs[df11::kGemmMaxMats];
+    const df11_status st = gemm_jobs(mats, n_mats, true, jobs);
+    if (st != DF11_OK) return st;
+    df11::GemmShape sh;
+    const df11::LaunchStatus ls = df11::gemm_launch_shape(jobs, n_mats, m, &sh);
+    if (ls != df11::LaunchStatus::kOk) return from_launch(ls);
+    if (grid) *grid = sh.grid;
+    if (block) *block = sh.block;
+    if (smem_bytes) *smem_bytes = sh.smem;
     return DF11_OK;
 }
 

@@ -37,87 +37,10 @@
 
 #include "df11.h"
 #include "launch.h"
+#include "walk.cuh"
 
 namespace df11 {
 namespace {
-
-// ------------------------------------------------------------------ PTX helpers
-
-__device__ __forceinline__ uint32_t smem_addr(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void fence_mbar_init() {
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t tx) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(tx)
-                 : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ uint64_t global_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Waits for the phase of `parity` to complete; false after limit_ns (the
-// launch's DecodeParams::wait_ns: 2 s, or 10 ms when its waits are made to
-// run out on purpose).
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (global_ns() - t0 > limit_ns) return false;
-    }
-    return true;
-}
-
-// 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
-// Both addresses 16-byte aligned, bytes a positive multiple of 16.
-__device__ __forceinline__ void bulk_load(void *smem_dst, const void *gmem_src, uint32_t bytes, uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_addr(smem_dst)),
-        "l"(gmem_src), "r"(bytes), "r"(smem_addr(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ void consumer_sync(int nthreads) {
-    asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
-}
-
-// Lets a kernel launched after this one with programmatic stream
-// serialization start as soon as SMs free up (no effect otherwise).  Decode
-// launches never consume a previous decode's output, so they trigger at once.
-__device__ __forceinline__ void allow_dependent_launch() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
-__device__ __forceinline__ void report(int *err, uint32_t bits) {
-    if (err && bits) atomicOr(err, static_cast<int>(bits));
-}
 
 // ------------------------------------------------------------------ shared memory plan
 
@@ -162,228 +85,6 @@ __host__ __device__ inline Plan make_plan(int chunk_bits, int chunks, uint32_t m
     p.off_exps = p.off_gaps + kStreamStages * up128(p.gaps_bytes);
     p.total = p.off_exps + p.exps_bytes;
     return p;
-}
-
-// ------------------------------------------------------------------ decoding a chunk
-
-struct Tables {
-    const uint32_t *meta;   // shared
-    const uint32_t *syms;   // shared
-    const uint16_t *lut_s;  // shared: hierarchical tables [0, n_lut_smem)
-    const uint16_t *lut_g;  // global: all hierarchical tables
-    int n_lut_smem;
-    int n_luts;
-};
-
-// One code through the hierarchical 256-entry tables; `win` holds the next 32
-// stream bits, most significant first.  Returns symbol | length << 8.  A bit
-// pattern that is no codeword (possible only for a one-symbol code or a
-// damaged stream), a pointer past the last table or a zero length (damaged
-// tables) is flagged and consumed as one 1-bit code, so every step advances.
-__device__ __forceinline__ uint32_t lut_decode(uint32_t win, const Tables &T, uint32_t &err) {
-    uint32_t e = T.lut_s[win >> 24];
-#pragma unroll 1
-    for (int lvl = 1; (e & kLutPointer) && lvl < 4; ++lvl) {
-        const int tbl = static_cast<int>(e & 0x7FFFu);
-        if (tbl >= T.n_luts) break;
-        const uint32_t ix = static_cast<uint32_t>(tbl) * kLutEntries + ((win >> (24 - 8 * lvl)) & 0xFFu);
-        e = tbl < T.n_lut_smem ? T.lut_s[ix] : __ldg(T.lut_g + ix);
-    }
-    if ((e & (kLutPointer | 0x4000u)) || !(e & 0x3F00u)) {
-        err |= DF11_DEV_ERR_CODE;
-        e = 1u << 8;
-    }
-    return e;
-}
-
-// A multi-symbol entry is used only when it consumes 1..12 bits, yields 1..4
-// symbols and its start mask has one bit per symbol starting at offset 0;
-// anything else (a damaged table) becomes the long-code sentinel, whose codes
-// the hierarchical tables then decode one at a time.
-__device__ __forceinline__ uint32_t sane_meta(uint32_t e) {
-    const uint32_t used = e & 0x7FFu, n = (e >> kMetaCountShift) & 0x1FFu, mask = e >> kMetaMaskShift;
-    const bool ok = used >= 1 && used <= kMultiBits && n >= 1 && n <= kMultiMaxSyms && (mask & 1u) &&
-                    static_cast<uint32_t>(__popc(mask)) == n && mask < (1u << used);
-    return ok ? e : kMetaLong;
-}
-
-// Multi-symbol table reads: shared-memory copies were checked when staged;
-// GM = true reads the image in global memory and checks each entry.
-template <bool GM>
-__device__ __forceinline__ uint32_t meta_at(const Tables &T, uint32_t idx) {
-    if constexpr (GM) return sane_meta(__ldg(T.meta + idx));
-    else return T.meta[idx];
-}
-
-template <bool GM>
-__device__ __forceinline__ uint32_t syms_at(const Tables &T, uint32_t idx) {
-    if constexpr (GM) return __ldg(T.syms + idx);
-    else return T.syms[idx];
-}
-
-// Number of an entry's codes that start before bit `room` of its window.
-__device__ __forceinline__ uint32_t starts_before(uint32_t mm, int room) {
-    return static_cast<uint32_t>(__popc((mm >> kMetaMaskShift) & ((1u << room) - 1u)));
-}
-
-// Field masks of a walker's accumulator acc = p | count << kMetaCountShift.
-constexpr uint32_t kPosMask = (1u << kMetaCountShift) - 1u;
-constexpr uint32_t kCountOne = 1u << kMetaCountShift;
-
-// Phase 1 (CTA-tile kernel): count the codes that start in each of this
-// thread's CPT chunks, with the chunk in registers.  Chunk c occupies
-// w[c*CW .. c*CW+CW-1] (earliest bit first) and w[c*CW+CW] is its look-ahead
-// word (the next chunk's first word).  Its walk starts at bit gap[c] and
-// counts codes that start before bit E[c].  The walk moves through the chunk
-// 32 bits at a time ("stage" k reads the word pair w[k], w[k+1]).  While a
-// whole 12-bit window lies before E, one lookup in the multi-symbol table
-// consumes up to 4 codes; in the last 11 bits before E the entry's start mask
-// counts only the codes that start before E; codes longer than 12 bits (the
-// sentinel entry) go through the hierarchical tables.  acc = p | count << 11
-// and an entry is consumed | count << 11 | mask << 20, so one add advances
-// both (the mask lands above the count field); the sentinel adds 1024 to p,
-// which ends the loop.  The CPT chunks advance in lockstep.
-template <int CW, int CPT, bool GM = false>
-__device__ __forceinline__ void count_codes(const uint32_t (&w)[CPT * CW + 1], const int (&gap)[CPT],
-                                            const int (&E)[CPT], const Tables &T, uint32_t (&cnt)[CPT],
-                                            uint32_t &err) {
-    uint32_t acc[CPT];
-#pragma unroll
-    for (int c = 0; c < CPT; ++c) acc[c] = static_cast<uint32_t>(gap[c]);
-#pragma unroll
-    for (int k = 0; k < CW; ++k) {
-        int lm[CPT], ls[CPT], er[CPT];
-#pragma unroll
-        for (int c = 0; c < CPT; ++c) {
-            er[c] = E[c] - 32 * k;
-            lm[c] = min(32, er[c] - (kMultiBits - 1));
-            ls[c] = min(32, er[c]);
-        }
-        for (;;) {
-            for (;;) {
-                bool act[CPT], any = false;
-#pragma unroll
-                for (int c = 0; c < CPT; ++c) {
-                    act[c] = static_cast<int>(acc[c] & kPosMask) < lm[c];
-                    any |= act[c];
-                }
-                if (!any) break;
-#pragma unroll
-                for (int c = 0; c < CPT; ++c) {
-                    if (act[c]) {
-                        const uint32_t win = __funnelshift_l(w[c * CW + k + 1], w[c * CW + k], acc[c]);
-                        acc[c] += meta_at<GM>(T, win >> (32 - kMultiBits));
-                    }
-                }
-            }
-            bool more = false;
-#pragma unroll
-            for (int c = 0; c < CPT; ++c) {
-                int p = static_cast<int>(acc[c] & kPosMask);
-                bool single = false;
-                if (p >= static_cast<int>(kMetaLong)) {  // sentinel: the first code is longer than 12 bits
-                    acc[c] -= kMetaLong;
-                    p -= kMetaLong;
-                    single = true;
-                } else if (p >= ls[c]) {
-                    continue;
-                }
-                const uint32_t win = __funnelshift_l(w[c * CW + k + 1], w[c * CW + k], p);
-                const uint32_t mm = single ? kMetaLong : meta_at<GM>(T, win >> (32 - kMultiBits));
-                if (mm & kMetaLong) {
-                    const uint32_t e = lut_decode(win, T, err);
-                    acc[c] += ((e >> 8) & 0x3Fu) + kCountOne;
-                } else {  // last bits before E: count only the codes that start before it
-                    acc[c] += (mm & 0xFu) + (starts_before(mm, er[c] - p) << kMetaCountShift);
-                }
-                more = true;
-            }
-            if (!more) break;
-        }
-#pragma unroll
-        for (int c = 0; c < CPT; ++c) acc[c] -= min(acc[c] & kPosMask, 32u);
-    }
-#pragma unroll
-    for (int c = 0; c < CPT; ++c) cnt[c] = (acc[c] >> kMetaCountShift) & 0x1FFu;
-}
-
-// ORs up to 4 symbol bytes `sy` (unused high bytes zero) into shared memory at
-// byte address out: the one or two 32-bit words they touch.  The exponent
-// buffer is zero before phase 2, so neighbouring chunks can OR into a word
-// they share and the zero high bytes leave other symbols intact.
-__device__ __forceinline__ void put_symbols(uint32_t sy, uint32_t out) {
-    const uint32_t a = out & ~3u, sh = (out & 3u) << 3;
-    asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(a), "r"(sy << sh) : "memory");
-    if (sh) asm volatile("red.shared.or.b32 [%0+4], %1;" ::"r"(a), "r"(__funnelshift_l(sy, 0u, sh)) : "memory");
-}
-
-// Phase 2 (CTA-tile kernel): decode chunk C again along the same path as
-// phase 1 and write its symbols from shared-memory byte address q on.
-template <int CW, int CPT, int C, bool GM = false>
-__device__ __forceinline__ void emit_codes(const uint32_t (&w)[CPT * CW + 1], int p, const int E, const Tables &T,
-                                           uint32_t q, uint32_t &err) {
-    uint32_t out = q;
-#pragma unroll
-    for (int k = 0; k < CW; ++k) {
-        const int er = E - 32 * k;
-        const int lm = min(32, er - (kMultiBits - 1));
-        const int ls = min(32, er);
-        const uint32_t hi = w[C * CW + k], lw = w[C * CW + k + 1];
-        for (;;) {
-            while (p < lm) {
-                const uint32_t win = __funnelshift_l(lw, hi, p);
-                const uint32_t idx = win >> (32 - kMultiBits);
-                const uint32_t mm = meta_at<GM>(T, idx);
-                p += static_cast<int>(mm & kPosMask);
-                put_symbols(syms_at<GM>(T, idx), out);
-                out += (mm >> kMetaCountShift) & 7u;
-            }
-            bool single = false;
-            if (p >= static_cast<int>(kMetaLong)) {
-                p -= kMetaLong;
-                single = true;
-            } else if (p >= ls) {
-                break;
-            }
-            const uint32_t win = __funnelshift_l(lw, hi, p);
-            const uint32_t idx = win >> (32 - kMultiBits);
-            const uint32_t mm = single ? kMetaLong : meta_at<GM>(T, idx);
-            if (mm & kMetaLong) {
-                const uint32_t e = lut_decode(win, T, err);
-                p += static_cast<int>((e >> 8) & 0x3Fu);
-                put_symbols(e & 0xFFu, out);
-                out += 1;
-            } else {
-                const uint32_t nv = starts_before(mm, er - p);
-                const uint32_t nb = 8u * nv;
-                const uint32_t sy = nb >= 32 ? syms_at<GM>(T, idx) : (syms_at<GM>(T, idx) & ((1u << nb) - 1u));
-                p += static_cast<int>(mm & 0xFu);
-                if (nv) put_symbols(sy, out);
-                out += nv;
-            }
-        }
-        p -= min(p, 32);
-    }
-}
-
-// ------------------------------------------------------------------ field merges
-
-// 4 plane bytes + 4 exponents -> 4 BF16 words (two 32-bit outputs).
-__device__ __forceinline__ void merge_bf16x4(uint32_t P, uint32_t X, uint32_t &o0, uint32_t &o1) {
-    const uint32_t hi = (P & 0x80808080u) | ((X >> 1) & 0x7F7F7F7Fu);  // sign | exponent[7:1]
-    const uint32_t lo = ((X << 7) & 0x80808080u) | (P & 0x7F7F7F7Fu);  // exponent[0] | mantissa
-    o0 = __byte_perm(lo, hi, 0x5140);
-    o1 = __byte_perm(lo, hi, 0x7362);
-}
-
-// 4 plane bytes (8 nibbles) + 8 exponents -> 8 E4M3 bytes.
-__device__ __forceinline__ void merge_e4m3x8(uint32_t P, uint32_t X0, uint32_t X1, uint32_t &o0, uint32_t &o1) {
-    const uint32_t nl = P & 0x0F0F0F0Fu;         // elements 0, 2, 4, 6
-    const uint32_t nh = (P >> 4) & 0x0F0F0F0Fu;  // elements 1, 3, 5, 7
-    const uint32_t n0 = __byte_perm(nl, nh, 0x5140);
-    const uint32_t n1 = __byte_perm(nl, nh, 0x7362);
-    o0 = ((n0 & 0x08080808u) << 4) | ((X0 << 3) & 0x78787878u) | (n0 & 0x07070707u);
-    o1 = ((n1 & 0x08080808u) << 4) | ((X1 << 3) & 0x78787878u) | (n1 & 0x07070707u);
 }
 
 __device__ __forceinline__ void st_global_v4(void *p, uint4 v) {
@@ -520,21 +221,8 @@ __device__ __forceinline__ void edge_groups(const uint4 (&pre)[kPrefetchGroups],
 // plane bytes [8j, 8j + 8) and 8 (BF16) or 16 (E4M3) exponents.  Lane L of
 // store round r takes half 32r + L, so each 16-byte store instruction of the
 // warp writes 512 contiguous bytes.
-__device__ __forceinline__ uint2 ld_global_stream_v2(const void *p) {
-    uint2 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
-    return v;
-}
-
-// The same load and the 16-byte store at a constant offset OFF from p (the
-// offset is part of the instruction: one address register serves every round).
-template <int OFF>
-__device__ __forceinline__ uint2 ld_global_stream_v2_at(const void *p) {
-    uint2 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2+%3];" : "=r"(v.x), "=r"(v.y) : "l"(p), "n"(OFF));
-    return v;
-}
-
+// The 16-byte store at a constant offset OFF from p (the offset is part of
+// the instruction: one address register serves every round).
 template <int OFF>
 __device__ __forceinline__ void st_global_v4_at(void *p, uint4 v) {
     asm volatile("st.global.v4.u32 [%0+%1], {%2, %3, %4, %5};" ::"l"(p), "n"(OFF), "r"(v.x), "r"(v.y), "r"(v.z),
@@ -611,11 +299,6 @@ __device__ __forceinline__ void merge_rounds(const uint2 *pre, uint32_t lane, ui
     ((lane + 32u * (U + 1) < nh ? merge_half_round<DT, U + 1>(pre[U + 1], x_l, out_l) : (void)0), ...);
 }
 
-template <int... U>
-__device__ __forceinline__ void prefetch_halves(uint2 *pre, const uint8_t *pl, uint32_t lane, uint32_t nhalf,
-                                                std::integer_sequence<int, U...>) {
-    ((lane + 32u * U < nhalf ? (void)(pre[U] = ld_global_stream_v2_at<256 * U>(pl)) : (void)0), ...);
-}
 
 // ------------------------------------------------------------------ kernel
 
@@ -881,10 +564,6 @@ __host__ __device__ inline WarpPlan make_warp_plan(int chunk_bits, int nwarp, ui
     return p;
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // Descriptor index of tile t (tiles of all tensors are numbered consecutively),
 // searching forward from `from`: a warp's tiles only increase.
 __device__ __forceinline__ int tensor_of(const DecodeParams &P, uint32_t t, int from = 0) {
@@ -1080,144 +759,6 @@ __global__ void __launch_bounds__(NWARP * 32, NWARP <= 8 ? 4 : 2)
             if (!mbar_wait(&full[s], (par >> s) & 1u, P.wait_ns)) err |= DF11_DEV_ERR_TIMEOUT;
     err = __reduce_or_sync(0xFFFFFFFFu, err);
     if (lane == 0) report(P.err, err);
-}
-
-// ------------------------------------------------------------------ byte-step kernel
-
-// Steps of the byte-step walk taken unconditionally by a chunk: its range is
-// CB + (next gap) - (gap) bits, at least CB - 31 (a gap is below 32), so every
-// chunk with a whole range takes its first (CB - 32) / 8 steps without
-// per-step checks.
-template <int CB>
-constexpr int kFixedSteps = (CB - 32) / 8;
-
-// Row base + byte k of x times the entry size, as a byte permute and a
-// multiply-add (the multiply-add issues on the FMA pipe).
-template <uint32_t ENTRY>
-__device__ __forceinline__ uint32_t step_addr(uint32_t x, int k, uint32_t base) {
-    const uint32_t b = __byte_perm(x, 0u, 0x4440u + static_cast<uint32_t>(3 - k));
-    uint32_t a;
-    asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(a) : "r"(b), "n"(ENTRY), "r"(base));
-    return a;
-}
-
-// Row field of the compact control words (row << 10: rows of 1 KB).
-constexpr uint32_t kCtlRowMask = kFsmRowMask >> 1;
-
-// The byte-step walk of one chunk.  The thread's codes occupy bits [g, g +
-// 8 * nfull + r) of the words w[0..CW] followed by w2 (earliest bit first):
-// from the first code start in the chunk to the first code start in the next
-// chunk (or the end of the stream).  Step j looks up byte j of that range in
-// the row of the tree node the previous step stopped on (the root first): the
-// entry lists the codes that end in the byte and the next row.  Steps below
-// NFIX are taken by every thread on the byte-step walk (kFixedSteps); the
-// others are predicated on nfull, and the warp stops after its longest range
-// (jmax steps).  A last partial byte (r bits) counts only
-// the codes whose end mask bit falls in its first r bits; those end exactly
-// at the range's end, so the codes of the next chunk are never counted.
-//
-// Phase 1 (byte_step_count) walks the compact control words (4 bytes per
-// entry, so a warp's random lookups spread over all 32 banks: end mask in
-// bits 0..7, row << 10, codes ended << 24, so adding whole words counts the
-// codes while the lower fields of at most 20 steps stay below bit 24) and
-// returns the number of codes; ctl_out receives the last control word, whose row is the
-// dead row (`dead`, in control-word form) when the walk left the tables or the
-// partial byte ends more than the 4 codes an entry holds (possible only with
-// a 1-bit codeword).
-template <int CB>
-__device__ __forceinline__ uint32_t byte_step_count(const uint32_t (&w)[CB / 32 + 1], uint32_t w2, int g, int nfull,
-                                                    int r, int jmax, const uint8_t *ctl_tab, uint32_t dead,
-                                                    uint32_t &ctl_out) {
-    constexpr int CW = CB / 32, NFIX = kFixedSteps<CB>;
-    uint32_t ctl = 0, cnt = 0;
-#pragma unroll
-    for (int m = 0; m <= CW; ++m) {
-        if (4 * m >= NFIX && 4 * m >= jmax) break;  // warp-uniform
-        const uint32_t x = __funnelshift_l(m < CW ? w[m + 1] : w2, w[m], static_cast<uint32_t>(g));
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int j = 4 * m + k;
-            if (j >= NFIX && j >= jmax) break;
-            const uint32_t e = *reinterpret_cast<const uint32_t *>(ctl_tab + step_addr<4>(x, k, ctl & kCtlRowMask));
-            if (j < NFIX || j < nfull) {
-                ctl = e;
-                cnt += e;  // the count field at bit 24 gathers the codes; the fields below it never carry into it
-            } else if (j == nfull) {
-                const uint32_t c = static_cast<uint32_t>(__popc(e & ((1u << r) - 1u)));
-                cnt += c << 24;
-                if (c > 4) ctl = dead;
-            }
-        }
-    }
-    ctl_out = ctl;
-    return cnt >> 24;
-}
-
-// Puts symbol bytes sy (c8 / 8 of them, unused bytes zero) after the f8 / 8
-// pending bytes of acc; a completed word goes to byte address wp.
-__device__ __forceinline__ void emit_word(uint32_t sy, uint32_t c8, uint32_t &acc, uint32_t &wp, uint32_t &f8) {
-    const uint32_t lo = acc | (sy << f8);
-    const uint32_t hi = __funnelshift_l(sy, 0u, f8);  // bytes pushed past the word
-    f8 += c8;
-    if (f8 >= 32u) {
-        asm volatile("st.shared.u32 [%0], %1;" ::"r"(wp), "r"(lo) : "memory");
-        wp += 4u;
-        f8 -= 32u;
-        acc = hi;
-    } else {
-        acc = lo;
-    }
-}
-
-// Phase 2: the same walk on the full entries {ctl, syms}, writing the symbols
-// in order from shared-memory byte address `out` on.  Symbols are assembled
-// in a register (acc holds f8 / 8 pending bytes, starting from acc0, the
-// current content of the word `out` falls in; unused bytes zero) and every
-// completed 32-bit word is stored with one plain store.  The word the range
-// starts in may hold earlier threads' bytes (stored as zeros here) and the
-// word it ends in later threads' bytes: that last, partial word is returned
-// in acc / wp / f8 and OR-ed in by the caller after a __syncwarp, so it
-// lands after every plain store of the warp and no store clears another
-// thread's bytes.  The buffer is zero outside the words written.  The
-// steps after the whole bytes only keep the entry of the last, partial byte
-// (j == nfull), whose codes are emitted once after the loop.  ctl_out
-// receives the last control word, whose row is the dead row (`dead`) when
-// the walk left the tables or the partial byte ends more than 4 codes.
-template <int CB>
-__device__ __forceinline__ void byte_step_emit(const uint32_t (&w)[CB / 32 + 1], uint32_t w2, int g, int nfull,
-                                               int r, int jmax, const uint8_t *tab, uint32_t out, uint32_t acc0,
-                                               uint32_t dead, uint32_t &acc, uint32_t &wp, uint32_t &f8,
-                                               uint32_t &ctl_out) {
-    constexpr int CW = CB / 32, NFIX = kFixedSteps<CB>;
-    uint32_t ctl = 0;
-    acc = acc0;
-    wp = out & ~3u;
-    f8 = (out & 3u) << 3;
-    uint2 ep = make_uint2(0u, 0u);
-#pragma unroll
-    for (int m = 0; m <= CW; ++m) {
-        if (4 * m >= NFIX && 4 * m >= jmax) break;  // warp-uniform
-        const uint32_t x = __funnelshift_l(m < CW ? w[m + 1] : w2, w[m], static_cast<uint32_t>(g));
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int j = 4 * m + k;
-            if (j >= NFIX && j >= jmax) break;
-            const uint2 e = *reinterpret_cast<const uint2 *>(tab + step_addr<8>(x, k, ctl & kFsmRowMask));
-            if (j < NFIX || j < nfull) {
-                ctl = e.x;
-                emit_word(e.y, e.x >> (kFsmCountShift - 3), acc, wp, f8);
-            } else if (j == nfull) {
-                ep = e;  // the partial byte: emitted once after the loop
-            }
-        }
-    }
-    if (r) {
-        const uint32_t ce = static_cast<uint32_t>(__popc(ep.x & ((1u << r) - 1u)));
-        const uint32_t c = min(ce, 4u);
-        emit_word(c ? ep.y & (0xFFFFFFFFu >> (32u - 8u * c)) : 0u, 8u * c, acc, wp, f8);
-        if (ce > 4) ctl = dead;
-    }
-    ctl_out = ctl;
 }
 
 // Shared memory of the byte-step kernel: the transition table (fsm_rows rows

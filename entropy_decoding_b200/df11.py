@@ -69,6 +69,13 @@ class DecodeOpts(ctypes.Structure):
                 ("overlap", ctypes.c_int32), ("diag_expire_waits", ctypes.c_int32), ("count_walk", ctypes.c_int32)]
 
 
+class GemmMatrix(ctypes.Structure):
+    _fields_ = [("weights", ctypes.c_void_p), ("k", ctypes.c_uint64), ("n", ctypes.c_uint64), ("x", ctypes.c_void_p),
+                ("y", ctypes.c_void_p)]
+
+
+GEMM_TILE_N, GEMM_TILE_K, GEMM_MAX_MATS, GEMM_MAX_BATCH = 128, 16, 8, 64
+
 WALKER_AUTO, WALKER_WINDOW, WALKER_BYTE_STEP = 0, 1, 2
 ENCODE_NO_CHUNK_COUNTS = 1  # encoder flag: leave out the chunk-counts section
 
@@ -115,6 +122,10 @@ _SIGS = {
     "df11_encode_device_noalloc": ([_P, _P, _U64, _I, _I, _I, _P, _U64, _P, ctypes.POINTER(EncodeResult)], _S),
     "df11_decode_host": ([_PP, _PP, _PP, _PP, _PP, _I, _P, _P], _S),
     "df11_decode_launch_shape": ([_PP, _I, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I)], _S),
+    "df11_gemm_tile_weights": ([_P, _U64, _U64, _P], _S),
+    "df11_decode_gemm": ([ctypes.POINTER(GemmMatrix), _I, _I, _P, _P], _S),
+    "df11_decode_gemm_launch_shape": ([ctypes.POINTER(GemmMatrix), _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I),
+                                       ctypes.POINTER(_I)], _S),
     "df11_rans_encode_group": ([_I, _PP, ctypes.POINTER(_U64), _I, _I, _I, _PP], _S),
     "df11_rans_group_free": ([_P], None),
     "df11_rans_group_freqs": ([_P, _P], _S),
@@ -428,6 +439,38 @@ def df11_encode_device_noalloc(cb: Codebook, src_ptr: int, n: int, chunk_bits: i
         e.result = r
         raise e
     return r
+
+
+# ----------------------------------------------------------------- decode fused into the consuming GEMM
+
+def df11_gemm_tile_weights(w: np.ndarray, k: int, n: int) -> np.ndarray:
+    """The operand-tile order of a K x N BF16 matrix (uint16 bits, row-major)."""
+    w = np.ascontiguousarray(w, dtype=np.uint16).reshape(-1)
+    if w.size != k * n:
+        raise ValueError("w must hold k * n weights")
+    out = np.empty(k * n, np.uint16)
+    _check(_lib.df11_gemm_tile_weights(w.ctypes.data, k, n, out.ctypes.data), "df11_gemm_tile_weights")
+    return out
+
+
+def _gemm_array(mats):
+    arr = (GemmMatrix * len(mats))()
+    for i, (blob, k, n, x_ptr, y_ptr) in enumerate(mats):
+        arr[i] = GemmMatrix(blob.handle.value, k, n, x_ptr or None, y_ptr or None)
+    return arr
+
+
+def df11_decode_gemm(mats, m: int, err_ptr: int | None = None, stream: int = 0):
+    """mats: (blob, K, N, x device pointer, y device pointer) per matrix; y += x W."""
+    _check(_lib.df11_decode_gemm(_gemm_array(mats), len(mats), m, err_ptr or None, stream or None), "df11_decode_gemm")
+
+
+def df11_decode_gemm_launch_shape(mats, m: int):
+    """(grid, threads per CTA, dynamic shared memory bytes); pointers may be 0."""
+    g, b, s = _I(), _I(), _I()
+    _check(_lib.df11_decode_gemm_launch_shape(_gemm_array(mats), len(mats), m, ctypes.byref(g), ctypes.byref(b),
+                                              ctypes.byref(s)), "df11_decode_gemm_launch_shape")
+    return g.value, b.value, s.value
 
 
 # ----------------------------------------------------------------- torch-side helpers (device memory only)

@@ -469,6 +469,62 @@ df11_status df11_encode_device_noalloc(const df11_codebook *cb, const void *src_
                                        df11_encode_result *result);
 
 /* ---------------------------------------------------------------------
+ * Decode fused into the consuming GEMM  ("Compressing LLMs without
+ * Compromise" summary page, ZipServ paragraph: decompression fused into the
+ * matrix multiply so the decoded weights go straight to the tensor cores;
+ * "Approaching Shannon Bound with Lossless LLM Weight Compression",
+ * Abstract: decoding aligned with the GEMM's tiling)
+ * ------------------------------------------------------------------ */
+
+/* Operand tile of the fused GEMM: 128 output rows x 16 reduction columns. */
+#define DF11_GEMM_TILE_N 128
+#define DF11_GEMM_TILE_K 16
+#define DF11_GEMM_MAX_MATS 8   /* matrices per df11_decode_gemm launch */
+#define DF11_GEMM_MAX_BATCH 64 /* rows of x */
+
+/* Writes the operand-tile order of a K x N BF16 weight matrix (host_w,
+ * row-major: element (k, n) at k * N + n, the layer mapping K inputs to N
+ * outputs) into host_tiled (K * N words, caller's buffer, not overlapping
+ * host_w): tile t = nb * (K / 16) + kb holds outputs n = 128 nb ..
+ * 128 nb + 127 and inputs k = 16 kb .. 16 kb + 15, element (r, c) at
+ * 2048 t + 16 r + c, i.e. host_w[(16 kb + c) * N + 128 nb + r].  Encoding the
+ * result with df11_encode gives the blob df11_decode_gemm consumes; decoding
+ * it with df11_decode gives back the tiled order.  K % 16 == 0 and
+ * N % 128 == 0, else DF11_EINVAL. */
+df11_status df11_gemm_tile_weights(const uint16_t *host_w, uint64_t k, uint64_t n, uint16_t *host_tiled);
+
+typedef struct {
+    const df11_blob *weights; /* bound blob of the tiled K x N matrix: BF16, the default layout
+                                 (128-bit chunks, 32-chunk tiles, chunk counts), host sections present */
+    uint64_t k, n;            /* K inputs (multiple of 16), N outputs (multiple of 128) */
+    const void *x;            /* device, M x K BF16 row-major, 16-byte aligned, rows K * 2 bytes apart */
+    float *y;                 /* device, M x N FP32 row-major, 4-byte aligned: y += x W */
+} df11_gemm_matrix;
+
+/* y_i += x_i W_i for every matrix of the launch, in ONE kernel launch on
+ * `stream`, asynchronously: the weights are decoded tile by tile into shared
+ * memory and multiplied there by the tensor cores (FP32 accumulation); the
+ * decoded weights never reach HBM.  y is accumulated with floating-point
+ * adds (the reduction over K is split between CTAs), so the caller zeroes y
+ * for a plain product, and the rounding order of y varies from run to run
+ * (every y element is within K * 2^-24 * sum_k |x_mk w_kn| of the exact
+ * product plus what y held).  The matrices share one code (one codebook),
+ * as in df11_decode.  M = m in 1..DF11_GEMM_MAX_BATCH; n_mats in
+ * 1..DF11_GEMM_MAX_MATS.  dev_err_flag as in df11_decode (its bits mean the
+ * y of that launch is not valid).  Never allocates, never synchronises.
+ * Errors: DF11_EINVAL (arguments, shapes, alignment, an unbound or
+ * GPU-encoded blob without host sections, mixed codes), DF11_EUNSUPPORTED
+ * (another dtype or layout, a code with a 1-bit codeword, tables too large
+ * for shared memory), DF11_ECUDA. */
+df11_status df11_decode_gemm(const df11_gemm_matrix *mats, int n_mats, int m, int *dev_err_flag,
+                             df11_stream stream);
+
+/* Grid, threads per CTA and dynamic shared memory of that launch on the
+ * current device (any output may be NULL); x and y are not read. */
+df11_status df11_decode_gemm_launch_shape(const df11_gemm_matrix *mats, int n_mats, int m, int *grid, int *block,
+                                          int *smem_bytes);
+
+/* ---------------------------------------------------------------------
  * rANS variant of the exponent coder
  * ------------------------------------------------------------------ */
 

@@ -19,7 +19,7 @@ def df11():
 
 
 STRUCTS = {"df11_blob_info": "BlobInfo", "df11_decode_opts": "DecodeOpts", "df11_encode_result": "EncodeResult",
-           "df11_rans_tensor_info": "RansTensorInfo"}
+           "df11_rans_tensor_info": "RansTensorInfo", "df11_gemm_matrix": "GemmMatrix"}
 CONSTANTS = {
     "DF11_OK": "DF11_OK", "DF11_EINVAL": "DF11_EINVAL", "DF11_ENOMEM": "DF11_ENOMEM", "DF11_ECUDA": "DF11_ECUDA",
     "DF11_ECORRUPT": "DF11_ECORRUPT", "DF11_EUNSUPPORTED": "DF11_EUNSUPPORTED",
@@ -31,6 +31,8 @@ CONSTANTS = {
     "DF11_ENCODE_NO_CHUNK_COUNTS": "ENCODE_NO_CHUNK_COUNTS",
     "DF11_NOALLOC_SCRATCH_BYTES": "NOALLOC_SCRATCH_BYTES", "DF11_NOALLOC_MAX_ELEMS": "NOALLOC_MAX_ELEMS",
     "DF11_RANS_TILE_DEFAULT": "RANS_TILE_DEFAULT",
+    "DF11_GEMM_TILE_N": "GEMM_TILE_N", "DF11_GEMM_TILE_K": "GEMM_TILE_K", "DF11_GEMM_MAX_MATS": "GEMM_MAX_MATS",
+    "DF11_GEMM_MAX_BATCH": "GEMM_MAX_BATCH",
 }
 
 

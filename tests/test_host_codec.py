@@ -421,3 +421,12 @@ def test_device_image_layout(df11):
     assert not words[s["stream"].size:].any()
     assert np.array_equal(img[lay["plane"]:lay["plane"] + info.plane_bytes], s["plane"])
     assert lay["total"] - lay["plane"] >= info.plane_bytes + 32
+
+
+@pytest.mark.parametrize("k,n", [(16, 128), (48, 384), (4096, 1024)])
+def test_gemm_tile_order_matches_oracle(df11, oracle_mod, k, n):
+    """The library's operand-tile permutation (host) against the oracle's."""
+    w = np.random.default_rng(k * n).integers(0, 1 << 16, k * n, dtype=np.uint16)
+    assert np.array_equal(df11.df11_gemm_tile_weights(w, k, n), oracle_mod.gemm_tile(w, k, n))
+    with pytest.raises(df11.Df11Error):
+        df11.df11_gemm_tile_weights(w[: (k - 1) * n], k - 1, n)
