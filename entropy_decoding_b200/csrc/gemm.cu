@@ -18,21 +18,21 @@
 // operand tiles by a shift, and nothing else of the container changes.
 //
 // One CTA per SM owns a contiguous range of operand tiles ("k-tiles"):
-//   * warps 0..27 decode the container's warp tiles that cover the range,
+//   * warps 0..23 decode the container's warp tiles that cover the range,
 //     round robin, with the byte-step walk (phase 2 into the warp's own
 //     exponent buffer, as in the decode kernel), and merge them with the raw
 //     sign+mantissa plane (prefetched into registers at tile start) straight
-//     into BF16 operand tiles in the 32-byte-swizzled K-major layout that
-//     tcgen05.mma reads (a ring of 4-KB slots: small slots keep many k-tiles
-//     in flight); a counter per operand slot hands a completed k-tile (2048
-//     weights placed) to the MMA warp;
-//   * warp 28 (lane 0) issues the copies of the activation tiles
-//     (cp.async.bulk.tensor with a 32-byte swizzle, no multicast; rows past
-//     M read as zeros) and the MMA of each k-tile (M = 128 output rows, N =
-//     M padded to 16, K = 16) into a TMEM accumulator, and
+//     into BF16 operand tiles in the swizzled K-major layout that
+//     tcgen05.mma reads (a ring of operand slots, rows of kGemmTileK weights,
+//     the swizzle as wide as a row); a counter per operand slot hands a
+//     completed k-tile (128 x kGemmTileK weights placed) to the MMA warp;
+//   * warp 24 (lane 0) issues the copies of the activation tiles
+//     (cp.async.bulk.tensor with the same swizzle, no multicast; rows past
+//     M read as zeros) and the MMAs of each k-tile (M = 128 output rows, N =
+//     M padded to 16, K = 16 each) into a TMEM accumulator, and
 //     frees each k-tile's slot once its MMAs completed (checked without
 //     blocking, so several k-tiles' MMAs are in flight);
-//   * warps 28..31 drain the accumulator (tcgen05.ld) into y with
+//   * warps 24..27 drain the accumulator (tcgen05.ld) into y with
 //     floating-point adds whenever the range leaves a block of 128 output
 //     rows: y's rows are split over CTAs along K, so y accumulates.
 // Every wait is bounded (%globaltimer); a timeout sets DF11_DEV_ERR_TIMEOUT
@@ -55,12 +55,17 @@
 namespace df11 {
 namespace {
 
-constexpr int kDecodeWarps = 28;  // warps 0..27 decode; 28..31 copy, multiply and drain
+constexpr int kDecodeWarps = 24;  // warps 0..23 decode; 24..27 copy, multiply and drain
 constexpr int kMmaWarp = kDecodeWarps;  // a multiple of 4: warps kMmaWarp + q reach TMEM lanes 32 q .. 32 q + 31
 constexpr int kGemmThreads = 32 * (kDecodeWarps + 4);
-constexpr uint32_t kKTile = kGemmTileN * kGemmTileK;  // 2048 weights
-constexpr int kKTileShift = 11;
-constexpr uint32_t kATileBytes = 2 * kKTile;  // BF16 operand tile: 128 rows of 32 bytes
+constexpr uint32_t kKTile = kGemmTileN * kGemmTileK;  // weights of one operand tile
+constexpr int kKTileShift = kGemmTileK == 16 ? 11 : (kGemmTileK == 32 ? 12 : 13);
+static_assert(kKTile == 1u << kKTileShift, "operand tile of 16, 32 or 64 columns");
+constexpr uint32_t kRowBytes = 2 * kGemmTileK;     // one operand row: the swizzle's width
+constexpr uint32_t kATileBytes = 2 * kKTile;       // BF16 operand tile: 128 rows
+constexpr uint32_t kSwzMask = kRowBytes / 16 - 1;  // 16-byte chunks of a row, less one
+// descriptor layout type of that swizzle (128 B: 2, 64 B: 4, 32 B: 6)
+constexpr uint64_t kSwzLayout = kRowBytes == 128 ? 2 : (kRowBytes == 64 ? 4 : 6);
 constexpr int kMaxASlots = 32, kMaxBSlots = 32;
 constexpr int kCB = 128;  // chunk bits of the containers the kernel reads
 constexpr uint32_t kTileBytes = 32 * kCB / 8;
@@ -78,13 +83,13 @@ struct GemmMat {
     uint32_t n_tiles;     // warp tiles of the container
     uint32_t tile_begin;  // launch-wide index of its first warp tile
     uint32_t kt_begin;    // launch-wide index of its first operand tile
-    uint32_t k_tiles;     // K / 16: operand tiles per block of 128 output rows
+    uint32_t k_tiles;     // K / kGemmTileK: operand tiles per block of 128 output rows
     uint32_t n_out;       // N
     uint32_t pad;
 };
 
 struct GemmParams {
-    CUtensorMap xmap[kGemmMaxMats];  // x of each matrix: 2-D, box 16 x mpad, 32-byte swizzle
+    CUtensorMap xmap[kGemmMaxMats];  // x of each matrix: 2-D, box kGemmTileK x mpad, row-wide swizzle
     const uint32_t *meta, *syms;     // 12-bit multi-symbol table (window-walk fallback)
     const uint16_t *lut;             // hierarchical tables
     const uint32_t *fsm;             // byte-step transition tables
@@ -103,7 +108,7 @@ struct GemmParams {
 // Shared memory, from a 1024-byte aligned base: the transition table, the
 // root hierarchical table, the control block, per decode warp its stage and
 // exponent buffer, the operand slots and the activation slots (1024-byte
-// aligned; the 32-byte swizzle needs 256).
+// aligned, as the swizzle needs).
 struct GemmPlan {
     uint32_t off_lut, off_ctrl, off_warps, warp_bytes, off_a, off_b, b_bytes, total;
 };
@@ -117,7 +122,7 @@ __host__ __device__ inline GemmPlan make_gemm_plan(int rows, int mpad, int a_slo
     p.off_warps = p.off_ctrl + kCtrlBytes;
     p.warp_bytes = kStageBytes + exps_bytes;
     p.off_a = up1024(p.off_warps + kDecodeWarps * p.warp_bytes);
-    p.b_bytes = static_cast<uint32_t>(mpad) * 32u;
+    p.b_bytes = static_cast<uint32_t>(mpad) * kRowBytes;
     p.off_b = p.off_a + static_cast<uint32_t>(a_slots) * kATileBytes;
     p.total = p.off_b + static_cast<uint32_t>(b_slots) * p.b_bytes;
     return p;
@@ -192,18 +197,19 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&v)[16]) {
 
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// Shared-memory matrix descriptor of a K-major operand in the 32-byte
-// swizzle (layout type 6): rows of 32 bytes (16 BF16, one MMA's K), 8-row
-// groups 256 bytes apart (stride byte offset), the leading byte offset
-// unused (1), descriptor version 1.
-__device__ __forceinline__ uint64_t sw32_desc(uint32_t saddr) {
-    return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (uint64_t{1} << 16) | (uint64_t{256 >> 4} << 32) |
-           (uint64_t{1} << 46) | (uint64_t{6} << 61);
+// Shared-memory matrix descriptor of a K-major operand in the row-wide
+// swizzle: rows of kRowBytes, 8-row groups 8 kRowBytes apart (stride byte
+// offset), the leading byte offset unused (1), descriptor version 1.  The
+// k-th MMA of a tile (K = 16) starts 32 k bytes into the rows.
+__device__ __forceinline__ uint64_t swz_desc(uint32_t saddr) {
+    return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (uint64_t{1} << 16) |
+           (static_cast<uint64_t>(8u * kRowBytes >> 4) << 32) | (uint64_t{1} << 46) | (kSwzLayout << 61);
 }
 
-// Byte offset o (from a 256-byte aligned base) in the 32-byte swizzle: the
-// 16-byte half of a 32-byte row flips with bit 2 of the row (bit 4 ^= bit 7).
-__device__ __forceinline__ uint32_t swz32(uint32_t o) { return o ^ (((o >> 7) & 1u) << 4); }
+// Byte offset o (from a 1024-byte aligned base) in the row-wide swizzle: the
+// 16-byte chunks of a row are permuted by the row's low bits (address bits
+// 4.. XOR bits 7..).
+__device__ __forceinline__ uint32_t swz(uint32_t o) { return o ^ (((o >> 7) & kSwzMask) << 4); }
 
 // Elements [lo, hi) of an 8-weight half (the others belong to a neighbouring
 // tile or lie outside the CTA's range), one 2-byte store each.
@@ -509,7 +515,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_kernel(const __gr
                 if (in_lo < in_hi) {
                     // its k-tiles' operand slots are free once the k-tiles SA before were multiplied
                     kr0 = static_cast<uint32_t>((in_lo - lo) >> kKTileShift);
-                    kr1 = static_cast<uint32_t>((in_hi - 1u - lo) >> kKTileShift);  // kr0 + 1 at most: span <= 2048
+                    kr1 = static_cast<uint32_t>((in_hi - 1u - lo) >> kKTileShift);  // kr0 + 1 at most
                     bool ok = true;
                     if (lane == 0)
                         ok = wait_gen(&C.a_free[dA.r(kr0)], dA.q(kr0), C, P.wait_ns) &&
@@ -523,7 +529,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_kernel(const __gr
                 // ---- merge: half j (8 weights: 8 plane bytes, 8 exponents) -> 16
                 // bytes of an operand row.  The operand slots form a ring of
                 // ring_w weights, 2 bytes each in order (a k-tile's 128 rows of
-                // 16 weights), in the 32-byte swizzle; the exponents are cleared
+                // kGemmTileK weights), swizzled; the exponents are cleared
                 // for the next tile.  Positions relative to the tile's first half
                 // (32-bit: a tile spans < 2^16 weights).
                 const uint64_t e_first = base + (h0 << 3);
@@ -535,12 +541,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_kernel(const __gr
                                                 : static_cast<uint32_t>(rel0) -
                                                       dA.q(static_cast<uint32_t>(rel0) >> kKTileShift) * ring_w;
                 const bool wraps = rbase + 8u * nh > ring_w;
-                // no wrap: round rr of a lane is 512 bytes after round 0 (16 rows on, same swizzle)
-                const uint32_t a_lane = swz32(2u * rbase + 16u * static_cast<uint32_t>(lane));
+                // no wrap: round rr of a lane is 512 bytes after round 0 (512 / kRowBytes rows on);
+                // its swizzle chunk flips by (4 & kSwzMask) between even and odd rounds
+                const uint32_t a_even = swz(2u * rbase + 16u * static_cast<uint32_t>(lane));
+                const uint32_t a_odd = a_even ^ ((4u & kSwzMask) << 4);
                 auto ring_off = [&](uint32_t jj) -> uint32_t {
                     uint32_t rp = rbase + 8u * jj;
                     if (rp >= ring_w) rp -= ring_w;
-                    return swz32(2u * rp);
+                    return swz(2u * rp);
                 };
                 auto merge_one = [&](uint32_t jj, uint2 p2, uint32_t aoff) {
                     uint2 *xp = reinterpret_cast<uint2 *>(s_exps + 8u * jj);
@@ -557,7 +565,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_kernel(const __gr
 #pragma unroll
                 for (int rr = 0; rr < kPrefetchHalves; ++rr) {
                     const uint32_t jj = static_cast<uint32_t>(lane) + 32u * rr;
-                    if (jj < nh) merge_one(jj, pre[rr], wraps ? ring_off(jj) : a_lane + 512u * rr);
+                    if (jj < nh) merge_one(jj, pre[rr], wraps ? ring_off(jj) : ((rr & 1) ? a_odd : a_even) + 512u * rr);
                 }
                 for (uint32_t jj = static_cast<uint32_t>(lane) + 32u * kPrefetchHalves; jj < nh; jj += 32)
                     merge_one(jj, ld_global_stream_v2(plane + 8u * jj), ring_off(jj));
@@ -631,7 +639,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_kernel(const __gr
                             tc_fence_after();
                             const uint32_t a0 = smem_addr(abase + dA.r(issued) * kATileBytes);
                             const uint32_t b0 = smem_addr(smem + plan.off_b + dB.r(issued) * plan.b_bytes);
-                            tc_mma(tmem, sw32_desc(a0), sw32_desc(b0), idesc, issued > kr ? 1u : 0u);
+#pragma unroll
+                            for (int k16 = 0; k16 < kGemmTileK / 16; ++k16)
+                                tc_mma(tmem, swz_desc(a0 + 32u * k16), swz_desc(b0 + 32u * k16), idesc,
+                                       (issued > kr || k16 > 0) ? 1u : 0u);
                             tc_commit(&C.mma_done[dA.r(issued)]);
                             ++issued;
                             prog = true;
@@ -823,14 +834,14 @@ LaunchStatus build_gemm(const GemmJob *jobs, int n, int m, int *err, bool with_m
     if (max_span > kKTile) return LaunchStatus::kUnsupported;  // a tile's codes must touch <= 2 operand tiles
     P.max_span = static_cast<uint32_t>(max_span);
     P.total_kt = static_cast<uint32_t>(kts);
-    // slots: as many (operand tile, activation tile) pairs as fit, 4..32 (an
-    // activation slot is refilled only after the MMA that read it retired, so
-    // a short activation ring would pace the MMAs)
+    // slots: 4 activation tiles (8 when an operand tile holds fewer than 64
+    // columns), operand tiles as many as fit, 4..32
     P.exps_bytes = gemm_exps_bytes(P.max_span);
+    P.b_slots = kGemmTileK >= 64 ? 4 : 8;
     const uint32_t budget = 227u * 1024u - 1024u;  // opt-in shared memory less the alignment slack
-    P.a_slots = P.b_slots = kMaxASlots;
+    P.a_slots = kMaxASlots;
     while (P.a_slots > 4 && make_gemm_plan(rows, P.mpad, P.a_slots, P.b_slots, P.exps_bytes).total > budget)
-        P.b_slots = --P.a_slots;
+        --P.a_slots;
     if (make_gemm_plan(rows, P.mpad, P.a_slots, P.b_slots, P.exps_bytes).total > budget)
         return LaunchStatus::kUnsupported;
     P.a_magic = static_cast<uint32_t>(((uint64_t{1} << 32) + P.a_slots - 1) / P.a_slots);
@@ -853,7 +864,10 @@ LaunchStatus build_gemm(const GemmJob *jobs, int n, int m, int *err, bool with_m
             const cuuint32_t box[2] = {static_cast<cuuint32_t>(kGemmTileK), static_cast<cuuint32_t>(P.mpad)};
             const cuuint32_t estr[2] = {1, 1};
             if (enc(&P.xmap[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(jobs[i].x), dims, strides, box,
-                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    kRowBytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                     : (kRowBytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B),
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
                 return LaunchStatus::kInvalid;
         }

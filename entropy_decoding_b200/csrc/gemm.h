@@ -10,10 +10,10 @@
 
 namespace df11 {
 
-// Operand tile of the weights: 128 output rows x 16 reduction columns (one
-// 32-byte swizzle row of BF16 per output row, one MMA's K), 2048 weights.
+// Operand tile of the weights: 128 output rows x 64 reduction columns (one
+// 128-byte swizzle row of BF16 per output row, four MMAs' K), 8192 weights.
 constexpr int kGemmTileN = 128;
-constexpr int kGemmTileK = 16;
+constexpr int kGemmTileK = 64;
 constexpr int kGemmMaxMats = 8;    // matrices per launch (sharing one code)
 constexpr int kGemmMaxBatch = 64;  // rows of x (the MMA's N, padded to 16)
 constexpr int kGemmMaxCtas = 256;
@@ -30,9 +30,9 @@ struct GemmShape {
 };
 
 // The operand-tile order of a K x N row-major matrix w (element (k, n) at
-// k * N + n): tile t = nb * (K / 16) + kb holds rows n = 128 nb .. 128 nb +
-// 127 and columns k = 16 kb .. 16 kb + 15, element (r, c) at position
-// 2048 t + 16 r + c.  K % 16 == 0 and N % 128 == 0.
+// k * N + n): tile t = nb * (K / 64) + kb holds rows n = 128 nb .. 128 nb +
+// 127 and columns k = 64 kb .. 64 kb + 63, element (r, c) at position
+// 8192 t + 64 r + c.  K % 64 == 0 and N % 128 == 0.
 void gemm_tile_weights(const uint16_t *w, uint64_t k, uint64_t n, uint16_t *tiled, int n_threads);
 
 LaunchStatus gemm_launch_shape(const GemmJob *jobs, int n, int m, GemmShape *out);

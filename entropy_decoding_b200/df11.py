@@ -74,7 +74,7 @@ class GemmMatrix(ctypes.Structure):
                 ("y", ctypes.c_void_p)]
 
 
-GEMM_TILE_N, GEMM_TILE_K, GEMM_MAX_MATS, GEMM_MAX_BATCH = 128, 16, 8, 64
+GEMM_TILE_N, GEMM_TILE_K, GEMM_MAX_MATS, GEMM_MAX_BATCH = 128, 64, 8, 64
 
 WALKER_AUTO, WALKER_WINDOW, WALKER_BYTE_STEP = 0, 1, 2
 ENCODE_NO_CHUNK_COUNTS = 1  # encoder flag: leave out the chunk-counts section

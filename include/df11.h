@@ -476,27 +476,27 @@ df11_status df11_encode_device_noalloc(const df11_codebook *cb, const void *src_
  * Abstract: decoding aligned with the GEMM's tiling)
  * ------------------------------------------------------------------ */
 
-/* Operand tile of the fused GEMM: 128 output rows x 16 reduction columns. */
+/* Operand tile of the fused GEMM: 128 output rows x 64 reduction columns. */
 #define DF11_GEMM_TILE_N 128
-#define DF11_GEMM_TILE_K 16
+#define DF11_GEMM_TILE_K 64
 #define DF11_GEMM_MAX_MATS 8   /* matrices per df11_decode_gemm launch */
 #define DF11_GEMM_MAX_BATCH 64 /* rows of x */
 
 /* Writes the operand-tile order of a K x N BF16 weight matrix (host_w,
  * row-major: element (k, n) at k * N + n, the layer mapping K inputs to N
  * outputs) into host_tiled (K * N words, caller's buffer, not overlapping
- * host_w): tile t = nb * (K / 16) + kb holds outputs n = 128 nb ..
- * 128 nb + 127 and inputs k = 16 kb .. 16 kb + 15, element (r, c) at
- * 2048 t + 16 r + c, i.e. host_w[(16 kb + c) * N + 128 nb + r].  Encoding the
+ * host_w): tile t = nb * (K / 64) + kb holds outputs n = 128 nb ..
+ * 128 nb + 127 and inputs k = 64 kb .. 64 kb + 63, element (r, c) at
+ * 8192 t + 64 r + c, i.e. host_w[(64 kb + c) * N + 128 nb + r].  Encoding the
  * result with df11_encode gives the blob df11_decode_gemm consumes; decoding
- * it with df11_decode gives back the tiled order.  K % 16 == 0 and
+ * it with df11_decode gives back the tiled order.  K % 64 == 0 and
  * N % 128 == 0, else DF11_EINVAL. */
 df11_status df11_gemm_tile_weights(const uint16_t *host_w, uint64_t k, uint64_t n, uint16_t *host_tiled);
 
 typedef struct {
     const df11_blob *weights; /* bound blob of the tiled K x N matrix: BF16, the default layout
                                  (128-bit chunks, 32-chunk tiles, chunk counts), host sections present */
-    uint64_t k, n;            /* K inputs (multiple of 16), N outputs (multiple of 128) */
+    uint64_t k, n;            /* K inputs (multiple of 64), N outputs (multiple of 128) */
     const void *x;            /* device, M x K BF16 row-major, 16-byte aligned, rows K * 2 bytes apart */
     float *y;                 /* device, M x N FP32 row-major, 4-byte aligned: y += x W */
 } df11_gemm_matrix;

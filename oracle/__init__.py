@@ -385,17 +385,18 @@ def rans_decompress(c: RansCompressed) -> np.ndarray:
 # with Lossless LLM Weight Compression", Abstract: decoding aligned with the
 # GEMM's tiling).  Fusing changes where the decoded weights go, not what is
 # computed: the result is the plain product y = x W of the exactly decoded
-# weights.  The pages give no tile shape; the reading here is one tcgen05
-# MMA's operand tile of 128 output rows x 16 reduction columns, each tile a
-# contiguous run of the encoded weights.
+# weights.  The pages give no tile shape; the reading here is a tcgen05
+# operand tile of 128 output rows x 64 reduction columns (one 128-byte
+# swizzle row of BF16 per output row), each tile a contiguous run of the
+# encoded weights.
 
-GEMM_TILE_N, GEMM_TILE_K = 128, 16
+GEMM_TILE_N, GEMM_TILE_K = 128, 64
 
 
 def gemm_tile(w: np.ndarray, k: int, n: int) -> np.ndarray:
     """Operand-tile order of a K x N matrix (row-major, element (k, n) at
-    k * N + n): tile t = nb * (K / 16) + kb holds W[16 kb + c][128 nb + r] at
-    position 2048 t + 16 r + c."""
+    k * N + n): tile t = nb * (K / 64) + kb holds W[64 kb + c][128 nb + r] at
+    position 8192 t + 64 r + c."""
     w = np.asarray(w).reshape(k, n)
     return w.reshape(k // GEMM_TILE_K, GEMM_TILE_K, n // GEMM_TILE_N, GEMM_TILE_N).transpose(2, 0, 3, 1).reshape(-1)
 

@@ -27,17 +27,17 @@ def test_tile_positions_match_hand_derivation():
         assert int(oracle.gemm_tile(w, k, n)[pos]) == value, (k, n, pos)
 
 
-@pytest.mark.parametrize("k,n", [(16, 128), (128, 384), (336, 256)])
+@pytest.mark.parametrize("k,n", [(64, 128), (128, 384), (320, 256)])
 def test_untile_inverts_tile(k, n):
     w = np.random.default_rng(k + n).integers(0, 1 << 16, k * n, dtype=np.uint16)
     t = oracle.gemm_tile(w, k, n)
     assert sorted(t.tolist()) == sorted(w.tolist())  # a permutation
     assert np.array_equal(oracle.gemm_untile(t, k, n).reshape(-1), w)
-    # every tile is one contiguous 2048-weight run of 128 output rows x 16 inputs
-    tiles = t.reshape(-1, 128, 16)
+    # every tile is one contiguous 8192-weight run of 128 output rows x 64 inputs
+    tiles = t.reshape(-1, 128, 64)
     W = w.reshape(k, n)
-    nb, kb = 1 % (n // 128), (k // 16) - 1
-    assert np.array_equal(tiles[nb * (k // 16) + kb], W[16 * kb: 16 * kb + 16, 128 * nb: 128 * nb + 128].T)
+    nb, kb = 1 % (n // 128), (k // 64) - 1
+    assert np.array_equal(tiles[nb * (k // 64) + kb], W[64 * kb: 64 * kb + 64, 128 * nb: 128 * nb + 128].T)
 
 
 def _bf16(v: float) -> int:

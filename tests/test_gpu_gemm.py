@@ -73,8 +73,8 @@ def _check(oracle_mod, y, x, w, m, k, n, what=""):
     assert not bad.any(), f"{what}: {int(bad.sum())} of {bad.size} outside the bound, first at {np.argwhere(bad)[:4]}"
 
 
-@pytest.mark.parametrize("k,n,m", [(16, 128, 1), (64, 128, 2), (256, 256, 16), (512, 384, 5), (1024, 512, 33),
-                                   (4096, 256, 64), (208, 640, 17), (48, 1152, 16)])
+@pytest.mark.parametrize("k,n,m", [(64, 128, 1), (128, 128, 2), (256, 256, 16), (512, 384, 5), (1024, 512, 33),
+                                   (4096, 256, 64), (192, 640, 17), (64, 1152, 16)])
 def test_single_matrix(df11, oracle_mod, k, n, m):
     w, x = _weights(k, n, k + n + m), _acts(m, k, k + n + m)
     tiled, (blob,) = _encode(df11, oracle_mod, [w], [(k, n)])
@@ -87,14 +87,14 @@ def test_single_matrix(df11, oracle_mod, k, n, m):
 
 
 def test_operand_tiles_split_between_ctas(df11, oracle_mod):
-    """2048 operand tiles over the SMs: CTA ranges start and end inside blocks
+    """512 operand tiles over the SMs: CTA ranges start and end inside blocks
     of 128 output rows (their y rows are summed by several CTAs) and inside
     warp tiles of the container."""
     k, n, m = 4096, 1024, 16
     w, x = _weights(k, n, 5), _acts(m, k, 5)
     _, (blob,) = _encode(df11, oracle_mod, [w], [(k, n)])
     grid, block, smem = df11.df11_decode_gemm_launch_shape([(blob, k, n, 0, 0)], m)
-    assert block % 128 == 0 and 1 < grid <= 148 and (k // 16) * (n // 128) % grid != 0
+    assert block % 128 == 0 and 1 < grid <= 148 and (k // 64) * (n // 128) % grid != 0
     (y,), err = _run(df11, [blob], [(k, n)], [x], m)
     assert err == 0
     _check(oracle_mod, y, x, w, m, k, n)
@@ -127,7 +127,7 @@ def test_against_decode_then_matmul(df11, oracle_mod):
     assert int(err.item()) == 0
     dec = out[: 2 * k * n].view(torch.int16).cpu().numpy().view(np.uint16)
     assert np.array_equal(dec, tiled[0])  # the tiled order, bit for bit
-    wd = out[: 2 * k * n].view(torch.bfloat16).reshape(n // 128, k // 16, 128, 16).permute(1, 3, 0, 2).reshape(k, n)
+    wd = out[: 2 * k * n].view(torch.bfloat16).reshape(n // 128, k // 64, 128, 64).permute(1, 3, 0, 2).reshape(k, n)
     xd = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16).reshape(m, k)
     ref = (xd.float() @ wd.float()).double().cpu().numpy()
     (y,), err = _run(df11, [blob], [(k, n)], [x], m)

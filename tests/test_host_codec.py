@@ -423,7 +423,7 @@ def test_device_image_layout(df11):
     assert lay["total"] - lay["plane"] >= info.plane_bytes + 32
 
 
-@pytest.mark.parametrize("k,n", [(16, 128), (48, 384), (4096, 1024)])
+@pytest.mark.parametrize("k,n", [(64, 128), (192, 384), (4096, 1024)])
 def test_gemm_tile_order_matches_oracle(df11, oracle_mod, k, n):
     """The library's operand-tile permutation (host) against the oracle's."""
     w = np.random.default_rng(k * n).integers(0, 1 << 16, k * n, dtype=np.uint16)
