@@ -306,9 +306,11 @@ df11_status df11_decode_ex(const df11_blob *const *blobs, void *const *dst_dev, 
         o.overlap = opts->overlap;
         o.diag_expire_waits = opts->diag_expire_waits;
         o.count_walk = opts->count_walk;
+        o.diag_check_bounds = opts->diag_check_bounds;
         if (o.chunks_per_thread < 0 || o.ctas_per_sm < 0 || o.warps_per_cta < 0 || o.walker < 0 ||
             o.walker > DF11_WALKER_BYTE_STEP || o.max_ctas < 0 || o.overlap < 0 || o.overlap > 1 ||
-            o.diag_expire_waits < 0 || o.diag_expire_waits > 1 || o.count_walk < 0 || o.count_walk > 1)
+            o.diag_expire_waits < 0 || o.diag_expire_waits > 1 || o.count_walk < 0 || o.count_walk > 1 ||
+            o.diag_check_bounds < 0 || o.diag_check_bounds > 1)
             return DF11_EINVAL;
     }
     return from_launch(df11::launch_decode(bs, dst_dev, n_blobs, dev_err_flag, o,

@@ -100,6 +100,11 @@ __device__ __forceinline__ uint4 ld_global_stream_v4(const void *p) {
     return v;
 }
 
+// One group's plane bytes, checked in the bounds-checked build (zeros outside).
+__device__ __forceinline__ uint4 plane_v4(const uint8_t *p, Guard &G) {
+    return G.pl(p, 16) ? ld_global_stream_v4(p) : make_uint4(0u, 0u, 0u, 0u);
+}
+
 __device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
@@ -127,11 +132,12 @@ __device__ __noinline__ void store_partial(uint8_t *out, uint4 a, uint4 b, uint3
 // [lo, hi) are the tile's elements relative to the first group's first element.
 template <int DT, bool PARTIAL = true>
 __device__ __forceinline__ void merge_group(uint4 p4, uint32_t i, uint8_t *s_exps, uint8_t *dst_tile, uint32_t lo,
-                                            uint32_t hi) {
+                                            uint32_t hi, Guard &G) {
     constexpr uint32_t GROUP = DT == 0 ? 16u : 32u;
     if constexpr (!PARTIAL) {
         if (i * GROUP < lo || i * GROUP + GROUP > hi) return;  // edge group: stored by edge_groups()
     }
+    if (!G.ex(s_exps + (DT == 0 ? 16u : 32u) * i, DT == 0 ? 16u : 32u)) return;
     uint4 a, b;
     if constexpr (DT == 0) {
         uint4 *xp = reinterpret_cast<uint4 *>(s_exps + 16 * i);
@@ -155,9 +161,11 @@ __device__ __forceinline__ void merge_group(uint4 p4, uint32_t i, uint8_t *s_exp
     const uint32_t e0 = i * GROUP;
     uint8_t *out = dst_tile + 32u * i;
     if (!PARTIAL || (e0 >= lo && e0 + GROUP <= hi)) {
-        st_global_v4(out, a);
-        st_global_v4(out + 16, b);
-    } else {
+        if (G.out(out, 32)) {
+            st_global_v4(out, a);
+            st_global_v4(out + 16, b);
+        }
+    } else if (G.out_elems(out, e0, GROUP, lo, hi, DT == 0 ? 2u : 1u)) {
         store_partial<DT>(out, a, b, e0, lo, hi);
     }
 }
@@ -168,7 +176,8 @@ __device__ __forceinline__ void merge_group(uint4 p4, uint32_t i, uint8_t *s_exp
 // (shuffled), its exponents from shared memory, which are then cleared.
 template <int DT>
 __device__ __forceinline__ void edge_groups(const uint4 (&pre)[kPrefetchGroups], const uint8_t *plane, uint32_t ng,
-                                            uint8_t *s_exps, uint8_t *dst_tile, uint32_t lo, uint32_t hi, int lane) {
+                                            uint8_t *s_exps, uint8_t *dst_tile, uint32_t lo, uint32_t hi, int lane,
+                                            Guard &G) {
     constexpr uint32_t GROUP = DT == 0 ? 16u : 32u;
     const uint32_t last = ng - 1;
     const bool head = lo != 0, tail = (hi % GROUP) != 0 && !(head && last == 0);
@@ -191,16 +200,17 @@ __device__ __forceinline__ void edge_groups(const uint4 (&pre)[kPrefetchGroups],
             v.z = __shfl_sync(0xFFFFFFFFu, mine.z, src);
             v.w = __shfl_sync(0xFFFFFFFFu, mine.w, src);
         } else {
-            v = ld_global_stream_v4(plane + 16u * g);
+            v = plane_v4(plane + 16u * g, G);
         }
 #pragma unroll
         for (uint32_t j0 = 0; j0 < GROUP; j0 += 32) {
             const uint32_t j = j0 + static_cast<uint32_t>(lane);
             if (j < GROUP) {
                 const uint32_t e = g * GROUP + j;
+                if (!G.ex(s_exps + e, 1)) continue;
                 const uint32_t x = s_exps[e];
                 s_exps[e] = 0;
-                if (e >= lo && e < hi) {
+                if (e >= lo && e < hi && G.out(dst_tile + e * (DT == 0 ? 2u : 1u), DT == 0 ? 2u : 1u)) {
                     const uint32_t wi = DT == 0 ? (j >> 2) : (j >> 3);
                     const uint32_t word = wi == 0 ? v.x : (wi == 1 ? v.y : (wi == 2 ? v.z : v.w));
                     if constexpr (DT == 0) {
@@ -247,9 +257,10 @@ __device__ __noinline__ void store_partial_half(uint8_t *out, uint4 a, uint32_t 
 
 template <int DT, bool PARTIAL>
 __device__ __forceinline__ void merge_half(uint2 p2, uint32_t j, uint8_t *s_exps, uint8_t *dst_tile, uint32_t lo,
-                                           uint32_t hi) {
+                                           uint32_t hi, Guard &G) {
     uint4 a;
     uint32_t e0;
+    if (!G.ex(s_exps + (DT == 0 ? 8u : 16u) * j, DT == 0 ? 8u : 16u)) return;
     if constexpr (DT == 0) {
         uint2 *xp = reinterpret_cast<uint2 *>(s_exps + 8 * j);
         const uint2 x2 = *xp;
@@ -267,16 +278,20 @@ __device__ __forceinline__ void merge_half(uint2 p2, uint32_t j, uint8_t *s_exps
     }
     uint8_t *out = dst_tile + 16u * j;
     constexpr uint32_t HALF = DT == 0 ? 8u : 16u;
-    if (!PARTIAL || (e0 >= lo && e0 + HALF <= hi)) st_global_v4(out, a);
-    else store_partial_half<DT>(out, a, e0, lo, hi);
+    if (!PARTIAL || (e0 >= lo && e0 + HALF <= hi)) {
+        if (G.out(out, 16)) st_global_v4(out, a);
+    } else if (G.out_elems(out, e0, HALF, lo, hi, DT == 0 ? 2u : 1u)) {
+        store_partial_half<DT>(out, a, e0, lo, hi);
+    }
 }
 
 // Round U (>= 1) of the merge for a lane: half j = lane + 32 U, whole (no
 // piecewise store).  x_l and out_l are the lane's round-0 addresses in the
 // exponent buffer and the tile's output.
 template <int DT, int U>
-__device__ __forceinline__ void merge_half_round(uint2 p2, uint8_t *x_l, uint8_t *out_l) {
+__device__ __forceinline__ void merge_half_round(uint2 p2, uint8_t *x_l, uint8_t *out_l, Guard &G) {
     uint4 a;
+    if (!G.ex(x_l + (DT == 0 ? 256 : 512) * U, DT == 0 ? 8u : 16u)) return;
     if constexpr (DT == 0) {
         uint2 *xp = reinterpret_cast<uint2 *>(x_l + 256 * U);
         const uint2 x2 = *xp;
@@ -290,13 +305,13 @@ __device__ __forceinline__ void merge_half_round(uint2 p2, uint8_t *x_l, uint8_t
         merge_e4m3x8(p2.x, x4.x, x4.y, a.x, a.y);
         merge_e4m3x8(p2.y, x4.z, x4.w, a.z, a.w);
     }
-    st_global_v4_at<512 * U>(out_l, a);
+    if (G.out(out_l + 512 * U, 16)) st_global_v4_at<512 * U>(out_l, a);
 }
 
 template <int DT, int... U>
 __device__ __forceinline__ void merge_rounds(const uint2 *pre, uint32_t lane, uint32_t nh, uint8_t *x_l, uint8_t *out_l,
-                                             std::integer_sequence<int, U...>) {
-    ((lane + 32u * (U + 1) < nh ? merge_half_round<DT, U + 1>(pre[U + 1], x_l, out_l) : (void)0), ...);
+                                             Guard &G, std::integer_sequence<int, U...>) {
+    ((lane + 32u * (U + 1) < nh ? merge_half_round<DT, U + 1>(pre[U + 1], x_l, out_l, G) : (void)0), ...);
 }
 
 
@@ -346,7 +361,8 @@ __global__ void __launch_bounds__(NTH + 32, (NTH + 32) * 3 <= 1024 ? 3 : 1)
         for (int i = tid; i < kMultiEntries * 4 / 16; i += NTH + 32) s[i] = __ldg(g + i);
         g = reinterpret_cast<const uint4 *>(P.lut);
         s = reinterpret_cast<uint4 *>(s_lut);
-        for (int i = tid; i < n_lut_smem * kLutEntries * 2 / 16; i += NTH + 32) s[i] = __ldg(g + i);
+        for (int i = tid; i < lut_stage_count(n_lut_smem, P.n_luts) * kLutEntries * 2 / 16; i += NTH + 32)
+            s[i] = __ldg(g + i);
         s = reinterpret_cast<uint4 *>(s_exps);
         for (uint32_t i = tid; i < plan.exps_bytes / 16; i += NTH + 32) s[i] = make_uint4(0, 0, 0, 0);
     }
@@ -381,13 +397,24 @@ __global__ void __launch_bounds__(NTH + 32, (NTH + 32) * 3 <= 1024 ? 3 : 1)
             while (ti + 1 < P.n_tensors && t >= P.t[ti + 1].tile_begin) ++ti;
             const TensorDesc &d = P.t[ti];
             const uint32_t lt = t - d.tile_begin;
-            uint64_t S = __ldg(d.out_off + lt);
-            const uint64_t E = __ldg(d.out_off + lt + 1);
+            uint32_t cerr = 0;
+            const bool src_ok =
+                in_bounds(lt, 2, static_cast<uint64_t>(d.n_tiles) + 1u, cerr) &&
+                in_bounds(static_cast<uint64_t>(lt) * TILE_BYTES, plan.stream_bytes,
+                          static_cast<uint64_t>(d.n_tiles) * TILE_BYTES + kStreamTail, cerr) &&
+                in_bounds(static_cast<uint64_t>(lt) * CHUNKS, plan.gaps_bytes,
+                          static_cast<uint64_t>(d.n_tiles) * CHUNKS + kGapsTail, cerr);
+            uint64_t S = src_ok ? __ldg(d.out_off + lt) : 0u;
+            const uint64_t E = src_ok ? __ldg(d.out_off + lt + 1) : 0u;
             uint32_t bad = 0;
             if (E < S || E > d.n || E - S > max_span) {
                 report(P.err, DF11_DEV_ERR_AUX);
                 bad = 1;
                 S = 0;
+            }
+            if (!src_ok) {
+                report(P.err, cerr);
+                bad = 1;
             }
             const uint32_t span = bad ? 0u : static_cast<uint32_t>(E - S);
             StageMeta &m = smeta[s];
@@ -396,15 +423,22 @@ __global__ void __launch_bounds__(NTH + 32, (NTH + 32) * 3 <= 1024 ? 3 : 1)
             m.tensor = static_cast<uint32_t>(ti);
             m.local_tile = lt;
             m.bad = bad;
-            mbar_arrive_expect_tx(&full_s[s], plan.stream_bytes + plan.gaps_bytes);
-            bulk_load(s_stream0 + s * stream_stride, d.stream + static_cast<uint64_t>(lt) * TILE_BYTES,
-                      plan.stream_bytes, &full_s[s]);
-            bulk_load(s_gaps0 + s * gaps_stride, d.gaps + static_cast<uint64_t>(lt) * CHUNKS, plan.gaps_bytes,
-                      &full_s[s]);
+            if (src_ok) {
+                mbar_arrive_expect_tx(&full_s[s], plan.stream_bytes + plan.gaps_bytes);
+                bulk_load(s_stream0 + s * stream_stride, d.stream + static_cast<uint64_t>(lt) * TILE_BYTES,
+                          plan.stream_bytes, &full_s[s]);
+                bulk_load(s_gaps0 + s * gaps_stride, d.gaps + static_cast<uint64_t>(lt) * CHUNKS, plan.gaps_bytes,
+                          &full_s[s]);
+            } else {
+                mbar_arrive(&full_s[s]);  // nothing copied: the tile is marked bad
+            }
             // the merge reads this tile's plane span from global memory: pull it into L2 now
             if (span) {
                 const uint64_t a0 = (S / GROUP) * 16u, a1 = ((S + span + GROUP - 1) / GROUP) * 16u;
-                prefetch_l2(d.plane + a0, static_cast<uint32_t>(a1 - a0));
+                Guard Gp;
+                Gp.tensor<DT>(d);
+                if (Gp.pl(d.plane + a0, a1 - a0)) prefetch_l2(d.plane + a0, static_cast<uint32_t>(a1 - a0));
+                if (Gp.flags()) report(P.err, Gp.flags());
             }
             armed |= 1u << s;
             last_parity = (last_parity & ~(1u << s)) | (ph << s);
@@ -417,8 +451,12 @@ __global__ void __launch_bounds__(NTH + 32, (NTH + 32) * 3 <= 1024 ? 3 : 1)
     }
 
     // ---------------- consumer warps
-    const Tables T{s_meta, s_syms, s_lut, P.lut, n_lut_smem, P.n_luts};
+    const Tables T{s_meta, s_syms, s_lut, P.lut, n_lut_smem, P.n_luts, smem_addr(s_exps),
+                   smem_addr(s_exps) + plan.exps_bytes};
     uint32_t err = 0;
+    in_bounds(0, static_cast<uint64_t>(max(n_lut_smem, 0)), static_cast<uint64_t>(max(P.n_luts, 0)), err);
+    Guard G;
+    G.buffer(s_exps, P.diag_bounds ? 0u : plan.exps_bytes);
     uint32_t k = 0;
     for (uint32_t t = blockIdx.x; t < P.total_tiles; t += gridDim.x, ++k) {
         const int s = static_cast<int>(k % kStreamStages);
@@ -427,6 +465,7 @@ __global__ void __launch_bounds__(NTH + 32, (NTH + 32) * 3 <= 1024 ? 3 : 1)
         const StageMeta m = smeta[s];
         const int ti = landed && m.tensor < static_cast<uint32_t>(P.n_tensors) ? static_cast<int>(m.tensor) : 0;
         const TensorDesc &d = P.t[ti];
+        G.tensor<DT>(d);
 
         // ---- the tile's plane span (16 bytes per group of GROUP elements): the
         // first kPrefetchGroups groups of this thread are loaded now, so they
@@ -439,13 +478,15 @@ __global__ void __launch_bounds__(NTH + 32, (NTH + 32) * 3 <= 1024 ? 3 : 1)
 #pragma unroll
         for (int u = 0; u < kPrefetchGroups; ++u) {
             const uint32_t i = tid + u * NTH;
-            if (i < ng) pre[u] = ld_global_stream_v4(plane + 16u * i);
+            if (i < ng) pre[u] = plane_v4(plane + 16u * i, G);
         }
 
         // ---- this thread's CPT consecutive chunks + one look-ahead word
         const uint8_t *sst = s_stream0 + s * stream_stride + tid * (CPT * CB / 8);
-        uint32_t w[CPT * CW + 1];
-        if constexpr ((CPT * CW) % 4 == 0) {
+        uint32_t w[CPT * CW + 1] = {};
+        const bool st_ok = in_bounds(static_cast<uint64_t>(tid) * (CPT * CB / 8), CPT * CB / 8 + 4, plan.stream_bytes, err);
+        if (!st_ok) {
+        } else if constexpr ((CPT * CW) % 4 == 0) {
 #pragma unroll
             for (int j = 0; j < CPT * CW / 4; ++j) {
                 const uint4 v = *reinterpret_cast<const uint4 *>(sst + 16 * j);
@@ -462,10 +503,11 @@ __global__ void __launch_bounds__(NTH + 32, (NTH + 32) * 3 <= 1024 ? 3 : 1)
         {
             const uint32_t nxt = __shfl_down_sync(0xFFFFFFFFu, w[0], 1);
             w[CPT * CW] =
-                lane == 31 ? *reinterpret_cast<const uint32_t *>(sst + CPT * CB / 8) : nxt;
+                lane == 31 ? (st_ok ? *reinterpret_cast<const uint32_t *>(sst + CPT * CB / 8) : 0u) : nxt;
         }
         int gap[CPT], E[CPT];
         const uint8_t *sg = s_gaps0 + s * gaps_stride + tid * CPT;
+        const bool sg_ok = in_bounds(static_cast<uint64_t>(tid) * CPT, CPT, plan.gaps_bytes, err);
         // stream bits of this tile from this thread's first chunk on (clamped)
         const int64_t rem64 = static_cast<int64_t>(d.total_bits) -
                               static_cast<int64_t>(m.local_tile) * (static_cast<int64_t>(CHUNKS) * CB) -
@@ -473,7 +515,7 @@ __global__ void __launch_bounds__(NTH + 32, (NTH + 32) * 3 <= 1024 ? 3 : 1)
         const int rem = rem64 > CPT * CB ? CPT * CB : (rem64 < 0 ? 0 : static_cast<int>(rem64));
 #pragma unroll
         for (int c = 0; c < CPT; ++c) {
-            const int g = sg[c];
+            const int g = sg_ok ? sg[c] : 0;
             if (g >= 32) err |= DF11_DEV_ERR_AUX;
             gap[c] = min(g, 63);
             E[c] = min(max(rem - c * CB, 0), CB);
@@ -532,13 +574,13 @@ __global__ void __launch_bounds__(NTH + 32, (NTH + 32) * 3 <= 1024 ? 3 : 1)
 #pragma unroll
             for (int u = 0; u < kPrefetchGroups; ++u) {
                 const uint32_t i = tid + u * NTH;
-                if (i < ng) merge_group<DT>(pre[u], i, s_exps, dst_tile, lo, hi);
+                if (i < ng) merge_group<DT>(pre[u], i, s_exps, dst_tile, lo, hi, G);
             }
             for (uint32_t i = tid + kPrefetchGroups * NTH; i < ng; i += NTH)
-                merge_group<DT>(ld_global_stream_v4(plane + 16u * i), i, s_exps, dst_tile, lo, hi);
+                merge_group<DT>(plane_v4(plane + 16u * i, G), i, s_exps, dst_tile, lo, hi, G);
         }
     }
-    report(P.err, err);
+    report(P.err, err | G.flags());
 }
 
 // ------------------------------------------------------------------ warp-tile kernel
@@ -613,7 +655,8 @@ __global__ void __launch_bounds__(NWARP * 32, NWARP <= 8 ? 4 : 2)
         for (int i = tid; i < kMultiEntries * 4 / 16; i += NWARP * 32) s[i] = __ldg(g + i);
         g = reinterpret_cast<const uint4 *>(P.lut);
         s = reinterpret_cast<uint4 *>(s_lut);
-        for (int i = tid; i < n_lut_smem * kLutEntries * 2 / 16; i += NWARP * 32) s[i] = __ldg(g + i);
+        for (int i = tid; i < lut_stage_count(n_lut_smem, P.n_luts) * kLutEntries * 2 / 16; i += NWARP * 32)
+            s[i] = __ldg(g + i);
         s = reinterpret_cast<uint4 *>(s_exps);
         for (uint32_t i = lane; i < plan.exps_bytes / 16; i += 32) s[i] = make_uint4(0, 0, 0, 0);
     }
@@ -636,9 +679,17 @@ __global__ void __launch_bounds__(NWARP * 32, NWARP <= 8 ? 4 : 2)
         const TensorDesc &d = P.t[ti_issue];
         const uint32_t lt = t - d.tile_begin;
         uint8_t *st = stage0 + s * plan.stage_bytes;
-        mbar_arrive_expect_tx(&full[s], TILE_BYTES + 16u + 32u);
-        bulk_load(st, d.stream + static_cast<uint64_t>(lt) * TILE_BYTES, TILE_BYTES + 16u, &full[s]);
-        bulk_load(st + TILE_BYTES + 16u, d.gaps + static_cast<uint64_t>(lt) * 32u, 32u, &full[s]);
+        uint32_t cerr = 0;
+        if (in_bounds(static_cast<uint64_t>(lt) * TILE_BYTES, TILE_BYTES + 16u,
+                      static_cast<uint64_t>(d.n_tiles) * TILE_BYTES + kStreamTail, cerr) &&
+            in_bounds(static_cast<uint64_t>(lt) * 32u, 32u, static_cast<uint64_t>(d.n_tiles) * 32u + kGapsTail, cerr)) {
+            mbar_arrive_expect_tx(&full[s], TILE_BYTES + 16u + 32u);
+            bulk_load(st, d.stream + static_cast<uint64_t>(lt) * TILE_BYTES, TILE_BYTES + 16u, &full[s]);
+            bulk_load(st + TILE_BYTES + 16u, d.gaps + static_cast<uint64_t>(lt) * 32u, 32u, &full[s]);
+        } else {
+            mbar_arrive(&full[s]);  // nothing copied: the stage keeps stale bytes, the error is reported
+            report(P.err, cerr);
+        }
     };
     if (!P.expire) {
         if (lane == 0) {
@@ -649,17 +700,23 @@ __global__ void __launch_bounds__(NWARP * 32, NWARP <= 8 ? 4 : 2)
         if (first + stride < P.total_tiles) issued |= 2u;
     }
 
-    const Tables T{s_meta, s_syms, s_lut, P.lut, n_lut_smem, P.n_luts};
+    const Tables T{s_meta, s_syms, s_lut, P.lut, n_lut_smem, P.n_luts, smem_addr(s_exps),
+                   smem_addr(s_exps) + plan.exps_bytes};
     uint32_t err = 0;
+    in_bounds(0, static_cast<uint64_t>(max(n_lut_smem, 0)), static_cast<uint64_t>(max(P.n_luts, 0)), err);
+    Guard G;
+    G.buffer(s_exps, P.diag_bounds ? 0u : plan.exps_bytes);
     uint32_t k = 0;
     for (uint32_t t = first; t < P.total_tiles; t += stride, ++k) {
         const int s = static_cast<int>(k & 1u);
         const uint32_t ph = (k >> 1) & 1u;
         ti_cur = tensor_of(P, t, ti_cur);
         const TensorDesc &d = P.t[ti_cur];
+        G.tensor<DT>(d);
         const uint32_t lt = t - d.tile_begin;
-        uint64_t S = __ldg(d.out_off + lt);
-        const uint64_t Eo = __ldg(d.out_off + lt + 1);
+        const bool oo = in_bounds(lt, 2, static_cast<uint64_t>(d.n_tiles) + 1u, err);
+        uint64_t S = oo ? __ldg(d.out_off + lt) : 1u;
+        const uint64_t Eo = oo ? __ldg(d.out_off + lt + 1) : 0u;
         const bool bad = Eo < S || Eo > d.n || Eo - S > max_span;
         if (bad) S = 0;
         const uint32_t span = bad ? 0u : static_cast<uint32_t>(Eo - S);
@@ -672,7 +729,7 @@ __global__ void __launch_bounds__(NWARP * 32, NWARP <= 8 ? 4 : 2)
 #pragma unroll
         for (int u = 0; u < kPrefetchGroups; ++u) {
             const uint32_t i = lane + 32u * u;
-            if (i < ng) pre[u] = ld_global_stream_v4(plane + 16u * i);
+            if (i < ng) pre[u] = plane_v4(plane + 16u * i, G);
         }
 
         const bool landed = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], ph, P.wait_ns));
@@ -681,6 +738,8 @@ __global__ void __launch_bounds__(NWARP * 32, NWARP <= 8 ? 4 : 2)
             break;
         }
         issued &= ~(1u << s);
+        // every stage read below stays inside the stage: 32 chunks, the look-ahead word, 32 gaps
+        in_bounds(TILE_BYTES + 16u, 32u, plan.stage_bytes, err);
         const uint8_t *st = stage0 + s * plan.stage_bytes;
         uint32_t w[CW + 1];
         if constexpr (CW % 4 == 0) {
@@ -745,14 +804,15 @@ __global__ void __launch_bounds__(NWARP * 32, NWARP <= 8 ? 4 : 2)
 #pragma unroll
             for (int u = 0; u < kPrefetchGroups; ++u) {
                 const uint32_t i = lane + 32u * u;
-                if (i < ng) merge_group<DT, false>(pre[u], i, s_exps, dst_tile, lo, hi);
+                if (i < ng) merge_group<DT, false>(pre[u], i, s_exps, dst_tile, lo, hi, G);
             }
             for (uint32_t i = lane + 32u * kPrefetchGroups; i < ng; i += 32)
-                merge_group<DT, false>(ld_global_stream_v4(plane + 16u * i), i, s_exps, dst_tile, lo, hi);
-            edge_groups<DT>(pre, plane, ng, s_exps, dst_tile, lo, hi, lane);
+                merge_group<DT, false>(plane_v4(plane + 16u * i, G), i, s_exps, dst_tile, lo, hi, G);
+            edge_groups<DT>(pre, plane, ng, s_exps, dst_tile, lo, hi, lane, G);
             __syncwarp();
         }
     }
+    err |= G.flags();
     // after an abort: wait (bounded) for copies that were issued but never consumed
     for (int s = 0; s < 2; ++s)
         if (issued & (1u << s))
@@ -872,18 +932,36 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         ti_issue = tensor_of(P, t, ti_issue);
         const TensorDesc &d = P.t[ti_issue];
         const uint32_t lt = t - d.tile_begin;
-        mbar_arrive_expect_tx(&full[0], STAGE_TX);
-        bulk_load(stage, d.stream + static_cast<uint64_t>(lt) * TILE_BYTES, TILE_BYTES + 16u, &full[0]);
-        bulk_load(stage + TILE_BYTES + 16u, d.gaps + static_cast<uint64_t>(lt) * 32u, 48u, &full[0]);
-        if constexpr (CNT) bulk_load(stage + TILE_BYTES + 64u, d.counts + static_cast<uint64_t>(lt) * 32u, 32u, &full[0]);
+        uint32_t cerr = 0;
+        if (in_bounds(static_cast<uint64_t>(lt) * TILE_BYTES, TILE_BYTES + 16u,
+                      static_cast<uint64_t>(d.n_tiles) * TILE_BYTES + kStreamTail, cerr) &&
+            in_bounds(static_cast<uint64_t>(lt) * 32u, 48u, static_cast<uint64_t>(d.n_tiles) * 32u + kGapsTail, cerr) &&
+            (!CNT || in_bounds(static_cast<uint64_t>(lt) * 32u, 32u, static_cast<uint64_t>(d.n_tiles) * 32u, cerr))) {
+            mbar_arrive_expect_tx(&full[0], STAGE_TX);
+            bulk_load(stage, d.stream + static_cast<uint64_t>(lt) * TILE_BYTES, TILE_BYTES + 16u, &full[0]);
+            bulk_load(stage + TILE_BYTES + 16u, d.gaps + static_cast<uint64_t>(lt) * 32u, 48u, &full[0]);
+            if constexpr (CNT)
+                bulk_load(stage + TILE_BYTES + 64u, d.counts + static_cast<uint64_t>(lt) * 32u, 32u, &full[0]);
+        } else {
+            mbar_arrive(&full[0]);  // nothing copied: the stage keeps stale bytes, the error is reported
+            report(P.err, cerr);
+        }
     };
     if (lane == 0 && t_begin < t_end && !P.expire) issue(t_begin);
     bool pending = t_begin < t_end && !P.expire;
 
     // the window walk of the fallback: 12-bit table in global memory, root
     // hierarchical table in shared memory
-    const Tables T{P.meta, P.syms, s_lut, P.lut, 1, P.n_luts};
+    const Tables T{P.meta, P.syms, s_lut, P.lut, 1, P.n_luts, smem_addr(s_exps), smem_addr(s_exps) + plan.exps_bytes};
     uint32_t err = 0;
+    // every stage read stays inside the stage: 32 chunks, the look-ahead
+    // words, 48 gaps, with stored counts 32 counts
+    in_bounds(0, STAGE_TX, plan.stage_bytes, err);
+    Guard G;
+    G.buffer(s_exps, P.diag_bounds ? 0u : plan.exps_bytes);
+    const uint32_t exps_lo = smem_addr(s_exps), exps_hi = exps_lo + plan.exps_bytes;
+    const uint32_t ctl_bytes = static_cast<uint32_t>(rows) * (kFsmRowBytes / 2);
+    const uint32_t fsm_bytes = static_cast<uint32_t>(rows) * kFsmRowBytes;
     uint32_t k = 0;
     // carried group: exponents of its elements [0, carry_n) at the buffer start
     uint32_t carry_n = 0;
@@ -893,8 +971,11 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
     auto flush_carry = [&]() {
         if (lane == 0) {
             const TensorDesc &dc = P.t[carry_ti];
-            merge_group<DT, true>(ld_global_stream_v4(dc.plane + carry_g * 16u), 0u, s_exps,
-                                  static_cast<uint8_t *>(dc.dst) + carry_g * 32u, 0u, carry_n);
+            Guard Gc = G;
+            Gc.tensor<DT>(dc);
+            merge_group<DT, true>(plane_v4(dc.plane + carry_g * 16u, Gc), 0u, s_exps,
+                                  static_cast<uint8_t *>(dc.dst) + carry_g * 32u, 0u, carry_n, Gc);
+            err |= Gc.flags();
         }
         carry_n = 0;
         __syncwarp();
@@ -903,9 +984,11 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
     for (uint32_t t = t_begin; t < t_end; ++t, ++k) {
         ti_cur = tensor_of(P, t, ti_cur);
         const TensorDesc &d = P.t[ti_cur];
+        G.tensor<DT>(d);
         const uint32_t lt = t - d.tile_begin;
-        uint64_t S = __ldg(d.out_off + lt);
-        const uint64_t Eo = __ldg(d.out_off + lt + 1);
+        const bool oo = in_bounds(lt, 2, static_cast<uint64_t>(d.n_tiles) + 1u, err);
+        uint64_t S = oo ? __ldg(d.out_off + lt) : 1u;
+        const uint64_t Eo = oo ? __ldg(d.out_off + lt + 1) : 0u;
         const bool bad = Eo - S > max_span || Eo > d.n;  // Eo < S wraps above max_span
         if (bad) S = 0;
         const uint32_t span = bad ? 0u : static_cast<uint32_t>(Eo - S);
@@ -919,7 +1002,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         // the tile's plane span: the first kPrefetchGroups groups of each lane now
         const uint8_t *plane = d.plane + g0 * 16u;
         uint2 pre[2 * kPrefetchGroups];
-        prefetch_halves(pre, plane + 8u * lane, lane, 2 * ng, std::make_integer_sequence<int, 2 * kPrefetchGroups>{});
+        prefetch_halves(pre, plane + 8u * lane, lane, 2 * ng, G, std::make_integer_sequence<int, 2 * kPrefetchGroups>{});
 
         const bool landed = __all_sync(0xFFFFFFFFu, mbar_wait(&full[0], k & 1u, P.wait_ns));
         if (!landed) {
@@ -986,7 +1069,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         } else {
             uint32_t ctl;
             const uint32_t dead_c = dead >> 1;
-            cnt = byte_step_count<CB>(w, w2, g & 31, nfull, r, jmax, smem + plan.off_ctl, dead_c, ctl);
+            cnt = byte_step_count<CB>(w, w2, g & 31, nfull, r, jmax, smem + plan.off_ctl, dead_c, ctl, ctl_bytes, err);
             slow = !whole || (ctl & kCtlRowMask) == dead_c;
         }
         if (__any_sync(0xFFFFFFFFu, slow)) {
@@ -1014,10 +1097,13 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
             const uint32_t qrel = s0 + incl - cnt;
             const uint32_t q = smem_addr(s_exps) + qrel;
             // the word a range starts in may hold carried exponents: start from it
-            const uint32_t acc0 = joined ? *reinterpret_cast<const uint32_t *>(s_exps + (qrel & ~3u)) : 0u;
+            const uint32_t acc0 =
+                joined && G.ex(s_exps + (qrel & ~3u), 4) ? *reinterpret_cast<const uint32_t *>(s_exps + (qrel & ~3u)) : 0u;
             __syncwarp();
             uint32_t acc = 0, wp = 0, f8 = 0, last = 0;
-            if (!slow) byte_step_emit<CB>(w, w2, g, nfull, r, jmax, smem, q, acc0, dead, acc, wp, f8, last);
+            if (!slow)
+                byte_step_emit<CB>(w, w2, g, nfull, r, jmax, smem, q, acc0, dead, acc, wp, f8, last, fsm_bytes, exps_lo,
+                                   exps_hi, err);
             // with stored counts: a walk that left the tables is redone with the
             // window walk below; a whole walk must end the stored number of codes
             // (8 bits of f8 per code: wp * 8 + f8 advanced by 8 per symbol from q * 8)
@@ -1027,7 +1113,8 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
                 if (!slow && !redo && (wp - q) * 8u + f8 != 8u * cnt) mism = true;
             }
             __syncwarp();  // every plain store of phase 2 before the OR-ed words
-            if (!slow && !redo && f8) asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(wp), "r"(acc) : "memory");
+            if (!slow && !redo && f8 && in_bounds(wp - exps_lo, 4, exps_hi - exps_lo, err))
+                asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(wp), "r"(acc) : "memory");
             if constexpr (CNT) {
                 if (__any_sync(0xFFFFFFFFu, redo)) {
                     if (redo) {
@@ -1052,17 +1139,19 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
             const bool keep = (hi % GROUP) != 0 && !(ng == 1 && lo != 0);
             const uint32_t nmerge = keep ? ng - 1 : ng;
             const uint32_t nh = 2u * nmerge;
-            if (static_cast<uint32_t>(lane) < nh) merge_half<DT, true>(pre[0], lane, s_exps, dst_tile, lo, hi);
-            merge_rounds<DT>(pre, lane, nh, s_exps + (DT == 0 ? 8u : 16u) * lane, dst_tile + 16u * lane,
+            if (static_cast<uint32_t>(lane) < nh) merge_half<DT, true>(pre[0], lane, s_exps, dst_tile, lo, hi, G);
+            merge_rounds<DT>(pre, lane, nh, s_exps + (DT == 0 ? 8u : 16u) * lane, dst_tile + 16u * lane, G,
                              std::make_integer_sequence<int, 2 * kPrefetchGroups - 1>{});
             for (uint32_t j = lane + 64u * kPrefetchGroups; j < nh; j += 32)
-                merge_half<DT, false>(ld_global_stream_v2(plane + 8u * j), j, s_exps, dst_tile, lo, hi);
+                merge_half<DT, false>(plane_v2(plane + 8u * j, G), j, s_exps, dst_tile, lo, hi, G);
             __syncwarp();
             if (keep) {
                 if (ng > 1 && lane < static_cast<int>(GROUP / 16u)) {  // move the group's exponents to the start
                     uint4 *src = reinterpret_cast<uint4 *>(s_exps + GROUP * (ng - 1)) + lane;
-                    reinterpret_cast<uint4 *>(s_exps)[lane] = *src;
-                    *src = make_uint4(0, 0, 0, 0);
+                    if (G.ex(src, 16) && G.ex(s_exps + 16 * lane, 16)) {
+                        reinterpret_cast<uint4 *>(s_exps)[lane] = *src;
+                        *src = make_uint4(0, 0, 0, 0);
+                    }
                 }
                 carry_n = hi % GROUP;
                 carry_g = g0 + ng - 1;
@@ -1086,7 +1175,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
     // after an abort: wait (bounded) for a copy that was issued but never consumed
     if (pending)
         if (!mbar_wait(&full[0], k & 1u, P.wait_ns)) err |= DF11_DEV_ERR_TIMEOUT;
-    err = __reduce_or_sync(0xFFFFFFFFu, err);
+    err = __reduce_or_sync(0xFFFFFFFFu, err | G.flags());
     if (lane == 0) report(P.err, err);
 }
 
@@ -1257,6 +1346,8 @@ LaunchStatus build_params(const Blob *const *blobs, void *const *dst, int n, int
     P.fsm = reinterpret_cast<const uint32_t *>(b0.dev_image + L0.fsm);
     P.fsm_rows = rows;
     P.expire = opt.diag_expire_waits ? 1 : 0;
+    P.diag_bounds = opt.diag_check_bounds ? 1 : 0;
+    P.pad = 0;
     P.wait_ns = opt.diag_expire_waits ? 10000000ull : 2000000000ull;
     P.err = err;
     P.n_luts = b0.cb->n_luts();

@@ -121,6 +121,8 @@ struct DecodeParams {
     int32_t n_tensors;
     uint32_t total_tiles;
     uint32_t max_span;  // largest per-tile span over the launch's tensors
+    int32_t diag_bounds;  // bounds-checked build: check exponent-buffer accesses against 0 bytes
+    int32_t pad;
     TensorDesc t[kMaxTensorsPerLaunch];
 };
 

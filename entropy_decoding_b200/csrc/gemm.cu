@@ -379,14 +379,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_kernel(const __gr
             mi_issue = mat_of_tile(P, v, mi_issue);
             const GemmMat &d = P.mt[mi_issue];
             const uint32_t lt = v - d.tile_begin;
-            mbar_arrive_expect_tx(full, kStageTx);
-            bulk_load(stage, d.stream + static_cast<uint64_t>(lt) * kTileBytes, kTileBytes + 16u, full);
-            bulk_load(stage + kTileBytes + 16u, d.gaps + static_cast<uint64_t>(lt) * 32u, 48u, full);
-            bulk_load(stage + kTileBytes + 64u, d.counts + static_cast<uint64_t>(lt) * 32u, 32u, full);
+            uint32_t cerr = 0;
+            if (in_bounds(static_cast<uint64_t>(lt) * kTileBytes, kTileBytes + 16u,
+                          static_cast<uint64_t>(d.n_tiles) * kTileBytes + kStreamTail, cerr) &&
+                in_bounds(static_cast<uint64_t>(lt) * 32u, 48u, static_cast<uint64_t>(d.n_tiles) * 32u + kGapsTail,
+                          cerr) &&
+                in_bounds(static_cast<uint64_t>(lt) * 32u, 32u, static_cast<uint64_t>(d.n_tiles) * 32u, cerr)) {
+                mbar_arrive_expect_tx(full, kStageTx);
+                bulk_load(stage, d.stream + static_cast<uint64_t>(lt) * kTileBytes, kTileBytes + 16u, full);
+                bulk_load(stage + kTileBytes + 16u, d.gaps + static_cast<uint64_t>(lt) * 32u, 48u, full);
+                bulk_load(stage + kTileBytes + 64u, d.counts + static_cast<uint64_t>(lt) * 32u, 32u, full);
+            } else {
+                mbar_arrive(full);  // nothing copied: the stage keeps stale bytes, the error is reported
+                report(P.err, cerr);
+            }
         };
         if (lane == 0 && v0 < v_hi) issue(v0);
         bool pending = v0 < v_hi;
-        const Tables T{P.meta, P.syms, s_lut, P.lut, 1, P.n_luts};
+        const Tables T{P.meta, P.syms, s_lut, P.lut, 1, P.n_luts, smem_addr(s_exps), smem_addr(s_exps) + P.exps_bytes};
+        // every stage read stays inside the stage: 32 chunks, the look-ahead
+        // words, 48 gaps, 32 counts
+        in_bounds(0, kStageTx, kStageBytes, err);
+        Guard G;
+        G.buffer(s_exps, P.exps_bytes);
+        const uint32_t exps_lo = smem_addr(s_exps), exps_hi = exps_lo + P.exps_bytes;
+        const uint32_t fsm_bytes = static_cast<uint32_t>(rows) * kFsmRowBytes, ring_bytes = SA * kATileBytes;
         // a k-tile slot receives n more weights; the warp that completes it hands it to the MMA warp
         auto placed = [&](uint32_t kr, uint32_t n) {
             const uint32_t sa = dA.r(kr);
@@ -400,9 +417,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_kernel(const __gr
         for (uint32_t v = v0; v < v_hi; v += kDecodeWarps, ++k) {
             mi_cur = mat_of_tile(P, v, mi_cur);
             const GemmMat &d = P.mt[mi_cur];
+            G.plane_of<0>(d.plane, d.n);
             const uint32_t lt = v - d.tile_begin;
-            uint64_t S = __ldg(d.out_off + lt);
-            const uint64_t Eo = __ldg(d.out_off + lt + 1);
+            const bool oo = in_bounds(lt, 2, static_cast<uint64_t>(d.n_tiles) + 1u, err);
+            uint64_t S = oo ? __ldg(d.out_off + lt) : 1u;
+            const uint64_t Eo = oo ? __ldg(d.out_off + lt + 1) : 0u;
             const bool bad = Eo - S > P.max_span || Eo > d.n;  // Eo < S wraps above max_span
             if (bad) S = 0;
             const uint32_t span = bad ? 0u : static_cast<uint32_t>(Eo - S);
@@ -412,7 +431,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_kernel(const __gr
             const uint32_t nh = span ? static_cast<uint32_t>(((S + span + 7u) >> 3) - h0) : 0u;
             const uint8_t *plane = d.plane + h0 * 8u;
             uint2 pre[kPrefetchHalves];
-            prefetch_halves(pre, plane + 8u * lane, lane, nh, std::make_integer_sequence<int, kPrefetchHalves>{});
+            prefetch_halves(pre, plane + 8u * lane, lane, nh, G, std::make_integer_sequence<int, kPrefetchHalves>{});
 
             const bool landed = __all_sync(0xFFFFFFFFu, mbar_wait(full, k & 1u, P.wait_ns));
             if (!landed) {
@@ -486,14 +505,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_kernel(const __gr
                 const uint32_t q = smem_addr(s_exps) + s0 + incl - cnt;
                 __syncwarp();
                 uint32_t acc = 0, wp = 0, f8 = 0, last = 0;
-                if (!slow) byte_step_emit<CB>(w, w2, g, nfull, r, jmax, smem, q, 0u, dead, acc, wp, f8, last);
+                if (!slow)
+                    byte_step_emit<CB>(w, w2, g, nfull, r, jmax, smem, q, 0u, dead, acc, wp, f8, last, fsm_bytes, exps_lo,
+                                       exps_hi, err);
                 bool redo = false;
                 if (!slow) {
                     redo = (last & kFsmRowMask) == dead;
                     if (!redo && (wp - q) * 8u + f8 != 8u * cnt) mism = true;
                 }
                 __syncwarp();  // every plain store before the OR-ed last words
-                if (!slow && !redo && f8) asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(wp), "r"(acc) : "memory");
+                if (!slow && !redo && f8 && in_bounds(wp - exps_lo, 4, exps_hi - exps_lo, err))
+                    asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(wp), "r"(acc) : "memory");
                 if (__any_sync(0xFFFFFFFFu, redo)) {
                     if (redo) {
                         const int gg[1] = {g}, ee[1] = {E};
@@ -551,6 +573,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_kernel(const __gr
                     return swz(2u * rp);
                 };
                 auto merge_one = [&](uint32_t jj, uint2 p2, uint32_t aoff) {
+                    if (!G.ex(s_exps + 8u * jj, 8) || !in_bounds(aoff, 16, ring_bytes, err)) return;
                     uint2 *xp = reinterpret_cast<uint2 *>(s_exps + 8u * jj);
                     const uint2 x2 = *xp;
                     *xp = make_uint2(0u, 0u);
@@ -568,7 +591,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_kernel(const __gr
                     if (jj < nh) merge_one(jj, pre[rr], wraps ? ring_off(jj) : ((rr & 1) ? a_odd : a_even) + 512u * rr);
                 }
                 for (uint32_t jj = static_cast<uint32_t>(lane) + 32u * kPrefetchHalves; jj < nh; jj += 32)
-                    merge_one(jj, ld_global_stream_v2(plane + 8u * jj), ring_off(jj));
+                    merge_one(jj, plane_v2(plane + 8u * jj, G), ring_off(jj));
                 fence_proxy_async_smem();  // the operand tiles are read by the tensor core (async proxy)
                 if (__any_sync(0xFFFFFFFFu, mism)) {
                     // a walk wrote past its stored range: clear the whole buffer (flagged below)
@@ -587,6 +610,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_kernel(const __gr
         // after an abort: wait (bounded) for a copy that was issued but never consumed
         if (pending)
             if (!mbar_wait(full, k & 1u, P.wait_ns)) err |= DF11_DEV_ERR_TIMEOUT;
+        err |= G.flags();
     } else {
         // =============================== warps 24..27: copies, MMAs, drain
         const int quarter = warp - kDecodeWarps;  // TMEM lanes 32 quarter .. 32 quarter + 31

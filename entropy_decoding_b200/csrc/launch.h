@@ -18,6 +18,7 @@ struct DecodeOptions {
     int overlap = 0;            // 1: programmatic dependent launch (no dependency on earlier stream work)
     int diag_expire_waits = 0;  // diagnostics: no copies, every wait runs out after 10 ms
     int count_walk = 0;         // 1: byte-step walker counts with a walk even when chunk counts are stored
+    int diag_check_bounds = 0;  // diagnostics (bounds-checked build only): the exponent buffer's checked bound is 0
 };
 
 constexpr int kDefaultChunksPerThread = 1;

@@ -18,8 +18,147 @@
 #include "df11.h"
 #include "df11_internal.h"
 
+// Bounds-checked debug build: compiled with -DDF11_CHECK=1 (libdf11_check.so),
+// every shared-memory index of the decode walks (table rows, stage, exponent
+// buffer, look-ahead) and every global read and write of the byte-step decode
+// is checked against its buffer or section; an access outside is skipped and
+// DF11_DEV_ERR_BOUNDS is ORed into the launch's error word.  The normal build
+// compiles every check away.
+#ifndef DF11_CHECK
+#define DF11_CHECK 0
+#endif
+
 namespace df11 {
 namespace {
+
+// [off, off + len) inside [0, cap)?  Always true in the normal build; in the
+// check build a violation sets DF11_DEV_ERR_BOUNDS in err.
+__device__ __forceinline__ bool in_bounds(uint64_t off, uint64_t len, uint64_t cap, uint32_t &err) {
+#if DF11_CHECK
+    if (off <= cap && len <= cap - off) return true;
+    err |= DF11_DEV_ERR_BOUNDS;
+    return false;
+#else
+    (void)off;
+    (void)len;
+    (void)cap;
+    (void)err;
+    return true;
+#endif
+}
+
+// The buffers a thread's merge touches: one tensor's output (n elements of 2
+// or 1 bytes) and readable plane (n or ceil(n / 2) bytes, padded to 16 bytes
+// plus the image's tail), and the shared-memory exponent buffer it decodes
+// into.  In the bounds-checked build every access is checked against them
+// (an access outside is skipped and recorded in err); in the normal build
+// the struct is empty and every check is true.
+struct Guard {
+#if DF11_CHECK
+    uintptr_t dst = 0, plane = 0, exps = 0;
+    uint64_t dst_bytes = 0, plane_bytes = 0;
+    uint32_t exps_bytes = 0, err = 0;
+
+    __device__ __forceinline__ bool span(const void *p, uint64_t len, uintptr_t base, uint64_t cap) {
+        return in_bounds(static_cast<uint64_t>(reinterpret_cast<uintptr_t>(p) - base), len, cap, err);
+    }
+#endif
+    // the plane of n elements
+    template <int DT>
+    __device__ __forceinline__ void plane_of(const uint8_t *p, uint64_t n) {
+#if DF11_CHECK
+        plane = reinterpret_cast<uintptr_t>(p);
+        plane_bytes = ((DT == 0 ? n : (n + 1) / 2) + 15u) / 16u * 16u + kPlaneTail;
+#else
+        (void)p;
+        (void)n;
+#endif
+    }
+    // a tensor's plane and output
+    template <int DT>
+    __device__ __forceinline__ void tensor(const TensorDesc &d) {
+        plane_of<DT>(d.plane, d.n);
+#if DF11_CHECK
+        dst = reinterpret_cast<uintptr_t>(d.dst);
+        dst_bytes = d.n * (DT == 0 ? 2u : 1u);
+#endif
+    }
+    __device__ __forceinline__ void buffer(const uint8_t *e, uint32_t bytes) {
+#if DF11_CHECK
+        exps = reinterpret_cast<uintptr_t>(e);
+        exps_bytes = bytes;
+#else
+        (void)e;
+        (void)bytes;
+#endif
+    }
+    // output bytes [p, p + len)
+    __device__ __forceinline__ bool out(const void *p, uint64_t len) {
+#if DF11_CHECK
+        return span(p, len, dst, dst_bytes);
+#else
+        (void)p;
+        (void)len;
+        return true;
+#endif
+    }
+    // the elements [lo, hi) of the ne elements (esz bytes each) of a unit
+    // starting at element e0, stored at p
+    __device__ __forceinline__ bool out_elems(const void *p, uint32_t e0, uint32_t ne, uint32_t lo, uint32_t hi,
+                                              uint32_t esz) {
+#if DF11_CHECK
+        const uint32_t a = max(e0, lo), b = min(e0 + ne, hi);
+        return a >= b || out(static_cast<const uint8_t *>(p) + (a - e0) * esz, static_cast<uint64_t>(b - a) * esz);
+#else
+        (void)p;
+        (void)e0;
+        (void)ne;
+        (void)lo;
+        (void)hi;
+        (void)esz;
+        return true;
+#endif
+    }
+    // plane bytes [p, p + len)
+    __device__ __forceinline__ bool pl(const void *p, uint64_t len) {
+#if DF11_CHECK
+        return span(p, len, plane, plane_bytes);
+#else
+        (void)p;
+        (void)len;
+        return true;
+#endif
+    }
+    // exponent-buffer bytes [p, p + len) (a generic pointer into shared memory)
+    __device__ __forceinline__ bool ex(const void *p, uint64_t len) {
+#if DF11_CHECK
+        return span(p, len, exps, exps_bytes);
+#else
+        (void)p;
+        (void)len;
+        return true;
+#endif
+    }
+    __device__ __forceinline__ uint32_t flags() const {
+#if DF11_CHECK
+        return err;
+#else
+        return 0u;
+#endif
+    }
+};
+
+// Hierarchical tables a kernel stages in shared memory: n_lut_smem, in the
+// bounds-checked build no more than the launch's n_luts.
+__device__ __forceinline__ int lut_stage_count(int n_lut_smem, int n_luts) {
+#if DF11_CHECK
+    return min(n_lut_smem, n_luts);
+#else
+    (void)n_luts;
+    return n_lut_smem;
+#endif
+}
+
 // ------------------------------------------------------------------ PTX helpers
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
@@ -108,6 +247,9 @@ struct Tables {
     const uint16_t *lut_g;  // global: all hierarchical tables
     int n_lut_smem;
     int n_luts;
+    // shared-memory byte addresses [out_lo, out_hi) the window walk may write
+    // symbols to (checked in the bounds-checked build only)
+    uint32_t out_lo = 0, out_hi = 0xFFFFFFFFu;
 };
 
 // One code through the hierarchical 256-entry tables; `win` holds the next 32
@@ -122,7 +264,11 @@ __device__ __forceinline__ uint32_t lut_decode(uint32_t win, const Tables &T, ui
         const int tbl = static_cast<int>(e & 0x7FFFu);
         if (tbl >= T.n_luts) break;
         const uint32_t ix = static_cast<uint32_t>(tbl) * kLutEntries + ((win >> (24 - 8 * lvl)) & 0xFFu);
-        e = tbl < T.n_lut_smem ? T.lut_s[ix] : __ldg(T.lut_g + ix);
+        if (tbl < T.n_lut_smem) {
+            e = in_bounds(ix, 1, static_cast<uint64_t>(T.n_lut_smem) * kLutEntries, err) ? T.lut_s[ix] : 0u;
+        } else {
+            e = in_bounds(ix, 1, static_cast<uint64_t>(T.n_luts) * kLutEntries, err) ? __ldg(T.lut_g + ix) : 0u;
+        }
     }
     if ((e & (kLutPointer | 0x4000u)) || !(e & 0x3F00u)) {
         err |= DF11_DEV_ERR_CODE;
@@ -145,13 +291,15 @@ __device__ __forceinline__ uint32_t sane_meta(uint32_t e) {
 // Multi-symbol table reads: shared-memory copies were checked when staged;
 // GM = true reads the image in global memory and checks each entry.
 template <bool GM>
-__device__ __forceinline__ uint32_t meta_at(const Tables &T, uint32_t idx) {
+__device__ __forceinline__ uint32_t meta_at(const Tables &T, uint32_t idx, uint32_t &err) {
+    if (!in_bounds(idx, 1, kMultiEntries, err)) return kMetaLong;
     if constexpr (GM) return sane_meta(__ldg(T.meta + idx));
     else return T.meta[idx];
 }
 
 template <bool GM>
-__device__ __forceinline__ uint32_t syms_at(const Tables &T, uint32_t idx) {
+__device__ __forceinline__ uint32_t syms_at(const Tables &T, uint32_t idx, uint32_t &err) {
+    if (!in_bounds(idx, 1, kMultiEntries, err)) return 0u;
     if constexpr (GM) return __ldg(T.syms + idx);
     else return T.syms[idx];
 }
@@ -207,7 +355,7 @@ __device__ __forceinline__ void count_codes(const uint32_t (&w)[CPT * CW + 1], c
                 for (int c = 0; c < CPT; ++c) {
                     if (act[c]) {
                         const uint32_t win = __funnelshift_l(w[c * CW + k + 1], w[c * CW + k], acc[c]);
-                        acc[c] += meta_at<GM>(T, win >> (32 - kMultiBits));
+                        acc[c] += meta_at<GM>(T, win >> (32 - kMultiBits), err);
                     }
                 }
             }
@@ -224,7 +372,7 @@ __device__ __forceinline__ void count_codes(const uint32_t (&w)[CPT * CW + 1], c
                     continue;
                 }
                 const uint32_t win = __funnelshift_l(w[c * CW + k + 1], w[c * CW + k], p);
-                const uint32_t mm = single ? kMetaLong : meta_at<GM>(T, win >> (32 - kMultiBits));
+                const uint32_t mm = single ? kMetaLong : meta_at<GM>(T, win >> (32 - kMultiBits), err);
                 if (mm & kMetaLong) {
                     const uint32_t e = lut_decode(win, T, err);
                     acc[c] += ((e >> 8) & 0x3Fu) + kCountOne;
@@ -246,8 +394,9 @@ __device__ __forceinline__ void count_codes(const uint32_t (&w)[CPT * CW + 1], c
 // byte address out: the one or two 32-bit words they touch.  The exponent
 // buffer is zero before phase 2, so neighbouring chunks can OR into a word
 // they share and the zero high bytes leave other symbols intact.
-__device__ __forceinline__ void put_symbols(uint32_t sy, uint32_t out) {
+__device__ __forceinline__ void put_symbols(uint32_t sy, uint32_t out, const Tables &T, uint32_t &err) {
     const uint32_t a = out & ~3u, sh = (out & 3u) << 3;
+    if (!in_bounds(a - T.out_lo, sh ? 8u : 4u, T.out_hi - T.out_lo, err)) return;
     asm volatile("red.shared.or.b32 [%0], %1;" ::"r"(a), "r"(sy << sh) : "memory");
     if (sh) asm volatile("red.shared.or.b32 [%0+4], %1;" ::"r"(a), "r"(__funnelshift_l(sy, 0u, sh)) : "memory");
 }
@@ -268,9 +417,9 @@ __device__ __forceinline__ void emit_codes(const uint32_t (&w)[CPT * CW + 1], in
             while (p < lm) {
                 const uint32_t win = __funnelshift_l(lw, hi, p);
                 const uint32_t idx = win >> (32 - kMultiBits);
-                const uint32_t mm = meta_at<GM>(T, idx);
+                const uint32_t mm = meta_at<GM>(T, idx, err);
                 p += static_cast<int>(mm & kPosMask);
-                put_symbols(syms_at<GM>(T, idx), out);
+                put_symbols(syms_at<GM>(T, idx, err), out, T, err);
                 out += (mm >> kMetaCountShift) & 7u;
             }
             bool single = false;
@@ -282,18 +431,18 @@ __device__ __forceinline__ void emit_codes(const uint32_t (&w)[CPT * CW + 1], in
             }
             const uint32_t win = __funnelshift_l(lw, hi, p);
             const uint32_t idx = win >> (32 - kMultiBits);
-            const uint32_t mm = single ? kMetaLong : meta_at<GM>(T, idx);
+            const uint32_t mm = single ? kMetaLong : meta_at<GM>(T, idx, err);
             if (mm & kMetaLong) {
                 const uint32_t e = lut_decode(win, T, err);
                 p += static_cast<int>((e >> 8) & 0x3Fu);
-                put_symbols(e & 0xFFu, out);
+                put_symbols(e & 0xFFu, out, T, err);
                 out += 1;
             } else {
                 const uint32_t nv = starts_before(mm, er - p);
                 const uint32_t nb = 8u * nv;
-                const uint32_t sy = nb >= 32 ? syms_at<GM>(T, idx) : (syms_at<GM>(T, idx) & ((1u << nb) - 1u));
+                const uint32_t sy = nb >= 32 ? syms_at<GM>(T, idx, err) : (syms_at<GM>(T, idx, err) & ((1u << nb) - 1u));
                 p += static_cast<int>(mm & 0xFu);
-                if (nv) put_symbols(sy, out);
+                if (nv) put_symbols(sy, out, T, err);
                 out += nv;
             }
         }
@@ -373,7 +522,7 @@ constexpr uint32_t kCtlRowMask = kFsmRowMask >> 1;
 template <int CB>
 __device__ __forceinline__ uint32_t byte_step_count(const uint32_t (&w)[CB / 32 + 1], uint32_t w2, int g, int nfull,
                                                     int r, int jmax, const uint8_t *ctl_tab, uint32_t dead,
-                                                    uint32_t &ctl_out) {
+                                                    uint32_t &ctl_out, uint32_t tab_bytes, uint32_t &err) {
     constexpr int CW = CB / 32, NFIX = kFixedSteps<CB>;
     uint32_t ctl = 0, cnt = 0;
 #pragma unroll
@@ -384,7 +533,8 @@ __device__ __forceinline__ uint32_t byte_step_count(const uint32_t (&w)[CB / 32 
         for (int k = 0; k < 4; ++k) {
             const int j = 4 * m + k;
             if (j >= NFIX && j >= jmax) break;
-            const uint32_t e = *reinterpret_cast<const uint32_t *>(ctl_tab + step_addr<4>(x, k, ctl & kCtlRowMask));
+            const uint32_t ea = step_addr<4>(x, k, ctl & kCtlRowMask);
+            const uint32_t e = in_bounds(ea, 4, tab_bytes, err) ? *reinterpret_cast<const uint32_t *>(ctl_tab + ea) : dead;
             if (j < NFIX || j < nfull) {
                 ctl = e;
                 cnt += e;  // the count field at bit 24 gathers the codes; the fields below it never carry into it
@@ -400,13 +550,16 @@ __device__ __forceinline__ uint32_t byte_step_count(const uint32_t (&w)[CB / 32 
 }
 
 // Puts symbol bytes sy (c8 / 8 of them, unused bytes zero) after the f8 / 8
-// pending bytes of acc; a completed word goes to byte address wp.
-__device__ __forceinline__ void emit_word(uint32_t sy, uint32_t c8, uint32_t &acc, uint32_t &wp, uint32_t &f8) {
+// pending bytes of acc; a completed word goes to byte address wp (inside
+// [lo_a, hi_a), checked in the bounds-checked build).
+__device__ __forceinline__ void emit_word(uint32_t sy, uint32_t c8, uint32_t &acc, uint32_t &wp, uint32_t &f8,
+                                          uint32_t lo_a, uint32_t hi_a, uint32_t &err) {
     const uint32_t lo = acc | (sy << f8);
     const uint32_t hi = __funnelshift_l(sy, 0u, f8);  // bytes pushed past the word
     f8 += c8;
     if (f8 >= 32u) {
-        asm volatile("st.shared.u32 [%0], %1;" ::"r"(wp), "r"(lo) : "memory");
+        if (in_bounds(wp - lo_a, 4, hi_a - lo_a, err))
+            asm volatile("st.shared.u32 [%0], %1;" ::"r"(wp), "r"(lo) : "memory");
         wp += 4u;
         f8 -= 32u;
         acc = hi;
@@ -433,7 +586,8 @@ template <int CB>
 __device__ __forceinline__ void byte_step_emit(const uint32_t (&w)[CB / 32 + 1], uint32_t w2, int g, int nfull,
                                                int r, int jmax, const uint8_t *tab, uint32_t out, uint32_t acc0,
                                                uint32_t dead, uint32_t &acc, uint32_t &wp, uint32_t &f8,
-                                               uint32_t &ctl_out) {
+                                               uint32_t &ctl_out, uint32_t tab_bytes, uint32_t lo_a, uint32_t hi_a,
+                                               uint32_t &err) {
     constexpr int CW = CB / 32, NFIX = kFixedSteps<CB>;
     uint32_t ctl = 0;
     acc = acc0;
@@ -448,10 +602,12 @@ __device__ __forceinline__ void byte_step_emit(const uint32_t (&w)[CB / 32 + 1],
         for (int k = 0; k < 4; ++k) {
             const int j = 4 * m + k;
             if (j >= NFIX && j >= jmax) break;
-            const uint2 e = *reinterpret_cast<const uint2 *>(tab + step_addr<8>(x, k, ctl & kFsmRowMask));
+            const uint32_t ea = step_addr<8>(x, k, ctl & kFsmRowMask);
+            const uint2 e =
+                in_bounds(ea, 8, tab_bytes, err) ? *reinterpret_cast<const uint2 *>(tab + ea) : make_uint2(dead, 0u);
             if (j < NFIX || j < nfull) {
                 ctl = e.x;
-                emit_word(e.y, e.x >> (kFsmCountShift - 3), acc, wp, f8);
+                emit_word(e.y, e.x >> (kFsmCountShift - 3), acc, wp, f8, lo_a, hi_a, err);
             } else if (j == nfull) {
                 ep = e;  // the partial byte: emitted once after the loop
             }
@@ -460,7 +616,7 @@ __device__ __forceinline__ void byte_step_emit(const uint32_t (&w)[CB / 32 + 1],
     if (r) {
         const uint32_t ce = static_cast<uint32_t>(__popc(ep.x & ((1u << r) - 1u)));
         const uint32_t c = min(ce, 4u);
-        emit_word(c ? ep.y & (0xFFFFFFFFu >> (32u - 8u * c)) : 0u, 8u * c, acc, wp, f8);
+        emit_word(c ? ep.y & (0xFFFFFFFFu >> (32u - 8u * c)) : 0u, 8u * c, acc, wp, f8, lo_a, hi_a, err);
         if (ce > 4) ctl = dead;
     }
     ctl_out = ctl;
@@ -489,8 +645,15 @@ __device__ __forceinline__ uint2 ld_global_stream_v2_at(const void *p) {
 // they arrive while the tile decodes.
 template <int... U>
 __device__ __forceinline__ void prefetch_halves(uint2 *pre, const uint8_t *pl, uint32_t lane, uint32_t nhalf,
-                                                std::integer_sequence<int, U...>) {
-    ((lane + 32u * U < nhalf ? (void)(pre[U] = ld_global_stream_v2_at<256 * U>(pl)) : (void)0), ...);
+                                                Guard &G, std::integer_sequence<int, U...>) {
+    ((lane + 32u * U < nhalf && G.pl(pl + 256 * U, 8) ? (void)(pre[U] = ld_global_stream_v2_at<256 * U>(pl))
+                                                       : (void)0),
+     ...);
+}
+
+// One half's plane bytes, checked in the bounds-checked build (zeros outside).
+__device__ __forceinline__ uint2 plane_v2(const uint8_t *p, Guard &G) {
+    return G.pl(p, 8) ? ld_global_stream_v2(p) : make_uint2(0u, 0u);
 }
 
 }  // namespace

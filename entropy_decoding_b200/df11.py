@@ -8,6 +8,11 @@ when libdf11.so has not been built (``python -m entropy_decoding_b200.build``).
 PyTorch is used only as a source of device memory and streams: device
 pointers are plain integers (``tensor.data_ptr()``), streams are
 ``torch.cuda.Stream.cuda_stream`` integers (0 = default stream).
+
+The environment variable DF11_LIBRARY=check loads libdf11_check.so instead:
+the same C-ABI with every decode access bounds-checked (an access outside
+its buffer or section is skipped and DEV_ERR_BOUNDS set in the launch's
+error word).  It is read once, at import.
 """
 from __future__ import annotations
 
@@ -19,18 +24,24 @@ import re
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libdf11.so")
+_VARIANTS = {"": "libdf11.so", "normal": "libdf11.so", "check": "libdf11_check.so"}
+_variant = os.environ.get("DF11_LIBRARY", "")
+if _variant not in _VARIANTS:
+    raise ImportError(f"DF11_LIBRARY={_variant!r}: expected one of 'normal', 'check'")
+CHECKED = _variant == "check"
+LIB_PATH = os.path.join(_HERE, _VARIANTS[_variant])
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "df11.h")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"libdf11.so not built at {LIB_PATH}; run `python -m entropy_decoding_b200.build`")
+    raise ImportError(f"{os.path.basename(LIB_PATH)} not built at {LIB_PATH}; "
+                      f"run `python -m entropy_decoding_b200.build{' --check' if CHECKED else ''}`")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
 DF11_OK, DF11_EINVAL, DF11_ENOMEM, DF11_ECUDA, DF11_ECORRUPT, DF11_EUNSUPPORTED = range(6)
 DF11_BF16, DF11_FP8_E4M3 = 0, 1
 DTYPES = {"bf16": DF11_BF16, "e4m3": DF11_FP8_E4M3}
-DEV_ERR_SPAN, DEV_ERR_CODE, DEV_ERR_AUX, DEV_ERR_TIMEOUT = 1, 2, 4, 8
+DEV_ERR_SPAN, DEV_ERR_CODE, DEV_ERR_AUX, DEV_ERR_TIMEOUT, DEV_ERR_BOUNDS = 1, 2, 4, 8, 16
 
 
 class Df11Error(RuntimeError):
@@ -66,7 +77,8 @@ class RansTensorInfo(ctypes.Structure):
 class DecodeOpts(ctypes.Structure):
     _fields_ = [("chunks_per_thread", ctypes.c_int32), ("ctas_per_sm", ctypes.c_int32),
                 ("warps_per_cta", ctypes.c_int32), ("walker", ctypes.c_int32), ("max_ctas", ctypes.c_int32),
-                ("overlap", ctypes.c_int32), ("diag_expire_waits", ctypes.c_int32), ("count_walk", ctypes.c_int32)]
+                ("overlap", ctypes.c_int32), ("diag_expire_waits", ctypes.c_int32), ("count_walk", ctypes.c_int32),
+                ("diag_check_bounds", ctypes.c_int32)]
 
 
 class GemmMatrix(ctypes.Structure):
@@ -326,9 +338,9 @@ def df11_decode(blobs, dst_ptrs, err_ptr: int | None = None, stream: int = 0):
 
 def df11_decode_ex(blobs, dst_ptrs, err_ptr: int | None = None, stream: int = 0, chunks_per_thread: int = 0,
                    ctas_per_sm: int = 0, warps_per_cta: int = 0, walker: int = 0, max_ctas: int = 0,
-                   overlap: int = 0, diag_expire_waits: int = 0, count_walk: int = 0):
+                   overlap: int = 0, diag_expire_waits: int = 0, count_walk: int = 0, diag_check_bounds: int = 0):
     o = DecodeOpts(chunks_per_thread, ctas_per_sm, warps_per_cta, walker, max_ctas, overlap, diag_expire_waits,
-                   count_walk)
+                   count_walk, diag_check_bounds)
     _check(_lib.df11_decode_ex(_ptr_array([b.handle.value for b in blobs]), _ptr_array(dst_ptrs), len(blobs),
                                err_ptr or None, stream or None, ctypes.byref(o)), "df11_decode_ex")
 

@@ -62,6 +62,9 @@ typedef enum {
 #define DF11_DEV_ERR_CODE 2u     /* the stream held a bit pattern that is no codeword */
 #define DF11_DEV_ERR_AUX 4u      /* an auxiliary value (gap, out_off) out of its valid range */
 #define DF11_DEV_ERR_TIMEOUT 8u  /* a bounded wait on an on-chip barrier gave up */
+#define DF11_DEV_ERR_BOUNDS 16u  /* bounds-checked debug build only (libdf11_check.so, built with
+                                    -DDF11_CHECK=1): a shared- or global-memory access fell outside
+                                    its buffer or section and was skipped; never set by libdf11.so */
 
 /* Same type as cudaStream_t; pass 0 for the legacy default stream. */
 typedef struct CUstream_st *df11_stream;
@@ -277,6 +280,12 @@ typedef struct {
                                   counts when every image of the launch stores them, else walk;
                                   1 = always walk each chunk once to count its codes first (the
                                   first phase of the two-phase kernel), ignoring stored counts */
+    int32_t diag_check_bounds; /* diagnostics, 0 in normal use; acts in libdf11_check.so only
+                                  (libdf11.so ignores it).  1: every exponent-buffer access of
+                                  the merge is checked against a bound of 0 bytes, so each is
+                                  refused and skipped: the launch writes no output and sets
+                                  DF11_DEV_ERR_BOUNDS (shows the checks are live, without a
+                                  fault) */
 } df11_decode_opts;
 
 /* How a decoding thread walks its chunk (both give the same output).

@@ -5,7 +5,8 @@ import torch
 
 
 def decode_gpu(df11, blobs, stream=None, guard: int = 64, chunks_per_thread: int = 0, ctas_per_sm: int = 0,
-               warps_per_cta: int = 0, walker: int = 0, max_ctas: int = 0, count_walk: int = 0):
+               warps_per_cta: int = 0, walker: int = 0, max_ctas: int = 0, count_walk: int = 0,
+               diag_check_bounds: int = 0):
     """Uploads the blobs, decodes them in ONE df11_decode launch and returns
     (outputs as numpy bit arrays, device error word, guards intact)."""
     s = stream or torch.cuda.current_stream()
@@ -21,7 +22,8 @@ def decode_gpu(df11, blobs, stream=None, guard: int = 64, chunks_per_thread: int
             views.append(buf[guard:guard + nbytes])
         err = torch.zeros(1, dtype=torch.int32, device="cuda")
         df11.df11_decode_ex(blobs, [v.data_ptr() for v in views], err.data_ptr(), s.cuda_stream,
-                            chunks_per_thread, ctas_per_sm, warps_per_cta, walker, max_ctas, count_walk=count_walk)
+                            chunks_per_thread, ctas_per_sm, warps_per_cta, walker, max_ctas, count_walk=count_walk,
+                            diag_check_bounds=diag_check_bounds)
     s.synchronize()
     outs, guards_ok = [], True
     for b, buf, v in zip(blobs, bufs, views):

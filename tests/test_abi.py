@@ -25,7 +25,7 @@ CONSTANTS = {
     "DF11_ECORRUPT": "DF11_ECORRUPT", "DF11_EUNSUPPORTED": "DF11_EUNSUPPORTED",
     "DF11_BF16": "DF11_BF16", "DF11_FP8_E4M3": "DF11_FP8_E4M3",
     "DF11_DEV_ERR_SPAN": "DEV_ERR_SPAN", "DF11_DEV_ERR_CODE": "DEV_ERR_CODE", "DF11_DEV_ERR_AUX": "DEV_ERR_AUX",
-    "DF11_DEV_ERR_TIMEOUT": "DEV_ERR_TIMEOUT",
+    "DF11_DEV_ERR_TIMEOUT": "DEV_ERR_TIMEOUT", "DF11_DEV_ERR_BOUNDS": "DEV_ERR_BOUNDS",
     "DF11_WALKER_AUTO": "WALKER_AUTO", "DF11_WALKER_WINDOW": "WALKER_WINDOW",
     "DF11_WALKER_BYTE_STEP": "WALKER_BYTE_STEP",
     "DF11_ENCODE_NO_CHUNK_COUNTS": "ENCODE_NO_CHUNK_COUNTS",

@@ -132,6 +132,33 @@ def test_parity_launch_options(df11, oracle_mod, layout_cpt, ctas):
     _roundtrip(df11, oracle_mod, make(), dt, cb, tt, cpt=cpt, ctas=ctas)
 
 
+# (chunk bits, tile threads, walker, chunk counts): the CTA-tile kernel, the
+# warp-tile window walk, the byte-step walk with stored counts and with the
+# count walk
+KERNELS = [(128, 256, 0, "stored"), (128, 32, 1, "stored"), (128, 32, 2, "stored"), (128, 32, 2, "walk")]
+
+
+@pytest.mark.parametrize("kernel", KERNELS)
+@pytest.mark.parametrize("dt", ["bf16", "e4m3"])
+def test_bounds_checks_are_live(df11, kernel, dt):
+    """diag_check_bounds: in the bounds-checked library every exponent-buffer
+    access of the merge is checked against a bound of 0 bytes, so each one is
+    refused: no output byte is written and DF11_DEV_ERR_BOUNDS is set.  The
+    normal library ignores the option and decodes exactly, with no flag."""
+    chunk_bits, tile_threads, walker, counts = kernel
+    x = synth.random_bits(50001, dt, 3) if dt == "bf16" else synth.normal_e4m3(np.random.SeedSequence(3), 50001)
+    blob = df11.df11_encode(df11.df11_build_codebook(dt, [x]), x, chunk_bits, tile_threads)
+    (out,), err, guards = decode_gpu(df11, [blob], walker=walker, count_walk=int(counts == "walk"),
+                                     diag_check_bounds=1)
+    assert guards
+    if df11.CHECKED:
+        assert err & df11.DEV_ERR_BOUNDS
+        fill = 0xA5A5 if dt == "bf16" else 0xA5
+        assert (out == fill).all()
+    else:
+        assert err == 0 and np.array_equal(out, x)
+
+
 def test_parity_32_bit_codes(df11, oracle_mod):
     """Fibonacci counts F1..F34: package-merge limits the code to 32 bits, so
     the decoder walks all four hierarchical levels."""
@@ -359,6 +386,9 @@ def test_corrupted_device_data_sets_error_flag(df11):
         e = int(err.item())
         g = buf.cpu().numpy()
         assert (g[:guard] == 0xA5).all() and (g[guard + nbytes:] == 0xA5).all()
+        # damaged data never sends an access outside its buffer or section
+        # (checked access by access in the bounds-checked library)
+        assert not e & df11.DEV_ERR_BOUNDS
         if what == "out_off":
             assert e & df11.DEV_ERR_AUX
         if what.startswith("count"):
@@ -408,7 +438,7 @@ def test_moved_chunk_count_is_caught_and_contained(df11, oracle_mod, count_walk)
     img[c] -= 1
     img[c + 1] += 1
     out, err, guards = _decode_bound_image(df11, blob, img, count_walk=count_walk)
-    assert guards
+    assert guards and not err & df11.DEV_ERR_BOUNDS
     if count_walk:
         assert err == 0 and np.array_equal(out, x)
         return

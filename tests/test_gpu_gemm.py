@@ -207,6 +207,7 @@ def test_corrupted_counts_are_flagged(df11, oracle_mod):
     (y,), err = _run(df11, [blob], [(k, n)], [x], m)
     assert err & df11.DEV_ERR_SPAN
     assert not err & df11.DEV_ERR_TIMEOUT
+    assert not err & df11.DEV_ERR_BOUNDS
 
 
 @pytest.mark.slow

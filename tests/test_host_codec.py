@@ -27,6 +27,18 @@ def test_library_exports_every_declared_symbol(df11):
     assert df11.df11_version() == 10000
 
 
+def test_check_library_exports_the_same_symbols(df11):
+    """The bounds-checked build (kernels compiled with -DDF11_CHECK=1) is a
+    drop-in twin of libdf11.so: same C-ABI, same version."""
+    from entropy_decoding_b200 import build
+    path = build.build(check=True)
+    lib = ctypes.CDLL(path)
+    for n in df11.exported_names():
+        assert hasattr(lib, n), n
+    lib.df11_version.restype = ctypes.c_int
+    assert lib.df11_version() == 10000
+
+
 def _cases():
     return {
         "normal": ("bf16", lambda: synth.single_matrix(0)[0].tensors[0].bits[:400000]),
