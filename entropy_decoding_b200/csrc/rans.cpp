@@ -45,7 +45,7 @@ bool rans_freqs(const uint64_t *counts, int nsym, uint32_t *freqs) {
 void rans_build_table(const uint32_t *freqs, int nsym, uint32_t *table) {
     uint32_t c = 0;
     for (int s = 0; s < nsym; ++s) {
-        for (uint32_t v = 0; v < freqs[s]; ++v) table[c + v] = static_cast<uint32_t>(s) | (freqs[s] - 1) << 8 | c << 20;
+        for (uint32_t v = 0; v < freqs[s]; ++v) table[c + v] = static_cast<uint32_t>(s) | (freqs[s] - 1) << 8 | v << 20;
         c += freqs[s];
     }
 }

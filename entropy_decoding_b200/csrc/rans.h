@@ -50,7 +50,7 @@ struct RansGroup {
     int nsym = 256;
     uint32_t tile_symbols = 16384;
     uint32_t freqs[256] = {};
-    uint32_t table[kRansM] = {};  // decode entry per slot: symbol | (f - 1) << 8 | c << 20
+    uint32_t table[kRansM] = {};  // decode entry per slot: symbol | (f - 1) << 8 | (slot - c) << 20
     std::vector<RansTensor> tensors;
     const uint8_t *dev_image = nullptr;
     uint64_t dev_cap = 0;

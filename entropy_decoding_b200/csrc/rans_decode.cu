@@ -3,12 +3,16 @@
 // One warp decodes one tile at a time (a contiguous run of tiles per warp):
 // its 32 lanes are the tile's 32 interleaved coders.  A step decodes 32
 // consecutive symbols, one per lane, through the 4096-entry slot table in
-// shared memory; the lanes whose state fell below 2^16 take the next words
-// of the tile's stream in lane order (a ballot and a population count give
-// each its word).  The words reach shared memory through a per-warp ring of
-// 1024 words filled 256 words at a time, each chunk loaded into registers one
-// refill ahead.  Every 8 steps (16 for E4M3) the warp merges the decoded
-// exponents with the raw plane and writes 16 bytes per lane.
+// shared memory (entry: symbol, f - 1 and slot - c, so the state update is
+// one multiply-add and one add); the lanes whose state fell below 2^16 take
+// the next words of the tile's stream in lane order (a ballot and a
+// population count give each its word).  The words reach shared memory
+// through a per-warp ring of 1024 words filled 256 words at a time, each
+// chunk loaded into registers one refill ahead; the ring's first words are
+// mirrored after its end, so a group of steps reads it without wrapping.
+// Every 16 steps the warp merges the decoded exponents with the raw plane
+// (loaded one group ahead) and writes 32 (BF16) or 16 (E4M3) bytes per lane.
+// Groups whose steps all have 32 symbols take a path without per-lane checks.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -16,6 +20,7 @@
 
 #include "df11.h"
 #include "df11_internal.h"
+#include "merge.cuh"
 #include "rans.h"
 
 namespace df11 {
@@ -60,44 +65,67 @@ __device__ __forceinline__ uint2 ld_nc_v2(const void *p) {
     return v;
 }
 
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// A ring word (written by this warp before the __syncwarp that precedes
+// the group; the address depends on the step's ballot, so the load cannot
+// move above it).
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+    uint16_t v;
+    asm("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+    return v;
+}
+
 __device__ __forceinline__ void st_v4(void *p, uint4 v) {
     asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                  : "memory");
 }
 
-// 4 plane bytes (sign << 7 | mantissa) and 4 exponents -> 4 BF16 (two words).
-__device__ __forceinline__ void bf16x4(uint32_t p, uint32_t e, uint32_t &w0, uint32_t &w1) {
-    const uint32_t hi = (p & 0x80808080u) | ((e >> 1) & 0x7F7F7F7Fu);  // sign | exponent bits 7..1
-    const uint32_t lo = ((e << 7) & 0x80808080u) | (p & 0x7F7F7F7Fu);  // exponent bit 0 | mantissa
-    w0 = __byte_perm(lo, hi, 0x5140);
-    w1 = __byte_perm(lo, hi, 0x7362);
-}
-
-// 4 plane nibbles (sign << 3 | mantissa, element i in bits 4i..4i+3) and 4
-// exponents -> 4 E4M3 bytes.
-__device__ __forceinline__ uint32_t e4m3x4(uint32_t nib, uint32_t e) {
-    uint32_t w = 0;
+// G steps of the tile's 32 coders from step k0 on.  FULL: every step has 32
+// symbols (no per-lane check); else lane j decodes in step k only when
+// 32 k + j < m.  x: the lane's state; ra: the shared-memory address of the
+// next word in the ring (below the ring's end at the group's start; the
+// mirror covers the group's reads); the exponents go to s_ex[32 s + lane].
+template <uint32_t G, bool FULL>
+__device__ __forceinline__ void decode_group(uint32_t &x, uint32_t &ra, uint32_t k0, uint32_t m, int lane,
+                                             uint32_t below, const uint32_t *s_tab, uint8_t *s_ex) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t q = (nib >> (4 * i)) & 0xFu, x = (e >> (8 * i)) & 0xFu;
-        w |= (((q & 8u) << 4) | (x << 3) | (q & 7u)) << (8 * i);
+    for (uint32_t s = 0; s < G; ++s) {
+        const uint32_t e = s_tab[x & (kRansM - 1u)];
+        const uint32_t q = x >> kRansBits;
+        uint32_t xn = q * ((e >> 8) & 0xFFFu) + q + (e >> 20);  // f floor(x / M) + slot - c
+        bool need;
+        if constexpr (FULL) {
+            need = xn < kRansL;
+        } else {
+            const bool act = (k0 + s) * 32u + static_cast<uint32_t>(lane) < m;
+            if (!act) xn = x;
+            need = act && xn < kRansL;
+        }
+        const uint32_t mask = __ballot_sync(0xFFFFFFFFu, need);
+        if (need) xn = __byte_perm(lds_u16(ra + 2u * __popc(mask & below)), xn, 0x5410);  // xn << 16 | word
+        ra += 2u * __popc(mask);
+        x = xn;
+        s_ex[s * 32u + lane] = static_cast<uint8_t>(e);
     }
-    return w;
 }
 
 template <int DT, int NWARP>
 __global__ void __launch_bounds__(NWARP * 32, 1) rans_decode_kernel(const __grid_constant__ RansParams P) {
-    constexpr uint32_t G = DT == 0 ? 8u : 16u;  // steps per merge group
+    constexpr uint32_t G = 16u;                 // steps per merge group
     constexpr uint32_t GW = G * 32u;             // symbols per group, and the most words it can take
-    constexpr uint32_t WARP_BYTES = kRing * 2u + GW;
+    constexpr uint32_t WARP_BYTES = (kRing + GW) * 2u + GW;
     extern __shared__ __align__(16) uint8_t smem[];
     uint32_t *s_tab = reinterpret_cast<uint32_t *>(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint16_t *ring = reinterpret_cast<uint16_t *>(smem + kRansM * 4u + warp * WARP_BYTES);
-    uint8_t *s_ex = smem + kRansM * 4u + warp * WARP_BYTES + kRing * 2u;
+    uint8_t *s_ex = smem + kRansM * 4u + warp * WARP_BYTES + (kRing + GW) * 2u;
     for (int i = tid; i < static_cast<int>(kRansM / 4); i += NWARP * 32)
         reinterpret_cast<uint4 *>(s_tab)[i] = __ldg(reinterpret_cast<const uint4 *>(P.table) + i);
     __syncthreads();
+    const uint32_t ring_addr = smem_u32(ring);
 
     const uint32_t nwt = gridDim.x * NWARP;
     const uint32_t per = (P.total_tiles + nwt - 1) / nwt;
@@ -126,62 +154,74 @@ __global__ void __launch_bounds__(NWARP * 32, 1) rans_decode_kernel(const __grid
             const uint64_t w0 = static_cast<uint64_t>(c) * kRansChunkWords + 8u * lane;
             return w0 + 8u <= avail ? ld_nc_v4(ws + w0) : make_uint4(0, 0, 0, 0);
         };
-        reinterpret_cast<uint4 *>(ring)[lane] = load_chunk(0);
+        // chunk c into its ring slot (c % 4), and into the mirror after the
+        // ring when the slot holds the ring's first GW words
+        auto put_chunk = [&](uint32_t c, uint4 v) {
+            const uint32_t slot = c & 3u;
+            reinterpret_cast<uint4 *>(ring + slot * kRansChunkWords)[lane] = v;
+            if (slot * kRansChunkWords < GW) reinterpret_cast<uint4 *>(ring + kRing + slot * kRansChunkWords)[lane] = v;
+        };
+        // the lane's plane bytes of the group starting at step k: 16 (BF16:
+        // weights 16 lane .. 16 lane + 15 of the group) or 8 (E4M3: 16 nibbles)
+        const uint8_t *pl_lane = d.plane + (DT == 0 ? e0 + 16u * lane : e0 / 2u + 8u * lane);
+        auto plane_of = [&](uint32_t k) -> uint4 {
+            if constexpr (DT == 0) {
+                return ld_nc_v4(pl_lane + 32u * k);
+            } else {
+                const uint2 v = ld_nc_v2(pl_lane + 16u * k);
+                return make_uint4(v.x, v.y, 0u, 0u);
+            }
+        };
+        put_chunk(0, load_chunk(0));
         uint4 pf = load_chunk(1);
         uint32_t loaded = 1;  // chunks [0, loaded) have entered the ring (the last 4 are in it)
         uint32_t ptr = 0;     // words taken
-        const uint32_t steps = (m + 31u) / 32u;
+        const uint32_t steps = (m + 31u) / 32u, full_steps = m / 32u;
         uint8_t *out = static_cast<uint8_t *>(d.dst);
+        uint4 pl = plane_of(0);
         for (uint32_t k0 = 0; k0 < steps; k0 += G) {
             // the ring must hold words [ptr, ptr + GW): refill by chunks; a
             // chunk's slot is reused only once every word of it was taken
             while (loaded * kRansChunkWords < ptr + GW) {
-                reinterpret_cast<uint4 *>(ring + (loaded & 3u) * kRansChunkWords)[lane] = pf;
+                put_chunk(loaded, pf);
                 ++loaded;
                 pf = load_chunk(loaded);
             }
             __syncwarp();
-            const uint64_t g0 = e0 + static_cast<uint64_t>(k0) * 32u;  // first weight of the group
-            const uint2 pl = ld_nc_v2(d.plane + (DT == 0 ? g0 : g0 / 2u) + 8u * lane);
-#pragma unroll
-            for (uint32_t s = 0; s < G; ++s) {
-                const bool act = (k0 + s) * 32u + lane < m;
-                const uint32_t slot = x & (kRansM - 1u);
-                const uint32_t e = s_tab[slot];
-                uint32_t xn = (((e >> 8) & 0xFFFu) + 1u) * (x >> kRansBits) + slot - (e >> 20);
-                if (!act) xn = x;
-                const bool need = act && xn < kRansL;
-                const uint32_t mask = __ballot_sync(0xFFFFFFFFu, need);
-                if (need) xn = (xn << 16) | ring[(ptr + __popc(mask & below)) & (kRing - 1u)];
-                ptr += __popc(mask);
-                x = xn;
-                s_ex[s * 32u + lane] = static_cast<uint8_t>(e);
-            }
+            // the next group's plane bytes now: they arrive while this group decodes
+            const uint4 pl_next = k0 + G < steps ? plane_of(k0 + G) : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t ra0 = ring_addr + 2u * (ptr & (kRing - 1u));
+            uint32_t ra = ra0;
+            if (k0 + G <= full_steps) decode_group<G, true>(x, ra, k0, m, lane, below, s_tab, s_ex);
+            else decode_group<G, false>(x, ra, k0, m, lane, below, s_tab, s_ex);
+            ptr += (ra - ra0) >> 1;
             __syncwarp();
             // merge: weights [g0, g0 + cnt) of the tile's output
+            const uint64_t g0 = e0 + static_cast<uint64_t>(k0) * 32u;
             const uint32_t cnt = min(GW, m - k0 * 32u);
             if constexpr (DT == 0) {
-                const uint2 ex = *reinterpret_cast<const uint2 *>(s_ex + 8u * lane);
-                uint4 o;
-                bf16x4(pl.x, ex.x, o.x, o.y);
-                bf16x4(pl.y, ex.y, o.z, o.w);
-                uint8_t *dp = out + 2u * (g0 + 8u * lane);
-                if (8u * lane + 8u <= cnt) {
+                const uint4 ex = *reinterpret_cast<const uint4 *>(s_ex + 16u * lane);
+                uint4 o, o2;
+                merge_bf16x4(pl.x, ex.x, o.x, o.y);
+                merge_bf16x4(pl.y, ex.y, o.z, o.w);
+                merge_bf16x4(pl.z, ex.z, o2.x, o2.y);
+                merge_bf16x4(pl.w, ex.w, o2.z, o2.w);
+                uint8_t *dp = out + 2u * (g0 + 16u * lane);
+                if (16u * lane + 16u <= cnt) {
                     st_v4(dp, o);
+                    st_v4(dp + 16, o2);
                 } else {
-                    const uint32_t v[4] = {o.x, o.y, o.z, o.w};
+                    const uint32_t v[8] = {o.x, o.y, o.z, o.w, o2.x, o2.y, o2.z, o2.w};
 #pragma unroll
-                    for (uint32_t j = 0; j < 8; ++j)
-                        if (8u * lane + j < cnt)
+                    for (uint32_t j = 0; j < 16; ++j)
+                        if (16u * lane + j < cnt)
                             reinterpret_cast<uint16_t *>(dp)[j] = static_cast<uint16_t>(v[j >> 1] >> (16 * (j & 1)));
                 }
             } else {
                 const uint4 ex = *reinterpret_cast<const uint4 *>(s_ex + 16u * lane);
                 uint4 o;
-                o.x = e4m3x4(pl.x, ex.x);
-                o.y = e4m3x4(pl.x >> 16, ex.y);
-                o.z = e4m3x4(pl.y, ex.z);
-                o.w = e4m3x4(pl.y >> 16, ex.w);
+                merge_e4m3x8(pl.x, ex.x, ex.y, o.x, o.y);
+                merge_e4m3x8(pl.y, ex.z, ex.w, o.z, o.w);
                 uint8_t *dp = out + g0 + 16u * lane;
                 if (16u * lane + 16u <= cnt) {
                     st_v4(dp, o);
@@ -192,6 +232,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1) rans_decode_kernel(const __grid
                         if (16u * lane + j < cnt) dp[j] = static_cast<uint8_t>(v[j >> 2] >> (8 * (j & 3)));
                 }
             }
+            pl = pl_next;
             __syncwarp();
         }
         // every coder back at 2^16, and the tile's words taken up to its padding
@@ -209,9 +250,9 @@ constexpr int kMaxDev = 64;
 bool g_rans_attr[kMaxDev][2] = {};
 int g_rans_sms[kMaxDev] = {};
 
-uint32_t rans_smem_bytes(int dtype) {
-    const uint32_t gw = (dtype == DF11_BF16 ? 8u : 16u) * 32u;
-    return kRansM * 4u + kRansWarps * (kRing * 2u + gw);
+uint32_t rans_smem_bytes(int) {
+    const uint32_t gw = 16u * 32u;
+    return kRansM * 4u + kRansWarps * ((kRing + gw) * 2u + gw);
 }
 
 }  // namespace

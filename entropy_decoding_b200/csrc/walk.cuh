@@ -17,6 +17,7 @@
 
 #include "df11.h"
 #include "df11_internal.h"
+#include "merge.cuh"
 
 // Bounds-checked debug build: compiled with -DDF11_CHECK=1 (libdf11_check.so),
 // every shared-memory index of the decode walks (table rows, stage, exponent
@@ -449,27 +450,6 @@ __device__ __forceinline__ void emit_codes(const uint32_t (&w)[CPT * CW + 1], in
         p -= min(p, 32);
     }
 }
-
-// ------------------------------------------------------------------ field merges
-
-// 4 plane bytes + 4 exponents -> 4 BF16 words (two 32-bit outputs).
-__device__ __forceinline__ void merge_bf16x4(uint32_t P, uint32_t X, uint32_t &o0, uint32_t &o1) {
-    const uint32_t hi = (P & 0x80808080u) | ((X >> 1) & 0x7F7F7F7Fu);  // sign | exponent[7:1]
-    const uint32_t lo = ((X << 7) & 0x80808080u) | (P & 0x7F7F7F7Fu);  // exponent[0] | mantissa
-    o0 = __byte_perm(lo, hi, 0x5140);
-    o1 = __byte_perm(lo, hi, 0x7362);
-}
-
-// 4 plane bytes (8 nibbles) + 8 exponents -> 8 E4M3 bytes.
-__device__ __forceinline__ void merge_e4m3x8(uint32_t P, uint32_t X0, uint32_t X1, uint32_t &o0, uint32_t &o1) {
-    const uint32_t nl = P & 0x0F0F0F0Fu;         // elements 0, 2, 4, 6
-    const uint32_t nh = (P >> 4) & 0x0F0F0F0Fu;  // elements 1, 3, 5, 7
-    const uint32_t n0 = __byte_perm(nl, nh, 0x5140);
-    const uint32_t n1 = __byte_perm(nl, nh, 0x7362);
-    o0 = ((n0 & 0x08080808u) << 4) | ((X0 << 3) & 0x78787878u) | (n0 & 0x07070707u);
-    o1 = ((n1 & 0x08080808u) << 4) | ((X1 << 3) & 0x78787878u) | (n1 & 0x07070707u);
-}
-
 
 // ------------------------------------------------------------------ async-proxy fence
 
