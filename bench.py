@@ -75,9 +75,12 @@ def parse_args():
     p.add_argument("--count-walk", action="store_true",
                    help="decode launch option: count each chunk's codes with a first walk even though the "
                         "images store chunk counts")
-    p.add_argument("--coder", choices=["huffman", "rans"], default="huffman",
+    p.add_argument("--coder", choices=["huffman", "rans", "fused_gemm"], default="huffman",
                    help="exponent coder: the Huffman container (default) or the rANS variant (decode from HBM "
-                        "only; no end-to-end, streaming, encoder or CPU measurements)")
+                        "only; no end-to-end, streaming, encoder or CPU measurements); fused_gemm: the decode "
+                        "fused into the consuming GEMM alone (y += x W on the block's seven matrices at M = "
+                        "--gemm-m, one launch per step, the Huffman container in operand-tile order)")
+    p.add_argument("--gemm-m", type=int, default=16, help="rows of x for --coder fused_gemm (1..64)")
     p.add_argument("--rans-tile", type=int, default=0, help="rANS symbols per tile (0 = library default)")
     p.add_argument("--no-overlap", dest="overlap", action="store_false",
                    help="launch the groups in plain stream order (default: each group's decode may start "
@@ -1115,6 +1118,104 @@ def run_rans(args, rank: int, world: int, local_rank: int):
     print(json.dumps(line), flush=True)
 
 
+def run_fused_gemm(args, rank: int, world: int, local_rank: int):
+    """The decode fused into the consuming GEMM alone: the block's seven
+    matrices encoded in operand-tile order with one code, then per step one
+    df11_decode_gemm launch (y += x W at M = --gemm-m), each after an L2
+    flush and timed with CUDA events; checked once against float32 matmuls
+    of the source weights (the exact decoded weights)."""
+    import torch
+    from entropy_decoding_b200 import df11
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    threads = host_threads(world)
+    m = args.gemm_m
+    t_setup = time.time()
+    blk = synth.transformer_block(args.seed)[0]
+    shapes = [tuple(t.shape) for t in blk.tensors]
+    ws = [t.bits for t in blk.tensors]
+    tiled = [df11.df11_gemm_tile_weights(w, k, n) for w, (k, n) in zip(ws, shapes)]
+    cb = df11.df11_build_codebook("bf16", tiled)
+    blobs = [df11.df11_encode(cb, t, 128, 32, threads) for t in tiled]
+    del tiled
+    g = np.random.default_rng(2024)
+    xs = [synth.to_bf16_bits(g.standard_normal(m * k).astype(np.float32)) for k, _ in shapes]
+    with torch.cuda.stream(stream):
+        for b in blobs:
+            df11.upload(b, stream)
+        xd = [torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16).reshape(m, k)
+              for x, (k, _) in zip(xs, shapes)]
+        ys = [torch.zeros(m * n, dtype=torch.float32, device=dev) for _, n in shapes]
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+        flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream.synchronize()
+    setup_s = time.time() - t_setup
+    mats = [(b, k, n, x.data_ptr(), y.data_ptr()) for b, (k, n), x, y in zip(blobs, shapes, xd, ys)]
+
+    def launch():
+        df11.df11_decode_gemm(mats, m, err.data_ptr(), stream.cuda_stream)
+
+    smi_index = torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            flush_buf.fill_(1)
+            launch()
+        stream.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        clocks = ClockSampler(smi_index)
+        clocks.start()
+        time.sleep(0.3)
+        for a, b in ev:
+            flush_buf.fill_(1)
+            a.record(stream)
+            launch()
+            b.record(stream)
+        stream.synchronize()
+        clk = clocks.stop()
+        ms = [a.elapsed_time(b) for a, b in ev]
+        for y in ys:
+            y.zero_()
+        launch()
+        stream.synchronize()
+    e = int(err.item())
+    assert e == 0, f"fused gemm: device error word {e}"
+    for y, x, w, (k, n) in zip(ys, xd, ws, shapes):
+        wv = torch.from_numpy(w.view(np.int16)).to(dev).view(torch.bfloat16).reshape(k, n).float()
+        ref = x.float() @ wv
+        scale = x.float().abs() @ wv.abs()
+        assert bool(((y.reshape(m, n) - ref).abs() <= 2 * (k + 16) * 2.0 ** -24 * scale).all()), "fused gemm"
+    if rank != 0:
+        return
+    nw = sum(k * n for k, n in shapes)
+    comp = 0
+    for b in blobs:
+        i = b.info()
+        comp += i.stream_bytes + i.plane_bytes + i.gaps_bytes + i.out_off_bytes + i.counts_bytes
+    algo = comp + sum(2 * m * k + 8 * m * n for k, n in shapes)
+    med = statistics.median(ms)
+    peak, peak_src = hbm_peak()
+    shape = df11.df11_decode_gemm_launch_shape([(b, k, n, 0, 0) for b, (k, n) in zip(blobs, shapes)], m)
+    line = {
+        "metric": "fused decode + GEMM weights/s", "value": world * nw / (med / 1e3), "unit": "weights/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": med,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1/sqrt(fan_in)) weights and N(0,1) activations, random init)",
+        "config": {"workload": f"one Llama-3-8B-shaped transformer block, 7 matrices [in, out], y += x W at "
+                               f"M = {m}, one fused launch per step", "batch_m": m, "seed": args.seed,
+                   "l2": f"flushed: {L2_FLUSH_BYTES >> 20} MB written before every timed launch"},
+        "bytes_per_weight": algo / nw,
+        "roofline": {"bound": "hbm", "achieved": algo / (med / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                     "frac": algo / (med / 1e3) / 1e9 / peak, "peak_source": peak_src, "traffic": None,
+                     "algorithmic_bytes": algo, "kernel": "decode_gemm_kernel",
+                     "launch": {"grid": shape[0], "block": shape[1], "smem_bytes": shape[2]}},
+        "ms_min": min(ms), "cpu_baseline": None, "e2e": None, "gpu_launches": args.steps, "clocks": clk,
+        "setup_s": setup_s,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse_args()
     rank, world, local_rank = rank_env()
@@ -1130,6 +1231,8 @@ def main():
     try:
         if args.coder == "rans":
             run_rans(args, rank, world, local_rank)
+        elif args.coder == "fused_gemm":
+            run_fused_gemm(args, rank, world, local_rank)
         else:
             run_ours(args, rank, world, local_rank)
     finally:
