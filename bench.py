@@ -41,7 +41,9 @@ from entropy_decoding_b200 import synth  # noqa: E402
 
 METRIC = "decompressed BF16 GB/s"
 HBM_FALLBACK_GBS = 6650.0
-KERNEL_SRC = os.path.join(ROOT, "entropy_decoding_b200", "csrc", "decode.cu")
+# the decode kernels' source: decode.cu and the device headers it includes
+KERNEL_SRC = [os.path.join(ROOT, "entropy_decoding_b200", "csrc", f)
+              for f in ("decode.cu", "walk.cuh", "merge.cuh", "df11_internal.h")]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
 
 
@@ -193,8 +195,11 @@ def hbm_peak():
 
 
 def kernel_hash() -> str:
-    with open(KERNEL_SRC, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    h = hashlib.sha256()
+    for path in KERNEL_SRC:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def traffic_per_weight():

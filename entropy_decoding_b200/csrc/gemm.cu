@@ -12,13 +12,13 @@
 // launch for all matrices that share a code.
 //
 // Layout.  The weights are encoded in operand-tile order (gemm.h): every
-// operand tile of 128 output rows x 16 reduction columns is a contiguous run
-// of 2048 weights of the ordinary container (stream, gaps, chunk counts,
+// operand tile of 128 output rows x 64 reduction columns is a contiguous run
+// of 8192 weights of the ordinary container (stream, gaps, chunk counts,
 // out_off per warp tile, plane).  So the decode's output positions map to
 // operand tiles by a shift, and nothing else of the container changes.
 //
 // One CTA per SM owns a contiguous range of operand tiles ("k-tiles"):
-//   * warps 0..23 decode the container's warp tiles that cover the range,
+//   * warps 0..19 decode the container's warp tiles that cover the range,
 //     round robin, with the byte-step walk (phase 2 into the warp's own
 //     exponent buffer, as in the decode kernel), and merge them with the raw
 //     sign+mantissa plane (prefetched into registers at tile start) straight
@@ -26,13 +26,13 @@
 //     tcgen05.mma reads (a ring of operand slots, rows of kGemmTileK weights,
 //     the swizzle as wide as a row); a counter per operand slot hands a
 //     completed k-tile (128 x kGemmTileK weights placed) to the MMA warp;
-//   * warp 24 (lane 0) issues the copies of the activation tiles
+//   * warp 20 (lane 0) issues the copies of the activation tiles
 //     (cp.async.bulk.tensor with the same swizzle, no multicast; rows past
 //     M read as zeros) and the MMAs of each k-tile (M = 128 output rows, N =
 //     M padded to 16, K = 16 each) into a TMEM accumulator, and
 //     frees each k-tile's slot once its MMAs completed (checked without
 //     blocking, so several k-tiles' MMAs are in flight);
-//   * warps 24..27 drain the accumulator (tcgen05.ld) into y with
+//   * warps 20..23 drain the accumulator (tcgen05.ld) into y with
 //     floating-point adds whenever the range leaves a block of 128 output
 //     rows: y's rows are split over CTAs along K, so y accumulates.
 // Every wait is bounded (%globaltimer); a timeout sets DF11_DEV_ERR_TIMEOUT
@@ -55,7 +55,7 @@
 namespace df11 {
 namespace {
 
-constexpr int kDecodeWarps = 24;  // warps 0..23 decode; 24..27 copy, multiply and drain
+constexpr int kDecodeWarps = 20;  // warps 0..19 decode; 20..23 copy, multiply and drain
 constexpr int kMmaWarp = kDecodeWarps;  // a multiple of 4: warps kMmaWarp + q reach TMEM lanes 32 q .. 32 q + 31
 constexpr int kGemmThreads = 32 * (kDecodeWarps + 4);
 constexpr uint32_t kKTile = kGemmTileN * kGemmTileK;  // weights of one operand tile
@@ -612,7 +612,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_kernel(const __gr
             if (!mbar_wait(full, k & 1u, P.wait_ns)) err |= DF11_DEV_ERR_TIMEOUT;
         err |= G.flags();
     } else {
-        // =============================== warps 24..27: copies, MMAs, drain
+        // =============================== warps 20..23: copies, MMAs, drain
         const int quarter = warp - kDecodeWarps;  // TMEM lanes 32 quarter .. 32 quarter + 31
         const uint32_t tmem = C.tmem;
         const bool issuer = warp == kMmaWarp;
