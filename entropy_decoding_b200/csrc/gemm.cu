@@ -858,10 +858,12 @@ LaunchStatus build_gemm(const GemmJob *jobs, int n, int m, int *err, bool with_m
     if (max_span > kKTile) return LaunchStatus::kUnsupported;  // a tile's codes must touch <= 2 operand tiles
     P.max_span = static_cast<uint32_t>(max_span);
     P.total_kt = static_cast<uint32_t>(kts);
-    // slots: 4 activation tiles (8 when an operand tile holds fewer than 64
-    // columns), operand tiles as many as fit, 4..32
+    // slots: 3 activation tiles (8 when an operand tile holds fewer than 64
+    // columns), operand tiles as many as fit, 4..32 (3 activation slots
+    // instead of 4 leave room for a seventh operand slot on the block at
+    // M = 16: 0.305 vs 0.311 ms)
     P.exps_bytes = gemm_exps_bytes(P.max_span);
-    P.b_slots = kGemmTileK >= 64 ? 4 : 8;
+    P.b_slots = kGemmTileK >= 64 ? 3 : 8;
     const uint32_t budget = 227u * 1024u - 1024u;  // opt-in shared memory less the alignment slack
     P.a_slots = kMaxASlots;
     while (P.a_slots > 4 && make_gemm_plan(rows, P.mpad, P.a_slots, P.b_slots, P.exps_bytes).total > budget)
