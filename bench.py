@@ -43,7 +43,7 @@ METRIC = "decompressed BF16 GB/s"
 HBM_FALLBACK_GBS = 6650.0
 # the decode kernels' source: decode.cu and the device headers it includes
 KERNEL_SRC = [os.path.join(ROOT, "entropy_decoding_b200", "csrc", f)
-              for f in ("decode.cu", "walk.cuh", "merge.cuh", "df11_internal.h")]
+              for f in ("decode.cu", "walk.cuh", "merge.cuh", "check.cuh", "df11_internal.h")]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
 
 

@@ -30,7 +30,7 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 SOURCES_CU = ["decode.cu", "encode.cu", "rans_decode.cu", "gemm.cu"]
 SOURCES_CPP = ["codec.cpp", "capi.cpp", "rans.cpp"]
-HEADERS = ["df11_internal.h", "codec.h", "launch.h", "encode.h", "rans.h", "walk.cuh", "gemm.h", "merge.cuh"]
+HEADERS = ["df11_internal.h", "codec.h", "launch.h", "encode.h", "rans.h", "walk.cuh", "gemm.h", "merge.cuh", "check.cuh"]
 
 
 def _newer(target: str, deps: list[str]) -> bool:

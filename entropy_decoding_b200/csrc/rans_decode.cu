@@ -18,6 +18,7 @@
 #include <cstdint>
 #include <mutex>
 
+#include "check.cuh"
 #include "df11.h"
 #include "df11_internal.h"
 #include "merge.cuh"
@@ -88,9 +89,12 @@ __device__ __forceinline__ void st_v4(void *p, uint4 v) {
 // 32 k + j < m.  x: the lane's state; ra: the shared-memory address of the
 // next word in the ring (below the ring's end at the group's start; the
 // mirror covers the group's reads); the exponents go to s_ex[32 s + lane].
+// Ring reads are checked against [ring_lo, ring_lo + ring_bytes) in the
+// bounds-checked build.
 template <uint32_t G, bool FULL>
 __device__ __forceinline__ void decode_group(uint32_t &x, uint32_t &ra, uint32_t k0, uint32_t m, int lane,
-                                             uint32_t below, const uint32_t *s_tab, uint8_t *s_ex) {
+                                             uint32_t below, const uint32_t *s_tab, uint8_t *s_ex, uint32_t ring_lo,
+                                             uint32_t ring_bytes, uint32_t &err) {
 #pragma unroll
     for (uint32_t s = 0; s < G; ++s) {
         const uint32_t e = s_tab[x & (kRansM - 1u)];
@@ -105,7 +109,9 @@ __device__ __forceinline__ void decode_group(uint32_t &x, uint32_t &ra, uint32_t
             need = act && xn < kRansL;
         }
         const uint32_t mask = __ballot_sync(0xFFFFFFFFu, need);
-        if (need) xn = __byte_perm(lds_u16(ra + 2u * __popc(mask & below)), xn, 0x5410);  // xn << 16 | word
+        const uint32_t wa = ra + 2u * __popc(mask & below);
+        if (need && in_bounds(wa - ring_lo, 2, ring_bytes, err))
+            xn = __byte_perm(lds_u16(wa), xn, 0x5410);  // xn << 16 | word
         ra += 2u * __popc(mask);
         x = xn;
         s_ex[s * 32u + lane] = static_cast<uint8_t>(e);
@@ -140,12 +146,19 @@ __global__ void __launch_bounds__(NWARP * 32, 1) rans_decode_kernel(const __grid
         const uint32_t lt = t - d.tile_begin;
         const uint64_t e0 = static_cast<uint64_t>(lt) * P.tile_symbols;
         const uint32_t m = static_cast<uint32_t>(min(static_cast<uint64_t>(P.tile_symbols), d.n - e0));
+        if (!in_bounds(lt, 2, static_cast<uint64_t>(d.n_tiles) + 1u, err)) continue;
         const uint64_t wb = d.tile_words[lt], we = d.tile_words[lt + 1];
         if (wb > we || we > d.words_len || (wb & 7u)) {
             err |= DF11_DEV_ERR_AUX;
             continue;
         }
-        uint32_t x = d.states[static_cast<uint64_t>(lt) * 32u + lane];
+        uint32_t x = in_bounds(static_cast<uint64_t>(lt) * 32u + lane, 1, static_cast<uint64_t>(d.n_tiles) * 32u, err)
+                         ? d.states[static_cast<uint64_t>(lt) * 32u + lane]
+                         : kRansL;
+        // readable plane bytes (the section plus its tail) and output bytes,
+        // for the bounds-checked build
+        const uint64_t plane_cap = (DT == 0 ? d.n : (d.n + 1) / 2) + kRansPlaneTail;
+        const uint64_t out_cap = d.n * (DT == 0 ? 2u : 1u);
         const uint16_t *ws = d.words + wb;  // 16-byte aligned: wb is a multiple of 8 words
         const uint64_t avail = d.words_len + kRansWordsTail - wb;
         // chunk c = words [256 c, 256 c + 256) of the tile, lane's 8 of them;
@@ -165,6 +178,8 @@ __global__ void __launch_bounds__(NWARP * 32, 1) rans_decode_kernel(const __grid
         // weights 16 lane .. 16 lane + 15 of the group) or 8 (E4M3: 16 nibbles)
         const uint8_t *pl_lane = d.plane + (DT == 0 ? e0 + 16u * lane : e0 / 2u + 8u * lane);
         auto plane_of = [&](uint32_t k) -> uint4 {
+            const uint64_t off = static_cast<uint64_t>(pl_lane - d.plane) + (DT == 0 ? 32u : 16u) * k;
+            if (!in_bounds(off, DT == 0 ? 16u : 8u, plane_cap, err)) return make_uint4(0u, 0u, 0u, 0u);
             if constexpr (DT == 0) {
                 return ld_nc_v4(pl_lane + 32u * k);
             } else {
@@ -192,8 +207,10 @@ __global__ void __launch_bounds__(NWARP * 32, 1) rans_decode_kernel(const __grid
             const uint4 pl_next = k0 + G < steps ? plane_of(k0 + G) : make_uint4(0u, 0u, 0u, 0u);
             const uint32_t ra0 = ring_addr + 2u * (ptr & (kRing - 1u));
             uint32_t ra = ra0;
-            if (k0 + G <= full_steps) decode_group<G, true>(x, ra, k0, m, lane, below, s_tab, s_ex);
-            else decode_group<G, false>(x, ra, k0, m, lane, below, s_tab, s_ex);
+            if (k0 + G <= full_steps)
+                decode_group<G, true>(x, ra, k0, m, lane, below, s_tab, s_ex, ring_addr, (kRing + GW) * 2u, err);
+            else
+                decode_group<G, false>(x, ra, k0, m, lane, below, s_tab, s_ex, ring_addr, (kRing + GW) * 2u, err);
             ptr += (ra - ra0) >> 1;
             __syncwarp();
             // merge: weights [g0, g0 + cnt) of the tile's output
@@ -207,7 +224,9 @@ __global__ void __launch_bounds__(NWARP * 32, 1) rans_decode_kernel(const __grid
                 merge_bf16x4(pl.z, ex.z, o2.x, o2.y);
                 merge_bf16x4(pl.w, ex.w, o2.z, o2.w);
                 uint8_t *dp = out + 2u * (g0 + 16u * lane);
-                if (16u * lane + 16u <= cnt) {
+                const uint32_t nw = 16u * lane < cnt ? min(16u, cnt - 16u * lane) : 0u;  // weights this lane stores
+                if (!in_bounds(2u * (g0 + 16u * lane), 2u * nw, out_cap, err)) {
+                } else if (16u * lane + 16u <= cnt) {
                     st_v4(dp, o);
                     st_v4(dp + 16, o2);
                 } else {
@@ -223,7 +242,9 @@ __global__ void __launch_bounds__(NWARP * 32, 1) rans_decode_kernel(const __grid
                 merge_e4m3x8(pl.x, ex.x, ex.y, o.x, o.y);
                 merge_e4m3x8(pl.y, ex.z, ex.w, o.z, o.w);
                 uint8_t *dp = out + g0 + 16u * lane;
-                if (16u * lane + 16u <= cnt) {
+                const uint32_t nw = 16u * lane < cnt ? min(16u, cnt - 16u * lane) : 0u;  // weights this lane stores
+                if (!in_bounds(g0 + 16u * lane, nw, out_cap, err)) {
+                } else if (16u * lane + 16u <= cnt) {
                     st_v4(dp, o);
                 } else {
                     const uint32_t v[4] = {o.x, o.y, o.z, o.w};

@@ -15,38 +15,13 @@
 #include <cstdint>
 #include <utility>
 
+#include "check.cuh"
 #include "df11.h"
 #include "df11_internal.h"
 #include "merge.cuh"
 
-// Bounds-checked debug build: compiled with -DDF11_CHECK=1 (libdf11_check.so),
-// every shared-memory index of the decode walks (table rows, stage, exponent
-// buffer, look-ahead) and every global read and write of the byte-step decode
-// is checked against its buffer or section; an access outside is skipped and
-// DF11_DEV_ERR_BOUNDS is ORed into the launch's error word.  The normal build
-// compiles every check away.
-#ifndef DF11_CHECK
-#define DF11_CHECK 0
-#endif
-
 namespace df11 {
 namespace {
-
-// [off, off + len) inside [0, cap)?  Always true in the normal build; in the
-// check build a violation sets DF11_DEV_ERR_BOUNDS in err.
-__device__ __forceinline__ bool in_bounds(uint64_t off, uint64_t len, uint64_t cap, uint32_t &err) {
-#if DF11_CHECK
-    if (off <= cap && len <= cap - off) return true;
-    err |= DF11_DEV_ERR_BOUNDS;
-    return false;
-#else
-    (void)off;
-    (void)len;
-    (void)cap;
-    (void)err;
-    return true;
-#endif
-}
 
 // The buffers a thread's merge touches: one tensor's output (n elements of 2
 // or 1 bytes) and readable plane (n or ceil(n / 2) bytes, padded to 16 bytes

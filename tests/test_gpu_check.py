@@ -6,8 +6,8 @@ checked against its bound.  An access outside is skipped and
 DF11_DEV_ERR_BOUNDS is set in the launch's error word; nothing traps.
 
 The small-case GPU suites (decode, GPU encode, the decode fused into the
-GEMM) run against it in a child process (the binding picks its library once,
-at import, from DF11_LIBRARY).  Their parity tests demand an error word of 0,
+GEMM, the rANS decode) run against it in a child process (the binding picks
+its library once, at import, from DF11_LIBRARY).  Their parity tests demand an error word of 0,
 their corruption tests demand no DF11_DEV_ERR_BOUNDS, and
 test_bounds_checks_are_live demands that a bound made 0 bytes is reported."""
 import os
@@ -19,7 +19,7 @@ import pytest
 pytestmark = pytest.mark.gpu
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-SUITES = ["tests/test_gpu_decode.py", "tests/test_gpu_encode.py", "tests/test_gpu_gemm.py"]
+SUITES = ["tests/test_gpu_decode.py", "tests/test_gpu_encode.py", "tests/test_gpu_gemm.py", "tests/test_gpu_rans.py"]
 
 
 @pytest.fixture(scope="module")

@@ -126,6 +126,9 @@ def test_damaged_data_flagged(df11):
         h = buf.cpu().numpy()
         assert (h[:guard] == 0xA5).all() and (h[guard + nbytes:] == 0xA5).all()
         assert e & (df11.DEV_ERR_SPAN if what == "state" else df11.DEV_ERR_AUX)
+        # damaged data never sends an access outside its buffer or section
+        # (checked access by access in the bounds-checked library)
+        assert not e & df11.DEV_ERR_BOUNDS
     # the same group uploaded again decodes exactly
     (out,), err, ok = _decode(df11, g, [x])
     assert err == 0 and ok and np.array_equal(out, x)
