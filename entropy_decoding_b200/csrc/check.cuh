@@ -35,5 +35,10 @@ __device__ __forceinline__ bool in_bounds(uint64_t off, uint64_t len, uint64_t c
 #endif
 }
 
+// The same for an access that may be empty (an empty one is always inside).
+__device__ __forceinline__ bool in_bounds_or_empty(uint64_t off, uint64_t len, uint64_t cap, uint32_t &err) {
+    return len == 0 || in_bounds(off, len, cap, err);
+}
+
 }  // namespace
 }  // namespace df11

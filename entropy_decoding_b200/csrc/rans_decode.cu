@@ -225,7 +225,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1) rans_decode_kernel(const __grid
                 merge_bf16x4(pl.w, ex.w, o2.z, o2.w);
                 uint8_t *dp = out + 2u * (g0 + 16u * lane);
                 const uint32_t nw = 16u * lane < cnt ? min(16u, cnt - 16u * lane) : 0u;  // weights this lane stores
-                if (!in_bounds(2u * (g0 + 16u * lane), 2u * nw, out_cap, err)) {
+                if (!in_bounds_or_empty(2u * (g0 + 16u * lane), 2u * nw, out_cap, err)) {
                 } else if (16u * lane + 16u <= cnt) {
                     st_v4(dp, o);
                     st_v4(dp + 16, o2);
@@ -243,7 +243,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1) rans_decode_kernel(const __grid
                 merge_e4m3x8(pl.y, ex.z, ex.w, o.z, o.w);
                 uint8_t *dp = out + g0 + 16u * lane;
                 const uint32_t nw = 16u * lane < cnt ? min(16u, cnt - 16u * lane) : 0u;  // weights this lane stores
-                if (!in_bounds(g0 + 16u * lane, nw, out_cap, err)) {
+                if (!in_bounds_or_empty(g0 + 16u * lane, nw, out_cap, err)) {
                 } else if (16u * lane + 16u <= cnt) {
                     st_v4(dp, o);
                 } else {
