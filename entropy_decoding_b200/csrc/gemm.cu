@@ -260,8 +260,6 @@ struct SlotDiv {
     __device__ __forceinline__ uint32_t r(uint32_t x) const { return x - q(x) * d; }
 };
 
-// Waits until *ctr >= target (an acquire); false when the CTA aborted or the
-// wait ran past limit_ns (which aborts the CTA).
 // Acquire load, release add (shared memory, CTA scope): a release orders
 // every write the thread saw before it (the warp's, after a __syncwarp).
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t *p) {
