@@ -927,9 +927,16 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
     const uint32_t t_begin = min((blockIdx.x * NWARP + warp) * per, P.total_tiles);
     const uint32_t t_end = min(t_begin + per, P.total_tiles);
     int ti_issue = tensor_of(P, t_begin), ti_cur = ti_issue;
+    // the first tile of the tensor after ti: a warp's run stays in one tensor
+    // for most tiles, so the descriptor search runs only when it crosses one
+    auto next_begin = [&](int ti) -> uint32_t { return ti + 1 < P.n_tensors ? P.t[ti + 1].tile_begin : 0xFFFFFFFFu; };
+    uint32_t nb_issue = next_begin(ti_issue), nb_cur = nb_issue;
     // lane 0: copy tile t's stream slice and gaps into the stage
     auto issue = [&](uint32_t t) {
-        ti_issue = tensor_of(P, t, ti_issue);
+        if (t >= nb_issue) {
+            ti_issue = tensor_of(P, t, ti_issue);
+            nb_issue = next_begin(ti_issue);
+        }
         const TensorDesc &d = P.t[ti_issue];
         const uint32_t lt = t - d.tile_begin;
         uint32_t cerr = 0;
@@ -982,7 +989,10 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
     };
 
     for (uint32_t t = t_begin; t < t_end; ++t, ++k) {
-        ti_cur = tensor_of(P, t, ti_cur);
+        if (t >= nb_cur) {
+            ti_cur = tensor_of(P, t, ti_cur);
+            nb_cur = next_begin(ti_cur);
+        }
         const TensorDesc &d = P.t[ti_cur];
         G.tensor<DT>(d);
         const uint32_t lt = t - d.tile_begin;
