@@ -1058,10 +1058,16 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         // ---- this thread's range of codes
         // stream bits from this thread's chunk on: the tile's remainder (64-bit,
         // warp-uniform) clamped to [-1, 32 CB + 256], then 32-bit per thread
-        // (no range reaches past CB + 255 bits of its chunk)
-        const int64_t trem = static_cast<int64_t>(d.total_bits) - static_cast<int64_t>(lt) * (32 * CB);
-        const int rem = static_cast<int>(max(min(trem, static_cast<int64_t>(32 * CB + 256)), static_cast<int64_t>(-1))) -
-                        lane * CB;
+        // (no range reaches past CB + 255 bits of its chunk).  Only a tensor's
+        // last tile can hold fewer: every other tile is followed by one whose
+        // first gap is at most the bits left after this tile, so its lanes'
+        // ranges come out the same with the clamp's upper value
+        int rem0 = 32 * CB + 256;
+        if (lt + 1u >= d.n_tiles) {
+            const int64_t trem = static_cast<int64_t>(d.total_bits) - static_cast<int64_t>(lt) * (32 * CB);
+            rem0 = static_cast<int>(max(min(trem, static_cast<int64_t>(32 * CB + 256)), static_cast<int64_t>(-1)));
+        }
+        const int rem = rem0 - lane * CB;
         const int E = min(max(rem, 0), CB);
         if (graw >= 32) err |= DF11_DEV_ERR_AUX;
         const int g = min(graw, 63);
