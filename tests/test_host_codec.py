@@ -39,6 +39,26 @@ def test_check_library_exports_the_same_symbols(df11):
     assert lib.df11_version() == 10000
 
 
+def test_library_choice_from_the_environment(df11):
+    """DF11_LIBRARY picks the library at import: 'check' loads the
+    bounds-checked twin, anything unknown is refused."""
+    import os
+    import subprocess
+    import sys
+    from entropy_decoding_b200 import build
+    build.build(check=True)
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = "from entropy_decoding_b200 import df11; print(df11.CHECKED, os.path.basename(df11.LIB_PATH))"
+    for var, want in (("check", "True libdf11_check.so"), ("normal", "False libdf11.so"), ("", "False libdf11.so")):
+        env = dict(os.environ, DF11_LIBRARY=var)
+        r = subprocess.run([sys.executable, "-c", "import os; " + code], cwd=root, env=env, capture_output=True,
+                           text=True, timeout=300)
+        assert r.returncode == 0 and r.stdout.strip() == want, (var, r.stdout, r.stderr[-500:])
+    r = subprocess.run([sys.executable, "-c", "import entropy_decoding_b200.df11"], cwd=root,
+                       env=dict(os.environ, DF11_LIBRARY="bogus"), capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0 and "DF11_LIBRARY" in r.stderr
+
+
 def _cases():
     return {
         "normal": ("bf16", lambda: synth.single_matrix(0)[0].tensors[0].bits[:400000]),
