@@ -29,10 +29,11 @@
 //   * warp 20 (lane 0) issues the copies of the activation tiles
 //     (cp.async.bulk.tensor with the same swizzle, no multicast; rows past
 //     M read as zeros) and the MMAs of each k-tile (M = 128 output rows, N =
-//     M padded to 16, K = 16 each) into a TMEM accumulator, and
+//     M padded to 16, K = 16 each; one TMEM accumulator per MMA of a tile,
+//     so they do not wait for each other), and
 //     frees each k-tile's slot once its MMAs completed (checked without
 //     blocking, so several k-tiles' MMAs are in flight);
-//   * warps 20..23 drain the accumulator (tcgen05.ld) into y with
+//   * warps 20..23 drain the accumulators (tcgen05.ld) into y with
 //     floating-point adds whenever the range leaves a block of 128 output
 //     rows: y's rows are split over CTAs along K, so y accumulates.
 // Every wait is bounded (%globaltimer); a timeout sets DF11_DEV_ERR_TIMEOUT
@@ -328,7 +329,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_kernel(const __gr
     const uint32_t cta = blockIdx.x;
     const uint32_t kt_lo = P.cta_kt[cta], kt_hi = P.cta_kt[cta + 1], n_kt = kt_hi - kt_lo;
     const uint64_t lo = static_cast<uint64_t>(kt_lo) * kKTile, hi = static_cast<uint64_t>(kt_hi) * kKTile;
-    const uint32_t ncols = P.mpad <= 32 ? 32u : 64u;
+    // TMEM: one FP32 accumulator of mpad columns per MMA of a tile (K = 16
+    // each, kGemmTileK / 16 of them), so a tile's MMAs do not wait for each
+    // other's results; the drain adds them up.  A power of two >= 32 columns.
+    constexpr uint32_t kAccs = kGemmTileK / 16;
+    const uint32_t acc_cols = kAccs * static_cast<uint32_t>(P.mpad);
+    const uint32_t ncols = acc_cols <= 32 ? 32u : acc_cols <= 64 ? 64u : acc_cols <= 128 ? 128u : 256u;
 
     // ---- set-up: tables (a row index past the last row is redirected to the
     // dead row), zeroed control block, stages and exponent buffers
@@ -663,8 +669,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_kernel(const __gr
                             const uint32_t b0 = smem_addr(smem + plan.off_b + dB.r(issued) * plan.b_bytes);
 #pragma unroll
                             for (int k16 = 0; k16 < kGemmTileK / 16; ++k16)
-                                tc_mma(tmem, swz_desc(a0 + 32u * k16), swz_desc(b0 + 32u * k16), idesc,
-                                       (issued > kr || k16 > 0) ? 1u : 0u);
+                                tc_mma(tmem + static_cast<uint32_t>(k16) * static_cast<uint32_t>(P.mpad),
+                                       swz_desc(a0 + 32u * k16), swz_desc(b0 + 32u * k16), idesc,
+                                       issued > kr ? 1u : 0u);
                             tc_commit(&C.mma_done[dA.r(issued)]);
                             ++issued;
                             prog = true;
@@ -693,7 +700,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_kernel(const __gr
                 aborted = __shfl_sync(0xFFFFFFFFu, aborted, 0);
                 n_x = __shfl_sync(0xFFFFFFFFu, n_x, 0);
             }
-            // drain the accumulator of this block of rows into y
+            // drain the accumulators of this block of rows into y
             named_sync(1, 128);  // warps kMmaWarp .. kMmaWarp + 3
             const bool skip = __shfl_sync(0xFFFFFFFFu, ld_vol(&C.abort), 0) != 0;
             if (!skip) {
@@ -701,11 +708,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) decode_gemm_kernel(const __gr
                 float *yc = d.y + static_cast<uint64_t>(nb) * kGemmTileN + 32u * quarter + lane;
                 for (int c0 = 0; c0 < P.mpad; c0 += 16) {
                     uint32_t vv[16];
+                    float sum[16];
                     tc_ld16(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + static_cast<uint32_t>(c0), vv);
                     tc_wait_ld();
 #pragma unroll
+                    for (int j = 0; j < 16; ++j) sum[j] = __uint_as_float(vv[j]);
+                    for (uint32_t a = 1; a < kAccs; ++a) {
+                        tc_ld16(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + a * static_cast<uint32_t>(P.mpad) +
+                                    static_cast<uint32_t>(c0), vv);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) sum[j] += __uint_as_float(vv[j]);
+                    }
+#pragma unroll
                     for (int j = 0; j < 16; ++j)
-                        if (c0 + j < P.m) atomicAdd(yc + static_cast<uint64_t>(c0 + j) * d.n_out, __uint_as_float(vv[j]));
+                        if (c0 + j < P.m) atomicAdd(yc + static_cast<uint64_t>(c0 + j) * d.n_out, sum[j]);
                 }
             }
             tc_fence_before();
