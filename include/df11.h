@@ -516,8 +516,9 @@ typedef struct {
  * decoded weights never reach HBM.  y is accumulated with floating-point
  * adds (the reduction over K is split between CTAs), so the caller zeroes y
  * for a plain product, and the rounding order of y varies from run to run
- * (every y element is within K * 2^-24 * sum_k |x_mk w_kn| of the exact
- * product plus what y held).  The matrices share one code (one codebook),
+ * (every y element is within (K + 16) * 2^-24 * sum_k |x_mk w_kn| of the
+ * exact product plus what y held: K products added in FP32, plus the adds of
+ * a tile's four accumulators and of the CTAs that share the reduction).  The matrices share one code (one codebook),
  * as in df11_decode.  M = m in 1..DF11_GEMM_MAX_BATCH; n_mats in
  * 1..DF11_GEMM_MAX_MATS.  dev_err_flag as in df11_decode (its bits mean the
  * y of that launch is not valid).  Never allocates, never synchronises.
